@@ -1,0 +1,132 @@
+"""Seeded synthetic inputs for the bidirectional Mamba mixer layer.
+
+This module only draws random numbers; it holds none of the layer's
+arithmetic, so both the CUDA path and the fp64 oracle can be fed from it.
+
+Distributions (the layer's already-projected inputs and S4D-real-initialised
+parameters, as the throughput workloads use them):
+
+  x, z, dt_raw             ~ N(0, 1)                       [b, L, D]  (dt per direction)
+  B, C                     ~ N(0, 1) per direction          [b, L, N]
+  dt_bias[r, d]            = log(expm1(s)), s log-uniform in [1e-3, 1e-1]
+                             (so that softplus(dt_bias) = s)
+  A[r, d, n]               = -(n + 1)                        (S4D-real)
+  D[r, d]                  = 1
+  conv_w[r, d, k], conv_b  ~ U(-0.5, 0.5)
+  separate parameters for the forward (r = 0) and reverse (r = 1) layers.
+
+Draw order from one ``torch.Generator`` seeded with ``seed`` (fixed, so a
+seed names one input set):
+  bias_f, bias_b, w_f, b_f, w_b, b_b, x, z, dt_f, dt_b, B_f, C_f, B_b, C_b
+Floating tensors are drawn in fp32 and then rounded (RNE) to the I/O dtype;
+the oracle receives exactly the rounded values widened to fp64.  A CPU
+generator and a CUDA generator give different streams for the same seed, so
+``device`` is part of an input set's name.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+D_CONV = 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One named synthetic workload (sizes, dtype and seed)."""
+    name: str
+    batch: int
+    L: int
+    d_inner: int
+    d_state: int = 16
+    dtype: str = "bf16"          # I/O dtype of x, z, dt, B, C and out
+    seed: int = 0
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.L
+
+    @property
+    def elements(self) -> int:
+        return self.batch * self.L * self.d_inner
+
+
+# The workloads the layer is specified on.
+TINY = Workload("tiny_b1_L256_D64_fp32", 1, 256, 64, 16, "fp32", 0)
+LAYER_1P3B = Workload("layer_1p3b_b8_L2048_D4096_bf16", 8, 2048, 4096, 16, "bf16", 1)
+LONG_SEQ = {L: Workload(f"long_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 2)
+            for L in (4096, 16384, 65536, 131072)}
+BLOCK_CACHED = Workload("block_cached_b16_P65536_G32_D4096_bf16", 16, 32, 4096, 16, "bf16", 4,
+                        extra={"prefix": 65536, "block": 32, "blocks": 16, "steps_per_block": 128})
+DENOISER_SWEEP = {L: Workload(f"denoiser_48x128_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 3,
+                              extra={"layers": 48, "steps": 128})
+                  for L in (2048, 8192, 32768, 131072)}
+
+
+def torch_dtype(name: str) -> torch.dtype:
+    return {"fp32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def make_params(D: int, N: int, g: torch.Generator, device="cpu") -> dict:
+    """Parameters of both directions (fp32).  Draws bias_f, bias_b, w_f, b_f, w_b, b_b."""
+    lo, hi = math.log(1e-3), math.log(1e-1)
+    bias = []
+    for _ in range(2):
+        s = torch.exp(torch.rand(D, generator=g, device=device, dtype=torch.float64) * (hi - lo) + lo)
+        bias.append(torch.log(torch.expm1(s)).float())
+    w, cb = [], []
+    for _ in range(2):
+        w.append(torch.rand(D, D_CONV, generator=g, device=device) - 0.5)
+        cb.append(torch.rand(D, generator=g, device=device) - 0.5)
+    A = -torch.arange(1, N + 1, device=device, dtype=torch.float32).repeat(2, D, 1).contiguous()
+    return {
+        "A": A,                                             # [2, D, N]
+        "D": torch.ones(2, D, device=device),               # [2, D]
+        "dt_bias": torch.stack(bias).contiguous(),          # [2, D]
+        "conv_w": torch.stack(w).contiguous(),              # [2, D, 4]
+        "conv_b": torch.stack(cb).contiguous(),             # [2, D]
+    }
+
+
+def make_inputs(batch: int, L: int, D: int, N: int, dtype: str, g: torch.Generator,
+                device="cpu") -> dict:
+    """Layer inputs.  Draws x, z, dt_f, dt_b, B_f, C_f, B_b, C_b."""
+    td = torch_dtype(dtype)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=device, dtype=torch.float32).to(td)
+
+    x = randn(batch, L, D)
+    z = randn(batch, L, D)
+    dt = torch.empty(2, batch, L, D, device=device, dtype=td)
+    dt[0] = randn(batch, L, D)
+    dt[1] = randn(batch, L, D)
+    B = torch.empty(2, batch, L, N, device=device, dtype=td)
+    C = torch.empty(2, batch, L, N, device=device, dtype=td)
+    B[0] = randn(batch, L, N)
+    C[0] = randn(batch, L, N)
+    B[1] = randn(batch, L, N)
+    C[1] = randn(batch, L, N)
+    return {"x": x, "z": z, "dt": dt, "B": B, "C": C}
+
+
+def make_case(batch: int, L: int, D: int, N: int = 16, dtype: str = "bf16", seed: int = 0,
+              device="cpu"):
+    """(inputs, params) for one layer call, drawn in the documented order."""
+    g = _gen(seed, device)
+    params = make_params(D, N, g, device)
+    inputs = make_inputs(batch, L, D, N, dtype, g, device)
+    return inputs, params
+
+
+def make_workload(w: Workload, device="cpu"):
+    return make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device)
