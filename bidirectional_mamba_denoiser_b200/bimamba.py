@@ -1,0 +1,204 @@
+"""Python binding of the C ABI in include/bimamba.h (ctypes, marshalling only).
+
+Each function has the name of the C entry point it calls.  Tensors are torch
+tensors on the CUDA device; torch allocates outputs and workspaces and
+supplies the current stream.  Every step of the layer runs in the CUDA
+library: if ``libbimamba.so`` is missing this module raises on import, and
+there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB_PATH = _build.LIB
+
+BIMAMBA_OK = 0
+BIMAMBA_ERR_INVALID_ARG = -1
+BIMAMBA_ERR_UNSUPPORTED = -2
+BIMAMBA_ERR_MISALIGNED = -3
+BIMAMBA_ERR_WORKSPACE = -4
+BIMAMBA_ERR_CUDA = -5
+
+BIMAMBA_F32 = 0
+BIMAMBA_BF16 = 1
+
+BIMAMBA_FWD_ONLY = 0x1
+BIMAMBA_REV_ONLY = 0x2
+BIMAMBA_LANES_SHIFT = 8
+
+D_STATE = 16
+
+
+class BimambaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
+
+
+class Inputs(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("z", ctypes.c_void_p), ("dt", ctypes.c_void_p * 2),
+                ("B", ctypes.c_void_p * 2), ("C", ctypes.c_void_p * 2), ("dtype", ctypes.c_int)]
+
+
+class FwdState(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_void_p), ("conv_x", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is not built; run `python -c \"import __graft_entry__ as g; g.build()\"` "
+                          "or `python bidirectional_mamba_denoiser_b200/build.py`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, U, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint, ctypes.c_size_t
+    lib.bimamba_workspace_bytes.argtypes = [I, I64, I, I, U]
+    lib.bimamba_workspace_bytes.restype = SZ
+    lib.bimamba_layer_fwd.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
+                                      I, I64, I, I, U, P, SZ, P]
+    lib.bimamba_layer_fwd.restype = I
+    lib.bimamba_prefix_state.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), I, I64, I, I,
+                                         ctypes.POINTER(FwdState), P]
+    lib.bimamba_prefix_state.restype = I
+    lib.bimamba_block_step.argtypes = [ctypes.POINTER(FwdState), ctypes.POINTER(Inputs), I, ctypes.POINTER(Params),
+                                       P, I, I, I, I, ctypes.POINTER(FwdState), U, P]
+    lib.bimamba_block_step.restype = I
+    lib.bimamba_status_string.argtypes = [I]
+    lib.bimamba_status_string.restype = ctypes.c_char_p
+    lib.bimamba_abi_version.restype = I
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.bimamba_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return BIMAMBA_F32
+    if t == torch.bfloat16:
+        return BIMAMBA_BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors passed to the CUDA library must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _pair(t):
+    """A per-direction input: a [2, ...] tensor or a (fwd, rev) pair."""
+    if isinstance(t, (tuple, list)):
+        return t[0], t[1]
+    return t[0], t[1]
+
+
+def make_params(params: dict) -> Params:
+    return Params(_ptr(params["A"]), _ptr(params["D"]), _ptr(params["dt_bias"]),
+                  _ptr(params["conv_w"]), _ptr(params.get("conv_b")))
+
+
+def make_inputs(x, z, dt, B, C) -> Inputs:
+    dt0, dt1 = _pair(dt)
+    B0, B1 = _pair(B)
+    C0, C1 = _pair(C)
+    inp = Inputs()
+    inp.x = _ptr(x)
+    inp.z = _ptr(z)
+    inp.dt[0], inp.dt[1] = _ptr(dt0), _ptr(dt1)
+    inp.B[0], inp.B[1] = _ptr(B0), _ptr(B1)
+    inp.C[0], inp.C[1] = _ptr(C0), _ptr(C1)
+    inp.dtype = _dtype_code(x.dtype)
+    return inp
+
+
+def bimamba_workspace_bytes(batch: int, L: int, d_inner: int, d_state: int = D_STATE, flags: int = 0) -> int:
+    return int(lib.bimamba_workspace_bytes(batch, L, d_inner, d_state, flags))
+
+
+def bimamba_layer_fwd(x, z, dt, B, C, params: dict, out=None, out_dtype=None, flags: int = 0,
+                      workspace=None, stream=None):
+    """Full-sequence bidirectional layer.  x, z [b, L, D]; dt [2, b, L, D];
+    B, C [2, b, L, 16]; params as produced by workloads.make_params (on the
+    device).  Returns out [b, L, D]."""
+    b, L, D = x.shape
+    N = (B[0] if isinstance(B, (tuple, list)) else B).shape[-1]
+    if out is None:
+        out = torch.empty(b, L, D, device=x.device, dtype=out_dtype or x.dtype)
+    need = bimamba_workspace_bytes(b, L, D, N, flags)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
+    inp = make_inputs(x, z, dt, B, C)
+    par = make_params(params)
+    rc = lib.bimamba_layer_fwd(ctypes.byref(inp), ctypes.byref(par), _ptr(out), _dtype_code(out.dtype),
+                               b, L, D, N, flags, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_layer_fwd", rc)
+    return out
+
+
+def bimamba_prefix_state(x, dt, B, params: dict, h_out=None, conv_x_out=None, stream=None):
+    """Forward scan over the prefix x [b, P, D] (dt, B: the forward direction's,
+    [b, P, D] / [b, P, 16], or [2, ...] stacks whose first entry is used).
+    Returns (h [b, D, 16] fp32, conv_x [b, 3, D])."""
+    b, P, D = x.shape
+    dt0 = dt[0] if (isinstance(dt, (tuple, list)) or dt.dim() == 4) else dt
+    B0 = B[0] if (isinstance(B, (tuple, list)) or B.dim() == 4) else B
+    N = B0.shape[-1]
+    if h_out is None:
+        h_out = torch.empty(b, D, N, device=x.device, dtype=torch.float32)
+    if conv_x_out is None:
+        conv_x_out = torch.empty(b, 3, D, device=x.device, dtype=x.dtype)
+    inp = Inputs()
+    inp.x = _ptr(x)
+    inp.dt[0] = _ptr(dt0)
+    inp.B[0] = _ptr(B0)
+    inp.dtype = _dtype_code(x.dtype)
+    par = make_params(params)
+    st = FwdState(_ptr(h_out), _ptr(conv_x_out))
+    rc = lib.bimamba_prefix_state(ctypes.byref(inp), ctypes.byref(par), b, P, D, N, ctypes.byref(st),
+                                  _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_prefix_state", rc)
+    return h_out, conv_x_out
+
+
+def bimamba_block_step(state, x, z, dt, B, C, params: dict, out=None, out_dtype=None, new_state=None,
+                       flags: int = 0, stream=None):
+    """One step on the active block x [b, G, D] from state = (h, conv_x).
+    new_state = (h, conv_x) tensors to commit into (may be `state` itself)."""
+    b, G, D = x.shape
+    N = state[0].shape[-1]
+    if out is None:
+        out = torch.empty(b, G, D, device=x.device, dtype=out_dtype or x.dtype)
+    inp = make_inputs(x, z, dt, B, C)
+    par = make_params(params)
+    st = FwdState(_ptr(state[0]), _ptr(state[1]))
+    ns = FwdState(_ptr(new_state[0]), _ptr(new_state[1])) if new_state is not None else None
+    rc = lib.bimamba_block_step(ctypes.byref(st), ctypes.byref(inp), G, ctypes.byref(par), _ptr(out),
+                                _dtype_code(out.dtype), b, D, N, ctypes.byref(ns) if ns is not None else None,
+                                flags, _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_block_step", rc)
+    return out

@@ -1,0 +1,317 @@
+// bimamba_api.cu -- the C ABI (include/bimamba.h): argument checks, launch
+// shapes and kernel dispatch.  All arithmetic lives in scan_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "bimamba.h"
+#include "scan_kernels.cuh"
+
+namespace {
+
+using bimamba::KParams;
+using bf16 = __nv_bfloat16;
+
+constexpr int kT = 16;       // tokens per chunk (full layer, prefix)
+constexpr int kWPD = 4;      // warps per direction per CTA (full layer)
+constexpr int kWPB = 8;      // warps per CTA (prefix, block step)
+constexpr int kTBlock = 64;  // longest block of the block step
+constexpr int kMaxBatch = 65535;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t elem_size(bimamba_dtype_t t) { return t == BIMAMBA_F32 ? 4 : 2; }
+
+bool dtype_ok(int t) { return t == BIMAMBA_F32 || t == BIMAMBA_BF16; }
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+int ensure_smem(const void* fn, size_t bytes) {
+    if (bytes <= 48 * 1024) return BIMAMBA_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({fn, dev})) return BIMAMBA_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return BIMAMBA_ERR_CUDA;
+    done.insert({fn, dev});
+    return BIMAMBA_OK;
+}
+
+int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? BIMAMBA_OK : BIMAMBA_ERR_CUDA;
+}
+
+// Lanes per channel: the smallest power of two that gives about one resident
+// thread slot per SM thread (148 SMs x 1024), at most 8.
+int pick_lanes(int64_t chains, unsigned flags) {
+    const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    if (forced) return (int)forced;
+    const int64_t target = 148LL * 1024;
+    int g = 1;
+    while (g < 8 && chains * g < target) g *= 2;
+    return g;
+}
+
+bool lanes_ok(unsigned flags) {
+    const unsigned f = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    return f == 0 || f == 1 || f == 2 || f == 4 || f == 8 || f == 16;
+}
+
+int check_params(const bimamba_params_t* p) {
+    if (!p || !p->A || !p->D || !p->dt_bias || !p->conv_w) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_w, 4) ||
+        (p->conv_b && !aligned(p->conv_b, 4)))
+        return BIMAMBA_ERR_MISALIGNED;
+    return BIMAMBA_OK;
+}
+
+void fill_params(KParams& k, const bimamba_params_t* p) {
+    k.A = p->A;
+    k.Dskip = p->D;
+    k.dt_bias = p->dt_bias;
+    k.conv_w = p->conv_w;
+    k.conv_b = p->conv_b;
+}
+
+// ---- full layer dispatch
+
+template <int G, typename Tin, typename Tout>
+int launch_layer(const KParams& k, cudaStream_t st) {
+    constexpr int CW = kWPD * (32 / G);
+    const void* fn = reinterpret_cast<const void*>(&bimamba::layer_kernel<G, kT, kWPD, Tin, Tout>);
+    const size_t smem = sizeof(float) * bimamba::layer_smem_floats<G, kT, kWPD>();
+    int rc = ensure_smem(fn, smem);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + CW - 1) / CW), (unsigned)k.batch);
+    bimamba::layer_kernel<G, kT, kWPD, Tin, Tout><<<grid, 2 * kWPD * 32, smem, st>>>(k);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+int layer_by_lanes(int g, const KParams& k, cudaStream_t st) {
+    switch (g) {
+        case 1: return launch_layer<1, Tin, Tout>(k, st);
+        case 2: return launch_layer<2, Tin, Tout>(k, st);
+        case 4: return launch_layer<4, Tin, Tout>(k, st);
+        case 8: return launch_layer<8, Tin, Tout>(k, st);
+        case 16: return launch_layer<16, Tin, Tout>(k, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+// ---- prefix dispatch
+
+template <int G, typename Tin>
+int launch_prefix(const KParams& k, cudaStream_t st) {
+    constexpr int CW = kWPB * (32 / G);
+    const void* fn = reinterpret_cast<const void*>(&bimamba::prefix_kernel<G, kT, kWPB, Tin>);
+    const size_t smem = sizeof(float) * bimamba::prefix_smem_floats<G, kT, kWPB>();
+    int rc = ensure_smem(fn, smem);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + CW - 1) / CW), (unsigned)k.batch);
+    bimamba::prefix_kernel<G, kT, kWPB, Tin><<<grid, kWPB * 32, smem, st>>>(k);
+    return launch_status();
+}
+
+template <typename Tin>
+int prefix_by_lanes(int g, const KParams& k, cudaStream_t st) {
+    switch (g) {
+        case 1: return launch_prefix<1, Tin>(k, st);
+        case 2: return launch_prefix<2, Tin>(k, st);
+        case 4: return launch_prefix<4, Tin>(k, st);
+        case 8: return launch_prefix<8, Tin>(k, st);
+        case 16: return launch_prefix<16, Tin>(k, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+// ---- block-step dispatch
+
+template <int G, int TB, typename Tin, typename Tout>
+int launch_block(const KParams& k, cudaStream_t st) {
+    constexpr int CW = kWPB * (32 / G);
+    const void* fn = reinterpret_cast<const void*>(&bimamba::block_kernel<G, TB, kWPB, Tin, Tout>);
+    const size_t smem = sizeof(float) * bimamba::block_smem_floats<G, TB, kWPB>();
+    int rc = ensure_smem(fn, smem);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + CW - 1) / CW), (unsigned)k.batch);
+    bimamba::block_kernel<G, TB, kWPB, Tin, Tout><<<grid, kWPB * 32, smem, st>>>(k);
+    return launch_status();
+}
+
+// The whole block is one chunk held in registers, so at least 4 lanes share
+// a channel (at most 16 tokens per lane); blocks of up to 32 tokens use the
+// smaller shared-memory footprint.
+template <typename Tin, typename Tout>
+int block_by_lanes(int g, const KParams& k, cudaStream_t st) {
+    if (g < 4) g = 4;
+    if (k.L <= 32) {
+        switch (g) {
+            case 4: return launch_block<4, 32, Tin, Tout>(k, st);
+            case 8: return launch_block<8, 32, Tin, Tout>(k, st);
+            case 16: return launch_block<16, 32, Tin, Tout>(k, st);
+        }
+    } else {
+        switch (g) {
+            case 4: return launch_block<4, kTBlock, Tin, Tout>(k, st);
+            case 8: return launch_block<8, kTBlock, Tin, Tout>(k, st);
+            case 16: return launch_block<16, kTBlock, Tin, Tout>(k, st);
+        }
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+int check_inputs(const bimamba_inputs_t* in, bool need_reverse, bool need_z_c) {
+    if (!in || !in->x || !in->dt[0] || !in->B[0]) return BIMAMBA_ERR_INVALID_ARG;
+    if (need_z_c && (!in->z || !in->C[0])) return BIMAMBA_ERR_INVALID_ARG;
+    if (need_reverse && (!in->dt[1] || !in->B[1] || !in->C[1])) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(in->dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    const size_t a = elem_size(in->dtype);
+    const void* ptrs[8] = {in->x, in->z, in->dt[0], in->dt[1], in->B[0], in->B[1], in->C[0], in->C[1]};
+    for (const void* q : ptrs)
+        if (q && !aligned(q, a)) return BIMAMBA_ERR_MISALIGNED;
+    return BIMAMBA_OK;
+}
+
+void fill_inputs(KParams& k, const bimamba_inputs_t* in) {
+    k.x = in->x;
+    k.z = in->z;
+    for (int r = 0; r < 2; ++r) {
+        k.dt[r] = in->dt[r];
+        k.B[r] = in->B[r];
+        k.C[r] = in->C[r];
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int bimamba_abi_version(void) { return 1; }
+
+const char* bimamba_status_string(int status) {
+    switch (status) {
+        case BIMAMBA_OK: return "ok";
+        case BIMAMBA_ERR_INVALID_ARG: return "invalid argument (null pointer or bad size)";
+        case BIMAMBA_ERR_UNSUPPORTED: return "unsupported (d_state, dtype, block length or flag)";
+        case BIMAMBA_ERR_MISALIGNED: return "pointer not aligned to its element size";
+        case BIMAMBA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case BIMAMBA_ERR_CUDA: return "CUDA launch or attribute call failed";
+    }
+    return "unknown status";
+}
+
+size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags) {
+    (void)flags;
+    if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || d_state != bimamba::kNState) return 0;
+    return (size_t)batch * (size_t)L * (size_t)d_inner * sizeof(float);
+}
+
+int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, void* out,
+                      bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner, int d_state,
+                      unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
+    if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
+    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK;
+    if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
+    if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    int rc = check_inputs(in, true, true);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (!aligned(out, elem_size(out_dtype))) return BIMAMBA_ERR_MISALIGNED;
+    const size_t need = bimamba_workspace_bytes(batch, L, d_inner, d_state, flags);
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return BIMAMBA_ERR_WORKSPACE;
+
+    KParams k = {};
+    fill_inputs(k, in);
+    fill_params(k, p);
+    k.out = out;
+    k.ws = static_cast<float*>(workspace);
+    k.L = L;
+    k.M = L / 2;
+    k.D = d_inner;
+    k.batch = batch;
+    k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
+    k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    const int g = pick_lanes(2LL * batch * d_inner, flags);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if (in_bf && out_bf) return layer_by_lanes<bf16, bf16>(g, k, st);
+    if (in_bf) return layer_by_lanes<bf16, float>(g, k, st);
+    if (out_bf) return layer_by_lanes<float, bf16>(g, k, st);
+    return layer_by_lanes<float, float>(g, k, st);
+}
+
+int bimamba_prefix_state(const bimamba_inputs_t* prefix, const bimamba_params_t* p, int batch, int64_t P,
+                         int d_inner, int d_state, bimamba_fwd_state_t* state_out, void* cuda_stream) {
+    if (batch <= 0 || batch > kMaxBatch || P <= 0 || d_inner <= 0) return BIMAMBA_ERR_INVALID_ARG;
+    if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
+    int rc = check_inputs(prefix, false, false);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (!state_out || !state_out->h || !state_out->conv_x) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(state_out->h, 4) || !aligned(state_out->conv_x, elem_size(prefix->dtype)))
+        return BIMAMBA_ERR_MISALIGNED;
+
+    KParams k = {};
+    fill_inputs(k, prefix);
+    fill_params(k, p);
+    k.h_out = state_out->h;
+    k.tail_out = state_out->conv_x;
+    k.L = P;
+    k.D = d_inner;
+    k.batch = batch;
+    k.dir_scale[0] = k.dir_scale[1] = 1.f;
+    const int g = pick_lanes((int64_t)batch * d_inner, 0);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (prefix->dtype == BIMAMBA_BF16) return prefix_by_lanes<bf16>(g, k, st);
+    return prefix_by_lanes<float>(g, k, st);
+}
+
+int bimamba_block_step(const bimamba_fwd_state_t* prefix_state, const bimamba_inputs_t* block, int block_len,
+                       const bimamba_params_t* p, void* out, bimamba_dtype_t out_dtype, int batch, int d_inner,
+                       int d_state, bimamba_fwd_state_t* new_state, unsigned flags, void* cuda_stream) {
+    if (batch <= 0 || batch > kMaxBatch || d_inner <= 0 || !out || block_len <= 0) return BIMAMBA_ERR_INVALID_ARG;
+    if (d_state != bimamba::kNState || block_len > kTBlock) return BIMAMBA_ERR_UNSUPPORTED;
+    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK;
+    if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
+    if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    int rc = check_inputs(block, true, true);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (!prefix_state || !prefix_state->h || !prefix_state->conv_x) return BIMAMBA_ERR_INVALID_ARG;
+    if (new_state && (!new_state->h || !new_state->conv_x)) return BIMAMBA_ERR_INVALID_ARG;
+    const size_t a = elem_size(block->dtype);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(prefix_state->h, 4) || !aligned(prefix_state->conv_x, a))
+        return BIMAMBA_ERR_MISALIGNED;
+    if (new_state && (!aligned(new_state->h, 4) || !aligned(new_state->conv_x, a))) return BIMAMBA_ERR_MISALIGNED;
+
+    KParams k = {};
+    fill_inputs(k, block);
+    fill_params(k, p);
+    k.out = out;
+    k.h_in = prefix_state->h;
+    k.tail_in = prefix_state->conv_x;
+    k.h_out = new_state ? new_state->h : nullptr;
+    k.tail_out = new_state ? new_state->conv_x : nullptr;
+    k.L = block_len;
+    k.D = d_inner;
+    k.batch = batch;
+    k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
+    k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    const int g = pick_lanes((int64_t)batch * d_inner, flags);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const bool in_bf = block->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if (in_bf && out_bf) return block_by_lanes<bf16, bf16>(g, k, st);
+    if (in_bf) return block_by_lanes<bf16, float>(g, k, st);
+    if (out_bf) return block_by_lanes<float, bf16>(g, k, st);
+    return block_by_lanes<float, float>(g, k, st);
+}
+
+}  // extern "C"

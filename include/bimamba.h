@@ -1,0 +1,145 @@
+/*
+ * bimamba.h -- C ABI of the B200 (sm_100a) bidirectional Mamba mixer layer.
+ *
+ * The layer is the sequence mixer of DiffuMamba's masked-diffusion denoiser
+ * ("DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone",
+ * arXiv 2511.15927v4, §3.2 Eq. (4)-(6), App. A.1 Eq. (7)-(9)): two
+ * independent Mamba layers, one over the sequence left to right and one right
+ * to left, whose outputs are added.  Its inputs are the already-projected
+ * x, z, dt, B, C.  Per batch row b, channel d and direction r (0 = forward,
+ * 1 = reverse):
+ *
+ *   u_r[t]     = silu(conv_b[r][d] + sum_{k<4} conv_w[r][d][k] * x[t - 3 + k])   (r = 0)
+ *              = silu(conv_b[r][d] + sum_{k<4} conv_w[r][d][k] * x[t + 3 - k])   (r = 1)
+ *                (zero outside [0, L): causal / anti-causal width-4 conv, §3.2)
+ *   delta_r[t] = softplus(dt_r[t] + dt_bias[r][d])
+ *   h_n        = exp(delta_r[t] * A[r][d][n]) * h_n + delta_r[t] * B_r[t][n] * u_r[t]
+ *                over t = 0..L-1 (r = 0, Eq. (4)) or t = L-1..0 (r = 1, Eq. (5)), h = 0 first
+ *   y_r[t]     = sum_n C_r[t][n] * h_n + D[r][d] * u_r[t]
+ *   out[t]     = (y_0[t] + y_1[t]) * silu(z[t])                   (Eq. (6), SiLU(z) gate)
+ *
+ * The block step is the block-cached decoding form (§4.3: right-to-left
+ * state updates stay inside the current block while the cached forward states
+ * carry across blocks; "Training Hybrid Block Diffusion Language Models with
+ * Partial Bidirectionality", arXiv 2607.02805, abstract: restricting the
+ * reverse scan to the active block makes caching across blocks exact).
+ *
+ * Conventions for every entry point:
+ *  - All tensors are caller-owned device memory, row-major and contiguous in
+ *    the layouts given below.  The library allocates nothing, never
+ *    synchronises the stream and never reads device data on the host.
+ *  - Work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and runs asynchronously; errors of the kernels themselves appear
+ *    at the caller's next synchronisation.
+ *  - Return value 0 (BIMAMBA_OK) or a negative BIMAMBA_ERR_* code; nothing is
+ *    launched when a check fails.  No C++ exception crosses this boundary.
+ *  - Outputs must not alias inputs, except where stated (state commit).
+ *  - d_state must be 16 (the state dimension of the layer's S4D-real
+ *    parameterisation); other values return BIMAMBA_ERR_UNSUPPORTED.
+ *  - Pointers must be aligned to their element size.
+ */
+#ifndef BIMAMBA_H
+#define BIMAMBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BIMAMBA_OK                0
+#define BIMAMBA_ERR_INVALID_ARG  (-1)  /* NULL pointer, size <= 0, size too large */
+#define BIMAMBA_ERR_UNSUPPORTED  (-2)  /* d_state != 16, unknown dtype or flag    */
+#define BIMAMBA_ERR_MISALIGNED   (-3)  /* a pointer not aligned to its element    */
+#define BIMAMBA_ERR_WORKSPACE    (-4)  /* workspace NULL or smaller than needed   */
+#define BIMAMBA_ERR_CUDA         (-5)  /* a CUDA launch or attribute call failed  */
+
+/* Element type of x, z, dt, B, C, the conv tail and the output. */
+typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
+
+/* flags (bitwise OR) */
+#define BIMAMBA_FWD_ONLY   0x1u   /* y_1 taken as 0: out = y_0 * silu(z) (test aid) */
+#define BIMAMBA_REV_ONLY   0x2u   /* y_0 taken as 0: out = y_1 * silu(z) (test aid) */
+/* Bits 8..12 select the number of lanes that share one channel's 16 states
+ * (1, 2, 4, 8 or 16; 0 = chosen from the problem size).  A tuning knob: the
+ * result does not depend on it beyond fp32 rounding order. */
+#define BIMAMBA_LANES_SHIFT 8
+#define BIMAMBA_LANES_MASK  (0x1fu << BIMAMBA_LANES_SHIFT)
+
+/* Parameters of both directions, fp32 device pointers, index 0 = forward. */
+typedef struct {
+    const float *A;        /* [2][d_inner][d_state]   state matrix diagonal (negative) */
+    const float *D;        /* [2][d_inner]            skip weight                       */
+    const float *dt_bias;  /* [2][d_inner]            added to dt before softplus       */
+    const float *conv_w;   /* [2][d_inner][4]         conv taps, see the formula above  */
+    const float *conv_b;   /* [2][d_inner] or NULL    conv bias (NULL reads as 0)       */
+} bimamba_params_t;
+
+/* Layer inputs, device pointers of type `dtype`.  x and z are shared by the
+ * two directions; dt, B and C are per direction (dt[1] may equal dt[0], and
+ * likewise for B and C, to share them). */
+typedef struct {
+    const void *x;         /* [batch][L][d_inner]  */
+    const void *z;         /* [batch][L][d_inner]  */
+    const void *dt[2];     /* [batch][L][d_inner]  raw step size, before bias and softplus */
+    const void *B[2];      /* [batch][L][d_state]  */
+    const void *C[2];      /* [batch][L][d_state]  */
+    bimamba_dtype_t dtype;
+} bimamba_inputs_t;
+
+/* The cached forward state a block step starts from. */
+typedef struct {
+    float *h;              /* [batch][d_inner][d_state] fp32: forward scan state          */
+    void *conv_x;          /* [batch][3][d_inner] of the inputs' dtype: x of the last
+                              three prefix tokens, oldest first (zeros before token 0)   */
+} bimamba_fwd_state_t;
+
+/* Bytes of device workspace bimamba_layer_fwd needs: one fp32 per
+ * (batch, token, channel) for the half-sequence partial outputs the two
+ * directions hand each other.  Returns 0 for invalid sizes. */
+size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags);
+
+/* Full-sequence bidirectional layer (§3.2 Eq. (4)-(6)).
+ *   in          inputs; in->dtype is the input element type
+ *   p           parameters
+ *   out         [batch][L][d_inner] of out_dtype
+ *   workspace   >= bimamba_workspace_bytes(...) bytes of device memory, 16-byte
+ *               aligned, contents ignored on entry and undefined on exit
+ * One kernel launch. */
+int bimamba_layer_fwd(const bimamba_inputs_t *in, const bimamba_params_t *p,
+                      void *out, bimamba_dtype_t out_dtype,
+                      int batch, int64_t L, int d_inner, int d_state, unsigned flags,
+                      void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/* Forward-only scan over a prefix of P tokens from a zero state (§4.3: the
+ * cache a decoded block leaves behind).  Reads prefix->x, prefix->dt[0],
+ * prefix->B[0] (z, C and the reverse inputs are not read and may be NULL).
+ * Writes state_out->h and state_out->conv_x.  One kernel launch. */
+int bimamba_prefix_state(const bimamba_inputs_t *prefix, const bimamba_params_t *p,
+                         int batch, int64_t P, int d_inner, int d_state,
+                         bimamba_fwd_state_t *state_out, void *cuda_stream);
+
+/* One denoising step on the active block of block_len tokens (§4.3; the
+ * follow-up's abstract).  The forward direction starts from *prefix_state;
+ * the reverse direction sees the block alone (zero state after its last token,
+ * conv zero-padded past its end).  out: [batch][block_len][d_inner] of
+ * out_dtype.  If new_state is not NULL the forward state after the block is
+ * written there (commit); new_state may be prefix_state itself (in place).
+ * block_len must be in [1, 64].  One kernel launch. */
+int bimamba_block_step(const bimamba_fwd_state_t *prefix_state, const bimamba_inputs_t *block,
+                       int block_len, const bimamba_params_t *p,
+                       void *out, bimamba_dtype_t out_dtype,
+                       int batch, int d_inner, int d_state,
+                       bimamba_fwd_state_t *new_state, unsigned flags, void *cuda_stream);
+
+/* Human-readable text for a status code (static storage). */
+const char *bimamba_status_string(int status);
+
+/* ABI version: bumps when a signature or layout above changes. */
+int bimamba_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BIMAMBA_H */

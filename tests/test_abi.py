@@ -1,0 +1,178 @@
+"""The C ABI on the host: symbols, sizes and argument checks (no kernel runs).
+
+Every call here fails a check before anything is launched: the pointers are
+fake addresses that no code ever dereferences.  Each case breaks exactly one
+rule, and the rule checked before it is satisfied, so the expected status
+names the check that must fire.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bidirectional_mamba_denoiser_b200 import bimamba as bm
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bimamba.h")
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+NULL = object()        # "pass a NULL struct pointer"
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bimamba_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("bimamba_layer_fwd", "bimamba_prefix_state", "bimamba_block_step",
+              "bimamba_workspace_bytes", "bimamba_status_string", "bimamba_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(bm._LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_status_strings():
+    assert bm.lib.bimamba_abi_version() == 1
+    for s in (0, -1, -2, -3, -4, -5):
+        assert bm.status_string(s) and bm.status_string(s) != "unknown status"
+    assert bm.status_string(-99) == "unknown status"
+
+
+def test_workspace_bytes():
+    assert bm.bimamba_workspace_bytes(8, 2048, 4096) == 8 * 2048 * 4096 * 4
+    assert bm.bimamba_workspace_bytes(1, 1, 1) == 4
+    assert bm.bimamba_workspace_bytes(0, 10, 10) == 0
+    assert bm.bimamba_workspace_bytes(1, 0, 10) == 0
+    assert bm.bimamba_workspace_bytes(1, 10, 10, d_state=8) == 0
+
+
+def _inputs(dtype=bm.BIMAMBA_BF16, base=FAKE):
+    inp = bm.Inputs()
+    inp.x, inp.z = base, base + 0x1000
+    inp.dt[0], inp.dt[1] = base + 0x2000, base + 0x3000
+    inp.B[0], inp.B[1] = base + 0x4000, base + 0x5000
+    inp.C[0], inp.C[1] = base + 0x6000, base + 0x7000
+    inp.dtype = dtype
+    return inp
+
+
+def _params():
+    return bm.Params(FAKE + 0x10000, FAKE + 0x11000, FAKE + 0x12000, FAKE + 0x13000, FAKE + 0x14000)
+
+
+def _byref(s):
+    return None if s is NULL else ctypes.byref(s)
+
+
+def _layer(inp=None, par=None, out=FAKE + 0x20000, out_dtype=bm.BIMAMBA_BF16, batch=2, L=64, D=32, N=16,
+           flags=0, ws=FAKE + 0x30000, ws_bytes=None, broken=True):
+    # Refuse to issue a call in which nothing was broken: with every argument
+    # valid the library would launch a kernel on the fake addresses.
+    assert broken, "a validation case must break some argument"
+    inp = _inputs() if inp is None else inp
+    par = _params() if par is None else par
+    if ws_bytes is None:
+        ws_bytes = bm.bimamba_workspace_bytes(max(batch, 1), max(L, 1), max(D, 1)) or 16
+    return bm.lib.bimamba_layer_fwd(_byref(inp), _byref(par), out, out_dtype, batch, L, D, N, flags, ws,
+                                    ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(batch=70000), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(L=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(L=-5), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(D=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(out=None), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(N=8), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(N=32), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(flags=0x4), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(flags=3 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(out_dtype=7), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(inp=NULL), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(par=NULL), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(out=FAKE + 0x20001), bm.BIMAMBA_ERR_MISALIGNED),
+    (dict(ws=None), bm.BIMAMBA_ERR_WORKSPACE),
+    (dict(ws=FAKE + 0x30008), bm.BIMAMBA_ERR_WORKSPACE),
+    (dict(ws_bytes=100), bm.BIMAMBA_ERR_WORKSPACE),
+])
+def test_layer_rejects(kw, status):
+    assert kw
+    assert _layer(**kw) == status
+
+
+def test_layer_rejects_bad_inputs_and_params():
+    inp = _inputs()
+    inp.z = None
+    assert _layer(inp=inp) == bm.BIMAMBA_ERR_INVALID_ARG
+    inp = _inputs()
+    inp.C[1] = None
+    assert _layer(inp=inp) == bm.BIMAMBA_ERR_INVALID_ARG
+    inp = _inputs()
+    inp.dtype = 5
+    assert _layer(inp=inp) == bm.BIMAMBA_ERR_UNSUPPORTED
+    inp = _inputs()
+    inp.dt[1] = FAKE + 0x3001  # odd address for a 2-byte element
+    assert _layer(inp=inp) == bm.BIMAMBA_ERR_MISALIGNED
+    inp = _inputs(dtype=bm.BIMAMBA_F32)
+    inp.B[0] = FAKE + 0x4002  # 2-byte aligned, 4-byte element
+    assert _layer(inp=inp) == bm.BIMAMBA_ERR_MISALIGNED
+    par = _params()
+    par.A = None
+    assert _layer(par=par) == bm.BIMAMBA_ERR_INVALID_ARG
+    par = _params()
+    par.conv_w = FAKE + 0x13002
+    assert _layer(par=par) == bm.BIMAMBA_ERR_MISALIGNED
+
+
+def _state(h=FAKE + 0x40000, cx=FAKE + 0x41000):
+    return bm.FwdState(h, cx)
+
+
+def _prefix(inp=None, par=None, batch=2, P=64, D=32, N=16, st=None):
+    inp = _inputs() if inp is None else inp
+    par = _params() if par is None else par
+    st = _state() if st is None else st
+    return bm.lib.bimamba_prefix_state(_byref(inp), _byref(par), batch, P, D, N, _byref(st), None)
+
+
+def test_prefix_rejects():
+    assert _prefix(batch=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _prefix(P=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _prefix(N=4) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _prefix(st=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _prefix(st=_state(h=None)) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _prefix(st=_state(h=FAKE + 0x40002)) == bm.BIMAMBA_ERR_MISALIGNED
+    inp = _inputs()
+    inp.x = None
+    assert _prefix(inp=inp) == bm.BIMAMBA_ERR_INVALID_ARG
+
+
+def _block(st=None, inp=None, G=32, par=None, out=FAKE + 0x20000, out_dtype=bm.BIMAMBA_BF16, batch=2, D=32,
+           N=16, new=NULL, flags=0):
+    st = _state() if st is None else st
+    inp = _inputs() if inp is None else inp
+    par = _params() if par is None else par
+    return bm.lib.bimamba_block_step(_byref(st), _byref(inp), G, _byref(par), out, out_dtype, batch, D, N,
+                                     _byref(new), flags, None)
+
+
+def test_block_rejects():
+    assert _block(G=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(G=65) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _block(batch=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(N=15) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _block(out=None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(st=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(new=_state(cx=None)) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(new=_state(cx=FAKE + 0x41001)) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _block(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _block(flags=0x100000) == bm.BIMAMBA_ERR_UNSUPPORTED

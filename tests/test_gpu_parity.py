@@ -1,0 +1,235 @@
+"""The CUDA path (through the C ABI) against the fp64 oracle, on a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bidirectional_mamba_denoiser_b200 import workloads as W
+from tests import parity_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bm():
+    from bidirectional_mamba_denoiser_b200 import bimamba
+    return bimamba
+
+
+def run_layer(bm, inp, par, out_dtype, flags=0):
+    d = U.to_device(inp)
+    p = U.to_device(par)
+    out = bm.bimamba_layer_fwd(d["x"], d["z"], d["dt"], d["B"], d["C"], p, out_dtype=out_dtype, flags=flags)
+    torch.cuda.synchronize()
+    return U.to_cpu64(out)
+
+
+def test_tiny_fp32_case(bm):
+    """b=1, L=256, D=64, fp32 in and out, seed 0: normwise <= 1e-5."""
+    inp, par = W.make_workload(W.TINY)
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+@pytest.mark.parametrize("lanes", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 17, 24)])
+def test_bf16_ragged_every_lane_split(bm, shape, lanes):
+    """Ragged L (not a multiple of the 16-token chunk) and ragged D (not a
+    multiple of the channels a CTA covers), each lane split."""
+    b, L, D = shape
+    inp, par = W.make_case(b, L, D, 16, "bf16", seed=100 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = lanes << 8
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= U.GUARD
+    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+    assert U.bf16_out_ok(got16, ref)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 15, 16, 31, 32, 33])
+def test_short_sequences(bm, L):
+    inp, par = W.make_case(2, L, 16, 16, "fp32", seed=7 + L)
+    ref = oracle.layer_fwd(inp, par)
+    for lanes in (1, 4, 16):
+        got = run_layer(bm, inp, par, torch.float32, lanes << 8)
+        assert U.normwise(got, ref) <= U.TOL_FP32, (L, lanes)
+
+
+@pytest.mark.parametrize("flag", ["fwd", "rev"])
+def test_single_direction_flags(bm, flag):
+    """FWD_ONLY / REV_ONLY give y_0 * silu(z) / y_1 * silu(z) (Eq. (6) additivity)."""
+    inp, par = W.make_case(2, 130, 24, 16, "fp32", seed=3)
+    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
+    ref = oracle.layer_fwd(inp, par, flags=f)
+    got = run_layer(bm, inp, par, torch.float32, bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+def test_conv_bias_absent(bm):
+    inp, par = W.make_case(1, 90, 16, 16, "fp32", seed=4)
+    par = dict(par)
+    par["conv_b"] = None
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+def test_general_A_and_D(bm):
+    """A not of the S4D-real form and D != 1: nothing may rely on either."""
+    inp, par = W.make_case(2, 200, 40, 16, "fp32", seed=5)
+    g = torch.Generator().manual_seed(9)
+    par = dict(par)
+    par["A"] = -torch.exp(torch.rand(par["A"].shape, generator=g) * 5.0 - 3.0)
+    par["D"] = torch.rand(par["D"].shape, generator=g) * 2.0 - 1.0
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+def test_repeatable(bm):
+    """Same inputs, same bits: no reduction order depends on timing."""
+    inp, par = W.make_case(2, 300, 64, 16, "bf16", seed=6)
+    a = run_layer(bm, inp, par, torch.bfloat16)
+    b = run_layer(bm, inp, par, torch.bfloat16)
+    assert np.array_equal(a, b)
+
+
+def _sampled_layer_check(bm, w: W.Workload, nchan: int, flags=0):
+    inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device="cuda")
+    out32 = bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par,
+                                 out_dtype=torch.float32, flags=flags)
+    out16 = bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par,
+                                 out_dtype=torch.bfloat16, flags=flags)
+    torch.cuda.synchronize()
+    chans = U.sample_channels(w.d_inner, nchan, seed=w.seed)
+    si, sp = U.channel_subset(inp, par, chans)
+    ref = oracle.layer_fwd(si, sp)
+    idx = torch.as_tensor(chans, device="cuda")
+    g32 = U.to_cpu64(out32.index_select(-1, idx))
+    g16 = U.to_cpu64(out16.index_select(-1, idx))
+    return U.normwise(g32, ref), U.bf16_out_ok(g16, ref)
+
+
+def test_layer_1p3b_shape_sampled(bm):
+    """b=8, L=2048, D=4096, bf16, seed 1 -- the launch configuration the
+    bench times; 48 channels of every batch row against the oracle."""
+    err, ok16 = _sampled_layer_check(bm, W.LAYER_1P3B, 48)
+    assert err <= U.GUARD and ok16
+
+
+@pytest.mark.parametrize("L", [4096, 65536, 131072])
+def test_long_sequence_sampled(bm, L):
+    """b=1, D=4096, bf16, seed 2 at long L; 12 channels against the oracle."""
+    err, ok16 = _sampled_layer_check(bm, W.LONG_SEQ[L], 12)
+    assert err <= U.TOL_BF16 and ok16
+    assert err <= U.GUARD
+
+
+# ------------------------------------------------------------------ block step
+
+def _slice_tokens(inp, lo, hi):
+    return {k: (v[:, :, lo:hi] if k in ("dt", "B", "C") else v[:, lo:hi]).contiguous()
+            for k, v in inp.items() if v is not None}
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_block_chain_matches_oracle(bm, dtype):
+    """Prefix of 512 tokens, then 16 blocks of 32 committed one after another
+    (L = 1024 in all): every block's output and the committed state against
+    the oracle's own block chain."""
+    b, D, P, G = 2, 40, 512, 32
+    inp, par = W.make_case(b, P + 16 * G, D, 16, dtype, seed=21)
+    pre = _slice_tokens(inp, 0, P)
+    h_ref, t_ref = oracle.prefix_state(pre, par)
+    dpar = U.to_device(par)
+    dpre = U.to_device(pre)
+    h, tail = bm.bimamba_prefix_state(dpre["x"], dpre["dt"], dpre["B"], dpar)
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(h), h_ref) <= U.GUARD
+    assert np.array_equal(U.to_cpu64(tail), t_ref)
+    tol = U.TOL_FP32 if dtype == "fp32" else U.GUARD
+    for k in range(16):
+        blk = _slice_tokens(inp, P + k * G, P + (k + 1) * G)
+        ref, h_ref, t_ref = oracle.block_step(h_ref, t_ref, blk, par, commit=True)
+        dblk = U.to_device(blk)
+        out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
+                                    out_dtype=torch.float32, new_state=(h, tail))
+        torch.cuda.synchronize()
+        assert U.normwise(U.to_cpu64(out), ref) <= tol, k
+        assert U.normwise(U.to_cpu64(h), h_ref) <= U.GUARD, k
+        assert np.array_equal(U.to_cpu64(tail), t_ref), k
+
+
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 31, 33, 64])
+def test_block_step_ragged_lengths(bm, G):
+    b, D, P = 2, 24, 70
+    inp, par = W.make_case(b, P + G, D, 16, "fp32", seed=30 + G)
+    pre, blk = _slice_tokens(inp, 0, P), _slice_tokens(inp, P, P + G)
+    h_ref, t_ref = oracle.prefix_state(pre, par)
+    ref, h2_ref, t2_ref = oracle.block_step(h_ref, t_ref, blk, par, commit=True)
+    dpar, dpre, dblk = U.to_device(par), U.to_device(pre), U.to_device(blk)
+    h, tail = bm.bimamba_prefix_state(dpre["x"], dpre["dt"], dpre["B"], dpar)
+    h2, t2 = torch.empty_like(h), torch.empty_like(tail)
+    out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
+                                out_dtype=torch.float32, new_state=(h2, t2))
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(out), ref) <= U.TOL_FP32
+    assert U.normwise(U.to_cpu64(h2), h2_ref) <= U.TOL_FP32
+    assert np.array_equal(U.to_cpu64(t2), t2_ref)
+    # without commit the cached state is left alone
+    h_before = h.clone()
+    bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
+                          out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(h, h_before)
+
+
+def test_block_step_flags(bm):
+    b, D, P, G = 1, 16, 40, 32
+    inp, par = W.make_case(b, P + G, D, 16, "fp32", seed=41)
+    pre, blk = _slice_tokens(inp, 0, P), _slice_tokens(inp, P, P + G)
+    h_ref, t_ref = oracle.prefix_state(pre, par)
+    dpar, dpre, dblk = U.to_device(par), U.to_device(pre), U.to_device(blk)
+    h, tail = bm.bimamba_prefix_state(dpre["x"], dpre["dt"], dpre["B"], dpar)
+    for f_or, f_bm in ((oracle.FWD_ONLY, bm.BIMAMBA_FWD_ONLY), (oracle.REV_ONLY, bm.BIMAMBA_REV_ONLY)):
+        ref = oracle.block_step(h_ref, t_ref, blk, par, flags=f_or)
+        out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
+                                    out_dtype=torch.float32, flags=f_bm)
+        torch.cuda.synchronize()
+        assert U.normwise(U.to_cpu64(out), ref) <= U.TOL_FP32
+
+
+def test_block_cached_full_prefix_sampled(bm):
+    """b=16, P=65536, D=4096, bf16: the prefix state over the full prefix and
+    two committed block steps of 32 tokens, on 8 sampled channels."""
+    w = W.BLOCK_CACHED
+    P, G = w.extra["prefix"], w.extra["block"]
+    inp, par = W.make_case(w.batch, P + 2 * G, w.d_inner, 16, "bf16", w.seed, device="cuda")
+    pre = {"x": inp["x"][:, :P], "dt": inp["dt"][0, :, :P].contiguous(), "B": inp["B"][0, :, :P].contiguous()}
+    h, tail = bm.bimamba_prefix_state(pre["x"].contiguous(), pre["dt"], pre["B"], par)
+    chans = U.sample_channels(w.d_inner, 8, seed=5)
+    idx = torch.as_tensor(chans, device="cuda")
+    si, sp = U.channel_subset(inp, par, chans)
+    spre = _slice_tokens(si, 0, P)
+    h_ref, t_ref = oracle.prefix_state(spre, sp)
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(h.index_select(1, idx)), h_ref) <= U.GUARD
+    assert np.array_equal(U.to_cpu64(tail.index_select(-1, idx)), t_ref)
+    for k in range(2):
+        blk = _slice_tokens(inp, P + k * G, P + (k + 1) * G)
+        out = bm.bimamba_block_step((h, tail), blk["x"], blk["z"], blk["dt"], blk["B"], blk["C"], par,
+                                    out_dtype=torch.float32, new_state=(h, tail))
+        sblk = _slice_tokens(si, P + k * G, P + (k + 1) * G)
+        ref, h_ref, t_ref = oracle.block_step(h_ref, t_ref, sblk, sp, commit=True)
+        torch.cuda.synchronize()
+        assert U.normwise(U.to_cpu64(out.index_select(-1, idx)), ref) <= U.GUARD
+        assert U.normwise(U.to_cpu64(h.index_select(1, idx)), h_ref) <= U.GUARD
+
+
+def test_workspace_too_small_is_rejected(bm):
+    inp, par = W.make_case(1, 64, 16, 16, "bf16", seed=1, device="cuda")
+    ws = torch.empty(100, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bm.BimambaError) as e:
+        bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, workspace=ws)
+    assert e.value.status == bm.BIMAMBA_ERR_WORKSPACE
