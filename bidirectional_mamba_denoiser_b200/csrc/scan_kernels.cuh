@@ -211,18 +211,22 @@ struct DirScan {
         __syncwarp();
     }
 
-    // Stage x and B/C rows of steps [0, n) (token tc + dir * s).
+    // Stage x and B (and, with LOAD_C, C) rows of steps [0, n) (token
+    // tc + dir * s).  Without LOAD_C the C pointer is never dereferenced.
+    template <bool LOAD_C>
     __device__ __forceinline__ void stage(int64_t tc, int dir, int n) {
         for (int e = lane; e < n * Ge::CPW; e += 32) {
             const int s = e / Ge::CPW, cc = e % Ge::CPW;
             const int64_t t = tc + (int64_t)dir * s;
             xs[(3 + s) * Ge::CPW + cc] = (c0 + cc < D) ? ldf(X, (rowbase + t) * D + c0 + cc) : 0.f;
         }
-        const Tin* src = (lane < kNState) ? Bp : Cp;
-        const int col = lane & (kNState - 1);
-        for (int s = 0; s < n; ++s) {
-            const int64_t t = tc + (int64_t)dir * s;
-            bc[s * 2 * kNState + lane] = ldf(src, (rowbase + t) * kNState + col);
+        if (LOAD_C || lane < kNState) {
+            const Tin* src = (lane < kNState) ? Bp : Cp;
+            const int col = lane & (kNState - 1);
+            for (int s = 0; s < n; ++s) {
+                const int64_t t = tc + (int64_t)dir * s;
+                bc[s * 2 * kNState + lane] = ldf(src, (rowbase + t) * kNState + col);
+            }
         }
         __syncwarp();
     }
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(2 * WPD * 32) layer_kernel(const KParams p) {
         for (int64_t done = 0; done < count; done += T) {
             const int n = (int)((count - done < T) ? (count - done) : T);
             const int64_t tc = tstart + dir * done;
-            sc.stage(tc, dir, n);
+            sc.template stage<true>(tc, dir, n);
             float du[Ge::EPL], yv[Ge::EPL];
             sc.elements(tc, dir, n, du);
             sc.template scan<true>(n, yv);
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(WPB * 32) prefix_kernel(const KParams p) {
 #pragma unroll 1
     for (int64_t done = 0; done < P; done += T) {
         const int n = (int)((P - done < T) ? (P - done) : T);
-        sc.stage(done, 1, n);
+        sc.template stage<false>(done, 1, n);
         float du[Ge::EPL], yv[Ge::EPL];
         sc.elements(done, 1, n, du);
         sc.template scan<false>(n, yv);
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(WPB * 32) block_kernel(const KParams p) {
     }
     __syncwarp();
     {
-        sc.stage(0, 1, n);
+        sc.template stage<true>(0, 1, n);
         float du[Ge::EPL], yv[Ge::EPL];
         sc.elements(0, 1, n, du);
         sc.template scan<true>(n, yv);
@@ -477,7 +481,7 @@ __global__ void __launch_bounds__(WPB * 32) block_kernel(const KParams p) {
     sc.set_direction(p, 1);
     {
         const int64_t tc = n - 1;
-        sc.stage(tc, -1, n);
+        sc.template stage<true>(tc, -1, n);
         float du[Ge::EPL], yv[Ge::EPL];
         sc.elements(tc, -1, n, du);
         sc.template scan<true>(n, yv);
