@@ -30,6 +30,7 @@ BIMAMBA_BF16 = 1
 BIMAMBA_FWD_ONLY = 0x1
 BIMAMBA_REV_ONLY = 0x2
 BIMAMBA_LANES_SHIFT = 8
+BIMAMBA_NO_TMA = 0x4000
 
 D_STATE = 16
 
@@ -74,10 +75,17 @@ def _load():
     lib.bimamba_status_string.argtypes = [I]
     lib.bimamba_status_string.restype = ctypes.c_char_p
     lib.bimamba_abi_version.restype = I
+    lib.bimamba_device_error.argtypes = [I]
+    lib.bimamba_device_error.restype = I
     return lib
 
 
 lib = _load()
+
+
+def bimamba_device_error(reset: bool = True) -> int:
+    """The device error word (0 = no kernel gave up waiting); synchronises."""
+    return int(lib.bimamba_device_error(1 if reset else 0))
 
 
 def status_string(status: int) -> str:

@@ -1,12 +1,15 @@
 // bimamba_api.cu -- the C ABI (include/bimamba.h): argument checks, launch
 // shapes and kernel dispatch.  All arithmetic lives in scan_kernels.cuh.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 #include <set>
+#include <type_traits>
 #include <utility>
 
 #include "bimamba.h"
+#include "layer_tma.cuh"
 #include "scan_kernels.cuh"
 
 namespace {
@@ -165,6 +168,139 @@ int block_by_lanes(int g, const KParams& k, cudaStream_t st) {
     return BIMAMBA_ERR_UNSUPPORTED;
 }
 
+// ---- TMA-fed kernels
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// 3-D map over a [batch][rows][inner] row-major tensor; the box is
+// {box_inner, box_rows, 1}; out-of-range elements of a box read as zero.
+bool map3d(CUtensorMap* m, const void* ptr, bool is_bf16, uint64_t inner, uint64_t rows, uint64_t batch,
+           uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    const uint64_t esz = is_bf16 ? 2 : 4;
+    cuuint64_t dims[3] = {inner, rows, batch};
+    cuuint64_t strides[2] = {inner * esz, inner * rows * esz};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+             const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tma_eligible(const bimamba_inputs_t* in, int d_inner, bool need_reverse, bool need_z_c) {
+    const size_t esz = elem_size(in->dtype);
+    if ((d_inner * esz) % 16 != 0) return false;
+    const void* ptrs[8] = {in->x, in->dt[0], in->B[0], need_z_c ? in->z : in->x, need_z_c ? in->C[0] : in->x,
+                           need_reverse ? in->dt[1] : in->x, need_reverse ? in->B[1] : in->x,
+                           need_reverse ? in->C[1] : in->x};
+    for (const void* q : ptrs)
+        if (!aligned(q, 16)) return false;
+    return true;
+}
+
+constexpr int kTT = 32;  // tokens per chunk of the TMA kernels
+constexpr int kTWD = 4;  // warps per direction per CTA
+constexpr int kTNS = 2;  // pipeline stages
+
+template <int G, typename Tin>
+bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool reverse,
+               bool gated) {
+    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    const bool bf = std::is_same<Tin, bf16>::value;
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, kTT + 3);
+    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, Ge::CW, kTT);
+    ok = ok && map3d(&m.B[0], in->B[0], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+    if (gated) {
+        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, kTT);
+        ok = ok && map3d(&m.C[0], in->C[0], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+    } else {
+        m.z = m.x;
+        m.C[0] = m.B[0];
+    }
+    if (reverse) {
+        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, Ge::CW, kTT);
+        ok = ok && map3d(&m.B[1], in->B[1], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+        ok = ok && map3d(&m.C[1], in->C[1], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+    } else {
+        m.dt[1] = m.dt[0];
+        m.B[1] = m.B[0];
+        m.C[1] = m.C[0];
+    }
+    return ok;
+}
+
+template <int G, typename Tin, typename Tout>
+int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    bimamba::LayerMaps maps;
+    if (!fill_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::layer_tma_kernel<G, kTT, kTWD, kTNS, Tin, Tout>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, 2 * kTWD * 32, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+int layer_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    switch (g) {
+        case 4: return launch_layer_tma<4, Tin, Tout>(k, in, st);
+        case 8: return launch_layer_tma<8, Tin, Tout>(k, in, st);
+        case 16: return launch_layer_tma<16, Tin, Tout>(k, in, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+template <int G, typename Tin>
+int launch_prefix_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    bimamba::LayerMaps maps;
+    if (!fill_maps<G, Tin>(maps, in, k.batch, k.L, k.D, false, false)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::prefix_tma_kernel<G, kTT, kTWD, kTNS, Tin>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, kTWD * 32, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+template <typename Tin>
+int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    switch (g) {
+        case 4: return launch_prefix_tma<4, Tin>(k, in, st);
+        case 8: return launch_prefix_tma<8, Tin>(k, in, st);
+        case 16: return launch_prefix_tma<16, Tin>(k, in, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+// Lanes per channel of the TMA kernels: 4, 8 or 16 (same rule as pick_lanes).
+int pick_lanes_tma(int64_t chains, unsigned flags) {
+    const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    if (forced) return (int)forced;
+    const int64_t target = 148LL * 1024;
+    int g = 4;
+    while (g < 16 && chains * g < target) g *= 2;
+    return g;
+}
+
 int check_inputs(const bimamba_inputs_t* in, bool need_reverse, bool need_z_c) {
     if (!in || !in->x || !in->dt[0] || !in->B[0]) return BIMAMBA_ERR_INVALID_ARG;
     if (need_z_c && (!in->z || !in->C[0])) return BIMAMBA_ERR_INVALID_ARG;
@@ -205,6 +341,16 @@ const char* bimamba_status_string(int status) {
     return "unknown status";
 }
 
+int bimamba_device_error(int reset) {
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, bimamba::g_device_error, sizeof(word)) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(bimamba::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    }
+    return (int)word;
+}
+
 size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags) {
     (void)flags;
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || d_state != bimamba::kNState) return 0;
@@ -216,7 +362,7 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
                       unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
-    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK;
+    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -238,9 +384,17 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     k.batch = batch;
     k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
-    const int g = pick_lanes(2LL * batch * d_inner, flags);
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
+        const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
+        if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, k, in, st);
+        if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, k, in, st);
+        if (out_bf) return layer_tma_by_lanes<float, bf16>(gt, k, in, st);
+        return layer_tma_by_lanes<float, float>(gt, k, in, st);
+    }
+    const int g = pick_lanes(2LL * batch * d_inner, flags);
     if (in_bf && out_bf) return layer_by_lanes<bf16, bf16>(g, k, st);
     if (in_bf) return layer_by_lanes<bf16, float>(g, k, st);
     if (out_bf) return layer_by_lanes<float, bf16>(g, k, st);
@@ -267,8 +421,13 @@ int bimamba_prefix_state(const bimamba_inputs_t* prefix, const bimamba_params_t*
     k.D = d_inner;
     k.batch = batch;
     k.dir_scale[0] = k.dir_scale[1] = 1.f;
-    const int g = pick_lanes((int64_t)batch * d_inner, 0);
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (tma_eligible(prefix, d_inner, false, false)) {
+        const int gt = pick_lanes_tma((int64_t)batch * d_inner, 0);
+        if (prefix->dtype == BIMAMBA_BF16) return prefix_tma_by_lanes<bf16>(gt, k, prefix, st);
+        return prefix_tma_by_lanes<float>(gt, k, prefix, st);
+    }
+    const int g = pick_lanes((int64_t)batch * d_inner, 0);
     if (prefix->dtype == BIMAMBA_BF16) return prefix_by_lanes<bf16>(g, k, st);
     return prefix_by_lanes<float>(g, k, st);
 }

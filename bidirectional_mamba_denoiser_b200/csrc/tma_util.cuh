@@ -1,0 +1,82 @@
+// tma_util.cuh -- sm_100a tensor-memory-accelerator (TMA) loads, mbarriers and
+// named barriers, in inline PTX.
+//
+// Only plain (non-multicast) TMA loads are issued: every tile is fetched by
+// the CTA that uses it, from this GPU's own memory.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace bimamba {
+
+// Error word of the library on each device (bit flags, see kErr*).  A wait
+// that gives up sets a bit here instead of hanging; the host reads it with
+// bimamba_device_error().
+__device__ unsigned int g_device_error;
+constexpr unsigned kErrTmaTimeout = 1u;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async proxy (TMA unit).
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of the barrier to complete, for at most about
+// `limit_cycles` SM clocks.  On timeout the device error word records it and
+// the caller carries on (its data is then garbage, but every thread still
+// reaches every later barrier, so the kernel ends).
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  long long limit_cycles = 4000000000LL) {
+    if (mbar_try_wait(bar, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit_cycles) {
+            atomicOr(&g_device_error, kErrTmaTimeout);
+            return;
+        }
+    }
+}
+
+// 3-D tiled TMA load into shared memory, completing on `bar` (transaction
+// bytes).  Coordinates are element indices, innermost first; a box that
+// reaches outside the tensor reads zeros there.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+}  // namespace bimamba

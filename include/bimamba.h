@@ -66,6 +66,11 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * result does not depend on it beyond fp32 rounding order. */
 #define BIMAMBA_LANES_SHIFT 8
 #define BIMAMBA_LANES_MASK  (0x1fu << BIMAMBA_LANES_SHIFT)
+/* Use the kernel that stages tiles with ordinary loads instead of the
+ * TMA-fed one (test aid; the TMA kernel is otherwise chosen whenever every
+ * x/z/dt/B/C pointer is 16-byte aligned and a row of d_inner elements is a
+ * whole number of 16-byte units). */
+#define BIMAMBA_NO_TMA      0x4000u
 
 /* Parameters of both directions, fp32 device pointers, index 0 = forward. */
 typedef struct {
@@ -132,6 +137,13 @@ int bimamba_block_step(const bimamba_fwd_state_t *prefix_state, const bimamba_in
                        void *out, bimamba_dtype_t out_dtype,
                        int batch, int d_inner, int d_state,
                        bimamba_fwd_state_t *new_state, unsigned flags, void *cuda_stream);
+
+/* Read (and, if reset != 0, clear) the error word of the current device.
+ * Kernels never wait without bound: a wait for a tile that gives up after
+ * about two seconds sets bit 0 (a tile load that never arrived) and the kernel
+ * finishes with undefined output instead of hanging.  Synchronises the
+ * device.  Returns the word, or BIMAMBA_ERR_CUDA if it cannot be read. */
+int bimamba_device_error(int reset);
 
 /* Human-readable text for a status code (static storage). */
 const char *bimamba_status_string(int status);

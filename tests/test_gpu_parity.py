@@ -24,36 +24,66 @@ def run_layer(bm, inp, par, out_dtype, flags=0):
     return U.to_cpu64(out)
 
 
-def test_tiny_fp32_case(bm):
-    """b=1, L=256, D=64, fp32 in and out, seed 0: normwise <= 1e-5."""
+@pytest.mark.parametrize("flags", [0, 0x4000])
+def test_tiny_fp32_case(bm, flags):
+    """b=1, L=256, D=64, fp32 in and out, seed 0: normwise <= 1e-5 (both kernels)."""
     inp, par = W.make_workload(W.TINY)
     ref = oracle.layer_fwd(inp, par)
-    got = run_layer(bm, inp, par, torch.float32)
+    got = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got, ref) <= U.TOL_FP32
 
 
 @pytest.mark.parametrize("lanes", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 17, 24)])
-def test_bf16_ragged_every_lane_split(bm, shape, lanes):
-    """Ragged L (not a multiple of the 16-token chunk) and ragged D (not a
-    multiple of the channels a CTA covers), each lane split."""
+def test_bf16_ragged_staged_kernel(bm, shape, lanes):
+    """The kernel without TMA staging: ragged L (not a multiple of its
+    16-token chunk) and ragged D (not a multiple of a CTA's channels), each
+    lane split."""
     b, L, D = shape
     inp, par = W.make_case(b, L, D, 16, "bf16", seed=100 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    flags = lanes << 8
+    flags = (lanes << 8) | bm.BIMAMBA_NO_TMA
     got32 = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got32, ref) <= U.GUARD
     got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
     assert U.bf16_out_ok(got16, ref)
 
 
-@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 15, 16, 31, 32, 33])
+@pytest.mark.parametrize("lanes", [4, 8, 16])
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 32, 32), (1, 64, 48), (1, 65, 8)])
+def test_bf16_ragged_tma_kernel(bm, shape, lanes):
+    """The TMA-fed kernel (32-token chunks): one, two and three chunks, a
+    ragged last chunk, and channel counts that leave the last CTA's tile
+    partly empty."""
+    b, L, D = shape
+    inp, par = W.make_case(b, L, D, 16, "bf16", seed=200 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = lanes << 8
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= U.GUARD
+    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+    assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
+def test_unaligned_channel_count_uses_staged_kernel(bm):
+    """d_inner = 20: a bf16 row is not a whole number of 16-byte units, so
+    the library must take the kernel without TMA -- and still be right."""
+    inp, par = W.make_case(2, 70, 20, 16, "bf16", seed=11)
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32)
+    assert U.normwise(got, ref) <= U.GUARD
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 15, 16, 31, 32, 33, 63, 64, 65, 96, 97])
 def test_short_sequences(bm, L):
     inp, par = W.make_case(2, L, 16, 16, "fp32", seed=7 + L)
     ref = oracle.layer_fwd(inp, par)
-    for lanes in (1, 4, 16):
-        got = run_layer(bm, inp, par, torch.float32, lanes << 8)
-        assert U.normwise(got, ref) <= U.TOL_FP32, (L, lanes)
+    for flags in (1 << 8 | bm.BIMAMBA_NO_TMA, 4 << 8 | bm.BIMAMBA_NO_TMA, 16 << 8 | bm.BIMAMBA_NO_TMA,
+                  4 << 8, 8 << 8, 16 << 8):
+        got = run_layer(bm, inp, par, torch.float32, flags)
+        assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
 
 
 @pytest.mark.parametrize("flag", ["fwd", "rev"])
