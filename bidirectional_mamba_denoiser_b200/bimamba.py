@@ -31,6 +31,7 @@ BIMAMBA_FWD_ONLY = 0x1
 BIMAMBA_REV_ONLY = 0x2
 BIMAMBA_LANES_SHIFT = 8
 BIMAMBA_NO_TMA = 0x4000
+BIMAMBA_CHUNK_SHIFT = 16
 
 D_STATE = 16
 

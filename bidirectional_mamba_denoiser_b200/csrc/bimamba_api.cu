@@ -214,29 +214,28 @@ bool tma_eligible(const bimamba_inputs_t* in, int d_inner, bool need_reverse, bo
     return true;
 }
 
-constexpr int kTT = 32;  // tokens per chunk of the TMA kernels
 constexpr int kTWD = 4;  // warps per direction per CTA
 constexpr int kTNS = 2;  // pipeline stages
 
-template <int G, typename Tin>
+template <int G, int T, typename Tin>
 bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool reverse,
                bool gated) {
-    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
     const bool bf = std::is_same<Tin, bf16>::value;
-    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, kTT + 3);
-    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, Ge::CW, kTT);
-    ok = ok && map3d(&m.B[0], in->B[0], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, T + 3);
+    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, Ge::CW, T);
+    ok = ok && map3d(&m.B[0], in->B[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     if (gated) {
-        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, kTT);
-        ok = ok && map3d(&m.C[0], in->C[0], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, T);
+        ok = ok && map3d(&m.C[0], in->C[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     } else {
         m.z = m.x;
         m.C[0] = m.B[0];
     }
     if (reverse) {
-        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, Ge::CW, kTT);
-        ok = ok && map3d(&m.B[1], in->B[1], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
-        ok = ok && map3d(&m.C[1], in->C[1], bf, bimamba::kNState, L, batch, bimamba::kNState, kTT);
+        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, Ge::CW, T);
+        ok = ok && map3d(&m.B[1], in->B[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
+        ok = ok && map3d(&m.C[1], in->C[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     } else {
         m.dt[1] = m.dt[0];
         m.B[1] = m.B[0];
@@ -245,12 +244,12 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
-template <int G, typename Tin, typename Tout>
+template <int G, int T, typename Tin, typename Tout>
 int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
     bimamba::LayerMaps maps;
-    if (!fill_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_tma_kernel<G, kTT, kTWD, kTNS, Tin, Tout>;
+    if (!fill_maps<G, T, Tin>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::layer_tma_kernel<G, T, kTWD, kTNS, Tin, Tout>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -259,21 +258,30 @@ int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t 
 }
 
 template <typename Tin, typename Tout>
-int layer_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    switch (g) {
-        case 4: return launch_layer_tma<4, Tin, Tout>(k, in, st);
-        case 8: return launch_layer_tma<8, Tin, Tout>(k, in, st);
-        case 16: return launch_layer_tma<16, Tin, Tout>(k, in, st);
+int layer_tma_by_lanes(int g, int t, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    if (t == 16) {
+        switch (g) {
+            case 4: return launch_layer_tma<4, 16, Tin, Tout>(k, in, st);
+            case 8: return launch_layer_tma<8, 16, Tin, Tout>(k, in, st);
+            case 16: return launch_layer_tma<16, 16, Tin, Tout>(k, in, st);
+        }
+    } else {
+        switch (g) {
+            case 4: return launch_layer_tma<4, 32, Tin, Tout>(k, in, st);
+            case 8: return launch_layer_tma<8, 32, Tin, Tout>(k, in, st);
+            case 16: return launch_layer_tma<16, 32, Tin, Tout>(k, in, st);
+        }
     }
     return BIMAMBA_ERR_UNSUPPORTED;
 }
 
 template <int G, typename Tin>
 int launch_prefix_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::TmaGeo<G, kTT, kTWD, kTNS, Tin>;
+    constexpr int T = 32;
+    using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
     bimamba::LayerMaps maps;
-    if (!fill_maps<G, Tin>(maps, in, k.batch, k.L, k.D, false, false)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::prefix_tma_kernel<G, kTT, kTWD, kTNS, Tin>;
+    if (!fill_maps<G, T, Tin>(maps, in, k.batch, k.L, k.D, false, false)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::prefix_tma_kernel<G, T, kTWD, kTNS, Tin>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -289,6 +297,12 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
         case 16: return launch_prefix_tma<16, Tin>(k, in, st);
     }
     return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+// Chunk length of the TMA kernel: forced by the flags, else 32.
+int pick_chunk_tma(unsigned flags) {
+    const unsigned f = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
+    return f == 1 ? 16 : 32;
 }
 
 // Lanes per channel of the TMA kernels: 4, 8 or 16 (same rule as pick_lanes).
@@ -362,7 +376,9 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
                       unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
-    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA;
+    const unsigned known =
+        BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA | BIMAMBA_CHUNK_MASK;
+    if (((flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -389,10 +405,11 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
         const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
-        if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, k, in, st);
-        if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, k, in, st);
-        if (out_bf) return layer_tma_by_lanes<float, bf16>(gt, k, in, st);
-        return layer_tma_by_lanes<float, float>(gt, k, in, st);
+        const int tt = pick_chunk_tma(flags);
+        if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, tt, k, in, st);
+        if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, tt, k, in, st);
+        if (out_bf) return layer_tma_by_lanes<float, bf16>(gt, tt, k, in, st);
+        return layer_tma_by_lanes<float, float>(gt, tt, k, in, st);
     }
     const int g = pick_lanes(2LL * batch * d_inner, flags);
     if (in_bf && out_bf) return layer_by_lanes<bf16, bf16>(g, k, st);

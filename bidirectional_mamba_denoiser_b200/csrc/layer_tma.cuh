@@ -4,24 +4,34 @@
 //
 // One CTA = one batch row x CW channels.  Warps [0, NWD) run the forward
 // direction and warps [NWD, 2*NWD) the reverse direction over the same
-// channels; each warp covers CPW = 32/G channels with G lanes per channel.
+// channels; each warp covers CPW = 32/G channels with G lanes per channel,
+// each lane holding S = 16/G of a channel's states.
 //
-// Per direction the sequence is cut into chunks of T tokens on one grid
-// shared by both directions (chunk k = tokens [kT, kT+T)).  Each chunk's x
-// (with the 3-token conv halo), dt, B, C -- and z when the chunk is gated --
-// arrive by 3-D TMA loads into an NS-stage shared-memory ring; a box that
-// reaches outside [0, L) is zero-filled, which is exactly the conv's zero
-// padding at the sequence ends.  Per chunk the direction's warps convert B/C
-// to fp32 pairs once (shared by all its channels), meet at one named
-// barrier, and the group leader then refills the stage the previous chunk
-// used (every warp of the group is past it).  Tokens >= L in the last chunk
-// get delta = 0 and zero drive, so their scan step is the identity.
+// Both directions cut the sequence into the same chunks of T tokens
+// (chunk k = tokens [kT, kT+T)) and walk them in "step space": step s of
+// chunk k is token kT + s (forward) or kT + T-1-s (reverse), so the reverse
+// conv is the causal conv over tokens read backwards; nothing is flipped in
+// memory.  Each chunk's x (with the 3-token conv halo), dt, B, C -- and z
+// when the chunk is gated -- arrive by 3-D TMA loads into an NS-stage
+// shared-memory ring; a box reaching outside [0, L) reads zeros, which is
+// the conv's zero padding at both sequence ends.  Per chunk a direction's
+// warps convert B/C to fp32 once (shared by all its channels) and meet at
+// one named barrier, after which the group leader refills the stage the
+// previous chunk used.  Steps whose token is >= L get delta = 0 and no
+// drive, so they leave the state exactly unchanged.
 //
-// Full layer: the forward group walks chunks 0..nc-1 and the reverse group
-// nc-1..0.  Chunks [0, nc/2) are the forward group's first half and the
-// rest the reverse group's; each stores its fp32 y over its first half to
-// the workspace, both groups meet at one barrier, and each then finishes the
-// other half, adding the partner's y and applying the SiLU(z) gate.
+// Per chunk a warp (1) computes conv + SiLU, softplus and D*u for its
+// elements into shared memory, (2) advances its states step by step with
+// packed f32x2 arithmetic and one MUFU exp2 per state, and after every G
+// steps combines the C.h partial sums across the G lanes (shuffle
+// transpose-reduce) so that each lane owns one finished step, which it
+// writes out at once.
+//
+// Full layer: the forward group walks chunks 0..nc-1, the reverse group
+// nc-1..0.  Until they meet (the forward group after nc/2 chunks) each
+// stores its fp32 y to the workspace; after one CTA barrier each finishes
+// the other half, adding the partner's y (fetched by cp.async) and applying
+// the SiLU(z) gate.
 #pragma once
 
 #include "scan_kernels.cuh"
@@ -41,6 +51,7 @@ constexpr int align128(int v) { return (v + 127) & ~127; }
 
 template <int G, int T, int NWD, int NS, typename Tin>
 struct TmaGeo {
+    static_assert(G == 4 || G == 8 || G == 16, "lanes per channel");
     static_assert(T % G == 0 && T <= 253, "chunk");
     static constexpr int CPW = 32 / G;                    // channels per warp
     static constexpr int S = kNState / G;                 // states per lane
@@ -51,28 +62,62 @@ struct TmaGeo {
     static constexpr int DTB = align128(T * CW * ESZ);
     static constexpr int BB = align128(T * kNState * ESZ);
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;   // x, dt, z, B, C
-    static constexpr int BC32 = T * kNState * 2 * 4;      // one fp32 (B, C) pair buffer
-    static constexpr int ED = T * CPW * 8;                // per warp: (delta, delta*u)
+    static constexpr int BC32 = T * kNState * 2 * 4;      // one fp32 B/C buffer
+    static constexpr int ED2 = T * CPW * 8;               // per warp: (delta, delta*u)
+    static constexpr int EDU = T * CPW * 4;               // per warp: D*u
+    static constexpr int OWS = T * CPW * 4;               // per warp: partner's y
+    static constexpr int WARP_BYTES = ED2 + EDU + OWS;
     static constexpr int DIR_BYTES = NS * STAGE + 2 * BC32;
-    static constexpr int BAR_OFF = 2 * DIR_BYTES + 2 * NWD * ED;
+    static constexpr int WARP_OFF = 2 * DIR_BYTES;
+    static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;  // + alignment slack
     static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
     static constexpr uint32_t TX_Z = (uint32_t)(T * CW * ESZ);
     static_assert((CW * ESZ) % 16 == 0, "TMA box rows must be whole 16-byte units");
 };
 
-// Per-lane state of one warp scanning one direction over CPW channels.
+// fp32 B/C layout per token: 8 quads (B_2p, B_2p+1, C_2p, C_2p+1), so that a
+// lane's state pairs and their B and C are register pairs.
+__device__ __forceinline__ int bc_quad_index(int n) { return (n >> 1) * 4 + (n & 1); }
+
+template <int T, typename Tin>
+__device__ __forceinline__ void convert_bc(const Tin* Bt, const Tin* Ct, float* bc, int tid, int nthreads,
+                                           bool with_c) {
+    for (int e = tid; e < T * kNState; e += nthreads) {
+        const int row = e >> 4, n = e & 15;
+        float* q = bc + row * 2 * kNState + bc_quad_index(n);
+        q[0] = ldf(Bt, e);
+        if (with_c) q[2] = ldf(Ct, e);
+    }
+}
+
+// Asynchronous global -> shared copy of BYTES (8 or 16; both addresses
+// aligned to BYTES); with pred false nothing is read and zeros are written.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void* dst, const void* src, bool pred) {
+    static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
+    const int n = pred ? BYTES : 0;
+    if constexpr (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
+                     : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
+                     : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// One warp's scan of one direction over CPW channels.
 template <int G, int T, int NWD, int NS, typename Tin, int DIR>
 struct TmaWorker {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
-    int lane, c, j, d, cc;  // cc: channel index inside the CTA tile
+    int c, j, cc, d;  // cc: channel inside the CTA tile; d: global channel
     bool dvalid;
-    float A2[Ge::S];
+    float A2[Ge::S];  // A * log2(e) of this lane's states
     float w[4], cb, bias, Dd;
     float h[Ge::S];
 
-    __device__ __forceinline__ void setup(const KParams& p, int ct0, int wg, int lane_) {
-        lane = lane_;
+    __device__ __forceinline__ void setup(const KParams& p, int ct0, int wg, int lane) {
         c = lane % Ge::CPW;
         j = lane / Ge::CPW;
         cc = wg * Ge::CPW + c;
@@ -91,74 +136,71 @@ struct TmaWorker {
         Dd = dvalid ? p.Dskip[rd] : 0.f;
     }
 
-    // token of step s of chunk k
-    __device__ __forceinline__ int64_t token(int k, int s) const {
-        return DIR == 0 ? (int64_t)k * T + s : (int64_t)k * T + (T - 1 - s);
-    }
+    // tile row (token - kT) of step s
+    static __device__ __forceinline__ int row_of(int s) { return DIR == 0 ? s : T - 1 - s; }
 
-    // conv + SiLU and softplus of this lane's steps; (delta, delta*u) to ed,
-    // D*u to du.  Steps whose token is >= L become identity steps.
-    __device__ __forceinline__ void elements(const Tin* xt, const Tin* dtt, int k, int64_t L, float2* ed,
-                                             float (&du)[Ge::EPL]) {
-#pragma unroll
+    // conv + SiLU and softplus of this lane's steps j, j+G, ...; steps
+    // outside [s_lo, s_hi) (tokens >= L) become identity steps.
+    __device__ __forceinline__ void elements(const Tin* xt, const Tin* dtt, int s_lo, int s_hi, float2* ed2,
+                                             float* edu) {
+#pragma unroll 2
         for (int e = 0; e < Ge::EPL; ++e) {
             const int s = j + G * e;
-            const bool valid = token(k, s) < L;
+            // step s-3+q is x-tile row s+q (forward) or T+2-s-q (reverse)
             float cv = cb;
-            if (DIR == 0) {
-                // tile row rho holds token kT - 3 + rho: taps t-3..t are rows s..s+3
 #pragma unroll
-                for (int q = 0; q < 4; ++q) cv = fmaf(w[q], ldf(xt, (s + q) * Ge::CW + cc), cv);
-            } else {
-                // tile row rho holds token kT + rho; token t = kT + T-1-s; tap q reads t+3-q
-#pragma unroll
-                for (int q = 0; q < 4; ++q) cv = fmaf(w[q], ldf(xt, (T + 2 - s - q) * Ge::CW + cc), cv);
+            for (int q = 0; q < 4; ++q) {
+                const int xr = DIR == 0 ? s + q : T + 2 - s - q;
+                cv = fmaf(w[q], ldf(xt, xr * Ge::CW + cc), cv);
             }
-            const int trow = DIR == 0 ? s : T - 1 - s;
             const float u = silu(cv);
-            const float dl = softplus(ldf(dtt, trow * Ge::CW + cc) + bias);
-            ed[s * Ge::CPW + c] = valid ? make_float2(dl, dl * u) : make_float2(0.f, 0.f);
-            du[e] = valid ? Dd * u : 0.f;
+            const float dl = softplus(ldf(dtt, row_of(s) * Ge::CW + cc) + bias);
+            const bool valid = s >= s_lo && s < s_hi;
+            ed2[s * Ge::CPW + c] = valid ? make_float2(dl, dl * u) : make_float2(0.f, 0.f);
+            edu[s * Ge::CPW + c] = valid ? Dd * u : 0.f;
         }
     }
 
-    // Advance the state over the T steps; yv[e] = sum_n C h of step j + G*e.
+    // Advance the states over steps G*e .. G*e+G-1; returns, for this lane,
+    // sum_n C h of step G*e + j (WITH_Y) after the cross-lane combination.
     template <bool WITH_Y>
-    __device__ __forceinline__ void scan(const float2* ed, const float* bc, float (&yv)[Ge::EPL]) {
+    __device__ __forceinline__ float step_group(int e, const float2* ed2, const float* bc) {
+        float pp[G];
 #pragma unroll
-        for (int e = 0; e < Ge::EPL; ++e) {
-            float pp[G];
+        for (int g = 0; g < G; ++g) {
+            const int s = G * e + g;
+            const float2 q2 = ed2[s * Ge::CPW + c];
+            const float* row = bc + row_of(s) * 2 * kNState;
+            float acc = 0.f;
+            if constexpr (Ge::S == 1) {
+                const float ea = ex2_approx(q2.x * A2[0]);
+                h[0] = fmaf(ea, h[0], q2.y * row[bc_quad_index(j)]);
+                if constexpr (WITH_Y) acc = row[bc_quad_index(j) + 2] * h[0];
+            } else {
+                const float2 dd = make_float2(q2.x, q2.x);
+                const float2 du = make_float2(q2.y, q2.y);
+                float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const int s = G * e + g;
-                const int row = DIR == 0 ? s : T - 1 - s;
-                const float2 q2 = ed[s * Ge::CPW + c];
-                const float* bcr = bc + row * 2 * kNState + 2 * j * Ge::S;  // (B, C) pairs of my states
-                float bcv[2 * Ge::S];
-                load_states<2 * Ge::S>(bcr, bcv);
-                float acc = 0.f;
-#pragma unroll
-                for (int q = 0; q < Ge::S; ++q) {
-                    const float ea = ex2_approx(q2.x * A2[q]);
-                    h[q] = fmaf(ea, h[q], q2.y * bcv[2 * q]);
-                    if constexpr (WITH_Y) acc = fmaf(bcv[2 * q + 1], h[q], acc);
+                for (int pq = 0; pq < Ge::S / 2; ++pq) {
+                    const float4 bcq = *reinterpret_cast<const float4*>(row + (j * Ge::S / 2 + pq) * 4);
+                    const float2 v = mul2(dd, make_float2(A2[2 * pq], A2[2 * pq + 1]));
+                    const float2 ea = make_float2(ex2_approx(v.x), ex2_approx(v.y));
+                    const float2 drive = mul2(du, make_float2(bcq.x, bcq.y));
+                    const float2 hh = fma2(ea, make_float2(h[2 * pq], h[2 * pq + 1]), drive);
+                    h[2 * pq] = hh.x;
+                    h[2 * pq + 1] = hh.y;
+                    if constexpr (WITH_Y) acc2 = fma2(make_float2(bcq.z, bcq.w), hh, acc2);
                 }
-                pp[g] = acc;
+                acc = acc2.x + acc2.y;
             }
-            if constexpr (WITH_Y) yv[e] = group_transpose_reduce<G, Ge::CPW>(pp, j);
+            pp[g] = acc;
         }
+        if constexpr (WITH_Y)
+            return group_transpose_reduce<G, Ge::CPW>(pp, j);
+        else
+            return 0.f;
     }
 };
-
-// Convert a chunk's B and C tiles (T x 16 each, token order) into fp32
-// (B_n, C_n) pairs, cooperatively over `nthreads` threads.
-template <int T, typename Tin>
-__device__ __forceinline__ void convert_bc(const Tin* Bt, const Tin* Ct, float* bc, int tid, int nthreads) {
-    for (int e = tid; e < T * kNState; e += nthreads) {
-        bc[2 * e] = ldf(Bt, e);
-        bc[2 * e + 1] = ldf(Ct, e);
-    }
-}
 
 template <int G, int T, int NWD, int NS, typename Tin>
 __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char* dir_base, uint64_t* full, int r,
@@ -180,9 +222,13 @@ template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR>
 __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
+    using Wk = TmaWorker<G, T, NWD, NS, Tin, DIR>;
     unsigned char* dir_base = base + DIR * Ge::DIR_BYTES;
     float* bc32 = reinterpret_cast<float*>(dir_base + NS * Ge::STAGE);
-    float2* ed = reinterpret_cast<float2*>(base + 2 * Ge::DIR_BYTES + (DIR * NWD + wg) * Ge::ED);
+    unsigned char* wbase = base + Ge::WARP_OFF + (DIR * NWD + wg) * Ge::WARP_BYTES;
+    float2* ed2 = reinterpret_cast<float2*>(wbase);
+    float* edu = reinterpret_cast<float*>(wbase + Ge::ED2);
+    float* ows = reinterpret_cast<float*>(wbase + Ge::ED2 + Ge::EDU);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + Ge::BAR_OFF) + DIR * NS;
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
@@ -194,11 +240,9 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     const bool leader = (wg == 0 && lane == 0);
     const int gtid = wg * 32 + lane;
     const float scale = p.dir_scale[DIR];
-    const float* WSr = p.ws;
-    float* WSw = p.ws;
-    Tout* OUT = static_cast<Tout*>(p.out);
+    const int c0w = ct0 + wg * Ge::CPW;  // first channel of this warp
 
-    TmaWorker<G, T, NWD, NS, Tin, DIR> wk;
+    Wk wk;
     wk.setup(p, ct0, wg, lane);
 
     if (leader) {
@@ -216,6 +260,28 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
             __threadfence_block();
             named_bar_sync(3, 2 * NWD * 32);
         }
+        // valid steps of this chunk: tokens < L
+        const int nvalid = (int)((L - (int64_t)k * T < T) ? (L - (int64_t)k * T) : T);
+        const int s_lo = DIR == 0 ? 0 : T - nvalid;
+        const int s_hi = DIR == 0 ? nvalid : T;
+        const int64_t chunk_row = (int64_t)b * L + (int64_t)k * T;  // global row of the chunk's token kT
+
+        // partner's y of this chunk -> shared memory (waited for before the scan),
+        // in pieces of PC = min(4, CPW) channels.  D is a multiple of 4 on this
+        // path and c0w a multiple of PC, so a piece that starts inside a row
+        // ends inside it and is aligned to its size.
+        if (gated) {
+            constexpr int PC = Ge::CPW < 4 ? Ge::CPW : 4;
+            constexpr int PIECES = Ge::CPW / PC;
+            for (int e = lane; e < T * PIECES; e += 32) {
+                const int r = e / PIECES, q = e % PIECES;
+                const bool ok = (int64_t)k * T + r < L && c0w + PC * q < D;
+                const float* src = p.ws + (chunk_row + (ok ? r : 0)) * D + (ok ? c0w + PC * q : 0);
+                cp_async<PC * 4>(ows + r * Ge::CPW + PC * q, src, ok);
+            }
+            cp_async_commit();
+        }
+
         const int st = i % NS;
         mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1));
         const unsigned char* sb = dir_base + st * Ge::STAGE;
@@ -225,36 +291,32 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
         float* bc = bc32 + (i & 1) * (T * kNState * 2);
-        convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32);
+        convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
         named_bar_sync(1 + DIR, NWD * 32);
         if (leader && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
             issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2,
                                             i2 >= meet, ct0, b);
         }
-        // the partner's y over this chunk, fetched now and used after the scan
-        float other[Ge::EPL];
-#pragma unroll
-        for (int e = 0; e < Ge::EPL; ++e) {
-            const int64_t t = wk.token(k, wk.j + G * e);
-            other[e] = (gated && t < L && wk.dvalid) ? WSr[((int64_t)b * L + t) * D + wk.d] : 0.f;
-        }
-        float du[Ge::EPL], yv[Ge::EPL];
-        wk.elements(xt, dtt, k, L, ed, du);
+
+        wk.elements(xt, dtt, s_lo, s_hi, ed2, edu);
+        if (gated) cp_async_wait_all();
         __syncwarp();
-        wk.template scan<true>(ed, bc, yv);
-#pragma unroll
+
+        float* wsw = p.ws + chunk_row * D + wk.d;
+        Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
+#pragma unroll 2
         for (int e = 0; e < Ge::EPL; ++e) {
-            const int s = wk.j + G * e;
-            const int64_t t = wk.token(k, s);
-            if (t < L && wk.dvalid) {
-                const int64_t idx = ((int64_t)b * L + t) * D + wk.d;
-                const float y = (yv[e] + du[e]) * scale;
+            const float yr = wk.template step_group<true>(e, ed2, bc);
+            const int s = G * e + wk.j;
+            if (s >= s_lo && s < s_hi && wk.dvalid) {
+                const int tr = Wk::row_of(s);  // token - kT
+                const float y = (yr + edu[s * Ge::CPW + wk.c]) * scale;
                 if (!gated) {
-                    WSw[idx] = y;
+                    wsw[(int64_t)tr * D] = y;
                 } else {
-                    const int trow = DIR == 0 ? s : T - 1 - s;
-                    stf(OUT, idx, (y + other[e]) * silu(ldf(zt, trow * Ge::CW + wk.cc)));
+                    const float zv = ldf(zt, tr * Ge::CW + wk.cc);
+                    stf(outw, (int64_t)tr * D, (y + ows[tr * Ge::CPW + wk.c]) * silu(zv));
                 }
             }
         }
@@ -266,15 +328,14 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     }
 }
 
-// Resident CTAs per SM the register budget is sized for (shared memory
-// allows about this many at T = 32, bf16).
-template <int G>
+// Resident CTAs per SM the register budget is sized for.
+template <int G, int T>
 constexpr int layer_min_blocks() {
-    return G >= 16 ? 4 : 3;
+    return (T <= 16 || G >= 16) ? 4 : 3;
 }
 
 template <int G, int T, int NWD, int NS, typename Tin, typename Tout>
-__global__ void __launch_bounds__(2 * NWD * 32, layer_min_blocks<G>())
+__global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     layer_tma_kernel(const __grid_constant__ LayerMaps maps, const KParams p) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
@@ -297,8 +358,8 @@ __global__ void __launch_bounds__(2 * NWD * 32, layer_min_blocks<G>())
 
 // Forward scan over P = p.L tokens from zero; writes the final state and the
 // last three x of the prefix.  One CTA = one batch row x CW channels, NWD
-// warps, the same chunk ring as the layer (the reverse-direction half of the
-// shared memory is unused).  C and z are not read.
+// forward warps and the same chunk ring as the layer (only the forward
+// half of its shared memory is used).  C and z are not read.
 template <int G, int T, int NWD, int NS, typename Tin>
 __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_constant__ LayerMaps maps,
                                                               const KParams p) {
@@ -314,7 +375,9 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
     }
     __syncthreads();
     float* bc32 = reinterpret_cast<float*>(base + NS * Ge::STAGE);
-    float2* ed = reinterpret_cast<float2*>(base + 2 * Ge::DIR_BYTES + wg * Ge::ED);
+    unsigned char* wbase = base + Ge::WARP_OFF + wg * Ge::WARP_BYTES;
+    float2* ed2 = reinterpret_cast<float2*>(wbase);
+    float* edu = reinterpret_cast<float*>(wbase + Ge::ED2);
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
     const int64_t P = p.L;
@@ -346,13 +409,14 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         float* bc = bc32 + (i & 1) * (T * kNState * 2);
-        for (int e = wg * 32 + lane; e < T * kNState; e += NWD * 32) bc[2 * e] = ldf(Bt, e);
+        convert_bc<T, Tin>(Bt, Bt, bc, wg * 32 + lane, NWD * 32, false);
         named_bar_sync(1, NWD * 32);
         if (leader && i >= 1 && i - 1 + NS < nc) issue(i - 1 + NS);
-        float du[Ge::EPL], yv[Ge::EPL];
-        wk.elements(xt, dtt, i, P, ed, du);
+        const int nvalid = (int)((P - (int64_t)i * T < T) ? (P - (int64_t)i * T) : T);
+        wk.elements(xt, dtt, 0, nvalid, ed2, edu);
         __syncwarp();
-        wk.template scan<false>(ed, bc, yv);
+#pragma unroll 2
+        for (int e = 0; e < Ge::EPL; ++e) wk.template step_group<false>(e, ed2, bc);
         __syncwarp();
     }
     if (wk.dvalid) {

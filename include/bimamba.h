@@ -71,6 +71,11 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * x/z/dt/B/C pointer is 16-byte aligned and a row of d_inner elements is a
  * whole number of 16-byte units). */
 #define BIMAMBA_NO_TMA      0x4000u
+/* Bits 16..17 select the chunk length of the TMA-fed kernel (0 = chosen from
+ * the problem size, 1 = 16 tokens, 2 = 32 tokens).  A tuning knob like the
+ * lane count. */
+#define BIMAMBA_CHUNK_SHIFT 16
+#define BIMAMBA_CHUNK_MASK  (0x3u << BIMAMBA_CHUNK_SHIFT)
 
 /* Parameters of both directions, fp32 device pointers, index 0 = forward. */
 typedef struct {

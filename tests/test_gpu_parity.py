@@ -49,17 +49,18 @@ def test_bf16_ragged_staged_kernel(bm, shape, lanes):
     assert U.bf16_out_ok(got16, ref)
 
 
+@pytest.mark.parametrize("chunk", [1, 2])
 @pytest.mark.parametrize("lanes", [4, 8, 16])
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
                                    (1, 32, 32), (1, 64, 48), (1, 65, 8)])
-def test_bf16_ragged_tma_kernel(bm, shape, lanes):
-    """The TMA-fed kernel (32-token chunks): one, two and three chunks, a
-    ragged last chunk, and channel counts that leave the last CTA's tile
-    partly empty."""
+def test_bf16_ragged_tma_kernel(bm, shape, lanes, chunk):
+    """The TMA-fed kernel with 16- and 32-token chunks: one, two and three
+    chunks, a ragged last chunk, and channel counts that leave the last
+    CTA's tile partly empty."""
     b, L, D = shape
     inp, par = W.make_case(b, L, D, 16, "bf16", seed=200 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    flags = lanes << 8
+    flags = (lanes << 8) | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
     got32 = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got32, ref) <= U.GUARD
     got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
@@ -81,7 +82,7 @@ def test_short_sequences(bm, L):
     inp, par = W.make_case(2, L, 16, 16, "fp32", seed=7 + L)
     ref = oracle.layer_fwd(inp, par)
     for flags in (1 << 8 | bm.BIMAMBA_NO_TMA, 4 << 8 | bm.BIMAMBA_NO_TMA, 16 << 8 | bm.BIMAMBA_NO_TMA,
-                  4 << 8, 8 << 8, 16 << 8):
+                  4 << 8, 8 << 8, 16 << 8, 4 << 8 | 1 << 16, 16 << 8 | 1 << 16):
         got = run_layer(bm, inp, par, torch.float32, flags)
         assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
 
