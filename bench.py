@@ -46,6 +46,7 @@ def parse_args():
     ap.add_argument("--L", type=int, default=65536, help="sequence length of --workload long")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="TMA chunk length selector: 0 auto, 1 = 16, 2 = 32")
+    ap.add_argument("--family", type=int, default=0, help="kernel family: 0 auto, 1 chunked, 2 per-token fused")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
@@ -183,7 +184,8 @@ def run_ours(args, rank, world, local):
     from bidirectional_mamba_denoiser_b200 import bimamba as bm
     w = workload_of(args)
     dev = torch.device("cuda", local)
-    flags = ((args.lanes << bm.BIMAMBA_LANES_SHIFT) if args.lanes else 0) | (args.chunk << bm.BIMAMBA_CHUNK_SHIFT)
+    flags = (((args.lanes << bm.BIMAMBA_LANES_SHIFT) if args.lanes else 0) | (args.chunk << bm.BIMAMBA_CHUNK_SHIFT)
+             | (args.family << bm.BIMAMBA_FAMILY_SHIFT))
     sets = [W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed + 1000 * i + rank, device=dev)
             for i in range(2)]
     out = torch.empty(w.batch, w.L, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))

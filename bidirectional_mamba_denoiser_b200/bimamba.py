@@ -32,6 +32,7 @@ BIMAMBA_REV_ONLY = 0x2
 BIMAMBA_LANES_SHIFT = 8
 BIMAMBA_NO_TMA = 0x4000
 BIMAMBA_CHUNK_SHIFT = 16
+BIMAMBA_FAMILY_SHIFT = 18
 
 D_STATE = 16
 

@@ -9,6 +9,7 @@
 #include <utility>
 
 #include "bimamba.h"
+#include "layer_fused.cuh"
 #include "layer_tma.cuh"
 #include "scan_kernels.cuh"
 
@@ -299,6 +300,81 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
     return BIMAMBA_ERR_UNSUPPORTED;
 }
 
+// ---- per-token fused kernels (many channels)
+
+template <typename Tin>
+bool fill_fused_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool layer) {
+    constexpr int T = 16, CW = 32;
+    const bool bf = std::is_same<Tin, bf16>::value;
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, CW, T + 3);
+    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, CW, T);
+    ok = ok && map3d(&m.B[0], in->B[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
+    if (layer) {
+        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, CW, T);
+        ok = ok && map3d(&m.C[0], in->C[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
+        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, CW, T);
+        ok = ok && map3d(&m.B[1], in->B[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
+        ok = ok && map3d(&m.C[1], in->C[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
+    } else {
+        m.z = m.x;
+        m.C[0] = m.B[0];
+        m.dt[1] = m.dt[0];
+        m.B[1] = m.B[0];
+        m.C[1] = m.B[0];
+    }
+    return ok;
+}
+
+template <int G, typename Tin, typename Tout>
+int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::FusedGeo<G, Tin>;
+    bimamba::FusedMaps maps;
+    if (!fill_fused_maps<Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, 64, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+int fused_layer_by_group(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    switch (g) {
+        case 2: return launch_fused_layer<2, Tin, Tout>(k, in, st);
+        case 4: return launch_fused_layer<4, Tin, Tout>(k, in, st);
+        case 8: return launch_fused_layer<8, Tin, Tout>(k, in, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
+}
+
+template <int G, typename Tin>
+int launch_fused_prefix(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::FusedGeo<G, Tin>;
+    bimamba::FusedMaps maps;
+    if (!fill_fused_maps<Tin>(maps, in, k.batch, k.L, k.D, false)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::fused_prefix_kernel<G, Tin>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, 32, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+// Kernel family of the TMA path: forced by the flags, else the per-token
+// fused kernel when one lane per channel and direction still gives at least
+// 8 warps per SM, otherwise the chunked kernel.
+int pick_family(int64_t lanes_total, unsigned flags) {
+    const unsigned f = (flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT;
+    if (f) return (int)f;
+    return lanes_total >= 148LL * 8 * 32 ? 2 : 1;
+}
+
+int pick_group_fused(unsigned flags) {
+    const unsigned f = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    return f ? (int)f : 4;
+}
+
 // Chunk length of the TMA kernel: forced by the flags, else 32.
 int pick_chunk_tma(unsigned flags) {
     const unsigned f = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
@@ -376,8 +452,9 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
                       unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
-    const unsigned known =
-        BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA | BIMAMBA_CHUNK_MASK;
+    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
+                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK;
+    if (((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if (((flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
@@ -403,6 +480,15 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    const int fam = pick_family(2LL * batch * d_inner, flags);
+    if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && (forced == 0 || forced == 2 || forced == 4 || forced == 8) &&
+        tma_eligible(in, d_inner, true, true)) {
+        const int gf = pick_group_fused(flags);
+        if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, k, in, st);
+        if (in_bf) return fused_layer_by_group<bf16, float>(gf, k, in, st);
+        if (out_bf) return fused_layer_by_group<float, bf16>(gf, k, in, st);
+        return fused_layer_by_group<float, float>(gf, k, in, st);
+    }
     if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
         const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
         const int tt = pick_chunk_tma(flags);
@@ -439,6 +525,10 @@ int bimamba_prefix_state(const bimamba_inputs_t* prefix, const bimamba_params_t*
     k.batch = batch;
     k.dir_scale[0] = k.dir_scale[1] = 1.f;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (tma_eligible(prefix, d_inner, false, false) && pick_family((int64_t)batch * d_inner, 0) == 2) {
+        if (prefix->dtype == BIMAMBA_BF16) return launch_fused_prefix<4, bf16>(k, prefix, st);
+        return launch_fused_prefix<4, float>(k, prefix, st);
+    }
     if (tma_eligible(prefix, d_inner, false, false)) {
         const int gt = pick_lanes_tma((int64_t)batch * d_inner, 0);
         if (prefix->dtype == BIMAMBA_BF16) return prefix_tma_by_lanes<bf16>(gt, k, prefix, st);

@@ -91,21 +91,6 @@ __device__ __forceinline__ void convert_bc(const Tin* Bt, const Tin* Ct, float* 
     }
 }
 
-// Asynchronous global -> shared copy of BYTES (8 or 16; both addresses
-// aligned to BYTES); with pred false nothing is read and zeros are written.
-template <int BYTES>
-__device__ __forceinline__ void cp_async(void* dst, const void* src, bool pred) {
-    static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
-    const int n = pred ? BYTES : 0;
-    if constexpr (BYTES == 16)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
-                     : "memory");
-    else
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
-                     : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // One warp's scan of one direction over CPW channels.
 template <int G, int T, int NWD, int NS, typename Tin, int DIR>

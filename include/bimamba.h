@@ -76,6 +76,13 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * lane count. */
 #define BIMAMBA_CHUNK_SHIFT 16
 #define BIMAMBA_CHUNK_MASK  (0x3u << BIMAMBA_CHUNK_SHIFT)
+/* Bits 18..19 select the TMA-fed kernel family (0 = chosen from the problem
+ * size).  1: chunked -- G lanes share one channel's states, for few channels
+ * (batch 1, long sequences).  2: per-token fused -- one lane per channel,
+ * groups of G lanes share B/C across G channels, for many channels.  With
+ * family 2 the lane field (bits 8..12) is the group size (2, 4 or 8). */
+#define BIMAMBA_FAMILY_SHIFT 18
+#define BIMAMBA_FAMILY_MASK  (0x3u << BIMAMBA_FAMILY_SHIFT)
 
 /* Parameters of both directions, fp32 device pointers, index 0 = forward. */
 typedef struct {

@@ -96,6 +96,7 @@ def _layer(inp=None, par=None, out=FAKE + 0x20000, out_dtype=bm.BIMAMBA_BF16, ba
     (dict(flags=0x4), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_CHUNK_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY), bm.BIMAMBA_ERR_INVALID_ARG),
     (dict(out_dtype=7), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(inp=NULL), bm.BIMAMBA_ERR_INVALID_ARG),

@@ -24,7 +24,7 @@ def run_layer(bm, inp, par, out_dtype, flags=0):
     return U.to_cpu64(out)
 
 
-@pytest.mark.parametrize("flags", [0, 0x4000])
+@pytest.mark.parametrize("flags", [0, 0x4000, 1 << 18, 2 << 18])
 def test_tiny_fp32_case(bm, flags):
     """b=1, L=256, D=64, fp32 in and out, seed 0: normwise <= 1e-5 (both kernels)."""
     inp, par = W.make_workload(W.TINY)
@@ -60,7 +60,25 @@ def test_bf16_ragged_tma_kernel(bm, shape, lanes, chunk):
     b, L, D = shape
     inp, par = W.make_case(b, L, D, 16, "bf16", seed=200 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    flags = (lanes << 8) | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
+    flags = (lanes << 8) | (chunk << bm.BIMAMBA_CHUNK_SHIFT) | (1 << bm.BIMAMBA_FAMILY_SHIFT)
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= U.GUARD
+    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+    assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
+@pytest.mark.parametrize("group", [2, 4, 8])
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 16, 32), (1, 32, 64), (2, 17, 96)])
+def test_bf16_ragged_fused_kernel(bm, shape, group):
+    """The per-token fused kernel (16-token chunks, one lane per channel,
+    B/C shared by groups of lanes): one, two and many chunks, ragged last
+    chunks and a last CTA whose 32 channels are partly past d_inner."""
+    b, L, D = shape
+    inp, par = W.make_case(b, L, D, 16, "bf16", seed=300 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = (group << 8) | (2 << bm.BIMAMBA_FAMILY_SHIFT)
     got32 = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got32, ref) <= U.GUARD
     got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
@@ -82,7 +100,8 @@ def test_short_sequences(bm, L):
     inp, par = W.make_case(2, L, 16, 16, "fp32", seed=7 + L)
     ref = oracle.layer_fwd(inp, par)
     for flags in (1 << 8 | bm.BIMAMBA_NO_TMA, 4 << 8 | bm.BIMAMBA_NO_TMA, 16 << 8 | bm.BIMAMBA_NO_TMA,
-                  4 << 8, 8 << 8, 16 << 8, 4 << 8 | 1 << 16, 16 << 8 | 1 << 16):
+                  4 << 8 | 1 << 18, 8 << 8 | 1 << 18, 16 << 8 | 1 << 18, 4 << 8 | 1 << 16 | 1 << 18,
+                  16 << 8 | 1 << 16 | 1 << 18, 2 << 8 | 2 << 18, 4 << 8 | 2 << 18, 8 << 8 | 2 << 18):
         got = run_layer(bm, inp, par, torch.float32, flags)
         assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
 
@@ -142,10 +161,12 @@ def _sampled_layer_check(bm, w: W.Workload, nchan: int, flags=0):
     return U.normwise(g32, ref), U.bf16_out_ok(g16, ref)
 
 
-def test_layer_1p3b_shape_sampled(bm):
+@pytest.mark.parametrize("flags", [0, 1 << 18])
+def test_layer_1p3b_shape_sampled(bm, flags):
     """b=8, L=2048, D=4096, bf16, seed 1 -- the launch configuration the
-    bench times; 48 channels of every batch row against the oracle."""
-    err, ok16 = _sampled_layer_check(bm, W.LAYER_1P3B, 48)
+    bench times (flags 0) and the chunked kernel; 48 channels of every batch
+    row against the oracle."""
+    err, ok16 = _sampled_layer_check(bm, W.LAYER_1P3B, 48, flags)
     assert err <= U.GUARD and ok16
 
 
