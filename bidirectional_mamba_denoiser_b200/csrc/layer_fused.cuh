@@ -139,30 +139,42 @@ struct FusedWarp {
         x2 = ldf(xt, xrow_of(-1) * Ge::CW + lane);
     }
 
-    // One step: per-token work of the own channel, the group's state
-    // updates, and the own channel's y (sum C h + D u) returned.
-    template <bool WITH_Y>
-    __device__ __forceinline__ float step(int s, bool valid, const Tin* xt, const Tin* dtt, const Tin* Bt,
-                                          const Tin* Ct) {
+    // Per-token work of the own channel at step s: step size, drive and
+    // D*u (zero for an identity step).  Independent of the scan, so it is
+    // computed one step ahead of the state updates that use it.
+    struct Elem {
+        float dl, du, Du;
+    };
+    __device__ __forceinline__ Elem element(int s, bool valid, const Tin* xt, const Tin* dtt) {
         const float x3 = ldf(xt, xrow_of(s) * Ge::CW + lane);
         float cv = fmaf(w[0], x0, cb);
         cv = fmaf(w[1], x1, cv);
         cv = fmaf(w[2], x2, cv);
         cv = fmaf(w[3], x3, cv);
         x0 = x1; x1 = x2; x2 = x3;
-        const int row = row_of(s);
         const float u = silu(cv);
-        const float dl0 = softplus(ldf(dtt, row * Ge::CW + lane) + bias);
-        const float dl = valid ? dl0 : 0.f;
-        const float du = valid ? dl0 * u : 0.f;
+        const float dl = softplus(ldf(dtt, row_of(s) * Ge::CW + lane) + bias);
+        Elem e;
+        e.dl = valid ? dl : 0.f;
+        e.du = valid ? dl * u : 0.f;
+        e.Du = valid ? Dd * u : 0.f;
+        return e;
+    }
+
+    // State updates of step s for the group's G channels (their step sizes
+    // gathered from the group's lanes); returns sum_n C h of the own channel
+    // (WITH_Y), before the D skip.
+    template <bool WITH_Y>
+    __device__ __forceinline__ float scan(int s, const Elem& e, const Tin* Bt, const Tin* Ct) {
+        const int row = row_of(s);
         float bv[S], cvv[S];
         load_row<S>(Bt + row * kNState + j * S, bv);
         if constexpr (WITH_Y) load_row<S>(Ct + row * kNState + j * S, cvv);
         float acc[G];
 #pragma unroll
         for (int q = 0; q < G; ++q) {
-            const float dq = __shfl_sync(0xffffffffu, dl, q, G);
-            const float uq = __shfl_sync(0xffffffffu, du, q, G);
+            const float dq = __shfl_sync(0xffffffffu, e.dl, q, G);
+            const float uq = __shfl_sync(0xffffffffu, e.du, q, G);
             const float2 dd = make_float2(dq, dq);
             const float2 uu = make_float2(uq, uq);
             float2 acc2 = make_float2(0.f, 0.f);
@@ -178,12 +190,10 @@ struct FusedWarp {
             }
             acc[q] = acc2.x + acc2.y;
         }
-        if constexpr (WITH_Y) {
-            const float y = group_transpose_reduce<G, 1>(acc, j);
-            return y + (valid ? Dd * u : 0.f);
-        } else {
+        if constexpr (WITH_Y)
+            return group_transpose_reduce<G, 1>(acc, j);
+        else
             return 0.f;
-        }
     }
 };
 
@@ -269,10 +279,13 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         wp.window(xt);
         float* wsw = p.ws + chunk_row * D + wp.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wp.d;
+        typename Wp::Elem nxt = wp.element(0, 0 >= s_lo && 0 < s_hi, xt, dtt);
 #pragma unroll 2
         for (int s = 0; s < T; ++s) {
             const bool valid = s >= s_lo && s < s_hi;
-            const float y = wp.template step<true>(s, valid, xt, dtt, Bt, Ct) * scale;
+            const typename Wp::Elem cur = nxt;
+            if (s + 1 < T) nxt = wp.element(s + 1, s + 1 >= s_lo && s + 1 < s_hi, xt, dtt);
+            const float y = (wp.template scan<true>(s, cur, Bt, Ct) + cur.Du) * scale;
             if (valid && wp.dvalid) {
                 const int tr = Wp::row_of(s);
                 if (!gated) {
@@ -355,8 +368,13 @@ __global__ void __launch_bounds__(32, 16) fused_prefix_kernel(const __grid_const
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         wp.window(xt);
+        auto nxt = wp.element(0, 0 < nvalid, xt, dtt);
 #pragma unroll 2
-        for (int s = 0; s < T; ++s) wp.template step<false>(s, s < nvalid, xt, dtt, Bt, Bt);
+        for (int s = 0; s < T; ++s) {
+            const auto cur = nxt;
+            if (s + 1 < T) nxt = wp.element(s + 1, s + 1 < nvalid, xt, dtt);
+            wp.template scan<false>(s, cur, Bt, Bt);
+        }
         __syncwarp();
     }
     // the group's G channels x my S states
