@@ -68,6 +68,9 @@ def _load():
     lib.bimamba_layer_fwd.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
                                       I, I64, I, I, U, P, SZ, P]
     lib.bimamba_layer_fwd.restype = I
+    lib.bimamba_layer_fwd_noalloc.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
+                                              I, I64, I, I, U, P]
+    lib.bimamba_layer_fwd_noalloc.restype = I
     lib.bimamba_prefix_state.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), I, I64, I, I,
                                          ctypes.POINTER(FwdState), P]
     lib.bimamba_prefix_state.restype = I
@@ -165,6 +168,26 @@ def bimamba_layer_fwd(x, z, dt, B, C, params: dict, out=None, out_dtype=None, fl
                                _stream(stream))
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba_layer_fwd", rc)
+    return out
+
+
+def bimamba_layer_fwd_noalloc(x, z, dt, B, C, params: dict, out=None, out_dtype=None, flags: int = 0,
+                              stream=None):
+    """bimamba_layer_fwd for callers that cannot allocate device memory: the
+    library's built-in 64 MiB scratch replaces the workspace (batch * L *
+    d_inner <= 16,777,216).  Calls that overlap on the GPU race on that
+    scratch.  ``out`` is still the caller's; pass it in to allocate nothing
+    here either."""
+    b, L, D = x.shape
+    N = (B[0] if isinstance(B, (tuple, list)) else B).shape[-1]
+    if out is None:
+        out = torch.empty(b, L, D, device=x.device, dtype=out_dtype or x.dtype)
+    inp = make_inputs(x, z, dt, B, C)
+    par = make_params(params)
+    rc = lib.bimamba_layer_fwd_noalloc(ctypes.byref(inp), ctypes.byref(par), _ptr(out), _dtype_code(out.dtype),
+                                       b, L, D, N, flags, _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_layer_fwd_noalloc", rc)
     return out
 
 

@@ -586,3 +586,56 @@ int bimamba_block_step(const bimamba_fwd_state_t* prefix_state, const bimamba_in
 }
 
 }  // extern "C"
+
+// ---- full layer without a caller-provided workspace
+//
+// Some callers have no device allocator to hand: a plugin loaded into a host
+// application that owns every byte of GPU memory, or a program that reaches
+// this library only through the C ABI from a language with no CUDA memory
+// API.  They cannot supply the workspace bimamba_layer_fwd needs, so this
+// entry point uses a fixed scratch array that lives in the library itself.
+
+// Scratch for the half-sequence partial outputs, 64 MiB on every device that
+// loads this library, kept until the process exits.  In host code this name
+// is only a stand-in for the symbol: its device address comes from
+// cudaGetSymbolAddress below, never from the name itself.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[64u << 20];
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = sizeof(g_noalloc_scratch);
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+int noalloc_scratch(void** addr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BIMAMBA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BIMAMBA_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return BIMAMBA_OK;
+}
+
+}  // namespace
+
+extern "C" int bimamba_layer_fwd_noalloc(const bimamba_inputs_t* in, const bimamba_params_t* p, void* out,
+                                         bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner,
+                                         int d_state, unsigned flags, void* cuda_stream) {
+    const size_t need = bimamba_workspace_bytes(batch, L, d_inner, d_state, flags);
+    if (need == 0)  // invalid sizes: let the full entry point name the problem (nothing is launched)
+        return bimamba_layer_fwd(in, p, out, out_dtype, batch, L, d_inner, d_state, flags, nullptr, 0,
+                                 cuda_stream);
+    if (need > kNoallocScratchBytes) return BIMAMBA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    return bimamba_layer_fwd(in, p, out, out_dtype, batch, L, d_inner, d_state, flags, scratch,
+                             kNoallocScratchBytes, cuda_stream);
+}

@@ -129,6 +129,29 @@ int bimamba_layer_fwd(const bimamba_inputs_t *in, const bimamba_params_t *p,
                       int batch, int64_t L, int d_inner, int d_state, unsigned flags,
                       void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* The full layer for callers that cannot allocate device memory -- a plugin
+ * inside a host application that owns all GPU memory, or a caller that
+ * reaches this library only through the C ABI with no CUDA allocator -- and
+ * so cannot hand bimamba_layer_fwd a workspace.  The paper has no
+ * counterpart: this is an interface convenience, computing exactly what
+ * bimamba_layer_fwd computes.
+ *   Instead of a caller's workspace it uses a scratch array built into the
+ * library: 64 MiB that every GPU loading the library holds until the process
+ * exits.  It therefore accepts batch * L * d_inner <= 16,777,216 (the
+ * workspace bimamba_workspace_bytes reports must fit in 64 MiB) and returns
+ * BIMAMBA_ERR_WORKSPACE above that.  It allocates and frees nothing.
+ *   The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls on a device share the one array: the
+ * kernel writes every scratch value before reading it, so nothing needs
+ * clearing between calls, but two calls whose kernels overlap on the GPU
+ * (other streams, or other host threads) race on it and give undefined
+ * output.  Other arguments, checks and errors: as bimamba_layer_fwd. */
+int bimamba_layer_fwd_noalloc(const bimamba_inputs_t *in, const bimamba_params_t *p,
+                              void *out, bimamba_dtype_t out_dtype,
+                              int batch, int64_t L, int d_inner, int d_state, unsigned flags,
+                              void *cuda_stream);
+
 /* Forward-only scan over a prefix of P tokens from a zero state (§4.3: the
  * cache a decoded block leaves behind).  Reads prefix->x, prefix->dt[0],
  * prefix->B[0] (z, C and the reverse inputs are not read and may be NULL).
