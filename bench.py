@@ -1,18 +1,26 @@
 #!/usr/bin/env python
 """Throughput of the bidirectional Mamba mixer layer on B200.
 
-Default workload: one layer call at batch 8, L = 2048, d_inner = 4096,
-d_state = 16, bf16 I/O with fp32 state (the 1.3B-model layer shape), on
-synthetic seeded inputs.  A step is one bimamba_layer_fwd call (one kernel
-launch: conv, softplus, both scan directions, D skip, sum and gate).
-
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload layer|long] [--L L]
+                  [--workload layer|long|block|sweep] [--L L]
 
-Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs its
-own replica of the workload on its own GPU -- the layer has no exchange step
-across batch rows or channels -- and value is the total over ranks divided
-by the slowest rank's device time.
+Workloads (synthetic seeded inputs, bf16 I/O, fp32 state, d_state 16):
+  layer  (default) one layer call at batch 8, L 2048, d_inner 4096 -- the 1.3B
+         layer shape; a step is one bimamba_layer_fwd (one kernel launch:
+         conv, softplus, both scan directions, D skip, sum and gate)
+  long   the same at batch 1 and L = --L (default 65536)
+  block  block-cached decoding at batch 16, d_inner 4096: the forward state of
+         a 65536-token prefix is built once, then a step is one
+         bimamba_block_step over a 32-token block (commit every 128th step);
+         steps are replayed from a CUDA graph
+  sweep  a denoiser-shaped stack: one step is 48 layer calls at batch 1,
+         L = --L (default 8192), each layer with its own inputs; the line adds
+         the mixer time of a full 128-step generation
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
+replica on its own GPU -- the layer has no exchange step across batch rows or
+channels -- and value is the total over ranks divided by the slowest rank's
+device time (scaling "weak").
 """
 from __future__ import annotations
 
@@ -35,47 +43,73 @@ from bidirectional_mamba_denoiser_b200 import workloads as W  # noqa: E402
 METRIC = "bi-Mamba layer Mtokens/s"
 UNIT = "Mtokens/s"
 
+SMS = 148
+MUFU_PER_SM_CLK = 16          # special-function-unit lanes per SM per clock (B200)
+MUFU_PER_ELEM_LAYER = 42      # 32 state exps + 2x(SiLU 2 + softplus 2) + gate SiLU 2
+MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus 2
 
-def parse_args():
+# DRAM bytes (read + write) per launch from the ncu capture summarised in
+# profiles/ -- the workload and kernel they were taken on; anything else null.
+NCU_TRAFFIC = {
+    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1306.8e6,
+}
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "long"], default="layer")
-    ap.add_argument("--L", type=int, default=65536, help="sequence length of --workload long")
-    ap.add_argument("--lanes", type=int, default=0, help="lanes per channel (0 = library's choice)")
-    ap.add_argument("--chunk", type=int, default=0, help="TMA chunk length selector: 0 auto, 1 = 16, 2 = 32")
+    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep"], default="layer")
+    ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep")
+    ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
+    ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
     ap.add_argument("--family", type=int, default=0, help="kernel family: 0 auto, 1 chunked, 2 per-token fused")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def workload_of(args) -> W.Workload:
-    return W.LAYER_1P3B if args.workload == "layer" else W.LONG_SEQ.get(args.L) or \
-        W.Workload(f"long_b1_L{args.L}_D4096_bf16", 1, args.L, 4096, 16, "bf16", 2)
+    if args.workload == "layer":
+        return W.LAYER_1P3B
+    if args.workload == "block":
+        return W.BLOCK_CACHED
+    if args.workload == "sweep":
+        L = args.L or 8192
+        return W.DENOISER_SWEEP.get(L) or W.Workload(f"denoiser_48x128_b1_L{L}_D4096_bf16", 1, L, 4096, 16,
+                                                     "bf16", 3, extra={"layers": 48, "steps": 128})
+    L = args.L or 65536
+    return W.LONG_SEQ.get(L) or W.Workload(f"long_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 2)
 
 
-def algorithmic_bytes(w: W.Workload) -> int:
-    """Bytes the layer must move once: x, z, dt_f, dt_b read and out written
+def layer_bytes(batch: int, L: int, D: int, N: int, esz: int) -> int:
+    """Bytes one layer call must move: x, z, dt_f, dt_b read and out written
     per (token, channel); B_f, C_f, B_b, C_b read per token."""
-    e = 2 if w.dtype == "bf16" else 4
-    return w.batch * w.L * (w.d_inner * 5 * e + 4 * w.d_state * e)
+    return batch * L * (D * 5 * esz + 4 * N * esz)
+
+
+def block_bytes(w: W.Workload, esz: int = 2) -> int:
+    """One block step: the block's inputs and output, the cached state (fp32)
+    and conv tail read; the commit's writes are amortised over the steps of a
+    block."""
+    b, G, D, N = w.batch, w.extra["block"], w.d_inner, w.d_state
+    state = b * D * N * 4 + b * 3 * D * esz
+    return layer_bytes(b, G, D, N, esz) + state + state // w.extra["steps_per_block"]
 
 
 def load_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
-        with open(path) as f:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             pk = json.load(f)
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
 
 
-# ---------------------------------------------------------------- distributed
+# ---------------------------------------------------------------- ranks
 
 def dist_init(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -96,12 +130,18 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """The largest of every rank's v (timing is the slowest rank's)."""
     if world == 1:
         return v
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    t = torch.tensor([v], device=device, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds_max: float, scale: float = 1e-6) -> float:
+    """Units all ranks processed over the slowest rank's time (weak scaling)."""
+    return world * units_per_rank / seconds_max * scale
 
 
 # ---------------------------------------------------------------- clocks
@@ -138,7 +178,7 @@ class ClockSampler:
         rows = []
         with open(self.path) as f:
             for line in f:
-                parts = [p.strip() for p in line.split(",")]
+                parts = [q.strip() for q in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
@@ -155,11 +195,54 @@ class ClockSampler:
                 "power_w_max": max(r[2] for r in loaded), "samples": len(loaded), "reasons": reasons}
 
 
+def timed(step, steps: int, warmup: int, world: int, dev, stream):
+    """Device time of `steps` calls of step(i) after `warmup` untimed ones:
+    CUDA events on the launch stream, barrier + synchronize on both sides.
+    Returns (ms on this rank, clocks)."""
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index or 0)
+    sampler.start()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop()
+    return e0.elapsed_time(e1), clocks
+
+
+def roofline(mufu_ops: float, launch_ms: float, clocks, workload: str, kernel: str):
+    """The binding roof of this path is the special-function unit (one exp
+    per state update): achieved MUFU operations per second against the unit
+    count x clock."""
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = SMS * MUFU_PER_SM_CLK * mhz * 1e6 / 1e9
+    achieved = mufu_ops / (launch_ms / 1e3) / 1e9
+    return {"bound": "alu", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "Gop/s (MUFU)",
+            "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get((workload, kernel)),
+            "peak_source": f"148 SMs x 16 MUFU lanes/clk x {mhz:.0f} MHz", "kernel": kernel}
+
+
+def hbm_fraction(bytes_per_launch: float, launch_ms: float):
+    peak, src = load_peaks()
+    achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
+    return {"achieved_gbs": round(achieved, 1), "peak_gbs": peak, "frac": round(achieved / peak, 4),
+            "peak_source": src, "algorithmic_bytes_per_launch": int(bytes_per_launch)}
+
+
 # ---------------------------------------------------------------- cpu baseline (the oracle)
 
 def oracle_sample_rate(w: W.Workload, inputs, params, budget_s: float):
-    """The fp64 oracle, timed on a channel sample of the same inputs;
-    returns (Mtokens/s scaled to the whole layer, channels, seconds, threads)."""
+    """The fp64 oracle on a channel sample of the same inputs, scaled to the
+    whole layer: (Mtokens/s, channels, seconds, threads)."""
     import oracle
     from tests import parity_util as U
     threads = oracle.max_threads()
@@ -175,110 +258,167 @@ def oracle_sample_rate(w: W.Workload, inputs, params, budget_s: float):
         nch = int(min(w.d_inner, max(nch + 1, nch * budget_s / max(dt, 1e-3))))
         nch = max(threads, (nch // threads) * threads)
     layer_s = dt * w.d_inner / len(chans)
-    return w.tokens / layer_s / 1e6, len(chans), dt, threads
+    return w.batch * w.L / layer_s / 1e6, len(chans), dt, threads
 
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args, rank, world, local):
-    from bidirectional_mamba_denoiser_b200 import bimamba as bm
-    w = workload_of(args)
-    dev = torch.device("cuda", local)
-    flags = (((args.lanes << bm.BIMAMBA_LANES_SHIFT) if args.lanes else 0) | (args.chunk << bm.BIMAMBA_CHUNK_SHIFT)
-             | (args.family << bm.BIMAMBA_FAMILY_SHIFT))
+def flags_of(args, bm):
+    return (((args.lanes << bm.BIMAMBA_LANES_SHIFT) if args.lanes else 0) | (args.chunk << bm.BIMAMBA_CHUNK_SHIFT)
+            | (args.family << bm.BIMAMBA_FAMILY_SHIFT))
+
+
+def kernel_name(w: W.Workload, args) -> str:
+    if args.workload == "block":
+        return "block_kernel"
+    fam = args.family or (2 if 2 * w.batch * w.d_inner >= SMS * 8 * 32 else 1)
+    return "fused_layer_kernel" if fam == 2 else "layer_tma_kernel"
+
+
+def run_layer_like(args, w, bm, rank, world, dev, stream):
+    """layer / long / sweep: steps of bimamba_layer_fwd."""
+    flags = flags_of(args, bm)
+    nsets = w.extra.get("layers", 2) if args.workload == "sweep" else 2
     sets = [W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed + 1000 * i + rank, device=dev)
-            for i in range(2)]
+            for i in range(nsets)]
     out = torch.empty(w.batch, w.L, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
     ws = torch.empty(bm.bimamba_workspace_bytes(w.batch, w.L, w.d_inner, w.d_state), device=dev,
                      dtype=torch.uint8)
-    stream = torch.cuda.current_stream(dev)
+    calls = nsets if args.workload == "sweep" else 1
 
     def step(i):
-        inp, par = sets[i & 1]
-        bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, out=out, flags=flags,
-                             workspace=ws, stream=stream)
+        for c in range(calls):
+            inp, par = sets[(i * calls + c) % nsets]
+            bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, out=out, flags=flags,
+                                 workspace=ws, stream=stream)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    sampler = ClockSampler(local)
-    sampler.start()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
+    ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
     ms_max = max_over_ranks(ms, world)
-    ms_per_step = ms_max / args.steps
-    value = world * w.tokens * args.steps / (ms_max / 1e3) / 1e6
+    call_ms = ms / args.steps / calls
+    elems = w.batch * w.L * w.d_inner
+    res = {
+        "value": whole_job_rate(w.batch * w.L * calls * args.steps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / args.steps,
+        "gpu_launches": args.steps * calls,
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args)),
+        "hbm": hbm_fraction(layer_bytes(w.batch, w.L, w.d_inner, w.d_state, 2), call_ms),
+        "clocks": clocks,
+    }
+    if args.workload == "sweep":
+        res["sequence_mixer_s"] = round(call_ms * w.extra["layers"] * w.extra["steps"] / 1e3, 4)
+        res["sequence_note"] = f"{w.extra['layers']} layers x {w.extra['steps']} steps x {call_ms:.4f} ms per call"
 
-    # roofline of the (only) kernel: algorithmic bytes per launch / launch time
-    peak, peak_src = load_peaks()
-    achieved = algorithmic_bytes(w) / (ms / args.steps / 1e3) / 1e9
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_src,
-            "kernel": "layer_kernel", "algorithmic_bytes_per_launch": algorithmic_bytes(w)}
-
-    # end to end: host (pinned) inputs -> device, the C-ABI call, result -> host
-    e2e = None
     if not args.no_e2e:
         inp, par = sets[0]
         host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}
         dbuf = {k: torch.empty_like(v) for k, v in inp.items()}
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in host.values())
-        d2h = hout.numel() * hout.element_size()
         k2 = max(3, min(args.steps, 20))
 
-        def e2e_step():
+        def e2e_step(i):
             for k in host:
                 dbuf[k].copy_(host[k], non_blocking=True)
-            bm.bimamba_layer_fwd(dbuf["x"], dbuf["z"], dbuf["dt"], dbuf["B"], dbuf["C"], par, out=out,
-                                 flags=flags, workspace=ws, stream=stream)
+            bm.bimamba_layer_fwd(dbuf["x"], dbuf["z"], dbuf["dt"], dbuf["B"], dbuf["C"], par, out=out, flags=flags,
+                                 workspace=ws, stream=stream)
             hout.copy_(out, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(k2):
-            e2e_step()
-        a1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms2 = max_over_ranks(a0.elapsed_time(a1), world)
-        e2e = {"value": round(world * w.tokens * k2 / (ms2 / 1e3) / 1e6, 4), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k2}
-
-    cpu = None
+        ms2, _ = timed(e2e_step, k2, 2, world, dev, stream)
+        res["e2e"] = {"value": round(whole_job_rate(w.batch * w.L * k2, world, max_over_ranks(ms2, world) / 1e3), 4),
+                      "unit": UNIT, "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": k2}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp, par = sets[0]
         v, nch, secs, thr = oracle_sample_rate(w, inp, par, args.cpu_budget)
-        cpu = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
-               "sample": f"{nch} of {w.d_inner} channels x {w.batch} batch rows x L={w.L} "
-                         f"({secs:.1f} s), scaled by {w.d_inner}/{nch}"}
+        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+                               "sample": f"{nch} of {w.d_inner} channels x {w.batch} batch rows x L={w.L} "
+                                         f"({secs:.1f} s), scaled by {w.d_inner}/{nch}"}
+    return res
 
+
+def run_block(args, w, bm, rank, world, dev, stream):
+    """block: a prefix state, then block steps replayed from a CUDA graph."""
+    P, G, spb = w.extra["prefix"], w.extra["block"], w.extra["steps_per_block"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + rank)
+    par = W.make_params(w.d_inner, w.d_state, g, dev)
+    pre = W.make_inputs(w.batch, P, w.d_inner, w.d_state, w.dtype, g, dev)
+    h = torch.empty(w.batch, w.d_inner, w.d_state, device=dev, dtype=torch.float32)
+    tail = torch.empty(w.batch, 3, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
+    torch.cuda.synchronize(dev)
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    bm.bimamba_prefix_state(pre["x"], pre["dt"], pre["B"], par, h_out=h, conv_x_out=tail, stream=stream)
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    prefix_ms = p0.elapsed_time(p1)
+    del pre
+    torch.cuda.empty_cache()
+    pool = [W.make_inputs(w.batch, G, w.d_inner, w.d_state, w.dtype, g, dev) for _ in range(8)]
+    out = torch.empty(w.batch, G, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
+
+    def one(i):
+        blk = pool[i % len(pool)]
+        commit = (i % spb) == spb - 1
+        bm.bimamba_block_step((h, tail), blk["x"], blk["z"], blk["dt"], blk["B"], blk["C"], par, out=out,
+                              new_state=(h, tail) if commit else None, stream=stream)
+
+    # one block's steps captured once (the decoding loop's shape) and replayed
+    for i in range(2):
+        one(i)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(spb):
+            one(i)
+    reps = max(1, args.steps // spb)
+
+    def step(_):
+        graph.replay()
+
+    ms, clocks = timed(step, reps, max(1, args.warmup // spb), world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    nsteps = reps * spb
+    step_ms = ms / nsteps
+    elems = w.batch * G * w.d_inner
+    del graph
+    return {
+        "value": whole_job_rate(w.batch * G * nsteps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / nsteps, "gpu_launches": nsteps,
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, step_ms, clocks, w.name, "block_kernel"),
+        "hbm": hbm_fraction(block_bytes(w), step_ms), "clocks": clocks,
+        "prefix_state_ms": round(prefix_ms, 3),
+        "prefix_mufu_frac": roofline(MUFU_PER_ELEM_FWD * w.batch * P * w.d_inner, prefix_ms, clocks, w.name,
+                                     "prefix")["frac"],
+        "steps_timed": nsteps, "graph": f"{spb} block steps per CUDA graph replay",
+    }
+
+
+def run_ours(args, rank, world, local):
+    from bidirectional_mamba_denoiser_b200 import bimamba as bm
+    w = workload_of(args)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    if args.workload == "block":
+        side = torch.cuda.Stream(dev)  # graphs cannot be captured on the legacy default stream
+        with torch.cuda.stream(side):
+            res = run_block(args, w, bm, rank, world, dev, side)
+    else:
+        res = run_layer_like(args, w, bm, rank, world, dev, stream)
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "metric": METRIC, "value": round(res.pop("value"), 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(res.pop("ms_per_step"), 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                        "d_state": w.d_state, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (two rotating input sets)"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
-            "hbm_gbs_algorithmic": round(achieved, 1),
+                       "l2": "inputs larger than L2 (rotating input sets)" if args.workload != "block"
+                       else "block inputs rotate over 8 sets (state stays L2-resident, as in decoding)"},
+            "roofline": res.pop("roofline"), "cpu_baseline": res.pop("cpu_baseline", None),
+            "e2e": res.pop("e2e", None), "gpu_launches": res.pop("gpu_launches"), "clocks": res.pop("clocks"),
         }
+        line.update(res)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -287,16 +427,19 @@ def run_ours(args, rank, world, local):
 # ---------------------------------------------------------------- reference arm (the oracle)
 
 def run_reference(args, rank, world):
+    """The fp64 CPU oracle, timed on the host cores on a channel sample of the
+    same workload (rank 0 only; other ranks exit without work)."""
     if rank != 0:
-        return
+        return None
     import oracle
     from tests import parity_util as U
     w = workload_of(args)
+    if args.workload == "block":
+        w = W.Workload(w.name, w.batch, w.extra["block"], w.d_inner, w.d_state, w.dtype, w.seed)
     inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed,
                            device="cuda" if torch.cuda.is_available() else "cpu")
     threads = oracle.max_threads()
     per_step = min(30.0, 150.0 / max(1, args.steps + args.warmup))
-    # size one step's channel sample to about per_step seconds
     nch = max(1, threads)
     chans = U.sample_channels(w.d_inner, nch, seed=7)
     si, sp = U.channel_subset(inp, par, chans)
@@ -313,9 +456,9 @@ def run_reference(args, rank, world):
         oracle.layer_fwd(si, sp)
     secs = time.perf_counter() - t0
     layer_s = secs / args.steps * w.d_inner / len(chans)
-    value = w.tokens / layer_s / 1e6
-    sample = f"{len(chans)} of {w.d_inner} channels x {w.batch} batch rows x L={w.L} per step, scaled by " \
-             f"{w.d_inner}/{len(chans)}"
+    value = w.batch * w.L / layer_s / 1e6
+    sample = (f"{len(chans)} of {w.d_inner} channels x {w.batch} batch rows x L={w.L} per step, scaled by "
+              f"{w.d_inner}/{len(chans)}")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(layer_s * 1e3, 3),
@@ -327,6 +470,7 @@ def run_reference(args, rank, world):
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return line
 
 
 def main():

@@ -23,6 +23,8 @@ constexpr int kWPD = 4;      // warps per direction per CTA (full layer)
 constexpr int kWPB = 8;      // warps per CTA (prefix, block step)
 constexpr int kTBlock = 64;  // longest block of the block step
 constexpr int kMaxBatch = 65535;
+constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 1.965 GHz
+constexpr long long kStarveWaitCycles = 200000LL;  // ~0.1 ms: the starved test gives up fast
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -341,6 +343,7 @@ int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_
 template <typename Tin, typename Tout>
 int fused_layer_by_group(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     switch (g) {
+        case 1: return launch_fused_layer<1, Tin, Tout>(k, in, st);
         case 2: return launch_fused_layer<2, Tin, Tout>(k, in, st);
         case 4: return launch_fused_layer<4, Tin, Tout>(k, in, st);
         case 8: return launch_fused_layer<8, Tin, Tout>(k, in, st);
@@ -458,7 +461,7 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
-                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK;
+                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE;
     if (((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if (((flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -482,11 +485,14 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     k.batch = batch;
     k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    k.starve = (flags & BIMAMBA_TEST_STARVE) ? 1 : 0;
+    k.wait_limit = k.starve ? kStarveWaitCycles : kWaitCycles;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int fam = pick_family(2LL * batch * d_inner, flags);
-    if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && (forced == 0 || forced == 2 || forced == 4 || forced == 8) &&
+    const bool group_ok = forced == 0 || forced == 1 || forced == 2 || forced == 4 || forced == 8;
+    if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
         tma_eligible(in, d_inner, true, true)) {
         const int gf = pick_group_fused(flags);
         if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, k, in, st);
@@ -529,6 +535,7 @@ int bimamba_prefix_state(const bimamba_inputs_t* prefix, const bimamba_params_t*
     k.D = d_inner;
     k.batch = batch;
     k.dir_scale[0] = k.dir_scale[1] = 1.f;
+    k.wait_limit = kWaitCycles;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     if (tma_eligible(prefix, d_inner, false, false) && pick_family((int64_t)batch * d_inner, 0) == 2) {
         if (prefix->dtype == BIMAMBA_BF16) return launch_fused_prefix<4, bf16>(k, prefix, st);

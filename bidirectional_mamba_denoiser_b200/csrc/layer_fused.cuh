@@ -40,7 +40,7 @@ struct FusedMaps {
 
 template <int G, typename Tin>
 struct FusedGeo {
-    static_assert(G == 2 || G == 4 || G == 8, "lanes per group");
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "lanes per group");
     static constexpr int T = 16;                // tokens per chunk
     static constexpr int NS = 2;                // ring stages per direction
     static constexpr int S = kNState / G;       // states per lane
@@ -51,7 +51,10 @@ struct FusedGeo {
     static constexpr int BB = ((T * kNState * ESZ) + 127) & ~127;
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
     static constexpr int OWS = T * CW * 4;               // partner's y of a chunk
-    static constexpr int WARP_BYTES = NS * STAGE + OWS;
+    // With G == 1 every lane needs all 16 B and C of a token: they are
+    // converted to fp32 once per chunk (T x 32 floats) instead of per use.
+    static constexpr int BCF = G == 1 ? T * 2 * kNState * 4 : 0;
+    static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF;
     static constexpr int BAR_OFF = 2 * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
     static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
@@ -164,6 +167,30 @@ struct FusedWarp {
     // State updates of step s for the group's G channels (their step sizes
     // gathered from the group's lanes); returns sum_n C h of the own channel
     // (WITH_Y), before the D skip.
+    // G == 1: the lane's own channel, all 16 states; B and C of the token
+    // come as fp32 from the per-chunk buffer bcf ([T][B 16 | C 16]).
+    template <bool WITH_Y>
+    __device__ __forceinline__ float scan1(int s, const Elem& e, const float* bcf) {
+        const float* rowp = bcf + row_of(s) * 2 * kNState;
+        float bv[kNState], cvv[kNState];
+        load_states<kNState>(rowp, bv);
+        if constexpr (WITH_Y) load_states<kNState>(rowp + kNState, cvv);
+        const float2 dd = make_float2(e.dl, e.dl);
+        const float2 uu = make_float2(e.du, e.du);
+        float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int sp = 0; sp < kNState; sp += 2) {
+            const float2 v = mul2(dd, make_float2(A2[0][sp], A2[0][sp + 1]));
+            const float2 ea = make_float2(ex2_approx(v.x), ex2_approx(v.y));
+            const float2 drive = mul2(uu, make_float2(bv[sp], bv[sp + 1]));
+            const float2 hh = fma2(ea, make_float2(h[0][sp], h[0][sp + 1]), drive);
+            h[0][sp] = hh.x;
+            h[0][sp + 1] = hh.y;
+            if constexpr (WITH_Y) acc2 = fma2(make_float2(cvv[sp], cvv[sp + 1]), hh, acc2);
+        }
+        return acc2.x + acc2.y;
+    }
+
     template <bool WITH_Y>
     __device__ __forceinline__ float scan(int s, const Elem& e, const Tin* Bt, const Tin* Ct) {
         const int row = row_of(s);
@@ -197,10 +224,23 @@ struct FusedWarp {
     }
 };
 
+// B and C rows of a chunk (T x 16 each, token order) -> fp32 [T][B 16 | C 16],
+// one warp; lane l handles state l % 16 of B (l < 16) or C (l >= 16).
+template <int T, typename Tin>
+__device__ __forceinline__ void fused_convert_bc(const Tin* Bt, const Tin* Ct, float* bcf, int lane, bool with_c) {
+    const int n = lane & (kNState - 1);
+    const bool isc = lane >= kNState;
+    if (isc && !with_c) return;
+    const Tin* src = isc ? Ct : Bt;
+#pragma unroll 4
+    for (int r = 0; r < T; ++r) bcf[r * 2 * kNState + lane] = ldf(src, r * kNState + n);
+}
+
 template <int G, typename Tin>
 __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char* wbase, uint64_t* full, int r,
-                                            int i, int k, bool gated, int ct0, int b) {
+                                            int i, int k, bool gated, int ct0, int b, int starve) {
     using Ge = FusedGeo<G, Tin>;
+    if (starve) return;
     const int st = i % Ge::NS;
     unsigned char* sb = wbase + st * Ge::STAGE;
     uint64_t* bar = full + st;
@@ -221,6 +261,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     using Wp = FusedWarp<G, Tin, Tout, DIR, true>;
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
+    float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + Ge::BAR_OFF) + DIR * NS;
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
@@ -235,7 +276,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     wp.setup(p, ct0, lane);
     if (lane == 0)
         for (int i = 0; i < NS && i < nc; ++i)
-            fused_issue<G, Tin>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b);
+            fused_issue<G, Tin>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b, p.starve);
 
 #pragma unroll 1
     for (int i = 0; i < nc; ++i) {
@@ -248,7 +289,8 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         // the previous chunk's stage is free (this warp is past it): refill it
         if (lane == 0 && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
-            fused_issue<G, Tin>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b);
+            fused_issue<G, Tin>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b,
+                                p.starve);
         }
         const int nvalid = (int)((L - (int64_t)k * T < T) ? (L - (int64_t)k * T) : T);
         const int s_lo = DIR == 0 ? 0 : T - nvalid;
@@ -265,7 +307,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             cp_async_commit();
         }
         const int st = i % NS;
-        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1));
+        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
         const unsigned char* sb = wbase + st * Ge::STAGE;
         const Tin* xt = reinterpret_cast<const Tin*>(sb);
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);
@@ -274,6 +316,11 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
         if (gated) {
             cp_async_wait_all();
+            __syncwarp();
+        }
+        if constexpr (G == 1) {
+            __syncwarp();
+            fused_convert_bc<T, Tin>(Bt, Ct, bcf, lane, true);
             __syncwarp();
         }
         wp.window(xt);
@@ -285,7 +332,12 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             const bool valid = s >= s_lo && s < s_hi;
             const typename Wp::Elem cur = nxt;
             if (s + 1 < T) nxt = wp.element(s + 1, s + 1 >= s_lo && s + 1 < s_hi, xt, dtt);
-            const float y = (wp.template scan<true>(s, cur, Bt, Ct) + cur.Du) * scale;
+            float yr;
+            if constexpr (G == 1)
+                yr = wp.template scan1<true>(s, cur, bcf);
+            else
+                yr = wp.template scan<true>(s, cur, Bt, Ct);
+            const float y = (yr + cur.Du) * scale;
             if (valid && wp.dvalid) {
                 const int tr = Wp::row_of(s);
                 if (!gated) {
@@ -345,6 +397,7 @@ __global__ void __launch_bounds__(32, 16) fused_prefix_kernel(const __grid_const
     const int nc = (int)((P + T - 1) / T);
     constexpr uint32_t TX = (uint32_t)(((T + 3) * Ge::CW + T * Ge::CW + T * kNState) * Ge::ESZ);
     auto issue = [&](int i) {
+        if (p.starve) return;
         const int st = i % NS;
         unsigned char* sb = base + st * Ge::STAGE;
         uint64_t* bar = full + st;
@@ -362,7 +415,7 @@ __global__ void __launch_bounds__(32, 16) fused_prefix_kernel(const __grid_const
         if (lane == 0 && i >= 1 && i - 1 + NS < nc) issue(i - 1 + NS);
         const int nvalid = (int)((P - (int64_t)i * T < T) ? (P - (int64_t)i * T) : T);
         const int st = i % NS;
-        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1));
+        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
         const unsigned char* sb = base + st * Ge::STAGE;
         const Tin* xt = reinterpret_cast<const Tin*>(sb);
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);

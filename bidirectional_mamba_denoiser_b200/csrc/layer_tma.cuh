@@ -189,8 +189,9 @@ struct TmaWorker {
 
 template <int G, int T, int NWD, int NS, typename Tin>
 __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char* dir_base, uint64_t* full, int r,
-                                            int i, int k, bool gated, int ct0, int b) {
+                                            int i, int k, bool gated, int ct0, int b, int starve) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
+    if (starve) return;
     const int st = i % NS;
     unsigned char* sb = dir_base + st * Ge::STAGE;
     uint64_t* bar = full + st;
@@ -233,7 +234,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     if (leader) {
         for (int i = 0; i < NS && i < nc; ++i) {
             const int k = DIR == 0 ? i : nc - 1 - i;
-            issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i, k, i >= meet, ct0, b);
+            issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i, k, i >= meet, ct0, b, p.starve);
         }
     }
 
@@ -268,7 +269,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         }
 
         const int st = i % NS;
-        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1));
+        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
         const unsigned char* sb = dir_base + st * Ge::STAGE;
         const Tin* xt = reinterpret_cast<const Tin*>(sb);
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);
@@ -281,7 +282,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         if (leader && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
             issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2,
-                                            i2 >= meet, ct0, b);
+                                            i2 >= meet, ct0, b, p.starve);
         }
 
         wk.elements(xt, dtt, s_lo, s_hi, ed2, edu);
@@ -371,6 +372,7 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
     constexpr uint32_t TX = (uint32_t)(((T + 3) * Ge::CW + T * Ge::CW + T * kNState) * Ge::ESZ);
 
     auto issue = [&](int i) {
+        if (p.starve) return;
         const int st = i % NS;
         unsigned char* sb = base + st * Ge::STAGE;
         uint64_t* bar = full + st;
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
 #pragma unroll 1
     for (int i = 0; i < nc; ++i) {
         const int st = i % NS;
-        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1));
+        mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
         const unsigned char* sb = base + st * Ge::STAGE;
         const Tin* xt = reinterpret_cast<const Tin*>(sb);
         const Tin* dtt = reinterpret_cast<const Tin*>(sb + Ge::XB);

@@ -123,6 +123,8 @@ struct KParams {
     int D;
     int batch;
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
+    long long wait_limit;  // SM clocks a wait for a tile may take before it gives up
+    int starve;            // test aid: issue no tile loads, so every such wait gives up
 };
 
 // ---------------------------------------------------------------- geometry

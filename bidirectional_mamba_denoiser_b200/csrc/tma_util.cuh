@@ -51,8 +51,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // `limit_cycles` SM clocks.  On timeout the device error word records it and
 // the caller carries on (its data is then garbage, but every thread still
 // reaches every later barrier, so the kernel ends).
-__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  long long limit_cycles = 4000000000LL) {
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit_cycles) {
     if (mbar_try_wait(bar, parity)) return;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {

@@ -80,9 +80,14 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * size).  1: chunked -- G lanes share one channel's states, for few channels
  * (batch 1, long sequences).  2: per-token fused -- one lane per channel,
  * groups of G lanes share B/C across G channels, for many channels.  With
- * family 2 the lane field (bits 8..12) is the group size (2, 4 or 8). */
+ * family 2 the lane field (bits 8..12) is the group size (1, 2, 4 or 8). */
 #define BIMAMBA_FAMILY_SHIFT 18
 #define BIMAMBA_FAMILY_MASK  (0x3u << BIMAMBA_FAMILY_SHIFT)
+/* Test aid for the failure path: the TMA-fed kernels issue no tile loads,
+ * so every wait for a tile gives up (after ~0.1 ms instead of ~2 s); the
+ * kernel still finishes, its output is undefined, and bit 0 of
+ * bimamba_device_error() is set.  bimamba_layer_fwd only. */
+#define BIMAMBA_TEST_STARVE 0x100000u
 
 /* Parameters of both directions, fp32 device pointers, index 0 = forward. */
 typedef struct {

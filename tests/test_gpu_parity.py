@@ -68,7 +68,7 @@ def test_bf16_ragged_tma_kernel(bm, shape, lanes, chunk):
     assert bm.bimamba_device_error() == 0
 
 
-@pytest.mark.parametrize("group", [2, 4, 8])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
                                    (1, 16, 32), (1, 32, 64), (2, 17, 96)])
 def test_bf16_ragged_fused_kernel(bm, shape, group):
@@ -101,7 +101,8 @@ def test_short_sequences(bm, L):
     ref = oracle.layer_fwd(inp, par)
     for flags in (1 << 8 | bm.BIMAMBA_NO_TMA, 4 << 8 | bm.BIMAMBA_NO_TMA, 16 << 8 | bm.BIMAMBA_NO_TMA,
                   4 << 8 | 1 << 18, 8 << 8 | 1 << 18, 16 << 8 | 1 << 18, 4 << 8 | 1 << 16 | 1 << 18,
-                  16 << 8 | 1 << 16 | 1 << 18, 2 << 8 | 2 << 18, 4 << 8 | 2 << 18, 8 << 8 | 2 << 18):
+                  16 << 8 | 1 << 16 | 1 << 18, 1 << 8 | 2 << 18, 2 << 8 | 2 << 18, 4 << 8 | 2 << 18,
+                  8 << 8 | 2 << 18):
         got = run_layer(bm, inp, par, torch.float32, flags)
         assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
 
