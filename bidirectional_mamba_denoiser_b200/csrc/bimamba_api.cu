@@ -304,9 +304,11 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
 
 // ---- per-token fused kernels (many channels)
 
-template <typename Tin>
+// The boxes come from the kernel's own geometry, so the bytes each TMA load
+// delivers always equal what the kernel's barrier expects.
+template <int G, typename Tin>
 bool fill_fused_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool layer) {
-    constexpr int T = 16, CW = 32;
+    constexpr int T = bimamba::FusedGeo<G, Tin>::T, CW = bimamba::FusedGeo<G, Tin>::CW;
     const bool bf = std::is_same<Tin, bf16>::value;
     bool ok = map3d(&m.x, in->x, bf, D, L, batch, CW, T + 3);
     ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, CW, T);
@@ -331,7 +333,7 @@ template <int G, typename Tin, typename Tout>
 int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     using Ge = bimamba::FusedGeo<G, Tin>;
     bimamba::FusedMaps maps;
-    if (!fill_fused_maps<Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
+    if (!fill_fused_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
     auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
@@ -355,7 +357,7 @@ template <int G, typename Tin>
 int launch_fused_prefix(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     using Ge = bimamba::FusedGeo<G, Tin>;
     bimamba::FusedMaps maps;
-    if (!fill_fused_maps<Tin>(maps, in, k.batch, k.L, k.D, false)) return BIMAMBA_ERR_CUDA;
+    if (!fill_fused_maps<G, Tin>(maps, in, k.batch, k.L, k.D, false)) return BIMAMBA_ERR_CUDA;
     auto kern = &bimamba::fused_prefix_kernel<G, Tin>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
@@ -389,14 +391,15 @@ int pick_chunk_tma(unsigned flags, int lanes) {
     return lanes >= 8 ? 32 : 16;
 }
 
-// Lanes per channel of the TMA kernels: 4, 8 or 16 (same rule as pick_lanes).
+// Lanes per channel of the chunked kernel: 4 when that gives about one
+// thread slot per SM thread (148 SMs x 1024), else 8.  16 lanes (one state
+// each) measured slower than 8 even at batch 1 (10.0 ms against 7.1 ms at
+// L 65536, d_inner 4096): its per-state reduction overhead outweighs the
+// extra parallelism.
 int pick_lanes_tma(int64_t chains, unsigned flags) {
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     if (forced) return (int)forced;
-    const int64_t target = 148LL * 1024;
-    int g = 4;
-    while (g < 16 && chains * g < target) g *= 2;
-    return g;
+    return chains * 4 >= 148LL * 1024 ? 4 : 8;
 }
 
 int check_inputs(const bimamba_inputs_t* in, bool need_reverse, bool need_z_c) {

@@ -59,6 +59,7 @@ struct FusedGeo {
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
     static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
     static constexpr uint32_t TX_Z = (uint32_t)(T * CW * ESZ);
+    static_assert(T + 3 <= 256 && CW <= 256, "TMA box dimensions");
 };
 
 // S consecutive B (or C) values of a token row, as fp32.
