@@ -9,6 +9,7 @@
 #include <utility>
 
 #include "bimamba.h"
+#include "block_fused.cuh"
 #include "layer_fused.cuh"
 #include "layer_tma.cuh"
 #include "scan_kernels.cuh"
@@ -402,6 +403,19 @@ int pick_lanes_tma(int64_t chains, unsigned flags) {
     return chains * 4 >= 148LL * 1024 ? 4 : 8;
 }
 
+// ---- block step on the per-token fused layout (the default)
+
+template <typename Tin, typename Tout>
+int launch_fused_block(const KParams& k, cudaStream_t st) {
+    auto kern = &bimamba::fused_block_kernel<Tin, Tout>;
+    const size_t smem = 2 * sizeof(float) * (size_t)bimamba::block_dir_floats((int)k.L);
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), 2 * sizeof(float) * bimamba::block_dir_floats(kTBlock));
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + 31) / 32), (unsigned)k.batch);
+    kern<<<grid, 64, smem, st>>>(k);
+    return launch_status();
+}
+
 int check_inputs(const bimamba_inputs_t* in, bool need_reverse, bool need_z_c) {
     if (!in || !in->x || !in->dt[0] || !in->B[0]) return BIMAMBA_ERR_INVALID_ARG;
     if (need_z_c && (!in->z || !in->C[0])) return BIMAMBA_ERR_INVALID_ARG;
@@ -586,9 +600,15 @@ int bimamba_block_step(const bimamba_fwd_state_t* prefix_state, const bimamba_in
     k.batch = batch;
     k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
-    const int g = pick_lanes((int64_t)batch * d_inner, flags);
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = block->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if ((flags & BIMAMBA_LANES_MASK) == 0) {
+        if (in_bf && out_bf) return launch_fused_block<bf16, bf16>(k, st);
+        if (in_bf) return launch_fused_block<bf16, float>(k, st);
+        if (out_bf) return launch_fused_block<float, bf16>(k, st);
+        return launch_fused_block<float, float>(k, st);
+    }
+    const int g = pick_lanes((int64_t)batch * d_inner, flags);
     if (in_bf && out_bf) return block_by_lanes<bf16, bf16>(g, k, st);
     if (in_bf) return block_by_lanes<bf16, float>(g, k, st);
     if (out_bf) return block_by_lanes<float, bf16>(g, k, st);

@@ -171,7 +171,9 @@ int bimamba_prefix_state(const bimamba_inputs_t *prefix, const bimamba_params_t 
  * conv zero-padded past its end).  out: [batch][block_len][d_inner] of
  * out_dtype.  If new_state is not NULL the forward state after the block is
  * written there (commit); new_state may be prefix_state itself (in place).
- * block_len must be in [1, 64].  One kernel launch. */
+ * block_len must be in [1, 64].  One kernel launch.  A non-zero lane field in
+ * flags (bits 8..12) selects the earlier kernel that splits a channel's states
+ * over that many lanes (test aid). */
 int bimamba_block_step(const bimamba_fwd_state_t *prefix_state, const bimamba_inputs_t *block,
                        int block_len, const bimamba_params_t *p,
                        void *out, bimamba_dtype_t out_dtype,

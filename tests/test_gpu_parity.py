@@ -186,8 +186,9 @@ def _slice_tokens(inp, lo, hi):
             for k, v in inp.items() if v is not None}
 
 
+@pytest.mark.parametrize("lanes", [0, 4])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_block_chain_matches_oracle(bm, dtype):
+def test_block_chain_matches_oracle(bm, dtype, lanes):
     """Prefix of 512 tokens, then 16 blocks of 32 committed one after another
     (L = 1024 in all): every block's output and the committed state against
     the oracle's own block chain."""
@@ -207,15 +208,16 @@ def test_block_chain_matches_oracle(bm, dtype):
         ref, h_ref, t_ref = oracle.block_step(h_ref, t_ref, blk, par, commit=True)
         dblk = U.to_device(blk)
         out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                                    out_dtype=torch.float32, new_state=(h, tail))
+                                    out_dtype=torch.float32, new_state=(h, tail), flags=lanes << 8)
         torch.cuda.synchronize()
         assert U.normwise(U.to_cpu64(out), ref) <= tol, k
         assert U.normwise(U.to_cpu64(h), h_ref) <= U.GUARD, k
         assert np.array_equal(U.to_cpu64(tail), t_ref), k
 
 
+@pytest.mark.parametrize("lanes", [0, 8])
 @pytest.mark.parametrize("G", [1, 2, 3, 5, 31, 33, 64])
-def test_block_step_ragged_lengths(bm, G):
+def test_block_step_ragged_lengths(bm, G, lanes):
     b, D, P = 2, 24, 70
     inp, par = W.make_case(b, P + G, D, 16, "fp32", seed=30 + G)
     pre, blk = _slice_tokens(inp, 0, P), _slice_tokens(inp, P, P + G)
@@ -225,7 +227,7 @@ def test_block_step_ragged_lengths(bm, G):
     h, tail = bm.bimamba_prefix_state(dpre["x"], dpre["dt"], dpre["B"], dpar)
     h2, t2 = torch.empty_like(h), torch.empty_like(tail)
     out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                                out_dtype=torch.float32, new_state=(h2, t2))
+                                out_dtype=torch.float32, new_state=(h2, t2), flags=lanes << 8)
     torch.cuda.synchronize()
     assert U.normwise(U.to_cpu64(out), ref) <= U.TOL_FP32
     assert U.normwise(U.to_cpu64(h2), h2_ref) <= U.TOL_FP32
