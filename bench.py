@@ -62,7 +62,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["layer", "long", "block", "sweep"], default="layer")
-    ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep")
+    ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
     ap.add_argument("--family", type=int, default=0, help="kernel family: 0 auto, 1 chunked, 2 per-token fused")
@@ -76,6 +76,10 @@ def workload_of(args) -> W.Workload:
     if args.workload == "layer":
         return W.LAYER_1P3B
     if args.workload == "block":
+        if args.L:  # a shorter cached prefix (same block steps)
+            w = W.BLOCK_CACHED
+            return W.Workload(f"block_cached_b{w.batch}_P{args.L}_G{w.L}_D{w.d_inner}_{w.dtype}", w.batch, w.L,
+                              w.d_inner, w.d_state, w.dtype, w.seed, extra={**w.extra, "prefix": args.L})
         return W.BLOCK_CACHED
     if args.workload == "sweep":
         L = args.L or 8192

@@ -416,6 +416,27 @@ int launch_fused_block(const KParams& k, cudaStream_t st) {
     return launch_status();
 }
 
+template <typename Tin, typename Tout>
+int launch_async_block(const KParams& k, cudaStream_t st) {
+    auto kern = &bimamba::async_block_kernel<Tin, Tout>;
+    const size_t smem = (size_t)bimamba::async_block_smem<Tin>((int)k.L);
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), (size_t)bimamba::async_block_smem<Tin>(kTBlock));
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + 31) / 32), (unsigned)k.batch);
+    kern<<<grid, 64, smem, st>>>(k);
+    return launch_status();
+}
+
+// The cp.async-staged block kernel copies 16-byte pieces of 32-channel rows:
+// every row must start on a 16-byte boundary.
+bool async_block_eligible(const bimamba_inputs_t* in, const void* tail, int d_inner) {
+    if ((d_inner * elem_size(in->dtype)) % 16 != 0) return false;
+    const void* ptrs[9] = {in->x, in->z, in->dt[0], in->dt[1], in->B[0], in->B[1], in->C[0], in->C[1], tail};
+    for (const void* q : ptrs)
+        if (!aligned(q, 16)) return false;
+    return true;
+}
+
 int check_inputs(const bimamba_inputs_t* in, bool need_reverse, bool need_z_c) {
     if (!in || !in->x || !in->dt[0] || !in->B[0]) return BIMAMBA_ERR_INVALID_ARG;
     if (need_z_c && (!in->z || !in->C[0])) return BIMAMBA_ERR_INVALID_ARG;
@@ -573,7 +594,7 @@ int bimamba_block_step(const bimamba_fwd_state_t* prefix_state, const bimamba_in
                        int d_state, bimamba_fwd_state_t* new_state, unsigned flags, void* cuda_stream) {
     if (batch <= 0 || batch > kMaxBatch || d_inner <= 0 || !out || block_len <= 0) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState || block_len > kTBlock) return BIMAMBA_ERR_UNSUPPORTED;
-    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK;
+    const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -602,6 +623,13 @@ int bimamba_block_step(const bimamba_fwd_state_t* prefix_state, const bimamba_in
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = block->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if ((flags & BIMAMBA_LANES_MASK) == 0 && !(flags & BIMAMBA_NO_TMA) &&
+        async_block_eligible(block, prefix_state->conv_x, d_inner)) {
+        if (in_bf && out_bf) return launch_async_block<bf16, bf16>(k, st);
+        if (in_bf) return launch_async_block<bf16, float>(k, st);
+        if (out_bf) return launch_async_block<float, bf16>(k, st);
+        return launch_async_block<float, float>(k, st);
+    }
     if ((flags & BIMAMBA_LANES_MASK) == 0) {
         if (in_bf && out_bf) return launch_fused_block<bf16, bf16>(k, st);
         if (in_bf) return launch_fused_block<bf16, float>(k, st);

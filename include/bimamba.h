@@ -171,9 +171,13 @@ int bimamba_prefix_state(const bimamba_inputs_t *prefix, const bimamba_params_t 
  * conv zero-padded past its end).  out: [batch][block_len][d_inner] of
  * out_dtype.  If new_state is not NULL the forward state after the block is
  * written there (commit); new_state may be prefix_state itself (in place).
- * block_len must be in [1, 64].  One kernel launch.  A non-zero lane field in
- * flags (bits 8..12) selects the earlier kernel that splits a channel's states
- * over that many lanes (test aid). */
+ * block_len must be in [1, 64].  One kernel launch.  The block's rows are
+ * staged with asynchronous 16-byte copies when every x/z/dt/B/C pointer and
+ * prefix_state->conv_x is 16-byte aligned and a row of d_inner elements is a
+ * whole number of 16-byte units; otherwise, or with BIMAMBA_NO_TMA, with
+ * ordinary loads.  A non-zero lane field in flags (bits 8..12) selects the
+ * earlier kernel that splits a channel's states over that many lanes (test
+ * aid).  The results do not depend on the kernel beyond fp32 rounding order. */
 int bimamba_block_step(const bimamba_fwd_state_t *prefix_state, const bimamba_inputs_t *block,
                        int block_len, const bimamba_params_t *p,
                        void *out, bimamba_dtype_t out_dtype,

@@ -10,6 +10,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a) and the built CUDA library")
+    # the tests load the in-tree library: rebuild it when a source is newer
+    from bidirectional_mamba_denoiser_b200 import build
+    if build.stale():
+        build.build()
 
 
 def _has_cuda():

@@ -186,9 +186,14 @@ def _slice_tokens(inp, lo, hi):
             for k, v in inp.items() if v is not None}
 
 
-@pytest.mark.parametrize("lanes", [0, 4])
+# block-step kernels: 0 = rows staged by cp.async, NO_TMA = ordinary loads,
+# a lane count = the kernel that splits a channel's states over lanes
+BLOCK_KERNELS = {"async": 0, "plain": 0x4000, "split4": 4 << 8, "split8": 8 << 8}
+
+
+@pytest.mark.parametrize("kernel", ["async", "plain", "split4"])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_block_chain_matches_oracle(bm, dtype, lanes):
+def test_block_chain_matches_oracle(bm, dtype, kernel):
     """Prefix of 512 tokens, then 16 blocks of 32 committed one after another
     (L = 1024 in all): every block's output and the committed state against
     the oracle's own block chain."""
@@ -208,17 +213,20 @@ def test_block_chain_matches_oracle(bm, dtype, lanes):
         ref, h_ref, t_ref = oracle.block_step(h_ref, t_ref, blk, par, commit=True)
         dblk = U.to_device(blk)
         out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                                    out_dtype=torch.float32, new_state=(h, tail), flags=lanes << 8)
+                                    out_dtype=torch.float32, new_state=(h, tail), flags=BLOCK_KERNELS[kernel])
         torch.cuda.synchronize()
         assert U.normwise(U.to_cpu64(out), ref) <= tol, k
         assert U.normwise(U.to_cpu64(h), h_ref) <= U.GUARD, k
         assert np.array_equal(U.to_cpu64(tail), t_ref), k
 
 
-@pytest.mark.parametrize("lanes", [0, 8])
+@pytest.mark.parametrize("kernel", ["async", "plain", "split8"])
 @pytest.mark.parametrize("G", [1, 2, 3, 5, 31, 33, 64])
-def test_block_step_ragged_lengths(bm, G, lanes):
-    b, D, P = 2, 24, 70
+@pytest.mark.parametrize("D", [24, 18])
+def test_block_step_ragged_lengths(bm, G, kernel, D):
+    """d_inner 18 (72-byte rows) cannot take 16-byte copies: the default then
+    falls back to ordinary loads."""
+    b, P = 2, 70
     inp, par = W.make_case(b, P + G, D, 16, "fp32", seed=30 + G)
     pre, blk = _slice_tokens(inp, 0, P), _slice_tokens(inp, P, P + G)
     h_ref, t_ref = oracle.prefix_state(pre, par)
@@ -227,7 +235,7 @@ def test_block_step_ragged_lengths(bm, G, lanes):
     h, tail = bm.bimamba_prefix_state(dpre["x"], dpre["dt"], dpre["B"], dpar)
     h2, t2 = torch.empty_like(h), torch.empty_like(tail)
     out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                                out_dtype=torch.float32, new_state=(h2, t2), flags=lanes << 8)
+                                out_dtype=torch.float32, new_state=(h2, t2), flags=BLOCK_KERNELS[kernel])
     torch.cuda.synchronize()
     assert U.normwise(U.to_cpu64(out), ref) <= U.TOL_FP32
     assert U.normwise(U.to_cpu64(h2), h2_ref) <= U.TOL_FP32
@@ -235,12 +243,13 @@ def test_block_step_ragged_lengths(bm, G, lanes):
     # without commit the cached state is left alone
     h_before = h.clone()
     bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                          out_dtype=torch.float32)
+                          out_dtype=torch.float32, flags=BLOCK_KERNELS[kernel])
     torch.cuda.synchronize()
     assert torch.equal(h, h_before)
 
 
-def test_block_step_flags(bm):
+@pytest.mark.parametrize("kernel", ["async", "plain"])
+def test_block_step_flags(bm, kernel):
     b, D, P, G = 1, 16, 40, 32
     inp, par = W.make_case(b, P + G, D, 16, "fp32", seed=41)
     pre, blk = _slice_tokens(inp, 0, P), _slice_tokens(inp, P, P + G)
@@ -250,7 +259,7 @@ def test_block_step_flags(bm):
     for f_or, f_bm in ((oracle.FWD_ONLY, bm.BIMAMBA_FWD_ONLY), (oracle.REV_ONLY, bm.BIMAMBA_REV_ONLY)):
         ref = oracle.block_step(h_ref, t_ref, blk, par, flags=f_or)
         out = bm.bimamba_block_step((h, tail), dblk["x"], dblk["z"], dblk["dt"], dblk["B"], dblk["C"], dpar,
-                                    out_dtype=torch.float32, flags=f_bm)
+                                    out_dtype=torch.float32, flags=f_bm | BLOCK_KERNELS[kernel])
         torch.cuda.synchronize()
         assert U.normwise(U.to_cpu64(out), ref) <= U.TOL_FP32
 
