@@ -50,8 +50,15 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 
 # DRAM bytes (read + write) per launch from the ncu capture summarised in
 # profiles/ -- the workload and kernel they were taken on; anything else null.
+# The chunked kernel's figure was taken at L 16384 and scaled by the token
+# count (its traffic is linear in L); the block step's at a 4096-token prefix
+# (a step reads the same bytes whatever the prefix length).
 NCU_TRAFFIC = {
-    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1306.8e6,
+    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1304.8e6,
+    ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1414.2e6,
+    ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1414.2e6,
+    ("block_cached_b16_P65536_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
+    ("block_cached_b16_P4096_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
 }
 
 
@@ -274,7 +281,7 @@ def flags_of(args, bm):
 
 def kernel_name(w: W.Workload, args) -> str:
     if args.workload == "block":
-        return "block_kernel"
+        return "async_block_kernel"
     fam = args.family or (2 if 2 * w.batch * w.d_inner >= SMS * 8 * 32 else 1)
     return "fused_layer_kernel" if fam == 2 else "layer_tma_kernel"
 
@@ -348,6 +355,8 @@ def run_block(args, w, bm, rank, world, dev, stream):
     pre = W.make_inputs(w.batch, P, w.d_inner, w.d_state, w.dtype, g, dev)
     h = torch.empty(w.batch, w.d_inner, w.d_state, device=dev, dtype=torch.float32)
     tail = torch.empty(w.batch, 3, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
+    # one untimed call first: the first launch of a kernel also loads its module
+    bm.bimamba_prefix_state(pre["x"], pre["dt"], pre["B"], par, h_out=h, conv_x_out=tail, stream=stream)
     torch.cuda.synchronize(dev)
     p0 = torch.cuda.Event(enable_timing=True)
     p1 = torch.cuda.Event(enable_timing=True)
@@ -389,7 +398,7 @@ def run_block(args, w, bm, rank, world, dev, stream):
     return {
         "value": whole_job_rate(w.batch * G * nsteps, world, ms_max / 1e3),
         "ms_per_step": ms_max / nsteps, "gpu_launches": nsteps,
-        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, step_ms, clocks, w.name, "block_kernel"),
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, step_ms, clocks, w.name, kernel_name(w, args)),
         "hbm": hbm_fraction(block_bytes(w), step_ms), "clocks": clocks,
         "prefix_state_ms": round(prefix_ms, 3),
         "prefix_mufu_frac": roofline(MUFU_PER_ELEM_FWD * w.batch * P * w.d_inner, prefix_ms, clocks, w.name,
