@@ -18,6 +18,16 @@ parameters, as the throughput workloads use them):
 Draw order from one ``torch.Generator`` seeded with ``seed`` (fixed, so a
 seed names one input set):
   bias_f, bias_b, w_f, b_f, w_b, b_b, x, z, dt_f, dt_b, B_f, C_f, B_b, C_b
+
+The Mamba-2 mixer at the pages' shape (H heads of P channels, one group of B
+and C with N states, conv over the C_conv = H*P + 2N channels of xBC):
+
+  xbc_r (x | B | C per direction), z, dt_raw ~ N(0, 1)   [b, L, C_conv], [b, L, H*P], [b, L, H]
+  dt_bias[r, h]            = log(expm1(s)), s log-uniform in [1e-3, 1e-1]
+  A[r, h]                  = -a, a ~ U(1, 16)               (Mamba-2 initialisation range)
+  D[r, h]                  = 1
+  conv_w[r, c, k], conv_b  ~ U(-0.5, 0.5)
+  draw order: bias_f, bias_b, A_f, A_b, w_f, b_f, w_b, b_b, xbc_f, xbc_b, z, dt_f, dt_b
 Floating tensors are drawn in fp32 and then rounded (RNE) to the I/O dtype;
 the oracle receives exactly the rounded values widened to fp64.  A CPU
 generator and a CUDA generator give different streams for the same seed, so
@@ -130,3 +140,63 @@ def make_case(batch: int, L: int, D: int, N: int = 16, dtype: str = "bf16", seed
 
 def make_workload(w: Workload, device="cpu"):
     return make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device)
+
+
+# ---------------------------------------------------------------- Mamba-2 mixer
+
+def make_mamba2_params(H: int, P: int, N: int, g: torch.Generator, device="cpu") -> dict:
+    """Parameters of both directions (fp32).  Draws bias_f, bias_b, A_f, A_b, w_f, b_f, w_b, b_b."""
+    CH = H * P + 2 * N
+    lo, hi = math.log(1e-3), math.log(1e-1)
+    bias = []
+    for _ in range(2):
+        s = torch.exp(torch.rand(H, generator=g, device=device, dtype=torch.float64) * (hi - lo) + lo)
+        bias.append(torch.log(torch.expm1(s)).float())
+    A = [-(1.0 + 15.0 * torch.rand(H, generator=g, device=device)) for _ in range(2)]
+    w, cb = [], []
+    for _ in range(2):
+        w.append(torch.rand(CH, D_CONV, generator=g, device=device) - 0.5)
+        cb.append(torch.rand(CH, generator=g, device=device) - 0.5)
+    return {
+        "A": torch.stack(A).contiguous(),                   # [2, H]
+        "D": torch.ones(2, H, device=device),               # [2, H]
+        "dt_bias": torch.stack(bias).contiguous(),          # [2, H]
+        "conv_w": torch.stack(w).contiguous(),              # [2, CH, 4]
+        "conv_b": torch.stack(cb).contiguous(),             # [2, CH]
+    }
+
+
+def make_mamba2_inputs(batch: int, L: int, H: int, P: int, N: int, dtype: str, g: torch.Generator,
+                       device="cpu") -> dict:
+    """Mixer inputs.  Draws xbc_f, xbc_b, z, dt_f, dt_b."""
+    td = torch_dtype(dtype)
+    CH = H * P + 2 * N
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=device, dtype=torch.float32).to(td)
+
+    xbc = torch.empty(2, batch, L, CH, device=device, dtype=td)
+    xbc[0] = randn(batch, L, CH)
+    xbc[1] = randn(batch, L, CH)
+    z = randn(batch, L, H * P)
+    dt = torch.empty(2, batch, L, H, device=device, dtype=td)
+    dt[0] = randn(batch, L, H)
+    dt[1] = randn(batch, L, H)
+    return {"xbc": xbc, "z": z, "dt": dt}
+
+
+def make_mamba2_case(batch: int, L: int, H: int, P: int, N: int, dtype: str = "bf16", seed: int = 0,
+                     device="cpu"):
+    """(inputs, params) for one Mamba-2 mixer call, drawn in the documented order."""
+    g = _gen(seed, device)
+    params = make_mamba2_params(H, P, N, g, device)
+    inputs = make_mamba2_inputs(batch, L, H, P, N, dtype, g, device)
+    return inputs, params
+
+
+# The pages' 1.3B denoiser layer: d_inner 3840 = 120 heads x 32, d_state 128.
+MAMBA2_1P3B = Workload("mamba2_1p3b_b8_L2048_H120x32_N128_bf16", 8, 2048, 3840, 128, "bf16", 5,
+                       extra={"nheads": 120, "headdim": 32})
+MAMBA2_LONG = {L: Workload(f"mamba2_b1_L{L}_H120x32_N128_bf16", 1, L, 3840, 128, "bf16", 6,
+                           extra={"nheads": 120, "headdim": 32})
+               for L in (4096, 16384, 65536)}

@@ -21,6 +21,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bimamba_oracle.c")
+_SRC2 = os.path.join(_HERE, "mamba2_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 FWD_ONLY = 1
@@ -45,11 +46,28 @@ MUTATIONS = {
 }
 
 
+MUTATIONS2 = {
+    1: "B and C skip the conv",
+    2: "A taken from the next head",
+    3: "delta taken from the next head",
+    4: "reverse conv made causal",
+    5: "C reads the state before the update",
+    6: "D skip dropped",
+    7: "B read from the C slice",
+    8: "dt bias dropped",
+    9: "reverse direction walks forwards",
+    10: "delta missing on the drive",
+    11: "gate is silu of the sum times z",
+    12: "x channels laid out p-major instead of head-major",
+}
+
+
 def build(force: bool = False) -> str:
     """Compile liboracle.so with gcc (-O2, OpenMP, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC2))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-               "-fno-fast-math", "-o", _LIB, _SRC, "-lm"]
+               "-fno-fast-math", "-o", _LIB, _SRC, _SRC2, "-lm"]
         subprocess.run(cmd, check=True)
     return _LIB
 
@@ -72,6 +90,9 @@ def _load():
         lib.oracle_prefix_state.restype = I
         lib.oracle_block_step.argtypes = [I, Lg, I, I, P, P] + [P] * 13 + [U, P, P, P, P, P]
         lib.oracle_block_step.restype = I
+        lib.oracle2_layer_fwd.argtypes = [I, Lg, I, I, I] + [P] * 10 + [U, P, P, P]
+        lib.oracle2_layer_fwd.restype = I
+        lib.oracle2_set_mutation.argtypes = [I]
         lib.oracle_set_mutation.argtypes = [I]
         lib.oracle_get_mutation.restype = I
         lib.oracle_set_threads.argtypes = [I]
@@ -96,6 +117,11 @@ def _ptr(a):
 def set_mutation(m: int) -> None:
     """Plant mistake ``m`` (see MUTATIONS) in the oracle; 0 restores it."""
     _load().oracle_set_mutation(int(m))
+
+
+def set_mutation2(m: int) -> None:
+    """Plant mistake ``m`` (see MUTATIONS2) in the Mamba-2 oracle; 0 restores it."""
+    _load().oracle2_set_mutation(int(m))
 
 
 def set_threads(n: int) -> None:
@@ -201,3 +227,38 @@ def block_step(h, tail, inp: dict, params: dict, flags: int = 0, commit: bool = 
     if return_dirs:
         res += [yf, yr]
     return res[0] if len(res) == 1 else tuple(res)
+
+
+# ---------------------------------------------------------------- Mamba-2 mixer
+
+def mamba2_dims(inp: dict):
+    """(batch, L, H, P, N) of a Mamba-2 input dict."""
+    dt, z, xbc = inp["dt"], inp["z"], inp["xbc"]
+    b, L, H = dt.shape[1], dt.shape[2], dt.shape[3]
+    HP = z.shape[-1]
+    P = HP // H
+    N = (xbc.shape[-1] - HP) // 2
+    return b, L, H, P, N
+
+
+def mamba2_layer_fwd(inp: dict, params: dict, flags: int = 0, return_dirs: bool = False):
+    """Full-sequence bidirectional Mamba-2 mixer (mamba2_oracle.c).
+
+    inp: xbc [2, b, L, H*P + 2N] (per direction: x | B | C before the conv);
+         z [b, L, H*P]; dt [2, b, L, H]
+    params: A, D, dt_bias [2, H]; conv_w [2, H*P + 2N, 4]; conv_b [2, H*P + 2N] or None
+    Returns out [b, L, H*P] (and y_fwd, y_rev when return_dirs).
+    """
+    b, L, H, P, N = mamba2_dims(inp)
+    xbc, z, dt = _f64(inp["xbc"]), _f64(inp["z"]), _f64(inp["dt"])
+    x0, x1 = np.ascontiguousarray(xbc[0]), np.ascontiguousarray(xbc[1])
+    dt0, dt1 = np.ascontiguousarray(dt[0]), np.ascontiguousarray(dt[1])
+    A, Dk, bias, w, cb = _params(params)
+    out = np.empty((b, L, H * P), np.float64)
+    yf = np.empty_like(out) if return_dirs else None
+    yr = np.empty_like(out) if return_dirs else None
+    rc = _load().oracle2_layer_fwd(b, L, H, P, N, *map(_ptr, (x0, x1, z, dt0, dt1, A, Dk, bias, w, cb)),
+                                   flags, _ptr(out), _ptr(yf), _ptr(yr))
+    if rc != 0:
+        raise RuntimeError("oracle2_layer_fwd failed")
+    return (out, yf, yr) if return_dirs else out
