@@ -36,6 +36,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from bidirectional_mamba_denoiser_b200 import workloads as W  # noqa: E402
@@ -68,7 +69,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep"], default="layer")
+    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "mamba2", "mamba2_long"],
+                    default="layer")
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
@@ -82,6 +84,12 @@ def parse_args(argv=None):
 def workload_of(args) -> W.Workload:
     if args.workload == "layer":
         return W.LAYER_1P3B
+    if args.workload == "mamba2":
+        return W.MAMBA2_1P3B
+    if args.workload == "mamba2_long":
+        L = args.L or 16384
+        return W.MAMBA2_LONG.get(L) or W.Workload(f"mamba2_b1_L{L}_H120x32_N128_bf16", 1, L, 3840, 128, "bf16",
+                                                  6, extra={"nheads": 120, "headdim": 32})
     if args.workload == "block":
         if args.L:  # a shorter cached prefix (same block steps)
             w = W.BLOCK_CACHED
@@ -407,6 +415,102 @@ def run_block(args, w, bm, rank, world, dev, stream):
     }
 
 
+# ---------------------------------------------------------------- Mamba-2 mixer
+
+FP32_FMA_PER_SM_CLK = 128     # FP32 lanes per SM per clock (B200), one FMA each
+
+
+def mamba2_bytes(batch: int, L: int, H: int, P: int, N: int, esz: int = 2) -> int:
+    """Bytes one Mamba-2 mixer call must move: xBC of both directions, z, dt of
+    both directions read and out written."""
+    CH = H * P + 2 * N
+    return batch * L * (2 * CH + H * P + 2 * H + H * P) * esz
+
+
+def roofline_fma(flops: float, call_ms: float, clocks, workload: str, kernel: str):
+    """Binding roof of the Mamba-2 scan on CUDA cores: FP32 FMA throughput,
+    148 SMs x 128 lanes x 2 flops x the SM clock."""
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = SMS * FP32_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
+    achieved = flops / (call_ms / 1e3) / 1e12
+    return {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 2), "unit": "TFLOP/s (FP32 FMA)",
+            "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get((workload, kernel)),
+            "peak_source": f"148 SMs x {FP32_FMA_PER_SM_CLK} FP32 lanes x 2 x {mhz:.0f} MHz", "kernel": kernel}
+
+
+def mamba2_oracle_rate(w: W.Workload, inputs, params, budget_s: float):
+    """The fp64 oracle on a sample of heads, scaled to all heads:
+    (Mtokens/s, heads, seconds, threads)."""
+    import oracle
+    from tests import parity_util as U
+    H = w.extra["nheads"]
+    threads = oracle.max_threads()
+    k = 1
+    while True:
+        heads = sorted({int(h) for h in np.linspace(0, H - 1, k)})
+        si, sp, _ = U.head_subset(inputs, params, heads)
+        t0 = time.perf_counter()
+        oracle.mamba2_layer_fwd(si, sp)
+        dt = time.perf_counter() - t0
+        if dt >= 0.3 * budget_s or len(heads) >= H:
+            break
+        k = int(min(H, max(k + 1, k * 0.6 * budget_s / max(dt, 1e-3))))
+    layer_s = dt * H / len(heads)
+    return w.batch * w.L / layer_s / 1e6, len(heads), dt, threads
+
+
+def run_mamba2(args, w, bm, rank, world, dev, stream):
+    """mamba2 / mamba2_long: steps of bimamba2_layer_fwd (three launches each)."""
+    H, P, N = w.extra["nheads"], w.extra["headdim"], w.d_state
+    sets = [W.make_mamba2_case(w.batch, w.L, H, P, N, w.dtype, w.seed + 1000 * i + rank, device=dev)
+            for i in range(2)]
+    out = torch.empty(w.batch, w.L, H * P, device=dev, dtype=W.torch_dtype(w.dtype))
+    ws = torch.empty(bm.bimamba2_workspace_bytes(w.batch, w.L, H, P, N), device=dev, dtype=torch.uint8)
+
+    def step(i):
+        inp, par = sets[i % 2]
+        bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out=out, workspace=ws, stream=stream)
+
+    ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    call_ms = ms / args.steps
+    tokens = w.batch * w.L
+    flops = 4.0 * P * N * H * 2 * tokens  # two FMAs per state per token and direction
+    res = {
+        "value": whole_job_rate(tokens * args.steps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / args.steps,
+        "gpu_launches": 3 * args.steps,
+        "roofline": roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel"),
+        "hbm": hbm_fraction(mamba2_bytes(w.batch, w.L, H, P, N), call_ms),
+        "clocks": clocks,
+        "flops_per_token": int(flops / tokens),
+    }
+    if not args.no_e2e:
+        inp, par = sets[0]
+        host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}
+        dbuf = {k: torch.empty_like(v) for k, v in inp.items()}
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        k2 = max(3, min(args.steps, 20))
+
+        def e2e_step(i):
+            for k in host:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            bm.bimamba2_layer_fwd(dbuf["xbc"], dbuf["z"], dbuf["dt"], par, out=out, workspace=ws, stream=stream)
+            hout.copy_(out, non_blocking=True)
+
+        ms2, _ = timed(e2e_step, k2, 2, world, dev, stream)
+        res["e2e"] = {"value": round(whole_job_rate(tokens * k2, world, max_over_ranks(ms2, world) / 1e3), 4),
+                      "unit": UNIT, "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": k2}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp, par = sets[0]
+        v, nh, secs, thr = mamba2_oracle_rate(w, inp, par, args.cpu_budget)
+        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+                               "sample": f"{nh} of {H} heads x {w.batch} batch rows x L={w.L} ({secs:.1f} s), "
+                                         f"scaled by {H}/{nh}"}
+    return res
+
+
 def run_ours(args, rank, world, local):
     from bidirectional_mamba_denoiser_b200 import bimamba as bm
     w = workload_of(args)
@@ -416,6 +520,8 @@ def run_ours(args, rank, world, local):
         side = torch.cuda.Stream(dev)  # graphs cannot be captured on the legacy default stream
         with torch.cuda.stream(side):
             res = run_block(args, w, bm, rank, world, dev, side)
+    elif args.workload in ("mamba2", "mamba2_long"):
+        res = run_mamba2(args, w, bm, rank, world, dev, stream)
     else:
         res = run_layer_like(args, w, bm, rank, world, dev, stream)
     if rank == 0:
@@ -449,8 +555,10 @@ def run_reference(args, rank, world):
     w = workload_of(args)
     if args.workload == "block":
         w = W.Workload(w.name, w.batch, w.extra["block"], w.d_inner, w.d_state, w.dtype, w.seed)
-    inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed,
-                           device="cuda" if torch.cuda.is_available() else "cpu")
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if args.workload in ("mamba2", "mamba2_long"):
+        return run_reference_mamba2(args, w, world, dev)
+    inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device=dev)
     threads = oracle.max_threads()
     per_step = min(30.0, 150.0 / max(1, args.steps + args.warmup))
     nch = max(1, threads)
@@ -478,6 +586,45 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                    "d_state": w.d_state, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def run_reference_mamba2(args, w, world, dev):
+    """The reference arm for the Mamba-2 workloads: the fp64 oracle on a sample
+    of heads per step, scaled to all heads."""
+    import oracle
+    from tests import parity_util as U
+    H, P, N = w.extra["nheads"], w.extra["headdim"], w.d_state
+    inp, par = W.make_mamba2_case(w.batch, w.L, H, P, N, w.dtype, w.seed, device=dev)
+    threads = oracle.max_threads()
+    per_step = min(30.0, 150.0 / max(1, args.steps + args.warmup))
+    si, sp, _ = U.head_subset(inp, par, [0])
+    t0 = time.perf_counter()
+    oracle.mamba2_layer_fwd(si, sp)
+    t1 = time.perf_counter() - t0
+    k = int(max(1, min(H, per_step / max(t1, 1e-3))))
+    heads = sorted({int(h) for h in np.linspace(0, H - 1, k)})
+    si, sp, _ = U.head_subset(inp, par, heads)
+    for _ in range(args.warmup):
+        oracle.mamba2_layer_fwd(si, sp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.mamba2_layer_fwd(si, sp)
+    secs = time.perf_counter() - t0
+    layer_s = secs / args.steps * H / len(heads)
+    value = w.batch * w.L / layer_s / 1e6
+    sample = f"{len(heads)} of {H} heads x {w.batch} batch rows x L={w.L} per step, scaled by {H}/{len(heads)}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(layer_s * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
+                   "d_state": w.d_state, "nheads": H, "headdim": P, "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -58,6 +58,16 @@ class FwdState(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("conv_x", ctypes.c_void_p)]
 
 
+class Params2(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
+
+
+class Inputs2(ctypes.Structure):
+    _fields_ = [("xbc", ctypes.c_void_p * 2), ("z", ctypes.c_void_p), ("dt", ctypes.c_void_p * 2),
+                ("dtype", ctypes.c_int)]
+
+
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is not built; run `python -c \"import __graft_entry__ as g; g.build()\"` "
@@ -78,6 +88,11 @@ def _load():
     lib.bimamba_block_step.argtypes = [ctypes.POINTER(FwdState), ctypes.POINTER(Inputs), I, ctypes.POINTER(Params),
                                        P, I, I, I, I, ctypes.POINTER(FwdState), U, P]
     lib.bimamba_block_step.restype = I
+    lib.bimamba2_workspace_bytes.argtypes = [I, I64, I, I, I]
+    lib.bimamba2_workspace_bytes.restype = SZ
+    lib.bimamba2_layer_fwd.argtypes = [ctypes.POINTER(Inputs2), ctypes.POINTER(Params2), P, I,
+                                       I, I64, I, I, I, U, P, SZ, P]
+    lib.bimamba2_layer_fwd.restype = I
     lib.bimamba_status_string.argtypes = [I]
     lib.bimamba_status_string.restype = ctypes.c_char_p
     lib.bimamba_abi_version.restype = I
@@ -235,4 +250,47 @@ def bimamba_block_step(state, x, z, dt, B, C, params: dict, out=None, out_dtype=
                                 flags, _stream(stream))
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba_block_step", rc)
+    return out
+
+
+# ---------------------------------------------------------------- Mamba-2 mixer
+
+M2_HEADDIM = 32
+M2_D_STATE = 128
+
+
+def bimamba2_workspace_bytes(batch: int, L: int, nheads: int, headdim: int = M2_HEADDIM,
+                             d_state: int = M2_D_STATE) -> int:
+    return int(lib.bimamba2_workspace_bytes(batch, L, nheads, headdim, d_state))
+
+
+def bimamba2_layer_fwd(xbc, z, dt, params: dict, out=None, out_dtype=None, flags: int = 0,
+                       workspace=None, stream=None):
+    """Full-sequence bidirectional Mamba-2 mixer.  xbc [2, b, L, H*P + 2N]
+    (or a (fwd, rev) pair); z [b, L, H*P]; dt [2, b, L, H] (or a pair);
+    params as produced by workloads.make_mamba2_params (on the device).
+    Returns out [b, L, H*P]."""
+    x0, x1 = _pair(xbc)
+    d0, d1 = _pair(dt)
+    b, L, H = d0.shape
+    HP = z.shape[-1]
+    P = HP // H
+    N = (x0.shape[-1] - HP) // 2
+    if out is None:
+        out = torch.empty(b, L, HP, device=z.device, dtype=out_dtype or z.dtype)
+    need = bimamba2_workspace_bytes(b, L, H, P, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=z.device, dtype=torch.uint8)
+    inp = Inputs2()
+    inp.xbc[0], inp.xbc[1] = _ptr(x0), _ptr(x1)
+    inp.z = _ptr(z)
+    inp.dt[0], inp.dt[1] = _ptr(d0), _ptr(d1)
+    inp.dtype = _dtype_code(z.dtype)
+    par = Params2(_ptr(params["A"]), _ptr(params["D"]), _ptr(params["dt_bias"]),
+                  _ptr(params["conv_w"]), _ptr(params.get("conv_b")))
+    rc = lib.bimamba2_layer_fwd(ctypes.byref(inp), ctypes.byref(par), _ptr(out), _dtype_code(out.dtype),
+                                b, L, H, P, N, flags, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba2_layer_fwd", rc)
     return out

@@ -12,6 +12,7 @@
 #include "block_fused.cuh"
 #include "layer_fused.cuh"
 #include "layer_tma.cuh"
+#include "mamba2.cuh"
 #include "scan_kernels.cuh"
 
 namespace {
@@ -703,3 +704,108 @@ extern "C" int bimamba_layer_fwd_noalloc(const bimamba_inputs_t* in, const bimam
     return bimamba_layer_fwd(in, p, out, out_dtype, batch, L, d_inner, d_state, flags, scratch,
                              kNoallocScratchBytes, cuda_stream);
 }
+
+// ---- Mamba-2 mixer
+
+namespace {
+
+size_t m2_round(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+struct M2Layout {
+    size_t v, dl, yf, total;
+};
+
+// Workspace: conv features [2][batch][L][CH], step sizes [2][batch][H][L],
+// forward output [batch][L][H*P], all fp32, each part 256-byte aligned.
+M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
+    const size_t CH = (size_t)H * P + 2 * (size_t)N;
+    M2Layout l;
+    l.v = 0;
+    l.dl = m2_round(2 * (size_t)batch * (size_t)L * CH * 4);
+    l.yf = l.dl + m2_round(2 * (size_t)batch * (size_t)H * (size_t)L * 4);
+    l.total = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
+    return l;
+}
+
+bool m2_sizes_ok(int batch, int64_t L, int H) {
+    // grid limits: 2 * batch (z) and nheads (x) at most 65535; L bounded so
+    // that token indices stay far inside int64 and the prep grid's x.
+    return batch >= 1 && 2 * (int64_t)batch <= 65535 && L >= 1 && L <= (int64_t)1 << 31 && H >= 1 && H <= 65535;
+}
+
+template <typename Tin, typename Tout>
+int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
+    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 127) / 128),
+                  (unsigned)(2 * k.batch));
+    bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const dim3 g2((unsigned)k.H, (unsigned)k.batch);
+    bimamba::m2_scan_kernel<0, Tin, Tout><<<g2, 32, 0, st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    bimamba::m2_scan_kernel<1, Tin, Tout><<<g2, 32, 0, st>>>(k);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state) {
+    if (!m2_sizes_ok(batch, L, nheads) || headdim <= 0 || d_state <= 0) return 0;
+    return m2_layout(batch, L, nheads, headdim, d_state).total;
+}
+
+int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, void* out,
+                       bimamba_dtype_t out_dtype, int batch, int64_t L, int nheads, int headdim, int d_state,
+                       unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    if (!in || !p || !out || !m2_sizes_ok(batch, L, nheads)) return BIMAMBA_ERR_INVALID_ARG;
+    if (headdim != bimamba::kM2P || d_state != bimamba::kM2N) return BIMAMBA_ERR_UNSUPPORTED;
+    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_UNSUPPORTED;
+    if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(in->dtype) || !dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    const void* ptrs[5] = {in->xbc[0], in->xbc[1], in->z, in->dt[0], in->dt[1]};
+    const size_t a = elem_size(in->dtype);
+    for (const void* q : ptrs) {
+        if (!q) return BIMAMBA_ERR_INVALID_ARG;
+        if (!aligned(q, a)) return BIMAMBA_ERR_MISALIGNED;
+    }
+    if (!aligned(in->z, 16)) return BIMAMBA_ERR_MISALIGNED;  // z rows are staged in 16-byte copies
+    if (!p->A || !p->D || !p->dt_bias || !p->conv_w) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_w, 4) ||
+        (p->conv_b && !aligned(p->conv_b, 4)) || !aligned(out, elem_size(out_dtype)))
+        return BIMAMBA_ERR_MISALIGNED;
+    const M2Layout lay = m2_layout(batch, L, nheads, headdim, d_state);
+    if (!workspace || workspace_bytes < lay.total) return BIMAMBA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BIMAMBA_ERR_MISALIGNED;
+
+    bimamba::M2Params k = {};
+    for (int r = 0; r < 2; ++r) {
+        k.xbc[r] = in->xbc[r];
+        k.dt[r] = in->dt[r];
+    }
+    k.z = in->z;
+    k.A = p->A;
+    k.Dskip = p->D;
+    k.dt_bias = p->dt_bias;
+    k.conv_w = p->conv_w;
+    k.conv_b = p->conv_b;
+    k.out = out;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    k.V = reinterpret_cast<float*>(ws + lay.v);
+    k.DL = reinterpret_cast<float*>(ws + lay.dl);
+    k.YF = reinterpret_cast<float*>(ws + lay.yf);
+    k.L = L;
+    k.H = nheads;
+    k.CH = nheads * headdim + 2 * d_state;
+    k.batch = batch;
+    k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
+    k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if (in_bf && out_bf) return launch_m2<bf16, bf16>(k, st);
+    if (in_bf) return launch_m2<bf16, float>(k, st);
+    if (out_bf) return launch_m2<float, bf16>(k, st);
+    return launch_m2<float, float>(k, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,258 @@
+// mamba2.cuh -- the bidirectional Mamba-2 mixer at the shape of DiffuMamba's
+// own denoiser ("DiffuMamba: High-Throughput Diffusion LMs with Mamba
+// Backbone", §3.2 Eq. (4)-(6); App. C Table 8: Mamba-2 mixers, state
+// dimension 128, conv dimension 4, no weight tie between directions; App. C
+// Table 12: d_inner 3840, a conv over the 4096 channels of x, B and C, one
+// group of B and C for 120 heads of 32 channels).
+//
+// Per direction r, batch row b and head h (P = 32 channels, N = 128 states):
+//   v = silu(conv_r(xbc_r))   over x | B | C (causal forward, anti-causal reverse)
+//   delta[t] = softplus(dt_r[t][h] + dt_bias_r[h])
+//   S[p][n] <- exp(delta A_h) S[p][n] + delta x[t][p] B[t][n]
+//   y_r[t][p] = sum_n C[t][n] S[p][n] + D_h x[t][p]
+//   out = (y_0 + y_1) * silu(z)
+//
+// Three launches: m2_prep_kernel writes the conv + SiLU features of both
+// directions and the per-head step sizes (fp32, to the workspace) -- B and C
+// are shared by every head, so they are computed once, not once per head;
+// m2_scan_kernel<0, ...> runs the forward scans and stores y_0;
+// m2_scan_kernel<1, ...> runs the reverse scans, adds y_0 and applies the gate.
+//
+// Scan: one warp per (batch row, head).  Lane (pb, nb) = (lane / 8, lane % 8)
+// holds rows 8pb..8pb+7 x the 16 states {32i + 4nb + j : i, j < 4} of the
+// head's 32 x 128 state, 128 registers; interleaving the states in groups of
+// 4 makes every 16-byte B/C load of the 8 lanes of a row block one
+// conflict-free shared-memory wavefront.  The state is kept divided by the running product of the
+// decays, S~ = S / a_cum, so that a token costs one FMA per state for the
+// update (S~ += (delta x / a_cum) B) and one for the readout (C . S~, times
+// a_cum afterwards), instead of a multiply and two FMAs.  Before a_cum drops
+// below 2^-60 the product is folded into S~ (a branch uniform over the warp:
+// delta and A are the head's), so 1 / a_cum stays finite.  Rows of 8 partial
+// C . S~ sums are combined over the 8 lanes of a row block by a transpose-
+// reduce, after which every lane owns one (token, channel) output.  Token
+// rows of x, B, C and delta (and, in reverse, the forward y and z of the
+// head's channels) stream through a 2-stage shared-memory ring by cp.async;
+// tokens past the end read zeros, so delta = 0 there and the step leaves the
+// state exactly unchanged.
+#pragma once
+
+#include "scan_kernels.cuh"
+#include "tma_util.cuh"
+
+namespace bimamba {
+
+constexpr int kM2P = 32;    // channels per head (headdim)
+constexpr int kM2N = 128;   // states per channel (d_state)
+constexpr int kM2T = 8;     // tokens per staged chunk of the scan
+constexpr int kM2PrepT = 8;   // tokens per thread of the prep kernel
+constexpr float kM2Floor = 8.673617379884035e-19f;  // 2^-60
+
+struct M2Params {
+    const void* xbc[2];    // [batch][L][CH] per direction, CH = H*P + 2N
+    const void* z;         // [batch][L][H*P]
+    const void* dt[2];     // [batch][L][H]
+    const float* A;        // [2][H]
+    const float* Dskip;    // [2][H]
+    const float* dt_bias;  // [2][H]
+    const float* conv_w;   // [2][CH][4]
+    const float* conv_b;   // [2][CH] or nullptr
+    void* out;             // [batch][L][H*P]
+    float* V;              // [2][batch][L][CH]   conv + SiLU features
+    float* DL;             // [2][batch][H][L]    step sizes
+    float* YF;             // [batch][L][H*P]     forward y
+    int64_t L;
+    int H, CH, batch;
+    float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
+};
+
+// grid (ceil(L / 8), ceil(CH / 128), 2 * batch), block 128: thread = one
+// channel of one direction over 8 tokens; its 11 input rows (8 + the 3-row
+// conv halo) are loaded first, independently, then the 8 outputs computed.
+template <typename Tin>
+__global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
+    constexpr int TT = kM2PrepT;
+    const int c = blockIdx.y * 128 + threadIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.x * TT;
+    const int r = blockIdx.z / p.batch, b = blockIdx.z % p.batch;
+    const int64_t L = p.L;
+    const int CH = p.CH, H = p.H;
+    if (c < CH) {
+        const Tin* X = static_cast<const Tin*>(p.xbc[r]) + (int64_t)b * L * CH + c;
+        const float* w = p.conv_w + ((int64_t)r * CH + c) * 4;
+        const float w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3];
+        const float cb = p.conv_b ? p.conv_b[r * CH + c] : 0.f;
+        float* V = p.V + ((int64_t)r * p.batch + b) * L * CH + c;
+        // window[k] = x[t0 - 3 + k] (forward) or x[t0 + k] (reverse), zero outside [0, L)
+        float xw[TT + 3];
+        const int64_t base = r == 0 ? t0 - 3 : t0;
+#pragma unroll
+        for (int k = 0; k < TT + 3; ++k) {
+            const int64_t i = base + k;
+            xw[k] = (i >= 0 && i < L) ? ldf(X, i * CH) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < TT; ++k) {
+            const int64_t t = t0 + k;
+            // forward: taps 0..3 on x[t-3..t] = xw[k..k+3]; reverse: tap k on x[t+3-k] = xw[k+3-tap]
+            const float v = r == 0 ? fmaf(w3, xw[k + 3], fmaf(w2, xw[k + 2], fmaf(w1, xw[k + 1], fmaf(w0, xw[k], cb))))
+                                   : fmaf(w3, xw[k], fmaf(w2, xw[k + 1], fmaf(w1, xw[k + 2], fmaf(w0, xw[k + 3], cb))));
+            if (t < L) V[t * CH] = silu(v);
+        }
+    }
+    if (blockIdx.y == 0) {
+        for (int h = threadIdx.x; h < H; h += 128) {
+            const Tin* DT = static_cast<const Tin*>(p.dt[r]) + (int64_t)b * L * H + h;
+            const float bias = p.dt_bias[r * H + h];
+            float* DLh = p.DL + (((int64_t)r * p.batch + b) * H + h) * L;
+#pragma unroll
+            for (int k = 0; k < TT; ++k) {
+                const int64_t t = t0 + k;
+                if (t < L) DLh[t] = softplus(ldf(DT, t * H) + bias);
+            }
+        }
+    }
+}
+
+// grid (H, batch), block 32: one warp scans one head of one batch row in
+// direction DIR.  DIR 0 stores y_0 to p.YF; DIR 1 adds it and gates.
+template <int DIR, typename Tin, typename Tout>
+__global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
+    constexpr int P = kM2P, N = kM2N, T = kM2T;
+    __shared__ __align__(16) float xs[2][T][P];
+    __shared__ __align__(16) float bs[2][T][N];
+    __shared__ __align__(16) float cs[2][T][N];
+    __shared__ __align__(16) float ds[2][T];
+    // reverse only: the forward y and z of this head's channels
+    __shared__ __align__(16) float ys[DIR == 1 ? 2 : 1][DIR == 1 ? T : 1][P];
+    __shared__ __align__(16) Tin zs[DIR == 1 ? 2 : 1][DIR == 1 ? T : 1][P];
+    const int lane = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int pb = lane >> 3, nb = lane & 7;
+    const int64_t L = p.L;
+    const int H = p.H, CH = p.CH, HP = H * P;
+    const float* Vb = p.V + ((int64_t)DIR * p.batch + b) * L * CH;
+    const float* Dh = p.DL + (((int64_t)DIR * p.batch + b) * H + h) * L;
+    const int nc = (int)((L + T - 1) / T);
+
+    // chunk i of the walk (chunk k = tokens [kT, kT+T)) into ring slot buf
+    auto stage = [&](int i, int buf) {
+        const int64_t row0 = (int64_t)(DIR == 0 ? i : nc - 1 - i) * T;
+        for (int e = lane; e < T * (P / 4); e += 32) {
+            const int rr = e / (P / 4), q = e % (P / 4);
+            const bool ok = row0 + rr < L;
+            cp_async<16>(&xs[buf][rr][4 * q], Vb + (ok ? row0 + rr : 0) * CH + h * P + 4 * q, ok);
+        }
+        for (int e = lane; e < T * (N / 4); e += 32) {
+            const int rr = e / (N / 4), q = e % (N / 4);
+            const bool ok = row0 + rr < L;
+            const float* row = Vb + (ok ? row0 + rr : 0) * CH + HP;
+            cp_async<16>(&bs[buf][rr][4 * q], row + 4 * q, ok);
+            cp_async<16>(&cs[buf][rr][4 * q], row + N + 4 * q, ok);
+        }
+        if (lane < T) {
+            const bool ok = row0 + lane < L;
+            cp_async<4>(&ds[buf][lane], Dh + (ok ? row0 + lane : 0), ok);
+        }
+        if constexpr (DIR == 1) {
+            constexpr int ZP = P * (int)sizeof(Tin) / 16;  // 16-byte pieces of a z row
+            for (int e = lane; e < T * (P / 4); e += 32) {
+                const int rr = e / (P / 4), q = e % (P / 4);
+                const bool ok = row0 + rr < L;
+                const int64_t o = ((int64_t)b * L + (ok ? row0 + rr : 0)) * HP + (int64_t)h * P;
+                cp_async<16>(&ys[buf][rr][4 * q], p.YF + o + 4 * q, ok);
+            }
+            for (int e = lane; e < T * ZP; e += 32) {
+                const int rr = e / ZP, q = e % ZP;
+                const bool ok = row0 + rr < L;
+                const int64_t o = ((int64_t)b * L + (ok ? row0 + rr : 0)) * HP + (int64_t)h * P;
+                cp_async<16>(reinterpret_cast<unsigned char*>(&zs[buf][rr][0]) + 16 * q,
+                             reinterpret_cast<const unsigned char*>(static_cast<const Tin*>(p.z) + o) + 16 * q, ok);
+            }
+        }
+        cp_async_commit();
+    };
+
+    const float A2 = p.A[DIR * H + h] * kLog2e;
+    const float Dskip = p.Dskip[DIR * H + h];
+    const float scale = p.dir_scale[DIR];
+    float S[8][16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int n = 0; n < 16; ++n) S[i][n] = 0.f;
+    float acum = 1.f;
+
+    stage(0, 0);
+    if (nc > 1) stage(1, 1);
+#pragma unroll 1
+    for (int i = 0; i < nc; ++i) {
+        const int buf = i & 1;
+        if (i + 1 < nc)
+            cp_async_wait_pending<1>();
+        else
+            cp_async_wait_pending<0>();
+        __syncwarp();
+        const int64_t row0 = (int64_t)(DIR == 0 ? i : nc - 1 - i) * T;
+#pragma unroll 1
+        for (int s = 0; s < T; ++s) {
+            const int rr = DIR == 0 ? s : T - 1 - s;
+            const float dl = ds[buf][rr];
+            const float na = acum * ex2_approx(dl * A2);
+            if (na < kM2Floor) {  // fold the decay product into the state
+#pragma unroll
+                for (int i2 = 0; i2 < 8; ++i2)
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) S[i2][n] *= na;
+                acum = 1.f;
+            } else {
+                acum = na;
+            }
+            const float sc = dl * rcp_approx(acum);
+            float xd[8], bv[16], cv[16];
+            {
+                const float4 x0 = *reinterpret_cast<const float4*>(&xs[buf][rr][8 * pb]);
+                const float4 x1 = *reinterpret_cast<const float4*>(&xs[buf][rr][8 * pb + 4]);
+                xd[0] = x0.x * sc; xd[1] = x0.y * sc; xd[2] = x0.z * sc; xd[3] = x0.w * sc;
+                xd[4] = x1.x * sc; xd[5] = x1.y * sc; xd[6] = x1.z * sc; xd[7] = x1.w * sc;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 b4 = *reinterpret_cast<const float4*>(&bs[buf][rr][32 * q + 4 * nb]);
+                const float4 c4 = *reinterpret_cast<const float4*>(&cs[buf][rr][32 * q + 4 * nb]);
+                bv[4 * q] = b4.x; bv[4 * q + 1] = b4.y; bv[4 * q + 2] = b4.z; bv[4 * q + 3] = b4.w;
+                cv[4 * q] = c4.x; cv[4 * q + 1] = c4.y; cv[4 * q + 2] = c4.z; cv[4 * q + 3] = c4.w;
+            }
+            float acc[8];
+#pragma unroll
+            for (int i2 = 0; i2 < 8; ++i2) {
+                const float2 xx = make_float2(xd[i2], xd[i2]);
+                float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int n = 0; n < 16; n += 2) {
+                    const float2 hh = fma2(xx, make_float2(bv[n], bv[n + 1]), make_float2(S[i2][n], S[i2][n + 1]));
+                    S[i2][n] = hh.x;
+                    S[i2][n + 1] = hh.y;
+                    a2 = fma2(make_float2(cv[n], cv[n + 1]), hh, a2);
+                }
+                acc[i2] = a2.x + a2.y;
+            }
+            const float yr = group_transpose_reduce<8, 1>(acc, nb);  // row 8pb + nb
+            const int64_t t = row0 + rr;
+            if (t < L) {
+                const int prow = 8 * pb + nb;
+                const float y = (acum * yr + Dskip * xs[buf][rr][prow]) * scale;
+                const int64_t o = ((int64_t)b * L + t) * HP + (int64_t)h * P + prow;
+                if constexpr (DIR == 0) {
+                    p.YF[o] = y;
+                } else {
+                    const float zv = ldf(&zs[buf][rr][0], prow);
+                    stf(static_cast<Tout*>(p.out), o, (ys[buf][rr][prow] + y) * silu(zv));
+                }
+            }
+        }
+        __syncwarp();
+        if (i + 2 < nc) stage(i + 2, buf);
+    }
+}
+
+}  // namespace bimamba

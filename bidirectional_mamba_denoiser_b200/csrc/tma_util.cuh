@@ -74,21 +74,29 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// Asynchronous global -> shared copy of BYTES (8 or 16; both addresses
+// Asynchronous global -> shared copy of BYTES (4, 8 or 16; both addresses
 // aligned to BYTES); with pred false nothing is read and zeros are written.
 template <int BYTES>
 __device__ __forceinline__ void cp_async(void* dst, const void* src, bool pred) {
-    static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
+    static_assert(BYTES == 4 || BYTES == 8 || BYTES == 16, "cp.async size");
     const int n = pred ? BYTES : 0;
     if constexpr (BYTES == 16)
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
                      : "memory");
-    else
+    else if constexpr (BYTES == 8)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
+                     : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(n)
                      : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Wait until at most N of this thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_pending() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -184,6 +184,57 @@ int bimamba_block_step(const bimamba_fwd_state_t *prefix_state, const bimamba_in
                        int batch, int d_inner, int d_state,
                        bimamba_fwd_state_t *new_state, unsigned flags, void *cuda_stream);
 
+/* ---------------------------------------------------------------- Mamba-2
+ * The bidirectional Mamba-2 mixer at the shape of the pages' own denoiser
+ * ("DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone", §3.2
+ * Eq. (4)-(6); App. C Table 8: Mamba-2, state dimension 128, conv dimension
+ * 4, no weight tie between directions; App. C Table 12: d_inner 3840 = 120
+ * heads x 32, conv over the x | B | C channels, one group of B and C).  Per
+ * direction r, batch row b, head h (headdim P, d_state N, conv channels
+ * CH = nheads*P + 2N):
+ *   v = silu(conv_r(xbc_r))            causal (r = 0) / anti-causal (r = 1),
+ *                                      zero outside [0, L); x | B | C = v
+ *   delta[t] = softplus(dt_r[t][h] + dt_bias_r[h])
+ *   S[p][n] <- exp(delta A_r[h]) S[p][n] + delta x[t][h*P+p] B[t][n]
+ *   y_r[t][h*P+p] = sum_n C[t][n] S[p][n] + D_r[h] x[t][h*P+p]
+ *   out[t] = (y_0[t] + y_1[t]) * silu(z[t])
+ * The gated RMSNorm and out_proj of a Mamba-2 block are not part of this
+ * call.  This version supports headdim 32 and d_state 128 (the pages'
+ * shape; anything else returns BIMAMBA_ERR_UNSUPPORTED). */
+
+/* Parameters of both directions, fp32 device pointers, index 0 = forward. */
+typedef struct {
+    const float *A;        /* [2][nheads] (negative: the decay is exp(delta*A)) */
+    const float *D;        /* [2][nheads] */
+    const float *dt_bias;  /* [2][nheads] */
+    const float *conv_w;   /* [2][CH][4]: forward tap k multiplies x[t-3+k], reverse tap k x[t+3-k] */
+    const float *conv_b;   /* [2][CH] or NULL (= 0) */
+} bimamba2_params_t;
+
+/* Inputs, device pointers of `dtype`, row-major. */
+typedef struct {
+    const void *xbc[2];    /* [batch][L][CH] per direction (the same pointer twice = shared) */
+    const void *z;         /* [batch][L][nheads*headdim], 16-byte aligned */
+    const void *dt[2];     /* [batch][L][nheads] per direction */
+    bimamba_dtype_t dtype;
+} bimamba2_inputs_t;
+
+/* Bytes of device workspace bimamba2_layer_fwd needs (fp32 conv features of
+ * both directions, step sizes, the forward output); 0 for invalid sizes. */
+size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state);
+
+/* The full-sequence Mamba-2 mixer.  out: [batch][L][nheads*headdim] of
+ * out_dtype, must not alias an input.  flags: BIMAMBA_FWD_ONLY or
+ * BIMAMBA_REV_ONLY (test aids) or 0.  workspace: device memory of at least
+ * bimamba2_workspace_bytes(), 256-byte aligned, caller-owned.  Three kernel
+ * launches on cuda_stream (conv features, forward scan, reverse scan +
+ * combine + gate); nothing is launched when a check fails.  Returns
+ * BIMAMBA_OK or a negative status. */
+int bimamba2_layer_fwd(const bimamba2_inputs_t *in, const bimamba2_params_t *p,
+                       void *out, bimamba_dtype_t out_dtype,
+                       int batch, int64_t L, int nheads, int headdim, int d_state,
+                       unsigned flags, void *workspace, size_t workspace_bytes, void *cuda_stream);
+
 /* Read (and, if reset != 0, clear) the error word of the current device.
  * Kernels never wait without bound: a wait for a tile that gives up after
  * about two seconds sets bit 0 (a tile load that never arrived) and the kernel

@@ -75,3 +75,25 @@ def sample_channels(D: int, k: int, seed: int) -> list[int]:
     while len(picks) < min(k, D):
         picks.add(int(rng.integers(0, D)))
     return sorted(picks)
+
+
+def head_subset(inp: dict, par: dict, heads, P: int = 32, N: int = 128):
+    """The exact Mamba-2 sub-problem on `heads` (heads are independent once B
+    and C, shared by all heads after their own conv, are kept whole).
+    Returns (inputs, params, the output channels of those heads)."""
+    H = inp["dt"].shape[-1]
+    HP = H * P
+    dev = inp["z"].device
+    hidx = torch.as_tensor(list(heads), device=dev, dtype=torch.long)
+    xch = torch.cat([torch.arange(h * P, (h + 1) * P, device=dev) for h in heads])
+    cch = torch.cat([xch, torch.arange(HP, HP + 2 * N, device=dev)])
+    si = {"xbc": inp["xbc"].index_select(-1, cch).cpu(),
+          "z": inp["z"].index_select(-1, xch).cpu(),
+          "dt": inp["dt"].index_select(-1, hidx).cpu()}
+    pd = par["A"].device
+    sp = {"A": par["A"].index_select(1, hidx.to(pd)).cpu(),
+          "D": par["D"].index_select(1, hidx.to(pd)).cpu(),
+          "dt_bias": par["dt_bias"].index_select(1, hidx.to(pd)).cpu(),
+          "conv_w": par["conv_w"].index_select(1, cch.to(pd)).cpu(),
+          "conv_b": par["conv_b"].index_select(1, cch.to(pd)).cpu() if par.get("conv_b") is not None else None}
+    return si, sp, xch.cpu().numpy()

@@ -22,13 +22,14 @@ NULL = object()        # "pass a NULL struct pointer"
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bimamba_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(bimamba2?_[a-z_]+)\s*\(", text)))
 
 
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("bimamba_layer_fwd", "bimamba_prefix_state", "bimamba_block_step",
-              "bimamba_workspace_bytes", "bimamba_status_string", "bimamba_abi_version"):
+              "bimamba_workspace_bytes", "bimamba_status_string", "bimamba_abi_version",
+              "bimamba2_layer_fwd", "bimamba2_workspace_bytes"):
         assert n in names
 
 
@@ -178,3 +179,80 @@ def test_block_rejects():
     assert _block(new=_state(cx=FAKE + 0x41001)) == bm.BIMAMBA_ERR_MISALIGNED
     assert _block(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY) == bm.BIMAMBA_ERR_INVALID_ARG
     assert _block(flags=0x100000) == bm.BIMAMBA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- Mamba-2 mixer
+
+def _inputs2(dtype=bm.BIMAMBA_BF16, base=FAKE):
+    inp = bm.Inputs2()
+    inp.xbc[0], inp.xbc[1] = base, base + 0x10000
+    inp.z = base + 0x20000
+    inp.dt[0], inp.dt[1] = base + 0x30000, base + 0x31000
+    inp.dtype = dtype
+    return inp
+
+
+def _params2(base=FAKE + 0x40000):
+    return bm.Params2(base, base + 0x1000, base + 0x2000, base + 0x3000, base + 0x4000)
+
+
+def _m2(**broken):
+    # Refuse to issue a call in which nothing was broken: with every argument
+    # valid the library would launch kernels on the fake addresses.
+    assert broken, "a validation case must break some argument"
+    return _m2_call(**broken)
+
+
+def _m2_call(inp=None, par=None, out=FAKE + 0x50000, out_dtype=bm.BIMAMBA_BF16, batch=2, L=64, H=4, P=32, N=128,
+             flags=0, ws=FAKE + 0x100000, ws_bytes=None):
+    inp = _inputs2() if inp is None else inp
+    par = _params2() if par is None else par
+    if ws_bytes is None:
+        ws_bytes = bm.bimamba2_workspace_bytes(batch, L, H, P, N)
+    return bm.lib.bimamba2_layer_fwd(_byref(inp), _byref(par), out, out_dtype, batch, L, H, P, N, flags,
+                                     ws, ws_bytes, None)
+
+
+def test_mamba2_workspace_bytes():
+    # conv features 2*b*L*CH + step sizes 2*b*H*L + forward output b*L*H*P, fp32, 256-byte parts
+    b, L, H = 8, 2048, 120
+    CH = H * 32 + 256
+    want = 2 * b * L * CH * 4 + 2 * b * H * L * 4 + b * L * H * 32 * 4
+    assert bm.bimamba2_workspace_bytes(b, L, H) == want
+    assert bm.bimamba2_workspace_bytes(0, 10, 4) == 0
+    assert bm.bimamba2_workspace_bytes(1, 0, 4) == 0
+    assert bm.bimamba2_workspace_bytes(1, 10, 0) == 0
+
+
+def test_mamba2_rejects():
+    assert _m2(inp=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(par=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(out=None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(batch=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(L=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(H=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(P=64) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2(N=64) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2(flags=bm.BIMAMBA_NO_TMA) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2(inp=_inputs2(dtype=7)) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2(out_dtype=7) == bm.BIMAMBA_ERR_UNSUPPORTED
+    bad = _inputs2()
+    bad.z = None
+    assert _m2(inp=bad) == bm.BIMAMBA_ERR_INVALID_ARG
+    bad = _inputs2()
+    bad.dt[1] = FAKE + 0x31001
+    assert _m2(inp=bad) == bm.BIMAMBA_ERR_MISALIGNED
+    bad = _inputs2()
+    bad.z = FAKE + 0x20008  # element-aligned but not 16-byte aligned
+    assert _m2(inp=bad) == bm.BIMAMBA_ERR_MISALIGNED
+    par = _params2()
+    par.conv_w = None
+    assert _m2(par=par) == bm.BIMAMBA_ERR_INVALID_ARG
+    par = _params2()
+    par.A = FAKE + 0x40002
+    assert _m2(par=par) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2(out=FAKE + 0x50001) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2(ws=None) == bm.BIMAMBA_ERR_WORKSPACE
+    assert _m2(ws_bytes=bm.bimamba2_workspace_bytes(2, 64, 4) - 1) == bm.BIMAMBA_ERR_WORKSPACE
+    assert _m2(ws=FAKE + 0x100080) == bm.BIMAMBA_ERR_MISALIGNED

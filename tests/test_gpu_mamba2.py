@@ -1,0 +1,123 @@
+"""The Mamba-2 mixer's CUDA path (through the C ABI) against the fp64 oracle, on a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bidirectional_mamba_denoiser_b200 import workloads as W
+from tests import parity_util as U
+
+pytestmark = pytest.mark.gpu
+
+P, N = 32, 128
+
+
+@pytest.fixture(scope="module")
+def bm():
+    from bidirectional_mamba_denoiser_b200 import bimamba
+    return bimamba
+
+
+def run(bm, inp, par, out_dtype, flags=0):
+    d = U.to_device(inp)
+    p = U.to_device(par)
+    out = bm.bimamba2_layer_fwd(d["xbc"], d["z"], d["dt"], p, out_dtype=out_dtype, flags=flags)
+    torch.cuda.synchronize()
+    return U.to_cpu64(out)
+
+
+@pytest.mark.parametrize("shape", [(1, 37, 2), (2, 100, 3), (1, 8, 1), (1, 1, 2), (2, 257, 4), (1, 9, 2)])
+def test_small_fp32(bm, shape):
+    """fp32 in and out, ragged lengths around the 8-token chunk: normwise <= 1e-5."""
+    b, L, H = shape
+    inp, par = W.make_mamba2_case(b, L, H, P, N, "fp32", seed=50 + L)
+    got = run(bm, inp, par, torch.float32)
+    want = oracle.mamba2_layer_fwd(inp, par)
+    assert U.normwise(got, want) <= U.TOL_FP32
+
+
+def test_bf16_inputs(bm):
+    """bf16 in, fp32 state: fp32-output mode within 2e-3 (and the fp32
+    arithmetic guard); bf16-output mode within one bf16 rounding + 2e-3."""
+    inp, par = W.make_mamba2_case(2, 300, 4, P, N, "bf16", seed=61)
+    want = oracle.mamba2_layer_fwd(inp, par)
+    got32 = run(bm, inp, par, torch.float32)
+    err = U.normwise(got32, want)
+    assert err <= U.TOL_BF16 and err <= U.GUARD, err
+    got16 = run(bm, inp, par, torch.bfloat16)
+    assert U.bf16_out_ok(got16, want)
+
+
+@pytest.mark.parametrize("which", ["fwd", "rev"])
+def test_direction_flags(bm, which):
+    inp, par = W.make_mamba2_case(1, 70, 2, P, N, "fp32", seed=62)
+    f_or = oracle.FWD_ONLY if which == "fwd" else oracle.REV_ONLY
+    f_bm = bm.BIMAMBA_FWD_ONLY if which == "fwd" else bm.BIMAMBA_REV_ONLY
+    got = run(bm, inp, par, torch.float32, flags=f_bm)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par, flags=f_or)) <= U.TOL_FP32
+
+
+def test_shared_xbc_pointer(bm):
+    """The same xBC buffer for both directions (one in_proj)."""
+    inp, par = W.make_mamba2_case(1, 45, 2, P, N, "fp32", seed=63)
+    inp["xbc"][1] = inp["xbc"][0]
+    d, p = U.to_device(inp), U.to_device(par)
+    x = d["xbc"][0].contiguous()
+    out = bm.bimamba2_layer_fwd((x, x), d["z"], d["dt"], p, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(out), oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_FP32
+
+
+@pytest.mark.parametrize("dt_value", [4.0, -9.0])
+def test_extreme_step_sizes(bm, dt_value):
+    """Large steps (decay products fall below 2^-60 within a few tokens, so the
+    kernel folds them into the state again and again) and tiny steps (memory
+    over the whole sequence)."""
+    inp, par = W.make_mamba2_case(1, 150, 3, P, N, "fp32", seed=64)
+    inp["dt"][:] = dt_value
+    got = run(bm, inp, par, torch.float32)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_FP32
+
+
+def test_conv_bias_absent(bm):
+    inp, par = W.make_mamba2_case(1, 33, 2, P, N, "fp32", seed=65)
+    par = dict(par)
+    par["conv_b"] = None
+    d, p = U.to_device(inp), U.to_device(par)
+    out = bm.bimamba2_layer_fwd(d["xbc"], d["z"], d["dt"], p, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(out), oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_FP32
+
+
+def test_repeatable(bm):
+    inp, par = W.make_mamba2_case(2, 64, 3, P, N, "bf16", seed=66)
+    a = run(bm, inp, par, torch.float32)
+    b = run(bm, inp, par, torch.float32)
+    assert np.array_equal(a, b)
+
+
+def test_full_size_sampled_heads(bm):
+    """The pages' layer: b 8, L 2048, 120 heads x 32, N 128, bf16, in the
+    launch configuration the bench times; three heads against the oracle."""
+    w = W.MAMBA2_1P3B
+    H = w.extra["nheads"]
+    inp, par = W.make_mamba2_case(w.batch, w.L, H, P, N, "bf16", w.seed, device="cuda")
+    out32 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.float32)
+    out16 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    heads = [0, 77, H - 1]
+    si, sp, xch = U.head_subset(inp, par, heads)
+    want = oracle.mamba2_layer_fwd(si, sp)
+    idx = torch.as_tensor(xch, device="cuda")
+    got32 = U.to_cpu64(out32.index_select(-1, idx))
+    err = U.normwise(got32, want)
+    assert err <= U.TOL_BF16 and err <= U.GUARD, err
+    assert U.bf16_out_ok(U.to_cpu64(out16.index_select(-1, idx)), want)
+
+
+def test_workspace_too_small_is_rejected(bm):
+    inp, par = W.make_mamba2_case(1, 16, 2, P, N, "bf16", seed=1, device="cuda")
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bm.BimambaError) as e:
+        bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, workspace=ws)
+    assert e.value.status == bm.BIMAMBA_ERR_WORKSPACE
