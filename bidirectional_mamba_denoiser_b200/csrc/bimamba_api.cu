@@ -13,6 +13,7 @@
 #include "layer_fused.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
+#include "mamba2_ssd.cuh"
 #include "scan_kernels.cuh"
 
 namespace {
@@ -712,18 +713,22 @@ namespace {
 size_t m2_round(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct M2Layout {
-    size_t v, dl, yf, total;
+    size_t v, dl, yf, tiles, total;
 };
 
 // Workspace: conv features [2][batch][L][CH], step sizes [2][batch][H][L],
-// forward output [batch][L][H*P], all fp32, each part 256-byte aligned.
+// forward output [batch][L][H*P], all fp32, then the fp16 C/B tiles of the
+// tensor-core path [2][batch][ceil(L/128)][2][128 x 128]; each part 256-byte
+// aligned.
 M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
     const size_t CH = (size_t)H * P + 2 * (size_t)N;
+    const size_t nc = (size_t)((L + bimamba::kSQ - 1) / bimamba::kSQ);
     M2Layout l;
     l.v = 0;
     l.dl = m2_round(2 * (size_t)batch * (size_t)L * CH * 4);
     l.yf = l.dl + m2_round(2 * (size_t)batch * (size_t)H * (size_t)L * 4);
-    l.total = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
+    l.tiles = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
+    l.total = l.tiles + 2 * (size_t)batch * nc * 2 * (size_t)bimamba::kTileBytes;
     return l;
 }
 
@@ -731,6 +736,29 @@ bool m2_sizes_ok(int batch, int64_t L, int H) {
     // grid limits: 2 * batch (z) and nheads (x) at most 65535; L bounded so
     // that token indices stay far inside int64 and the prep grid's x.
     return batch >= 1 && 2 * (int64_t)batch <= 65535 && L >= 1 && L <= (int64_t)1 << 31 && H >= 1 && H <= 65535;
+}
+
+// Chunked dual form on the tensor cores: conv features, C/B tiles, forward
+// and reverse chunk scans (four launches).
+template <typename Tin, typename Tout>
+int launch_m2_ssd(const bimamba::M2Params& k, unsigned char* tiles, cudaStream_t st) {
+    auto k0 = &bimamba::m2_ssd_kernel<0, Tin, Tout>;
+    auto k1 = &bimamba::m2_ssd_kernel<1, Tin, Tout>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
+    if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k1), bimamba::kSsdSmem);
+    if (rc) return rc;
+    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 127) / 128),
+                  (unsigned)(2 * k.batch));
+    bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const unsigned nc = (unsigned)((k.L + bimamba::kSQ - 1) / bimamba::kSQ);
+    bimamba::m2_tiles_kernel<<<dim3(nc, (unsigned)k.batch, 2), 256, 0, st>>>(k, tiles);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const dim3 g2((unsigned)k.H, (unsigned)k.batch);
+    k0<<<g2, 128, bimamba::kSsdSmem, st>>>(k, tiles);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    k1<<<g2, 128, bimamba::kSsdSmem, st>>>(k, tiles);
+    return launch_status();
 }
 
 template <typename Tin, typename Tout>
@@ -760,7 +788,8 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
                        unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (!in || !p || !out || !m2_sizes_ok(batch, L, nheads)) return BIMAMBA_ERR_INVALID_ARG;
     if (headdim != bimamba::kM2P || d_state != bimamba::kM2N) return BIMAMBA_ERR_UNSUPPORTED;
-    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_NO_TMA | BIMAMBA_TEST_STARVE))
+        return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(in->dtype) || !dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
     const void* ptrs[5] = {in->xbc[0], in->xbc[1], in->z, in->dt[0], in->dt[1]};
@@ -800,8 +829,15 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     k.batch = batch;
     k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    k.starve = (flags & BIMAMBA_TEST_STARVE) ? 1 : 0;
+    k.wait_limit = k.starve ? kStarveWaitCycles : kWaitCycles;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
+        unsigned char* tiles = ws + lay.tiles;
+        if (out_bf) return launch_m2_ssd<bf16, bf16>(k, tiles, st);
+        return launch_m2_ssd<bf16, float>(k, tiles, st);
+    }
     if (in_bf && out_bf) return launch_m2<bf16, bf16>(k, st);
     if (in_bf) return launch_m2<bf16, float>(k, st);
     if (out_bf) return launch_m2<float, bf16>(k, st);

@@ -63,6 +63,8 @@ struct M2Params {
     int64_t L;
     int H, CH, batch;
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
+    long long wait_limit;  // SM clocks a wait for a tile or a product may take (tensor-core path)
+    int starve;            // test aid (tensor-core path): issue no tile copies, so every wait gives up
 };
 
 // grid (ceil(L / 8), ceil(CH / 128), 2 * batch), block 128: thread = one

@@ -1,0 +1,359 @@
+// mamba2_ssd.cuh -- the Mamba-2 mixer's scan in its chunked dual form on the
+// sm_100a tensor cores (tcgen05, fp16 operands, fp32 accumulation in TMEM).
+//
+// Per direction, batch row b and head h, the scan over a chunk of Q = 128
+// steps with a_t = delta_t A_h, c_t = sum_{u <= t} a_u (inside the chunk) and
+// the state S_ (P x N) carried in from the previous chunk is
+//   S_t = e^{c_t} S_ + sum_{s <= t} e^{c_t - c_s} delta_s x_s B_s^T
+//   y_t = e^{c_t} (C_t . S_) + sum_{s <= t} (C_t . B_s) e^{c_t - c_s} delta_s x_s + D x_t
+// (the same recurrence as the step-by-step scan, summed in closed form; the
+// state-space-dual view of Mamba-2 the pages cite).  Four matrix products:
+//   G   = C B^T                     (Q x Q, K = N)      -> TMEM cols [0, 128)
+//   Y2  = C S_^T                    (Q x P, K = N)      -> TMEM cols [160, 192)
+//   S^T = e^{c_end} S_^T + B^T W    (N x P, K = Q), W_s = e^{c_end - c_s} delta_s x_s
+//                                                        -> TMEM cols [192, 224)
+//   Y1  = M (delta x), M = G o e^{c_t - c_s} [s <= t]   (Q x P, K = Q)
+//                                                        -> TMEM cols [128, 160)
+//   y_t = Y1 + e^{c_t} Y2 + D x_t
+// One CTA = one (head, batch row) in one direction, 128 threads; thread t
+// owns step t of the chunk (TMEM lane t) for the per-step work and state
+// row n = t for the state epilogue.  The chunk's C and B arrive as fp16
+// tiles (laid out by m2_tiles_kernel in the canonical K-major form, rows in
+// step order so that the reverse direction needs no other code) by bulk
+// copies; the B tile of the next chunk is fetched as soon as the products
+// that read B are done, the C tile once M (which reuses C's buffer) has been
+// consumed, and each thread's x row and step size of the next chunk by
+// cp.async once this chunk's copies are in registers.  Every mbarrier wait
+// is bounded.
+//
+// Precision: fp16 operands (11-bit significands, like tf32) with fp32
+// accumulation; the carried state stays fp32 in TMEM.  Used for bf16 I/O
+// (within the 2e-3 bound); fp32 I/O runs the step-by-step CUDA-core scan.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "mamba2.cuh"
+#include "tcgen05_util.cuh"
+
+namespace bimamba {
+
+constexpr int kSQ = 128;                    // steps per chunk (= MMA M)
+constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
+// shared memory of m2_ssd_kernel
+constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
+              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90720, kSsdX = 90752, kSsdDL = 109184,
+              kSsdSmem = 109696;
+constexpr int kSsdXStride = 36;  // floats per x row in shared memory (144 B: conflict-free 16-byte accesses)
+
+// grid (nchunks, batch, 2), block 256: fp16 tiles of C and B per chunk, rows
+// in step order (reverse direction: step s of chunk k is token L-1-kQ-s),
+// zero rows past either end.  tiles: [2][batch][nchunks][C | B] x 32 KB.
+__global__ void __launch_bounds__(256) m2_tiles_kernel(const M2Params p, unsigned char* tiles) {
+    const int k = blockIdx.x, b = blockIdx.y, r = blockIdx.z;
+    const int64_t L = p.L;
+    const int CH = p.CH, HP = p.H * kM2P;
+    const int nc = (int)((L + kSQ - 1) / kSQ);
+    const float* Vb = p.V + ((int64_t)r * p.batch + b) * L * CH;
+    unsigned char* T = tiles + (((int64_t)r * p.batch + b) * nc + k) * (2 * kTileBytes);
+    for (int e = threadIdx.x; e < 2 * kSQ * (kM2N / 8); e += 256) {
+        const int which = e / (kSQ * (kM2N / 8));  // 0 = C, 1 = B
+        const int rem = e % (kSQ * (kM2N / 8));
+        const int s = rem / (kM2N / 8), g = rem % (kM2N / 8);
+        const int64_t tok = r == 0 ? (int64_t)k * kSQ + s : L - 1 - (int64_t)k * kSQ - s;
+        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+        if (tok >= 0 && tok < L) {
+            const float* src = Vb + tok * CH + HP + (which == 0 ? kM2N : 0) + 8 * g;
+            const float4 v0 = *reinterpret_cast<const float4*>(src);
+            const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+            __half2 h0 = __floats2half2_rn(v0.x, v0.y), h1 = __floats2half2_rn(v0.z, v0.w);
+            __half2 h2 = __floats2half2_rn(v1.x, v1.y), h3 = __floats2half2_rn(v1.z, v1.w);
+            packed = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+        }
+        *reinterpret_cast<uint4*>(T + which * kTileBytes + f16_kmajor(s, 8 * g, kM2N)) = packed;
+    }
+}
+
+// 8 fp32 values -> 8 fp16 in one 16-byte store.
+__device__ __forceinline__ void st_half8(unsigned char* dst, const float* v) {
+    __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+    __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
+    *reinterpret_cast<uint4*>(dst) =
+        make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                   *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+}
+
+// 32 outputs of one row: 16-byte stores.
+__device__ __forceinline__ void store_row32(float* dst, const float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * u], v[8 * q + 2 * u + 1]);
+            w[u] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// grid (H, batch), block 128, dynamic shared memory kSsdSmem.  DIR 0 stores
+// y_0 to p.YF; DIR 1 adds it and applies the gate.
+template <int DIR, typename Tin, typename Tout>
+__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const unsigned char* tiles) {
+    constexpr int Q = kSQ, P = kM2P;
+    extern __shared__ __align__(128) unsigned char sm[];
+    unsigned char* sC = sm + kSsdC;
+    unsigned char* sB = sm + kSsdB;
+    unsigned char* sDX = sm + kSsdDX;
+    unsigned char* sW = sm + kSsdW;
+    unsigned char* sS = sm + kSsdS;
+    float* c2s = reinterpret_cast<float*>(sm + kSsdC2);
+    float* wtot = reinterpret_cast<float*>(sm + kSsdTot);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSsdBar);  // B tile, C tile, products 1-3, product 4
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
+    float* sX = reinterpret_cast<float*>(sm + kSsdX);   // [128][kSsdXStride]: row t = x of step t
+    float* sDL = reinterpret_cast<float*>(sm + kSsdDL);  // [128]: step size of step t
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t L = p.L;
+    const int H = p.H, CH = p.CH, HP = H * P;
+    const int nc = (int)((L + Q - 1) / Q);
+    const unsigned char* tileb = tiles + ((int64_t)DIR * p.batch + b) * nc * (2 * kTileBytes);
+    const float* Vx = p.V + ((int64_t)DIR * p.batch + b) * L * CH + (int64_t)h * P;
+    const float* Dh = p.DL + (((int64_t)DIR * p.batch + b) * H + h) * L;
+    const float A2 = p.A[DIR * H + h] * kLog2e;
+    const float Dsk = p.Dskip[DIR * H + h];
+    const float scale = p.dir_scale[DIR];
+
+    if (t == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc<256>(tmem_slot);
+    for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sS)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    {
+        float zero[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) zero[i] = 0.f;
+        tmem_st32(tmem + 192 + lb, zero);  // state row n = t starts at 0
+    }
+    if (t == 0 && !p.starve) {
+        mbar_arrive_expect_tx(bars + 0, kTileBytes);
+        bulk_g2s(sB, tileb + kTileBytes, kTileBytes, bars + 0);
+        mbar_arrive_expect_tx(bars + 1, kTileBytes);
+        bulk_g2s(sC, tileb, kTileBytes, bars + 1);
+    }
+    // this thread's x row and step size of chunk kk, into sX / sDL (zeros past either end)
+    auto fetch_step = [&](int kk) {
+        const int64_t tk = DIR == 0 ? (int64_t)kk * Q + t : L - 1 - (int64_t)kk * Q - t;
+        const bool ok = tk >= 0 && tk < L;
+        const float* src = Vx + (ok ? tk : 0) * CH;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp_async<16>(sX + t * kSsdXStride + 4 * i, src + 4 * i, ok);
+        cp_async<4>(sDL + t, Dh + (ok ? tk : 0), ok);
+        cp_async_commit();
+    };
+    fetch_step(0);
+    const uint32_t aC = smem_addr(sC), aB = smem_addr(sB), aDX = smem_addr(sDX), aW = smem_addr(sW),
+                   aS = smem_addr(sS);
+    constexpr uint32_t ID_G = umma_idesc_f16(128, 128, false, false);
+    constexpr uint32_t ID_Y = umma_idesc_f16(128, 32, false, true);
+    constexpr uint32_t ID_S = umma_idesc_f16(128, 32, true, true);
+
+#pragma unroll 1
+    for (int k = 0; k < nc; ++k) {
+        const uint32_t ph = (uint32_t)(k & 1);
+        // ---- step t of chunk k: x, delta (and the reverse epilogue's y_0, z)
+        const int64_t tok = DIR == 0 ? (int64_t)k * Q + t : L - 1 - (int64_t)k * Q - t;
+        const bool valid = tok >= 0 && tok < L;
+        float x[32], yf[DIR == 1 ? 32 : 1];
+        uint4 zq[DIR == 1 ? 4 : 1];  // the reverse epilogue's z: 32 bf16
+        if constexpr (DIR == 1) {
+            if (valid) {  // loaded now, used at the end of the chunk
+                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
+                const float4* ysrc = reinterpret_cast<const float4*>(p.YF + o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v = ysrc[i];
+                    yf[4 * i] = v.x; yf[4 * i + 1] = v.y; yf[4 * i + 2] = v.z; yf[4 * i + 3] = v.w;
+                }
+                const uint4* zsrc = reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.z) + o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) zq[i] = zsrc[i];
+            }
+        }
+        cp_async_wait_all();  // own x row and step size (written and read by this thread only)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(sX + t * kSsdXStride + 4 * i);
+            x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+        }
+        const float dl = sDL[t];
+        // ---- c_t: inclusive scan of delta A (log2 units) over the chunk
+        float a = dl * A2;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, a, off);
+            if (lane >= off) a += v;
+        }
+        if (lane == 31) wtot[warp] = a;
+        __syncthreads();
+        float base = 0.f;
+        for (int w = 0; w < warp; ++w) base += wtot[w];
+        const float c = a + base;
+        const float cend = wtot[0] + wtot[1] + wtot[2] + wtot[3];
+        c2s[t] = c;
+        // ---- delta x and W rows of step t (MN-major [s][p])
+        {
+            const float wdec = ex2_approx(cend - c);
+            float dx[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dx[i] = dl * x[i];
+#pragma unroll
+            for (int pg = 0; pg < 4; ++pg) st_half8(sDX + f16_mnmajor(8 * pg, t, P), dx + 8 * pg);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dx[i] *= wdec;
+#pragma unroll
+            for (int pg = 0; pg < 4; ++pg) st_half8(sW + f16_mnmajor(8 * pg, t, P), dx + 8 * pg);
+        }
+        if (k + 1 < nc) fetch_step(k + 1);  // x is in registers now
+        // ---- carried state row n = t decays over the whole chunk
+        {
+            float s[32];
+            tmem_ld32(tmem + 192 + lb, s);
+            const float f = ex2_approx(cend);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[i] *= f;
+            tmem_st32(tmem + 192 + lb, s);
+        }
+        fence_async_smem();
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        // ---- G = C B^T, Y2 = C S_^T, S^T += B^T W
+        if (t == 0) {
+            mbar_wait_bounded(bars + 0, ph, p.wait_limit);
+            mbar_wait_bounded(bars + 1, ph, p.wait_limit);
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 0, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aB + ks * 256, 128, 2048), ID_G,
+                         ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 160, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aS + ks * 1024, 512, 128), ID_Y,
+                         ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 192, umma_desc(aB + ks * 4096, 2048, 128), umma_desc(aW + ks * 1024, 512, 128),
+                         ID_S, true);
+            umma_commit(bars + 2);
+        }
+        mbar_wait_bounded(bars + 2, ph, p.wait_limit);
+        tmem_fence_after_sync();
+        if (t == 0 && k + 1 < nc && !p.starve) {  // B's buffer is free: next chunk's B tile
+            mbar_arrive_expect_tx(bars + 0, kTileBytes);
+            bulk_g2s(sB, tileb + (int64_t)(k + 1) * 2 * kTileBytes + kTileBytes, kTileBytes, bars + 0);
+        }
+        // ---- M row t (into C's buffer, K-major [t][s]) and the new state row n = t
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+            float g[32];
+            if (j <= warp) {  // columns s >= 32j reach step t = 32 warp + lane only for j <= warp
+                tmem_ld32(tmem + 32 * j + lb, g);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int s = 32 * j + i;
+                    g[i] = s <= t ? g[i] * ex2_approx(c - c2s[s]) : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) g[i] = 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) st_half8(sC + f16_kmajor(t, 32 * j + 8 * q, Q), g + 8 * q);
+        }
+        {
+            float s[32];
+            tmem_ld32(tmem + 192 + lb, s);
+#pragma unroll
+            for (int pg = 0; pg < 4; ++pg) st_half8(sS + f16_mnmajor(8 * pg, t, P), s + 8 * pg);
+        }
+        fence_async_smem();
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        // ---- Y1 = M (delta x)
+        if (t == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 128, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aDX + ks * 1024, 512, 128), ID_Y,
+                         ks > 0);
+            umma_commit(bars + 3);
+        }
+        mbar_wait_bounded(bars + 3, ph, p.wait_limit);
+        tmem_fence_after_sync();
+        if (t == 0 && k + 1 < nc && !p.starve) {  // C's buffer is free: next chunk's C tile
+            mbar_arrive_expect_tx(bars + 1, kTileBytes);
+            bulk_g2s(sC, tileb + (int64_t)(k + 1) * 2 * kTileBytes, kTileBytes, bars + 1);
+        }
+        // ---- output of step t
+        {
+            float y1[32], y2[32];
+            tmem_ld32(tmem + 128 + lb, y1);
+            tmem_ld32(tmem + 160 + lb, y2);
+            if (valid) {
+                const float e = ex2_approx(c);
+                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
+                if constexpr (DIR == 0) {
+                    float4* dst = reinterpret_cast<float4*>(p.YF + o);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float4 v;
+                        v.x = (y1[4 * i] + e * y2[4 * i] + Dsk * x[4 * i]) * scale;
+                        v.y = (y1[4 * i + 1] + e * y2[4 * i + 1] + Dsk * x[4 * i + 1]) * scale;
+                        v.z = (y1[4 * i + 2] + e * y2[4 * i + 2] + Dsk * x[4 * i + 2]) * scale;
+                        v.w = (y1[4 * i + 3] + e * y2[4 * i + 3] + Dsk * x[4 * i + 3]) * scale;
+                        dst[i] = v;
+                    }
+                } else {
+                    float ov[32];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t w4[4] = {zq[q].x, zq[q].y, zq[q].z, zq[q].w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            // bf16 -> fp32 is exact: the bf16 bits are the high half
+                            const float z0 = __uint_as_float(w4[u] << 16), z1 = __uint_as_float(w4[u] & 0xffff0000u);
+                            const int i = 8 * q + 2 * u;
+                            ov[i] = (yf[i] + (y1[i] + e * y2[i] + Dsk * x[i]) * scale) * silu(z0);
+                            ov[i + 1] = (yf[i + 1] + (y1[i + 1] + e * y2[i + 1] + Dsk * x[i + 1]) * scale) * silu(z1);
+                        }
+                    }
+                    store_row32(static_cast<Tout*>(p.out) + o, ov);
+                }
+            }
+        }
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+    }
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc<256>(tmem);
+}
+
+}  // namespace bimamba

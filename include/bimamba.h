@@ -224,11 +224,17 @@ typedef struct {
 size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state);
 
 /* The full-sequence Mamba-2 mixer.  out: [batch][L][nheads*headdim] of
- * out_dtype, must not alias an input.  flags: BIMAMBA_FWD_ONLY or
- * BIMAMBA_REV_ONLY (test aids) or 0.  workspace: device memory of at least
- * bimamba2_workspace_bytes(), 256-byte aligned, caller-owned.  Three kernel
- * launches on cuda_stream (conv features, forward scan, reverse scan +
- * combine + gate); nothing is launched when a check fails.  Returns
+ * out_dtype, must not alias an input.  workspace: device memory of at least
+ * bimamba2_workspace_bytes(), 256-byte aligned, caller-owned.
+ * bf16 inputs run the scan in its chunked dual form on the tensor cores
+ * (chunks of 128 steps; fp16 operands, fp32 accumulation and state; within
+ * 2e-3 of the exact result normwise): four launches (conv features, C/B
+ * tiles, forward, reverse + combine + gate).  fp32 inputs, or flags with
+ * BIMAMBA_NO_TMA, run the step-by-step scan on the CUDA cores in fp32: three
+ * launches.  Other flags: BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY (test aids);
+ * BIMAMBA_TEST_STARVE (tensor-core path: no tile copies are issued, every
+ * wait gives up after ~0.1 ms and sets bit 0 of bimamba_device_error(); the
+ * output is undefined).  Nothing is launched when a check fails.  Returns
  * BIMAMBA_OK or a negative status. */
 int bimamba2_layer_fwd(const bimamba2_inputs_t *in, const bimamba2_params_t *p,
                        void *out, bimamba_dtype_t out_dtype,

@@ -214,10 +214,11 @@ def _m2_call(inp=None, par=None, out=FAKE + 0x50000, out_dtype=bm.BIMAMBA_BF16, 
 
 
 def test_mamba2_workspace_bytes():
-    # conv features 2*b*L*CH + step sizes 2*b*H*L + forward output b*L*H*P, fp32, 256-byte parts
+    # conv features 2*b*L*CH + step sizes 2*b*H*L + forward output b*L*H*P, fp32,
+    # then fp16 C and B tiles of 128 x 128 per chunk of 128 steps and direction
     b, L, H = 8, 2048, 120
     CH = H * 32 + 256
-    want = 2 * b * L * CH * 4 + 2 * b * H * L * 4 + b * L * H * 32 * 4
+    want = 2 * b * L * CH * 4 + 2 * b * H * L * 4 + b * L * H * 32 * 4 + 2 * b * (L // 128) * 2 * 128 * 128 * 2
     assert bm.bimamba2_workspace_bytes(b, L, H) == want
     assert bm.bimamba2_workspace_bytes(0, 10, 4) == 0
     assert bm.bimamba2_workspace_bytes(1, 0, 4) == 0
@@ -233,7 +234,8 @@ def test_mamba2_rejects():
     assert _m2(H=0) == bm.BIMAMBA_ERR_INVALID_ARG
     assert _m2(P=64) == bm.BIMAMBA_ERR_UNSUPPORTED
     assert _m2(N=64) == bm.BIMAMBA_ERR_UNSUPPORTED
-    assert _m2(flags=bm.BIMAMBA_NO_TMA) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2(flags=0x4) == bm.BIMAMBA_ERR_UNSUPPORTED  # no such flag
+    assert _m2(flags=1 << 8) == bm.BIMAMBA_ERR_UNSUPPORTED  # lane field: not a Mamba-2 option
     assert _m2(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY) == bm.BIMAMBA_ERR_INVALID_ARG
     assert _m2(inp=_inputs2(dtype=7)) == bm.BIMAMBA_ERR_UNSUPPORTED
     assert _m2(out_dtype=7) == bm.BIMAMBA_ERR_UNSUPPORTED

@@ -36,16 +36,62 @@ def test_small_fp32(bm, shape):
     assert U.normwise(got, want) <= U.TOL_FP32
 
 
-def test_bf16_inputs(bm):
-    """bf16 in, fp32 state: fp32-output mode within 2e-3 (and the fp32
-    arithmetic guard); bf16-output mode within one bf16 rounding + 2e-3."""
+# bf16 inputs run the chunked dual form on the tensor cores (fp16 operands,
+# bound 2e-3); BIMAMBA_NO_TMA selects the step-by-step CUDA-core scan, which
+# also meets the fp32-arithmetic guard.
+PATHS = {"tensor": (0, U.TOL_BF16), "cuda_core": (0x4000, U.GUARD)}
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_bf16_inputs(bm, path):
+    """bf16 in, fp32 state: fp32-output mode within the path's bound;
+    bf16-output mode within one bf16 rounding + 2e-3."""
+    flags, tol = PATHS[path]
     inp, par = W.make_mamba2_case(2, 300, 4, P, N, "bf16", seed=61)
     want = oracle.mamba2_layer_fwd(inp, par)
-    got32 = run(bm, inp, par, torch.float32)
+    got32 = run(bm, inp, par, torch.float32, flags=flags)
     err = U.normwise(got32, want)
-    assert err <= U.TOL_BF16 and err <= U.GUARD, err
-    got16 = run(bm, inp, par, torch.bfloat16)
+    assert err <= tol, err
+    got16 = run(bm, inp, par, torch.bfloat16, flags=flags)
     assert U.bf16_out_ok(got16, want)
+
+
+@pytest.mark.parametrize("L", [1, 2, 127, 128, 129, 256, 383])
+def test_tensor_path_ragged_lengths(bm, L):
+    """Chunks of 128 steps: lengths around the chunk edge, both directions."""
+    inp, par = W.make_mamba2_case(2, L, 3, P, N, "bf16", seed=70 + L)
+    got = run(bm, inp, par, torch.float32)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
+
+
+@pytest.mark.parametrize("which", ["fwd", "rev"])
+def test_tensor_path_direction_flags(bm, which):
+    inp, par = W.make_mamba2_case(1, 200, 2, P, N, "bf16", seed=71)
+    f_or = oracle.FWD_ONLY if which == "fwd" else oracle.REV_ONLY
+    f_bm = bm.BIMAMBA_FWD_ONLY if which == "fwd" else bm.BIMAMBA_REV_ONLY
+    got = run(bm, inp, par, torch.float32, flags=f_bm)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par, flags=f_or)) <= U.TOL_BF16
+
+
+@pytest.mark.parametrize("dt_value", [4.0, -9.0])
+def test_tensor_path_extreme_step_sizes(bm, dt_value):
+    inp, par = W.make_mamba2_case(1, 300, 2, P, N, "bf16", seed=72)
+    inp["dt"][:] = dt_value
+    got = run(bm, inp, par, torch.float32)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
+
+
+def test_tensor_path_starved_waits_give_up(bm):
+    """With BIMAMBA_TEST_STARVE no tile copy is issued: every wait for a tile
+    gives up after ~0.1 ms, bit 0 of the device error word is set, the
+    kernel finishes, and the context still works afterwards."""
+    inp, par = W.make_mamba2_case(1, 130, 2, P, N, "bf16", seed=73)
+    assert bm.bimamba_device_error(reset=True) >= 0
+    run(bm, inp, par, torch.float32, flags=bm.BIMAMBA_TEST_STARVE)
+    assert bm.bimamba_device_error(reset=True) & 1
+    got = run(bm, inp, par, torch.float32)
+    assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
+    assert bm.bimamba_device_error(reset=True) == 0
 
 
 @pytest.mark.parametrize("which", ["fwd", "rev"])
@@ -102,17 +148,17 @@ def test_full_size_sampled_heads(bm):
     w = W.MAMBA2_1P3B
     H = w.extra["nheads"]
     inp, par = W.make_mamba2_case(w.batch, w.L, H, P, N, "bf16", w.seed, device="cuda")
-    out32 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.float32)
-    out16 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.bfloat16)
-    torch.cuda.synchronize()
     heads = [0, 77, H - 1]
     si, sp, xch = U.head_subset(inp, par, heads)
     want = oracle.mamba2_layer_fwd(si, sp)
     idx = torch.as_tensor(xch, device="cuda")
-    got32 = U.to_cpu64(out32.index_select(-1, idx))
-    err = U.normwise(got32, want)
-    assert err <= U.TOL_BF16 and err <= U.GUARD, err
-    assert U.bf16_out_ok(U.to_cpu64(out16.index_select(-1, idx)), want)
+    for flags, tol in PATHS.values():
+        out32 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.float32, flags=flags)
+        out16 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.bfloat16, flags=flags)
+        torch.cuda.synchronize()
+        err = U.normwise(U.to_cpu64(out32.index_select(-1, idx)), want)
+        assert err <= tol, (flags, err)
+        assert U.bf16_out_ok(U.to_cpu64(out16.index_select(-1, idx)), want)
 
 
 def test_workspace_too_small_is_rejected(bm):
