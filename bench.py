@@ -438,6 +438,29 @@ def roofline_fma(flops: float, call_ms: float, clocks, workload: str, kernel: st
             "peak_source": f"148 SMs x {FP32_FMA_PER_SM_CLK} FP32 lanes x 2 x {mhz:.0f} MHz", "kernel": kernel}
 
 
+def roofline_tensor(flops: float, call_ms: float, workload: str, kernel: str):
+    """Tensor-core roof of the chunked dual form: executed MMA flops per call
+    against the measured dense bf16 rate (fp16 operands run at the same rate)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured bf16 dense (burst), fp16 at the same rate"
+    except Exception:
+        peak, src = 1590.0, "fallback bf16 dense (burst), fp16 at the same rate"
+    achieved = flops / (call_ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get((workload, kernel)), "peak_source": src,
+            "kernel": kernel}
+
+
+def mamba2_ssd_flops(batch: int, L: int, H: int, P: int, N: int, Q: int = 128) -> float:
+    """MMA flops of one dual-form call: per chunk of Q steps, head and
+    direction G = C B^T (Q x Q x N), C S^T (Q x P x N), B^T W (N x P x Q) and
+    M (delta x) (Q x P x Q), at 2 flops per multiply-add."""
+    nc = (L + Q - 1) // Q
+    per_chunk = 2.0 * (Q * Q * N + Q * P * N + N * P * Q + Q * P * Q)
+    return per_chunk * nc * H * batch * 2
+
+
 def mamba2_oracle_rate(w: W.Workload, inputs, params, budget_s: float):
     """The fp64 oracle on a sample of heads, scaled to all heads:
     (Mtokens/s, heads, seconds, threads)."""
@@ -475,16 +498,22 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     ms_max = max_over_ranks(ms, world)
     call_ms = ms / args.steps
     tokens = w.batch * w.L
-    flops = 4.0 * P * N * H * 2 * tokens  # two FMAs per state per token and direction
+    flops = 4.0 * P * N * H * 2 * tokens  # the recurrence: two FMAs per state per token and direction
+    tensor_path = w.dtype == "bf16"
     res = {
         "value": whole_job_rate(tokens * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
-        "gpu_launches": 3 * args.steps,
-        "roofline": roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel"),
+        "gpu_launches": (4 if tensor_path else 3) * args.steps,
         "hbm": hbm_fraction(mamba2_bytes(w.batch, w.L, H, P, N), call_ms),
         "clocks": clocks,
-        "flops_per_token": int(flops / tokens),
+        "recurrence_flops_per_token": int(flops / tokens),
     }
+    if tensor_path:
+        res["roofline"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
+                                          "m2_prep + m2_tiles + 2 x m2_ssd_kernel")
+        res["fp32_equivalent"] = roofline_fma(flops, call_ms, clocks, w.name, "recurrence-equivalent")
+    else:
+        res["roofline"] = roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel")
     if not args.no_e2e:
         inp, par = sets[0]
         host = {k: v.to("cpu").pin_memory() for k, v in inp.items()}

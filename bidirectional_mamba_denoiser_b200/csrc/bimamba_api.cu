@@ -747,7 +747,7 @@ int launch_m2_ssd(const bimamba::M2Params& k, unsigned char* tiles, cudaStream_t
     int rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
     if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k1), bimamba::kSsdSmem);
     if (rc) return rc;
-    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 127) / 128),
+    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
                   (unsigned)(2 * k.batch));
     bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
@@ -763,7 +763,7 @@ int launch_m2_ssd(const bimamba::M2Params& k, unsigned char* tiles, cudaStream_t
 
 template <typename Tin, typename Tout>
 int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
-    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 127) / 128),
+    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
                   (unsigned)(2 * k.batch));
     bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
@@ -798,10 +798,11 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
         if (!q) return BIMAMBA_ERR_INVALID_ARG;
         if (!aligned(q, a)) return BIMAMBA_ERR_MISALIGNED;
     }
-    if (!aligned(in->z, 16)) return BIMAMBA_ERR_MISALIGNED;  // z rows are staged in 16-byte copies
+    // xBC rows, conv taps and z rows move in 16-byte pieces
+    if (!aligned(in->z, 16) || !aligned(in->xbc[0], 16) || !aligned(in->xbc[1], 16)) return BIMAMBA_ERR_MISALIGNED;
     if (!p->A || !p->D || !p->dt_bias || !p->conv_w) return BIMAMBA_ERR_INVALID_ARG;
-    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_w, 4) ||
-        (p->conv_b && !aligned(p->conv_b, 4)) || !aligned(out, elem_size(out_dtype)))
+    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_w, 16) ||
+        (p->conv_b && !aligned(p->conv_b, 4)) || !aligned(out, 16))
         return BIMAMBA_ERR_MISALIGNED;
     const M2Layout lay = m2_layout(batch, L, nheads, headdim, d_state);
     if (!workspace || workspace_bytes < lay.total) return BIMAMBA_ERR_WORKSPACE;

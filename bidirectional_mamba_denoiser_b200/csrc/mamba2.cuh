@@ -67,38 +67,78 @@ struct M2Params {
     int starve;            // test aid (tensor-core path): issue no tile copies, so every wait gives up
 };
 
-// grid (ceil(L / 8), ceil(CH / 128), 2 * batch), block 128: thread = one
-// channel of one direction over 8 tokens; its 11 input rows (8 + the 3-row
-// conv halo) are loaded first, independently, then the 8 outputs computed.
+// 8 consecutive channels of one row as fp32 (one 16-byte load for bf16).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
+        v[2 * u] = __uint_as_float(w[u] << 16);
+        v[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// grid (ceil(L / 8), ceil(CH / 1024), 2 * batch), block 128: thread = 8
+// consecutive channels of one direction over 8 tokens; its 11 input rows
+// (8 + the 3-row conv halo) are loaded first, 16 bytes at a time, then the
+// 64 outputs computed and stored as 16-byte rows.  Needs CH % 8 == 0 and
+// 16-byte aligned rows (CH * sizeof(Tin) % 16 == 0, aligned xbc).
 template <typename Tin>
 __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     constexpr int TT = kM2PrepT;
-    const int c = blockIdx.y * 128 + threadIdx.x;
+    const int c0 = (blockIdx.y * 128 + threadIdx.x) * 8;
     const int64_t t0 = (int64_t)blockIdx.x * TT;
     const int r = blockIdx.z / p.batch, b = blockIdx.z % p.batch;
     const int64_t L = p.L;
     const int CH = p.CH, H = p.H;
-    if (c < CH) {
-        const Tin* X = static_cast<const Tin*>(p.xbc[r]) + (int64_t)b * L * CH + c;
-        const float* w = p.conv_w + ((int64_t)r * CH + c) * 4;
-        const float w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3];
-        const float cb = p.conv_b ? p.conv_b[r * CH + c] : 0.f;
-        float* V = p.V + ((int64_t)r * p.batch + b) * L * CH + c;
-        // window[k] = x[t0 - 3 + k] (forward) or x[t0 + k] (reverse), zero outside [0, L)
-        float xw[TT + 3];
+    if (c0 < CH) {
+        const Tin* X = static_cast<const Tin*>(p.xbc[r]) + (int64_t)b * L * CH + c0;
+        float w[8][4], cb[8];
+        {
+            const float4* wp = reinterpret_cast<const float4*>(p.conv_w + ((int64_t)r * CH + c0) * 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 v = wp[q];
+                w[q][0] = v.x; w[q][1] = v.y; w[q][2] = v.z; w[q][3] = v.w;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) cb[q] = p.conv_b ? p.conv_b[r * CH + c0 + q] : 0.f;
+        }
+        float* V = p.V + ((int64_t)r * p.batch + b) * L * CH + c0;
+        // xw[k] = row t0 - 3 + k (forward) or t0 + k (reverse), zero outside [0, L)
+        float xw[TT + 3][8];
         const int64_t base = r == 0 ? t0 - 3 : t0;
 #pragma unroll
         for (int k = 0; k < TT + 3; ++k) {
             const int64_t i = base + k;
-            xw[k] = (i >= 0 && i < L) ? ldf(X, i * CH) : 0.f;
+            if (i >= 0 && i < L) {
+                load8(X + i * CH, xw[k]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xw[k][q] = 0.f;
+            }
         }
 #pragma unroll
         for (int k = 0; k < TT; ++k) {
             const int64_t t = t0 + k;
-            // forward: taps 0..3 on x[t-3..t] = xw[k..k+3]; reverse: tap k on x[t+3-k] = xw[k+3-tap]
-            const float v = r == 0 ? fmaf(w3, xw[k + 3], fmaf(w2, xw[k + 2], fmaf(w1, xw[k + 1], fmaf(w0, xw[k], cb))))
-                                   : fmaf(w3, xw[k], fmaf(w2, xw[k + 1], fmaf(w1, xw[k + 2], fmaf(w0, xw[k + 3], cb))));
-            if (t < L) V[t * CH] = silu(v);
+            if (t >= L) break;
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                // forward: tap j on x[t-3+j] = xw[k+j]; reverse: tap j on x[t+3-j] = xw[k+3-j]
+                const float a = r == 0 ? fmaf(w[q][3], xw[k + 3][q], fmaf(w[q][2], xw[k + 2][q],
+                                             fmaf(w[q][1], xw[k + 1][q], fmaf(w[q][0], xw[k][q], cb[q]))))
+                                       : fmaf(w[q][3], xw[k][q], fmaf(w[q][2], xw[k + 1][q],
+                                             fmaf(w[q][1], xw[k + 2][q], fmaf(w[q][0], xw[k + 3][q], cb[q]))));
+                v[q] = silu(a);
+            }
+            float4* dst = reinterpret_cast<float4*>(V + t * CH);
+            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
     }
     if (blockIdx.y == 0) {

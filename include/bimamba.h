@@ -207,13 +207,13 @@ typedef struct {
     const float *A;        /* [2][nheads] (negative: the decay is exp(delta*A)) */
     const float *D;        /* [2][nheads] */
     const float *dt_bias;  /* [2][nheads] */
-    const float *conv_w;   /* [2][CH][4]: forward tap k multiplies x[t-3+k], reverse tap k x[t+3-k] */
+    const float *conv_w;   /* [2][CH][4], 16-byte aligned: forward tap k multiplies x[t-3+k], reverse tap k x[t+3-k] */
     const float *conv_b;   /* [2][CH] or NULL (= 0) */
 } bimamba2_params_t;
 
 /* Inputs, device pointers of `dtype`, row-major. */
 typedef struct {
-    const void *xbc[2];    /* [batch][L][CH] per direction (the same pointer twice = shared) */
+    const void *xbc[2];    /* [batch][L][CH] per direction (the same pointer twice = shared), 16-byte aligned */
     const void *z;         /* [batch][L][nheads*headdim], 16-byte aligned */
     const void *dt[2];     /* [batch][L][nheads] per direction */
     bimamba_dtype_t dtype;
@@ -224,7 +224,7 @@ typedef struct {
 size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state);
 
 /* The full-sequence Mamba-2 mixer.  out: [batch][L][nheads*headdim] of
- * out_dtype, must not alias an input.  workspace: device memory of at least
+ * out_dtype, 16-byte aligned, must not alias an input.  workspace: device memory of at least
  * bimamba2_workspace_bytes(), 256-byte aligned, caller-owned.
  * bf16 inputs run the scan in its chunked dual form on the tensor cores
  * (chunks of 128 steps; fp16 operands, fp32 accumulation and state; within

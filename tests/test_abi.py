@@ -248,13 +248,19 @@ def test_mamba2_rejects():
     bad = _inputs2()
     bad.z = FAKE + 0x20008  # element-aligned but not 16-byte aligned
     assert _m2(inp=bad) == bm.BIMAMBA_ERR_MISALIGNED
+    bad = _inputs2()
+    bad.xbc[1] = FAKE + 0x10008
+    assert _m2(inp=bad) == bm.BIMAMBA_ERR_MISALIGNED
+    par = _params2()
+    par.conv_w = FAKE + 0x43008
+    assert _m2(par=par) == bm.BIMAMBA_ERR_MISALIGNED
     par = _params2()
     par.conv_w = None
     assert _m2(par=par) == bm.BIMAMBA_ERR_INVALID_ARG
     par = _params2()
     par.A = FAKE + 0x40002
     assert _m2(par=par) == bm.BIMAMBA_ERR_MISALIGNED
-    assert _m2(out=FAKE + 0x50001) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2(out=FAKE + 0x50008) == bm.BIMAMBA_ERR_MISALIGNED
     assert _m2(ws=None) == bm.BIMAMBA_ERR_WORKSPACE
     assert _m2(ws_bytes=bm.bimamba2_workspace_bytes(2, 64, 4) - 1) == bm.BIMAMBA_ERR_WORKSPACE
     assert _m2(ws=FAKE + 0x100080) == bm.BIMAMBA_ERR_MISALIGNED
