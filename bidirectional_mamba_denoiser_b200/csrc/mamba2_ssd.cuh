@@ -43,7 +43,8 @@ constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
 // shared memory of m2_ssd_kernel
 constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
               kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90720, kSsdX = 90752, kSsdDL = 109184,
-              kSsdSmem = 109696;
+              kSsdE = 109696, kSsdSmem = 110208;
+constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
 constexpr int kSsdXStride = 36;  // floats per x row in shared memory (144 B: conflict-free 16-byte accesses)
 
 // grid (nchunks, batch, 2), block 256: fp16 tiles of C and B per chunk, rows
@@ -120,6 +121,8 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
     float* sX = reinterpret_cast<float*>(sm + kSsdX);   // [128][kSsdXStride]: row t = x of step t
     float* sDL = reinterpret_cast<float*>(sm + kSsdDL);  // [128]: step size of step t
+    float* sE = reinterpret_cast<float*>(sm + kSsdE);    // [128]: 2^(c of step 32j - c of step s), s in block j
+    int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t L = p.L;
@@ -181,20 +184,8 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
         const bool valid = tok >= 0 && tok < L;
         float x[32], yf[DIR == 1 ? 32 : 1];
         uint4 zq[DIR == 1 ? 4 : 1];  // the reverse epilogue's z: 32 bf16
-        if constexpr (DIR == 1) {
-            if (valid) {  // loaded now, used at the end of the chunk
-                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
-                const float4* ysrc = reinterpret_cast<const float4*>(p.YF + o);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 v = ysrc[i];
-                    yf[4 * i] = v.x; yf[4 * i + 1] = v.y; yf[4 * i + 2] = v.z; yf[4 * i + 3] = v.w;
-                }
-                const uint4* zsrc = reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.z) + o);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) zq[i] = zsrc[i];
-            }
-        }
+        uint32_t sraw[32];
+        tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
         cp_async_wait_all();  // own x row and step size (written and read by this thread only)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -216,6 +207,13 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
         const float c = a + base;
         const float cend = wtot[0] + wtot[1] + wtot[2] + wtot[3];
         c2s[t] = c;
+        {
+            // block j = warp: step s's factor 2^(c_{32j} - c_s) >= 1, usable while the span is small
+            const float cref = __shfl_sync(0xffffffffu, c, 0);
+            sE[t] = ex2_approx(fminf(cref - c, kSsdSpanMax));
+            const float span = cref - __shfl_sync(0xffffffffu, c, 31);
+            if (lane == 0) bigspan[warp] = span > kSsdSpanMax ? 1 : 0;
+        }
         // ---- delta x and W rows of step t (MN-major [s][p])
         {
             const float wdec = ex2_approx(cend - c);
@@ -232,12 +230,26 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
         if (k + 1 < nc) fetch_step(k + 1);  // x is in registers now
         // ---- carried state row n = t decays over the whole chunk
         {
+            tmem_wait_ld(sraw);
             float s[32];
-            tmem_ld32(tmem + 192 + lb, s);
             const float f = ex2_approx(cend);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] *= f;
+            for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(sraw[i]) * f;
             tmem_st32(tmem + 192 + lb, s);
+        }
+        if constexpr (DIR == 1) {
+            if (valid) {  // the epilogue's y_0 and z, in flight while the products run
+                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
+                const float4* ysrc = reinterpret_cast<const float4*>(p.YF + o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v = ysrc[i];
+                    yf[4 * i] = v.x; yf[4 * i + 1] = v.y; yf[4 * i + 2] = v.z; yf[4 * i + 3] = v.w;
+                }
+                const uint4* zsrc = reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.z) + o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) zq[i] = zsrc[i];
+            }
         }
         fence_async_smem();
         tmem_fence_before_sync();
@@ -269,28 +281,53 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
             bulk_g2s(sB, tileb + (int64_t)(k + 1) * 2 * kTileBytes + kTileBytes, kTileBytes, bars + 0);
         }
         // ---- M row t (into C's buffer, K-major [t][s]) and the new state row n = t
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-            float g[32];
-            if (j <= warp) {  // columns s >= 32j reach step t = 32 warp + lane only for j <= warp
-                tmem_ld32(tmem + 32 * j + lb, g);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int s = 32 * j + i;
-                    g[i] = s <= t ? g[i] * ex2_approx(c - c2s[s]) : 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) g[i] = 0.f;
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) st_half8(sC + f16_kmajor(t, 32 * j + 8 * q, Q), g + 8 * q);
-        }
+        // columns s >= 32j reach step t = 32 warp + lane only for j <= warp;
+        // e^(c_t - c_s) = 2^(c_t - c_{32j}) 2^(c_{32j} - c_s) while block j's span is small
         {
-            float s[32];
-            tmem_ld32(tmem + 192 + lb, s);
+            uint32_t sn[32];
+            tmem_ld32_async(tmem + 192 + lb, sn);
+#pragma unroll 1
+            for (int j = 0; j < 4; j += 2) {
+                uint32_t g0[32], g1[32];
+                if (j <= warp) tmem_ld32_async(tmem + 32 * j + lb, g0);
+                if (j + 1 <= warp) tmem_ld32_async(tmem + 32 * (j + 1) + lb, g1);
+                tmem_wait_ld(g0);
+                tmem_wait_ld(g1);
 #pragma unroll
-            for (int pg = 0; pg < 4; ++pg) st_half8(sS + f16_mnmajor(8 * pg, t, P), s + 8 * pg);
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int jb = j + jj;
+                    uint32_t (&gr)[32] = jj == 0 ? g0 : g1;
+                    float m[32];
+                    if (jb <= warp) {
+                        const float cref = c2s[32 * jb];
+                        if (!bigspan[jb]) {
+                            const float F = ex2_approx(c - cref);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const int s = 32 * jb + i;
+                                m[i] = s <= t ? __uint_as_float(gr[i]) * (F * sE[s]) : 0.f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const int s = 32 * jb + i;
+                                m[i] = s <= t ? __uint_as_float(gr[i]) * ex2_approx(c - c2s[s]) : 0.f;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) m[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) st_half8(sC + f16_kmajor(t, 32 * jb + 8 * q, Q), m + 8 * q);
+                }
+            }
+            tmem_wait_ld(sn);
+            float sv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(sn[i]);
+#pragma unroll
+            for (int pg = 0; pg < 4; ++pg) st_half8(sS + f16_mnmajor(8 * pg, t, P), sv + 8 * pg);
         }
         fence_async_smem();
         tmem_fence_before_sync();
@@ -312,9 +349,17 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
         }
         // ---- output of step t
         {
+            uint32_t r1[32], r2[32];
+            tmem_ld32_async(tmem + 128 + lb, r1);
+            tmem_ld32_async(tmem + 160 + lb, r2);
+            tmem_wait_ld(r1);
+            tmem_wait_ld(r2);
             float y1[32], y2[32];
-            tmem_ld32(tmem + 128 + lb, y1);
-            tmem_ld32(tmem + 160 + lb, y2);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                y1[i] = __uint_as_float(r1[i]);
+                y2[i] = __uint_as_float(r2[i]);
+            }
             if (valid) {
                 const float e = ex2_approx(c);
                 const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
