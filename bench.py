@@ -69,7 +69,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "mamba2", "mamba2_long"],
+    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "mamba2", "mamba2_long"],
                     default="layer")
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
@@ -84,6 +84,8 @@ def parse_args(argv=None):
 def workload_of(args) -> W.Workload:
     if args.workload == "layer":
         return W.LAYER_1P3B
+    if args.workload == "decode":
+        return W.BLOCK_DECODE
     if args.workload == "mamba2":
         return W.MAMBA2_1P3B
     if args.workload == "mamba2_long":
@@ -288,7 +290,7 @@ def flags_of(args, bm):
 
 
 def kernel_name(w: W.Workload, args) -> str:
-    if args.workload == "block":
+    if args.workload in ("block", "decode"):
         return "async_block_kernel"
     fam = args.family or (2 if 2 * w.batch * w.d_inner >= SMS * 8 * 32 else 1)
     return "fused_layer_kernel" if fam == 2 else "layer_tma_kernel"
@@ -540,15 +542,67 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     return res
 
 
+def run_decode(args, w, bm, rank, world, dev, stream):
+    """decode: block-cached decoding through a stack of layers, one cached
+    state per layer; each block (steps x layers block steps, commits on the
+    last step) replays as one CUDA graph."""
+    from bidirectional_mamba_denoiser_b200 import decode
+    layers, P, G, K = w.extra["layers"], w.extra["prefix"], w.extra["block"], w.extra["steps_per_block"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + rank)
+    params = [W.make_params(w.d_inner, w.d_state, g, dev) for _ in range(layers)]
+    dec = decode.BlockDecoder(params, w.batch, w.d_inner, W.torch_dtype(w.dtype), dev)
+    pre = W.make_inputs(w.batch, P, w.d_inner, w.d_state, w.dtype, g, dev)
+    torch.cuda.synchronize(dev)
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    dec.prefill(lambda layer: pre, P, stream=stream)  # one prompt, each layer its own parameters
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    prefill_ms = p0.elapsed_time(p1)
+    del pre
+    torch.cuda.empty_cache()
+    pool = [W.make_inputs(w.batch, G, w.d_inner, w.d_state, w.dtype, g, dev) for _ in range(8)]
+    out = torch.empty(layers, w.batch, G, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
+
+    def inputs(s, layer):
+        return pool[(s * layers + layer) % len(pool)]
+
+    dec.block(K, inputs, out, stream=stream)  # one eager block (module loads, first launches)
+    torch.cuda.synchronize(dev)
+    graph = dec.capture_block(K, inputs, out, stream)
+    reps = max(1, args.steps // K)
+
+    def step(_):
+        graph.replay()
+
+    ms, clocks = timed(step, reps, max(1, args.warmup // K), world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    calls = reps * K * layers
+    call_ms = ms / calls
+    elems = w.batch * G * w.d_inner
+    del graph
+    return {
+        "value": whole_job_rate(w.batch * G * calls, world, ms_max / 1e3),
+        "ms_per_step": ms_max / (reps * K), "gpu_launches": calls,
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args)),
+        "hbm": hbm_fraction(block_bytes(w), call_ms), "clocks": clocks,
+        "generated_tokens_per_s": round(w.batch * G * reps * world / (ms_max / 1e3), 1),
+        "prefill_ms": round(prefill_ms, 3), "layers": layers, "steps_per_block": K,
+        "graph": f"one block = {K} steps x {layers} layers = {K * layers} block steps per CUDA graph replay",
+    }
+
+
 def run_ours(args, rank, world, local):
     from bidirectional_mamba_denoiser_b200 import bimamba as bm
     w = workload_of(args)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    if args.workload == "block":
+    if args.workload in ("block", "decode"):
         side = torch.cuda.Stream(dev)  # graphs cannot be captured on the legacy default stream
         with torch.cuda.stream(side):
-            res = run_block(args, w, bm, rank, world, dev, side)
+            res = (run_block if args.workload == "block" else run_decode)(args, w, bm, rank, world, dev, side)
     elif args.workload in ("mamba2", "mamba2_long"):
         res = run_mamba2(args, w, bm, rank, world, dev, stream)
     else:
@@ -561,7 +615,7 @@ def run_ours(args, rank, world, local):
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                        "d_state": w.d_state, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (rotating input sets)" if args.workload != "block"
+                       "l2": "inputs larger than L2 (rotating input sets)" if args.workload not in ("block", "decode")
                        else "block inputs rotate over 8 sets (state stays L2-resident, as in decoding)"},
             "roofline": res.pop("roofline"), "cpu_baseline": res.pop("cpu_baseline", None),
             "e2e": res.pop("e2e", None), "gpu_launches": res.pop("gpu_launches"), "clocks": res.pop("clocks"),

@@ -71,6 +71,10 @@ LONG_SEQ = {L: Workload(f"long_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 2)
             for L in (4096, 16384, 65536, 131072)}
 BLOCK_CACHED = Workload("block_cached_b16_P65536_G32_D4096_bf16", 16, 32, 4096, 16, "bf16", 4,
                         extra={"prefix": 65536, "block": 32, "blocks": 16, "steps_per_block": 128})
+# Block-cached decoding through a stack of layers (the pages' 1.3B denoiser
+# has 24 blocks), one cache per layer; the per-step shape of BLOCK_CACHED.
+BLOCK_DECODE = Workload("decode_24layers_b16_P65536_G32_K128_D4096_bf16", 16, 32, 4096, 16, "bf16", 7,
+                        extra={"layers": 24, "prefix": 65536, "block": 32, "steps_per_block": 128})
 DENOISER_SWEEP = {L: Workload(f"denoiser_48x128_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 3,
                               extra={"layers": 48, "steps": 128})
                   for L in (2048, 8192, 32768, 131072)}
