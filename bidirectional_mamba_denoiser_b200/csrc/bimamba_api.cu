@@ -716,8 +716,9 @@ struct M2Layout {
     size_t v, dl, yf, tiles, total;
 };
 
-// Workspace: conv features [2][batch][L][CH], step sizes [2][batch][H][L],
-// forward output [batch][L][H*P], all fp32, then the fp16 C/B tiles of the
+// Workspace: conv features [2][batch][L][CH] fp32 (the tensor-core path keeps
+// only x there, as fp16 [2][batch][L][H*P]), step sizes [2][batch][H][L],
+// forward output [batch][L][H*P], both fp32, then the fp16 C/B tiles of the
 // tensor-core path [2][batch][ceil(L/128)][2][128 x 128]; each part 256-byte
 // aligned.
 M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
@@ -738,26 +739,32 @@ bool m2_sizes_ok(int batch, int64_t L, int H) {
     return batch >= 1 && 2 * (int64_t)batch <= 65535 && L >= 1 && L <= (int64_t)1 << 31 && H >= 1 && H <= 65535;
 }
 
-// Chunked dual form on the tensor cores: conv features, C/B tiles, forward
-// and reverse chunk scans (four launches).
+// Chunked dual form on the tensor cores: conv features (x in fp16, C/B as
+// chunk tiles), forward and reverse chunk scans (three launches; when L is
+// not a whole number of chunks, the last chunk's tiles are cleared first so
+// that its rows past the end read zeros).
 template <typename Tin, typename Tout>
-int launch_m2_ssd(const bimamba::M2Params& k, unsigned char* tiles, cudaStream_t st) {
+int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
     auto k0 = &bimamba::m2_ssd_kernel<0, Tin, Tout>;
     auto k1 = &bimamba::m2_ssd_kernel<1, Tin, Tout>;
     int rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
     if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k1), bimamba::kSsdSmem);
     if (rc) return rc;
+    const int64_t nc = (k.L + bimamba::kSQ - 1) / bimamba::kSQ;
+    if (k.L % bimamba::kSQ) {
+        const size_t pair = 2 * (size_t)bimamba::kTileBytes;
+        if (cudaMemset2DAsync(k.tiles + (nc - 1) * pair, (size_t)nc * pair, 0, pair, (size_t)(2 * k.batch), st) !=
+            cudaSuccess)
+            return BIMAMBA_ERR_CUDA;
+    }
     const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
                   (unsigned)(2 * k.batch));
-    bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
-    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    const unsigned nc = (unsigned)((k.L + bimamba::kSQ - 1) / bimamba::kSQ);
-    bimamba::m2_tiles_kernel<<<dim3(nc, (unsigned)k.batch, 2), 256, 0, st>>>(k, tiles);
+    bimamba::m2_prep_kernel<Tin, true><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
     const dim3 g2((unsigned)k.H, (unsigned)k.batch);
-    k0<<<g2, 128, bimamba::kSsdSmem, st>>>(k, tiles);
+    k0<<<g2, 128, bimamba::kSsdSmem, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    k1<<<g2, 128, bimamba::kSsdSmem, st>>>(k, tiles);
+    k1<<<g2, 128, bimamba::kSsdSmem, st>>>(k);
     return launch_status();
 }
 
@@ -765,7 +772,7 @@ template <typename Tin, typename Tout>
 int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
     const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
                   (unsigned)(2 * k.batch));
-    bimamba::m2_prep_kernel<Tin><<<g1, 128, 0, st>>>(k);
+    bimamba::m2_prep_kernel<Tin, false><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
     const dim3 g2((unsigned)k.H, (unsigned)k.batch);
     bimamba::m2_scan_kernel<0, Tin, Tout><<<g2, 32, 0, st>>>(k);
@@ -835,9 +842,10 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
-        unsigned char* tiles = ws + lay.tiles;
-        if (out_bf) return launch_m2_ssd<bf16, bf16>(k, tiles, st);
-        return launch_m2_ssd<bf16, float>(k, tiles, st);
+        k.tiles = ws + lay.tiles;
+        k.X16 = reinterpret_cast<__half*>(ws + lay.v);  // in place of the fp32 features
+        if (out_bf) return launch_m2_ssd<bf16, bf16>(k, st);
+        return launch_m2_ssd<bf16, float>(k, st);
     }
     if (in_bf && out_bf) return launch_m2<bf16, bf16>(k, st);
     if (in_bf) return launch_m2<bf16, float>(k, st);

@@ -36,7 +36,10 @@
 // state exactly unchanged.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "scan_kernels.cuh"
+#include "tcgen05_util.cuh"
 #include "tma_util.cuh"
 
 namespace bimamba {
@@ -65,29 +68,54 @@ struct M2Params {
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
     long long wait_limit;  // SM clocks a wait for a tile or a product may take (tensor-core path)
     int starve;            // test aid (tensor-core path): issue no tile copies, so every wait gives up
+    // tensor-core path: the prep kernel writes x as fp16 ([2][batch][L][H*P], in V's place) and the
+    // fp16 C/B tiles ([2][batch][ceil(L/128)][C | B] x 128 x 128, rows in step order) instead of V
+    __half* X16;
+    unsigned char* tiles;
 };
 
-// 8 consecutive channels of one row as fp32 (one 16-byte load for bf16).
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 q = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
-        v[2 * u] = __uint_as_float(w[u] << 16);
-        v[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+// 8 consecutive channels of one row, kept as loaded (bf16: one 16-byte
+// word, unpacked on use) to hold the prep kernel's 11 rows in few registers.
+template <typename Tin>
+struct Row8;
+template <>
+struct Row8<__nv_bfloat16> {
+    uint4 q;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { q = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { q = make_uint4(0u, 0u, 0u, 0u); }
+    // bf16 -> fp32 is exact: the bf16 bits are the high half
+    __device__ __forceinline__ float get(int i) const {
+        const uint32_t w = i < 2 ? q.x : i < 4 ? q.y : i < 6 ? q.z : q.w;
+        return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
     }
-}
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
+};
+template <>
+struct Row8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = *reinterpret_cast<const float4*>(p);
+        b = *reinterpret_cast<const float4*>(p + 4);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float get(int i) const {
+        const float4& v = i < 4 ? a : b;
+        const int j = i & 3;
+        return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+    }
+};
+
+constexpr int kM2Chunk = 128;  // steps per chunk of the tensor-core path
 
 // grid (ceil(L / 8), ceil(CH / 1024), 2 * batch), block 128: thread = 8
 // consecutive channels of one direction over 8 tokens; its 11 input rows
 // (8 + the 3-row conv halo) are loaded first, 16 bytes at a time, then the
 // 64 outputs computed and stored as 16-byte rows.  Needs CH % 8 == 0 and
 // 16-byte aligned rows (CH * sizeof(Tin) % 16 == 0, aligned xbc).
-template <typename Tin>
+// TILES = false: every channel to V (fp32).  TILES = true (tensor-core
+// path): x channels to X16 (fp16) and B, C channels as fp16 rows of the
+// chunk tiles at the token's step (forward: token t is step t; reverse:
+// step L-1-t), in the canonical K-major layout.
+template <typename Tin, bool TILES>
 __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     constexpr int TT = kM2PrepT;
     const int c0 = (blockIdx.y * 128 + threadIdx.x) * 8;
@@ -110,17 +138,15 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
         }
         float* V = p.V + ((int64_t)r * p.batch + b) * L * CH + c0;
         // xw[k] = row t0 - 3 + k (forward) or t0 + k (reverse), zero outside [0, L)
-        float xw[TT + 3][8];
+        Row8<Tin> xw[TT + 3];
         const int64_t base = r == 0 ? t0 - 3 : t0;
 #pragma unroll
         for (int k = 0; k < TT + 3; ++k) {
             const int64_t i = base + k;
-            if (i >= 0 && i < L) {
-                load8(X + i * CH, xw[k]);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) xw[k][q] = 0.f;
-            }
+            if (i >= 0 && i < L)
+                xw[k].load(X + i * CH);
+            else
+                xw[k].zero();
         }
 #pragma unroll
         for (int k = 0; k < TT; ++k) {
@@ -130,15 +156,35 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 // forward: tap j on x[t-3+j] = xw[k+j]; reverse: tap j on x[t+3-j] = xw[k+3-j]
-                const float a = r == 0 ? fmaf(w[q][3], xw[k + 3][q], fmaf(w[q][2], xw[k + 2][q],
-                                             fmaf(w[q][1], xw[k + 1][q], fmaf(w[q][0], xw[k][q], cb[q]))))
-                                       : fmaf(w[q][3], xw[k][q], fmaf(w[q][2], xw[k + 1][q],
-                                             fmaf(w[q][1], xw[k + 2][q], fmaf(w[q][0], xw[k + 3][q], cb[q]))));
+                const float a = r == 0 ? fmaf(w[q][3], xw[k + 3].get(q), fmaf(w[q][2], xw[k + 2].get(q),
+                                             fmaf(w[q][1], xw[k + 1].get(q), fmaf(w[q][0], xw[k].get(q), cb[q]))))
+                                       : fmaf(w[q][3], xw[k].get(q), fmaf(w[q][2], xw[k + 1].get(q),
+                                             fmaf(w[q][1], xw[k + 2].get(q), fmaf(w[q][0], xw[k + 3].get(q), cb[q]))));
                 v[q] = silu(a);
             }
-            float4* dst = reinterpret_cast<float4*>(V + t * CH);
-            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+            if constexpr (!TILES) {
+                float4* dst = reinterpret_cast<float4*>(V + t * CH);
+                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else {
+                const __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+                const __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
+                const uint4 q = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                                           *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+                const int HP = H * kM2P;
+                if (c0 < HP) {
+                    *reinterpret_cast<uint4*>(p.X16 + (((int64_t)r * p.batch + b) * L + t) * HP + c0) = q;
+                } else {
+                    const bool isB = c0 < HP + kM2N;
+                    const int n0 = c0 - HP - (isB ? 0 : kM2N);
+                    const int64_t step = r == 0 ? t : L - 1 - t;
+                    const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
+                    unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + step / kM2Chunk) *
+                                                     (2 * kM2Chunk * kM2N * 2);
+                    *reinterpret_cast<uint4*>(T + (isB ? kM2Chunk * kM2N * 2 : 0) +
+                                              f16_kmajor((int)(step % kM2Chunk), n0, kM2N)) = q;
+                }
+            }
         }
     }
     if (blockIdx.y == 0) {

@@ -18,8 +18,9 @@
 // One CTA = one (head, batch row) in one direction, 128 threads; thread t
 // owns step t of the chunk (TMEM lane t) for the per-step work and state
 // row n = t for the state epilogue.  The chunk's C and B arrive as fp16
-// tiles (laid out by m2_tiles_kernel in the canonical K-major form, rows in
-// step order so that the reverse direction needs no other code) by bulk
+// tiles (in the canonical K-major form, rows in
+// step order so that the reverse direction needs no other code; written by
+// m2_prep_kernel<Tin, true>) by bulk
 // copies; the B tile of the next chunk is fetched as soon as the products
 // that read B are done, the C tile once M (which reuses C's buffer) has been
 // consumed, and each thread's x row and step size of the next chunk by
@@ -38,43 +39,14 @@
 
 namespace bimamba {
 
-constexpr int kSQ = 128;                    // steps per chunk (= MMA M)
+constexpr int kSQ = kM2Chunk;               // steps per chunk (= MMA M)
 constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
 // shared memory of m2_ssd_kernel
 constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
-              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90720, kSsdX = 90752, kSsdDL = 109184,
-              kSsdE = 109696, kSsdSmem = 110208;
+              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90720, kSsdX = 90752, kSsdDL = 100992,
+              kSsdE = 101504, kSsdSmem = 102016;
 constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
-constexpr int kSsdXStride = 36;  // floats per x row in shared memory (144 B: conflict-free 16-byte accesses)
-
-// grid (nchunks, batch, 2), block 256: fp16 tiles of C and B per chunk, rows
-// in step order (reverse direction: step s of chunk k is token L-1-kQ-s),
-// zero rows past either end.  tiles: [2][batch][nchunks][C | B] x 32 KB.
-__global__ void __launch_bounds__(256) m2_tiles_kernel(const M2Params p, unsigned char* tiles) {
-    const int k = blockIdx.x, b = blockIdx.y, r = blockIdx.z;
-    const int64_t L = p.L;
-    const int CH = p.CH, HP = p.H * kM2P;
-    const int nc = (int)((L + kSQ - 1) / kSQ);
-    const float* Vb = p.V + ((int64_t)r * p.batch + b) * L * CH;
-    unsigned char* T = tiles + (((int64_t)r * p.batch + b) * nc + k) * (2 * kTileBytes);
-    for (int e = threadIdx.x; e < 2 * kSQ * (kM2N / 8); e += 256) {
-        const int which = e / (kSQ * (kM2N / 8));  // 0 = C, 1 = B
-        const int rem = e % (kSQ * (kM2N / 8));
-        const int s = rem / (kM2N / 8), g = rem % (kM2N / 8);
-        const int64_t tok = r == 0 ? (int64_t)k * kSQ + s : L - 1 - (int64_t)k * kSQ - s;
-        uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-        if (tok >= 0 && tok < L) {
-            const float* src = Vb + tok * CH + HP + (which == 0 ? kM2N : 0) + 8 * g;
-            const float4 v0 = *reinterpret_cast<const float4*>(src);
-            const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
-            __half2 h0 = __floats2half2_rn(v0.x, v0.y), h1 = __floats2half2_rn(v0.z, v0.w);
-            __half2 h2 = __floats2half2_rn(v1.x, v1.y), h3 = __floats2half2_rn(v1.z, v1.w);
-            packed = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                                *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-        }
-        *reinterpret_cast<uint4*>(T + which * kTileBytes + f16_kmajor(s, 8 * g, kM2N)) = packed;
-    }
-}
+constexpr int kSsdXStride = 40;  // halves per x row in shared memory (80 B: conflict-free 16-byte accesses)
 
 // 8 fp32 values -> 8 fp16 in one 16-byte store.
 __device__ __forceinline__ void st_half8(unsigned char* dst, const float* v) {
@@ -107,7 +79,7 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)
 // grid (H, batch), block 128, dynamic shared memory kSsdSmem.  DIR 0 stores
 // y_0 to p.YF; DIR 1 adds it and applies the gate.
 template <int DIR, typename Tin, typename Tout>
-__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const unsigned char* tiles) {
+__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     constexpr int Q = kSQ, P = kM2P;
     extern __shared__ __align__(128) unsigned char sm[];
     unsigned char* sC = sm + kSsdC;
@@ -119,17 +91,17 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
     float* wtot = reinterpret_cast<float*>(sm + kSsdTot);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSsdBar);  // B tile, C tile, products 1-3, product 4
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
-    float* sX = reinterpret_cast<float*>(sm + kSsdX);   // [128][kSsdXStride]: row t = x of step t
+    __half* sX = reinterpret_cast<__half*>(sm + kSsdX);  // [128][kSsdXStride]: row t = x of step t (fp16)
     float* sDL = reinterpret_cast<float*>(sm + kSsdDL);  // [128]: step size of step t
     float* sE = reinterpret_cast<float*>(sm + kSsdE);    // [128]: 2^(c of step 32j - c of step s), s in block j
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t L = p.L;
-    const int H = p.H, CH = p.CH, HP = H * P;
+    const int H = p.H, HP = H * P;
     const int nc = (int)((L + Q - 1) / Q);
-    const unsigned char* tileb = tiles + ((int64_t)DIR * p.batch + b) * nc * (2 * kTileBytes);
-    const float* Vx = p.V + ((int64_t)DIR * p.batch + b) * L * CH + (int64_t)h * P;
+    const unsigned char* tileb = p.tiles + ((int64_t)DIR * p.batch + b) * nc * (2 * kTileBytes);
+    const __half* Vx = p.X16 + ((int64_t)DIR * p.batch + b) * L * HP + (int64_t)h * P;
     const float* Dh = p.DL + (((int64_t)DIR * p.batch + b) * H + h) * L;
     const float A2 = p.A[DIR * H + h] * kLog2e;
     const float Dsk = p.Dskip[DIR * H + h];
@@ -163,9 +135,9 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
     auto fetch_step = [&](int kk) {
         const int64_t tk = DIR == 0 ? (int64_t)kk * Q + t : L - 1 - (int64_t)kk * Q - t;
         const bool ok = tk >= 0 && tk < L;
-        const float* src = Vx + (ok ? tk : 0) * CH;
+        const __half* src = Vx + (ok ? tk : 0) * HP;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cp_async<16>(sX + t * kSsdXStride + 4 * i, src + 4 * i, ok);
+        for (int i = 0; i < 4; ++i) cp_async<16>(sX + t * kSsdXStride + 8 * i, src + 8 * i, ok);
         cp_async<4>(sDL + t, Dh + (ok ? tk : 0), ok);
         cp_async_commit();
     };
@@ -188,9 +160,15 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p, const 
         tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
         cp_async_wait_all();  // own x row and step size (written and read by this thread only)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 v = *reinterpret_cast<const float4*>(sX + t * kSsdXStride + 4 * i);
-            x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sX + t * kSsdXStride + 8 * i);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
+                x[8 * i + 2 * u] = f.x;
+                x[8 * i + 2 * u + 1] = f.y;
+            }
         }
         const float dl = sDL[t];
         // ---- c_t: inclusive scan of delta A (log2 units) over the chunk
