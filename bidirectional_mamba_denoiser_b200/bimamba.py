@@ -63,6 +63,10 @@ class Params2(ctypes.Structure):
                 ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
 
 
+class FwdState2(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_void_p), ("conv_xbc", ctypes.c_void_p)]
+
+
 class Inputs2(ctypes.Structure):
     _fields_ = [("xbc", ctypes.c_void_p * 2), ("z", ctypes.c_void_p), ("dt", ctypes.c_void_p * 2),
                 ("dtype", ctypes.c_int)]
@@ -93,6 +97,12 @@ def _load():
     lib.bimamba2_layer_fwd.argtypes = [ctypes.POINTER(Inputs2), ctypes.POINTER(Params2), P, I,
                                        I, I64, I, I, I, U, P, SZ, P]
     lib.bimamba2_layer_fwd.restype = I
+    lib.bimamba2_prefix_state.argtypes = [ctypes.POINTER(Inputs2), ctypes.POINTER(Params2), I, I64, I, I, I,
+                                          ctypes.POINTER(FwdState2), P, SZ, P]
+    lib.bimamba2_prefix_state.restype = I
+    lib.bimamba2_block_step.argtypes = [ctypes.POINTER(FwdState2), ctypes.POINTER(Inputs2), I64, ctypes.POINTER(Params2),
+                                        P, I, I, I, I, I, ctypes.POINTER(FwdState2), U, P, SZ, P]
+    lib.bimamba2_block_step.restype = I
     lib.bimamba_status_string.argtypes = [I]
     lib.bimamba_status_string.restype = ctypes.c_char_p
     lib.bimamba_abi_version.restype = I
@@ -293,4 +303,75 @@ def bimamba2_layer_fwd(xbc, z, dt, params: dict, out=None, out_dtype=None, flags
                                 _stream(stream))
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba2_layer_fwd", rc)
+    return out
+
+
+def _params2(params: dict) -> Params2:
+    return Params2(_ptr(params["A"]), _ptr(params["D"]), _ptr(params["dt_bias"]), _ptr(params["conv_w"]),
+                   _ptr(params.get("conv_b")))
+
+
+def _workspace2(workspace, batch, L, H, P, N, device):
+    need = bimamba2_workspace_bytes(batch, L, H, P, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=device, dtype=torch.uint8)
+    return workspace
+
+
+def bimamba2_prefix_state(xbc, dt, params: dict, S_out=None, conv_out=None, workspace=None, stream=None):
+    """Forward scan of the Mamba-2 mixer over a prefix: xbc, dt of the forward
+    direction ([b, P, CH], [b, P, H], or [2, ...] stacks whose first entry is
+    used).  Returns (S [b, H, 32, N] fp32, conv_xbc [b, 3, CH])."""
+    x0 = xbc[0] if (isinstance(xbc, (tuple, list)) or xbc.dim() == 4) else xbc
+    d0 = dt[0] if (isinstance(dt, (tuple, list)) or dt.dim() == 4) else dt
+    b, L, CH = x0.shape
+    H = d0.shape[-1]
+    P = M2_HEADDIM
+    N = (CH - H * P) // 2
+    if S_out is None:
+        S_out = torch.empty(b, H, P, N, device=x0.device, dtype=torch.float32)
+    if conv_out is None:
+        conv_out = torch.empty(b, 3, CH, device=x0.device, dtype=x0.dtype)
+    workspace = _workspace2(workspace, b, L, H, P, N, x0.device)
+    inp = Inputs2()
+    inp.xbc[0] = _ptr(x0)
+    inp.dt[0] = _ptr(d0)
+    inp.dtype = _dtype_code(x0.dtype)
+    par = _params2(params)
+    st = FwdState2(_ptr(S_out), _ptr(conv_out))
+    rc = lib.bimamba2_prefix_state(ctypes.byref(inp), ctypes.byref(par), b, L, H, P, N, ctypes.byref(st),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba2_prefix_state", rc)
+    return S_out, conv_out
+
+
+def bimamba2_block_step(state, xbc, z, dt, params: dict, out=None, out_dtype=None, new_state=None, flags: int = 0,
+                        workspace=None, stream=None):
+    """One denoising step of the Mamba-2 mixer on the active block from
+    state = (S, conv_xbc): xbc [2, b, G, CH] (or a pair), z [b, G, H*P],
+    dt [2, b, G, H].  new_state = (S, conv_xbc) to commit into (may be
+    `state` itself).  Returns out [b, G, H*P]."""
+    x0, x1 = _pair(xbc)
+    d0, d1 = _pair(dt)
+    b, G, H = d0.shape
+    HP = z.shape[-1]
+    P = HP // H
+    N = (x0.shape[-1] - HP) // 2
+    if out is None:
+        out = torch.empty(b, G, HP, device=z.device, dtype=out_dtype or z.dtype)
+    workspace = _workspace2(workspace, b, G, H, P, N, z.device)
+    inp = Inputs2()
+    inp.xbc[0], inp.xbc[1] = _ptr(x0), _ptr(x1)
+    inp.z = _ptr(z)
+    inp.dt[0], inp.dt[1] = _ptr(d0), _ptr(d1)
+    inp.dtype = _dtype_code(z.dtype)
+    par = _params2(params)
+    st = FwdState2(_ptr(state[0]), _ptr(state[1]))
+    ns = FwdState2(_ptr(new_state[0]), _ptr(new_state[1])) if new_state is not None else None
+    rc = lib.bimamba2_block_step(ctypes.byref(st), ctypes.byref(inp), G, ctypes.byref(par), _ptr(out),
+                                 _dtype_code(out.dtype), b, H, P, N, ctypes.byref(ns) if ns is not None else None,
+                                 flags, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba2_block_step", rc)
     return out

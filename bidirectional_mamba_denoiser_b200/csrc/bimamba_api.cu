@@ -781,9 +781,138 @@ int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
     return launch_status();
 }
 
+// Shared checks of the Mamba-2 entry points: parameters and the 16-byte
+// alignment the kernels' vector accesses need.
+int m2_check_params(const bimamba2_params_t* p) {
+    if (!p || !p->A || !p->D || !p->dt_bias || !p->conv_w) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_w, 16) ||
+        (p->conv_b && !aligned(p->conv_b, 4)))
+        return BIMAMBA_ERR_MISALIGNED;
+    return BIMAMBA_OK;
+}
+
+int m2_check_state(const bimamba2_fwd_state_t* s) {
+    if (!s || !s->S || !s->conv_xbc) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(s->S, 16) || !aligned(s->conv_xbc, 16)) return BIMAMBA_ERR_MISALIGNED;
+    return BIMAMBA_OK;
+}
+
+void m2_fill_params(bimamba::M2Params& k, const bimamba2_params_t* p) {
+    k.A = p->A;
+    k.Dskip = p->D;
+    k.dt_bias = p->dt_bias;
+    k.conv_w = p->conv_w;
+    k.conv_b = p->conv_b;
+}
+
 }  // namespace
 
 extern "C" {
+
+int bimamba2_prefix_state(const bimamba2_inputs_t* prefix, const bimamba2_params_t* p, int batch, int64_t P,
+                          int nheads, int headdim, int d_state, bimamba2_fwd_state_t* state_out, void* workspace,
+                          size_t workspace_bytes, void* cuda_stream) {
+    if (!prefix || !m2_sizes_ok(batch, P, nheads)) return BIMAMBA_ERR_INVALID_ARG;
+    if (headdim != bimamba::kM2P || d_state != bimamba::kM2N) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!dtype_ok(prefix->dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!prefix->xbc[0] || !prefix->dt[0]) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(prefix->xbc[0], 16) || !aligned(prefix->dt[0], elem_size(prefix->dtype))) return BIMAMBA_ERR_MISALIGNED;
+    int rc = m2_check_params(p);
+    if (rc) return rc;
+    if ((rc = m2_check_state(state_out))) return rc;
+    const M2Layout lay = m2_layout(batch, P, nheads, headdim, d_state);
+    if (!workspace || workspace_bytes < lay.total) return BIMAMBA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BIMAMBA_ERR_MISALIGNED;
+    bimamba::M2Params k = {};
+    k.xbc[0] = k.xbc[1] = prefix->xbc[0];
+    k.dt[0] = k.dt[1] = prefix->dt[0];
+    m2_fill_params(k, p);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    k.V = reinterpret_cast<float*>(ws + lay.v);
+    k.DL = reinterpret_cast<float*>(ws + lay.dl);
+    k.L = P;
+    k.H = nheads;
+    k.CH = nheads * headdim + 2 * d_state;
+    k.batch = batch;
+    k.dir_scale[0] = k.dir_scale[1] = 1.f;
+    k.S_out = state_out->S;
+    k.tail_out = state_out->conv_xbc;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const dim3 g1((unsigned)((P + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
+                  (unsigned)batch);  // direction 0 only
+    const dim3 g2((unsigned)nheads, (unsigned)batch);
+    const dim3 g3((unsigned)((k.CH + 127) / 128), (unsigned)batch);
+    if (prefix->dtype == BIMAMBA_BF16) {
+        bimamba::m2_prep_kernel<bf16, false><<<g1, 128, 0, st>>>(k);
+        bimamba::m2_scan_kernel<0, bf16, float><<<g2, 32, 0, st>>>(k);
+        bimamba::m2_tail_kernel<bf16><<<g3, 128, 0, st>>>(k);
+    } else {
+        bimamba::m2_prep_kernel<float, false><<<g1, 128, 0, st>>>(k);
+        bimamba::m2_scan_kernel<0, float, float><<<g2, 32, 0, st>>>(k);
+        bimamba::m2_tail_kernel<float><<<g3, 128, 0, st>>>(k);
+    }
+    return launch_status();
+}
+
+int bimamba2_block_step(const bimamba2_fwd_state_t* prefix_state, const bimamba2_inputs_t* block, int64_t block_len,
+                        const bimamba2_params_t* p, void* out, bimamba_dtype_t out_dtype, int batch, int nheads,
+                        int headdim, int d_state, bimamba2_fwd_state_t* new_state, unsigned flags, void* workspace,
+                        size_t workspace_bytes, void* cuda_stream) {
+    if (!block || !out || !m2_sizes_ok(batch, block_len, nheads)) return BIMAMBA_ERR_INVALID_ARG;
+    if (headdim != bimamba::kM2P || d_state != bimamba::kM2N) return BIMAMBA_ERR_UNSUPPORTED;
+    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_UNSUPPORTED;
+    if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(block->dtype) || !dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    const void* ptrs[5] = {block->xbc[0], block->xbc[1], block->z, block->dt[0], block->dt[1]};
+    for (const void* q : ptrs) {
+        if (!q) return BIMAMBA_ERR_INVALID_ARG;
+        if (!aligned(q, elem_size(block->dtype))) return BIMAMBA_ERR_MISALIGNED;
+    }
+    if (!aligned(block->z, 16) || !aligned(block->xbc[0], 16) || !aligned(block->xbc[1], 16) || !aligned(out, 16))
+        return BIMAMBA_ERR_MISALIGNED;
+    int rc = m2_check_params(p);
+    if (rc) return rc;
+    if ((rc = m2_check_state(prefix_state))) return rc;
+    if (new_state && (rc = m2_check_state(new_state))) return rc;
+    const M2Layout lay = m2_layout(batch, block_len, nheads, headdim, d_state);
+    if (!workspace || workspace_bytes < lay.total) return BIMAMBA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BIMAMBA_ERR_MISALIGNED;
+    bimamba::M2Params k = {};
+    for (int r = 0; r < 2; ++r) {
+        k.xbc[r] = block->xbc[r];
+        k.dt[r] = block->dt[r];
+    }
+    k.z = block->z;
+    m2_fill_params(k, p);
+    k.out = out;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    k.V = reinterpret_cast<float*>(ws + lay.v);
+    k.DL = reinterpret_cast<float*>(ws + lay.dl);
+    k.YF = reinterpret_cast<float*>(ws + lay.yf);
+    k.L = block_len;
+    k.H = nheads;
+    k.CH = nheads * headdim + 2 * d_state;
+    k.batch = batch;
+    k.dir_scale[0] = (flags & BIMAMBA_REV_ONLY) ? 0.f : 1.f;
+    k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
+    k.S_in = prefix_state->S;
+    k.tail_in = prefix_state->conv_xbc;
+    k.S_out = new_state ? new_state->S : nullptr;
+    k.tail_out = new_state ? new_state->conv_xbc : nullptr;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    const bool in_bf = block->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
+    if (in_bf && out_bf) rc = launch_m2<bf16, bf16>(k, st);
+    else if (in_bf) rc = launch_m2<bf16, float>(k, st);
+    else if (out_bf) rc = launch_m2<float, bf16>(k, st);
+    else rc = launch_m2<float, float>(k, st);
+    if (rc || !new_state) return rc;
+    const dim3 g3((unsigned)((k.CH + 127) / 128), (unsigned)batch);
+    if (in_bf)
+        bimamba::m2_tail_kernel<bf16><<<g3, 128, 0, st>>>(k);
+    else
+        bimamba::m2_tail_kernel<float><<<g3, 128, 0, st>>>(k);
+    return launch_status();
+}
 
 size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state) {
     if (!m2_sizes_ok(batch, L, nheads) || headdim <= 0 || d_state <= 0) return 0;

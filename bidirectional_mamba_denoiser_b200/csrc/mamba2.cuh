@@ -72,6 +72,13 @@ struct M2Params {
     // fp16 C/B tiles ([2][batch][ceil(L/128)][C | B] x 128 x 128, rows in step order) instead of V
     __half* X16;
     unsigned char* tiles;
+    // block-cached decoding (step-by-step scan): the forward direction's cached
+    // state [batch][H][P][N] fp32 and conv tail [batch][3][CH] (xBC rows before
+    // token 0, oldest first); nullptr = zero state / zero halo / no commit
+    const float* S_in;
+    float* S_out;
+    const void* tail_in;
+    void* tail_out;
 };
 
 // 8 consecutive channels of one row, kept as loaded (bf16: one 16-byte
@@ -140,11 +147,14 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
         // xw[k] = row t0 - 3 + k (forward) or t0 + k (reverse), zero outside [0, L)
         Row8<Tin> xw[TT + 3];
         const int64_t base = r == 0 ? t0 - 3 : t0;
+        const Tin* tail = r == 0 && p.tail_in ? static_cast<const Tin*>(p.tail_in) + (int64_t)b * 3 * CH + c0 : nullptr;
 #pragma unroll
         for (int k = 0; k < TT + 3; ++k) {
             const int64_t i = base + k;
             if (i >= 0 && i < L)
                 xw[k].load(X + i * CH);
+            else if (i < 0 && tail)  // forward halo from the cached tail (rows -3..-1)
+                xw[k].load(tail + (3 + i) * CH);
             else
                 xw[k].zero();
         }
@@ -263,11 +273,23 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
     const float A2 = p.A[DIR * H + h] * kLog2e;
     const float Dskip = p.Dskip[DIR * H + h];
     const float scale = p.dir_scale[DIR];
+    // S[i][4q+j] = state (row 8pb + i, state 32q + 4nb + j)
     float S[8][16];
+    const int64_t sbase = ((int64_t)b * H + h) * P * N;
+    if (DIR == 0 && p.S_in) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int n = 0; n < 16; ++n) S[i][n] = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(p.S_in + sbase + (8 * pb + i) * N + 32 * q + 4 * nb);
+                S[i][4 * q] = v.x; S[i][4 * q + 1] = v.y; S[i][4 * q + 2] = v.z; S[i][4 * q + 3] = v.w;
+            }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int n = 0; n < 16; ++n) S[i][n] = 0.f;
+    }
     float acum = 1.f;
 
     stage(0, 0);
@@ -331,7 +353,7 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
                 const float y = (acum * yr + Dskip * xs[buf][rr][prow]) * scale;
                 const int64_t o = ((int64_t)b * L + t) * HP + (int64_t)h * P + prow;
                 if constexpr (DIR == 0) {
-                    p.YF[o] = y;
+                    if (p.YF) p.YF[o] = y;  // no y for a prefix scan
                 } else {
                     const float zv = ldf(&zs[buf][rr][0], prow);
                     stf(static_cast<Tout*>(p.out), o, (ys[buf][rr][prow] + y) * silu(zv));
@@ -341,6 +363,39 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
         __syncwarp();
         if (i + 2 < nc) stage(i + 2, buf);
     }
+    // commit: the forward state after the last token (each element written by the lane that read it)
+    if (DIR == 0 && p.S_out) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4*>(p.S_out + sbase + (8 * pb + i) * N + 32 * q + 4 * nb) =
+                    make_float4(acum * S[i][4 * q], acum * S[i][4 * q + 1], acum * S[i][4 * q + 2], acum * S[i][4 * q + 3]);
+    }
+}
+
+// grid (ceil(CH / 128), batch), block 128: the forward conv tail after L more
+// tokens of xBC (direction 0): rows L-3..L-1, reaching back into the old tail
+// when L < 3.  Each thread reads its channel's three rows before writing, so
+// tail_out may be tail_in.
+template <typename Tin>
+__global__ void __launch_bounds__(128) m2_tail_kernel(const M2Params p) {
+    const int c = blockIdx.x * 128 + threadIdx.x;
+    const int b = blockIdx.y;
+    if (c >= p.CH) return;
+    const int64_t L = p.L;
+    const int CH = p.CH;
+    const Tin* X = static_cast<const Tin*>(p.xbc[0]) + (int64_t)b * L * CH + c;
+    const Tin* old = p.tail_in ? static_cast<const Tin*>(p.tail_in) + (int64_t)b * 3 * CH + c : nullptr;
+    Tin v[3];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+        const int64_t t = L - 3 + q;
+        v[q] = t >= 0 ? X[t * CH] : (old ? old[(t + 3) * CH] : cvt_from<Tin>(0.f));
+    }
+    Tin* out = static_cast<Tin*>(p.tail_out) + (int64_t)b * 3 * CH + c;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) out[q * CH] = v[q];
 }
 
 }  // namespace bimamba

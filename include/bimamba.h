@@ -241,6 +241,43 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t *in, const bimamba2_params_t *p,
                        int batch, int64_t L, int nheads, int headdim, int d_state,
                        unsigned flags, void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* Cached forward state of the Mamba-2 mixer for block-cached decoding
+ * ([DM] §4.3; [BD] abstract: the reverse scan restricted to the active block
+ * makes the forward state an exact cache). */
+typedef struct {
+    float *S;          /* [batch][nheads][headdim][d_state] fp32, 16-byte aligned */
+    void *conv_xbc;    /* [batch][3][CH] of the input dtype, 16-byte aligned: the forward
+                          direction's last three xBC rows, oldest first */
+} bimamba2_fwd_state_t;
+
+/* Forward scan of the Mamba-2 mixer over a prefix of P tokens from a zero
+ * state: writes state_out->S and state_out->conv_xbc.  Reads prefix->xbc[0]
+ * and prefix->dt[0] (the rest may be NULL).  workspace: at least
+ * bimamba2_workspace_bytes(batch, P, ...) bytes, 256-byte aligned.  Three
+ * launches (conv features, forward scan with the final state, conv tail);
+ * step-by-step scan on the CUDA cores in fp32. */
+int bimamba2_prefix_state(const bimamba2_inputs_t *prefix, const bimamba2_params_t *p,
+                          int batch, int64_t P, int nheads, int headdim, int d_state,
+                          bimamba2_fwd_state_t *state_out, void *workspace, size_t workspace_bytes,
+                          void *cuda_stream);
+
+/* One denoising step of the Mamba-2 mixer on the active block of block_len
+ * tokens: the forward direction continues from *prefix_state (its conv reads
+ * the cached tail before the block), the reverse direction sees the block
+ * alone (zero state after its last token, conv zero-padded past its end);
+ * out = (y_0 + y_1) * silu(z), [batch][block_len][nheads*headdim].  If
+ * new_state is not NULL the forward state and conv tail after the block are
+ * written there (commit); new_state may be prefix_state itself.  workspace:
+ * at least bimamba2_workspace_bytes(batch, block_len, ...) bytes.  Flags:
+ * BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY or 0.  Step-by-step scan on the CUDA
+ * cores in fp32; 3 launches, 4 with a commit. */
+int bimamba2_block_step(const bimamba2_fwd_state_t *prefix_state, const bimamba2_inputs_t *block,
+                        int64_t block_len, const bimamba2_params_t *p,
+                        void *out, bimamba_dtype_t out_dtype,
+                        int batch, int nheads, int headdim, int d_state,
+                        bimamba2_fwd_state_t *new_state, unsigned flags,
+                        void *workspace, size_t workspace_bytes, void *cuda_stream);
+
 /* Read (and, if reset != 0, clear) the error word of the current device.
  * Kernels never wait without bound: a wait for a tile that gives up after
  * about two seconds sets bit 0 (a tile load that never arrived) and the kernel

@@ -264,3 +264,55 @@ def test_mamba2_rejects():
     assert _m2(ws=None) == bm.BIMAMBA_ERR_WORKSPACE
     assert _m2(ws_bytes=bm.bimamba2_workspace_bytes(2, 64, 4) - 1) == bm.BIMAMBA_ERR_WORKSPACE
     assert _m2(ws=FAKE + 0x100080) == bm.BIMAMBA_ERR_MISALIGNED
+
+
+def _state2(base=FAKE + 0x200000):
+    return bm.FwdState2(base, base + 0x100000)
+
+
+def _m2_prefix(**broken):
+    assert broken, "a validation case must break some argument"
+    kw = dict(inp=None, par=None, batch=2, P=64, H=4, Pd=32, N=128, state=None, ws=FAKE + 0x400000, ws_bytes=None)
+    kw.update(broken)
+    inp = _inputs2() if kw["inp"] is None else kw["inp"]
+    par = _params2() if kw["par"] is None else kw["par"]
+    st = _state2() if kw["state"] is None else kw["state"]
+    wsb = kw["ws_bytes"] if kw["ws_bytes"] is not None else bm.bimamba2_workspace_bytes(2, 64, 4)
+    return bm.lib.bimamba2_prefix_state(_byref(inp), _byref(par), kw["batch"], kw["P"], kw["H"], kw["Pd"], kw["N"],
+                                        _byref(st), kw["ws"], wsb, None)
+
+
+def _m2_block(**broken):
+    assert broken, "a validation case must break some argument"
+    kw = dict(state=None, inp=None, G=32, par=None, out=FAKE + 0x50000, out_dtype=bm.BIMAMBA_BF16, batch=2, H=4,
+              Pd=32, N=128, new=None, flags=0, ws=FAKE + 0x400000, ws_bytes=None)
+    kw.update(broken)
+    st = _state2() if kw["state"] is None else kw["state"]
+    inp = _inputs2() if kw["inp"] is None else kw["inp"]
+    par = _params2() if kw["par"] is None else kw["par"]
+    wsb = kw["ws_bytes"] if kw["ws_bytes"] is not None else bm.bimamba2_workspace_bytes(2, 32, 4)
+    new = kw["new"]
+    return bm.lib.bimamba2_block_step(_byref(st), _byref(inp), kw["G"], _byref(par), kw["out"], kw["out_dtype"],
+                                      kw["batch"], kw["H"], kw["Pd"], kw["N"], None if new is None else _byref(new),
+                                      kw["flags"], kw["ws"], wsb, None)
+
+
+def test_mamba2_prefix_and_block_rejects():
+    assert _m2_prefix(inp=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_prefix(P=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_prefix(N=64) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2_prefix(state=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_prefix(state=bm.FwdState2(FAKE + 0x200008, FAKE + 0x300000)) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2_prefix(ws_bytes=16) == bm.BIMAMBA_ERR_WORKSPACE
+    bad = _inputs2()
+    bad.xbc[0] = FAKE + 0x8
+    assert _m2_prefix(inp=bad) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2_block(state=NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_block(G=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_block(out=None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_block(flags=bm.BIMAMBA_NO_TMA) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert _m2_block(flags=3) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_block(new=bm.FwdState2(FAKE + 0x200000, None)) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _m2_block(new=bm.FwdState2(FAKE + 0x200000, FAKE + 0x300008)) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _m2_block(ws=None) == bm.BIMAMBA_ERR_WORKSPACE
+    assert _m2_block(out=FAKE + 0x50008) == bm.BIMAMBA_ERR_MISALIGNED

@@ -167,3 +167,51 @@ def test_workspace_too_small_is_rejected(bm):
     with pytest.raises(bm.BimambaError) as e:
         bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, workspace=ws)
     assert e.value.status == bm.BIMAMBA_ERR_WORKSPACE
+
+
+def _tok(inp, lo, hi):
+    """Tokens [lo, hi) of a Mamba-2 input dict (xbc, dt: [2, b, L, .]; z: [b, L, .])."""
+    return {"xbc": inp["xbc"][:, :, lo:hi].contiguous(), "z": inp["z"][:, lo:hi].contiguous(),
+            "dt": inp["dt"][:, :, lo:hi].contiguous()}
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_block_chain_from_prefix_state(bm, dtype):
+    """Prefix of 100 tokens, then two committed blocks of 37.  Expected values
+    from the layer oracle by the definition of the block step: the forward
+    part is the full-sequence forward over prefix + blocks restricted to the
+    block, the reverse part is the layer on the block alone.  The second
+    block's output checks the first commit's state; the tail is compared
+    bit for bit."""
+    b, H, Pn, G = 2, 3, 100, 37
+    inp, par = W.make_mamba2_case(b, Pn + 2 * G, H, P, N, dtype, seed=80)
+    d, p = U.to_device(inp), U.to_device(par)
+    pre = _tok(d, 0, Pn)
+    S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
+    tol = U.TOL_FP32 if dtype == "fp32" else U.GUARD
+    for k in range(2):
+        lo, hi = Pn + k * G, Pn + (k + 1) * G
+        blk = _tok(d, lo, hi)
+        out = bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=torch.float32,
+                                     new_state=(S, tail))
+        torch.cuda.synchronize()
+        _, yf, _ = oracle.mamba2_layer_fwd(_tok(inp, 0, hi), par, return_dirs=True)
+        bi = _tok(inp, lo, hi)
+        _, _, yr = oracle.mamba2_layer_fwd(bi, par, return_dirs=True)
+        z = bi["z"].double().numpy()
+        want = (yf[:, lo:hi] + yr) * (z / (1.0 + np.exp(-z)))
+        assert U.normwise(U.to_cpu64(out), want) <= tol, k
+        want_tail = inp["xbc"][0, :, hi - 3:hi].double().numpy()
+        assert np.array_equal(U.to_cpu64(tail), want_tail), k
+
+
+def test_block_step_without_commit_leaves_state(bm):
+    inp, par = W.make_mamba2_case(1, 60, 2, P, N, "fp32", seed=81)
+    d, p = U.to_device(inp), U.to_device(par)
+    pre = _tok(d, 0, 40)
+    S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
+    S0, t0 = S.clone(), tail.clone()
+    blk = _tok(d, 40, 60)
+    bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(S, S0) and torch.equal(tail, t0)
