@@ -69,8 +69,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "mamba2", "mamba2_long"],
-                    default="layer")
+    ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "decode_mamba2", "mamba2",
+                                           "mamba2_long"], default="layer")
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
@@ -86,6 +86,8 @@ def workload_of(args) -> W.Workload:
         return W.LAYER_1P3B
     if args.workload == "decode":
         return W.BLOCK_DECODE
+    if args.workload == "decode_mamba2":
+        return W.BLOCK_DECODE_M2
     if args.workload == "mamba2":
         return W.MAMBA2_1P3B
     if args.workload == "mamba2_long":
@@ -586,22 +588,35 @@ def run_decode(args, w, bm, rank, world, dev, stream):
     last step) replays as one CUDA graph."""
     from bidirectional_mamba_denoiser_b200 import decode
     layers, P, G, K = w.extra["layers"], w.extra["prefix"], w.extra["block"], w.extra["steps_per_block"]
+    mixer = w.extra.get("mixer", "mamba1")
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed + rank)
-    params = [W.make_params(w.d_inner, w.d_state, g, dev) for _ in range(layers)]
-    dec = decode.BlockDecoder(params, w.batch, w.d_inner, W.torch_dtype(w.dtype), dev)
-    pre = W.make_inputs(w.batch, P, w.d_inner, w.d_state, w.dtype, g, dev)
+    if mixer == "mamba1":
+        params = [W.make_params(w.d_inner, w.d_state, g, dev) for _ in range(layers)]
+        dec = decode.BlockDecoder(params, w.batch, w.d_inner, W.torch_dtype(w.dtype), dev)
+        pre = W.make_inputs(w.batch, P, w.d_inner, w.d_state, w.dtype, g, dev)
+        pws = None
+    else:
+        H, Pd = w.extra["nheads"], w.extra["headdim"]
+        params = [W.make_mamba2_params(H, Pd, w.d_state, g, dev) for _ in range(layers)]
+        dec = decode.BlockDecoder(params, w.batch, w.d_inner, W.torch_dtype(w.dtype), dev, d_state=w.d_state,
+                                  mixer="mamba2", nheads=H, block_len=G)
+        pre = W.make_mamba2_inputs(w.batch, P, H, Pd, w.d_state, w.dtype, g, dev)
+        pws = torch.empty(bm.bimamba2_workspace_bytes(w.batch, P, H, Pd, w.d_state), device=dev, dtype=torch.uint8)
     torch.cuda.synchronize(dev)
     p0 = torch.cuda.Event(enable_timing=True)
     p1 = torch.cuda.Event(enable_timing=True)
     p0.record(stream)
-    dec.prefill(lambda layer: pre, P, stream=stream)  # one prompt, each layer its own parameters
+    dec.prefill(lambda layer: pre, P, stream=stream, workspace=pws)  # one prompt, each layer its own parameters
     p1.record(stream)
     torch.cuda.synchronize(dev)
     prefill_ms = p0.elapsed_time(p1)
-    del pre
+    del pre, pws
     torch.cuda.empty_cache()
-    pool = [W.make_inputs(w.batch, G, w.d_inner, w.d_state, w.dtype, g, dev) for _ in range(8)]
+    if mixer == "mamba1":
+        pool = [W.make_inputs(w.batch, G, w.d_inner, w.d_state, w.dtype, g, dev) for _ in range(8)]
+    else:
+        pool = [W.make_mamba2_inputs(w.batch, G, H, Pd, w.d_state, w.dtype, g, dev) for _ in range(8)]
     out = torch.empty(layers, w.batch, G, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
 
     def inputs(s, layer):
@@ -621,11 +636,21 @@ def run_decode(args, w, bm, rank, world, dev, stream):
     call_ms = ms / calls
     elems = w.batch * G * w.d_inner
     del graph
+    if mixer == "mamba1":
+        launches = calls
+        roof = roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args))
+        hbm = hbm_fraction(block_bytes(w), call_ms)
+    else:
+        # conv features, forward and reverse scans per call; a commit adds the conv tail
+        launches = reps * (3 * K * layers + layers)
+        roof = roofline_fma(4.0 * Pd * w.d_state * H * 2 * w.batch * G, call_ms, clocks, w.name,
+                            "m2_prep + 2 x m2_scan_kernel (block step)")
+        state = w.batch * H * Pd * w.d_state * 4 + w.batch * 3 * (w.d_inner + 2 * w.d_state) * 2
+        hbm = hbm_fraction(mamba2_bytes(w.batch, G, H, Pd, w.d_state) + state + state // K, call_ms)
     return {
         "value": whole_job_rate(w.batch * G * calls, world, ms_max / 1e3),
-        "ms_per_step": ms_max / (reps * K), "gpu_launches": calls,
-        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args)),
-        "hbm": hbm_fraction(block_bytes(w), call_ms), "clocks": clocks,
+        "ms_per_step": ms_max / (reps * K), "gpu_launches": launches,
+        "roofline": roof, "hbm": hbm, "clocks": clocks,
         "generated_tokens_per_s": round(w.batch * G * reps * world / (ms_max / 1e3), 1),
         "prefill_ms": round(prefill_ms, 3), "layers": layers, "steps_per_block": K,
         "graph": f"one block = {K} steps x {layers} layers = {K * layers} block steps per CUDA graph replay",
@@ -637,7 +662,7 @@ def run_ours(args, rank, world, local):
     w = workload_of(args)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    if args.workload in ("block", "decode"):
+    if args.workload in ("block", "decode", "decode_mamba2"):
         side = torch.cuda.Stream(dev)  # graphs cannot be captured on the legacy default stream
         with torch.cuda.stream(side):
             res = (run_block if args.workload == "block" else run_decode)(args, w, bm, rank, world, dev, side)
@@ -653,7 +678,8 @@ def run_ours(args, rank, world, local):
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                        "d_state": w.d_state, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (rotating input sets)" if args.workload not in ("block", "decode")
+                       "l2": "inputs larger than L2 (rotating input sets)"
+                       if args.workload not in ("block", "decode", "decode_mamba2")
                        else "block inputs rotate over 8 sets (state stays L2-resident, as in decoding)"},
             "roofline": res.pop("roofline"), "cpu_baseline": res.pop("cpu_baseline", None),
             "e2e": res.pop("e2e", None), "gpu_launches": res.pop("gpu_launches"), "clocks": res.pop("clocks"),

@@ -75,6 +75,11 @@ BLOCK_CACHED = Workload("block_cached_b16_P65536_G32_D4096_bf16", 16, 32, 4096, 
 # has 24 blocks), one cache per layer; the per-step shape of BLOCK_CACHED.
 BLOCK_DECODE = Workload("decode_24layers_b16_P65536_G32_K128_D4096_bf16", 16, 32, 4096, 16, "bf16", 7,
                         extra={"layers": 24, "prefix": 65536, "block": 32, "steps_per_block": 128})
+# The same decoding through 24 Mamba-2 mixers at the pages' shape (a shorter
+# prompt: the prefix scan's fp32 workspace grows with its length).
+BLOCK_DECODE_M2 = Workload("decode_mamba2_24layers_b16_P8192_G32_K128_H120x32_N128_bf16", 16, 32, 3840, 128, "bf16",
+                           8, extra={"layers": 24, "prefix": 8192, "block": 32, "steps_per_block": 128,
+                                     "nheads": 120, "headdim": 32, "mixer": "mamba2"})
 DENOISER_SWEEP = {L: Workload(f"denoiser_48x128_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 3,
                               extra={"layers": 48, "steps": 128})
                   for L in (2048, 8192, 32768, 131072)}

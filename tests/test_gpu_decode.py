@@ -88,3 +88,52 @@ def test_block_decoding_matches_oracle_chain(graph):
             assert U.normwise(U.to_cpu64(outs[k][l]), ref) <= U.TOL_FP32, (l, k)
         assert U.normwise(U.to_cpu64(dec.h[l]), h) <= U.TOL_FP32, l
         assert np.array_equal(U.to_cpu64(dec.tail[l]), t), l
+
+
+def test_mamba2_block_decoding_matches_layer_oracle():
+    """Two layers of the Mamba-2 mixer, prefix of 60 tokens, 2 blocks x 2
+    steps of 20: every step's output against the layer oracle by the
+    definition of the block step, the conv tails bit-exact."""
+    layers, b, H, Pn, G, K = 2, 1, 2, 60, 20, 2
+    P, N = 32, 128
+    total = Pn + 2 * K * G
+    cases = [W.make_mamba2_case(b, total, H, P, N, "fp32", seed=95 + i) for i in range(layers)]
+    dev = [(U.to_device(inp), U.to_device(par)) for inp, par in cases]
+    dec = decode.BlockDecoder([p for _, p in dev], batch=b, d_inner=H * P, dtype=torch.float32, device="cuda",
+                              d_state=N, mixer="mamba2", nheads=H, block_len=G)
+
+    def tok(inp, lo, hi):
+        return {"xbc": inp["xbc"][:, :, lo:hi].contiguous(), "z": inp["z"][:, lo:hi].contiguous(),
+                "dt": inp["dt"][:, :, lo:hi].contiguous()}
+
+    dec.prefill(lambda l: tok(dev[l][0], 0, Pn), Pn)
+    out = torch.empty(layers, b, G, H * P, device="cuda")
+    state = {"k": 0}
+
+    def inputs(s, l):
+        lo = Pn + (state["k"] * K + s) * G
+        return tok(dev[l][0], lo, lo + G)
+
+    for k in range(2):
+        state["k"] = k
+        for s in range(K):
+            dec.step(s, K, inputs, out)
+            torch.cuda.synchronize()
+            lo = Pn + (k * K + s) * G
+            for l, (inp, par) in enumerate(cases):
+                # forward from the cache = the full forward over the committed tokens (the prompt
+                # and, of each finished block, its last step's tokens) followed by this block
+                parts = [tok(inp, 0, Pn)] + [tok(inp, Pn + (kk * K + K - 1) * G, Pn + (kk * K + K) * G)
+                                             for kk in range(k)]
+                blk = tok(inp, lo, lo + G)
+                seq = {n: torch.cat([q[n] for q in parts + [blk]], dim=2 if n != "z" else 1)
+                       for n in ("xbc", "z", "dt")}
+                _, yf, _ = oracle.mamba2_layer_fwd(seq, par, return_dirs=True)
+                _, _, yr = oracle.mamba2_layer_fwd(blk, par, return_dirs=True)
+                zz = blk["z"].double().numpy()
+                want = (yf[:, -G:] + yr) * (zz / (1.0 + np.exp(-zz)))
+                assert U.normwise(U.to_cpu64(out[l]), want) <= U.TOL_FP32, (k, s, l)
+    for l, (inp, _) in enumerate(cases):
+        # the last commit was block 1's last step: tokens up to Pn + (K + K - 1) G + G
+        last = Pn + (K + K - 1) * G + G
+        assert np.array_equal(U.to_cpu64(dec.tail[l]), inp["xbc"][0, :, last - 3:last].double().numpy())
