@@ -556,7 +556,7 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     }
     if tensor_path:
         res["roofline"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
-                                          "m2_prep + m2_tiles + 2 x m2_ssd_kernel")
+                                          "m2_prep + 2 x m2_ssd_kernel")
         res["fp32_equivalent"] = roofline_fma(flops, call_ms, clocks, w.name, "recurrence-equivalent")
     else:
         res["roofline"] = roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel")

@@ -43,7 +43,7 @@ constexpr int kSQ = kM2Chunk;               // steps per chunk (= MMA M)
 constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
 // shared memory of m2_ssd_kernel
 constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
-              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90720, kSsdX = 90752, kSsdDL = 100992,
+              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90728, kSsdX = 90752, kSsdDL = 100992,
               kSsdE = 101504, kSsdSmem = 102016;
 constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
 constexpr int kSsdXStride = 40;  // halves per x row in shared memory (80 B: conflict-free 16-byte accesses)
@@ -57,23 +57,14 @@ __device__ __forceinline__ void st_half8(unsigned char* dst, const float* v) {
                    *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
 }
 
-// 32 outputs of one row: 16-byte stores.
-__device__ __forceinline__ void store_row32(float* dst, const float (&v)[32]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+// 4 consecutive outputs: one 16-byte (fp32) or 8-byte (bf16) store.
+__device__ __forceinline__ void store4(float* dst, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
 }
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)[32]) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * u], v[8 * q + 2 * u + 1]);
-            w[u] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&v)[4]) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
 }
 
 // grid (H, batch), block 128, dynamic shared memory kSsdSmem.  DIR 0 stores
@@ -89,7 +80,7 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     unsigned char* sS = sm + kSsdS;
     float* c2s = reinterpret_cast<float*>(sm + kSsdC2);
     float* wtot = reinterpret_cast<float*>(sm + kSsdTot);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSsdBar);  // B tile, C tile, products 1-3, product 4
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSsdBar);  // B tile, C tile, G + Y2, Y1, S
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
     __half* sX = reinterpret_cast<__half*>(sm + kSsdX);  // [128][kSsdXStride]: row t = x of step t (fp16)
     float* sDL = reinterpret_cast<float*>(sm + kSsdDL);  // [128]: step size of step t
@@ -108,7 +99,7 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     const float scale = p.dir_scale[DIR];
 
     if (t == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
         fence_barrier_init();
     }
     if (warp == 0) tmem_alloc<256>(tmem_slot);
@@ -151,11 +142,12 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
 #pragma unroll 1
     for (int k = 0; k < nc; ++k) {
         const uint32_t ph = (uint32_t)(k & 1);
-        // ---- step t of chunk k: x, delta (and the reverse epilogue's y_0, z)
-        const int64_t tok = DIR == 0 ? (int64_t)k * Q + t : L - 1 - (int64_t)k * Q - t;
-        const bool valid = tok >= 0 && tok < L;
-        float x[32], yf[DIR == 1 ? 32 : 1];
-        uint4 zq[DIR == 1 ? 4 : 1];  // the reverse epilogue's z: 32 bf16
+        // ---- step t of chunk k: x and delta
+        float x[32];
+        // the reverse epilogue's y_0 and z in the row-contiguous mapping of the output stores:
+        // row 32 warp + 4 i + lane / 8, channels 4 (lane % 8) .. + 3
+        float4 yfc[DIR == 1 ? 8 : 1];
+        uint2 zc[DIR == 1 ? 8 : 1];
         uint32_t sraw[32];
         tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
         cp_async_wait_all();  // own x row and step size (written and read by this thread only)
@@ -180,6 +172,22 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         }
         if (lane == 31) wtot[warp] = a;
         __syncthreads();
+        // ---- G = C B^T and Y2 = C S_^T need only the tiles and the state of the previous
+        // chunk: they run on the tensor cores while the steps below are computed
+        if (t == 0) {
+            mbar_wait_bounded(bars + 0, ph, p.wait_limit);
+            mbar_wait_bounded(bars + 1, ph, p.wait_limit);
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 0, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aB + ks * 256, 128, 2048), ID_G,
+                         ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_f16(tmem + 160, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aS + ks * 1024, 512, 128), ID_Y,
+                         ks > 0);
+            umma_commit(bars + 2);
+        }
         float base = 0.f;
         for (int w = 0; w < warp; ++w) base += wtot[w];
         const float c = a + base;
@@ -215,44 +223,34 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
             for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(sraw[i]) * f;
             tmem_st32(tmem + 192 + lb, s);
         }
-        if constexpr (DIR == 1) {
-            if (valid) {  // the epilogue's y_0 and z, in flight while the products run
-                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
-                const float4* ysrc = reinterpret_cast<const float4*>(p.YF + o);
+        if constexpr (DIR == 1) {  // in flight while the products run
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 v = ysrc[i];
-                    yf[4 * i] = v.x; yf[4 * i + 1] = v.y; yf[4 * i + 2] = v.z; yf[4 * i + 3] = v.w;
+            for (int i = 0; i < 8; ++i) {
+                const int r = 32 * warp + 4 * i + (lane >> 3);
+                const int64_t tk = L - 1 - (int64_t)k * Q - r;
+                yfc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                zc[i] = make_uint2(0u, 0u);
+                if (tk >= 0) {
+                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
+                    yfc[i] = *reinterpret_cast<const float4*>(p.YF + o);
+                    zc[i] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
                 }
-                const uint4* zsrc = reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.z) + o);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) zq[i] = zsrc[i];
             }
         }
         fence_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
         tmem_fence_after_sync();
-        // ---- G = C B^T, Y2 = C S_^T, S^T += B^T W
+        // ---- S^T += B^T W (onto the decayed state)
         if (t == 0) {
-            mbar_wait_bounded(bars + 0, ph, p.wait_limit);
-            mbar_wait_bounded(bars + 1, ph, p.wait_limit);
-            tmem_fence_after_sync();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 0, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aB + ks * 256, 128, 2048), ID_G,
-                         ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 160, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aS + ks * 1024, 512, 128), ID_Y,
-                         ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 umma_f16(tmem + 192, umma_desc(aB + ks * 4096, 2048, 128), umma_desc(aW + ks * 1024, 512, 128),
                          ID_S, true);
-            umma_commit(bars + 2);
+            umma_commit(bars + 4);
         }
         mbar_wait_bounded(bars + 2, ph, p.wait_limit);
+        mbar_wait_bounded(bars + 4, ph, p.wait_limit);
         tmem_fence_after_sync();
         if (t == 0 && k + 1 < nc && !p.starve) {  // B's buffer is free: next chunk's B tile
             mbar_arrive_expect_tx(bars + 0, kTileBytes);
@@ -325,48 +323,49 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
             mbar_arrive_expect_tx(bars + 1, kTileBytes);
             bulk_g2s(sC, tileb + (int64_t)(k + 1) * 2 * kTileBytes, kTileBytes, bars + 1);
         }
-        // ---- output of step t
+        // ---- output of step t: the row goes through this warp's 32-row staging block (the
+        // delta x / W buffers, free once Y1 is done; 16-byte chunks XOR-swizzled by row) and is
+        // stored row-contiguously, four whole 128-byte rows per warp instruction
         {
             uint32_t r1[32], r2[32];
             tmem_ld32_async(tmem + 128 + lb, r1);
             tmem_ld32_async(tmem + 160 + lb, r2);
             tmem_wait_ld(r1);
             tmem_wait_ld(r2);
-            float y1[32], y2[32];
+            const float e = ex2_approx(c);
+            float4* stg = reinterpret_cast<float4*>(sDX) + warp * 256;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                y1[i] = __uint_as_float(r1[i]);
-                y2[i] = __uint_as_float(r2[i]);
+            for (int q = 0; q < 8; ++q) {
+                float4 v;
+                v.x = (__uint_as_float(r1[4 * q]) + e * __uint_as_float(r2[4 * q]) + Dsk * x[4 * q]) * scale;
+                v.y = (__uint_as_float(r1[4 * q + 1]) + e * __uint_as_float(r2[4 * q + 1]) + Dsk * x[4 * q + 1]) * scale;
+                v.z = (__uint_as_float(r1[4 * q + 2]) + e * __uint_as_float(r2[4 * q + 2]) + Dsk * x[4 * q + 2]) * scale;
+                v.w = (__uint_as_float(r1[4 * q + 3]) + e * __uint_as_float(r2[4 * q + 3]) + Dsk * x[4 * q + 3]) * scale;
+                stg[lane * 8 + (q ^ (lane & 7))] = v;
             }
-            if (valid) {
-                const float e = ex2_approx(c);
-                const int64_t o = ((int64_t)b * L + tok) * HP + (int64_t)h * P;
-                if constexpr (DIR == 0) {
-                    float4* dst = reinterpret_cast<float4*>(p.YF + o);
+            __syncwarp();
+            const int cq = lane & 7;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        float4 v;
-                        v.x = (y1[4 * i] + e * y2[4 * i] + Dsk * x[4 * i]) * scale;
-                        v.y = (y1[4 * i + 1] + e * y2[4 * i + 1] + Dsk * x[4 * i + 1]) * scale;
-                        v.z = (y1[4 * i + 2] + e * y2[4 * i + 2] + Dsk * x[4 * i + 2]) * scale;
-                        v.w = (y1[4 * i + 3] + e * y2[4 * i + 3] + Dsk * x[4 * i + 3]) * scale;
-                        dst[i] = v;
+            for (int i = 0; i < 8; ++i) {
+                const int r = 4 * i + (lane >> 3);
+                const float4 v = stg[r * 8 + (cq ^ (r & 7))];
+                const int step = 32 * warp + r;
+                const int64_t tk = DIR == 0 ? (int64_t)k * Q + step : L - 1 - (int64_t)k * Q - step;
+                if (tk >= 0 && tk < L) {
+                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * cq;
+                    if constexpr (DIR == 0) {
+                        *reinterpret_cast<float4*>(p.YF + o) = v;
+                    } else {
+                        // bf16 -> fp32 is exact: the bf16 bits are the high half
+                        const float z0 = __uint_as_float(zc[i].x << 16), z1 = __uint_as_float(zc[i].x & 0xffff0000u);
+                        const float z2 = __uint_as_float(zc[i].y << 16), z3 = __uint_as_float(zc[i].y & 0xffff0000u);
+                        float ov[4];
+                        ov[0] = (yfc[i].x + v.x) * silu(z0);
+                        ov[1] = (yfc[i].y + v.y) * silu(z1);
+                        ov[2] = (yfc[i].z + v.z) * silu(z2);
+                        ov[3] = (yfc[i].w + v.w) * silu(z3);
+                        store4(static_cast<Tout*>(p.out) + o, ov);
                     }
-                } else {
-                    float ov[32];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t w4[4] = {zq[q].x, zq[q].y, zq[q].z, zq[q].w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            // bf16 -> fp32 is exact: the bf16 bits are the high half
-                            const float z0 = __uint_as_float(w4[u] << 16), z1 = __uint_as_float(w4[u] & 0xffff0000u);
-                            const int i = 8 * q + 2 * u;
-                            ov[i] = (yf[i] + (y1[i] + e * y2[i] + Dsk * x[i]) * scale) * silu(z0);
-                            ov[i + 1] = (yf[i + 1] + (y1[i + 1] + e * y2[i + 1] + Dsk * x[i + 1]) * scale) * silu(z1);
-                        }
-                    }
-                    store_row32(static_cast<Tout*>(p.out) + o, ov);
                 }
             }
         }
