@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         uint2 zc[DIR == 1 ? 8 : 1];
         uint32_t sraw[32];
         tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
+        // the next chunk's tiles into L2 a chunk ahead of their copies into shared memory
+        if (t == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
         cp_async_wait_all();  // own x row and step size (written and read by this thread only)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -278,10 +280,21 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
                         const float cref = c2s[32 * jb];
                         if (!bigspan[jb]) {
                             const float F = ex2_approx(c - cref);
+                            const float2 FF = make_float2(F, F);
+                            const float4* e4 = reinterpret_cast<const float4*>(sE + 32 * jb);
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const int s = 32 * jb + i;
-                                m[i] = s <= t ? __uint_as_float(gr[i]) * (F * sE[s]) : 0.f;
+                            for (int i = 0; i < 32; i += 4) {
+                                const float4 ev = e4[i / 4];
+                                const float2 m01 = mul2(make_float2(__uint_as_float(gr[i]), __uint_as_float(gr[i + 1])),
+                                                        mul2(FF, make_float2(ev.x, ev.y)));
+                                const float2 m23 = mul2(make_float2(__uint_as_float(gr[i + 2]), __uint_as_float(gr[i + 3])),
+                                                        mul2(FF, make_float2(ev.z, ev.w)));
+                                m[i] = m01.x; m[i + 1] = m01.y; m[i + 2] = m23.x; m[i + 3] = m23.y;
+                            }
+                            if (jb == warp) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (i > lane) m[i] = 0.f;
                             }
                         } else {
 #pragma unroll
