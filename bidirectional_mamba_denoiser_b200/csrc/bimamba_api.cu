@@ -739,10 +739,11 @@ bool m2_sizes_ok(int batch, int64_t L, int H) {
     return batch >= 1 && 2 * (int64_t)batch <= 65535 && L >= 1 && L <= (int64_t)1 << 31 && H >= 1 && H <= 65535;
 }
 
-// Chunked dual form on the tensor cores: conv features (x in fp16, C/B as
-// chunk tiles), forward and reverse chunk scans (three launches; when L is
-// not a whole number of chunks, the last chunk's tiles are cleared first so
-// that its rows past the end read zeros).
+// Chunked dual form on the tensor cores: the C/B chunk tiles, then the
+// forward and reverse chunk scans, which compute the x features and step
+// sizes themselves (three launches; when L is not a whole number of chunks,
+// the last chunk's tiles are cleared first so that its rows past the end read
+// zeros).
 template <typename Tin, typename Tout>
 int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
     auto k0 = &bimamba::m2_ssd_kernel<0, Tin, Tout>;
@@ -757,8 +758,8 @@ int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
             cudaSuccess)
             return BIMAMBA_ERR_CUDA;
     }
-    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
-                  (unsigned)(2 * k.batch));
+    const int64_t tok_per_cta = 4 * bimamba::kM2PrepT;
+    const dim3 g1((unsigned)((k.L + tok_per_cta - 1) / tok_per_cta), 1u, (unsigned)(2 * k.batch));
     bimamba::m2_prep_kernel<Tin, true><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
     const dim3 g2((unsigned)k.H, (unsigned)k.batch);
@@ -972,7 +973,6 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
         k.tiles = ws + lay.tiles;
-        k.X16 = reinterpret_cast<__half*>(ws + lay.v);  // in place of the fp32 features
         if (out_bf) return launch_m2_ssd<bf16, bf16>(k, st);
         return launch_m2_ssd<bf16, float>(k, st);
     }

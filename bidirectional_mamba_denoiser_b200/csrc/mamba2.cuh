@@ -68,9 +68,8 @@ struct M2Params {
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
     long long wait_limit;  // SM clocks a wait for a tile or a product may take (tensor-core path)
     int starve;            // test aid (tensor-core path): issue no tile copies, so every wait gives up
-    // tensor-core path: the prep kernel writes x as fp16 ([2][batch][L][H*P], in V's place) and the
-    // fp16 C/B tiles ([2][batch][ceil(L/128)][C | B] x 128 x 128, rows in step order) instead of V
-    __half* X16;
+    // tensor-core path: the prep kernel writes only the fp16 C/B tiles
+    // ([2][batch][ceil(L/128)][C | B] x 128 x 128, rows in step order)
     unsigned char* tiles;
     // block-cached decoding (step-by-step scan): the forward direction's cached
     // state [batch][H][P][N] fp32 and conv tail [batch][3][CH] (xBC rows before
@@ -113,23 +112,25 @@ struct Row8<float> {
 
 constexpr int kM2Chunk = 128;  // steps per chunk of the tensor-core path
 
-// grid (ceil(L / 8), ceil(CH / 1024), 2 * batch), block 128: thread = 8
-// consecutive channels of one direction over 8 tokens; its 11 input rows
-// (8 + the 3-row conv halo) are loaded first, 16 bytes at a time, then the
-// 64 outputs computed and stored as 16-byte rows.  Needs CH % 8 == 0 and
-// 16-byte aligned rows (CH * sizeof(Tin) % 16 == 0, aligned xbc).
-// TILES = false: every channel to V (fp32).  TILES = true (tensor-core
-// path): x channels to X16 (fp16) and B, C channels as fp16 rows of the
-// chunk tiles at the token's step (forward: token t is step t; reverse:
+// Thread = 8 consecutive channels of one direction over 8 tokens; its 11
+// input rows (8 + the 3-row conv halo) are loaded first, 16 bytes at a time,
+// then the 64 outputs computed and stored as 16-byte rows.  Needs CH % 8 == 0
+// and 16-byte aligned rows (CH * sizeof(Tin) % 16 == 0, aligned xbc).
+// TILES = false: grid (ceil(L / 8), ceil(CH / 1024), 2 * batch), block 128;
+// every channel to V (fp32) and the step sizes to DL.  TILES = true
+// (tensor-core path, whose scan kernel computes the x channels and step
+// sizes itself): grid (ceil(L / 32), 1, 2 * batch), block 128 = 4 token
+// groups x the 32 threads of the B and C channels, written as fp16 rows of
+// the chunk tiles at the token's step (forward: token t is step t; reverse:
 // step L-1-t), in the canonical K-major layout.
 template <typename Tin, bool TILES>
 __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     constexpr int TT = kM2PrepT;
-    const int c0 = (blockIdx.y * 128 + threadIdx.x) * 8;
-    const int64_t t0 = (int64_t)blockIdx.x * TT;
-    const int r = blockIdx.z / p.batch, b = blockIdx.z % p.batch;
     const int64_t L = p.L;
     const int CH = p.CH, H = p.H;
+    const int c0 = TILES ? H * kM2P + (int)(threadIdx.x & 31) * 8 : (blockIdx.y * 128 + threadIdx.x) * 8;
+    const int64_t t0 = TILES ? ((int64_t)blockIdx.x * 4 + (threadIdx.x >> 5)) * TT : (int64_t)blockIdx.x * TT;
+    const int r = blockIdx.z / p.batch, b = blockIdx.z % p.batch;
     if (c0 < CH) {
         const Tin* X = static_cast<const Tin*>(p.xbc[r]) + (int64_t)b * L * CH + c0;
         float w[8][4], cb[8];
@@ -182,22 +183,18 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
                 const uint4 q = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
                                            *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
                 const int HP = H * kM2P;
-                if (c0 < HP) {
-                    *reinterpret_cast<uint4*>(p.X16 + (((int64_t)r * p.batch + b) * L + t) * HP + c0) = q;
-                } else {
-                    const bool isB = c0 < HP + kM2N;
-                    const int n0 = c0 - HP - (isB ? 0 : kM2N);
-                    const int64_t step = r == 0 ? t : L - 1 - t;
-                    const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
-                    unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + step / kM2Chunk) *
-                                                     (2 * kM2Chunk * kM2N * 2);
-                    *reinterpret_cast<uint4*>(T + (isB ? kM2Chunk * kM2N * 2 : 0) +
-                                              f16_kmajor((int)(step % kM2Chunk), n0, kM2N)) = q;
-                }
+                const bool isB = c0 < HP + kM2N;
+                const int n0 = c0 - HP - (isB ? 0 : kM2N);
+                const int64_t step = r == 0 ? t : L - 1 - t;
+                const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
+                unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + step / kM2Chunk) *
+                                                 (2 * kM2Chunk * kM2N * 2);
+                *reinterpret_cast<uint4*>(T + (isB ? kM2Chunk * kM2N * 2 : 0) +
+                                          f16_kmajor((int)(step % kM2Chunk), n0, kM2N)) = q;
             }
         }
     }
-    if (blockIdx.y == 0) {
+    if (!TILES && blockIdx.y == 0) {
         for (int h = threadIdx.x; h < H; h += 128) {
             const Tin* DT = static_cast<const Tin*>(p.dt[r]) + (int64_t)b * L * H + h;
             const float bias = p.dt_bias[r * H + h];

@@ -17,15 +17,19 @@
 //   y_t = Y1 + e^{c_t} Y2 + D x_t
 // One CTA = one (head, batch row) in one direction, 128 threads; thread t
 // owns step t of the chunk (TMEM lane t) for the per-step work and state
-// row n = t for the state epilogue.  The chunk's C and B arrive as fp16
-// tiles (in the canonical K-major form, rows in
-// step order so that the reverse direction needs no other code; written by
-// m2_prep_kernel<Tin, true>) by bulk
-// copies; the B tile of the next chunk is fetched as soon as the products
-// that read B are done, the C tile once M (which reuses C's buffer) has been
-// consumed, and each thread's x row and step size of the next chunk by
-// cp.async once this chunk's copies are in registers.  Every mbarrier wait
-// is bounded.
+// row n = t for the state epilogue.  The per-step work starts from the
+// inputs: the head's 32 xBC channels of step t arrive raw by cp.async into a
+// shared-memory ring of 3 + 128 rows (the first three hold the last three
+// steps of the previous chunk, the conv's halo, in step order -- so that the
+// causal forward and the anti-causal reverse conv are the same code), thread
+// t computes the conv + SiLU of its step from rows t..t+3, and its step size
+// softplus(dt + bias) from dt.  The chunk's C and B arrive as fp16 tiles (in
+// the canonical K-major form, rows in step order so that the reverse
+// direction needs no other code; written by m2_prep_kernel<Tin, true>) by
+// bulk copies; the B tile of the next chunk is fetched as soon as the
+// products that read B are done, the C tile once M (which reuses C's
+// buffer) has been consumed, and the next chunk's xBC rows and step sizes
+// once this chunk's conv has read them.  Every mbarrier wait is bounded.
 //
 // Precision: fp16 operands (11-bit significands, like tf32) with fp32
 // accumulation; the carried state stays fp32 in TMEM.  Used for bf16 I/O
@@ -43,10 +47,10 @@ constexpr int kSQ = kM2Chunk;               // steps per chunk (= MMA M)
 constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
 // shared memory of m2_ssd_kernel
 constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
-              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90728, kSsdX = 90752, kSsdDL = 100992,
-              kSsdE = 101504, kSsdSmem = 102016;
+              kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90728, kSsdX = 90752, kSsdE = 101232,
+              kSsdCW = 101744, kSsdCB = 102256, kSsdSmem = 102384;
 constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
-constexpr int kSsdXStride = 40;  // halves per x row in shared memory (80 B: conflict-free 16-byte accesses)
+constexpr int kSsdXStride = 40;  // bf16 per xBC row in shared memory (80 B: conflict-free 16-byte accesses)
 
 // 8 fp32 values -> 8 fp16 in one 16-byte store.
 __device__ __forceinline__ void st_half8(unsigned char* dst, const float* v) {
@@ -72,6 +76,7 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&v)[4]) 
 template <int DIR, typename Tin, typename Tout>
 __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     constexpr int Q = kSQ, P = kM2P;
+    static_assert(sizeof(Tin) == 2, "the dual form reads bf16 inputs");
     extern __shared__ __align__(128) unsigned char sm[];
     unsigned char* sC = sm + kSsdC;
     unsigned char* sB = sm + kSsdB;
@@ -82,9 +87,10 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     float* wtot = reinterpret_cast<float*>(sm + kSsdTot);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kSsdBar);  // B tile, C tile, G + Y2, Y1, S
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
-    __half* sX = reinterpret_cast<__half*>(sm + kSsdX);  // [128][kSsdXStride]: row t = x of step t (fp16)
-    float* sDL = reinterpret_cast<float*>(sm + kSsdDL);  // [128]: step size of step t
-    float* sE = reinterpret_cast<float*>(sm + kSsdE);    // [128]: 2^(c of step 32j - c of step s), s in block j
+    Tin* sX = reinterpret_cast<Tin*>(sm + kSsdX);      // [3 + 128][kSsdXStride]: row 3 + s = xBC of step s
+    float* sE = reinterpret_cast<float*>(sm + kSsdE);  // [128]: 2^(c of step 32j - c of step s), s in block j
+    float4* sCW = reinterpret_cast<float4*>(sm + kSsdCW);  // [32]: conv taps of the head's channels
+    float* sCB = reinterpret_cast<float*>(sm + kSsdCB);    // [32]: conv bias
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int h = blockIdx.x, b = blockIdx.y;
@@ -92,8 +98,10 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     const int H = p.H, HP = H * P;
     const int nc = (int)((L + Q - 1) / Q);
     const unsigned char* tileb = p.tiles + ((int64_t)DIR * p.batch + b) * nc * (2 * kTileBytes);
-    const __half* Vx = p.X16 + ((int64_t)DIR * p.batch + b) * L * HP + (int64_t)h * P;
-    const float* Dh = p.DL + (((int64_t)DIR * p.batch + b) * H + h) * L;
+    const int CH = p.CH;
+    const Tin* Xr = static_cast<const Tin*>(p.xbc[DIR]) + (int64_t)b * L * CH + (int64_t)h * P;
+    const Tin* DTr = static_cast<const Tin*>(p.dt[DIR]) + (int64_t)b * L * H + h;
+    const float bias = p.dt_bias[DIR * H + h];
     const float A2 = p.A[DIR * H + h] * kLog2e;
     const float Dsk = p.Dskip[DIR * H + h];
     const float scale = p.dir_scale[DIR];
@@ -104,6 +112,13 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     }
     if (warp == 0) tmem_alloc<256>(tmem_slot);
     for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sS)[e] = make_uint4(0u, 0u, 0u, 0u);
+    if (t < P) {
+        const int64_t ch = (int64_t)DIR * CH + (int64_t)h * P + t;
+        sCW[t] = reinterpret_cast<const float4*>(p.conv_w)[ch];
+        sCB[t] = p.conv_b ? p.conv_b[ch] : 0.f;
+    }
+    if (t < 3 * 4)  // the first chunk's halo: zeros (before token 0 forward, past token L-1 in reverse)
+        reinterpret_cast<uint4*>(sX + (t >> 2) * kSsdXStride)[t & 3] = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
     tmem_fence_before_sync();
     __syncthreads();
@@ -122,15 +137,19 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         mbar_arrive_expect_tx(bars + 1, kTileBytes);
         bulk_g2s(sC, tileb, kTileBytes, bars + 1);
     }
-    // this thread's x row and step size of chunk kk, into sX / sDL (zeros past either end)
+    // step t of chunk kk: the head's xBC row into row 3 + t of sX (zeros past either end) and
+    // dt into a register, used one chunk later
+    float dt_next = 0.f;
+    bool ok_next = false;
     auto fetch_step = [&](int kk) {
         const int64_t tk = DIR == 0 ? (int64_t)kk * Q + t : L - 1 - (int64_t)kk * Q - t;
         const bool ok = tk >= 0 && tk < L;
-        const __half* src = Vx + (ok ? tk : 0) * HP;
+        const Tin* src = Xr + (ok ? tk : 0) * CH;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cp_async<16>(sX + t * kSsdXStride + 8 * i, src + 8 * i, ok);
-        cp_async<4>(sDL + t, Dh + (ok ? tk : 0), ok);
+        for (int i = 0; i < 4; ++i) cp_async<16>(sX + (3 + t) * kSsdXStride + 8 * i, src + 8 * i, ok);
         cp_async_commit();
+        dt_next = ok ? ldf(DTr, tk * H) : 0.f;
+        ok_next = ok;
     };
     fetch_step(0);
     const uint32_t aC = smem_addr(sC), aB = smem_addr(sB), aDX = smem_addr(sDX), aW = smem_addr(sW),
@@ -150,21 +169,35 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         uint2 zc[DIR == 1 ? 8 : 1];
         uint32_t sraw[32];
         tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
+        const float dtk = dt_next;
+        const bool okk = ok_next;
         // the next chunk's tiles into L2 a chunk ahead of their copies into shared memory
         if (t == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
-        cp_async_wait_all();  // own x row and step size (written and read by this thread only)
+        cp_async_wait_all();
+        __syncthreads();  // every xBC row of the chunk is in shared memory
+        // conv + SiLU of step t: rows t..t+3 hold steps t-3..t, and tap j multiplies step t-3+j in
+        // both directions (the reverse scan's steps run backwards in time)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint4 v = *reinterpret_cast<const uint4*>(sX + t * kSsdXStride + 8 * i);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            uint4 rw[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[u]));
-                x[8 * i + 2 * u] = f.x;
-                x[8 * i + 2 * u + 1] = f.y;
+            for (int j = 0; j < 4; ++j) rw[j] = *reinterpret_cast<const uint4*>(sX + (t + j) * kSsdXStride + 8 * i);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int ch = 8 * i + u;
+                const float4 w = sCW[ch];
+                float a = sCB[ch];
+                const float wj[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t word = u < 2 ? rw[j].x : u < 4 ? rw[j].y : u < 6 ? rw[j].z : rw[j].w;
+                    // bf16 -> fp32 is exact: the bf16 bits are the high half
+                    a = fmaf(wj[j], __uint_as_float((u & 1) ? (word & 0xffff0000u) : (word << 16)), a);
+                }
+                x[ch] = silu(a);
             }
         }
-        const float dl = sDL[t];
+        const float dl = okk ? softplus(dtk + bias) : 0.f;
         // ---- c_t: inclusive scan of delta A (log2 units) over the chunk
         float a = dl * A2;
 #pragma unroll
@@ -174,6 +207,12 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         }
         if (lane == 31) wtot[warp] = a;
         __syncthreads();
+        if (t >= Q - 3) {  // the conv has read every row: the last three steps become the next halo
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                reinterpret_cast<uint4*>(sX + (t + 3 - Q) * kSsdXStride)[i] =
+                    reinterpret_cast<const uint4*>(sX + (t + 3) * kSsdXStride)[i];
+        }
         // ---- G = C B^T and Y2 = C S_^T need only the tiles and the state of the previous
         // chunk: they run on the tensor cores while the steps below are computed
         if (t == 0) {
@@ -215,7 +254,7 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
 #pragma unroll
             for (int pg = 0; pg < 4; ++pg) st_half8(sW + f16_mnmajor(8 * pg, t, P), dx + 8 * pg);
         }
-        if (k + 1 < nc) fetch_step(k + 1);  // x is in registers now
+        if (k + 1 < nc) fetch_step(k + 1);  // the conv and the halo copy are done with this chunk's rows
         // ---- carried state row n = t decays over the whole chunk
         {
             tmem_wait_ld(sraw);
