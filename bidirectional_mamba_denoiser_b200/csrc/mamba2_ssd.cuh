@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSsdTmem);
     Tin* sX = reinterpret_cast<Tin*>(sm + kSsdX);      // [3 + 128][kSsdXStride]: row 3 + s = xBC of step s
     float* sE = reinterpret_cast<float*>(sm + kSsdE);  // [128]: 2^(c of step 32j - c of step s), s in block j
-    float4* sCW = reinterpret_cast<float4*>(sm + kSsdCW);  // [32]: conv taps of the head's channels
+    float* sCW = reinterpret_cast<float*>(sm + kSsdCW);  // [4][32]: conv tap j of the head's channel p
     float* sCB = reinterpret_cast<float*>(sm + kSsdCB);    // [32]: conv bias
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -114,7 +114,11 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sS)[e] = make_uint4(0u, 0u, 0u, 0u);
     if (t < P) {
         const int64_t ch = (int64_t)DIR * CH + (int64_t)h * P + t;
-        sCW[t] = reinterpret_cast<const float4*>(p.conv_w)[ch];
+        const float4 w = reinterpret_cast<const float4*>(p.conv_w)[ch];
+        sCW[t] = w.x;
+        sCW[32 + t] = w.y;
+        sCW[64 + t] = w.z;
+        sCW[96 + t] = w.w;
         sCB[t] = p.conv_b ? p.conv_b[ch] : 0.f;
     }
     if (t < 3 * 4)  // the first chunk's halo: zeros (before token 0 forward, past token L-1 in reverse)
@@ -178,23 +182,31 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         // conv + SiLU of step t: rows t..t+3 hold steps t-3..t, and tap j multiplies step t-3+j in
         // both directions (the reverse scan's steps run backwards in time)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 rw[4];
+        for (int i = 0; i < 4; ++i) {  // channels 8i .. 8i+7, in pairs
+            float2 acc[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) rw[j] = *reinterpret_cast<const uint4*>(sX + (t + j) * kSsdXStride + 8 * i);
+            for (int q = 0; q < 2; ++q) {
+                const float4 cb = reinterpret_cast<const float4*>(sCB)[2 * i + q];
+                acc[2 * q] = make_float2(cb.x, cb.y);
+                acc[2 * q + 1] = make_float2(cb.z, cb.w);
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int ch = 8 * i + u;
-                const float4 w = sCW[ch];
-                float a = sCB[ch];
-                const float wj[4] = {w.x, w.y, w.z, w.w};
+            for (int j = 0; j < 4; ++j) {
+                const uint4 rw = *reinterpret_cast<const uint4*>(sX + (t + j) * kSsdXStride + 8 * i);
+                const uint32_t wd[4] = {rw.x, rw.y, rw.z, rw.w};
+                const float4 w0 = reinterpret_cast<const float4*>(sCW + 32 * j)[2 * i];
+                const float4 w1 = reinterpret_cast<const float4*>(sCW + 32 * j)[2 * i + 1];
+                const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                                      make_float2(w1.z, w1.w)};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t word = u < 2 ? rw[j].x : u < 4 ? rw[j].y : u < 6 ? rw[j].z : rw[j].w;
-                    // bf16 -> fp32 is exact: the bf16 bits are the high half
-                    a = fmaf(wj[j], __uint_as_float((u & 1) ? (word & 0xffff0000u) : (word << 16)), a);
-                }
-                x[ch] = silu(a);
+                for (int u = 0; u < 4; ++u)  // bf16 -> fp32 is exact: the bf16 bits are the high half
+                    acc[u] = fma2(wp[u], make_float2(__uint_as_float(wd[u] << 16), __uint_as_float(wd[u] & 0xffff0000u)),
+                                  acc[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                x[8 * i + 2 * u] = silu(acc[u].x);
+                x[8 * i + 2 * u + 1] = silu(acc[u].y);
             }
         }
         const float dl = okk ? softplus(dtk + bias) : 0.f;
