@@ -70,7 +70,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "decode_mamba2", "mamba2",
-                                           "mamba2_long"], default="layer")
+                                           "mamba2_long", "sharded"], default="layer")
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
@@ -90,6 +90,8 @@ def workload_of(args) -> W.Workload:
         return W.BLOCK_DECODE_M2
     if args.workload == "mamba2":
         return W.MAMBA2_1P3B
+    if args.workload == "sharded":
+        return W.SHARDED_SEQ
     if args.workload == "mamba2_long":
         L = args.L or 16384
         return W.MAMBA2_LONG.get(L) or W.Workload(f"mamba2_b1_L{L}_H120x32_N128_bf16", 1, L, 3840, 128, "bf16",
@@ -657,6 +659,65 @@ def run_decode(args, w, bm, rank, world, dev, stream):
     }
 
 
+def run_sharded(args, w, bm, rank, world, dev, stream):
+    """One sequence of w.L tokens cut into `world` contiguous segments, one
+    per rank: per step each rank runs the sequence-sharded layer on its
+    segment (halo and aggregate all-gathers over NCCL, two carry passes and
+    the carry composition in the CUDA library).  Strong scaling.  Rank 0
+    also times, on its own GPU, one rank's share at 2, 4 and 8 segments (the
+    collectives replaced by stacking), for the projection to more GPUs."""
+    from bidirectional_mamba_denoiser_b200 import sharded as SH
+    flags = flags_of(args, bm)
+    ops = SH.CudaOps(flags)
+    Ls = w.L // world
+    seg, par = W.make_case(w.batch, Ls, w.d_inner, w.d_state, w.dtype, w.seed + rank, device=dev)
+
+    def step(i):
+        if world > 1:
+            SH.sharded_layer_fwd(seg, par, ops=ops)
+        else:
+            SH.emulate_sharded(seg, par, [Ls], ops=ops)
+
+    ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    step_ms = ms / args.steps
+    elems = w.batch * (Ls + 2 * SH.HALO) * w.d_inner
+    res = {
+        "value": whole_job_rate(w.batch * Ls * args.steps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / args.steps, "gpu_launches": 3 * args.steps, "scaling": "strong",
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, step_ms / 2, clocks, w.name, kernel_name(w, args)),
+        "clocks": clocks,
+        "method": "two layer passes per segment (from zero for the aggregates, then from the composed carries)",
+    }
+    del seg
+    torch.cuda.empty_cache()
+    if rank == 0:
+        proj = {}
+        for R in (2, 4, 8):
+            n = w.L // R
+            one, p1 = W.make_case(w.batch, n, w.d_inner, w.d_state, w.dtype, w.seed + 100 + R, device=dev)
+            h_all = torch.zeros(R, 2, w.batch, w.d_inner, w.d_state, device=dev)
+            ds_all = torch.zeros(R, 2, w.batch, w.d_inner, device=dev)
+            edges = torch.stack([SH.halo_edges(one)] * R)
+            mid = R // 2  # a middle segment: both halos and both carries are real
+
+            def share(i):
+                ext = SH.extend_segment(one, *SH.neighbour_halos(edges, mid))
+                SH.pass_from_zero(ext, p1, ops)
+                SH.pass_with_carries(ext, p1, h_all, ds_all, mid, ops)
+
+            k = max(3, args.steps // 4)
+            ms_r, _ = timed(share, k, 2, 1, dev, stream)
+            proj[str(R)] = {"per_rank_ms": round(ms_r / k, 3),
+                            "projected_value": round(w.batch * w.L / (ms_r / k) / 1e3, 3)}
+            del one
+            torch.cuda.empty_cache()
+        res["emulated_ranks"] = proj
+        res["emulated_note"] = ("one rank's segment of L/R tokens timed on this GPU; projected_value = L / that "
+                                "time, before the two all-gathers (a few hundred KB each)")
+    return res
+
+
 def run_ours(args, rank, world, local):
     from bidirectional_mamba_denoiser_b200 import bimamba as bm
     w = workload_of(args)
@@ -668,16 +729,19 @@ def run_ours(args, rank, world, local):
             res = (run_block if args.workload == "block" else run_decode)(args, w, bm, rank, world, dev, side)
     elif args.workload in ("mamba2", "mamba2_long"):
         res = run_mamba2(args, w, bm, rank, world, dev, stream)
+    elif args.workload == "sharded":
+        res = run_sharded(args, w, bm, rank, world, dev, stream)
     else:
         res = run_layer_like(args, w, bm, rank, world, dev, stream)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(res.pop("value"), 4), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(res.pop("ms_per_step"), 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": True, "scaling": res.pop("scaling", "weak"), "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
-                       "d_state": w.d_state, "parallelism": f"replicas{world}",
+                       "d_state": w.d_state,
+                       "parallelism": f"sequence{world}" if args.workload == "sharded" else f"replicas{world}",
                        "l2": "inputs larger than L2 (rotating input sets)"
                        if args.workload not in ("block", "decode", "decode_mamba2")
                        else "block inputs rotate over 8 sets (state stays L2-resident, as in decoding)"},

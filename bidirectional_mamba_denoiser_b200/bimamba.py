@@ -58,6 +58,10 @@ class FwdState(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("conv_x", ctypes.c_void_p)]
 
 
+class Carry(ctypes.Structure):
+    _fields_ = [("h_in", ctypes.c_void_p * 2), ("h_out", ctypes.c_void_p * 2), ("delta_sum", ctypes.c_void_p * 2)]
+
+
 class Params2(ctypes.Structure):
     _fields_ = [("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
                 ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p)]
@@ -83,6 +87,11 @@ def _load():
     lib.bimamba_layer_fwd.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
                                       I, I64, I, I, U, P, SZ, P]
     lib.bimamba_layer_fwd.restype = I
+    lib.bimamba_layer_fwd_carry.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), ctypes.POINTER(Carry), P,
+                                            I, I, I64, I, I, U, P, SZ, P]
+    lib.bimamba_layer_fwd_carry.restype = I
+    lib.bimamba_compose_carries.argtypes = [P, P, ctypes.POINTER(Params), I, I, I, I, I, P, P]
+    lib.bimamba_compose_carries.restype = I
     lib.bimamba_layer_fwd_noalloc.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
                                               I, I64, I, I, U, P]
     lib.bimamba_layer_fwd_noalloc.restype = I
@@ -194,6 +203,58 @@ def bimamba_layer_fwd(x, z, dt, B, C, params: dict, out=None, out_dtype=None, fl
                                _stream(stream))
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba_layer_fwd", rc)
+    return out
+
+
+def _dir_pair(t):
+    """None, a [2, ...] tensor or a (fwd, rev) pair (entries may be None) ->
+    two device pointers (or None)."""
+    if t is None:
+        return None, None
+    if isinstance(t, (tuple, list)):
+        return _ptr(t[0]), _ptr(t[1])
+    return _ptr(t[0]), _ptr(t[1])
+
+
+def bimamba_layer_fwd_carry(x, z, dt, B, C, params: dict, h_in=None, h_out=None, delta_sum=None, out=None,
+                            out_dtype=None, flags: int = 0, workspace=None, stream=None):
+    """bimamba_layer_fwd with scan carries.  h_in, h_out: [2, b, D, 16] fp32
+    (or (fwd, rev) pairs, entries may be None): the states entering / leaving
+    each direction; delta_sum: [2, b, D] fp32, each direction's sum of step
+    sizes.  Returns out [b, L, D]."""
+    b, L, D = x.shape
+    N = (B[0] if isinstance(B, (tuple, list)) else B).shape[-1]
+    if out is None:
+        out = torch.empty(b, L, D, device=x.device, dtype=out_dtype or x.dtype)
+    need = bimamba_workspace_bytes(b, L, D, N, flags)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=x.device, dtype=torch.uint8)
+    inp = make_inputs(x, z, dt, B, C)
+    par = make_params(params)
+    car = Carry()
+    car.h_in[0], car.h_in[1] = _dir_pair(h_in)
+    car.h_out[0], car.h_out[1] = _dir_pair(h_out)
+    car.delta_sum[0], car.delta_sum[1] = _dir_pair(delta_sum)
+    rc = lib.bimamba_layer_fwd_carry(ctypes.byref(inp), ctypes.byref(par), ctypes.byref(car), _ptr(out),
+                                     _dtype_code(out.dtype), b, L, D, N, flags, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_layer_fwd_carry", rc)
+    return out
+
+
+def bimamba_compose_carries(h_out_all, delta_sum_all, params: dict, seg: int, out=None, stream=None):
+    """The carries entering segment ``seg``: h_out_all [nseg, 2, b, D, 16] and
+    delta_sum_all [nseg, 2, b, D] (every segment's run from zero).  Returns
+    h_in [2, b, D, 16] fp32."""
+    nseg, _, b, D, N = h_out_all.shape
+    if out is None:
+        out = torch.empty(2, b, D, N, device=h_out_all.device, dtype=torch.float32)
+    par = make_params(params)
+    rc = lib.bimamba_compose_carries(_ptr(h_out_all), _ptr(delta_sum_all), ctypes.byref(par), nseg, seg, b, D, N,
+                                     _ptr(out), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_compose_carries", rc)
     return out
 
 

@@ -10,6 +10,7 @@
 
 #include "bimamba.h"
 #include "block_fused.cuh"
+#include "carry.cuh"
 #include "layer_fused.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
@@ -256,17 +257,29 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
-template <int G, int T, typename Tin, typename Tout>
+template <int G, int T, typename Tin, typename Tout, bool CARRY = false>
 int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
     bimamba::LayerMaps maps;
     if (!fill_maps<G, T, Tin>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_tma_kernel<G, T, kTWD, kTNS, Tin, Tout>;
+    auto kern = &bimamba::layer_tma_kernel<G, T, kTWD, kTNS, Tin, Tout, CARRY>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
     kern<<<grid, 2 * kTWD * 32, Ge::SMEM, st>>>(maps, k);
     return launch_status();
+}
+
+// With carries: 16-token chunks at 4 lanes per channel, 32 at 8 and 16 (the
+// automatic choice; the chunk flag is not honoured).
+template <typename Tin, typename Tout>
+int layer_tma_carry_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    switch (g) {
+        case 4: return launch_layer_tma<4, 16, Tin, Tout, true>(k, in, st);
+        case 8: return launch_layer_tma<8, 32, Tin, Tout, true>(k, in, st);
+        case 16: return launch_layer_tma<16, 32, Tin, Tout, true>(k, in, st);
+    }
+    return BIMAMBA_ERR_UNSUPPORTED;
 }
 
 template <typename Tin, typename Tout>
@@ -338,12 +351,12 @@ bool fill_fused_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batc
     return ok;
 }
 
-template <int G, typename Tin, typename Tout>
+template <int G, typename Tin, typename Tout, bool CARRY = false>
 int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     using Ge = bimamba::FusedGeo<G, Tin>;
     bimamba::FusedMaps maps;
     if (!fill_fused_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout>;
+    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout, CARRY>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -501,9 +514,14 @@ size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, u
     return (size_t)batch * (size_t)L * (size_t)d_inner * sizeof(float);
 }
 
-int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, void* out,
-                      bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner, int d_state,
-                      unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer, optionally with carries (carry may be null; its pointers may be null).
+int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const bimamba_carry_t* carry,
+                   void* out, bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner, int d_state,
+                   unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
@@ -533,6 +551,17 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
     k.starve = (flags & BIMAMBA_TEST_STARVE) ? 1 : 0;
     k.wait_limit = k.starve ? kStarveWaitCycles : kWaitCycles;
+    bool with_carry = false;
+    if (carry) {
+        for (int r = 0; r < 2; ++r) {
+            if (!aligned(carry->h_in[r], 4) || !aligned(carry->h_out[r], 4) || !aligned(carry->delta_sum[r], 4))
+                return BIMAMBA_ERR_MISALIGNED;
+            k.carry_in[r] = carry->h_in[r];
+            k.carry_out[r] = carry->h_out[r];
+            k.delta_sum[r] = carry->delta_sum[r];
+            with_carry = with_carry || carry->h_in[r] || carry->h_out[r] || carry->delta_sum[r];
+        }
+    }
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
@@ -540,6 +569,12 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     const bool group_ok = forced == 0 || forced == 1 || forced == 2 || forced == 4 || forced == 8;
     if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
         tma_eligible(in, d_inner, true, true)) {
+        if (with_carry) {  // carries: the 2-lane groups (the group size changes only the speed)
+            if (in_bf && out_bf) return launch_fused_layer<2, bf16, bf16, true>(k, in, st);
+            if (in_bf) return launch_fused_layer<2, bf16, float, true>(k, in, st);
+            if (out_bf) return launch_fused_layer<2, float, bf16, true>(k, in, st);
+            return launch_fused_layer<2, float, float, true>(k, in, st);
+        }
         const int gf = pick_group_fused(flags);
         if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, k, in, st);
         if (in_bf) return fused_layer_by_group<bf16, float>(gf, k, in, st);
@@ -548,17 +583,60 @@ int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, voi
     }
     if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
         const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
+        if (with_carry) {
+            if (in_bf && out_bf) return layer_tma_carry_by_lanes<bf16, bf16>(gt, k, in, st);
+            if (in_bf) return layer_tma_carry_by_lanes<bf16, float>(gt, k, in, st);
+            if (out_bf) return layer_tma_carry_by_lanes<float, bf16>(gt, k, in, st);
+            return layer_tma_carry_by_lanes<float, float>(gt, k, in, st);
+        }
         const int tt = pick_chunk_tma(flags, gt);
         if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, tt, k, in, st);
         if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, tt, k, in, st);
         if (out_bf) return layer_tma_by_lanes<float, bf16>(gt, tt, k, in, st);
         return layer_tma_by_lanes<float, float>(gt, tt, k, in, st);
     }
+    if (with_carry) return BIMAMBA_ERR_UNSUPPORTED;  // carries live in the TMA-fed kernel families
     const int g = pick_lanes(2LL * batch * d_inner, flags);
     if (in_bf && out_bf) return layer_by_lanes<bf16, bf16>(g, k, st);
     if (in_bf) return layer_by_lanes<bf16, float>(g, k, st);
     if (out_bf) return layer_by_lanes<float, bf16>(g, k, st);
     return layer_by_lanes<float, float>(g, k, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int bimamba_layer_fwd(const bimamba_inputs_t* in, const bimamba_params_t* p, void* out,
+                      bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner, int d_state,
+                      unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    return layer_fwd_impl(in, p, nullptr, out, out_dtype, batch, L, d_inner, d_state, flags, workspace,
+                          workspace_bytes, cuda_stream);
+}
+
+int bimamba_layer_fwd_carry(const bimamba_inputs_t* in, const bimamba_params_t* p, const bimamba_carry_t* carry,
+                            void* out, bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner, int d_state,
+                            unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    if (!carry) return BIMAMBA_ERR_INVALID_ARG;
+    if (flags & BIMAMBA_NO_TMA) return BIMAMBA_ERR_UNSUPPORTED;
+    return layer_fwd_impl(in, p, carry, out, out_dtype, batch, L, d_inner, d_state, flags, workspace,
+                          workspace_bytes, cuda_stream);
+}
+
+int bimamba_compose_carries(const float* h_out_all, const float* delta_sum_all, const bimamba_params_t* p,
+                            int nseg, int seg, int batch, int d_inner, int d_state, float* h_in, void* cuda_stream) {
+    if (!h_out_all || !delta_sum_all || !h_in || nseg < 1 || seg < 0 || seg >= nseg || batch <= 0 ||
+        batch > kMaxBatch || d_inner <= 0)
+        return BIMAMBA_ERR_INVALID_ARG;
+    if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!p || !p->A) return BIMAMBA_ERR_INVALID_ARG;
+    if (!aligned(h_out_all, 4) || !aligned(delta_sum_all, 4) || !aligned(h_in, 4) || !aligned(p->A, 4))
+        return BIMAMBA_ERR_MISALIGNED;
+    const int64_t n = (int64_t)batch * d_inner * bimamba::kNState;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    bimamba::compose_carries_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(h_out_all, delta_sum_all, p->A,
+                                                                              nseg, seg, batch, d_inner, h_in);
+    return launch_status();
 }
 
 int bimamba_prefix_state(const bimamba_inputs_t* prefix, const bimamba_params_t* p, int batch, int64_t P,

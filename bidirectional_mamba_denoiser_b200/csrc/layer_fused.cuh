@@ -254,11 +254,12 @@ __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
-template <int G, typename Tin, typename Tout, int DIR>
+// CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
+template <int G, typename Tin, typename Tout, int DIR, bool CARRY>
 __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, const KParams& p, unsigned char* base,
                                                       int lane) {
     using Ge = FusedGeo<G, Tin>;
-    constexpr int T = Ge::T, NS = Ge::NS;
+    constexpr int T = Ge::T, NS = Ge::NS, S = Ge::S;
     using Wp = FusedWarp<G, Tin, Tout, DIR, true>;
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
@@ -275,6 +276,18 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
 
     Wp wp;
     wp.setup(p, ct0, lane);
+    const int gbase = ct0 + lane - wp.j;  // first channel of this lane's group
+    if (CARRY && p.carry_in[DIR]) {
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            if (gbase + q < D) {
+                const float* ci = p.carry_in[DIR] + ((int64_t)b * D + gbase + q) * kNState + wp.j * S;
+#pragma unroll
+                for (int s = 0; s < S; ++s) wp.h[q][s] = ci[s];
+            }
+        }
+    }
+    float dsum = 0.f;  // step sizes of the own channel so far
     if (lane == 0)
         for (int i = 0; i < NS && i < nc; ++i)
             fused_issue<G, Tin>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b, p.starve);
@@ -332,6 +345,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         for (int s = 0; s < T; ++s) {
             const bool valid = s >= s_lo && s < s_hi;
             const typename Wp::Elem cur = nxt;
+            if constexpr (CARRY) dsum += cur.dl;  // 0 past the end
             if (s + 1 < T) nxt = wp.element(s + 1, s + 1 >= s_lo && s + 1 < s_hi, xt, dtt);
             float yr;
             if constexpr (G == 1)
@@ -355,9 +369,20 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         __threadfence_block();
         named_bar_sync(1, 64);
     }
+    if (CARRY && p.carry_out[DIR]) {
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            if (gbase + q < D) {
+                float* co = p.carry_out[DIR] + ((int64_t)b * D + gbase + q) * kNState + wp.j * S;
+#pragma unroll
+                for (int s = 0; s < S; ++s) co[s] = wp.h[q][s];
+            }
+        }
+    }
+    if (CARRY && p.delta_sum[DIR] && wp.dvalid) p.delta_sum[DIR][(int64_t)b * D + wp.d] = dsum;
 }
 
-template <int G, typename Tin, typename Tout>
+template <int G, typename Tin, typename Tout, bool CARRY = false>
 __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constant__ FusedMaps maps, const KParams p) {
     using Ge = FusedGeo<G, Tin>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
@@ -371,9 +396,9 @@ __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constan
     }
     __syncthreads();
     if (warp == 0)
-        fused_layer_direction<G, Tin, Tout, 0>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 0, CARRY>(maps, p, base, lane);
     else
-        fused_layer_direction<G, Tin, Tout, 1>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 1, CARRY>(maps, p, base, lane);
 }
 
 // Forward scan over P = p.L tokens from zero: final state and conv tail.

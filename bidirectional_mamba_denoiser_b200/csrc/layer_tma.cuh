@@ -101,8 +101,10 @@ struct TmaWorker {
     float A2[Ge::S];  // A * log2(e) of this lane's states
     float w[4], cb, bias, Dd;
     float h[Ge::S];
+    float dsum;  // step sizes of this lane's steps (j, j+G, ...) so far
 
     __device__ __forceinline__ void setup(const KParams& p, int ct0, int wg, int lane) {
+        dsum = 0.f;
         c = lane % Ge::CPW;
         j = lane / Ge::CPW;
         cc = wg * Ge::CPW + c;
@@ -125,7 +127,9 @@ struct TmaWorker {
     static __device__ __forceinline__ int row_of(int s) { return DIR == 0 ? s : T - 1 - s; }
 
     // conv + SiLU and softplus of this lane's steps j, j+G, ...; steps
-    // outside [s_lo, s_hi) (tokens >= L) become identity steps.
+    // outside [s_lo, s_hi) (tokens >= L) become identity steps.  DSUM: also
+    // add the valid step sizes to dsum.
+    template <bool DSUM = false>
     __device__ __forceinline__ void elements(const Tin* xt, const Tin* dtt, int s_lo, int s_hi, float2* ed2,
                                              float* edu) {
 #pragma unroll 2
@@ -141,6 +145,7 @@ struct TmaWorker {
             const float u = silu(cv);
             const float dl = softplus(ldf(dtt, row_of(s) * Ge::CW + cc) + bias);
             const bool valid = s >= s_lo && s < s_hi;
+            if constexpr (DSUM) dsum += valid ? dl : 0.f;
             ed2[s * Ge::CPW + c] = valid ? make_float2(dl, dl * u) : make_float2(0.f, 0.f);
             edu[s * Ge::CPW + c] = valid ? Dd * u : 0.f;
         }
@@ -204,7 +209,8 @@ __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR>
+// CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY>
 __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
@@ -230,6 +236,11 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
 
     Wk wk;
     wk.setup(p, ct0, wg, lane);
+    if (CARRY && p.carry_in[DIR] && wk.dvalid) {
+        const float* ci = p.carry_in[DIR] + ((int64_t)b * D + wk.d) * kNState + wk.j * Ge::S;
+#pragma unroll
+        for (int q = 0; q < Ge::S; ++q) wk.h[q] = ci[q];
+    }
 
     if (leader) {
         for (int i = 0; i < NS && i < nc; ++i) {
@@ -285,7 +296,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
                                             i2 >= meet, ct0, b, p.starve);
         }
 
-        wk.elements(xt, dtt, s_lo, s_hi, ed2, edu);
+        wk.template elements<CARRY>(xt, dtt, s_lo, s_hi, ed2, edu);
         if (gated) cp_async_wait_all();
         __syncwarp();
 
@@ -312,6 +323,17 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         __threadfence_block();
         named_bar_sync(3, 2 * NWD * 32);
     }
+    if (CARRY && p.carry_out[DIR] && wk.dvalid) {
+        float* co = p.carry_out[DIR] + ((int64_t)b * D + wk.d) * kNState + wk.j * Ge::S;
+#pragma unroll
+        for (int q = 0; q < Ge::S; ++q) co[q] = wk.h[q];
+    }
+    if (CARRY && p.delta_sum[DIR]) {  // the G lanes of a channel are CPW apart
+        float ds = wk.dsum;
+#pragma unroll
+        for (int off = Ge::CPW; off < 32; off <<= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+        if (wk.j == 0 && wk.dvalid) p.delta_sum[DIR][(int64_t)b * D + wk.d] = ds;
+    }
 }
 
 // Resident CTAs per SM the register budget is sized for.
@@ -320,7 +342,7 @@ constexpr int layer_min_blocks() {
     return (T <= 16 || G >= 16) ? 4 : 3;
 }
 
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout>
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false>
 __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     layer_tma_kernel(const __grid_constant__ LayerMaps maps, const KParams p) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
@@ -335,9 +357,9 @@ __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     }
     __syncthreads();
     if (warp < NWD)
-        layer_direction<G, T, NWD, NS, Tin, Tout, 0>(maps, p, base, warp, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY>(maps, p, base, warp, lane);
     else
-        layer_direction<G, T, NWD, NS, Tin, Tout, 1>(maps, p, base, warp - NWD, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY>(maps, p, base, warp - NWD, lane);
 }
 
 // ---------------------------------------------------------------- prefix

@@ -118,6 +118,10 @@ struct KParams {
     const void* tail_in;   // [batch][3][D]    (block step)
     float* h_out;          // [batch][D][16]   (prefix, block commit) or nullptr
     void* tail_out;        // [batch][3][D]    (prefix, block commit) or nullptr
+    // layer with carries (TMA kernel families), each [2] = per direction, nullptr = unused:
+    const float* carry_in[2];  // [batch][D][16]: state entering the direction's first step (else 0)
+    float* carry_out[2];       // [batch][D][16]: state after the direction's last step
+    float* delta_sum[2];       // [batch][D]: sum of the step sizes over the sequence
     int64_t L;             // sequence (or block) length
     int64_t M;             // meeting point of the two directions (layer)
     int D;

@@ -75,6 +75,10 @@ BLOCK_CACHED = Workload("block_cached_b16_P65536_G32_D4096_bf16", 16, 32, 4096, 
 # has 24 blocks), one cache per layer; the per-step shape of BLOCK_CACHED.
 BLOCK_DECODE = Workload("decode_24layers_b16_P65536_G32_K128_D4096_bf16", 16, 32, 4096, 16, "bf16", 7,
                         extra={"layers": 24, "prefix": 65536, "block": 32, "steps_per_block": 128})
+# One sequence of 262,144 tokens cut into contiguous segments, one per GPU
+# (the sequence-sharded scan; total work fixed as the GPU count grows).
+SHARDED_SEQ = Workload("sharded_b1_L262144_D4096_bf16", 1, 262144, 4096, 16, "bf16", 8)
+
 # The same decoding through 24 Mamba-2 mixers at the pages' shape (a shorter
 # prompt: the prefix scan's fp32 workspace grows with its length).
 BLOCK_DECODE_M2 = Workload("decode_mamba2_24layers_b16_P8192_G32_K128_H120x32_N128_bf16", 16, 32, 3840, 128, "bf16",

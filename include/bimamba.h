@@ -134,6 +134,58 @@ int bimamba_layer_fwd(const bimamba_inputs_t *in, const bimamba_params_t *p,
                       int batch, int64_t L, int d_inner, int d_state, unsigned flags,
                       void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* Scan carries of one layer call (a segment of a longer sequence).  Each
+ * [2] is per direction (0 forward, 1 reverse); every pointer may be NULL
+ * (unused).  Device memory, fp32, caller-owned, 4-byte aligned.
+ *   h_in       [batch][d_inner][d_state]: the state entering the direction's
+ *              first step (forward: before token 0; reverse: after token L-1),
+ *              instead of zero
+ *   h_out      [batch][d_inner][d_state]: the state after the direction's last
+ *              step (forward: after token L-1; reverse: after token 0)
+ *   delta_sum  [batch][d_inner]: sum over the L tokens of the direction's step
+ *              size softplus(dt + dt_bias) */
+typedef struct {
+    const float *h_in[2];
+    float *h_out[2];
+    float *delta_sum[2];
+} bimamba_carry_t;
+
+/* bimamba_layer_fwd with carries: the recurrences of §3.2 Eq. (4)-(5) start
+ * from carry->h_in and report their final states and step-size sums.  With
+ * these a sequence cut into segments (one per GPU) is scanned exactly: run
+ * each segment from zero for h_out and delta_sum, compose the carries with
+ * bimamba_compose_carries, run again from them.  The conv still reads zeros
+ * outside [0, L): a segment's inputs are extended by the three neighbouring
+ * tokens on each side with dt = -inf there (step size exactly 0, so those
+ * tokens leave the state unchanged and only feed the conv).  h_in may alias
+ * h_out only if both are the same direction's (each state word is read
+ * before it is written, by the same thread).  Runs the TMA-fed kernel
+ * families only: inputs that bimamba_layer_fwd would run on its fallback
+ * kernels (pointers not 16-byte aligned, d_inner % 8 != 0, or flags with
+ * BIMAMBA_NO_TMA or a fallback lane count) return BIMAMBA_ERR_UNSUPPORTED; with
+ * carries the per-token family runs 2-lane groups and the chunked family its
+ * automatic chunk length, whatever the lane-group and chunk flags ask.
+ * carry == NULL returns BIMAMBA_ERR_INVALID_ARG.  Other arguments, checks
+ * and errors: as bimamba_layer_fwd.  One kernel launch. */
+int bimamba_layer_fwd_carry(const bimamba_inputs_t *in, const bimamba_params_t *p, const bimamba_carry_t *carry,
+                            void *out, bimamba_dtype_t out_dtype,
+                            int batch, int64_t L, int d_inner, int d_state, unsigned flags,
+                            void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/* The carries entering segment `seg` of a sequence cut into nseg segments
+ * (in token order), from every segment's bimamba_layer_fwd_carry run from
+ * zero: since each step is affine in the state, a segment run from state h
+ * ends in exp(A * delta_sum) * h + h_out.
+ *   h_out_all      [nseg][2][batch][d_inner][d_state]: segment j's h_out[0], h_out[1]
+ *   delta_sum_all  [nseg][2][batch][d_inner]: segment j's delta_sum[0], delta_sum[1]
+ *   p              only p->A is read
+ *   h_in           [2][batch][d_inner][d_state] out: forward = fold of segments
+ *                  0..seg-1, reverse = fold of segments nseg-1..seg+1 (zero at the ends)
+ * Device pointers, fp32, 4-byte aligned; h_in must not alias the inputs.
+ * One kernel launch. */
+int bimamba_compose_carries(const float *h_out_all, const float *delta_sum_all, const bimamba_params_t *p,
+                            int nseg, int seg, int batch, int d_inner, int d_state, float *h_in, void *cuda_stream);
+
 /* The full layer for callers that cannot allocate device memory -- a plugin
  * inside a host application that owns all GPU memory, or a caller that
  * reaches this library only through the C ABI with no CUDA allocator -- and

@@ -316,3 +316,49 @@ def test_mamba2_prefix_and_block_rejects():
     assert _m2_block(new=bm.FwdState2(FAKE + 0x200000, FAKE + 0x300008)) == bm.BIMAMBA_ERR_MISALIGNED
     assert _m2_block(ws=None) == bm.BIMAMBA_ERR_WORKSPACE
     assert _m2_block(out=FAKE + 0x50008) == bm.BIMAMBA_ERR_MISALIGNED
+
+
+def _carry(**ptrs):
+    c = bm.Carry()
+    for name, (a, b) in ptrs.items():
+        getattr(c, name)[0], getattr(c, name)[1] = a, b
+    return c
+
+
+def _layer_carry(carry, flags=0, **kw):
+    inp, par = _inputs(), _params()
+    ws_bytes = bm.bimamba_workspace_bytes(2, 64, 32)
+    return bm.lib.bimamba_layer_fwd_carry(ctypes.byref(inp), ctypes.byref(par), _byref(carry), FAKE + 0x20000,
+                                          bm.BIMAMBA_BF16, kw.get("batch", 2), 64, 32, 16, flags, FAKE + 0x30000,
+                                          ws_bytes, None)
+
+
+def test_layer_carry_rejects():
+    # no carry struct; NO_TMA (carries live in the TMA-fed kernels); a misaligned carry pointer;
+    # the layer's own checks still apply (batch 0)
+    assert _layer_carry(NULL) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert _layer_carry(_carry(h_out=(FAKE + 0x40000, None)), flags=bm.BIMAMBA_NO_TMA) == bm.BIMAMBA_ERR_UNSUPPORTED
+    for name in ("h_in", "h_out", "delta_sum"):
+        assert _layer_carry(_carry(**{name: (None, FAKE + 0x40002)})) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _layer_carry(_carry(h_out=(FAKE + 0x40000, None)), batch=0) == bm.BIMAMBA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(h_all=None), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(ds_all=None), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(h_in=None), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(nseg=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(seg=-1), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(seg=4), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(batch=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(D=0), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(N=8), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(par=NULL), bm.BIMAMBA_ERR_INVALID_ARG),
+    (dict(h_in=FAKE + 0x50002), bm.BIMAMBA_ERR_MISALIGNED),
+])
+def test_compose_carries_rejects(kw, status):
+    a = dict(h_all=FAKE, ds_all=FAKE + 0x1000, par=_params(), nseg=4, seg=1, batch=2, D=32, N=16,
+             h_in=FAKE + 0x50000)
+    a.update(kw)
+    assert bm.lib.bimamba_compose_carries(a["h_all"], a["ds_all"], _byref(a["par"]), a["nseg"], a["seg"],
+                                          a["batch"], a["D"], a["N"], a["h_in"], None) == status
