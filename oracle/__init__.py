@@ -262,3 +262,6 @@ def mamba2_layer_fwd(inp: dict, params: dict, flags: int = 0, return_dirs: bool 
     if rc != 0:
         raise RuntimeError("oracle2_layer_fwd failed")
     return (out, yf, yr) if return_dirs else out
+
+
+from .proj import adaln, in_proj, out_proj  # noqa: E402  (the layer's neighbours, plain numpy)
