@@ -70,7 +70,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "decode_mamba2", "mamba2",
-                                           "mamba2_long", "sharded"], default="layer")
+                                           "mamba2_long", "sharded", "proj"], default="layer")
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
@@ -92,6 +92,8 @@ def workload_of(args) -> W.Workload:
         return W.MAMBA2_1P3B
     if args.workload == "sharded":
         return W.SHARDED_SEQ
+    if args.workload == "proj":
+        return W.PROJ_1P3B
     if args.workload == "mamba2_long":
         L = args.L or 16384
         return W.MAMBA2_LONG.get(L) or W.Workload(f"mamba2_b1_L{L}_H120x32_N128_bf16", 1, L, 3840, 128, "bf16",
@@ -718,6 +720,54 @@ def run_sharded(args, w, bm, rank, world, dev, stream):
     return res
 
 
+def run_proj(args, w, bm, rank, world, dev, stream):
+    """The layer's neighbours at the 1.3B shape: AdaLN of the hidden states,
+    the input projection into the layer's inputs, and the output projection
+    of a layer output, per step.  Two input sets alternate (each above L2).
+    Each op is also timed alone, for its own roofline."""
+    dm, D = w.extra["d_model"], w.d_inner
+    M = w.batch * w.L
+    cases = [W.make_proj_case(w.batch, w.L, dm, D, w.d_state, w.seed + 10 * i + rank, device=dev) for i in range(2)]
+    a = torch.empty(w.batch, w.L, dm, device=dev, dtype=torch.bfloat16)
+    ins = bm.bimamba_in_proj(a, cases[0]["w_in"], D)
+    o = torch.empty(w.batch, w.L, dm, device=dev, dtype=torch.bfloat16)
+
+    def op_adaln(i):
+        c = cases[i & 1]
+        bm.bimamba_adaln(c["h"], c["gamma"], c["beta"], out=a, stream=stream)
+
+    def op_in(i):
+        bm.bimamba_in_proj(a, cases[i & 1]["w_in"], D, out=ins, stream=stream)
+
+    def op_out(i):
+        c = cases[i & 1]
+        bm.bimamba_out_proj(c["y"], c["w_out"], out=o, stream=stream)
+
+    def step(i):
+        op_adaln(i)
+        op_in(i)
+        op_out(i)
+
+    ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    per = {}
+    for name, fn in (("adaln", op_adaln), ("in_proj", op_in), ("out_proj", op_out)):
+        t, _ = timed(fn, args.steps, args.warmup, 1, dev, stream)
+        per[name] = t / args.steps
+    f_in = 2.0 * M * dm * (4 * D + 4 * w.d_state)
+    f_out = 2.0 * M * D * dm
+    roof = roofline_tensor(f_in, per["in_proj"], w.name, "gemm_bf16_kernel (input projection)")
+    adaln_bytes = M * dm * 2 * 2
+    return {
+        "value": whole_job_rate(M * args.steps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / args.steps, "gpu_launches": 3 * args.steps, "roofline": roof, "clocks": clocks,
+        "kernels_ms": {k: round(v, 4) for k, v in per.items()},
+        "out_proj_roofline": roofline_tensor(f_out, per["out_proj"], w.name, "gemm_bf16_kernel (output projection)"),
+        "adaln_hbm": hbm_fraction(adaln_bytes, per["adaln"]),
+        "note": "value = tokens through AdaLN + input projection + output projection per second",
+    }
+
+
 def run_ours(args, rank, world, local):
     from bidirectional_mamba_denoiser_b200 import bimamba as bm
     w = workload_of(args)
@@ -731,6 +781,8 @@ def run_ours(args, rank, world, local):
         res = run_mamba2(args, w, bm, rank, world, dev, stream)
     elif args.workload == "sharded":
         res = run_sharded(args, w, bm, rank, world, dev, stream)
+    elif args.workload == "proj":
+        res = run_proj(args, w, bm, rank, world, dev, stream)
     else:
         res = run_layer_like(args, w, bm, rank, world, dev, stream)
     if rank == 0:

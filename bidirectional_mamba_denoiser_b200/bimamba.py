@@ -92,6 +92,12 @@ def _load():
     lib.bimamba_layer_fwd_carry.restype = I
     lib.bimamba_compose_carries.argtypes = [P, P, ctypes.POINTER(Params), I, I, I, I, I, P, P]
     lib.bimamba_compose_carries.restype = I
+    lib.bimamba_adaln.argtypes = [P, P, P, P, I, I64, I, ctypes.c_float, P]
+    lib.bimamba_adaln.restype = I
+    lib.bimamba_in_proj.argtypes = [P, P, I, I64, I, I, I, P, P, P, P, P, P]
+    lib.bimamba_in_proj.restype = I
+    lib.bimamba_out_proj.argtypes = [P, P, I, I64, I, I, P, P]
+    lib.bimamba_out_proj.restype = I
     lib.bimamba_layer_fwd_noalloc.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), P, I,
                                               I, I64, I, I, U, P]
     lib.bimamba_layer_fwd_noalloc.restype = I
@@ -255,6 +261,48 @@ def bimamba_compose_carries(h_out_all, delta_sum_all, params: dict, seg: int, ou
                                      _ptr(out), _stream(stream))
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba_compose_carries", rc)
+    return out
+
+
+def bimamba_adaln(x, gamma, beta, eps: float = 1e-5, out=None, stream=None):
+    """AdaLN: gamma[b] * (x - mean) / sqrt(var + eps) + beta[b] per token row.
+    x [b, L, d] bf16; gamma, beta [b, d] fp32.  Returns [b, L, d] bf16."""
+    b, L, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    rc = lib.bimamba_adaln(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(out), b, L, d, eps, _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_adaln", rc)
+    return out
+
+
+def bimamba_in_proj(a, w_in, d_inner: int, d_state: int = D_STATE, out: dict | None = None, stream=None) -> dict:
+    """Input projection into the layer's input arrays: a [b, L, d_model] bf16,
+    w_in [4 d_inner + 4 d_state, d_model] bf16.  Returns {"x", "z" [b, L, D];
+    "dt" [2, b, L, D]; "B", "C" [2, b, L, d_state]} (bf16)."""
+    b, L, dm = a.shape
+    if out is None:
+        kw = dict(device=a.device, dtype=a.dtype)
+        out = {"x": torch.empty(b, L, d_inner, **kw), "z": torch.empty(b, L, d_inner, **kw),
+               "dt": torch.empty(2, b, L, d_inner, **kw), "B": torch.empty(2, b, L, d_state, **kw),
+               "C": torch.empty(2, b, L, d_state, **kw)}
+    rc = lib.bimamba_in_proj(_ptr(a), _ptr(w_in), b, L, dm, d_inner, d_state, _ptr(out["x"]), _ptr(out["z"]),
+                             _ptr(out["dt"]), _ptr(out["B"]), _ptr(out["C"]), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_in_proj", rc)
+    return out
+
+
+def bimamba_out_proj(y, w_out, out=None, stream=None):
+    """Output projection: y [b, L, d_inner] bf16, w_out [d_model, d_inner]
+    bf16.  Returns [b, L, d_model] bf16."""
+    b, L, D = y.shape
+    dm = w_out.shape[0]
+    if out is None:
+        out = torch.empty(b, L, dm, device=y.device, dtype=y.dtype)
+    rc = lib.bimamba_out_proj(_ptr(y), _ptr(w_out), b, L, D, dm, _ptr(out), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_out_proj", rc)
     return out
 
 

@@ -15,6 +15,7 @@
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
 #include "mamba2_ssd.cuh"
+#include "proj.cuh"
 #include "scan_kernels.cuh"
 
 namespace {
@@ -1061,3 +1062,99 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
 }
 
 }  // extern "C"
+
+// ---- the layer's neighbours: AdaLN and the projections
+
+namespace {
+
+// 2-D map over a row-major bf16 [rows][inner] matrix, box {64, box_rows},
+// 128-byte swizzle (the layout the GEMM's descriptors expect).
+bool map2d_sw128(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)bimamba::kGemmBK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_gemm(const void* a, const void* w, const bimamba::GemmParams& gp, cudaStream_t st) {
+    CUtensorMap ma, mw;
+    if (!map2d_sw128(&ma, a, (uint64_t)gp.K, (uint64_t)gp.M, bimamba::kGemmBM) ||
+        !map2d_sw128(&mw, w, (uint64_t)gp.K, (uint64_t)gp.N, bimamba::kGemmBN))
+        return BIMAMBA_ERR_CUDA;
+    const void* fn = reinterpret_cast<const void*>(&bimamba::gemm_bf16_kernel);
+    int rc = ensure_smem(fn, bimamba::kGemmSmem);
+    if (rc) return rc;
+    const dim3 grid((unsigned)((gp.N + bimamba::kGemmBN - 1) / bimamba::kGemmBN),
+                    (unsigned)((gp.M + bimamba::kGemmBM - 1) / bimamba::kGemmBM));
+    bimamba::gemm_bf16_kernel<<<grid, 128, bimamba::kGemmSmem, st>>>(ma, mw, gp);
+    return launch_status();
+}
+
+// rows = batch * L within the GEMM grid's reach (ceil(rows / 128) <= 65535).
+bool proj_rows_ok(int batch, int64_t L) {
+    return batch >= 1 && batch <= kMaxBatch && L >= 1 && (int64_t)batch * L <= (int64_t)65535 * bimamba::kGemmBM;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bimamba_adaln(const void* x, const float* gamma, const float* beta, void* out, int batch, int64_t L, int d,
+                  float eps, void* cuda_stream) {
+    if (!x || !gamma || !beta || !out || batch < 1 || batch > kMaxBatch || L < 1 || d < 8 || !(eps > 0.f) ||
+        (int64_t)batch * L > 0x7fffffffLL)
+        return BIMAMBA_ERR_INVALID_ARG;
+    if (d % 8) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gamma, 4) || !aligned(beta, 4)) return BIMAMBA_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    bimamba::adaln_kernel<<<(unsigned)((int64_t)batch * L), 256, 0, st>>>(
+        static_cast<const bf16*>(x), gamma, beta, static_cast<bf16*>(out), L, d, eps);
+    return launch_status();
+}
+
+int bimamba_in_proj(const void* a, const void* w_in, int batch, int64_t L, int d_model, int d_inner, int d_state,
+                    void* x, void* z, void* dt, void* B, void* C, void* cuda_stream) {
+    if (!a || !w_in || !x || !z || !dt || !B || !C || !proj_rows_ok(batch, L) || d_model < 1 || d_inner < 1)
+        return BIMAMBA_ERR_INVALID_ARG;
+    if (d_state != bimamba::kNState || d_model % bimamba::kGemmBK || d_inner % 8) return BIMAMBA_ERR_UNSUPPORTED;
+    for (const void* q : {a, w_in, (const void*)x, (const void*)z, (const void*)dt, (const void*)B, (const void*)C})
+        if (!aligned(q, 16)) return BIMAMBA_ERR_MISALIGNED;
+    bimamba::GemmParams gp = {};
+    gp.M = (int)((int64_t)batch * L);
+    gp.N = 4 * d_inner + 4 * d_state;
+    gp.K = d_model;
+    gp.scatter = 1;
+    gp.x = static_cast<bf16*>(x);
+    gp.z = static_cast<bf16*>(z);
+    gp.dt = static_cast<bf16*>(dt);
+    gp.Bm = static_cast<bf16*>(B);
+    gp.Cm = static_cast<bf16*>(C);
+    gp.D = d_inner;
+    gp.Ns = d_state;
+    gp.wait_limit = kWaitCycles;
+    return launch_gemm(a, w_in, gp, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int bimamba_out_proj(const void* y, const void* w_out, int batch, int64_t L, int d_inner, int d_model, void* out,
+                     void* cuda_stream) {
+    if (!y || !w_out || !out || !proj_rows_ok(batch, L) || d_model < 1 || d_inner < 1)
+        return BIMAMBA_ERR_INVALID_ARG;
+    if (d_inner % bimamba::kGemmBK || d_model % 8) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!aligned(y, 16) || !aligned(w_out, 16) || !aligned(out, 16)) return BIMAMBA_ERR_MISALIGNED;
+    bimamba::GemmParams gp = {};
+    gp.M = (int)((int64_t)batch * L);
+    gp.N = d_model;
+    gp.K = d_inner;
+    gp.scatter = 0;
+    gp.C = static_cast<bf16*>(out);
+    gp.wait_limit = kWaitCycles;
+    return launch_gemm(y, w_out, gp, static_cast<cudaStream_t>(cuda_stream));
+}
+
+}  // extern "C"
+

@@ -1,0 +1,214 @@
+// proj.cuh -- the mixer layer's neighbours ("DiffuMamba: High-Throughput
+// Diffusion LMs with Mamba Backbone", App. A.1 Eq. (10)-(11) and Table 12):
+// the timestep-conditioned AdaLN in front of the mixer, the input projection
+// that produces the layer's inputs, and the output projection after it.
+//
+// AdaLN (Eq. (10)): out = gamma_b * (x - mu(x)) / sigma(x) + beta_b per token
+// row, gamma and beta per batch row, sigma = sqrt(var + eps); one CTA per
+// row, fp32 statistics (two passes over the row: mean, then centred squares).
+//
+// The projections are one GEMM kernel on the tcgen05 tensor cores:
+// C[m][n] = sum_k A[m][k] W[n][k], bf16 operands, fp32 accumulation in TMEM,
+// bf16 results.  A CTA computes a 128 x 256 tile: a producer thread streams
+// 128 x 64 A and 256 x 64 W tiles by TMA (128-byte swizzle) through a
+// 4-stage shared-memory ring, one thread issues the MMAs of each stage
+// (4 x K = 16) and frees the stage by tcgen05.commit, and after the last
+// stage the four warps read the accumulator rows of their TMEM lanes and
+// store them.  Every wait is bounded.  The epilogue either writes C as is
+// (output projection: A is the layer's gated output) or scatters each 8-column
+// group straight into the mixer's input arrays (input projection: columns
+// [x | z | dt_f | dt_b | B_f | C_f | B_b | C_b]), so the layer reads them with
+// no split or copy in between.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "tcgen05_util.cuh"
+#include "tma_util.cuh"
+
+namespace bimamba {
+
+// ---------------------------------------------------------------- AdaLN
+
+// grid (rows), block 256; d % 8 == 0; rows = batch * L, batch row = row / L.
+__global__ void __launch_bounds__(256) adaln_kernel(const __nv_bfloat16* x, const float* gamma, const float* beta,
+                                                    __nv_bfloat16* out, int64_t L, int d, float eps) {
+    __shared__ float red[8];
+    const int64_t row = blockIdx.x;
+    const int b = (int)(row / L);
+    const __nv_bfloat16* xr = x + row * d;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    auto block_sum = [&](float v) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        __syncthreads();  // red is free again
+        if (lane == 0) red[warp] = v;
+        __syncthreads();
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += red[w];
+        return s;
+    };
+    auto load8 = [&](int c, float (&v)[8]) {
+        const uint4 q = *reinterpret_cast<const uint4*>(xr + c);
+        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
+            v[2 * u] = __uint_as_float(w4[u] << 16);
+            v[2 * u + 1] = __uint_as_float(w4[u] & 0xffff0000u);
+        }
+    };
+    float s = 0.f;
+    for (int c = 8 * t; c < d; c += 8 * 256) {
+        float v[8];
+        load8(c, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += v[u];
+    }
+    const float mu = block_sum(s) / (float)d;
+    float q = 0.f;
+    for (int c = 8 * t; c < d; c += 8 * 256) {
+        float v[8];
+        load8(c, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) q = fmaf(v[u] - mu, v[u] - mu, q);
+    }
+    const float rstd = rsqrtf(block_sum(q) / (float)d + eps);
+    const float* g = gamma + (int64_t)b * d;
+    const float* be = beta + (int64_t)b * d;
+    for (int c = 8 * t; c < d; c += 8 * 256) {
+        float v[8];
+        load8(c, v);
+        uint32_t w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float a0 = fmaf(g[c + 2 * u], (v[2 * u] - mu) * rstd, be[c + 2 * u]);
+            const float a1 = fmaf(g[c + 2 * u + 1], (v[2 * u + 1] - mu) * rstd, be[c + 2 * u + 1]);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+            w4[u] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(out + row * d + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+}
+
+// ---------------------------------------------------------------- GEMM
+
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmATile = kGemmBM * kGemmBK * 2;    // 16 KB
+constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;    // 32 KB
+constexpr int kGemmStage = kGemmATile + kGemmBTile;  // 48 KB
+constexpr int kGemmBarOff = kGemmStages * kGemmStage;
+constexpr int kGemmSmem = kGemmBarOff + 128 + 1024;  // barriers + TMEM slot, and 1024-byte alignment slack
+
+struct GemmParams {
+    int M, N, K;
+    int scatter;              // 0: C [M][N]; 1: the mixer's input arrays
+    __nv_bfloat16* C;
+    // scatter: x, z [M][D]; dt [2][M][D]; Bm, Cm [2][M][Ns]
+    __nv_bfloat16 *x, *z, *dt, *Bm, *Cm;
+    int D, Ns;
+    long long wait_limit;
+};
+
+// 8 results (columns n .. n+7 of row m) to their place.
+__device__ __forceinline__ void gemm_store8(const GemmParams& p, int m, int n, const float* v) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+        w4[u] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    __nv_bfloat16* dst;
+    if (!p.scatter) {
+        dst = p.C + (int64_t)m * p.N + n;
+    } else {
+        const int64_t M = p.M, D = p.D, Ns = p.Ns;
+        if (n < 2 * D) {
+            dst = (n < D ? p.x + m * D + n : p.z + m * D + (n - D));
+        } else if (n < 4 * D) {
+            const int r = n < 3 * D ? 0 : 1;
+            dst = p.dt + (r * M + m) * D + (n - (2 + r) * D);
+        } else {
+            const int j = n - 4 * (int)D, seg = j / (int)Ns, c = j % (int)Ns;  // B_f, C_f, B_b, C_b
+            __nv_bfloat16* base = (seg & 1) ? p.Cm : p.Bm;
+            dst = base + ((int64_t)(seg >> 1) * M + m) * Ns + c;
+        }
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+}
+
+// grid (ceil(N / 256), ceil(M / 128)), block 128, dynamic shared memory kGemmSmem.
+// mapA: [M][K] bf16, box {64, 128}; mapW: [N][K] bf16, box {64, 256}; both
+// 128-byte swizzled.  K % 64 == 0; N % 8 == 0.
+__global__ void __launch_bounds__(128, 1) gemm_bf16_kernel(const __grid_constant__ CUtensorMap mapA,
+                                                           const __grid_constant__ CUtensorMap mapW,
+                                                           const GemmParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + kGemmBarOff);
+    uint64_t* empty = full + kGemmStages;
+    uint64_t* done = empty + kGemmStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
+    const int nk = p.K / kGemmBK;
+
+    if (t == 0) {
+        for (int i = 0; i < 2 * kGemmStages + 1; ++i) mbar_init(full + i, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc<256>(tmem_slot);
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (t == 0) {  // producer: A and W tiles of each K step into the ring
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % kGemmStages;
+            if (kt >= kGemmStages) mbar_wait_bounded(empty + s, (uint32_t)(((kt / kGemmStages) - 1) & 1), p.wait_limit);
+            unsigned char* st = base + s * kGemmStage;
+            mbar_arrive_expect_tx(full + s, kGemmStage);
+            tma_load_2d(st, &mapA, full + s, kt * kGemmBK, m0);
+            tma_load_2d(st + kGemmATile, &mapW, full + s, kt * kGemmBK, n0);
+        }
+    } else if (t == 32) {  // MMA issuer
+        constexpr uint32_t idesc = umma_idesc_bf16(kGemmBM, kGemmBN);
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % kGemmStages;
+            mbar_wait_bounded(full + s, (uint32_t)((kt / kGemmStages) & 1), p.wait_limit);
+            tmem_fence_after_sync();
+            const uint32_t a = smem_addr(base + s * kGemmStage), w = a + kGemmATile;
+#pragma unroll
+            for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                umma_f16(tmem, umma_desc_sw128(a + 32 * kk), umma_desc_sw128(w + 32 * kk), idesc, kt > 0 || kk > 0);
+            umma_commit(empty + s);  // the stage is free once these products have read it
+        }
+        umma_commit(done);
+    }
+    __syncwarp();
+    // epilogue: warp w owns accumulator rows 32w .. 32w+31 (its TMEM lanes)
+    mbar_wait_bounded(done, 0, p.wait_limit);
+    tmem_fence_after_sync();
+    const int m = m0 + warp * 32 + lane;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+    for (int c = 0; c < kGemmBN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lb + 32 * c, v);
+        if (m < p.M) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int n = n0 + 32 * c + 8 * g;
+                if (n < p.N) gemm_store8(p, m, n, v + 8 * g);
+            }
+        }
+    }
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc<256>(tmem);
+}
+
+}  // namespace bimamba

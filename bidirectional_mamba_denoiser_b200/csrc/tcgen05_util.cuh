@@ -37,6 +37,26 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// Descriptor of a K-major operand tile in the 128-byte swizzled layout that a
+// TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes (rows of 64 bf16 = 128 B,
+// 16-byte chunk c of row r at c ^ (r % 8), 8-row groups 1024 B apart; the
+// tile 1024-byte aligned).  Moving 16 elements along K inside the 128-byte
+// row adds 32 B to the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;             // leading byte offset: unused for a swizzled K-major tile
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: next group of 8 rows
+    d |= (uint64_t)1 << 46;             // descriptor version
+    d |= (uint64_t)2 << 61;             // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major), fp32 D.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor of kind::f16 with fp16 A and B, fp32 D.
 __host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                               // D format f32

@@ -74,6 +74,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 2-D tiled TMA load into shared memory, completing on `bar` (transaction
+// bytes); c0 is the inner (contiguous) coordinate.  A box reaching outside the
+// tensor reads zeros there.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
 // Asynchronous global -> shared copy of BYTES (4, 8 or 16; both addresses
 // aligned to BYTES); with pred false nothing is read and zeros are written.
 template <int BYTES>

@@ -75,6 +75,31 @@ BLOCK_CACHED = Workload("block_cached_b16_P65536_G32_D4096_bf16", 16, 32, 4096, 
 # has 24 blocks), one cache per layer; the per-step shape of BLOCK_CACHED.
 BLOCK_DECODE = Workload("decode_24layers_b16_P65536_G32_K128_D4096_bf16", 16, 32, 4096, 16, "bf16", 7,
                         extra={"layers": 24, "prefix": 65536, "block": 32, "steps_per_block": 128})
+def make_proj_case(batch: int, L: int, d_model: int, d_inner: int, N: int = 16, seed: int = 0, device="cpu") -> dict:
+    """Inputs of the layer's neighbours (bf16 activations and weights, fp32
+    modulation).  Draws h, gamma, beta, w_in, y, w_out: h, y ~ N(0, 1);
+    gamma ~ 1 + 0.1 N(0, 1), beta ~ 0.1 N(0, 1) per (batch row, feature);
+    weights ~ N(0, 1 / fan_in), so projected values are O(1)."""
+    g = _gen(seed, device)
+
+    def randn(*shape, scale=1.0):
+        return torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * scale
+
+    bf = torch.bfloat16
+    return {
+        "h": randn(batch, L, d_model).to(bf),
+        "gamma": (1.0 + randn(batch, d_model, scale=0.1)).contiguous(),
+        "beta": randn(batch, d_model, scale=0.1).contiguous(),
+        "w_in": randn(4 * d_inner + 4 * N, d_model, scale=d_model ** -0.5).to(bf),
+        "y": randn(batch, L, d_inner).to(bf),
+        "w_out": randn(d_model, d_inner, scale=d_inner ** -0.5).to(bf),
+    }
+
+
+# The projections around the 1.3B-shape layer: d_model 2048 -> d_inner 4096, b 8, L 2048.
+PROJ_1P3B = Workload("proj_1p3b_b8_L2048_dmodel2048_D4096_bf16", 8, 2048, 4096, 16, "bf16", 9,
+                     extra={"d_model": 2048})
+
 # One sequence of 262,144 tokens cut into contiguous segments, one per GPU
 # (the sequence-sharded scan; total work fixed as the GPU count grows).
 SHARDED_SEQ = Workload("sharded_b1_L262144_D4096_bf16", 1, 262144, 4096, 16, "bf16", 8)

@@ -330,6 +330,44 @@ int bimamba2_block_step(const bimamba2_fwd_state_t *prefix_state, const bimamba2
                         bimamba2_fwd_state_t *new_state, unsigned flags,
                         void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* ---- The layer's neighbours (App. A.1 Eq. (10)-(11), Table 12): AdaLN in
+ * front of the mixer and the projections around it.  bf16 in and out,
+ * device pointers, caller-owned, 16-byte aligned (gamma, beta: fp32, 4-byte).
+ * Rows are the batch * L tokens in [batch][L] order.  Nothing is launched when
+ * a check fails; returns BIMAMBA_OK or a negative status. */
+
+/* AdaLN (Eq. (10)): out[r] = gamma[b] * (x[r] - mu(x[r])) / sigma(x[r]) + beta[b]
+ * for every token row r of batch row b, mu and sigma^2 the mean and (biased)
+ * variance of the row's d values, sigma = sqrt(variance + eps).
+ *   x, out     [batch][L][d] bf16 (out must not alias x)
+ *   gamma, beta [batch][d] fp32: the timestep embedding's modulation
+ * d % 8 == 0 (else UNSUPPORTED); eps > 0.  One kernel launch. */
+int bimamba_adaln(const void *x, const float *gamma, const float *beta, void *out,
+                  int batch, int64_t L, int d, float eps, void *cuda_stream);
+
+/* The input projection, written straight into the layer's input arrays:
+ * for each token row r, y[r][n] = sum_k a[r][k] * w_in[n][k] (fp32
+ * accumulation on the tensor cores, rounded to bf16), with the columns n of
+ * w_in laid out as [x | z | dt_f | dt_b | B_f | C_f | B_b | C_b] (d_inner,
+ * d_inner, d_inner, d_inner, then d_state each: 4 d_inner + 4 d_state rows).
+ *   a      [batch][L][d_model]      (e.g. bimamba_adaln's output)
+ *   w_in   [4 d_inner + 4 d_state][d_model]
+ *   x, z   [batch][L][d_inner];  dt [2][batch][L][d_inner];  B, C [2][batch][L][d_state]
+ * (the layouts bimamba_layer_fwd reads, with dir_stride 0 for x and z).
+ * d_model % 64 == 0, d_inner % 8 == 0, d_state == 16 (else UNSUPPORTED);
+ * batch * L <= 8,388,480.  One kernel launch. */
+int bimamba_in_proj(const void *a, const void *w_in, int batch, int64_t L, int d_model, int d_inner, int d_state,
+                    void *x, void *z, void *dt, void *B, void *C, void *cuda_stream);
+
+/* The output projection of the layer's gated output (the sum of the two
+ * directions and the SiLU(z) gate are already applied by bimamba_layer_fwd):
+ * out[r][n] = sum_k y[r][k] * w_out[n][k], fp32 accumulation, bf16 result.
+ *   y      [batch][L][d_inner];  w_out [d_model][d_inner];  out [batch][L][d_model]
+ * d_inner % 64 == 0, d_model % 8 == 0 (else UNSUPPORTED); batch * L <= 8,388,480.
+ * One kernel launch. */
+int bimamba_out_proj(const void *y, const void *w_out, int batch, int64_t L, int d_inner, int d_model, void *out,
+                     void *cuda_stream);
+
 /* Read (and, if reset != 0, clear) the error word of the current device.
  * Kernels never wait without bound: a wait for a tile that gives up after
  * about two seconds sets bit 0 (a tile load that never arrived) and the kernel

@@ -362,3 +362,33 @@ def test_compose_carries_rejects(kw, status):
     a.update(kw)
     assert bm.lib.bimamba_compose_carries(a["h_all"], a["ds_all"], _byref(a["par"]), a["nseg"], a["seg"],
                                           a["batch"], a["D"], a["N"], a["h_in"], None) == status
+
+
+def test_neighbours_reject():
+    L = bm.lib
+    # AdaLN: null, sizes, d % 8, eps, misalignment
+    assert L.bimamba_adaln(None, FAKE, FAKE, FAKE, 2, 8, 64, 1e-5, None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 0, 8, 64, 1e-5, None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 2, 8, 64, 0.0, None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 2, 8, 60, 1e-5, None) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert L.bimamba_adaln(FAKE + 8, FAKE, FAKE, FAKE, 2, 8, 64, 1e-5, None) == bm.BIMAMBA_ERR_MISALIGNED
+    # input projection
+    ok = [FAKE, FAKE + 0x1000, 2, 8, 64, 32, 16] + [FAKE + 0x2000 * i for i in range(1, 6)] + [None]
+    def inp(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return L.bimamba_in_proj(*a)
+    assert inp(_0=None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert inp(_2=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert inp(_3=0) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert inp(_3=65535 * 128) == bm.BIMAMBA_ERR_INVALID_ARG  # 2 x that many rows: past the grid
+    assert inp(_4=96) == bm.BIMAMBA_ERR_UNSUPPORTED           # d_model % 64
+    assert inp(_5=36) == bm.BIMAMBA_ERR_UNSUPPORTED           # d_inner % 8
+    assert inp(_6=8) == bm.BIMAMBA_ERR_UNSUPPORTED            # d_state
+    assert inp(_9=FAKE + 0x6008) == bm.BIMAMBA_ERR_MISALIGNED
+    # output projection
+    assert L.bimamba_out_proj(FAKE, FAKE, 2, 8, 64, 32, None, None) == bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_out_proj(FAKE, FAKE, 2, 8, 72, 32, FAKE, None) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert L.bimamba_out_proj(FAKE, FAKE, 2, 8, 64, 36, FAKE, None) == bm.BIMAMBA_ERR_UNSUPPORTED
+    assert L.bimamba_out_proj(FAKE, FAKE + 4, 2, 8, 64, 32, FAKE, None) == bm.BIMAMBA_ERR_MISALIGNED
