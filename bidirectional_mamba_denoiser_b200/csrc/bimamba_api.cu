@@ -1109,11 +1109,21 @@ int bimamba_adaln(const void* x, const float* gamma, const float* beta, void* ou
     if (!x || !gamma || !beta || !out || batch < 1 || batch > kMaxBatch || L < 1 || d < 8 || !(eps > 0.f) ||
         (int64_t)batch * L > 0x7fffffffLL)
         return BIMAMBA_ERR_INVALID_ARG;
-    if (d % 8) return BIMAMBA_ERR_UNSUPPORTED;
-    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gamma, 4) || !aligned(beta, 4)) return BIMAMBA_ERR_MISALIGNED;
+    if (d % 8 || d > 8192) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gamma, 16) || !aligned(beta, 16))
+        return BIMAMBA_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-    bimamba::adaln_kernel<<<(unsigned)((int64_t)batch * L), 256, 0, st>>>(
-        static_cast<const bf16*>(x), gamma, beta, static_cast<bf16*>(out), L, d, eps);
+    const int64_t rows = (int64_t)batch * L;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    const bf16* xi = static_cast<const bf16*>(x);
+    bf16* o = static_cast<bf16*>(out);
+    const int cpl = (d + 255) / 256;  // 16-byte chunks per lane
+    if (cpl <= 1) bimamba::adaln_kernel<1><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
+    else if (cpl <= 2) bimamba::adaln_kernel<2><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
+    else if (cpl <= 4) bimamba::adaln_kernel<4><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
+    else if (cpl <= 8) bimamba::adaln_kernel<8><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
+    else if (cpl <= 16) bimamba::adaln_kernel<16><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
+    else bimamba::adaln_kernel<32><<<grid, 256, 0, st>>>(xi, gamma, beta, o, rows, L, d, eps);
     return launch_status();
 }
 

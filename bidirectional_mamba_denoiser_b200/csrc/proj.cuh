@@ -4,8 +4,9 @@
 // that produces the layer's inputs, and the output projection after it.
 //
 // AdaLN (Eq. (10)): out = gamma_b * (x - mu(x)) / sigma(x) + beta_b per token
-// row, gamma and beta per batch row, sigma = sqrt(var + eps); one CTA per
-// row, fp32 statistics (two passes over the row: mean, then centred squares).
+// row, gamma and beta per batch row, sigma = sqrt(var + eps); one warp per
+// row, fp32 statistics (the mean, then the centred squares, over the row held
+// in registers).
 //
 // The projections are one GEMM kernel on the tcgen05 tensor cores:
 // C[m][n] = sum_k A[m][k] W[n][k], bf16 operands, fp32 accumulation in TMEM,
@@ -31,60 +32,62 @@ namespace bimamba {
 
 // ---------------------------------------------------------------- AdaLN
 
-// grid (rows), block 256; d % 8 == 0; rows = batch * L, batch row = row / L.
+// One warp per token row, 8 rows per CTA of 256 threads: lane l holds the
+// 16-byte chunks l, l + 32, ... (CPL of them, d <= 256 CPL) in registers, so
+// the mean, the centred sum of squares and the output need one read of the
+// row and warp shuffles only.  d % 8 == 0; batch row = row / L.
+template <int CPL>
 __global__ void __launch_bounds__(256) adaln_kernel(const __nv_bfloat16* x, const float* gamma, const float* beta,
-                                                    __nv_bfloat16* out, int64_t L, int d, float eps) {
-    __shared__ float red[8];
-    const int64_t row = blockIdx.x;
-    const int b = (int)(row / L);
+                                                    __nv_bfloat16* out, int64_t rows, int64_t L, int d, float eps) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
     const __nv_bfloat16* xr = x + row * d;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    auto block_sum = [&](float v) {
+    float v[CPL][8];
+    float s = 0.f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        __syncthreads();  // red is free again
-        if (lane == 0) red[warp] = v;
-        __syncthreads();
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) s += red[w];
-        return s;
-    };
-    auto load8 = [&](int c, float (&v)[8]) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xr + c);
+    for (int i = 0; i < CPL; ++i) {
+        const int c = 8 * (lane + 32 * i);
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (c < d) q = *reinterpret_cast<const uint4*>(xr + c);
         const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
-            v[2 * u] = __uint_as_float(w4[u] << 16);
-            v[2 * u + 1] = __uint_as_float(w4[u] & 0xffff0000u);
+            v[i][2 * u] = __uint_as_float(w4[u] << 16);
+            v[i][2 * u + 1] = __uint_as_float(w4[u] & 0xffff0000u);
+            s += v[i][2 * u] + v[i][2 * u + 1];
         }
-    };
-    float s = 0.f;
-    for (int c = 8 * t; c < d; c += 8 * 256) {
-        float v[8];
-        load8(c, v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) s += v[u];
     }
-    const float mu = block_sum(s) / (float)d;
-    float q = 0.f;
-    for (int c = 8 * t; c < d; c += 8 * 256) {
-        float v[8];
-        load8(c, v);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) q = fmaf(v[u] - mu, v[u] - mu, q);
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    const float mu = s / (float)d;
+    float q2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        if (8 * (lane + 32 * i) < d) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) q2 = fmaf(v[i][u] - mu, v[i][u] - mu, q2);
+        }
     }
-    const float rstd = rsqrtf(block_sum(q) / (float)d + eps);
-    const float* g = gamma + (int64_t)b * d;
-    const float* be = beta + (int64_t)b * d;
-    for (int c = 8 * t; c < d; c += 8 * 256) {
-        float v[8];
-        load8(c, v);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, off);
+    const float rstd = rsqrtf(q2 / (float)d + eps);
+    const int64_t b = row / L;
+    const float* g = gamma + b * d;
+    const float* be = beta + b * d;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = 8 * (lane + 32 * i);
+        if (c >= d) continue;
+        const float4 g0 = *reinterpret_cast<const float4*>(g + c), g1 = *reinterpret_cast<const float4*>(g + c + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(be + c), b1 = *reinterpret_cast<const float4*>(be + c + 4);
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
         uint32_t w4[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const float a0 = fmaf(g[c + 2 * u], (v[2 * u] - mu) * rstd, be[c + 2 * u]);
-            const float a1 = fmaf(g[c + 2 * u + 1], (v[2 * u + 1] - mu) * rstd, be[c + 2 * u + 1]);
+            const float a0 = fmaf(gg[2 * u], (v[i][2 * u] - mu) * rstd, bb[2 * u]);
+            const float a1 = fmaf(gg[2 * u + 1], (v[i][2 * u + 1] - mu) * rstd, bb[2 * u + 1]);
             const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
             w4[u] = *reinterpret_cast<const uint32_t*>(&h);
         }

@@ -332,7 +332,7 @@ int bimamba2_block_step(const bimamba2_fwd_state_t *prefix_state, const bimamba2
 
 /* ---- The layer's neighbours (App. A.1 Eq. (10)-(11), Table 12): AdaLN in
  * front of the mixer and the projections around it.  bf16 in and out,
- * device pointers, caller-owned, 16-byte aligned (gamma, beta: fp32, 4-byte).
+ * device pointers, caller-owned, 16-byte aligned (gamma, beta: fp32).
  * Rows are the batch * L tokens in [batch][L] order.  Nothing is launched when
  * a check fails; returns BIMAMBA_OK or a negative status. */
 
@@ -340,8 +340,8 @@ int bimamba2_block_step(const bimamba2_fwd_state_t *prefix_state, const bimamba2
  * for every token row r of batch row b, mu and sigma^2 the mean and (biased)
  * variance of the row's d values, sigma = sqrt(variance + eps).
  *   x, out     [batch][L][d] bf16 (out must not alias x)
- *   gamma, beta [batch][d] fp32: the timestep embedding's modulation
- * d % 8 == 0 (else UNSUPPORTED); eps > 0.  One kernel launch. */
+ *   gamma, beta [batch][d] fp32, 16-byte aligned: the timestep embedding's modulation
+ * d % 8 == 0 and d <= 8192 (else UNSUPPORTED); eps > 0.  One kernel launch. */
 int bimamba_adaln(const void *x, const float *gamma, const float *beta, void *out,
                   int batch, int64_t L, int d, float eps, void *cuda_stream);
 

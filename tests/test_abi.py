@@ -372,6 +372,8 @@ def test_neighbours_reject():
     assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 2, 8, 64, 0.0, None) == bm.BIMAMBA_ERR_INVALID_ARG
     assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 2, 8, 60, 1e-5, None) == bm.BIMAMBA_ERR_UNSUPPORTED
     assert L.bimamba_adaln(FAKE + 8, FAKE, FAKE, FAKE, 2, 8, 64, 1e-5, None) == bm.BIMAMBA_ERR_MISALIGNED
+    assert L.bimamba_adaln(FAKE, FAKE + 4, FAKE, FAKE, 2, 8, 64, 1e-5, None) == bm.BIMAMBA_ERR_MISALIGNED
+    assert L.bimamba_adaln(FAKE, FAKE, FAKE, FAKE, 2, 8, 8200, 1e-5, None) == bm.BIMAMBA_ERR_UNSUPPORTED
     # input projection
     ok = [FAKE, FAKE + 0x1000, 2, 8, 64, 32, 16] + [FAKE + 0x2000 * i for i in range(1, 6)] + [None]
     def inp(**kw):
