@@ -756,13 +756,13 @@ def run_proj(args, w, bm, rank, world, dev, stream):
         per[name] = t / args.steps
     f_in = 2.0 * M * dm * (4 * D + 4 * w.d_state)
     f_out = 2.0 * M * D * dm
-    roof = roofline_tensor(f_in, per["in_proj"], w.name, "gemm_bf16_kernel (input projection)")
+    roof = roofline_tensor(f_in, per["in_proj"], w.name, "gemm_bf16_persistent_kernel (input projection)")
     adaln_bytes = M * dm * 2 * 2
     return {
         "value": whole_job_rate(M * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps, "gpu_launches": 3 * args.steps, "roofline": roof, "clocks": clocks,
         "kernels_ms": {k: round(v, 4) for k, v in per.items()},
-        "out_proj_roofline": roofline_tensor(f_out, per["out_proj"], w.name, "gemm_bf16_kernel (output projection)"),
+        "out_proj_roofline": roofline_tensor(f_out, per["out_proj"], w.name, "gemm_bf16_persistent_kernel (output projection)"),
         "adaln_hbm": hbm_fraction(adaln_bytes, per["adaln"]),
         "note": "value = tokens through AdaLN + input projection + output projection per second",
     }

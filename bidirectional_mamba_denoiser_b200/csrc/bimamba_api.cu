@@ -1086,12 +1086,16 @@ int launch_gemm(const void* a, const void* w, const bimamba::GemmParams& gp, cud
     if (!map2d_sw128(&ma, a, (uint64_t)gp.K, (uint64_t)gp.M, bimamba::kGemmBM) ||
         !map2d_sw128(&mw, w, (uint64_t)gp.K, (uint64_t)gp.N, bimamba::kGemmBN))
         return BIMAMBA_ERR_CUDA;
-    const void* fn = reinterpret_cast<const void*>(&bimamba::gemm_bf16_kernel);
+    const void* fn = reinterpret_cast<const void*>(&bimamba::gemm_bf16_persistent_kernel);
     int rc = ensure_smem(fn, bimamba::kGemmSmem);
     if (rc) return rc;
-    const dim3 grid((unsigned)((gp.N + bimamba::kGemmBN - 1) / bimamba::kGemmBN),
-                    (unsigned)((gp.M + bimamba::kGemmBM - 1) / bimamba::kGemmBM));
-    bimamba::gemm_bf16_kernel<<<grid, 128, bimamba::kGemmSmem, st>>>(ma, mw, gp);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BIMAMBA_ERR_CUDA;
+    const int64_t tiles = (int64_t)((gp.N + bimamba::kGemmBN - 1) / bimamba::kGemmBN) *
+                          ((gp.M + bimamba::kGemmBM - 1) / bimamba::kGemmBM);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    bimamba::gemm_bf16_persistent_kernel<<<grid, bimamba::kGemmPThreads, bimamba::kGemmSmem, st>>>(ma, mw, gp);
     return launch_status();
 }
 

@@ -10,12 +10,12 @@
 //
 // The projections are one GEMM kernel on the tcgen05 tensor cores:
 // C[m][n] = sum_k A[m][k] W[n][k], bf16 operands, fp32 accumulation in TMEM,
-// bf16 results.  A CTA computes a 128 x 256 tile: a producer thread streams
-// 128 x 64 A and 256 x 64 W tiles by TMA (128-byte swizzle) through a
-// 4-stage shared-memory ring, one thread issues the MMAs of each stage
-// (4 x K = 16) and frees the stage by tcgen05.commit, and after the last
-// stage the four warps read the accumulator rows of their TMEM lanes and
-// store them.  Every wait is bounded.  The epilogue either writes C as is
+// bf16 results, in 128 x 256 tiles: a producer thread streams 128 x 64 A and
+// 256 x 64 W tiles by TMA (128-byte swizzle) through a 4-stage shared-memory
+// ring, one thread issues the MMAs of each stage (4 x K = 16) and frees the
+// stage by tcgen05.commit, and four epilogue warps drain the accumulator --
+// persistent CTAs with two accumulators, so that a tile's stores overlap the
+// next tile's products.  Every wait is bounded.  The epilogue either writes C as is
 // (output projection: A is the layer's gated output) or scatters each 8-column
 // group straight into the mixer's input arrays (input projection: columns
 // [x | z | dt_f | dt_b | B_f | C_f | B_b | C_b]), so the layer reads them with
@@ -141,77 +141,110 @@ __device__ __forceinline__ void gemm_store8(const GemmParams& p, int m, int n, c
     *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
 }
 
-// grid (ceil(N / 256), ceil(M / 128)), block 128, dynamic shared memory kGemmSmem.
-// mapA: [M][K] bf16, box {64, 128}; mapW: [N][K] bf16, box {64, 256}; both
-// 128-byte swizzled.  K % 64 == 0; N % 8 == 0.
-__global__ void __launch_bounds__(128, 1) gemm_bf16_kernel(const __grid_constant__ CUtensorMap mapA,
-                                                           const __grid_constant__ CUtensorMap mapW,
-                                                           const GemmParams p) {
+// C = A W^T as a persistent kernel: grid = min(tiles, SMs), block 192, dynamic
+// shared memory kGemmSmem.  mapA: [M][K] bf16, box {64, 128}; mapW: [N][K]
+// bf16, box {64, 256}; both 128-byte swizzled.  K % 64 == 0; N % 8 == 0.
+// Warp 0 (one thread) streams the A / W tiles of every K step of every tile
+// this CTA owns (tiles blockIdx.x, blockIdx.x + gridDim.x, ...) through the
+// ring; warp 1 (one thread) issues the MMAs into one of two TMEM accumulators
+// (2 x 256 columns) and commits "accumulator full"; warps 2-5 drain the other
+// accumulator -- warp w reads TMEM lanes 32 (w % 4) .. +31 -- and hand it back
+// ("accumulator empty", one arrival per warp), so a tile's stores overlap the
+// next tile's products.  Tiles run along N first, so consecutive tiles of a CTA
+// reuse the A rows from L2.  Every wait is bounded.
+constexpr int kGemmPThreads = 192;
+
+__global__ void __launch_bounds__(kGemmPThreads, 1) gemm_bf16_persistent_kernel(
+    const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(base + kGemmBarOff);
     uint64_t* empty = full + kGemmStages;
-    uint64_t* done = empty + kGemmStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* acc_full = empty + kGemmStages;  // [2]
+    uint64_t* acc_empty = acc_full + 2;        // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
     const int nk = p.K / kGemmBK;
+    const int tiles_n = (p.N + kGemmBN - 1) / kGemmBN;
+    const int tiles = tiles_n * ((p.M + kGemmBM - 1) / kGemmBM);
 
     if (t == 0) {
-        for (int i = 0; i < 2 * kGemmStages + 1; ++i) mbar_init(full + i, 1);
+        for (int i = 0; i < 2 * kGemmStages + 2; ++i) mbar_init(full + i, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(acc_empty + 1, 4);
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc<256>(tmem_slot);
+    if (warp == 0) tmem_alloc<512>(tmem_slot);
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (t == 0) {  // producer: A and W tiles of each K step into the ring
-        for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kGemmStages;
-            if (kt >= kGemmStages) mbar_wait_bounded(empty + s, (uint32_t)(((kt / kGemmStages) - 1) & 1), p.wait_limit);
-            unsigned char* st = base + s * kGemmStage;
-            mbar_arrive_expect_tx(full + s, kGemmStage);
-            tma_load_2d(st, &mapA, full + s, kt * kGemmBK, m0);
-            tma_load_2d(st + kGemmATile, &mapW, full + s, kt * kGemmBK, n0);
+    if (t == 0) {  // producer
+        int g = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+            for (int kt = 0; kt < nk; ++kt, ++g) {
+                const int s = g % kGemmStages;
+                if (g >= kGemmStages) mbar_wait_bounded(empty + s, (uint32_t)(((g / kGemmStages) - 1) & 1), p.wait_limit);
+                unsigned char* st = base + s * kGemmStage;
+                mbar_arrive_expect_tx(full + s, kGemmStage);
+                tma_load_2d(st, &mapA, full + s, kt * kGemmBK, m0);
+                tma_load_2d(st + kGemmATile, &mapW, full + s, kt * kGemmBK, n0);
+            }
         }
     } else if (t == 32) {  // MMA issuer
         constexpr uint32_t idesc = umma_idesc_bf16(kGemmBM, kGemmBN);
-        for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kGemmStages;
-            mbar_wait_bounded(full + s, (uint32_t)((kt / kGemmStages) & 1), p.wait_limit);
+        int g = 0, i = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
+            const int acc = i & 1;
+            if (i >= 2) mbar_wait_bounded(acc_empty + acc, (uint32_t)(((i >> 1) - 1) & 1), p.wait_limit);
             tmem_fence_after_sync();
-            const uint32_t a = smem_addr(base + s * kGemmStage), w = a + kGemmATile;
+            const uint32_t d = tmem + 256 * acc;
+            for (int kt = 0; kt < nk; ++kt, ++g) {
+                const int s = g % kGemmStages;
+                mbar_wait_bounded(full + s, (uint32_t)((g / kGemmStages) & 1), p.wait_limit);
+                tmem_fence_after_sync();
+                const uint32_t a = smem_addr(base + s * kGemmStage), w = a + kGemmATile;
 #pragma unroll
-            for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                umma_f16(tmem, umma_desc_sw128(a + 32 * kk), umma_desc_sw128(w + 32 * kk), idesc, kt > 0 || kk > 0);
-            umma_commit(empty + s);  // the stage is free once these products have read it
+                for (int kk = 0; kk < kGemmBK / 16; ++kk)
+                    umma_f16(d, umma_desc_sw128(a + 32 * kk), umma_desc_sw128(w + 32 * kk), idesc, kt > 0 || kk > 0);
+                umma_commit(empty + s);
+            }
+            umma_commit(acc_full + acc);
         }
-        umma_commit(done);
+    } else if (warp >= 2) {  // epilogue
+        const int q = warp & 3;  // TMEM lane quadrant of this warp
+        const uint32_t lb = (uint32_t)(32 * q) << 16;
+        int i = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
+            const int acc = i & 1;
+            const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+            mbar_wait_bounded(acc_full + acc, (uint32_t)((i >> 1) & 1), p.wait_limit);
+            tmem_fence_after_sync();
+            const int m = m0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < kGemmBN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + 256 * acc + lb + 32 * c, v);
+                if (m < p.M) {
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {
+                        const int n = n0 + 32 * c + 8 * gq;
+                        if (n < p.N) gemm_store8(p, m, n, v + 8 * gq);
+                    }
+                }
+            }
+            tmem_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + acc);
+        }
     }
     __syncwarp();
-    // epilogue: warp w owns accumulator rows 32w .. 32w+31 (its TMEM lanes)
-    mbar_wait_bounded(done, 0, p.wait_limit);
-    tmem_fence_after_sync();
-    const int m = m0 + warp * 32 + lane;
-    const uint32_t lb = (uint32_t)(warp * 32) << 16;
-#pragma unroll 1
-    for (int c = 0; c < kGemmBN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lb + 32 * c, v);
-        if (m < p.M) {
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const int n = n0 + 32 * c + 8 * g;
-                if (n < p.N) gemm_store8(p, m, n, v + 8 * g);
-            }
-        }
-    }
     tmem_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc<256>(tmem);
+    if (warp == 0) tmem_dealloc<512>(tmem);
 }
 
 }  // namespace bimamba
