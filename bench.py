@@ -553,7 +553,7 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     res = {
         "value": whole_job_rate(tokens * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
-        "gpu_launches": (4 if tensor_path else 3) * args.steps,
+        "gpu_launches": 3 * args.steps,
         "hbm": hbm_fraction(mamba2_bytes(w.batch, w.L, H, P, N), call_ms),
         "clocks": clocks,
         "recurrence_flops_per_token": int(flops / tokens),
