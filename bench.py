@@ -553,14 +553,14 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     res = {
         "value": whole_job_rate(tokens * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (2 if tensor_path else 3) * args.steps,
         "hbm": hbm_fraction(mamba2_bytes(w.batch, w.L, H, P, N), call_ms),
         "clocks": clocks,
         "recurrence_flops_per_token": int(flops / tokens),
     }
     if tensor_path:
         res["roofline"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
-                                          "m2_prep + 2 x m2_ssd_kernel")
+                                          "m2_prep + m2_ssd_kernel (both directions, clusters of 2)")
         res["fp32_equivalent"] = roofline_fma(flops, call_ms, clocks, w.name, "recurrence-equivalent")
     else:
         res["roofline"] = roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel")

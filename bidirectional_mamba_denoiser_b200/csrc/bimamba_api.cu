@@ -819,28 +819,44 @@ bool m2_sizes_ok(int batch, int64_t L, int H) {
 }
 
 // Chunked dual form on the tensor cores: the C/B chunk tiles, then the
-// forward and reverse chunk scans, which compute the x features and step
-// sizes themselves (three launches; when L is not a whole number of chunks,
-// the last chunk's tiles are cleared first so that its rows past the end read
+// directions' chunk scans, which compute the x features and step sizes
+// themselves -- both in one launch as clusters of two CTAs that meet halfway
+// when one direction's grid leaves SMs idle, else the forward then the
+// reverse (two or three launches; when L is not a whole number of chunks, the
+// ragged chunk's tiles are cleared first so that its rows past the end read
 // zeros).
 template <typename Tin, typename Tout>
 int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
+    auto kc = &bimamba::m2_ssd_cluster_kernel<Tin, Tout>;
     auto k0 = &bimamba::m2_ssd_kernel<0, Tin, Tout>;
     auto k1 = &bimamba::m2_ssd_kernel<1, Tin, Tout>;
-    int rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
+    int rc = ensure_smem(reinterpret_cast<const void*>(kc), bimamba::kSsdSmem);
+    if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
     if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k1), bimamba::kSsdSmem);
     if (rc) return rc;
     const int64_t nc = (k.L + bimamba::kSQ - 1) / bimamba::kSQ;
-    if (k.L % bimamba::kSQ) {
+    if (k.L % bimamba::kSQ) {  // the ragged chunk: the forward's last, the reverse's first in step order
         const size_t pair = 2 * (size_t)bimamba::kTileBytes;
-        if (cudaMemset2DAsync(k.tiles + (nc - 1) * pair, (size_t)nc * pair, 0, pair, (size_t)(2 * k.batch), st) !=
-            cudaSuccess)
+        if (cudaMemset2DAsync(k.tiles + (nc - 1) * pair, (size_t)nc * pair, 0, pair, (size_t)k.batch, st) !=
+                cudaSuccess ||
+            cudaMemset2DAsync(k.tiles + (size_t)k.batch * nc * pair, (size_t)nc * pair, 0, pair, (size_t)k.batch,
+                              st) != cudaSuccess)
             return BIMAMBA_ERR_CUDA;
     }
     const int64_t tok_per_cta = 4 * bimamba::kM2PrepT;
     const dim3 g1((unsigned)((k.L + tok_per_cta - 1) / tok_per_cta), 1u, (unsigned)(2 * k.batch));
     bimamba::m2_prep_kernel<Tin, true><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    // one direction's grid within one wave (2 CTAs per SM): both directions at once, as
+    // clusters that meet halfway; else the forward, then the reverse (measured faster
+    // there: 0.80 against 0.89 ms at batch 8, L 2048, 120 heads)
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BIMAMBA_ERR_CUDA;
+    if ((int64_t)k.H * k.batch <= 2LL * sms) {
+        kc<<<dim3((unsigned)(2 * k.H), (unsigned)k.batch), 128, bimamba::kSsdSmem, st>>>(k);
+        return launch_status();
+    }
     const dim3 g2((unsigned)k.H, (unsigned)k.batch);
     k0<<<g2, 128, bimamba::kSsdSmem, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
@@ -1052,6 +1068,7 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
         k.tiles = ws + lay.tiles;
+        k.YB = reinterpret_cast<float*>(ws + lay.v);  // the fp32 feature region, unused on this path
         if (out_bf) return launch_m2_ssd<bf16, bf16>(k, st);
         return launch_m2_ssd<bf16, float>(k, st);
     }

@@ -63,6 +63,7 @@ struct M2Params {
     float* V;              // [2][batch][L][CH]   conv + SiLU features
     float* DL;             // [2][batch][H][L]    step sizes
     float* YF;             // [batch][L][H*P]     forward y
+    float* YB;             // [batch][L][H*P]     reverse y (tensor-core path: the reverse CTA's first half)
     int64_t L;
     int H, CH, batch;
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
@@ -122,7 +123,8 @@ constexpr int kM2Chunk = 128;  // steps per chunk of the tensor-core path
 // sizes itself): grid (ceil(L / 32), 1, 2 * batch), block 128 = 4 token
 // groups x the 32 threads of the B and C channels, written as fp16 rows of
 // the chunk tiles at the token's step (forward: token t is step t; reverse:
-// step L-1-t), in the canonical K-major layout.
+// step nc*128-1-t, the chunks of both directions covering the same tokens),
+// in the canonical K-major layout.
 template <typename Tin, bool TILES>
 __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     constexpr int TT = kM2PrepT;
@@ -185,8 +187,8 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
                 const int HP = H * kM2P;
                 const bool isB = c0 < HP + kM2N;
                 const int n0 = c0 - HP - (isB ? 0 : kM2N);
-                const int64_t step = r == 0 ? t : L - 1 - t;
                 const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
+                const int64_t step = r == 0 ? t : nc * kM2Chunk - 1 - t;  // chunks aligned in token space
                 unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + step / kM2Chunk) *
                                                  (2 * kM2Chunk * kM2N * 2);
                 *reinterpret_cast<uint4*>(T + (isB ? kM2Chunk * kM2N * 2 : 0) +

@@ -71,13 +71,30 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, const float (&v)[4]) 
         make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
 }
 
-// grid (H, batch), block 128, dynamic shared memory kSsdSmem.  DIR 0 stores
-// y_0 to p.YF; DIR 1 adds it and applies the gate.
-template <int DIR, typename Tin, typename Tout>
-__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
+// Both directions cut the sequence into the same chunks of Q tokens (chunk j
+// = tokens [jQ, jQ + Q)); the forward walks chunks 0 .. nc-1 with step t of
+// chunk j at token jQ + t, the reverse walks nc-1 .. 0 with step t at token
+// jQ + Q-1-t.  When L % Q != 0 the reverse's first chunk starts with steps
+// past the end, identity steps (step size 0, x zero).
+// Both directions of a (head, batch row) run as the two CTAs of a cluster.
+// Each walks its chunks in its own order; over the first half (forward:
+// chunks 0 .. nc/2 - 1; reverse: chunks nc-1 .. nc/2) it stores its y to the
+// workspace (p.YF forward, p.YB reverse).  The two then meet at a cluster
+// barrier (release / acquire: each sees the other's stores), and over the
+// second half each adds the partner's stored y to its own and applies the
+// SiLU(z) gate.  Every token is gated exactly once, by the direction that
+// reaches it second.
+__device__ __forceinline__ void cluster_meet() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// CL: the two directions run as a cluster and meet halfway (above).  Without
+// it the forward stores y for every chunk (p.YF) and the reverse, launched
+// after it, gates every chunk with that y.
+template <int DIR, typename Tin, typename Tout, bool CL>
+__device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm, const int h) {
     constexpr int Q = kSQ, P = kM2P;
     static_assert(sizeof(Tin) == 2, "the dual form reads bf16 inputs");
-    extern __shared__ __align__(128) unsigned char sm[];
     unsigned char* sC = sm + kSsdC;
     unsigned char* sB = sm + kSsdB;
     unsigned char* sDX = sm + kSsdDX;
@@ -93,10 +110,13 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     float* sCB = reinterpret_cast<float*>(sm + kSsdCB);    // [32]: conv bias
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int b = blockIdx.y;
     const int64_t L = p.L;
     const int H = p.H, HP = H * P;
     const int nc = (int)((L + Q - 1) / Q);
+    const int meetk = CL ? (DIR == 0 ? nc / 2 : nc - nc / 2) : (DIR == 0 ? nc : 0);  // chunks before the meeting
+    float* own_y = DIR == 0 ? p.YF : p.YB;
+    const float* partner_y = DIR == 0 ? p.YB : p.YF;
     const unsigned char* tileb = p.tiles + ((int64_t)DIR * p.batch + b) * nc * (2 * kTileBytes);
     const int CH = p.CH;
     const Tin* Xr = static_cast<const Tin*>(p.xbc[DIR]) + (int64_t)b * L * CH + (int64_t)h * P;
@@ -146,7 +166,7 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
     float dt_next = 0.f;
     bool ok_next = false;
     auto fetch_step = [&](int kk) {
-        const int64_t tk = DIR == 0 ? (int64_t)kk * Q + t : L - 1 - (int64_t)kk * Q - t;
+        const int64_t tk = DIR == 0 ? (int64_t)kk * Q + t : (int64_t)(nc - kk) * Q - 1 - t;
         const bool ok = tk >= 0 && tk < L;
         const Tin* src = Xr + (ok ? tk : 0) * CH;
 #pragma unroll
@@ -165,12 +185,14 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
 #pragma unroll 1
     for (int k = 0; k < nc; ++k) {
         const uint32_t ph = (uint32_t)(k & 1);
+        const bool gated = CL ? k >= meetk : DIR == 1;
+        if (CL && k == meetk) cluster_meet();
         // ---- step t of chunk k: x and delta
         float x[32];
-        // the reverse epilogue's y_0 and z in the row-contiguous mapping of the output stores:
+        // a gated chunk's partner y and z in the row-contiguous mapping of the output stores:
         // row 32 warp + 4 i + lane / 8, channels 4 (lane % 8) .. + 3
-        float4 yfc[DIR == 1 ? 8 : 1];
-        uint2 zc[DIR == 1 ? 8 : 1];
+        float4 yfc[8];
+        uint2 zc[8];
         uint32_t sraw[32];
         tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
         const float dtk = dt_next;
@@ -276,16 +298,16 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
             for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(sraw[i]) * f;
             tmem_st32(tmem + 192 + lb, s);
         }
-        if constexpr (DIR == 1) {  // in flight while the products run
+        if (gated) {  // in flight while the products run
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 32 * warp + 4 * i + (lane >> 3);
-                const int64_t tk = L - 1 - (int64_t)k * Q - r;
+                const int64_t tk = DIR == 0 ? (int64_t)k * Q + r : (int64_t)(nc - k) * Q - 1 - r;
                 yfc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 zc[i] = make_uint2(0u, 0u);
-                if (tk >= 0) {
+                if (tk >= 0 && tk < L) {
                     const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
-                    yfc[i] = *reinterpret_cast<const float4*>(p.YF + o);
+                    yfc[i] = *reinterpret_cast<const float4*>(partner_y + o);
                     zc[i] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
                 }
             }
@@ -414,11 +436,11 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
                 const int r = 4 * i + (lane >> 3);
                 const float4 v = stg[r * 8 + (cq ^ (r & 7))];
                 const int step = 32 * warp + r;
-                const int64_t tk = DIR == 0 ? (int64_t)k * Q + step : L - 1 - (int64_t)k * Q - step;
+                const int64_t tk = DIR == 0 ? (int64_t)k * Q + step : (int64_t)(nc - k) * Q - 1 - step;
                 if (tk >= 0 && tk < L) {
                     const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * cq;
-                    if constexpr (DIR == 0) {
-                        *reinterpret_cast<float4*>(p.YF + o) = v;
+                    if (!gated) {
+                        *reinterpret_cast<float4*>(own_y + o) = v;
                     } else {
                         // bf16 -> fp32 is exact: the bf16 bits are the high half
                         const float z0 = __uint_as_float(zc[i].x << 16), z1 = __uint_as_float(zc[i].x & 0xffff0000u);
@@ -437,9 +459,30 @@ __global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
         __syncthreads();
         tmem_fence_after_sync();
     }
+    if (CL && meetk >= nc) cluster_meet();  // a one-chunk sequence: the reverse CTA meets after its chunk
     tmem_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc<256>(tmem);
+}
+
+// grid (2 H, batch) in clusters of 2: CTA 2h runs head h forward, CTA 2h+1 in
+// reverse; block 128, dynamic shared memory kSsdSmem.  For calls whose
+// per-direction grid leaves SMs idle: both directions run at once.
+template <typename Tin, typename Tout>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 2) m2_ssd_cluster_kernel(const M2Params p) {
+    extern __shared__ __align__(128) unsigned char sm[];
+    if (blockIdx.x & 1)
+        m2_ssd_dir<1, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1));
+    else
+        m2_ssd_dir<0, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1));
+}
+
+// grid (H, batch), block 128, dynamic shared memory kSsdSmem: one direction;
+// the forward launch stores y_0, the reverse launch after it gates.
+template <int DIR, typename Tin, typename Tout>
+__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
+    extern __shared__ __align__(128) unsigned char sm[];
+    m2_ssd_dir<DIR, Tin, Tout, false>(p, sm, (int)blockIdx.x);
 }
 
 }  // namespace bimamba

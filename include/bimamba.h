@@ -280,10 +280,14 @@ size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, i
  * bimamba2_workspace_bytes(), 256-byte aligned, caller-owned.
  * bf16 inputs run the scan in its chunked dual form on the tensor cores
  * (chunks of 128 steps; fp16 operands, fp32 accumulation and state; within
- * 2e-3 of the exact result normwise): three launches (the C/B chunk tiles;
- * the forward chunks, which compute their x features and step sizes from
- * xbc and dt themselves; the reverse chunks + combine + gate), plus a
- * clearing of the last chunk's tiles when L % 128 != 0.  fp32 inputs, or flags with
+ * 2e-3 of the exact result normwise): the C/B chunk tiles, then the two
+ * directions' chunk scans, which compute their x features and step sizes
+ * from xbc and dt themselves: when batch * nheads <= 2 x the SM count both
+ * run in one launch as the two CTAs of a thread-block cluster (each stores
+ * its y over the first half of its walk and, after meeting at a cluster
+ * barrier, combines and gates over the second half), else the forward and
+ * then the reverse (which gates); plus a clearing of the ragged chunk's tiles
+ * when L % 128 != 0.  fp32 inputs, or flags with
  * BIMAMBA_NO_TMA, run the step-by-step scan on the CUDA cores in fp32: three
  * launches.  Other flags: BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY (test aids);
  * BIMAMBA_TEST_STARVE (tensor-core path: no tile copies are issued, every

@@ -56,6 +56,20 @@ def test_bf16_inputs(bm, path):
     assert U.bf16_out_ok(got16, want)
 
 
+@pytest.mark.parametrize("shape", [(3, 300, 120), (1, 383, 300), (3, 129, 100)])
+def test_tensor_path_both_launch_forms(bm, shape):
+    """batch * nheads above 2 x the SM count runs the forward and reverse
+    launches one after the other, at or below it one clustered launch whose
+    CTAs meet halfway: both, with ragged L (the chunks of the two directions
+    aligned in token space), within the 2e-3 bound."""
+    b, L, H = shape
+    inp, par = W.make_mamba2_case(b, L, H, P, N, "bf16", seed=66 + L)
+    want = oracle.mamba2_layer_fwd(inp, par)
+    got = run(bm, inp, par, torch.float32)
+    assert bm.bimamba_device_error() == 0
+    assert U.normwise(got, want) <= U.TOL_BF16
+
+
 @pytest.mark.parametrize("L", [1, 2, 127, 128, 129, 256, 383])
 def test_tensor_path_ragged_lengths(bm, L):
     """Chunks of 128 steps: lengths around the chunk edge, both directions."""
