@@ -792,14 +792,13 @@ namespace {
 size_t m2_round(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct M2Layout {
-    size_t v, dl, yf, tiles, total;
+    size_t v, dl, yf, yb, tiles, total;
 };
 
-// Workspace: conv features [2][batch][L][CH] fp32 (the tensor-core path keeps
-// only x there, as fp16 [2][batch][L][H*P]), step sizes [2][batch][H][L],
-// forward output [batch][L][H*P], both fp32, then the fp16 C/B tiles of the
-// tensor-core path [2][batch][ceil(L/128)][2][128 x 128]; each part 256-byte
-// aligned.
+// Workspace: conv features [2][batch][L][CH] fp32 (step-by-step path),
+// step sizes [2][batch][H][L], forward and reverse outputs [batch][L][H*P]
+// each, all fp32, then the fp16 C/B tiles of the tensor-core path
+// [2][batch][ceil(L/128)][2][128 x 128]; each part 256-byte aligned.
 M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
     const size_t CH = (size_t)H * P + 2 * (size_t)N;
     const size_t nc = (size_t)((L + bimamba::kSQ - 1) / bimamba::kSQ);
@@ -807,7 +806,8 @@ M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
     l.v = 0;
     l.dl = m2_round(2 * (size_t)batch * (size_t)L * CH * 4);
     l.yf = l.dl + m2_round(2 * (size_t)batch * (size_t)H * (size_t)L * 4);
-    l.tiles = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
+    l.yb = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
+    l.tiles = l.yb + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
     l.total = l.tiles + 2 * (size_t)batch * nc * 2 * (size_t)bimamba::kTileBytes;
     return l;
 }
@@ -870,10 +870,11 @@ int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
                   (unsigned)(2 * k.batch));
     bimamba::m2_prep_kernel<Tin, false><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    const dim3 g2((unsigned)k.H, (unsigned)k.batch);
-    bimamba::m2_scan_kernel<0, Tin, Tout><<<g2, 32, 0, st>>>(k);
+    bimamba::m2_scan_kernel<true, Tin><<<dim3((unsigned)(2 * k.H), (unsigned)k.batch), 32, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    bimamba::m2_scan_kernel<1, Tin, Tout><<<g2, 32, 0, st>>>(k);
+    const int64_t n4 = (int64_t)k.batch * k.L * k.H * bimamba::kM2P / 4;
+    const int64_t blocks = (n4 + 255) / 256;
+    bimamba::m2_combine_kernel<Tin, Tout><<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, st>>>(k);
     return launch_status();
 }
 
@@ -940,11 +941,11 @@ int bimamba2_prefix_state(const bimamba2_inputs_t* prefix, const bimamba2_params
     const dim3 g3((unsigned)((k.CH + 127) / 128), (unsigned)batch);
     if (prefix->dtype == BIMAMBA_BF16) {
         bimamba::m2_prep_kernel<bf16, false><<<g1, 128, 0, st>>>(k);
-        bimamba::m2_scan_kernel<0, bf16, float><<<g2, 32, 0, st>>>(k);
+        bimamba::m2_scan_kernel<false, bf16><<<g2, 32, 0, st>>>(k);
         bimamba::m2_tail_kernel<bf16><<<g3, 128, 0, st>>>(k);
     } else {
         bimamba::m2_prep_kernel<float, false><<<g1, 128, 0, st>>>(k);
-        bimamba::m2_scan_kernel<0, float, float><<<g2, 32, 0, st>>>(k);
+        bimamba::m2_scan_kernel<false, float><<<g2, 32, 0, st>>>(k);
         bimamba::m2_tail_kernel<float><<<g3, 128, 0, st>>>(k);
     }
     return launch_status();
@@ -985,6 +986,7 @@ int bimamba2_block_step(const bimamba2_fwd_state_t* prefix_state, const bimamba2
     k.V = reinterpret_cast<float*>(ws + lay.v);
     k.DL = reinterpret_cast<float*>(ws + lay.dl);
     k.YF = reinterpret_cast<float*>(ws + lay.yf);
+    k.YB = reinterpret_cast<float*>(ws + lay.yb);
     k.L = block_len;
     k.H = nheads;
     k.CH = nheads * headdim + 2 * d_state;
@@ -1056,6 +1058,7 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     k.V = reinterpret_cast<float*>(ws + lay.v);
     k.DL = reinterpret_cast<float*>(ws + lay.dl);
     k.YF = reinterpret_cast<float*>(ws + lay.yf);
+    k.YB = reinterpret_cast<float*>(ws + lay.yb);
     k.L = L;
     k.H = nheads;
     k.CH = nheads * headdim + 2 * d_state;
@@ -1068,7 +1071,6 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
         k.tiles = ws + lay.tiles;
-        k.YB = reinterpret_cast<float*>(ws + lay.v);  // the fp32 feature region, unused on this path
         if (out_bf) return launch_m2_ssd<bf16, bf16>(k, st);
         return launch_m2_ssd<bf16, float>(k, st);
     }

@@ -15,8 +15,8 @@
 // Three launches: m2_prep_kernel writes the conv + SiLU features of both
 // directions and the per-head step sizes (fp32, to the workspace) -- B and C
 // are shared by every head, so they are computed once, not once per head;
-// m2_scan_kernel<0, ...> runs the forward scans and stores y_0;
-// m2_scan_kernel<1, ...> runs the reverse scans, adds y_0 and applies the gate.
+// m2_scan_kernel<true, ...> runs the forward and reverse scans at once,
+// storing y_0 and y_1; m2_combine_kernel adds them and applies the gate.
 //
 // Scan: one warp per (batch row, head).  Lane (pb, nb) = (lane / 8, lane % 8)
 // holds rows 8pb..8pb+7 x the 16 states {32i + 4nb + j : i, j < 4} of the
@@ -210,20 +210,21 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     }
 }
 
-// grid (H, batch), block 32: one warp scans one head of one batch row in
-// direction DIR.  DIR 0 stores y_0 to p.YF; DIR 1 adds it and gates.
-template <int DIR, typename Tin, typename Tout>
+// block 32: one warp scans one head of one batch row in one direction and
+// stores its y (p.YF forward, p.YB reverse; not stored where null).  BOTH:
+// grid (2 H, batch), CTA 2h + r runs head h in direction r, so both
+// directions are in flight at once (m2_combine_kernel then adds and gates);
+// else grid (H, batch), forward only (a prefix scan).
+template <bool BOTH, typename Tin>
 __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
     constexpr int P = kM2P, N = kM2N, T = kM2T;
     __shared__ __align__(16) float xs[2][T][P];
     __shared__ __align__(16) float bs[2][T][N];
     __shared__ __align__(16) float cs[2][T][N];
     __shared__ __align__(16) float ds[2][T];
-    // reverse only: the forward y and z of this head's channels
-    __shared__ __align__(16) float ys[DIR == 1 ? 2 : 1][DIR == 1 ? T : 1][P];
-    __shared__ __align__(16) Tin zs[DIR == 1 ? 2 : 1][DIR == 1 ? T : 1][P];
     const int lane = threadIdx.x;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int DIR = BOTH ? (int)(blockIdx.x & 1) : 0;
+    const int h = BOTH ? (int)(blockIdx.x >> 1) : (int)blockIdx.x, b = blockIdx.y;
     const int pb = lane >> 3, nb = lane & 7;
     const int64_t L = p.L;
     const int H = p.H, CH = p.CH, HP = H * P;
@@ -250,28 +251,13 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
             const bool ok = row0 + lane < L;
             cp_async<4>(&ds[buf][lane], Dh + (ok ? row0 + lane : 0), ok);
         }
-        if constexpr (DIR == 1) {
-            constexpr int ZP = P * (int)sizeof(Tin) / 16;  // 16-byte pieces of a z row
-            for (int e = lane; e < T * (P / 4); e += 32) {
-                const int rr = e / (P / 4), q = e % (P / 4);
-                const bool ok = row0 + rr < L;
-                const int64_t o = ((int64_t)b * L + (ok ? row0 + rr : 0)) * HP + (int64_t)h * P;
-                cp_async<16>(&ys[buf][rr][4 * q], p.YF + o + 4 * q, ok);
-            }
-            for (int e = lane; e < T * ZP; e += 32) {
-                const int rr = e / ZP, q = e % ZP;
-                const bool ok = row0 + rr < L;
-                const int64_t o = ((int64_t)b * L + (ok ? row0 + rr : 0)) * HP + (int64_t)h * P;
-                cp_async<16>(reinterpret_cast<unsigned char*>(&zs[buf][rr][0]) + 16 * q,
-                             reinterpret_cast<const unsigned char*>(static_cast<const Tin*>(p.z) + o) + 16 * q, ok);
-            }
-        }
         cp_async_commit();
     };
 
     const float A2 = p.A[DIR * H + h] * kLog2e;
     const float Dskip = p.Dskip[DIR * H + h];
     const float scale = p.dir_scale[DIR];
+    float* const Y = DIR == 0 ? p.YF : p.YB;
     // S[i][4q+j] = state (row 8pb + i, state 32q + 4nb + j)
     float S[8][16];
     const int64_t sbase = ((int64_t)b * H + h) * P * N;
@@ -351,12 +337,7 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
                 const int prow = 8 * pb + nb;
                 const float y = (acum * yr + Dskip * xs[buf][rr][prow]) * scale;
                 const int64_t o = ((int64_t)b * L + t) * HP + (int64_t)h * P + prow;
-                if constexpr (DIR == 0) {
-                    if (p.YF) p.YF[o] = y;  // no y for a prefix scan
-                } else {
-                    const float zv = ldf(&zs[buf][rr][0], prow);
-                    stf(static_cast<Tout*>(p.out), o, (ys[buf][rr][prow] + y) * silu(zv));
-                }
+                if (Y) Y[o] = y;  // no y for a prefix scan
             }
         }
         __syncwarp();
@@ -370,6 +351,23 @@ __global__ void __launch_bounds__(32, 8) m2_scan_kernel(const M2Params p) {
             for (int q = 0; q < 4; ++q)
                 *reinterpret_cast<float4*>(p.S_out + sbase + (8 * pb + i) * N + 32 * q + 4 * nb) =
                     make_float4(acum * S[i][4 * q], acum * S[i][4 * q + 1], acum * S[i][4 * q + 2], acum * S[i][4 * q + 3]);
+    }
+}
+
+// grid-stride over the call's batch * L * H*P outputs, 4 per thread (H*P % 4
+// == 0): out = (y_0 + y_1) * silu(z) from p.YF and p.YB.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) m2_combine_kernel(const M2Params p) {
+    const int64_t n4 = (int64_t)p.batch * p.L * p.H * kM2P / 4;
+    const float4* yf = reinterpret_cast<const float4*>(p.YF);
+    const float4* yb = reinterpret_cast<const float4*>(p.YB);
+    const Tin* z = static_cast<const Tin*>(p.z);
+    Tout* out = static_cast<Tout*>(p.out);
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n4; i += (int64_t)gridDim.x * 256) {
+        const float4 a = yf[i], c = yb[i];
+        const float s[4] = {a.x + c.x, a.y + c.y, a.z + c.z, a.w + c.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) stf(out, 4 * i + u, s[u] * silu(ldf(z, 4 * i + u)));
     }
 }
 

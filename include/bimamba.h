@@ -272,7 +272,8 @@ typedef struct {
 } bimamba2_inputs_t;
 
 /* Bytes of device workspace bimamba2_layer_fwd needs (fp32 conv features of
- * both directions, step sizes, the forward output); 0 for invalid sizes. */
+ * both directions, step sizes, the forward and reverse outputs, the tensor
+ * path's C/B tiles); 0 for invalid sizes. */
 size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state);
 
 /* The full-sequence Mamba-2 mixer.  out: [batch][L][nheads*headdim] of
