@@ -821,6 +821,8 @@ def run_reference(args, rank, world):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     if args.workload in ("mamba2", "mamba2_long"):
         return run_reference_mamba2(args, w, world, dev)
+    if args.workload == "proj":
+        return run_reference_proj(args, w, world)
     inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device=dev)
     threads = oracle.max_threads()
     per_step = min(30.0, 150.0 / max(1, args.steps + args.warmup))
@@ -851,6 +853,47 @@ def run_reference(args, rank, world):
                    "d_state": w.d_state, "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def run_reference_proj(args, w, world):
+    """The reference arm for the neighbours: the fp64 oracle (AdaLN and both
+    projections, numpy) on a sample of token rows, scaled to all rows."""
+    import oracle
+    dm, D = w.extra["d_model"], w.d_inner
+    M = w.batch * w.L
+    c = W.make_proj_case(1, 256, dm, D, w.d_state, seed=w.seed)
+    per_step = min(30.0, 150.0 / max(1, args.steps + args.warmup))
+
+    def one(rows):
+        h, y = c["h"][:, :rows], c["y"][:, :rows]
+        a = oracle.adaln(h, c["gamma"], c["beta"])
+        oracle.in_proj(a, c["w_in"], D)
+        oracle.out_proj(y, c["w_out"])
+
+    t0 = time.perf_counter()
+    one(16)
+    t1 = time.perf_counter() - t0
+    rows = int(max(16, min(256, 16 * per_step / max(t1, 1e-3))))
+    for _ in range(args.warmup):
+        one(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one(rows)
+    secs = (time.perf_counter() - t0) / args.steps * M / rows
+    value = M / secs / 1e6
+    threads = oracle.max_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": D, "d_state": w.d_state,
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {M} token rows per step (numpy fp64), scaled by {M}/{rows}"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
