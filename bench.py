@@ -60,6 +60,7 @@ NCU_TRAFFIC = {
     ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1414.2e6,
     ("block_cached_b16_P65536_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
     ("block_cached_b16_P4096_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
+    ("proj_1p3b_b8_L2048_dmodel2048_D4096_bf16", "gemm_bf16_persistent_kernel (input projection)"): 1960.9e6,
 }
 
 
