@@ -24,8 +24,9 @@ Per rank, in order (all arithmetic in the CUDA library):
      entering states, then ``bimamba_layer_fwd_carry`` from them; the
      segment's rows of that output are the result.
 
-Two collectives, both all-gathers of a few hundred KB: the exchange step of
-a scan split along the sequence, nothing else.  ``sharded_layer_fwd`` runs
+The collectives are three small all-gathers (the halo rows, the final
+states, the step-size sums: a few hundred KB in all), the exchange step of a
+scan split along the sequence, and nothing else.  ``sharded_layer_fwd`` runs
 the steps under ``torch.distributed``; ``emulate_sharded`` runs them for all
 segments in one process (one device), with stacking in place of the
 collectives -- the same functions, so the single-device tests check the
