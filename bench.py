@@ -717,7 +717,7 @@ def run_sharded(args, w, bm, rank, world, dev, stream):
             torch.cuda.empty_cache()
         res["emulated_ranks"] = proj
         res["emulated_note"] = ("one rank's segment of L/R tokens timed on this GPU; projected_value = L / that "
-                                "time, before the two all-gathers (a few hundred KB each)")
+                                "time, before the three all-gathers (a few hundred KB in all)")
     return res
 
 
