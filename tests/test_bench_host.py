@@ -83,3 +83,22 @@ def test_roofline_fields():
     assert r["achieved"] == pytest.approx(ops / 1e-3 / 1e9, rel=1e-4)
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], abs=1e-4)
     assert bench.roofline(ops, 1.0, None, "layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel")["traffic"] > 0
+
+
+def test_every_workload_resolves_and_names_its_sizes():
+    for wl in ("layer", "long", "block", "sweep", "decode", "decode_mamba2", "mamba2", "mamba2_long", "sharded",
+               "proj"):
+        w = bench.workload_of(bench.parse_args(["--workload", wl]))
+        assert w.batch >= 1 and w.L >= 1 and w.d_inner >= 1
+        assert f"b{w.batch}" in w.name or "b8" in w.name or "b16" in w.name
+    assert bench.workload_of(bench.parse_args(["--workload", "sharded"])).L == 262144
+    assert bench.workload_of(bench.parse_args(["--workload", "proj"])).extra["d_model"] == 2048
+
+
+def test_tensor_roofline_and_flop_counts():
+    # dual form: 4 products per chunk, head and direction
+    Q, N, P = 128, 128, 32
+    per_chunk = 2.0 * (Q * Q * N + Q * P * N + N * P * Q + Q * P * Q)
+    assert bench.mamba2_ssd_flops(8, 2048, 120, P, N) == per_chunk * 16 * 120 * 8 * 2
+    r = bench.roofline_tensor(1.0e12, 1.0, "w", "k")  # 1 TFLOP in 1 ms = 1000 TFLOP/s
+    assert r["achieved"] == 1000.0 and abs(r["frac"] - 1000.0 / r["peak"]) < 1e-4 and r["bound"] == "tensor"
