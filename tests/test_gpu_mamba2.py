@@ -175,6 +175,25 @@ def test_full_size_sampled_heads(bm):
         assert U.bf16_out_ok(U.to_cpu64(out16.index_select(-1, idx)), want)
 
 
+def test_long_batch1_sampled_heads(bm):
+    """b 1, L 16,384, 120 heads (the clustered launch form of the tensor path:
+    both directions at once, meeting halfway), the bench's mamba2_long
+    configuration: three heads against the oracle on both paths."""
+    w = W.MAMBA2_LONG[16384]
+    H = w.extra["nheads"]
+    inp, par = W.make_mamba2_case(w.batch, w.L, H, P, N, "bf16", w.seed, device="cuda")
+    heads = [0, 60, H - 1]
+    si, sp, xch = U.head_subset(inp, par, heads)
+    want = oracle.mamba2_layer_fwd(si, sp)
+    idx = torch.as_tensor(xch, device="cuda")
+    for flags, tol in PATHS.values():
+        out32 = bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out_dtype=torch.float32, flags=flags)
+        torch.cuda.synchronize()
+        assert bm.bimamba_device_error() == 0
+        err = U.normwise(U.to_cpu64(out32.index_select(-1, idx)), want)
+        assert err <= tol, (flags, err)
+
+
 def test_workspace_too_small_is_rejected(bm):
     inp, par = W.make_mamba2_case(1, 16, 2, P, N, "bf16", seed=1, device="cuda")
     ws = torch.empty(1024, dtype=torch.uint8, device="cuda")

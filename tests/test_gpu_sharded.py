@@ -86,3 +86,19 @@ def test_zero_carries_change_nothing(bm, family):
     torch.cuda.synchronize()
     assert torch.equal(got, plain)
     assert torch.isfinite(h_out).all() and (ds > 0).all()
+
+
+def test_full_size_sampled_channels(bm):
+    """The bench's sharded workload (b 1, L 262,144, D 4096, bf16) cut into 4
+    segments of 65,536 (one rank's share at 4 GPUs), all channels on the GPU;
+    16 sampled channels against the oracle's full-sequence layer."""
+    w = W.SHARDED_SEQ
+    inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed, device="cuda")
+    got = SH.emulate_sharded(inp, par, [w.L // 4] * 4)
+    torch.cuda.synchronize()
+    assert bm.bimamba_device_error() == 0
+    chans = U.sample_channels(w.d_inner, 16, seed=3)
+    si, sp = U.channel_subset(inp, par, chans)
+    want = oracle.layer_fwd(si, sp)
+    idx = torch.as_tensor(chans, device="cuda")
+    assert U.bf16_out_ok(U.to_cpu64(got.index_select(-1, idx)), want)
