@@ -394,3 +394,37 @@ def test_neighbours_reject():
     assert L.bimamba_out_proj(FAKE, FAKE, 2, 8, 72, 32, FAKE, None) == bm.BIMAMBA_ERR_UNSUPPORTED
     assert L.bimamba_out_proj(FAKE, FAKE, 2, 8, 64, 36, FAKE, None) == bm.BIMAMBA_ERR_UNSUPPORTED
     assert L.bimamba_out_proj(FAKE, FAKE + 4, 2, 8, 64, 32, FAKE, None) == bm.BIMAMBA_ERR_MISALIGNED
+
+
+def test_header_serves_a_plain_c_program(tmp_path):
+    """A C99 program includes the header, links the library and calls it with
+    no torch and no C++: status strings, the ABI version, workspace queries
+    and a rejected call (nothing runs on a GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "bimamba.h"
+int main(void) {
+    if (bimamba_abi_version() != 1) return 1;
+    if (strlen(bimamba_status_string(BIMAMBA_ERR_INVALID_ARG)) == 0) return 2;
+    if (bimamba_workspace_bytes(8, 2048, 4096, 16, 0) != (size_t)8 * 2048 * 4096 * 4) return 3;
+    if (bimamba2_workspace_bytes(0, 10, 4, 32, 128) != 0) return 4;
+    /* a call with no inputs is rejected before anything is launched */
+    if (bimamba_layer_fwd(NULL, NULL, NULL, BIMAMBA_BF16, 1, 16, 32, 16, 0, NULL, 0, NULL) !=
+        BIMAMBA_ERR_INVALID_ARG) return 5;
+    printf("ok\n");
+    return 0;
+}
+""")
+    lib_dir = os.path.dirname(bm._LIB_PATH)
+    exe = tmp_path / "use_abi"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-L", lib_dir,
+                    "-lbimamba", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
