@@ -1,7 +1,6 @@
 """The block-cached decoding schedule on the host: which calls, in which
 order, and when each layer commits (a recording stand-in for the binding;
 no kernel runs)."""
-import types
 
 import torch
 

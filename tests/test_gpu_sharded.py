@@ -3,7 +3,6 @@ carry composition run through the C ABI (bimamba_layer_fwd_carry,
 bimamba_compose_carries), the collectives replaced by stacking
 (sharded.emulate_sharded, the same phase functions as the distributed path);
 the joined output against the fp64 oracle's full-sequence layer."""
-import numpy as np
 import pytest
 import torch
 
