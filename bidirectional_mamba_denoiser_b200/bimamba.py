@@ -118,6 +118,8 @@ def _load():
     lib.bimamba2_block_step.argtypes = [ctypes.POINTER(FwdState2), ctypes.POINTER(Inputs2), I64, ctypes.POINTER(Params2),
                                         P, I, I, I, I, I, ctypes.POINTER(FwdState2), U, P, SZ, P]
     lib.bimamba2_block_step.restype = I
+    lib.bimamba_features.argtypes = [ctypes.POINTER(Inputs), ctypes.POINTER(Params), I, I64, I, P, P, P]
+    lib.bimamba_features.restype = I
     lib.bimamba_status_string.argtypes = [I]
     lib.bimamba_status_string.restype = ctypes.c_char_p
     lib.bimamba_abi_version.restype = I
@@ -210,6 +212,24 @@ def bimamba_layer_fwd(x, z, dt, B, C, params: dict, out=None, out_dtype=None, fl
     if rc != BIMAMBA_OK:
         raise BimambaError("bimamba_layer_fwd", rc)
     return out
+
+
+def bimamba_features(x, dt, params: dict, stream=None):
+    """The layer's per-token features (diagnostic): x [b, L, D], dt [2, b, L, D]
+    (or a (fwd, rev) pair).  Returns (u, delta), each [2, b, L, D] fp32."""
+    b, L, D = x.shape
+    u = torch.empty(2, b, L, D, device=x.device, dtype=torch.float32)
+    delta = torch.empty_like(u)
+    dt0, dt1 = _pair(dt)
+    inp = Inputs()
+    inp.x = _ptr(x)
+    inp.dt[0], inp.dt[1] = _ptr(dt0), _ptr(dt1)
+    inp.dtype = _dtype_code(x.dtype)
+    par = make_params(params)
+    rc = lib.bimamba_features(ctypes.byref(inp), ctypes.byref(par), b, L, D, _ptr(u), _ptr(delta), _stream(stream))
+    if rc != BIMAMBA_OK:
+        raise BimambaError("bimamba_features", rc)
+    return u, delta
 
 
 def _dir_pair(t):

@@ -56,15 +56,28 @@ __device__ __forceinline__ float silu(float v) {
     return v * rcp_approx(1.f + ex2_approx(-v * kLog2e));
 }
 
-// softplus(v) = log(1 + e^v) = log2(1 + e^v) * ln 2; above 20 the result is
-// v to fp32 precision.  For small steps the rounding of 1 + e^v and the
-// absolute error of the approximate log2 give a relative error of the step
-// size of order 1e-4 at delta ~ 1e-3; through the scan that moves the output
-// by ~1e-6 of its largest value, far inside the fp32 and bf16 tolerances.
+// softplus(v) = log(1 + e^v), with e = e^v from one MUFU exp2, in three
+// ranges so that the step size keeps its relative accuracy however small:
+//  * e <= 1/16: log1p(e) by its alternating Taylor series
+//      e - e^2/2 + e^3/3 - e^4/4 + e^5/5 - e^6/6
+//    (Horner, FP32 pipe).  The first omitted term bounds the truncation by
+//    e^6/7 <= 8.5e-9 relative.  Forming 1 + e in fp32 would instead round
+//    away everything below 2^-24, which is all of e once v < -17.
+//  * 1/16 < e, v <= 20: log2(1 + e) * ln 2 (MUFU lg2).  The result is at
+//    least log(17/16) = 0.061 here, so the absolute error of the approximate
+//    log2 and the rounding of 1 + e stay a few 1e-6 of it.
+//  * v > 20: v (the remainder log1p(e^-v) < 2.1e-9 is below v's half ulp).
+// e^-inf = 0 makes softplus(-inf) exactly 0.
 __device__ __forceinline__ float softplus(float v) {
     const float e = ex2_approx(v * kLog2e);
+    float t = fmaf(e, -1.f / 6.f, 1.f / 5.f);
+    t = fmaf(e, t, -0.25f);
+    t = fmaf(e, t, 1.f / 3.f);
+    t = fmaf(e, t, -0.5f);
+    t = fmaf(e, t, 1.f);
+    const float series = e * t;
     const float via_log = lg2_approx(1.f + e) * kLn2;
-    return (v > 20.f) ? v : via_log;
+    return (v > 20.f) ? v : (e <= 0.0625f ? series : via_log);
 }
 
 // Packed two-lane fp32 arithmetic (sm_100a f32x2 instructions, round to
@@ -523,6 +536,42 @@ __global__ void __launch_bounds__(WPB * 32) block_kernel(const KParams p) {
                 stf(OUT, idx, y * silu(ldf(Z, idx)));
             }
         }
+    }
+}
+
+// ---------------------------------------------------------------- features
+
+// The per-token features of the layer written out (a diagnostic: the layer
+// kernels keep them in registers): u_r = silu(conv_r(x)) and
+// delta_r = softplus(dt_r + bias_r), with the conv accumulated in the same
+// order (bias, then taps 0..3) and the same silu / softplus as the scans.
+// One thread per (direction, row, token, channel); u, delta [2][batch][L][D].
+template <typename Tin>
+__global__ void __launch_bounds__(256) features_kernel(const Tin* __restrict__ x, const Tin* __restrict__ dt0,
+                                                       const Tin* __restrict__ dt1, const float* __restrict__ conv_w,
+                                                       const float* __restrict__ conv_b,
+                                                       const float* __restrict__ dt_bias, int batch, int64_t L,
+                                                       int D, float* __restrict__ u, float* __restrict__ delta) {
+    const int64_t per_dir = (int64_t)batch * L * D;
+    const int64_t total = 2 * per_dir;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int r = i >= per_dir ? 1 : 0;
+        const int64_t e = i - r * per_dir;  // (b, t, d) flat
+        const int d = (int)(e % D);
+        const int64_t bt = e / D;
+        const int64_t t = bt % L;
+        const int64_t rowbase = (bt - t) * D;  // element index of (b, 0, 0)
+        const int64_t rd = (int64_t)r * D + d;
+        float cv = conv_b ? conv_b[rd] : 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int64_t src = r == 0 ? t - 3 + k : t + 3 - k;
+            const float xv = (src >= 0 && src < L) ? ldf(x, rowbase + src * D + d) : 0.f;
+            cv = fmaf(conv_w[rd * 4 + k], xv, cv);
+        }
+        u[i] = silu(cv);
+        delta[i] = softplus(ldf(r == 0 ? dt0 : dt1, e) + dt_bias[rd]);
     }
 }
 

@@ -197,13 +197,19 @@ int bimamba_compose_carries(const float *h_out_all, const float *delta_sum_all, 
  * exits.  It therefore accepts batch * L * d_inner <= 16,777,216 (the
  * workspace bimamba_workspace_bytes reports must fit in 64 MiB) and returns
  * BIMAMBA_ERR_WORKSPACE above that.  It allocates and frees nothing.
- *   The first call on a device looks up the scratch array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  All calls on a device share the one array: the
- * kernel writes every scratch value before reading it, so nothing needs
- * clearing between calls, but two calls whose kernels overlap on the GPU
- * (other streams, or other host threads) race on it and give undefined
- * output.  Other arguments, checks and errors: as bimamba_layer_fwd. */
+ *   The first call in a CUDA context looks up the scratch array's device
+ * address (cudaGetSymbolAddress, with the device current) and caches it for
+ * that context; a context created anew (after cudaDeviceReset, say) looks it
+ * up again.  That first lookup may load the library's module into the
+ * context, which reserves the 64 MiB and may synchronise the device: make
+ * one call on each device before any stream capture or latency-sensitive
+ * work.  All calls on a device share the one array: the kernel writes every
+ * scratch value before reading it, so nothing needs clearing between calls,
+ * but two calls whose kernels overlap on the GPU (other streams, or other
+ * host threads) race on it and give undefined output.  Other arguments,
+ * checks and errors: as bimamba_layer_fwd, in the same order, the workspace
+ * check last (a problem too large for the scratch returns
+ * BIMAMBA_ERR_WORKSPACE only once every other argument has passed). */
 int bimamba_layer_fwd_noalloc(const bimamba_inputs_t *in, const bimamba_params_t *p,
                               void *out, bimamba_dtype_t out_dtype,
                               int batch, int64_t L, int d_inner, int d_state, unsigned flags,
@@ -374,6 +380,19 @@ int bimamba_in_proj(const void *a, const void *w_in, int batch, int64_t L, int d
  * One kernel launch. */
 int bimamba_out_proj(const void *y, const void *w_out, int batch, int64_t L, int d_inner, int d_model, void *out,
                      void *cuda_stream);
+
+/* The per-token features the layer computes before its scans, written out
+ * for inspection (a diagnostic: the layer kernels keep them in registers and
+ * never store them).  With the definitions at the top of this header:
+ *   u      [2][batch][L][d_inner] fp32 out: u_r[t] = silu(conv_r(x)[t])
+ *   delta  [2][batch][L][d_inner] fp32 out: delta_r[t] = softplus(dt_r[t] + dt_bias[r][d])
+ * computed by the same device code the layer, prefix and block-step kernels
+ * inline (conv accumulated bias first, then taps 0..3; the same silu and
+ * softplus).  Reads in->x, in->dt[0], in->dt[1] (z, B, C may be NULL) and
+ * p->conv_w, p->conv_b, p->dt_bias.  Pointers aligned to their element size.
+ * One kernel launch. */
+int bimamba_features(const bimamba_inputs_t *in, const bimamba_params_t *p, int batch, int64_t L, int d_inner,
+                     float *u, float *delta, void *cuda_stream);
 
 /* Read (and, if reset != 0, clear) the error word of the current device.
  * Kernels never wait without bound: a wait for a tile that gives up after
