@@ -97,7 +97,9 @@ def _layer(inp=None, par=None, out=FAKE + 0x20000, out_dtype=bm.BIMAMBA_BF16, ba
     (dict(flags=0x4), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_CHUNK_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
-    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
+    # the split-state family (3) runs 32- or 64-token chunks and 1 or 2 warps per direction
+    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT | 1 << bm.BIMAMBA_CHUNK_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
+    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT | 4 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY), bm.BIMAMBA_ERR_INVALID_ARG),
     (dict(out_dtype=7), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(inp=NULL), bm.BIMAMBA_ERR_INVALID_ARG),
@@ -428,3 +430,63 @@ int main(void) {
                     "-lbimamba", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_scratch_address_cache_is_keyed_by_context(tmp_path):
+    """The no-allocation entry point caches its scratch array's device address
+    per CUDA context.  A context destroyed and created anew (same device, new
+    context id) must miss the cache, so the address is looked up again; the
+    cache's own header is compiled here into a small C++ program."""
+    import shutil
+    import subprocess
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    csrc = os.path.join(os.path.dirname(bm._LIB_PATH), "csrc")
+    src = tmp_path / "cache.cc"
+    src.write_text(r"""
+#include <stdio.h>
+#include "context_cache.h"
+using bimamba::ContextAddressCache;
+int main() {
+    ContextAddressCache<4> c;
+    int a, b, d;
+    if (c.find({0, 7})) return 1;
+    c.put({0, 7}, &a);
+    if (c.find({0, 7}) != &a) return 2;
+    if (c.find({0, 8})) return 3;            /* same device, new context: miss */
+    if (c.find({1, 7})) return 4;            /* other device: miss */
+    c.put({0, 8}, &b);                       /* the new context's address */
+    if (c.find({0, 8}) != &b || c.find({0, 7}) != &a) return 5;
+    c.put({0, 8}, &d);                       /* an entry is replaced, not duplicated */
+    if (c.find({0, 8}) != &d) return 6;
+    for (unsigned long long id = 100; id < 110; ++id) c.put({2, id}, &a);  /* overflow: oldest evicted */
+    if (c.find({2, 109}) != &a) return 7;
+    if (c.find({2, 100})) return 8;
+    printf("ok\n");
+    return 0;
+}
+""")
+    exe = tmp_path / "cache"
+    subprocess.run([cxx, "-std=c++17", "-Wall", "-Werror", "-I", csrc, str(src), "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_features_rejects():
+    L = bm.lib
+    inp, par = _inputs(), _params()
+    assert L.bimamba_features(None, ctypes.byref(par), 2, 8, 32, FAKE, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_features(ctypes.byref(inp), None, 2, 8, 32, FAKE, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_features(ctypes.byref(inp), ctypes.byref(par), 0, 8, 32, FAKE, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_features(ctypes.byref(inp), ctypes.byref(par), 2, 8, 32, None, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_INVALID_ARG
+    assert L.bimamba_features(ctypes.byref(inp), ctypes.byref(par), 2, 8, 32, FAKE + 2, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_MISALIGNED
+    bad = _inputs()
+    bad.dtype = 9
+    assert L.bimamba_features(ctypes.byref(bad), ctypes.byref(par), 2, 8, 32, FAKE, FAKE + 0x100, None) == \
+        bm.BIMAMBA_ERR_UNSUPPORTED
