@@ -5,10 +5,12 @@
                   [--workload layer|long|block|sweep] [--L L]
 
 Workloads (synthetic seeded inputs, bf16 I/O, fp32 state, d_state 16):
-  layer  (default) one layer call at batch 8, L 2048, d_inner 4096 -- the 1.3B
-         layer shape; a step is one bimamba_layer_fwd (one kernel launch:
-         conv, softplus, both scan directions, D skip, sum and gate)
-  long   the same at batch 1 and L = --L (default 65536)
+  long   (default) one layer call at batch 1, d_inner 4096, L = --L (default
+         65536): the layer throughput against sequence length; a step is one
+         bimamba_layer_fwd (one kernel launch: conv, softplus, both scan
+         directions, D skip, sum and gate).  The line also carries the same
+         measurement at L = 4096, 16384, 65536 and 131072 ("l_sweep")
+  layer  the same at batch 8, L 2048 -- the 1.3B layer shape
   block  block-cached decoding at batch 16, d_inner 4096: the forward state of
          a 65536-token prefix is built once, then a step is one
          bimamba_block_step over a 32-token block (commit every 128th step);
@@ -71,13 +73,16 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["layer", "long", "block", "sweep", "decode", "decode_mamba2", "mamba2",
-                                           "mamba2_long", "sharded", "proj"], default="layer")
-    ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block")
+                                           "mamba2_long", "sharded", "proj"], default="long")
+    ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block/decode/decode_mamba2")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
     ap.add_argument("--family", type=int, default=0, help="kernel family: 0 auto, 1 chunked, 2 per-token fused")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-l-sweep", action="store_true", help="long: skip the per-L lines")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="long: scan the sequence as this many segments side by side, with carries (two passes)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     return ap.parse_args(argv)
 
@@ -85,10 +90,12 @@ def parse_args(argv=None):
 def workload_of(args) -> W.Workload:
     if args.workload == "layer":
         return W.LAYER_1P3B
-    if args.workload == "decode":
-        return W.BLOCK_DECODE
-    if args.workload == "decode_mamba2":
-        return W.BLOCK_DECODE_M2
+    if args.workload in ("decode", "decode_mamba2"):
+        w = W.BLOCK_DECODE if args.workload == "decode" else W.BLOCK_DECODE_M2
+        if args.L:  # a shorter prompt (same block steps)
+            return W.Workload(w.name.replace(f"_P{w.extra['prefix']}_", f"_P{args.L}_"), w.batch, w.L, w.d_inner,
+                              w.d_state, w.dtype, w.seed, extra={**w.extra, "prefix": args.L})
+        return w
     if args.workload == "mamba2":
         return W.MAMBA2_1P3B
     if args.workload == "sharded":
@@ -135,6 +142,26 @@ def load_peaks():
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def pool_size(input_bytes_per_set: int) -> int:
+    """Distinct input sets a step cycles through so that the sets' total
+    exceeds twice the L2 (each call's inputs then come from HBM)."""
+    return max(2, -(-2 * L2_BYTES // max(1, input_bytes_per_set)) + 1)
 
 
 # ---------------------------------------------------------------- ranks
@@ -305,6 +332,16 @@ def roofline(mufu_ops: float, launch_ms: float, clocks, workload: str, kernel: s
             "peak_source": f"148 SMs x 16 MUFU lanes/clk x {mhz:.0f} MHz", "kernel": kernel}
 
 
+def roofline_hbm(bytes_per_call: float, call_ms: float, workload: str, kernel: str):
+    """HBM roof: algorithmic bytes per call over its time, against the
+    measured copy bandwidth."""
+    peak, src = load_peaks()
+    achieved = bytes_per_call / (call_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get((workload, kernel)),
+            "peak_source": f"{src} HBM copy bandwidth", "kernel": kernel}
+
+
 def hbm_fraction(bytes_per_launch: float, launch_ms: float):
     peak, src = load_peaks()
     achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
@@ -349,16 +386,94 @@ def kernel_name(w: W.Workload, args) -> str:
     return "fused_layer_kernel" if fam == 2 else "layer_tma_kernel"
 
 
+def layer_input_bytes(batch: int, L: int, D: int, N: int, esz: int) -> int:
+    """Bytes of one layer call's inputs: x, z, dt_f, dt_b and B_f, C_f, B_b, C_b."""
+    return batch * L * (D * 4 * esz + 4 * N * esz)
+
+
+def l_sweep(args, bm, rank, world, dev, stream, flags, lengths=(4096, 16384, 65536, 131072)):
+    """The layer at batch 1, d_inner 4096 over sequence lengths: per L, two
+    rotating input sets (each far larger than L2), CUDA-event time per call,
+    Mtokens/s, algorithmic HBM fraction and MUFU fraction."""
+    rows = []
+    for L in lengths:
+        w = W.LONG_SEQ.get(L) or W.Workload(f"long_b1_L{L}_D4096_bf16", 1, L, 4096, 16, "bf16", 2)
+        sets = [W.make_case(w.batch, L, w.d_inner, w.d_state, w.dtype, w.seed + 1000 * i + rank, device=dev)
+                for i in range(2)]
+        out = torch.empty(w.batch, L, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
+        ws = torch.empty(bm.bimamba_workspace_bytes(w.batch, L, w.d_inner, w.d_state), device=dev,
+                         dtype=torch.uint8)
+
+        def step(i):
+            inp, par = sets[i % 2]
+            bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, out=out, flags=flags,
+                                 workspace=ws, stream=stream)
+
+        steps = max(5, min(args.steps, 50 * 65536 // L))
+        ms, clocks = timed(step, steps, max(3, args.warmup), world, dev, stream)
+        call_ms = max_over_ranks(ms, world) / steps
+        elems = w.batch * L * w.d_inner
+        rows.append({"L": L, "ms_per_call": round(call_ms, 4),
+                     "Mtokens_s": round(whole_job_rate(w.batch * L, world, call_ms / 1e3), 4),
+                     "hbm_frac": hbm_fraction(layer_bytes(w.batch, L, w.d_inner, w.d_state, 2), call_ms)["frac"],
+                     "mufu_frac": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name,
+                                           kernel_name(w, args))["frac"],
+                     "steps": steps, "sm_mhz": (clocks or {}).get("sm_mhz")})
+        del sets, out, ws
+        torch.cuda.empty_cache()
+    return rows
+
+
+def run_chunked(args, w, bm, rank, world, dev, stream):
+    """long --segments k: the batch-1 layer scanned as k segments side by side
+    (sharded.ChunkedLayer: a pass from zero, the carry composition, a second
+    pass), for comparison with the single-pass kernels.  The extended
+    segments are built before the timed region."""
+    from bidirectional_mamba_denoiser_b200 import sharded as SH
+    ops = SH.CudaOps(flags_of(args, bm))
+    plans = []
+    for i in range(2):
+        inp, par = W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed + 1000 * i + rank, device=dev)
+        plans.append(SH.ChunkedLayer(inp, par, args.segments, ops))
+        del inp
+    torch.cuda.empty_cache()
+
+    def step(i):
+        plans[i % 2].run()
+
+    ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
+    ms_max = max_over_ranks(ms, world)
+    call_ms = ms / args.steps
+    elems = w.batch * w.L * w.d_inner
+    return {
+        "value": whole_job_rate(w.batch * w.L * args.steps, world, ms_max / 1e3),
+        "ms_per_step": ms_max / args.steps,
+        "gpu_launches": args.steps * (2 + args.segments + 2),
+        "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, "fused_layer_kernel x 2 passes"),
+        "hbm": hbm_fraction(layer_bytes(w.batch, w.L, w.d_inner, w.d_state, 2), call_ms),
+        "clocks": clocks,
+        "schedule": f"{args.segments} segments of {w.L // args.segments} tokens as batch rows: pass from zero, "
+                    f"carry composition, pass from the carries (MUFU fraction counts one pass's work)",
+    }
+
+
 def run_layer_like(args, w, bm, rank, world, dev, stream):
-    """layer / long / sweep: steps of bimamba_layer_fwd."""
+    """layer / long / sweep: steps of bimamba_layer_fwd.  The sweep cycles its
+    48 layer calls through a pool of input sets (each set with its own
+    parameters) whose total exceeds twice the L2; the kernel's cost does not
+    depend on the values, so this stands in for fresh inputs per layer and
+    step."""
     flags = flags_of(args, bm)
-    nsets = w.extra.get("layers", 2) if args.workload == "sweep" else 2
+    if args.workload == "sweep":
+        nsets = pool_size(layer_input_bytes(w.batch, w.L, w.d_inner, w.d_state, 2))
+        calls = w.extra["layers"]
+    else:
+        nsets, calls = 2, 1
     sets = [W.make_case(w.batch, w.L, w.d_inner, w.d_state, w.dtype, w.seed + 1000 * i + rank, device=dev)
             for i in range(nsets)]
     out = torch.empty(w.batch, w.L, w.d_inner, device=dev, dtype=W.torch_dtype(w.dtype))
     ws = torch.empty(bm.bimamba_workspace_bytes(w.batch, w.L, w.d_inner, w.d_state), device=dev,
                      dtype=torch.uint8)
-    calls = nsets if args.workload == "sweep" else 1
 
     def step(i):
         for c in range(calls):
@@ -381,6 +496,8 @@ def run_layer_like(args, w, bm, rank, world, dev, stream):
     if args.workload == "sweep":
         res["sequence_mixer_s"] = round(call_ms * w.extra["layers"] * w.extra["steps"] / 1e3, 4)
         res["sequence_note"] = f"{w.extra['layers']} layers x {w.extra['steps']} steps x {call_ms:.4f} ms per call"
+        res["input_pool"] = (f"{nsets} input sets of {layer_input_bytes(w.batch, w.L, w.d_inner, w.d_state, 2)} "
+                             f"bytes, cycled by the 48 layer calls (total > 2 x L2)")
 
     if not args.no_e2e:
         inp, par = sets[0]
@@ -399,9 +516,14 @@ def run_layer_like(args, w, bm, rank, world, dev, stream):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp, par = sets[0]
         v, nch, secs, thr = oracle_sample_rate(w, inp, par, args.cpu_budget)
-        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "cpu_model": cpu_model(),
+                               "kind": "oracle",
                                "sample": f"{nch} of {w.d_inner} channels x {w.batch} batch rows x L={w.L} "
                                          f"({secs:.1f} s), scaled by {w.d_inner}/{nch}"}
+    if args.workload == "long" and not args.no_l_sweep:
+        del sets
+        torch.cuda.empty_cache()
+        res["l_sweep"] = l_sweep(args, bm, rank, world, dev, stream, flags)
     return res
 
 
@@ -560,8 +682,15 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
         "recurrence_flops_per_token": int(flops / tokens),
     }
     if tensor_path:
-        res["roofline"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
-                                          "m2_prep + m2_ssd_kernel (both directions, clusters of 2)")
+        # By the method's own work the call is bound by HBM: its algorithmic
+        # bytes take longer at the measured copy bandwidth than its recurrence
+        # flops at the tensor peak.  The dual form's executed MMA flops (a
+        # dense equivalent that also multiplies the masked zeros) are reported
+        # beside it.
+        res["roofline"] = roofline_hbm(mamba2_bytes(w.batch, w.L, H, P, N), call_ms, w.name,
+                                       "m2_prep + m2_ssd_kernel (both directions)")
+        res["tensor_executed"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
+                                                 "m2_ssd_kernel executed MMA")
         res["fp32_equivalent"] = roofline_fma(flops, call_ms, clocks, w.name, "recurrence-equivalent")
     else:
         res["roofline"] = roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel")
@@ -581,7 +710,8 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp, par = sets[0]
         v, nh, secs, thr = mamba2_oracle_rate(w, inp, par, args.cpu_budget)
-        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": thr, "cpu_model": cpu_model(),
+                               "kind": "oracle",
                                "sample": f"{nh} of {H} heads x {w.batch} batch rows x L={w.L} ({secs:.1f} s), "
                                          f"scaled by {H}/{nh}"}
     return res
@@ -784,6 +914,8 @@ def run_ours(args, rank, world, local):
         res = run_sharded(args, w, bm, rank, world, dev, stream)
     elif args.workload == "proj":
         res = run_proj(args, w, bm, rank, world, dev, stream)
+    elif args.workload == "long" and args.segments > 1:
+        res = run_chunked(args, w, bm, rank, world, dev, stream)
     else:
         res = run_layer_like(args, w, bm, rank, world, dev, stream)
     if rank == 0:
@@ -852,7 +984,8 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                    "d_state": w.d_state, "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "cpu_model": cpu_model(),
+                         "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -893,7 +1026,8 @@ def run_reference_proj(args, w, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": D, "d_state": w.d_state,
                    "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "cpu_model": cpu_model(),
+                         "kind": "oracle",
                          "sample": f"{rows} of {M} token rows per step (numpy fp64), scaled by {M}/{rows}"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -932,7 +1066,8 @@ def run_reference_mamba2(args, w, world, dev):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.d_inner,
                    "d_state": w.d_state, "nheads": H, "headdim": P, "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "cpu_model": cpu_model(),
+                         "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 #include <set>
 #include <type_traits>
@@ -11,7 +12,9 @@
 #include "bimamba.h"
 #include "block_fused.cuh"
 #include "carry.cuh"
+#include "context_cache.h"
 #include "layer_fused.cuh"
+#include "layer_split.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
 #include "mamba2_ssd.cuh"
@@ -325,6 +328,50 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
     return BIMAMBA_ERR_UNSUPPORTED;
 }
 
+// ---- split-state kernel (few channels: 4 lanes x 4 states per channel)
+
+constexpr int kSNS = 3;  // pipeline stages per direction
+
+template <int T, int NWD, typename Tin>
+bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
+    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin>;
+    const bool bf = std::is_same<Tin, bf16>::value;
+    constexpr int N = bimamba::kNState;
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, T + 3);
+    ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, T);
+    for (int r = 0; r < 2; ++r) {
+        ok = ok && map3d(&m.dt[r], in->dt[r], bf, D, L, batch, Ge::CW, T);
+        ok = ok && map3d(&m.B[r], in->B[r], bf, N, L, batch, N, T);
+        ok = ok && map3d(&m.C[r], in->C[r], bf, N, L, batch, N, T);
+    }
+    return ok;
+}
+
+template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false>
+int launch_layer_split(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin>;
+    bimamba::LayerMaps maps;
+    if (!fill_split_maps<T, NWD, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, 2 * NWD * 32, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+// Chunk of the split-state kernel: the chunk field's 2 = 32 tokens, 3 = 64
+// (0 = automatic: 32); warps per direction: the lane field (1 or 2; 0 = 1).
+template <typename Tin, typename Tout>
+int layer_split_by(unsigned flags, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    const unsigned ch = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
+    const unsigned nw = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    const int t = ch == 3 ? 64 : 32;
+    if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout>(k, in, st)
+                                : launch_layer_split<32, 2, Tin, Tout>(k, in, st);
+    return t == 64 ? launch_layer_split<64, 1, Tin, Tout>(k, in, st) : launch_layer_split<32, 1, Tin, Tout>(k, in, st);
+}
+
 // ---- per-token fused kernels (many channels)
 
 // The boxes come from the kernel's own geometry, so the bytes each TMA load
@@ -352,12 +399,12 @@ bool fill_fused_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batc
     return ok;
 }
 
-template <int G, typename Tin, typename Tout, bool CARRY = false>
+template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false>
 int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::FusedGeo<G, Tin>;
+    using Ge = bimamba::FusedGeo<G, Tin, F32BC>;
     bimamba::FusedMaps maps;
     if (!fill_fused_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout, CARRY>;
+    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout, CARRY, F32BC>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -366,7 +413,14 @@ int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_
 }
 
 template <typename Tin, typename Tout>
-int fused_layer_by_group(int g, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+int fused_layer_by_group(int g, bool f32bc, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    if (f32bc) {
+        switch (g) {
+            case 2: return launch_fused_layer<2, Tin, Tout, false, true>(k, in, st);
+            case 4: return launch_fused_layer<4, Tin, Tout, false, true>(k, in, st);
+        }
+        return BIMAMBA_ERR_UNSUPPORTED;
+    }
     switch (g) {
         case 1: return launch_fused_layer<1, Tin, Tout>(k, in, st);
         case 2: return launch_fused_layer<2, Tin, Tout>(k, in, st);
@@ -509,6 +563,30 @@ int bimamba_device_error(int reset) {
     return (int)word;
 }
 
+int bimamba_features(const bimamba_inputs_t* in, const bimamba_params_t* p, int batch, int64_t L, int d_inner,
+                     float* u, float* delta, void* cuda_stream) {
+    if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !u || !delta) return BIMAMBA_ERR_INVALID_ARG;
+    if (!in || !in->x || !in->dt[0] || !in->dt[1]) return BIMAMBA_ERR_INVALID_ARG;
+    if (!dtype_ok(in->dtype)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (!p || !p->conv_w || !p->dt_bias) return BIMAMBA_ERR_INVALID_ARG;
+    const size_t a = elem_size(in->dtype);
+    if (!aligned(in->x, a) || !aligned(in->dt[0], a) || !aligned(in->dt[1], a) || !aligned(u, 4) ||
+        !aligned(delta, 4) || !aligned(p->conv_w, 4) || !aligned(p->dt_bias, 4) || !aligned(p->conv_b, 4))
+        return BIMAMBA_ERR_MISALIGNED;
+    const int64_t total = 2LL * batch * L * d_inner;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 148LL * 16);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if (in->dtype == BIMAMBA_BF16)
+        bimamba::features_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(
+            static_cast<const bf16*>(in->x), static_cast<const bf16*>(in->dt[0]),
+            static_cast<const bf16*>(in->dt[1]), p->conv_w, p->conv_b, p->dt_bias, batch, L, d_inner, u, delta);
+    else
+        bimamba::features_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
+            static_cast<const float*>(in->x), static_cast<const float*>(in->dt[0]),
+            static_cast<const float*>(in->dt[1]), p->conv_w, p->conv_b, p->dt_bias, batch, L, d_inner, u, delta);
+    return launch_status();
+}
+
 size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags) {
     (void)flags;
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || d_state != bimamba::kNState) return 0;
@@ -527,8 +605,11 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
                            BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE;
-    if (((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
-    if (((flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT) == 3) return BIMAMBA_ERR_UNSUPPORTED;
+    const bool split_family = ((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3;
+    const unsigned chunk_field = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
+    const unsigned lane_field = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
+    if (!split_family && chunk_field == 3) return BIMAMBA_ERR_UNSUPPORTED;
+    if (split_family && (chunk_field == 1 || lane_field > 2)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -567,6 +648,19 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int fam = pick_family(2LL * batch * d_inner, flags);
+    if (fam == 3) {  // the split-state kernel: TMA-fed
+        if ((flags & BIMAMBA_NO_TMA) || !tma_eligible(in, d_inner, true, true)) return BIMAMBA_ERR_UNSUPPORTED;
+        if (with_carry) {  // carries: 32-token chunks, one warp per direction (the flags' choice is not honoured)
+            if (in_bf && out_bf) return launch_layer_split<32, 1, bf16, bf16, true>(k, in, st);
+            if (in_bf) return launch_layer_split<32, 1, bf16, float, true>(k, in, st);
+            if (out_bf) return launch_layer_split<32, 1, float, bf16, true>(k, in, st);
+            return launch_layer_split<32, 1, float, float, true>(k, in, st);
+        }
+        if (in_bf && out_bf) return layer_split_by<bf16, bf16>(flags, k, in, st);
+        if (in_bf) return layer_split_by<bf16, float>(flags, k, in, st);
+        if (out_bf) return layer_split_by<float, bf16>(flags, k, in, st);
+        return layer_split_by<float, float>(flags, k, in, st);
+    }
     const bool group_ok = forced == 0 || forced == 1 || forced == 2 || forced == 4 || forced == 8;
     if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
         tma_eligible(in, d_inner, true, true)) {
@@ -577,10 +671,11 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
             return launch_fused_layer<2, float, float, true>(k, in, st);
         }
         const int gf = pick_group_fused(flags);
-        if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, k, in, st);
-        if (in_bf) return fused_layer_by_group<bf16, float>(gf, k, in, st);
-        if (out_bf) return fused_layer_by_group<float, bf16>(gf, k, in, st);
-        return fused_layer_by_group<float, float>(gf, k, in, st);
+        const bool f32bc = chunk_field == 2;  // family 2: B/C widened once per chunk
+        if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, f32bc, k, in, st);
+        if (in_bf) return fused_layer_by_group<bf16, float>(gf, f32bc, k, in, st);
+        if (out_bf) return fused_layer_by_group<float, bf16>(gf, f32bc, k, in, st);
+        return fused_layer_by_group<float, float>(gf, f32bc, k, in, st);
     }
     if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
         const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
@@ -749,22 +844,54 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[64u << 20];
 namespace {
 
 constexpr size_t kNoallocScratchBytes = sizeof(g_noalloc_scratch);
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+bimamba::ContextAddressCache<64> g_noalloc_addr;
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_entry(const char* name) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(f);
+}
+
+// Id of the current context, or false if there is none (or the driver
+// cannot tell).
+bool current_context_id(unsigned long long* id) {
+    static const CtxGetCurrentFn get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context.  It is
+// looked up with cudaGetSymbolAddress (with the device current) the first
+// time a context calls, then cached under (device, context id): a context
+// destroyed and created again gets a new id, so its module's new address is
+// looked up afresh.  Without a context id the address is looked up on every
+// call.
 int noalloc_scratch(void** addr) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BIMAMBA_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BIMAMBA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BIMAMBA_ERR_CUDA;
-        g_noalloc_addr[dev] = p;
+    unsigned long long id = 0;
+    if (current_context_id(&id)) {
+        if (void* p = g_noalloc_addr.find({dev, id})) {
+            *addr = p;
+            return BIMAMBA_OK;
+        }
     }
-    *addr = g_noalloc_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BIMAMBA_ERR_CUDA;
+    // the lookup makes the device's primary context current if none was
+    if (current_context_id(&id)) g_noalloc_addr.put({dev, id}, p);
+    *addr = p;
     return BIMAMBA_OK;
 }
 
@@ -773,14 +900,15 @@ int noalloc_scratch(void** addr) {
 extern "C" int bimamba_layer_fwd_noalloc(const bimamba_inputs_t* in, const bimamba_params_t* p, void* out,
                                          bimamba_dtype_t out_dtype, int batch, int64_t L, int d_inner,
                                          int d_state, unsigned flags, void* cuda_stream) {
-    const size_t need = bimamba_workspace_bytes(batch, L, d_inner, d_state, flags);
-    if (need == 0)  // invalid sizes: let the full entry point name the problem (nothing is launched)
+    // Invalid sizes: the full entry point names the problem without touching the GPU.
+    if (bimamba_workspace_bytes(batch, L, d_inner, d_state, flags) == 0)
         return bimamba_layer_fwd(in, p, out, out_dtype, batch, L, d_inner, d_state, flags, nullptr, 0,
                                  cuda_stream);
-    if (need > kNoallocScratchBytes) return BIMAMBA_ERR_WORKSPACE;
     void* scratch = nullptr;
     const int rc = noalloc_scratch(&scratch);
     if (rc) return rc;
+    // The full entry point runs every check in its usual order; a problem too
+    // large for the scratch fails its last one, the workspace size.
     return bimamba_layer_fwd(in, p, out, out_dtype, batch, L, d_inner, d_state, flags, scratch,
                              kNoallocScratchBytes, cuda_stream);
 }

@@ -38,7 +38,9 @@ struct FusedMaps {
     CUtensorMap C[2];   // [batch][L][16]   box {16, T, 1}
 };
 
-template <int G, typename Tin>
+// F32BC: B and C are widened to fp32 once per chunk (into a per-warp buffer)
+// instead of at every use.
+template <int G, typename Tin, bool F32BC = false>
 struct FusedGeo {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "lanes per group");
     static constexpr int T = 16;                // tokens per chunk
@@ -51,9 +53,10 @@ struct FusedGeo {
     static constexpr int BB = ((T * kNState * ESZ) + 127) & ~127;
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
     static constexpr int OWS = T * CW * 4;               // partner's y of a chunk
-    // With G == 1 every lane needs all 16 B and C of a token: they are
-    // converted to fp32 once per chunk (T x 32 floats) instead of per use.
-    static constexpr int BCF = G == 1 ? T * 2 * kNState * 4 : 0;
+    // With G == 1 every lane needs all 16 B and C of a token, and with F32BC
+    // they are wanted as fp32 anyway: they are converted once per chunk
+    // (T x 32 floats) instead of per use.
+    static constexpr int BCF = (G == 1 || F32BC) ? T * 2 * kNState * 4 : 0;
     static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF;
     static constexpr int BAR_OFF = 2 * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
@@ -92,9 +95,9 @@ __device__ __forceinline__ void load_row(const float* p, float (&v)[S]) {
     load_states<S>(p, v);
 }
 
-template <int G, typename Tin, typename Tout, int DIR, bool LAYER>
+template <int G, typename Tin, typename Tout, int DIR, bool LAYER, bool F32BC = false>
 struct FusedWarp {
-    using Ge = FusedGeo<G, Tin>;
+    using Ge = FusedGeo<G, Tin, F32BC>;
     static constexpr int T = Ge::T, NS = Ge::NS, S = Ge::S;
 
     // own channel (per-token work and output)
@@ -193,11 +196,16 @@ struct FusedWarp {
     }
 
     template <bool WITH_Y>
-    __device__ __forceinline__ float scan(int s, const Elem& e, const Tin* Bt, const Tin* Ct) {
+    __device__ __forceinline__ float scan(int s, const Elem& e, const Tin* Bt, const Tin* Ct, const float* bcf) {
         const int row = row_of(s);
         float bv[S], cvv[S];
-        load_row<S>(Bt + row * kNState + j * S, bv);
-        if constexpr (WITH_Y) load_row<S>(Ct + row * kNState + j * S, cvv);
+        if constexpr (F32BC) {
+            load_states<S>(bcf + row * 2 * kNState + j * S, bv);
+            if constexpr (WITH_Y) load_states<S>(bcf + row * 2 * kNState + kNState + j * S, cvv);
+        } else {
+            load_row<S>(Bt + row * kNState + j * S, bv);
+            if constexpr (WITH_Y) load_row<S>(Ct + row * kNState + j * S, cvv);
+        }
         float acc[G];
 #pragma unroll
         for (int q = 0; q < G; ++q) {
@@ -205,7 +213,8 @@ struct FusedWarp {
             const float uq = __shfl_sync(0xffffffffu, e.du, q, G);
             const float2 dd = make_float2(dq, dq);
             const float2 uu = make_float2(uq, uq);
-            float2 acc2 = make_float2(0.f, 0.f);
+            // two accumulator pairs: half the dependent chain of the C.h sum
+            float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
             for (int sp = 0; sp < S; sp += 2) {
                 const float2 v = mul2(dd, make_float2(A2[q][sp], A2[q][sp + 1]));
@@ -214,9 +223,9 @@ struct FusedWarp {
                 const float2 hh = fma2(ea, make_float2(h[q][sp], h[q][sp + 1]), drive);
                 h[q][sp] = hh.x;
                 h[q][sp + 1] = hh.y;
-                if constexpr (WITH_Y) acc2 = fma2(make_float2(cvv[sp], cvv[sp + 1]), hh, acc2);
+                if constexpr (WITH_Y) acc2[(sp >> 1) & 1] = fma2(make_float2(cvv[sp], cvv[sp + 1]), hh, acc2[(sp >> 1) & 1]);
             }
-            acc[q] = acc2.x + acc2.y;
+            acc[q] = (acc2[0].x + acc2[1].x) + (acc2[0].y + acc2[1].y);
         }
         if constexpr (WITH_Y)
             return group_transpose_reduce<G, 1>(acc, j);
@@ -237,10 +246,10 @@ __device__ __forceinline__ void fused_convert_bc(const Tin* Bt, const Tin* Ct, f
     for (int r = 0; r < T; ++r) bcf[r * 2 * kNState + lane] = ldf(src, r * kNState + n);
 }
 
-template <int G, typename Tin>
+template <int G, typename Tin, bool F32BC = false>
 __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char* wbase, uint64_t* full, int r,
                                             int i, int k, bool gated, int ct0, int b, int starve) {
-    using Ge = FusedGeo<G, Tin>;
+    using Ge = FusedGeo<G, Tin, F32BC>;
     if (starve) return;
     const int st = i % Ge::NS;
     unsigned char* sb = wbase + st * Ge::STAGE;
@@ -255,12 +264,12 @@ __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int G, typename Tin, typename Tout, int DIR, bool CARRY>
+template <int G, typename Tin, typename Tout, int DIR, bool CARRY, bool F32BC>
 __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, const KParams& p, unsigned char* base,
                                                       int lane) {
-    using Ge = FusedGeo<G, Tin>;
+    using Ge = FusedGeo<G, Tin, F32BC>;
     constexpr int T = Ge::T, NS = Ge::NS, S = Ge::S;
-    using Wp = FusedWarp<G, Tin, Tout, DIR, true>;
+    using Wp = FusedWarp<G, Tin, Tout, DIR, true, F32BC>;
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
     float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS);
@@ -290,7 +299,8 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     float dsum = 0.f;  // step sizes of the own channel so far
     if (lane == 0)
         for (int i = 0; i < NS && i < nc; ++i)
-            fused_issue<G, Tin>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b, p.starve);
+            fused_issue<G, Tin, F32BC>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b,
+                                       p.starve);
 
 #pragma unroll 1
     for (int i = 0; i < nc; ++i) {
@@ -303,8 +313,8 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         // the previous chunk's stage is free (this warp is past it): refill it
         if (lane == 0 && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
-            fused_issue<G, Tin>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b,
-                                p.starve);
+            fused_issue<G, Tin, F32BC>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b,
+                                       p.starve);
         }
         const int nvalid = (int)((L - (int64_t)k * T < T) ? (L - (int64_t)k * T) : T);
         const int s_lo = DIR == 0 ? 0 : T - nvalid;
@@ -332,7 +342,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             cp_async_wait_all();
             __syncwarp();
         }
-        if constexpr (G == 1) {
+        if constexpr (G == 1 || F32BC) {
             __syncwarp();
             fused_convert_bc<T, Tin>(Bt, Ct, bcf, lane, true);
             __syncwarp();
@@ -351,7 +361,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             if constexpr (G == 1)
                 yr = wp.template scan1<true>(s, cur, bcf);
             else
-                yr = wp.template scan<true>(s, cur, Bt, Ct);
+                yr = wp.template scan<true>(s, cur, Bt, Ct, bcf);
             const float y = (yr + cur.Du) * scale;
             if (valid && wp.dvalid) {
                 const int tr = Wp::row_of(s);
@@ -382,9 +392,9 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     if (CARRY && p.delta_sum[DIR] && wp.dvalid) p.delta_sum[DIR][(int64_t)b * D + wp.d] = dsum;
 }
 
-template <int G, typename Tin, typename Tout, bool CARRY = false>
+template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false>
 __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constant__ FusedMaps maps, const KParams p) {
-    using Ge = FusedGeo<G, Tin>;
+    using Ge = FusedGeo<G, Tin, F32BC>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~static_cast<uintptr_t>(127));
@@ -396,9 +406,9 @@ __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constan
     }
     __syncthreads();
     if (warp == 0)
-        fused_layer_direction<G, Tin, Tout, 0, CARRY>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 0, CARRY, F32BC>(maps, p, base, lane);
     else
-        fused_layer_direction<G, Tin, Tout, 1, CARRY>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 1, CARRY, F32BC>(maps, p, base, lane);
 }
 
 // Forward scan over P = p.L tokens from zero: final state and conv tail.
@@ -452,7 +462,7 @@ __global__ void __launch_bounds__(32, 16) fused_prefix_kernel(const __grid_const
         for (int s = 0; s < T; ++s) {
             const auto cur = nxt;
             if (s + 1 < T) nxt = wp.element(s + 1, s + 1 < nvalid, xt, dtt);
-            wp.template scan<false>(s, cur, Bt, Bt);
+            wp.template scan<false>(s, cur, Bt, Bt, nullptr);
         }
         __syncwarp();
     }

@@ -165,3 +165,58 @@ def emulate_sharded(inputs: dict, params: dict, lengths: Sequence[int], ops=None
     h_all = torch.stack([a[0] for a in aggs])
     ds_all = torch.stack([a[1] for a in aggs])
     return torch.cat([pass_with_carries(e, params, h_all, ds_all, r, ops) for r, e in enumerate(exts)], dim=1)
+
+
+class ChunkedLayer:
+    """The layer over one long sequence (batch 1) cut into `nseg` equal
+    segments that one GPU scans side by side, as the rows of a batch: the
+    chunked form of the scan, with carries, inside one device.
+
+    ``__init__`` builds the extended segments once (each with its 3-token
+    halos, stacked into [nseg, Ls + 6, D] inputs); ``run`` is then the scan
+    itself: one layer pass from zero states for every segment's final states
+    and step-size sums, the composition of the carries entering each segment
+    (nseg small launches), and a second layer pass from them.  It exists to
+    measure this schedule against the single-pass kernels, which walk the
+    whole sequence in one chain per (channel, direction) and so need no
+    second pass."""
+
+    def __init__(self, inputs: dict, params: dict, nseg: int, ops=None):
+        x = inputs["x"]
+        if x.shape[0] != 1:
+            raise ValueError("the chunked form takes one sequence (batch 1)")
+        L = x.shape[1]
+        if L % nseg or L // nseg < HALO:
+            raise ValueError(f"L = {L} must split into {nseg} equal segments of at least {HALO} tokens")
+        self.ops = ops or CudaOps()
+        self.params = params
+        self.nseg, self.Ls = nseg, L // nseg
+        segs = split_sequence(inputs, [self.Ls] * nseg)
+        all_edges = torch.stack([halo_edges(s) for s in segs])
+        exts = [extend_segment(s, *neighbour_halos(all_edges, r)) for r, s in enumerate(segs)]
+        self.ext = {"x": torch.cat([e["x"] for e in exts], 0).contiguous(),
+                    "z": torch.cat([e["z"] for e in exts], 0).contiguous(),
+                    "dt": torch.cat([e["dt"] for e in exts], 1).contiguous(),
+                    "B": torch.cat([e["B"] for e in exts], 1).contiguous(),
+                    "C": torch.cat([e["C"] for e in exts], 1).contiguous()}
+        D, N = x.shape[2], inputs["B"].shape[-1]
+        dev = x.device
+        self.h_out = torch.empty(2, nseg, D, N, device=dev, dtype=self.ops.state_dtype)
+        self.ds = torch.empty(2, nseg, D, device=dev, dtype=self.ops.state_dtype)
+        self.h_all = torch.empty(nseg, 2, 1, D, N, device=dev, dtype=self.ops.state_dtype)
+        self.ds_all = torch.empty(nseg, 2, 1, D, device=dev, dtype=self.ops.state_dtype)
+        self.h_in = torch.empty(2, nseg, D, N, device=dev, dtype=self.ops.state_dtype)
+        self.y = torch.empty(nseg, self.Ls + 2 * HALO, D, device=dev, dtype=x.dtype)
+
+    def run(self) -> torch.Tensor:
+        """[nseg, Ls + 6, D]: each segment's extended rows of the layer output."""
+        self.ops.layer_carry(self.ext, self.params, h_out=self.h_out, delta_sum=self.ds)
+        self.h_all.copy_(self.h_out.permute(1, 0, 2, 3).unsqueeze(2))
+        self.ds_all.copy_(self.ds.permute(1, 0, 2).unsqueeze(2))
+        for s in range(self.nseg):
+            self.h_in[:, s] = self.ops.compose(self.h_all, self.ds_all, self.params, s)[:, 0]
+        return self.ops.layer_carry(self.ext, self.params, h_in=self.h_in, out=self.y)
+
+    def output(self, y: torch.Tensor) -> torch.Tensor:
+        """The layer output [1, L, D] from run()'s result."""
+        return y[:, HALO:HALO + self.Ls].reshape(1, self.nseg * self.Ls, y.shape[-1])

@@ -63,7 +63,9 @@ def test_layer_and_block_bytes():
 
 def test_workload_mapping():
     a = bench.parse_args([])
-    assert bench.workload_of(a) is W.LAYER_1P3B and a.steps >= 3 and a.warmup >= 3
+    # the default is the metric's own configuration: batch 1, d_inner 4096, L 65536
+    assert bench.workload_of(a) is W.LONG_SEQ[65536] and a.steps >= 3 and a.warmup >= 3
+    assert bench.workload_of(bench.parse_args(["--workload", "layer"])) is W.LAYER_1P3B
     assert bench.workload_of(bench.parse_args(["--workload", "long", "--L", "4096"])).L == 4096
     assert bench.workload_of(bench.parse_args(["--workload", "block"])) is W.BLOCK_CACHED
     sw = bench.workload_of(bench.parse_args(["--workload", "sweep", "--L", "32768"]))
@@ -102,3 +104,23 @@ def test_tensor_roofline_and_flop_counts():
     assert bench.mamba2_ssd_flops(8, 2048, 120, P, N) == per_chunk * 16 * 120 * 8 * 2
     r = bench.roofline_tensor(1.0e12, 1.0, "w", "k")  # 1 TFLOP in 1 ms = 1000 TFLOP/s
     assert r["achieved"] == 1000.0 and abs(r["frac"] - 1000.0 / r["peak"]) < 1e-4 and r["bound"] == "tensor"
+
+
+def test_sweep_pool_exceeds_twice_l2():
+    for L in (2048, 8192, 32768, 131072):
+        per_set = bench.layer_input_bytes(1, L, 4096, 16, 2)
+        r = bench.pool_size(per_set)
+        assert r >= 2 and r * per_set > 2 * bench.L2_BYTES
+    assert bench.pool_size(bench.layer_input_bytes(1, 2048, 4096, 16, 2)) == 5
+
+
+def test_hbm_roofline_fields():
+    r = bench.roofline_hbm(1.0e9, 1.0, "w", "k")  # 1 GB in 1 ms = 1000 GB/s
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["achieved"] == 1000.0
+    assert abs(r["frac"] - 1000.0 / r["peak"]) < 1e-4
+    # the Mamba-2 call at batch 8, L 2048: 528 MB of algorithmic traffic
+    assert bench.mamba2_bytes(8, 2048, 120, 32, 128) == 8 * 2048 * (2 * 4096 + 3840 + 240 + 3840) * 2
+
+
+def test_cpu_model_is_named():
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()

@@ -68,22 +68,92 @@ def test_bf16_ragged_tma_kernel(bm, shape, lanes, chunk):
     assert bm.bimamba_device_error() == 0
 
 
-@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("group", [1, 2, 4, 8, "2f", "4f"])
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
                                    (1, 16, 32), (1, 32, 64), (2, 17, 96)])
 def test_bf16_ragged_fused_kernel(bm, shape, group):
     """The per-token fused kernel (16-token chunks, one lane per channel,
-    B/C shared by groups of lanes): one, two and many chunks, ragged last
-    chunks and a last CTA whose 32 channels are partly past d_inner."""
+    B/C shared by groups of lanes; "f": B/C widened to fp32 once per chunk):
+    one, two and many chunks, ragged last chunks and a last CTA whose 32
+    channels are partly past d_inner."""
     b, L, D = shape
     inp, par = W.make_case(b, L, D, 16, "bf16", seed=300 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    flags = (group << 8) | (2 << bm.BIMAMBA_FAMILY_SHIFT)
+    f32bc = isinstance(group, str)
+    g = int(group[0]) if f32bc else group
+    flags = (g << 8) | (2 << bm.BIMAMBA_FAMILY_SHIFT) | ((2 << bm.BIMAMBA_CHUNK_SHIFT) if f32bc else 0)
     got32 = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got32, ref) <= U.GUARD
     got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
     assert U.bf16_out_ok(got16, ref)
     assert bm.bimamba_device_error() == 0
+
+
+SPLIT = 3 << 18  # the split-state kernel family (4 lanes x 4 states per channel)
+
+
+@pytest.mark.parametrize("chunk", [2, 3])  # 32 and 64 tokens
+@pytest.mark.parametrize("nwd", [1, 2])    # warps per direction per CTA
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 32, 32), (1, 64, 48), (1, 65, 8), (1, 200, 16)])
+def test_bf16_ragged_split_kernel(bm, shape, nwd, chunk):
+    """The split-state kernel: one, two and many chunks, a ragged last chunk
+    (both directions start their walk at a different end of it), and channel
+    counts that leave the last CTA's 8 or 16 channels partly empty."""
+    b, L, D = shape
+    inp, par = W.make_case(b, L, D, 16, "bf16", seed=400 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = SPLIT | (nwd << 8) | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= U.GUARD
+    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+    assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
+@pytest.mark.parametrize("L", [1, 3, 31, 32, 33, 63, 64, 65, 127, 129])
+@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16)])
+def test_split_kernel_fp32(bm, L, flags):
+    inp, par = W.make_case(2, L, 20, 16, "fp32", seed=500 + L)
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
+
+
+@pytest.mark.parametrize("flag", ["fwd", "rev"])
+def test_split_kernel_single_direction(bm, flag):
+    inp, par = W.make_case(1, 300, 24, 16, "fp32", seed=13)
+    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
+    ref = oracle.layer_fwd(inp, par, flags=f)
+    fl = bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY
+    got = run_layer(bm, inp, par, torch.float32, SPLIT | fl)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+def test_split_kernel_general_A_and_D(bm):
+    inp, par = W.make_case(1, 180, 32, 16, "fp32", seed=15)
+    g = torch.Generator().manual_seed(19)
+    par = dict(par)
+    par["A"] = -torch.exp(torch.rand(par["A"].shape, generator=g) * 5.0 - 3.0)
+    par["D"] = torch.rand(par["D"].shape, generator=g) * 2.0 - 1.0
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32, SPLIT | (2 << 8))
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+def test_split_kernel_rejects_staging(bm):
+    inp, par = W.make_case(1, 64, 16, 16, "bf16", seed=1, device="cuda")
+    with pytest.raises(bm.BimambaError) as e:
+        bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, flags=SPLIT | bm.BIMAMBA_NO_TMA)
+    assert e.value.status == bm.BIMAMBA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16)])
+@pytest.mark.parametrize("L", [4096, 65536])
+def test_long_sequence_split_sampled(bm, L, flags):
+    """b=1, D=4096, bf16, seed 2: the split-state kernel at long L."""
+    err, ok16 = _sampled_layer_check(bm, W.LONG_SEQ[L], 12, flags)
+    assert err <= U.GUARD and ok16
 
 
 def test_unaligned_channel_count_uses_staged_kernel(bm):

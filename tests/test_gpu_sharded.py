@@ -13,7 +13,7 @@ from tests import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
-FAMILIES = {"fused": 2 << 18, "chunked": 1 << 18}
+FAMILIES = {"fused": 2 << 18, "chunked": 1 << 18, "split": 3 << 18}
 
 
 @pytest.fixture(scope="module")
@@ -101,3 +101,21 @@ def test_full_size_sampled_channels(bm):
     want = oracle.layer_fwd(si, sp)
     idx = torch.as_tensor(chans, device="cuda")
     assert U.bf16_out_ok(U.to_cpu64(got.index_select(-1, idx)), want)
+
+
+@pytest.mark.parametrize("nseg", [2, 8])
+def test_chunked_layer_matches_single_pass(nseg):
+    """The batch-1 layer scanned as segments side by side with carries
+    (two passes) against the single-pass layer and the oracle."""
+    from bidirectional_mamba_denoiser_b200 import bimamba as bm
+    from bidirectional_mamba_denoiser_b200 import sharded as SH
+    inp, par = W.make_case(1, 1024, 64, 16, "fp32", seed=71)
+    ref = oracle.layer_fwd(inp, par)
+    d, p = U.to_device(inp), U.to_device(par)
+    plan = SH.ChunkedLayer(d, p, nseg)
+    got = plan.output(plan.run())
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(got), ref) <= U.TOL_FP32
+    one = bm.bimamba_layer_fwd(d["x"], d["z"], d["dt"], d["B"], d["C"], p, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert U.normwise(U.to_cpu64(got), U.to_cpu64(one)) <= U.TOL_FP32
