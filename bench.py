@@ -77,7 +77,9 @@ def parse_args(argv=None):
     ap.add_argument("--L", type=int, default=0, help="sequence length of --workload long/sweep; prefix length of --workload block/decode/decode_mamba2")
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
-    ap.add_argument("--family", type=int, default=0, help="kernel family: 0 auto, 1 chunked, 2 per-token fused")
+    ap.add_argument("--family", type=int, default=0,
+                    help="kernel family: 0 auto, 1 chunked, 2 per-token fused, 3 split-state")
+    ap.add_argument("--flags", type=lambda v: int(v, 0), default=0, help="further flag bits (tuning knobs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-l-sweep", action="store_true", help="long: skip the per-L lines")
@@ -376,7 +378,7 @@ def oracle_sample_rate(w: W.Workload, inputs, params, budget_s: float):
 
 def flags_of(args, bm):
     return (((args.lanes << bm.BIMAMBA_LANES_SHIFT) if args.lanes else 0) | (args.chunk << bm.BIMAMBA_CHUNK_SHIFT)
-            | (args.family << bm.BIMAMBA_FAMILY_SHIFT))
+            | (args.family << bm.BIMAMBA_FAMILY_SHIFT) | args.flags)
 
 
 def kernel_name(w: W.Workload, args) -> str:

@@ -14,6 +14,7 @@
 #include "carry.cuh"
 #include "context_cache.h"
 #include "layer_fused.cuh"
+#include "layer_fused2.cuh"
 #include "layer_split.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
@@ -331,6 +332,9 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
 // ---- split-state kernel (few channels: 4 lanes x 4 states per channel)
 
 constexpr int kSNS = 3;  // pipeline stages per direction
+// tuning knob: the alternative variant of a family (split-state: step sizes exchanged through shared
+// memory instead of shuffles; per-token fused: the kernel in phases, layer_fused2.cuh)
+constexpr unsigned kAltVariant = 0x2000u;
 
 template <int T, int NWD, typename Tin>
 bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
@@ -347,12 +351,12 @@ bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batc
     return ok;
 }
 
-template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false>
+template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false, bool XSM = false>
 int launch_layer_split(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin>;
+    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin, XSM>;
     bimamba::LayerMaps maps;
     if (!fill_split_maps<T, NWD, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY>;
+    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY, XSM>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -367,6 +371,12 @@ int layer_split_by(unsigned flags, const KParams& k, const bimamba_inputs_t* in,
     const unsigned ch = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
     const unsigned nw = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int t = ch == 3 ? 64 : 32;
+    if (flags & kAltVariant) {
+        if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout, false, true>(k, in, st)
+                                    : launch_layer_split<32, 2, Tin, Tout, false, true>(k, in, st);
+        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, true>(k, in, st)
+                       : launch_layer_split<32, 1, Tin, Tout, false, true>(k, in, st);
+    }
     if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout>(k, in, st)
                                 : launch_layer_split<32, 2, Tin, Tout>(k, in, st);
     return t == 64 ? launch_layer_split<64, 1, Tin, Tout>(k, in, st) : launch_layer_split<32, 1, Tin, Tout>(k, in, st);
@@ -441,6 +451,41 @@ int launch_fused_prefix(const KParams& k, const bimamba_inputs_t* in, cudaStream
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
     kern<<<grid, 32, Ge::SMEM, st>>>(maps, k);
     return launch_status();
+}
+
+// ---- per-token fused kernel in phases (fused2)
+
+template <int T, typename Tin>
+bool fill_fused2_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
+    const bool bf = std::is_same<Tin, bf16>::value;
+    constexpr int N = bimamba::kNState;
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, 32, T + 3);
+    ok = ok && map3d(&m.z, in->z, bf, D, L, batch, 32, T);
+    for (int r = 0; r < 2; ++r) {
+        ok = ok && map3d(&m.dt[r], in->dt[r], bf, D, L, batch, 32, T);
+        ok = ok && map3d(&m.B[r], in->B[r], bf, N, L, batch, N, T);
+        ok = ok && map3d(&m.C[r], in->C[r], bf, N, L, batch, N, T);
+    }
+    return ok;
+}
+
+template <int T, int NS, typename Tin, typename Tout, bool CARRY = false>
+int launch_fused2_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::Fused2Geo<T, NS, Tin>;
+    bimamba::FusedMaps maps;
+    if (!fill_fused2_maps<T, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::fused2_layer_kernel<T, NS, Tin, Tout, CARRY>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + 31) / 32), (unsigned)k.batch);
+    kern<<<grid, 64, Ge::SMEM, st>>>(maps, k);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+int fused2_by_chunk(unsigned chunk_field, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    if (chunk_field == 2) return launch_fused2_layer<8, 3, Tin, Tout>(k, in, st);
+    return launch_fused2_layer<16, 2, Tin, Tout>(k, in, st);
 }
 
 // Kernel family of the TMA path: forced by the flags, else the per-token
@@ -604,7 +649,7 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
-                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE;
+                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE | kAltVariant;
     const bool split_family = ((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3;
     const unsigned chunk_field = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
     const unsigned lane_field = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
@@ -671,6 +716,12 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
             return launch_fused_layer<2, float, float, true>(k, in, st);
         }
         const int gf = pick_group_fused(flags);
+        if (flags & kAltVariant) {  // family 2: the phased kernel
+            if (in_bf && out_bf) return fused2_by_chunk<bf16, bf16>(chunk_field, k, in, st);
+            if (in_bf) return fused2_by_chunk<bf16, float>(chunk_field, k, in, st);
+            if (out_bf) return fused2_by_chunk<float, bf16>(chunk_field, k, in, st);
+            return fused2_by_chunk<float, float>(chunk_field, k, in, st);
+        }
         const bool f32bc = chunk_field == 2;  // family 2: B/C widened once per chunk
         if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, f32bc, k, in, st);
         if (in_bf) return fused_layer_by_group<bf16, float>(gf, f32bc, k, in, st);

@@ -43,7 +43,9 @@
 
 namespace bimamba {
 
-template <int T, int NWD, int NS, typename Tin>
+// XSM: the step sizes and drives reach the scanning lanes through a per-warp
+// shared-memory buffer (one 8-byte load per step) instead of two shuffles.
+template <int T, int NWD, int NS, typename Tin, bool XSM = false>
 struct SplitGeo {
     static_assert(T % 4 == 0 && T + 3 <= 256, "chunk");
     static_assert(NWD == 1 || NWD == 2, "warps per direction");
@@ -58,9 +60,11 @@ struct SplitGeo {
     static constexpr int BB = align128(T * kNState * ESZ);
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
     static constexpr int OWS = T * CPW * 4;               // per warp: partner's y of a chunk
+    static constexpr int EDX = XSM ? T * CPW * 8 : 0;     // per warp: (delta, delta*u) of the chunk's steps
+    static constexpr int WARP_BYTES = OWS + EDX;
     static constexpr int DIR_BYTES = NS * STAGE;
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
-    static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * OWS;
+    static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;  // + alignment slack
     static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
     static constexpr uint32_t TX_Z = (uint32_t)(T * CW * ESZ);
@@ -95,9 +99,9 @@ __device__ __forceinline__ float reduce4(const float (&p)[4], int j) {
     return k + __shfl_xor_sync(0xffffffffu, s, 1);
 }
 
-template <int T, int NWD, int NS, typename Tin, int DIR>
+template <int T, int NWD, int NS, typename Tin, int DIR, bool XSM>
 struct SplitWorker {
-    using Ge = SplitGeo<T, NWD, NS, Tin>;
+    using Ge = SplitGeo<T, NWD, NS, Tin, XSM>;
     int c, j, cc, d;  // cc: channel inside the CTA tile; d: global channel
     bool dvalid;
     float A2[4];      // A * log2(e) of this lane's states
@@ -134,7 +138,7 @@ struct SplitWorker {
     // outside [s_lo, s_hi) (tokens >= L) become identity steps.  DSUM: also
     // add the valid step sizes to dsum.
     template <bool DSUM>
-    __device__ __forceinline__ void elements(const Tin* xt, const Tin* dtt, int s_lo, int s_hi) {
+    __device__ __forceinline__ void elements(const Tin* xt, const Tin* dtt, int s_lo, int s_hi, float2* edx) {
 #pragma unroll
         for (int e = 0; e < Ge::EPL; ++e) {
             const int s = j + 4 * e;
@@ -152,18 +156,26 @@ struct SplitWorker {
             dl[e] = valid ? dlt : 0.f;
             du[e] = valid ? dlt * u : 0.f;
             Du[e] = valid ? Dd * u : 0.f;
+            if constexpr (XSM) edx[s * Ge::CPW + c] = make_float2(dl[e], du[e]);
             if constexpr (DSUM) dsum += dl[e];
         }
     }
 
     // States over steps 4e..4e+3; returns sum_n C h of step 4e + j.
-    __device__ __forceinline__ float step_group(int e, const Tin* Bt, const Tin* Ct) {
+    __device__ __forceinline__ float step_group(int e, const Tin* Bt, const Tin* Ct, const float2* edx) {
         float pp[4];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const int s = 4 * e + g;
-            const float dq = __shfl_sync(0xffffffffu, dl[e], g, 4);
-            const float uq = __shfl_sync(0xffffffffu, du[e], g, 4);
+            float dq, uq;
+            if constexpr (XSM) {
+                const float2 q = edx[s * Ge::CPW + c];
+                dq = q.x;
+                uq = q.y;
+            } else {
+                dq = __shfl_sync(0xffffffffu, dl[e], g, 4);
+                uq = __shfl_sync(0xffffffffu, du[e], g, 4);
+            }
             float bv[4], cv[4];
             load_quad(Bt + row_of(s) * kNState, j, bv);
             load_quad(Ct + row_of(s) * kNState, j, cv);
@@ -189,7 +201,7 @@ struct SplitWorker {
 template <int T, int NWD, int NS, typename Tin>
 __device__ __forceinline__ void split_issue(const LayerMaps& maps, unsigned char* dir_base, uint64_t* full, int r,
                                             int i, int k, bool gated, int ct0, int b, int starve) {
-    using Ge = SplitGeo<T, NWD, NS, Tin>;
+    using Ge = SplitGeo<T, NWD, NS, Tin>;  // the stage layout does not depend on XSM
     if (starve) return;
     const int st = i % NS;
     unsigned char* sb = dir_base + st * Ge::STAGE;
@@ -204,13 +216,15 @@ __device__ __forceinline__ void split_issue(const LayerMaps& maps, unsigned char
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY>
+template <int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool XSM>
 __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
-    using Ge = SplitGeo<T, NWD, NS, Tin>;
-    using Wk = SplitWorker<T, NWD, NS, Tin, DIR>;
+    using Ge = SplitGeo<T, NWD, NS, Tin, XSM>;
+    using Wk = SplitWorker<T, NWD, NS, Tin, DIR, XSM>;
     unsigned char* dir_base = base + DIR * Ge::DIR_BYTES;
-    float* ows = reinterpret_cast<float*>(base + Ge::WARP_OFF + (DIR * NWD + wg) * Ge::OWS);
+    unsigned char* wbase = base + Ge::WARP_OFF + (DIR * NWD + wg) * Ge::WARP_BYTES;
+    float* ows = reinterpret_cast<float*>(wbase);
+    float2* edx = reinterpret_cast<float2*>(wbase + Ge::OWS);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + Ge::BAR_OFF) + DIR * NS;
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
@@ -269,17 +283,15 @@ __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KPa
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
 
-        wk.template elements<CARRY>(xt, dtt, s_lo, s_hi);
-        if (gated) {
-            cp_async_wait_all();
-            __syncwarp();
-        }
+        wk.template elements<CARRY>(xt, dtt, s_lo, s_hi, edx);
+        if (gated) cp_async_wait_all();
+        if (gated || XSM) __syncwarp();
 
         float* wsw = p.ws + chunk_row * D + wk.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
 #pragma unroll
         for (int e = 0; e < Ge::EPL; ++e) {
-            const float yr = wk.step_group(e, Bt, Ct);
+            const float yr = wk.step_group(e, Bt, Ct, edx);
             const int s = 4 * e + wk.j;
             if (s >= s_lo && s < s_hi && wk.dvalid) {
                 const int tr = Wk::row_of(s);  // token - kT
@@ -318,10 +330,10 @@ __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KPa
     }
 }
 
-template <int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false>
+template <int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool XSM = false>
 __global__ void __launch_bounds__(2 * NWD * 32) layer_split_kernel(const __grid_constant__ LayerMaps maps,
                                                                    const KParams p) {
-    using Ge = SplitGeo<T, NWD, NS, Tin>;
+    using Ge = SplitGeo<T, NWD, NS, Tin, XSM>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~static_cast<uintptr_t>(127));
@@ -333,9 +345,9 @@ __global__ void __launch_bounds__(2 * NWD * 32) layer_split_kernel(const __grid_
     }
     __syncthreads();
     if (warp < NWD)
-        split_direction<T, NWD, NS, Tin, Tout, 0, CARRY>(maps, p, base, warp, lane);
+        split_direction<T, NWD, NS, Tin, Tout, 0, CARRY, XSM>(maps, p, base, warp, lane);
     else
-        split_direction<T, NWD, NS, Tin, Tout, 1, CARRY>(maps, p, base, warp - NWD, lane);
+        split_direction<T, NWD, NS, Tin, Tout, 1, CARRY, XSM>(maps, p, base, warp - NWD, lane);
 }
 
 }  // namespace bimamba

@@ -89,6 +89,55 @@ def test_bf16_ragged_fused_kernel(bm, shape, group):
     assert bm.bimamba_device_error() == 0
 
 
+ALT = 0x2000  # a family's alternative variant (tuning knob)
+
+
+@pytest.mark.parametrize("chunk", [0, 2])  # 16- and 8-token chunks
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 16, 32), (1, 32, 64), (2, 17, 96), (1, 9, 32)])
+def test_bf16_ragged_fused2_kernel(bm, shape, chunk):
+    """The per-token fused kernel in phases (pre-pass of the chunk's per-token
+    work, then the scan): one, two and many chunks, ragged last chunks, a last
+    CTA whose 32 channels are partly past d_inner (and an odd channel count,
+    so a lane's partner channel can be past the end)."""
+    b, L, D = shape
+    inp, par = W.make_case(b, L, D, 16, "bf16", seed=600 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = (2 << bm.BIMAMBA_FAMILY_SHIFT) | ALT | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= U.GUARD
+    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+    assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
+@pytest.mark.parametrize("chunk", [0, 2])
+@pytest.mark.parametrize("L", [1, 7, 8, 9, 16, 17, 33, 100])
+def test_fused2_kernel_fp32(bm, L, chunk):
+    inp, par = W.make_case(2, L, 36, 16, "fp32", seed=700 + L)
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32, (2 << 18) | ALT | (chunk << 16))
+    assert U.normwise(got, ref) <= U.TOL_FP32, L
+
+
+@pytest.mark.parametrize("flag", ["fwd", "rev"])
+def test_fused2_kernel_single_direction(bm, flag):
+    inp, par = W.make_case(1, 200, 64, 16, "fp32", seed=17)
+    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
+    ref = oracle.layer_fwd(inp, par, flags=f)
+    fl = bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY
+    got = run_layer(bm, inp, par, torch.float32, (2 << 18) | ALT | fl)
+    assert U.normwise(got, ref) <= U.TOL_FP32
+
+
+@pytest.mark.parametrize("chunk", [2, 3])
+def test_split_kernel_smem_exchange(bm, chunk):
+    inp, par = W.make_case(2, 150, 40, 16, "bf16", seed=18)
+    ref = oracle.layer_fwd(inp, par)
+    got = run_layer(bm, inp, par, torch.float32, SPLIT | ALT | (chunk << 16))
+    assert U.normwise(got, ref) <= U.GUARD
+
+
 SPLIT = 3 << 18  # the split-state kernel family (4 lanes x 4 states per channel)
 
 
@@ -232,7 +281,7 @@ def _sampled_layer_check(bm, w: W.Workload, nchan: int, flags=0):
     return U.normwise(g32, ref), U.bf16_out_ok(g16, ref)
 
 
-@pytest.mark.parametrize("flags", [0, 1 << 18])
+@pytest.mark.parametrize("flags", [0, 1 << 18, (2 << 18) | 0x2000, (2 << 18) | 0x2000 | (2 << 16)])
 def test_layer_1p3b_shape_sampled(bm, flags):
     """b=8, L=2048, D=4096, bf16, seed 1 -- the launch configuration the
     bench times (flags 0) and the chunked kernel; 48 channels of every batch

@@ -112,6 +112,8 @@ LAYER_KERNELS = {
     "fused_g2": 2 << 8 | 2 << 18,
     "fused_g1": 1 << 8 | 2 << 18,
     "fused_g2_f32bc": 2 << 8 | 2 << 16 | 2 << 18,
+    "fused2_t16": 2 << 18 | 0x2000,
+    "fused2_t8": 2 << 18 | 0x2000 | 2 << 16,
     "chunked_g8": 8 << 8 | 1 << 18,
     "chunked_g4": 4 << 8 | 1 << 18,
     "staged": 4 << 8 | 0x4000,
