@@ -335,6 +335,7 @@ constexpr int kSNS = 3;  // pipeline stages per direction
 // tuning knob: the alternative variant of a family (split-state: step sizes exchanged through shared
 // memory instead of shuffles; per-token fused: the kernel in phases, layer_fused2.cuh)
 constexpr unsigned kAltVariant = 0x2000u;
+constexpr unsigned kAltVariant2 = 0x8000u;   // split-state: the scan step in phases (tuning knob)
 
 template <int T, int NWD, typename Tin>
 bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
@@ -351,12 +352,12 @@ bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batc
     return ok;
 }
 
-template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false, bool XSM = false>
+template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false, bool XSM = false, bool PHASED = false>
 int launch_layer_split(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
     using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin, XSM>;
     bimamba::LayerMaps maps;
     if (!fill_split_maps<T, NWD, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY, XSM>;
+    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY, XSM, PHASED>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -371,6 +372,12 @@ int layer_split_by(unsigned flags, const KParams& k, const bimamba_inputs_t* in,
     const unsigned ch = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
     const unsigned nw = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int t = ch == 3 ? 64 : 32;
+    if ((flags & kAltVariant) && (flags & kAltVariant2))  // shared-memory exchange, phased scan steps
+        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, true, true>(k, in, st)
+                       : launch_layer_split<32, 1, Tin, Tout, false, true, true>(k, in, st);
+    if (flags & kAltVariant2)  // phased scan steps
+        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, false, true>(k, in, st)
+                       : launch_layer_split<32, 1, Tin, Tout, false, false, true>(k, in, st);
     if (flags & kAltVariant) {
         if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout, false, true>(k, in, st)
                                     : launch_layer_split<32, 2, Tin, Tout, false, true>(k, in, st);
@@ -649,7 +656,8 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
-                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE | kAltVariant;
+                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE | kAltVariant |
+                           kAltVariant2;
     const bool split_family = ((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3;
     const unsigned chunk_field = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
     const unsigned lane_field = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;

@@ -161,7 +161,55 @@ struct SplitWorker {
         }
     }
 
-    // States over steps 4e..4e+3; returns sum_n C h of step 4e + j.
+    // States over steps 4e..4e+3; returns sum_n C h of step 4e + j.  In
+    // phases: every load of the four steps, then their 16 exps (which depend
+    // only on the step sizes), then the dependent updates -- so the exps can
+    // keep the special-function unit busy while the loads and the state
+    // chain wait.
+    __device__ __forceinline__ float step_group_phased(int e, const Tin* Bt, const Tin* Ct, const float2* edx) {
+        float dq[4], uq[4], bv[4][4], cv[4][4], ea[4][4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int s = 4 * e + g;
+            if constexpr (XSM) {
+                const float2 q = edx[s * Ge::CPW + c];
+                dq[g] = q.x;
+                uq[g] = q.y;
+            } else {
+                dq[g] = __shfl_sync(0xffffffffu, dl[e], g, 4);
+                uq[g] = __shfl_sync(0xffffffffu, du[e], g, 4);
+            }
+            load_quad(Bt + row_of(s) * kNState, j, bv[g]);
+            load_quad(Ct + row_of(s) * kNState, j, cv[g]);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const float2 dd = make_float2(dq[g], dq[g]);
+#pragma unroll
+            for (int q = 0; q < 4; q += 2) {
+                const float2 v = mul2(dd, make_float2(A2[q], A2[q + 1]));
+                ea[g][q] = ex2_approx(v.x);
+                ea[g][q + 1] = ex2_approx(v.y);
+            }
+        }
+        float pp[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const float2 uu = make_float2(uq[g], uq[g]);
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 4; q += 2) {
+                const float2 drive = mul2(uu, make_float2(bv[g][q], bv[g][q + 1]));
+                const float2 hh = fma2(make_float2(ea[g][q], ea[g][q + 1]), make_float2(h[q], h[q + 1]), drive);
+                h[q] = hh.x;
+                h[q + 1] = hh.y;
+                acc = fma2(make_float2(cv[g][q], cv[g][q + 1]), hh, acc);
+            }
+            pp[g] = acc.x + acc.y;
+        }
+        return reduce4(pp, j);
+    }
+
     __device__ __forceinline__ float step_group(int e, const Tin* Bt, const Tin* Ct, const float2* edx) {
         float pp[4];
 #pragma unroll
@@ -216,7 +264,7 @@ __device__ __forceinline__ void split_issue(const LayerMaps& maps, unsigned char
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool XSM>
+template <int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool XSM, bool PHASED>
 __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
     using Ge = SplitGeo<T, NWD, NS, Tin, XSM>;
@@ -291,7 +339,7 @@ __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KPa
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
 #pragma unroll
         for (int e = 0; e < Ge::EPL; ++e) {
-            const float yr = wk.step_group(e, Bt, Ct, edx);
+            const float yr = PHASED ? wk.step_group_phased(e, Bt, Ct, edx) : wk.step_group(e, Bt, Ct, edx);
             const int s = 4 * e + wk.j;
             if (s >= s_lo && s < s_hi && wk.dvalid) {
                 const int tr = Wk::row_of(s);  // token - kT
@@ -330,7 +378,8 @@ __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KPa
     }
 }
 
-template <int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool XSM = false>
+template <int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool XSM = false,
+          bool PHASED = false>
 __global__ void __launch_bounds__(2 * NWD * 32) layer_split_kernel(const __grid_constant__ LayerMaps maps,
                                                                    const KParams p) {
     using Ge = SplitGeo<T, NWD, NS, Tin, XSM>;
@@ -345,9 +394,9 @@ __global__ void __launch_bounds__(2 * NWD * 32) layer_split_kernel(const __grid_
     }
     __syncthreads();
     if (warp < NWD)
-        split_direction<T, NWD, NS, Tin, Tout, 0, CARRY, XSM>(maps, p, base, warp, lane);
+        split_direction<T, NWD, NS, Tin, Tout, 0, CARRY, XSM, PHASED>(maps, p, base, warp, lane);
     else
-        split_direction<T, NWD, NS, Tin, Tout, 1, CARRY, XSM>(maps, p, base, warp - NWD, lane);
+        split_direction<T, NWD, NS, Tin, Tout, 1, CARRY, XSM, PHASED>(maps, p, base, warp - NWD, lane);
 }
 
 }  // namespace bimamba

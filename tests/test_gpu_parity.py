@@ -130,12 +130,14 @@ def test_fused2_kernel_single_direction(bm, flag):
     assert U.normwise(got, ref) <= U.TOL_FP32
 
 
+@pytest.mark.parametrize("variant", [ALT, 0x8000, ALT | 0x8000])  # shared-memory exchange, phased steps, both
 @pytest.mark.parametrize("chunk", [2, 3])
-def test_split_kernel_smem_exchange(bm, chunk):
-    inp, par = W.make_case(2, 150, 40, 16, "bf16", seed=18)
-    ref = oracle.layer_fwd(inp, par)
-    got = run_layer(bm, inp, par, torch.float32, SPLIT | ALT | (chunk << 16))
-    assert U.normwise(got, ref) <= U.GUARD
+def test_split_kernel_variants(bm, chunk, variant):
+    for L, D in ((150, 40), (33, 8), (1, 16)):
+        inp, par = W.make_case(2, L, D, 16, "bf16", seed=18 + L)
+        ref = oracle.layer_fwd(inp, par)
+        got = run_layer(bm, inp, par, torch.float32, SPLIT | variant | (chunk << 16))
+        assert U.normwise(got, ref) <= U.GUARD, (L, D)
 
 
 SPLIT = 3 << 18  # the split-state kernel family (4 lanes x 4 states per channel)

@@ -61,6 +61,17 @@ def per_channel(got, want) -> float:
     return float(np.max(err / scale))
 
 
+def states_by_channel(h):
+    """[b, D, 16] states -> [b * 16, D]: a channel's states of every batch row
+    in its column.  Measured per channel like the outputs (not per batch row:
+    with a step size of 25 or 40 a row's state is essentially the single term
+    delta u B of its last token, so where that token's conv output nearly
+    cancels, the row's relative error reflects fp32 rounding of the conv, not
+    the scan)."""
+    h = np.asarray(h, dtype=np.float64)
+    return h.transpose(0, 2, 1).reshape(-1, h.shape[1])
+
+
 def tol_of(dtype):
     return U.TOL_FP32 if dtype == "fp32" else U.GUARD
 
@@ -157,10 +168,7 @@ def test_prefix_state_extreme_steps(bm, kernel, dtype, mode):
     d, p = U.to_device(inp), U.to_device(par)
     h, tail = bm.bimamba_prefix_state(d["x"], d["dt"][0].contiguous(), d["B"][0].contiguous(), p)
     torch.cuda.synchronize()
-    # per channel: the 16 states of a (row, channel) against their largest
-    got = U.to_cpu64(h).reshape(b * D, 16).T
-    want = h_ref.reshape(b * D, 16).T
-    assert per_channel(got, want) <= tol_of(dtype)
+    assert per_channel(states_by_channel(U.to_cpu64(h)), states_by_channel(h_ref)) <= tol_of(dtype)
     assert np.array_equal(U.to_cpu64(tail), t_ref)
     assert bm.bimamba_device_error() == 0
 
@@ -187,5 +195,4 @@ def test_block_step_extreme_steps(bm, kernel, dtype, mode):
                                     out_dtype=torch.float32, new_state=(h, tail), flags=BLOCK_KERNELS[kernel])
         torch.cuda.synchronize()
         assert per_channel(U.to_cpu64(out), ref) <= tol_of(dtype), k
-        got = U.to_cpu64(h).reshape(b * D, 16).T
-        assert per_channel(got, h_ref.reshape(b * D, 16).T) <= tol_of(dtype), k
+        assert per_channel(states_by_channel(U.to_cpu64(h)), states_by_channel(h_ref)) <= tol_of(dtype), k
