@@ -235,23 +235,23 @@ bool tma_eligible(const bimamba_inputs_t* in, int d_inner, bool need_reverse, bo
 constexpr int kTWD = 4;  // warps per direction per CTA
 constexpr int kTNS = 2;  // pipeline stages
 
-template <int G, int T, typename Tin>
+template <int G, int T, typename Tin, int NWD = kTWD>
 bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool reverse,
                bool gated) {
-    using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
+    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin>;
     const bool bf = std::is_same<Tin, bf16>::value;
-    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, T + 3);
-    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, Ge::CW, T);
+    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::XW, T + 3);
+    ok = ok && map3d(&m.dt[0], in->dt[0], bf, D, L, batch, Ge::XW, T);
     ok = ok && map3d(&m.B[0], in->B[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     if (gated) {
-        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, T);
+        ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::XW, T);
         ok = ok && map3d(&m.C[0], in->C[0], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     } else {
         m.z = m.x;
         m.C[0] = m.B[0];
     }
     if (reverse) {
-        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, Ge::CW, T);
+        ok = ok && map3d(&m.dt[1], in->dt[1], bf, D, L, batch, Ge::XW, T);
         ok = ok && map3d(&m.B[1], in->B[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
         ok = ok && map3d(&m.C[1], in->C[1], bf, bimamba::kNState, L, batch, bimamba::kNState, T);
     } else {
@@ -262,16 +262,16 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
-template <int G, int T, typename Tin, typename Tout, bool CARRY = false>
+template <int G, int T, typename Tin, typename Tout, bool CARRY = false, int NWD = kTWD, bool DIRECT = false>
 int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::TmaGeo<G, T, kTWD, kTNS, Tin>;
+    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin>;
     bimamba::LayerMaps maps;
-    if (!fill_maps<G, T, Tin>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_tma_kernel<G, T, kTWD, kTNS, Tin, Tout, CARRY>;
+    if (!fill_maps<G, T, Tin, NWD>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
-    kern<<<grid, 2 * kTWD * 32, Ge::SMEM, st>>>(maps, k);
+    kern<<<grid, 2 * NWD * 32, Ge::SMEM, st>>>(maps, k);
     return launch_status();
 }
 
@@ -745,6 +745,12 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
             return layer_tma_carry_by_lanes<float, float>(gt, k, in, st);
         }
         const int tt = pick_chunk_tma(flags, gt);
+        if ((flags & kAltVariant) && gt == 8) {  // one warp per direction, B/C read from the bf16 tile (tuning knob)
+            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true>(k, in, st);
+            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true>(k, in, st);
+            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true>(k, in, st);
+            return launch_layer_tma<8, 32, float, float, false, 1, true>(k, in, st);
+        }
         if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, tt, k, in, st);
         if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, tt, k, in, st);
         if (out_bf) return layer_tma_by_lanes<float, bf16>(gt, tt, k, in, st);

@@ -58,8 +58,11 @@ struct TmaGeo {
     static constexpr int EPL = T / G;                     // elements per lane per chunk
     static constexpr int CW = NWD * CPW;                  // channels per CTA
     static constexpr int ESZ = (int)sizeof(Tin);
-    static constexpr int XB = align128((T + 3) * CW * ESZ);
-    static constexpr int DTB = align128(T * CW * ESZ);
+    // channels per x/dt/z tile row: CW, widened to the aligned 16 bytes around
+    // the CTA's channels when CW of them are fewer (TMA rows are 16-byte units)
+    static constexpr int XW = CW * ESZ >= 16 ? CW : 16 / ESZ;
+    static constexpr int XB = align128((T + 3) * XW * ESZ);
+    static constexpr int DTB = align128(T * XW * ESZ);
     static constexpr int BB = align128(T * kNState * ESZ);
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;   // x, dt, z, B, C
     static constexpr int BC32 = T * kNState * 2 * 4;      // one fp32 B/C buffer
@@ -71,9 +74,9 @@ struct TmaGeo {
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
     static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;  // + alignment slack
-    static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
-    static constexpr uint32_t TX_Z = (uint32_t)(T * CW * ESZ);
-    static_assert((CW * ESZ) % 16 == 0, "TMA box rows must be whole 16-byte units");
+    static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * XW + T * XW + 2 * T * kNState) * ESZ);
+    static constexpr uint32_t TX_Z = (uint32_t)(T * XW * ESZ);
+    static_assert((XW * ESZ) % 16 == 0 && XW % CW == 0, "TMA box rows must be whole 16-byte units");
 };
 
 // fp32 B/C layout per token: 8 quads (B_2p, B_2p+1, C_2p, C_2p+1), so that a
@@ -97,6 +100,7 @@ template <int G, int T, int NWD, int NS, typename Tin, int DIR>
 struct TmaWorker {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
     int c, j, cc, d;  // cc: channel inside the CTA tile; d: global channel
+    int tc;           // column of the channel in the x/dt/z tiles
     bool dvalid;
     float A2[Ge::S];  // A * log2(e) of this lane's states
     float w[4], cb, bias, Dd;
@@ -109,6 +113,7 @@ struct TmaWorker {
         j = lane / Ge::CPW;
         cc = wg * Ge::CPW + c;
         d = ct0 + cc;
+        tc = ct0 % Ge::XW + cc;
         dvalid = d < p.D;
         const int64_t rd = (int64_t)DIR * p.D + (dvalid ? d : 0);
 #pragma unroll
@@ -140,10 +145,10 @@ struct TmaWorker {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int xr = DIR == 0 ? s + q : T + 2 - s - q;
-                cv = fmaf(w[q], ldf(xt, xr * Ge::CW + cc), cv);
+                cv = fmaf(w[q], ldf(xt, xr * Ge::XW + tc), cv);
             }
             const float u = silu(cv);
-            const float dl = softplus(ldf(dtt, row_of(s) * Ge::CW + cc) + bias);
+            const float dl = softplus(ldf(dtt, row_of(s) * Ge::XW + tc) + bias);
             const bool valid = s >= s_lo && s < s_hi;
             if constexpr (DSUM) dsum += valid ? dl : 0.f;
             ed2[s * Ge::CPW + c] = valid ? make_float2(dl, dl * u) : make_float2(0.f, 0.f);
@@ -151,10 +156,72 @@ struct TmaWorker {
         }
     }
 
+    // The S B (or C) values of states [jS, jS+S) of tile row r straight from
+    // a TMA tile of the input dtype (bf16 widened in registers: exact).
+    static __device__ __forceinline__ void tile_states(const Tin* t, int r, int jj, float (&v)[Ge::S]) {
+        const Tin* q = t + r * kNState + jj * Ge::S;
+        if constexpr (sizeof(Tin) == 4) {
+#pragma unroll
+            for (int i = 0; i < Ge::S; ++i) v[i] = ldf(q, i);
+        } else if constexpr (Ge::S == 2) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(q);
+            v[0] = __uint_as_float(w << 16);
+            v[1] = __uint_as_float(w & 0xffff0000u);
+        } else if constexpr (Ge::S == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(q);
+            v[0] = __uint_as_float(w.x << 16);
+            v[1] = __uint_as_float(w.x & 0xffff0000u);
+            v[2] = __uint_as_float(w.y << 16);
+            v[3] = __uint_as_float(w.y & 0xffff0000u);
+        } else {
+            v[0] = ldf(q, 0);
+        }
+    }
+
     // Advance the states over steps G*e .. G*e+G-1; returns, for this lane,
     // sum_n C h of step G*e + j (WITH_Y) after the cross-lane combination.
-    template <bool WITH_Y>
-    __device__ __forceinline__ float step_group(int e, const float2* ed2, const float* bc) {
+    // DIRECT: B and C come from the TMA tiles Bt, Ct instead of the fp32
+    // buffer bc.
+    template <bool WITH_Y, bool DIRECT = false>
+    __device__ __forceinline__ float step_group(int e, const float2* ed2, const float* bc, const Tin* Bt = nullptr,
+                                                const Tin* Ct = nullptr) {
+        if constexpr (DIRECT) {
+            float pp[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const int s = G * e + g;
+                const float2 q2 = ed2[s * Ge::CPW + c];
+                float bv[Ge::S], cv[Ge::S];
+                tile_states(Bt, row_of(s), j, bv);
+                if constexpr (WITH_Y) tile_states(Ct, row_of(s), j, cv);
+                float acc = 0.f;
+                if constexpr (Ge::S == 1) {
+                    const float ea = ex2_approx(q2.x * A2[0]);
+                    h[0] = fmaf(ea, h[0], q2.y * bv[0]);
+                    if constexpr (WITH_Y) acc = cv[0] * h[0];
+                } else {
+                    const float2 dd = make_float2(q2.x, q2.x);
+                    const float2 du = make_float2(q2.y, q2.y);
+                    float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int pq = 0; pq < Ge::S / 2; ++pq) {
+                        const float2 v = mul2(dd, make_float2(A2[2 * pq], A2[2 * pq + 1]));
+                        const float2 ea = make_float2(ex2_approx(v.x), ex2_approx(v.y));
+                        const float2 drive = mul2(du, make_float2(bv[2 * pq], bv[2 * pq + 1]));
+                        const float2 hh = fma2(ea, make_float2(h[2 * pq], h[2 * pq + 1]), drive);
+                        h[2 * pq] = hh.x;
+                        h[2 * pq + 1] = hh.y;
+                        if constexpr (WITH_Y) acc2 = fma2(make_float2(cv[2 * pq], cv[2 * pq + 1]), hh, acc2);
+                    }
+                    acc = acc2.x + acc2.y;
+                }
+                pp[g] = acc;
+            }
+            if constexpr (WITH_Y)
+                return group_transpose_reduce<G, Ge::CPW>(pp, j);
+            else
+                return 0.f;
+        }
         float pp[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -202,15 +269,16 @@ __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char
     uint64_t* bar = full + st;
     mbar_arrive_expect_tx(bar, Ge::TX_BASE + (gated ? Ge::TX_Z : 0u));
     const int row0 = k * T;
-    tma_load_3d(sb, &maps.x, bar, ct0, r == 0 ? row0 - 3 : row0, b);
-    tma_load_3d(sb + Ge::XB, &maps.dt[r], bar, ct0, row0, b);
-    if (gated) tma_load_3d(sb + Ge::XB + Ge::DTB, &maps.z, bar, ct0, row0, b);
+    const int x0 = ct0 - ct0 % Ge::XW;  // the aligned tile row around the CTA's channels
+    tma_load_3d(sb, &maps.x, bar, x0, r == 0 ? row0 - 3 : row0, b);
+    tma_load_3d(sb + Ge::XB, &maps.dt[r], bar, x0, row0, b);
+    if (gated) tma_load_3d(sb + Ge::XB + Ge::DTB, &maps.z, bar, x0, row0, b);
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB, &maps.B[r], bar, 0, row0, b);
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY>
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool DIRECT>
 __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
@@ -288,8 +356,13 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
         float* bc = bc32 + (i & 1) * (T * kNState * 2);
-        convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
-        named_bar_sync(1 + DIR, NWD * 32);
+        if constexpr (!DIRECT) convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
+        // every warp of the direction is past the previous chunk (and, unless
+        // DIRECT, the fp32 B/C rows of this one are written)
+        if constexpr (NWD == 1)
+            __syncwarp();
+        else
+            named_bar_sync(1 + DIR, NWD * 32);
         if (leader && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
             issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2,
@@ -304,7 +377,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
 #pragma unroll 2
         for (int e = 0; e < Ge::EPL; ++e) {
-            const float yr = wk.template step_group<true>(e, ed2, bc);
+            const float yr = wk.template step_group<true, DIRECT>(e, ed2, bc, Bt, Ct);
             const int s = G * e + wk.j;
             if (s >= s_lo && s < s_hi && wk.dvalid) {
                 const int tr = Wk::row_of(s);  // token - kT
@@ -312,7 +385,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
                 if (!gated) {
                     wsw[(int64_t)tr * D] = y;
                 } else {
-                    const float zv = ldf(zt, tr * Ge::CW + wk.cc);
+                    const float zv = ldf(zt, tr * Ge::XW + wk.tc);
                     stf(outw, (int64_t)tr * D, (y + ows[tr * Ge::CPW + wk.c]) * silu(zv));
                 }
             }
@@ -342,7 +415,7 @@ constexpr int layer_min_blocks() {
     return (T <= 16 || G >= 16) ? 4 : 3;
 }
 
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false>
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool DIRECT = false>
 __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     layer_tma_kernel(const __grid_constant__ LayerMaps maps, const KParams p) {
     using Ge = TmaGeo<G, T, NWD, NS, Tin>;
@@ -357,9 +430,9 @@ __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     }
     __syncthreads();
     if (warp < NWD)
-        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY>(maps, p, base, warp, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY, DIRECT>(maps, p, base, warp, lane);
     else
-        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY>(maps, p, base, warp - NWD, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY, DIRECT>(maps, p, base, warp - NWD, lane);
 }
 
 // ---------------------------------------------------------------- prefix
@@ -391,7 +464,8 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
     const int64_t P = p.L;
     const int nc = (int)((P + T - 1) / T);
     const bool leader = (wg == 0 && lane == 0);
-    constexpr uint32_t TX = (uint32_t)(((T + 3) * Ge::CW + T * Ge::CW + T * kNState) * Ge::ESZ);
+    constexpr uint32_t TX = (uint32_t)(((T + 3) * Ge::XW + T * Ge::XW + T * kNState) * Ge::ESZ);
+    const int x0 = ct0 - ct0 % Ge::XW;  // the aligned tile row around the CTA's channels
 
     auto issue = [&](int i) {
         if (p.starve) return;
@@ -399,8 +473,8 @@ __global__ void __launch_bounds__(NWD * 32) prefix_tma_kernel(const __grid_const
         unsigned char* sb = base + st * Ge::STAGE;
         uint64_t* bar = full + st;
         mbar_arrive_expect_tx(bar, TX);
-        tma_load_3d(sb, &maps.x, bar, ct0, i * T - 3, b);
-        tma_load_3d(sb + Ge::XB, &maps.dt[0], bar, ct0, i * T, b);
+        tma_load_3d(sb, &maps.x, bar, x0, i * T - 3, b);
+        tma_load_3d(sb + Ge::XB, &maps.dt[0], bar, x0, i * T, b);
         tma_load_3d(sb + Ge::XB + 2 * Ge::DTB, &maps.B[0], bar, 0, i * T, b);
     };
 

@@ -92,6 +92,27 @@ def test_bf16_ragged_fused_kernel(bm, shape, group):
 ALT = 0x2000  # a family's alternative variant (tuning knob)
 
 
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 32, 32), (1, 64, 48), (1, 65, 8), (1, 200, 20)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_ragged_chunked_direct_kernel(bm, shape, dtype):
+    """The chunked kernel with one warp per direction (4-channel CTAs whose
+    bf16 tiles are the aligned 8 channels around them) reading B/C straight
+    from the tiles."""
+    b, L, D = shape
+    if dtype == "fp32" and D % 4:
+        pytest.skip("fp32 rows must be 16-byte units for the TMA path")
+    inp, par = W.make_case(b, L, D, 16, dtype, seed=800 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    flags = (8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT) | ALT
+    got32 = run_layer(bm, inp, par, torch.float32, flags)
+    assert U.normwise(got32, ref) <= (U.GUARD if dtype == "bf16" else U.TOL_FP32)
+    if dtype == "bf16":
+        got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+        assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
 @pytest.mark.parametrize("chunk", [0, 2])  # 16- and 8-token chunks
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
                                    (1, 16, 32), (1, 32, 64), (2, 17, 96), (1, 9, 32)])
@@ -199,7 +220,7 @@ def test_split_kernel_rejects_staging(bm):
     assert e.value.status == bm.BIMAMBA_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16)])
+@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16), (8 << 8) | (1 << 18) | ALT])
 @pytest.mark.parametrize("L", [4096, 65536])
 def test_long_sequence_split_sampled(bm, L, flags):
     """b=1, D=4096, bf16, seed 2: the split-state kernel at long L."""
