@@ -57,9 +57,9 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 # count (its traffic is linear in L); the block step's at a 4096-token prefix
 # (a step reads the same bytes whatever the prefix length).
 NCU_TRAFFIC = {
-    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1304.8e6,
-    ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1414.2e6,
-    ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1414.2e6,
+
+    ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1464.2e6,
+    ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1464.2e6,
     ("block_cached_b16_P65536_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
     ("block_cached_b16_P4096_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
     ("proj_1p3b_b8_L2048_dmodel2048_D4096_bf16", "gemm_bf16_persistent_kernel (input projection)"): 1960.9e6,

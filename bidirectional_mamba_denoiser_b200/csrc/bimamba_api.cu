@@ -262,12 +262,13 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
-template <int G, int T, typename Tin, typename Tout, bool CARRY = false, int NWD = kTWD, bool DIRECT = false>
+template <int G, int T, typename Tin, typename Tout, bool CARRY = false, int NWD = kTWD, bool DIRECT = false,
+          bool FULL_UNROLL = false>
 int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin>;
+    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin, DIRECT>;
     bimamba::LayerMaps maps;
     if (!fill_maps<G, T, Tin, NWD>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT>;
+    auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT, FULL_UNROLL>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -730,7 +731,10 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
             if (out_bf) return fused2_by_chunk<float, bf16>(chunk_field, k, in, st);
             return fused2_by_chunk<float, float>(chunk_field, k, in, st);
         }
-        const bool f32bc = chunk_field == 2;  // family 2: B/C widened once per chunk
+        // B/C widened to fp32 once per chunk at 2 lanes per group (measured
+        // 1.164 against 1.176 ms at batch 8, L 2048); the chunk field's 1
+        // selects the per-use widening
+        const bool f32bc = gf == 2 ? chunk_field != 1 : chunk_field == 2;
         if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, f32bc, k, in, st);
         if (in_bf) return fused_layer_by_group<bf16, float>(gf, f32bc, k, in, st);
         if (out_bf) return fused_layer_by_group<float, bf16>(gf, f32bc, k, in, st);
@@ -738,18 +742,32 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     }
     if (!(flags & BIMAMBA_NO_TMA) && (forced == 0 || forced >= 4) && tma_eligible(in, d_inner, true, true)) {
         const int gt = pick_lanes_tma(2LL * batch * d_inner, flags);
+        // with carries the chunk length is the automatic one (the flag is not honoured)
+        const int tt = with_carry ? pick_chunk_tma(0, gt) : pick_chunk_tma(flags, gt);
+        // 8 lanes per channel with 32-token chunks: one warp per direction per
+        // CTA and B/C read straight from the tile (measured 6.79 against
+        // 7.20 ms at batch 1, L 65536, d_inner 4096: 1024 CTAs spread over the
+        // SMs evenly).  The alternative-variant flag keeps the 4-warp CTAs with
+        // B/C widened once per chunk.
+        if (gt == 8 && tt == 32 && !(flags & kAltVariant)) {
+            if (with_carry) {
+                if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, true>(k, in, st);
+                if (in_bf) return launch_layer_tma<8, 32, bf16, float, true, 1, true>(k, in, st);
+                if (out_bf) return launch_layer_tma<8, 32, float, bf16, true, 1, true>(k, in, st);
+                return launch_layer_tma<8, 32, float, float, true, 1, true>(k, in, st);
+            }
+            if (in_bf && out_bf && (flags & kAltVariant2))  // the group loop fully unrolled (tuning knob)
+                return launch_layer_tma<8, 32, bf16, bf16, false, 1, true, true>(k, in, st);
+            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true>(k, in, st);
+            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true>(k, in, st);
+            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true>(k, in, st);
+            return launch_layer_tma<8, 32, float, float, false, 1, true>(k, in, st);
+        }
         if (with_carry) {
             if (in_bf && out_bf) return layer_tma_carry_by_lanes<bf16, bf16>(gt, k, in, st);
             if (in_bf) return layer_tma_carry_by_lanes<bf16, float>(gt, k, in, st);
             if (out_bf) return layer_tma_carry_by_lanes<float, bf16>(gt, k, in, st);
             return layer_tma_carry_by_lanes<float, float>(gt, k, in, st);
-        }
-        const int tt = pick_chunk_tma(flags, gt);
-        if ((flags & kAltVariant) && gt == 8) {  // one warp per direction, B/C read from the bf16 tile (tuning knob)
-            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true>(k, in, st);
-            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true>(k, in, st);
-            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true>(k, in, st);
-            return launch_layer_tma<8, 32, float, float, false, 1, true>(k, in, st);
         }
         if (in_bf && out_bf) return layer_tma_by_lanes<bf16, bf16>(gt, tt, k, in, st);
         if (in_bf) return layer_tma_by_lanes<bf16, float>(gt, tt, k, in, st);

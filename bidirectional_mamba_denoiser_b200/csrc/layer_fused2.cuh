@@ -6,17 +6,19 @@
 // channel ct0 + l for the per-token work (conv + SiLU, softplus, D skip,
 // output).  Lanes pair up (l, l ^ 1): lane j of a pair holds states
 // [8j, 8j+8) of its own channel and of its partner's, so every B and C it
-// loads serves two channels, the partner's step size and drive arrive by one
-// shuffle, and one more shuffle completes each channel's C.h sum.
+// loads serves two channels, and one shuffle completes each channel's C.h
+// sum.
 //
 // Per chunk of T tokens, after its tiles have landed:
 //  1. B and C are widened to fp32 once ([T][B 16 | C 16], shared by the warp);
 //  2. every lane computes the per-token work of its channel for all T steps
-//     into registers -- T independent chains of conv, SiLU and softplus, so
-//     the special-function unit has work in flight while step 1's stores
-//     settle;
-//  3. the scan walks the T steps with every step size already at hand, so
-//     each step's 16 exps can issue as soon as the unit is free.
+//     -- T independent chains of conv, SiLU and softplus, so the
+//     special-function unit has work in flight -- into a per-warp buffer
+//     (step size, drive, D*u);
+//  3. the scan walks the T steps with every step size already at hand (its
+//     own and its partner's read from the buffer), so each step's 16 exps
+//     can issue as soon as the unit is free; the loop is not unrolled, which
+//     keeps its body in the instruction cache.
 // A CTA is one forward and one reverse warp over the same 32 channels; each
 // warp streams chunks of x (+3-token conv halo), dt, B, C (and z when gated)
 // through its own NS-stage TMA ring; boxes reaching outside [0, L) read
@@ -43,7 +45,9 @@ struct Fused2Geo {
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
     static constexpr int OWS = T * CW * 4;               // partner's y of a chunk
     static constexpr int BCF = T * 2 * kNState * 4;      // fp32 B | C rows of a chunk
-    static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF;
+    static constexpr int ED = T * CW * 8;                // (delta, delta*u) of the chunk's steps
+    static constexpr int EDU = T * CW * 4;               // D*u of the chunk's steps
+    static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF + ED + EDU;
     static constexpr int BAR_OFF = 2 * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
     static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
@@ -75,6 +79,8 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
     float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS);
+    float2* ed = reinterpret_cast<float2*>(wbase + NS * Ge::STAGE + Ge::OWS + Ge::BCF);
+    float* edu = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS + Ge::BCF + Ge::ED);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + Ge::BAR_OFF) + DIR * NS;
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
@@ -158,7 +164,6 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
         // 2. per-token work of the own channel for the chunk's T steps (step s:
         // token kT + s forward, kT + T-1-s reverse; the forward x tile starts
         // 3 tokens early)
-        float dl[T], du[T], Du[T];
         {
             float x0 = ldf(xt, (DIR == 0 ? 0 : T + 2) * Ge::CW + lane);
             float x1 = ldf(xt, (DIR == 0 ? 1 : T + 1) * Ge::CW + lane);
@@ -174,10 +179,9 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
                 const float u = silu(cv);
                 const float dlt = softplus(ldf(dtt, (DIR == 0 ? s : T - 1 - s) * Ge::CW + lane) + bias);
                 const bool valid = s >= s_lo && s < s_hi;
-                dl[s] = valid ? dlt : 0.f;
-                du[s] = valid ? dlt * u : 0.f;
-                Du[s] = valid ? Dd * u : 0.f;
-                if constexpr (CARRY) dsum += dl[s];
+                ed[s * Ge::CW + lane] = valid ? make_float2(dlt, dlt * u) : make_float2(0.f, 0.f);
+                edu[s * Ge::CW + lane] = valid ? Dd * u : 0.f;
+                if constexpr (CARRY) dsum += valid ? dlt : 0.f;
             }
         }
         if (gated) cp_async_wait_all();
@@ -186,16 +190,15 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
         // 3. the scan
         float* wsw = p.ws + chunk_row * D + d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + d;
-#pragma unroll
+#pragma unroll 1
         for (int s = 0; s < T; ++s) {
             const int row = DIR == 0 ? s : T - 1 - s;
-            const float dlp = __shfl_xor_sync(0xffffffffu, dl[s], 1);
-            const float dup = __shfl_xor_sync(0xffffffffu, du[s], 1);
+            const float2 eo = ed[s * Ge::CW + lane], ep = ed[s * Ge::CW + (lane ^ 1)];
             float bv[8], cvv[8];
             load_states<8>(bcf + row * 2 * kNState + 8 * j, bv);
             load_states<8>(bcf + row * 2 * kNState + kNState + 8 * j, cvv);
-            const float2 ddo = make_float2(dl[s], dl[s]), uuo = make_float2(du[s], du[s]);
-            const float2 ddp = make_float2(dlp, dlp), uup = make_float2(dup, dup);
+            const float2 ddo = make_float2(eo.x, eo.x), uuo = make_float2(eo.y, eo.y);
+            const float2 ddp = make_float2(ep.x, ep.x), uup = make_float2(ep.y, ep.y);
             float2 ao[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             float2 ap[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -204,10 +207,10 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
                 const float2 cq = make_float2(cvv[q], cvv[q + 1]);
                 const float2 vo = mul2(ddo, make_float2(A2o[q], A2o[q + 1]));
                 const float2 vp = mul2(ddp, make_float2(A2p[q], A2p[q + 1]));
-                const float2 eo = make_float2(ex2_approx(vo.x), ex2_approx(vo.y));
-                const float2 ep = make_float2(ex2_approx(vp.x), ex2_approx(vp.y));
-                const float2 no = fma2(eo, make_float2(ho[q], ho[q + 1]), mul2(uuo, bq));
-                const float2 np = fma2(ep, make_float2(hp[q], hp[q + 1]), mul2(uup, bq));
+                const float2 xo = make_float2(ex2_approx(vo.x), ex2_approx(vo.y));
+                const float2 xp = make_float2(ex2_approx(vp.x), ex2_approx(vp.y));
+                const float2 no = fma2(xo, make_float2(ho[q], ho[q + 1]), mul2(uuo, bq));
+                const float2 np = fma2(xp, make_float2(hp[q], hp[q + 1]), mul2(uup, bq));
                 ho[q] = no.x; ho[q + 1] = no.y;
                 hp[q] = np.x; hp[q + 1] = np.y;
                 ao[(q >> 1) & 1] = fma2(cq, no, ao[(q >> 1) & 1]);
@@ -217,7 +220,7 @@ __device__ __forceinline__ void fused2_direction(const FusedMaps& maps, const KP
             const float mine = (ao[0].x + ao[1].x) + (ao[0].y + ao[1].y);
             const float theirs = (ap[0].x + ap[1].x) + (ap[0].y + ap[1].y);
             const float yr = mine + __shfl_xor_sync(0xffffffffu, theirs, 1);
-            const float y = (yr + Du[s]) * scale;
+            const float y = (yr + edu[s * Ge::CW + lane]) * scale;
             if (s >= s_lo && s < s_hi && dvalid) {
                 if (!gated) {
                     wsw[(int64_t)row * D] = y;

@@ -44,7 +44,9 @@
 namespace bimamba {
 
 // XSM: the step sizes and drives reach the scanning lanes through a per-warp
-// shared-memory buffer (one 8-byte load per step) instead of two shuffles.
+// shared-memory buffer (one 8-byte load per step) instead of two shuffles,
+// and D*u likewise, so the scan loop need not be unrolled (a smaller loop
+// body stays in the instruction cache).
 template <int T, int NWD, int NS, typename Tin, bool XSM = false>
 struct SplitGeo {
     static_assert(T % 4 == 0 && T + 3 <= 256, "chunk");
@@ -61,7 +63,8 @@ struct SplitGeo {
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
     static constexpr int OWS = T * CPW * 4;               // per warp: partner's y of a chunk
     static constexpr int EDX = XSM ? T * CPW * 8 : 0;     // per warp: (delta, delta*u) of the chunk's steps
-    static constexpr int WARP_BYTES = OWS + EDX;
+    static constexpr int EDU = XSM ? T * CPW * 4 : 0;     // per warp: D*u of the chunk's steps
+    static constexpr int WARP_BYTES = OWS + EDX + EDU;
     static constexpr int DIR_BYTES = NS * STAGE;
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
     static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
@@ -156,7 +159,10 @@ struct SplitWorker {
             dl[e] = valid ? dlt : 0.f;
             du[e] = valid ? dlt * u : 0.f;
             Du[e] = valid ? Dd * u : 0.f;
-            if constexpr (XSM) edx[s * Ge::CPW + c] = make_float2(dl[e], du[e]);
+            if constexpr (XSM) {
+                edx[s * Ge::CPW + c] = make_float2(dl[e], du[e]);
+                reinterpret_cast<float*>(edx + T * Ge::CPW)[s * Ge::CPW + c] = Du[e];
+            }
             if constexpr (DSUM) dsum += dl[e];
         }
     }
@@ -337,19 +343,31 @@ __device__ __forceinline__ void split_direction(const LayerMaps& maps, const KPa
 
         float* wsw = p.ws + chunk_row * D + wk.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
-#pragma unroll
-        for (int e = 0; e < Ge::EPL; ++e) {
-            const float yr = PHASED ? wk.step_group_phased(e, Bt, Ct, edx) : wk.step_group(e, Bt, Ct, edx);
+        auto finish = [&](int e, float yr, float du_own) {
             const int s = 4 * e + wk.j;
             if (s >= s_lo && s < s_hi && wk.dvalid) {
                 const int tr = Wk::row_of(s);  // token - kT
-                const float y = (yr + wk.Du[e]) * scale;
+                const float y = (yr + du_own) * scale;
                 if (!gated) {
                     wsw[(int64_t)tr * D] = y;
                 } else {
                     const float zv = ldf(zt, tr * Ge::CW + wk.cc);
                     stf(outw, (int64_t)tr * D, (y + ows[tr * Ge::CPW + wk.c]) * silu(zv));
                 }
+            }
+        };
+        if constexpr (XSM) {
+            const float* edu = reinterpret_cast<const float*>(edx + T * Ge::CPW);
+#pragma unroll 2
+            for (int e = 0; e < Ge::EPL; ++e) {
+                const float yr = PHASED ? wk.step_group_phased(e, Bt, Ct, edx) : wk.step_group(e, Bt, Ct, edx);
+                finish(e, yr, edu[(4 * e + wk.j) * Ge::CPW + wk.c]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < Ge::EPL; ++e) {
+                const float yr = PHASED ? wk.step_group_phased(e, Bt, Ct, edx) : wk.step_group(e, Bt, Ct, edx);
+                finish(e, yr, wk.Du[e]);
             }
         }
         // every warp of this direction is done with stage st: refill it

@@ -49,7 +49,9 @@ struct LayerMaps {
 
 constexpr int align128(int v) { return (v + 127) & ~127; }
 
-template <int G, int T, int NWD, int NS, typename Tin>
+// DIRECT: B and C are read straight from the TMA tiles, so the fp32 B/C
+// buffers are not allocated.
+template <int G, int T, int NWD, int NS, typename Tin, bool DIRECT = false>
 struct TmaGeo {
     static_assert(G == 4 || G == 8 || G == 16, "lanes per channel");
     static_assert(T % G == 0 && T <= 253, "chunk");
@@ -70,7 +72,7 @@ struct TmaGeo {
     static constexpr int EDU = T * CPW * 4;               // per warp: D*u
     static constexpr int OWS = T * CPW * 4;               // per warp: partner's y
     static constexpr int WARP_BYTES = ED2 + EDU + OWS;
-    static constexpr int DIR_BYTES = NS * STAGE + 2 * BC32;
+    static constexpr int DIR_BYTES = NS * STAGE + (DIRECT ? 0 : 2 * BC32);
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
     static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;  // + alignment slack
@@ -278,10 +280,11 @@ __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool DIRECT>
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool DIRECT,
+          bool FULL_UNROLL = false>
 __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
-    using Ge = TmaGeo<G, T, NWD, NS, Tin>;
+    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT>;
     using Wk = TmaWorker<G, T, NWD, NS, Tin, DIR>;
     unsigned char* dir_base = base + DIR * Ge::DIR_BYTES;
     float* bc32 = reinterpret_cast<float*>(dir_base + NS * Ge::STAGE);
@@ -375,7 +378,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
 
         float* wsw = p.ws + chunk_row * D + wk.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
-#pragma unroll 2
+#pragma unroll (FULL_UNROLL ? Ge::EPL : 2)
         for (int e = 0; e < Ge::EPL; ++e) {
             const float yr = wk.template step_group<true, DIRECT>(e, ed2, bc, Bt, Ct);
             const int s = G * e + wk.j;
@@ -415,10 +418,11 @@ constexpr int layer_min_blocks() {
     return (T <= 16 || G >= 16) ? 4 : 3;
 }
 
-template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool DIRECT = false>
+template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool DIRECT = false,
+          bool FULL_UNROLL = false>
 __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     layer_tma_kernel(const __grid_constant__ LayerMaps maps, const KParams p) {
-    using Ge = TmaGeo<G, T, NWD, NS, Tin>;
+    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~static_cast<uintptr_t>(127));
@@ -430,9 +434,9 @@ __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     }
     __syncthreads();
     if (warp < NWD)
-        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY, DIRECT>(maps, p, base, warp, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY, DIRECT, FULL_UNROLL>(maps, p, base, warp, lane);
     else
-        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY, DIRECT>(maps, p, base, warp - NWD, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY, DIRECT, FULL_UNROLL>(maps, p, base, warp - NWD, lane);
 }
 
 // ---------------------------------------------------------------- prefix

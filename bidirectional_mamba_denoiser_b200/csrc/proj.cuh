@@ -150,9 +150,22 @@ __device__ __forceinline__ void gemm_store8(const GemmParams& p, int m, int n, c
 // (2 x 256 columns) and commits "accumulator full"; warps 2-5 drain the other
 // accumulator -- warp w reads TMEM lanes 32 (w % 4) .. +31 -- and hand it back
 // ("accumulator empty", one arrival per warp), so a tile's stores overlap the
-// next tile's products.  Tiles run along N first, so consecutive tiles of a CTA
-// reuse the A rows from L2.  Every wait is bounded.
+// next tile's products.  Tiles are taken in the banded order of
+// gemm_tile_origin.  Every wait is bounded.
 constexpr int kGemmPThreads = 192;
+constexpr int kGemmBand = 64;  // M tiles per band of the tile order
+
+// Tile t of the persistent order -> (m0, n0).  Tiles run M-fastest inside
+// bands of kGemmBand M tiles, band after band: the CTAs of one wave share a
+// few W column slices (each read from DRAM once per band) and a band's A
+// rows (kGemmBand x 128 rows) stay in L2 while the band sweeps N.
+__device__ __forceinline__ void gemm_tile_origin(int t, int tiles_m, int tiles_n, int& m0, int& n0) {
+    const int per_band = kGemmBand * tiles_n;
+    const int band = t / per_band, r = t % per_band;
+    const int bm = min(kGemmBand, tiles_m - band * kGemmBand);  // M tiles in this band
+    m0 = (band * kGemmBand + r % bm) * kGemmBM;
+    n0 = (r / bm) * kGemmBN;
+}
 
 __global__ void __launch_bounds__(kGemmPThreads, 1) gemm_bf16_persistent_kernel(
     const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, const GemmParams p) {
@@ -167,7 +180,8 @@ __global__ void __launch_bounds__(kGemmPThreads, 1) gemm_bf16_persistent_kernel(
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int nk = p.K / kGemmBK;
     const int tiles_n = (p.N + kGemmBN - 1) / kGemmBN;
-    const int tiles = tiles_n * ((p.M + kGemmBM - 1) / kGemmBM);
+    const int tiles_m = (p.M + kGemmBM - 1) / kGemmBM;
+    const int tiles = tiles_n * tiles_m;
 
     if (t == 0) {
         for (int i = 0; i < 2 * kGemmStages + 2; ++i) mbar_init(full + i, 1);
@@ -184,7 +198,8 @@ __global__ void __launch_bounds__(kGemmPThreads, 1) gemm_bf16_persistent_kernel(
     if (t == 0) {  // producer
         int g = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+            int m0, n0;
+            gemm_tile_origin(tile, tiles_m, tiles_n, m0, n0);
             for (int kt = 0; kt < nk; ++kt, ++g) {
                 const int s = g % kGemmStages;
                 if (g >= kGemmStages) mbar_wait_bounded(empty + s, (uint32_t)(((g / kGemmStages) - 1) & 1), p.wait_limit);
@@ -220,7 +235,8 @@ __global__ void __launch_bounds__(kGemmPThreads, 1) gemm_bf16_persistent_kernel(
         int i = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
             const int acc = i & 1;
-            const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+            int m0, n0;
+            gemm_tile_origin(tile, tiles_m, tiles_n, m0, n0);
             mbar_wait_bounded(acc_full + acc, (uint32_t)((i >> 1) & 1), p.wait_limit);
             tmem_fence_after_sync();
             const int m = m0 + 32 * q + lane;

@@ -84,7 +84,7 @@ def test_roofline_fields():
     assert r["peak"] == pytest.approx(148 * 16 * 1965e6 / 1e9, rel=1e-4)
     assert r["achieved"] == pytest.approx(ops / 1e-3 / 1e9, rel=1e-4)
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], abs=1e-4)
-    assert bench.roofline(ops, 1.0, None, "layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel")["traffic"] > 0
+    assert bench.roofline(ops, 1.0, None, "long_b1_L65536_D4096_bf16", "layer_tma_kernel")["traffic"] > 0
 
 
 def test_every_workload_resolves_and_names_its_sizes():

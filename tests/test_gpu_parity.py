@@ -68,20 +68,21 @@ def test_bf16_ragged_tma_kernel(bm, shape, lanes, chunk):
     assert bm.bimamba_device_error() == 0
 
 
-@pytest.mark.parametrize("group", [1, 2, 4, 8, "2f", "4f"])
+@pytest.mark.parametrize("group", [1, 2, 4, 8, "2u", "4f"])
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
                                    (1, 16, 32), (1, 32, 64), (2, 17, 96)])
 def test_bf16_ragged_fused_kernel(bm, shape, group):
     """The per-token fused kernel (16-token chunks, one lane per channel,
-    B/C shared by groups of lanes; "f": B/C widened to fp32 once per chunk):
-    one, two and many chunks, ragged last chunks and a last CTA whose 32
-    channels are partly past d_inner."""
+    B/C shared by groups of lanes; 2 lanes widen B/C to fp32 once per chunk
+    unless the chunk field is 1 ("u": per use), 4 lanes per use unless it
+    is 2 ("f")): one, two and many chunks, ragged last chunks and a last CTA
+    whose 32 channels are partly past d_inner."""
     b, L, D = shape
     inp, par = W.make_case(b, L, D, 16, "bf16", seed=300 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    f32bc = isinstance(group, str)
-    g = int(group[0]) if f32bc else group
-    flags = (g << 8) | (2 << bm.BIMAMBA_FAMILY_SHIFT) | ((2 << bm.BIMAMBA_CHUNK_SHIFT) if f32bc else 0)
+    g = int(group[0]) if isinstance(group, str) else group
+    chunk = {"u": 1, "f": 2}[group[1]] if isinstance(group, str) else 0
+    flags = (g << 8) | (2 << bm.BIMAMBA_FAMILY_SHIFT) | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
     got32 = run_layer(bm, inp, par, torch.float32, flags)
     assert U.normwise(got32, ref) <= U.GUARD
     got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
@@ -96,21 +97,22 @@ ALT = 0x2000  # a family's alternative variant (tuning knob)
                                    (1, 32, 32), (1, 64, 48), (1, 65, 8), (1, 200, 20)])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_ragged_chunked_direct_kernel(bm, shape, dtype):
-    """The chunked kernel with one warp per direction (4-channel CTAs whose
-    bf16 tiles are the aligned 8 channels around them) reading B/C straight
-    from the tiles."""
+    """The chunked kernel at 8 lanes per channel in both forms: one warp per
+    direction (4-channel CTAs whose bf16 tiles are the aligned 8 channels
+    around them) reading B/C straight from the tiles (the default), and the
+    4-warp CTAs with B/C widened once per chunk (the alternative flag)."""
     b, L, D = shape
     if dtype == "fp32" and D % 4:
         pytest.skip("fp32 rows must be 16-byte units for the TMA path")
     inp, par = W.make_case(b, L, D, 16, dtype, seed=800 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    flags = (8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT) | ALT
-    got32 = run_layer(bm, inp, par, torch.float32, flags)
-    assert U.normwise(got32, ref) <= (U.GUARD if dtype == "bf16" else U.TOL_FP32)
-    if dtype == "bf16":
-        got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
-        assert U.bf16_out_ok(got16, ref)
-    assert bm.bimamba_device_error() == 0
+    for flags in ((8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT), (8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT) | ALT):
+        got32 = run_layer(bm, inp, par, torch.float32, flags)
+        assert U.normwise(got32, ref) <= (U.GUARD if dtype == "bf16" else U.TOL_FP32), hex(flags)
+        if dtype == "bf16":
+            got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
+            assert U.bf16_out_ok(got16, ref)
+        assert bm.bimamba_device_error() == 0
 
 
 @pytest.mark.parametrize("chunk", [0, 2])  # 16- and 8-token chunks
