@@ -15,6 +15,7 @@
 #include "context_cache.h"
 #include "layer_fused.cuh"
 #include "layer_fused2.cuh"
+#include "layer_pscan.cuh"
 #include "layer_split.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
@@ -366,6 +367,32 @@ int launch_layer_split(const KParams& k, const bimamba_inputs_t* in, cudaStream_
     return launch_status();
 }
 
+// ---- chunked parallel scan (few channels: 8 pieces of 8 steps per channel and chunk)
+
+constexpr int kPNS = 2;  // pipeline stages per direction
+
+template <int NWD, typename Tin, typename Tout, bool CARRY = false>
+int launch_layer_pscan(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
+    using Ge = bimamba::PscanGeo<NWD, kPNS, Tin>;
+    const bool bf = std::is_same<Tin, bf16>::value;
+    constexpr int N = bimamba::kNState, T = Ge::T;
+    bimamba::LayerMaps m;
+    bool ok = map3d(&m.x, in->x, bf, k.D, k.L, k.batch, Ge::XW, T + 3);
+    ok = ok && map3d(&m.z, in->z, bf, k.D, k.L, k.batch, Ge::XW, T);
+    for (int r = 0; r < 2; ++r) {
+        ok = ok && map3d(&m.dt[r], in->dt[r], bf, k.D, k.L, k.batch, Ge::XW, T);
+        ok = ok && map3d(&m.B[r], in->B[r], bf, N, k.L, k.batch, N, T);
+        ok = ok && map3d(&m.C[r], in->C[r], bf, N, k.L, k.batch, N, T);
+    }
+    if (!ok) return BIMAMBA_ERR_CUDA;
+    auto kern = &bimamba::layer_pscan_kernel<NWD, kPNS, Tin, Tout, CARRY>;
+    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
+    if (rc) return rc;
+    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
+    kern<<<grid, 2 * NWD * 32, Ge::SMEM, st>>>(m, k);
+    return launch_status();
+}
+
 // Chunk of the split-state kernel: the chunk field's 2 = 32 tokens, 3 = 64
 // (0 = automatic: 32); warps per direction: the lane field (1 or 2; 0 = 1).
 template <typename Tin, typename Tout>
@@ -373,12 +400,7 @@ int layer_split_by(unsigned flags, const KParams& k, const bimamba_inputs_t* in,
     const unsigned ch = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
     const unsigned nw = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int t = ch == 3 ? 64 : 32;
-    if ((flags & kAltVariant) && (flags & kAltVariant2))  // shared-memory exchange, phased scan steps
-        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, true, true>(k, in, st)
-                       : launch_layer_split<32, 1, Tin, Tout, false, true, true>(k, in, st);
-    if (flags & kAltVariant2)  // phased scan steps
-        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, false, true>(k, in, st)
-                       : launch_layer_split<32, 1, Tin, Tout, false, false, true>(k, in, st);
+    if (flags & kAltVariant2) return launch_layer_pscan<2, Tin, Tout>(k, in, st);  // the chunked parallel scan
     if (flags & kAltVariant) {
         if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout, false, true>(k, in, st)
                                     : launch_layer_split<32, 2, Tin, Tout, false, true>(k, in, st);
@@ -747,21 +769,20 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
         // 8 lanes per channel with 32-token chunks: one warp per direction per
         // CTA and B/C read straight from the tile (measured 6.79 against
         // 7.20 ms at batch 1, L 65536, d_inner 4096: 1024 CTAs spread over the
-        // SMs evenly).  The alternative-variant flag keeps the 4-warp CTAs with
+        // SMs evenly),  The alternative-variant flag keeps the 4-warp CTAs with
         // B/C widened once per chunk.
         if (gt == 8 && tt == 32 && !(flags & kAltVariant)) {
+            // the group loop fully unrolled: 6.24 against 6.77 ms at the same size
             if (with_carry) {
-                if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, true>(k, in, st);
-                if (in_bf) return launch_layer_tma<8, 32, bf16, float, true, 1, true>(k, in, st);
-                if (out_bf) return launch_layer_tma<8, 32, float, bf16, true, 1, true>(k, in, st);
-                return launch_layer_tma<8, 32, float, float, true, 1, true>(k, in, st);
+                if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, true, true>(k, in, st);
+                if (in_bf) return launch_layer_tma<8, 32, bf16, float, true, 1, true, true>(k, in, st);
+                if (out_bf) return launch_layer_tma<8, 32, float, bf16, true, 1, true, true>(k, in, st);
+                return launch_layer_tma<8, 32, float, float, true, 1, true, true>(k, in, st);
             }
-            if (in_bf && out_bf && (flags & kAltVariant2))  // the group loop fully unrolled (tuning knob)
-                return launch_layer_tma<8, 32, bf16, bf16, false, 1, true, true>(k, in, st);
-            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true>(k, in, st);
-            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true>(k, in, st);
-            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true>(k, in, st);
-            return launch_layer_tma<8, 32, float, float, false, 1, true>(k, in, st);
+            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true, true>(k, in, st);
+            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true, true>(k, in, st);
+            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true, true>(k, in, st);
+            return launch_layer_tma<8, 32, float, float, false, 1, true, true>(k, in, st);
         }
         if (with_carry) {
             if (in_bf && out_bf) return layer_tma_carry_by_lanes<bf16, bf16>(gt, k, in, st);

@@ -153,7 +153,7 @@ def test_fused2_kernel_single_direction(bm, flag):
     assert U.normwise(got, ref) <= U.TOL_FP32
 
 
-@pytest.mark.parametrize("variant", [ALT, 0x8000, ALT | 0x8000])  # shared-memory exchange, phased steps, both
+@pytest.mark.parametrize("variant", [0, ALT])  # shuffles, shared-memory exchange
 @pytest.mark.parametrize("chunk", [2, 3])
 def test_split_kernel_variants(bm, chunk, variant):
     for L, D in ((150, 40), (33, 8), (1, 16)):
@@ -161,6 +161,44 @@ def test_split_kernel_variants(bm, chunk, variant):
         ref = oracle.layer_fwd(inp, par)
         got = run_layer(bm, inp, par, torch.float32, SPLIT | variant | (chunk << 16))
         assert U.normwise(got, ref) <= U.GUARD, (L, D)
+
+
+PSCAN = (3 << 18) | 0x8000  # the chunked parallel scan (8 pieces of 8 steps per channel and chunk)
+
+
+@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
+                                   (1, 64, 32), (1, 128, 48), (1, 65, 8), (1, 200, 20), (2, 129, 16), (1, 63, 8)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_ragged_pscan_kernel(bm, shape, dtype):
+    """The chunked parallel scan: chunks of 64 steps cut into 8 pieces whose
+    affine carries are combined by warp shuffles; one, two and many chunks,
+    ragged last chunks (where the reverse walk starts with identity steps),
+    and channel counts that leave the last CTA's 8 channels partly empty."""
+    b, L, D = shape
+    if dtype == "fp32" and D % 4:
+        pytest.skip("fp32 rows must be 16-byte units for the TMA path")
+    inp, par = W.make_case(b, L, D, 16, dtype, seed=900 + L + D)
+    ref = oracle.layer_fwd(inp, par)
+    got32 = run_layer(bm, inp, par, torch.float32, PSCAN)
+    assert U.normwise(got32, ref) <= (U.GUARD if dtype == "bf16" else U.TOL_FP32)
+    if dtype == "bf16":
+        got16 = run_layer(bm, inp, par, torch.bfloat16, PSCAN)
+        assert U.bf16_out_ok(got16, ref)
+    assert bm.bimamba_device_error() == 0
+
+
+@pytest.mark.parametrize("flag", ["fwd", "rev"])
+def test_pscan_single_direction_and_general_A(bm, flag):
+    inp, par = W.make_case(1, 300, 24, 16, "fp32", seed=23)
+    g = torch.Generator().manual_seed(29)
+    par = dict(par)
+    par["A"] = -torch.exp(torch.rand(par["A"].shape, generator=g) * 5.0 - 3.0)
+    par["D"] = torch.rand(par["D"].shape, generator=g) * 2.0 - 1.0
+    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
+    ref = oracle.layer_fwd(inp, par, flags=f)
+    fl = bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY
+    got = run_layer(bm, inp, par, torch.float32, PSCAN | fl)
+    assert U.normwise(got, ref) <= U.TOL_FP32
 
 
 SPLIT = 3 << 18  # the split-state kernel family (4 lanes x 4 states per channel)
@@ -222,7 +260,7 @@ def test_split_kernel_rejects_staging(bm):
     assert e.value.status == bm.BIMAMBA_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16), (8 << 8) | (1 << 18) | ALT])
+@pytest.mark.parametrize("flags", [SPLIT | ALT, (8 << 8) | (1 << 18) | ALT, PSCAN])
 @pytest.mark.parametrize("L", [4096, 65536])
 def test_long_sequence_split_sampled(bm, L, flags):
     """b=1, D=4096, bf16, seed 2: the split-state kernel at long L."""

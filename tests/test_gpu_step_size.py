@@ -130,6 +130,7 @@ LAYER_KERNELS = {
     "staged": 4 << 8 | 0x4000,
     "split_w1_t32": 3 << 18,
     "split_w2_t64": 2 << 8 | 3 << 16 | 3 << 18,
+    "pscan": 3 << 18 | 0x8000,
     "chunked_g8_4warp": 8 << 8 | 1 << 18 | 0x2000,
 }
 
