@@ -58,11 +58,12 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 # (a step reads the same bytes whatever the prefix length).
 NCU_TRAFFIC = {
 
-    ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1464.2e6,
-    ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1464.2e6,
+    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1305.4e6,
+    ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1473.0e6,
+    ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1473.0e6,
     ("block_cached_b16_P65536_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
     ("block_cached_b16_P4096_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
-    ("proj_1p3b_b8_L2048_dmodel2048_D4096_bf16", "gemm_bf16_persistent_kernel (input projection)"): 1960.9e6,
+    ("proj_1p3b_b8_L2048_dmodel2048_D4096_bf16", "gemm_bf16_persistent_kernel (input projection)"): 733.4e6,
 }
 
 
@@ -78,7 +79,7 @@ def parse_args(argv=None):
     ap.add_argument("--lanes", type=int, default=0, help="lanes per channel / group size (0 = library's choice)")
     ap.add_argument("--chunk", type=int, default=0, help="chunk length selector: 0 auto, 1 = 16, 2 = 32")
     ap.add_argument("--family", type=int, default=0,
-                    help="kernel family: 0 auto, 1 chunked, 2 per-token fused, 3 split-state")
+                    help="kernel family: 0 auto, 1 chunked, 2 per-token fused, 3 chunked parallel scan")
     ap.add_argument("--flags", type=lambda v: int(v, 0), default=0, help="further flag bits (tuning knobs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -385,7 +386,7 @@ def kernel_name(w: W.Workload, args) -> str:
     if args.workload in ("block", "decode"):
         return "async_block_kernel"
     fam = args.family or (2 if 2 * w.batch * w.d_inner >= SMS * 8 * 32 else 1)
-    return "fused_layer_kernel" if fam == 2 else "layer_tma_kernel"
+    return {2: "fused_layer_kernel", 3: "layer_pscan_kernel"}.get(fam, "layer_tma_kernel")
 
 
 def layer_input_bytes(batch: int, L: int, D: int, N: int, esz: int) -> int:

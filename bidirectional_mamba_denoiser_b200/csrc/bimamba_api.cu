@@ -14,9 +14,7 @@
 #include "carry.cuh"
 #include "context_cache.h"
 #include "layer_fused.cuh"
-#include "layer_fused2.cuh"
 #include "layer_pscan.cuh"
-#include "layer_split.cuh"
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
 #include "mamba2_ssd.cuh"
@@ -331,42 +329,6 @@ int prefix_tma_by_lanes(int g, const KParams& k, const bimamba_inputs_t* in, cud
     return BIMAMBA_ERR_UNSUPPORTED;
 }
 
-// ---- split-state kernel (few channels: 4 lanes x 4 states per channel)
-
-constexpr int kSNS = 3;  // pipeline stages per direction
-// tuning knob: the alternative variant of a family (split-state: step sizes exchanged through shared
-// memory instead of shuffles; per-token fused: the kernel in phases, layer_fused2.cuh)
-constexpr unsigned kAltVariant = 0x2000u;
-constexpr unsigned kAltVariant2 = 0x8000u;   // split-state: the scan step in phases (tuning knob)
-
-template <int T, int NWD, typename Tin>
-bool fill_split_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
-    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin>;
-    const bool bf = std::is_same<Tin, bf16>::value;
-    constexpr int N = bimamba::kNState;
-    bool ok = map3d(&m.x, in->x, bf, D, L, batch, Ge::CW, T + 3);
-    ok = ok && map3d(&m.z, in->z, bf, D, L, batch, Ge::CW, T);
-    for (int r = 0; r < 2; ++r) {
-        ok = ok && map3d(&m.dt[r], in->dt[r], bf, D, L, batch, Ge::CW, T);
-        ok = ok && map3d(&m.B[r], in->B[r], bf, N, L, batch, N, T);
-        ok = ok && map3d(&m.C[r], in->C[r], bf, N, L, batch, N, T);
-    }
-    return ok;
-}
-
-template <int T, int NWD, typename Tin, typename Tout, bool CARRY = false, bool XSM = false, bool PHASED = false>
-int launch_layer_split(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::SplitGeo<T, NWD, kSNS, Tin, XSM>;
-    bimamba::LayerMaps maps;
-    if (!fill_split_maps<T, NWD, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_split_kernel<T, NWD, kSNS, Tin, Tout, CARRY, XSM, PHASED>;
-    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
-    if (rc) return rc;
-    dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
-    kern<<<grid, 2 * NWD * 32, Ge::SMEM, st>>>(maps, k);
-    return launch_status();
-}
-
 // ---- chunked parallel scan (few channels: 8 pieces of 8 steps per channel and chunk)
 
 constexpr int kPNS = 2;  // pipeline stages per direction
@@ -391,25 +353,6 @@ int launch_layer_pscan(const KParams& k, const bimamba_inputs_t* in, cudaStream_
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
     kern<<<grid, 2 * NWD * 32, Ge::SMEM, st>>>(m, k);
     return launch_status();
-}
-
-// Chunk of the split-state kernel: the chunk field's 2 = 32 tokens, 3 = 64
-// (0 = automatic: 32); warps per direction: the lane field (1 or 2; 0 = 1).
-template <typename Tin, typename Tout>
-int layer_split_by(unsigned flags, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    const unsigned ch = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
-    const unsigned nw = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
-    const int t = ch == 3 ? 64 : 32;
-    if (flags & kAltVariant2) return launch_layer_pscan<2, Tin, Tout>(k, in, st);  // the chunked parallel scan
-    if (flags & kAltVariant) {
-        if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout, false, true>(k, in, st)
-                                    : launch_layer_split<32, 2, Tin, Tout, false, true>(k, in, st);
-        return t == 64 ? launch_layer_split<64, 1, Tin, Tout, false, true>(k, in, st)
-                       : launch_layer_split<32, 1, Tin, Tout, false, true>(k, in, st);
-    }
-    if (nw == 2) return t == 64 ? launch_layer_split<64, 2, Tin, Tout>(k, in, st)
-                                : launch_layer_split<32, 2, Tin, Tout>(k, in, st);
-    return t == 64 ? launch_layer_split<64, 1, Tin, Tout>(k, in, st) : launch_layer_split<32, 1, Tin, Tout>(k, in, st);
 }
 
 // ---- per-token fused kernels (many channels)
@@ -481,41 +424,6 @@ int launch_fused_prefix(const KParams& k, const bimamba_inputs_t* in, cudaStream
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
     kern<<<grid, 32, Ge::SMEM, st>>>(maps, k);
     return launch_status();
-}
-
-// ---- per-token fused kernel in phases (fused2)
-
-template <int T, typename Tin>
-bool fill_fused2_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D) {
-    const bool bf = std::is_same<Tin, bf16>::value;
-    constexpr int N = bimamba::kNState;
-    bool ok = map3d(&m.x, in->x, bf, D, L, batch, 32, T + 3);
-    ok = ok && map3d(&m.z, in->z, bf, D, L, batch, 32, T);
-    for (int r = 0; r < 2; ++r) {
-        ok = ok && map3d(&m.dt[r], in->dt[r], bf, D, L, batch, 32, T);
-        ok = ok && map3d(&m.B[r], in->B[r], bf, N, L, batch, N, T);
-        ok = ok && map3d(&m.C[r], in->C[r], bf, N, L, batch, N, T);
-    }
-    return ok;
-}
-
-template <int T, int NS, typename Tin, typename Tout, bool CARRY = false>
-int launch_fused2_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::Fused2Geo<T, NS, Tin>;
-    bimamba::FusedMaps maps;
-    if (!fill_fused2_maps<T, Tin>(maps, in, k.batch, k.L, k.D)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::fused2_layer_kernel<T, NS, Tin, Tout, CARRY>;
-    int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
-    if (rc) return rc;
-    dim3 grid((unsigned)((k.D + 31) / 32), (unsigned)k.batch);
-    kern<<<grid, 64, Ge::SMEM, st>>>(maps, k);
-    return launch_status();
-}
-
-template <typename Tin, typename Tout>
-int fused2_by_chunk(unsigned chunk_field, const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    if (chunk_field == 2) return launch_fused2_layer<8, 3, Tin, Tout>(k, in, st);
-    return launch_fused2_layer<16, 2, Tin, Tout>(k, in, st);
 }
 
 // Kernel family of the TMA path: forced by the flags, else the per-token
@@ -679,13 +587,9 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || !out) return BIMAMBA_ERR_INVALID_ARG;
     if (d_state != bimamba::kNState) return BIMAMBA_ERR_UNSUPPORTED;
     const unsigned known = BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_LANES_MASK | BIMAMBA_NO_TMA |
-                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE | kAltVariant |
-                           kAltVariant2;
-    const bool split_family = ((flags & BIMAMBA_FAMILY_MASK) >> BIMAMBA_FAMILY_SHIFT) == 3;
+                           BIMAMBA_CHUNK_MASK | BIMAMBA_FAMILY_MASK | BIMAMBA_TEST_STARVE | BIMAMBA_CHUNKED_WIDE;
     const unsigned chunk_field = (flags & BIMAMBA_CHUNK_MASK) >> BIMAMBA_CHUNK_SHIFT;
-    const unsigned lane_field = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
-    if (!split_family && chunk_field == 3) return BIMAMBA_ERR_UNSUPPORTED;
-    if (split_family && (chunk_field == 1 || lane_field > 2)) return BIMAMBA_ERR_UNSUPPORTED;
+    if (chunk_field == 3) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & ~known) || !lanes_ok(flags)) return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -724,18 +628,18 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     const unsigned forced = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
     const int fam = pick_family(2LL * batch * d_inner, flags);
-    if (fam == 3) {  // the split-state kernel: TMA-fed
+    if (fam == 3) {  // the chunked parallel scan: TMA-fed; the lane and chunk fields are not read
         if ((flags & BIMAMBA_NO_TMA) || !tma_eligible(in, d_inner, true, true)) return BIMAMBA_ERR_UNSUPPORTED;
-        if (with_carry) {  // carries: 32-token chunks, one warp per direction (the flags' choice is not honoured)
-            if (in_bf && out_bf) return launch_layer_split<32, 1, bf16, bf16, true>(k, in, st);
-            if (in_bf) return launch_layer_split<32, 1, bf16, float, true>(k, in, st);
-            if (out_bf) return launch_layer_split<32, 1, float, bf16, true>(k, in, st);
-            return launch_layer_split<32, 1, float, float, true>(k, in, st);
+        if (with_carry) {
+            if (in_bf && out_bf) return launch_layer_pscan<2, bf16, bf16, true>(k, in, st);
+            if (in_bf) return launch_layer_pscan<2, bf16, float, true>(k, in, st);
+            if (out_bf) return launch_layer_pscan<2, float, bf16, true>(k, in, st);
+            return launch_layer_pscan<2, float, float, true>(k, in, st);
         }
-        if (in_bf && out_bf) return layer_split_by<bf16, bf16>(flags, k, in, st);
-        if (in_bf) return layer_split_by<bf16, float>(flags, k, in, st);
-        if (out_bf) return layer_split_by<float, bf16>(flags, k, in, st);
-        return layer_split_by<float, float>(flags, k, in, st);
+        if (in_bf && out_bf) return launch_layer_pscan<2, bf16, bf16>(k, in, st);
+        if (in_bf) return launch_layer_pscan<2, bf16, float>(k, in, st);
+        if (out_bf) return launch_layer_pscan<2, float, bf16>(k, in, st);
+        return launch_layer_pscan<2, float, float>(k, in, st);
     }
     const bool group_ok = forced == 0 || forced == 1 || forced == 2 || forced == 4 || forced == 8;
     if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
@@ -747,12 +651,6 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
             return launch_fused_layer<2, float, float, true>(k, in, st);
         }
         const int gf = pick_group_fused(flags);
-        if (flags & kAltVariant) {  // family 2: the phased kernel
-            if (in_bf && out_bf) return fused2_by_chunk<bf16, bf16>(chunk_field, k, in, st);
-            if (in_bf) return fused2_by_chunk<bf16, float>(chunk_field, k, in, st);
-            if (out_bf) return fused2_by_chunk<float, bf16>(chunk_field, k, in, st);
-            return fused2_by_chunk<float, float>(chunk_field, k, in, st);
-        }
         // B/C widened to fp32 once per chunk at 2 lanes per group (measured
         // 1.164 against 1.176 ms at batch 8, L 2048); the chunk field's 1
         // selects the per-use widening
@@ -769,9 +667,10 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
         // 8 lanes per channel with 32-token chunks: one warp per direction per
         // CTA and B/C read straight from the tile (measured 6.79 against
         // 7.20 ms at batch 1, L 65536, d_inner 4096: 1024 CTAs spread over the
-        // SMs evenly),  The alternative-variant flag keeps the 4-warp CTAs with
+        // SMs evenly).  BIMAMBA_CHUNKED_WIDE keeps the 4-warp CTAs with B/C
+        // widened once per chunk.  The alternative-variant flag keeps the 4-warp CTAs with
         // B/C widened once per chunk.
-        if (gt == 8 && tt == 32 && !(flags & kAltVariant)) {
+        if (gt == 8 && tt == 32 && !(flags & BIMAMBA_CHUNKED_WIDE)) {
             // the group loop fully unrolled: 6.24 against 6.77 ms at the same size
             if (with_carry) {
                 if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, true, true>(k, in, st);

@@ -24,7 +24,8 @@
 //     into an NS-stage ring per direction (boxes outside [0, L) read zeros:
 //     the conv padding); the direction's warps widen B and C to fp32 once,
 //     state pairs interleaved and rows in step order, so a lane reads its
-//     piece's 8 B (or C) pairs with four 16-byte loads;
+//     piece's 8 B (or C) pairs with four 16-byte loads (pieces padded apart
+//     so that a channel's 8 lanes read distinct banks);
 //  2. each lane computes conv + SiLU, the step size and D*u of its 8 steps
 //     (a sliding conv window over 11 x rows) into registers;
 //  3. for each of the 8 state pairs (packed f32x2 arithmetic, one MUFU exp2
@@ -60,9 +61,15 @@ struct PscanGeo {
     static constexpr int DTB = align128(T * XW * ESZ);
     static constexpr int BB = align128(T * kNState * ESZ);
     static constexpr int STAGE = XB + 2 * DTB + 2 * BB;   // x, dt, z, B, C
-    static constexpr int BCF = 2 * T * kNState * 4;      // fp32 B then C: [pair 8][step T][2]
-    static constexpr int A2B = CW * kNState * 4;          // A * log2(e) of the CTA's channels
-    static constexpr int CRB = CW * kNState * 4;          // carried state of the CTA's channels
+    // fp32 B then C: [pair 8][piece 8][step 8][2], pieces padded to PS floats and
+    // pairs to QS, so that the 8 pieces of a channel read distinct banks
+    static constexpr int PS = 2 * PL + 4;
+    static constexpr int QS = 8 * PS + 4;
+    static constexpr int BCS = 8 * QS;                    // floats of B (or C)
+    static constexpr int BCF = 2 * BCS * 4;
+    static constexpr int AS = kNState + 2;                // floats per channel row of A and of the carry
+    static constexpr int A2B = CW * AS * 4;               // A * log2(e) of the CTA's channels
+    static constexpr int CRB = CW * AS * 4;               // carried state of the CTA's channels
     static constexpr int OWS = T * CPW * 4;               // per warp: partner's y of a chunk
     static constexpr int DIR_BYTES = NS * STAGE + BCF + A2B + CRB + NWD * OWS;
     static constexpr int BAR_OFF = 2 * DIR_BYTES;
@@ -91,8 +98,9 @@ __device__ __forceinline__ void pscan_issue(const LayerMaps& maps, unsigned char
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
-// B and C of the chunk's T rows -> fp32 [pair q][step][2] (rows in step
-// order), by the direction's NWD warps.
+// B and C of the chunk's T rows -> fp32 pairs in step order (the layout
+// above), by the direction's NWD warps; consecutive threads take consecutive
+// pairs of a row.
 template <int NWD, int NS, typename Tin, int DIR>
 __device__ __forceinline__ void pscan_widen_bc(const Tin* Bt, const Tin* Ct, float* bcf, int tid) {
     using Ge = PscanGeo<NWD, NS, Tin>;
@@ -102,7 +110,8 @@ __device__ __forceinline__ void pscan_widen_bc(const Tin* Bt, const Tin* Ct, flo
         const int row = (e / 8) % T, q = e % 8;
         const Tin* src = (which ? Ct : Bt) + row * kNState + 2 * q;
         const int step = DIR == 0 ? row : T - 1 - row;
-        *reinterpret_cast<float2*>(bcf + which * T * kNState + (q * T + step) * 2) =
+        const int pc = step / Ge::PL, j = step % Ge::PL;
+        *reinterpret_cast<float2*>(bcf + which * Ge::BCS + q * Ge::QS + pc * Ge::PS + 2 * j) =
             make_float2(ldf(src, 0), ldf(src, 1));
     }
 }
@@ -146,8 +155,9 @@ __device__ __forceinline__ void pscan_direction(const LayerMaps& maps, const KPa
     for (int e = tid; e < Ge::CW * kNState; e += NWD * 32) {
         const int ch = ct0 + e / kNState, n = e % kNState;
         const bool ok = ch < D;
-        a2s[e] = ok ? p.A[((int64_t)DIR * D + ch) * kNState + n] * kLog2e : 0.f;
-        crs[e] = (CARRY && ok && p.carry_in[DIR]) ? p.carry_in[DIR][((int64_t)b * D + ch) * kNState + n] : 0.f;
+        const int o = (e / kNState) * Ge::AS + n;
+        a2s[o] = ok ? p.A[((int64_t)DIR * D + ch) * kNState + n] * kLog2e : 0.f;
+        crs[o] = (CARRY && ok && p.carry_in[DIR]) ? p.carry_in[DIR][((int64_t)b * D + ch) * kNState + n] : 0.f;
     }
     float dsum = 0.f;  // step sizes of this lane's valid steps (carries)
 
@@ -237,16 +247,16 @@ __device__ __forceinline__ void pscan_direction(const LayerMaps& maps, const KPa
         float2 y[PL];
 #pragma unroll
         for (int j = 0; j < PL; ++j) y[j] = make_float2(0.f, 0.f);
-        const float* bfp = bcf + PL * pc * 2;                   // pair 0, my first step
-        const float* cfp = bcf + T * kNState + PL * pc * 2;
+        const float* bfp = bcf + pc * Ge::PS;                   // pair 0, my first step
+        const float* cfp = bcf + Ge::BCS + pc * Ge::PS;
 #pragma unroll 1
         for (int q = 0; q < 8; ++q) {
-            const float2 a2 = *reinterpret_cast<const float2*>(a2s + cc * kNState + 2 * q);
-            const float2 carry = *reinterpret_cast<const float2*>(crs + cc * kNState + 2 * q);
+            const float2 a2 = *reinterpret_cast<const float2*>(a2s + cc * Ge::AS + 2 * q);
+            const float2 carry = *reinterpret_cast<const float2*>(crs + cc * Ge::AS + 2 * q);
             float2 bp[PL];
 #pragma unroll
             for (int j = 0; j < PL; j += 2) {
-                const float4 v = *reinterpret_cast<const float4*>(bfp + q * T * 2 + 2 * j);
+                const float4 v = *reinterpret_cast<const float4*>(bfp + q * Ge::QS + 2 * j);
                 bp[j] = make_float2(v.x, v.y);
                 bp[j + 1] = make_float2(v.z, v.w);
             }
@@ -287,11 +297,11 @@ __device__ __forceinline__ void pscan_direction(const LayerMaps& maps, const KPa
             const float2 sin = fma2(Pe, carry, he);  // state entering my piece
             __syncwarp();                            // every lane has read the carry
             if (pc == PL - 1)                        // state after the chunk's last step
-                *reinterpret_cast<float2*>(crs + cc * kNState + 2 * q) = fma2(Pi, carry, hi);
+                *reinterpret_cast<float2*>(crs + cc * Ge::AS + 2 * q) = fma2(Pi, carry, hi);
             // the steps' states and C.h
 #pragma unroll
             for (int j = 0; j < PL; j += 2) {
-                const float4 cv = *reinterpret_cast<const float4*>(cfp + q * T * 2 + 2 * j);
+                const float4 cv = *reinterpret_cast<const float4*>(cfp + q * Ge::QS + 2 * j);
                 y[j] = fma2(make_float2(cv.x, cv.y), fma2(Pl[j], sin, hl[j]), y[j]);
                 y[j + 1] = fma2(make_float2(cv.z, cv.w), fma2(Pl[j + 1], sin, hl[j + 1]), y[j + 1]);
             }
@@ -331,7 +341,9 @@ __device__ __forceinline__ void pscan_direction(const LayerMaps& maps, const KPa
         __syncwarp();
         for (int e = lane; e < Ge::CPW * kNState; e += 32) {
             const int ch = c0w + e / kNState;
-            if (ch < D) p.carry_out[DIR][((int64_t)b * D + ch) * kNState + e % kNState] = crs[wg * Ge::CPW * kNState + e];
+            if (ch < D)
+                p.carry_out[DIR][((int64_t)b * D + ch) * kNState + e % kNState] =
+                    crs[(wg * Ge::CPW + e / kNState) * Ge::AS + e % kNState];
         }
     }
     if (CARRY && p.delta_sum[DIR]) {  // the 8 lanes of a channel are adjacent

@@ -80,9 +80,18 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * size).  1: chunked -- G lanes share one channel's states, for few channels
  * (batch 1, long sequences).  2: per-token fused -- one lane per channel,
  * groups of G lanes share B/C across G channels, for many channels.  With
- * family 2 the lane field (bits 8..12) is the group size (1, 2, 4 or 8). */
+ * family 2 the lane field (bits 8..12) is the group size (1, 2, 4 or 8); at 2
+ * lanes B/C are widened to fp32 once per chunk unless the chunk field is 1,
+ * at 4 only if it is 2.  3: chunked parallel scan -- per 64-token chunk a
+ * channel's 8 lanes scan 8-step pieces and combine their carries with warp
+ * shuffles (the lane and chunk fields are not read).  Tuning knobs: the
+ * result does not depend on the family beyond fp32 rounding order. */
 #define BIMAMBA_FAMILY_SHIFT 18
 #define BIMAMBA_FAMILY_MASK  (0x3u << BIMAMBA_FAMILY_SHIFT)
+/* Family 1 at 8 lanes per channel: 4 warps per direction per CTA with B/C
+ * widened to fp32 once per chunk, instead of one warp per direction reading
+ * B/C from the tile (tuning knob). */
+#define BIMAMBA_CHUNKED_WIDE 0x2000u
 /* Test aid for the failure path: the TMA-fed kernels issue no tile loads,
  * so every wait for a tile gives up (after ~0.1 ms instead of ~2 s); the
  * kernel still finishes, its output is undefined, and bit 0 of

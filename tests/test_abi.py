@@ -97,9 +97,6 @@ def _layer(inp=None, par=None, out=FAKE + 0x20000, out_dtype=bm.BIMAMBA_BF16, ba
     (dict(flags=0x4), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=3 << bm.BIMAMBA_CHUNK_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
-    # the split-state family (3) runs 32- or 64-token chunks and 1 or 2 warps per direction
-    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT | 1 << bm.BIMAMBA_CHUNK_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
-    (dict(flags=3 << bm.BIMAMBA_FAMILY_SHIFT | 4 << bm.BIMAMBA_LANES_SHIFT), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(flags=bm.BIMAMBA_FWD_ONLY | bm.BIMAMBA_REV_ONLY), bm.BIMAMBA_ERR_INVALID_ARG),
     (dict(out_dtype=7), bm.BIMAMBA_ERR_UNSUPPORTED),
     (dict(inp=NULL), bm.BIMAMBA_ERR_INVALID_ARG),

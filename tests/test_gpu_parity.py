@@ -90,7 +90,7 @@ def test_bf16_ragged_fused_kernel(bm, shape, group):
     assert bm.bimamba_device_error() == 0
 
 
-ALT = 0x2000  # a family's alternative variant (tuning knob)
+WIDE = 0x2000  # BIMAMBA_CHUNKED_WIDE
 
 
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
@@ -100,13 +100,13 @@ def test_ragged_chunked_direct_kernel(bm, shape, dtype):
     """The chunked kernel at 8 lanes per channel in both forms: one warp per
     direction (4-channel CTAs whose bf16 tiles are the aligned 8 channels
     around them) reading B/C straight from the tiles (the default), and the
-    4-warp CTAs with B/C widened once per chunk (the alternative flag)."""
+    4-warp CTAs with B/C widened once per chunk (BIMAMBA_CHUNKED_WIDE)."""
     b, L, D = shape
-    if dtype == "fp32" and D % 4:
-        pytest.skip("fp32 rows must be 16-byte units for the TMA path")
+    if D * (4 if dtype == "fp32" else 2) % 16:
+        pytest.skip("rows must be 16-byte units for the TMA-fed kernels")
     inp, par = W.make_case(b, L, D, 16, dtype, seed=800 + L + D)
     ref = oracle.layer_fwd(inp, par)
-    for flags in ((8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT), (8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT) | ALT):
+    for flags in ((8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT), (8 << 8) | (1 << bm.BIMAMBA_FAMILY_SHIFT) | WIDE):
         got32 = run_layer(bm, inp, par, torch.float32, flags)
         assert U.normwise(got32, ref) <= (U.GUARD if dtype == "bf16" else U.TOL_FP32), hex(flags)
         if dtype == "bf16":
@@ -115,55 +115,7 @@ def test_ragged_chunked_direct_kernel(bm, shape, dtype):
         assert bm.bimamba_device_error() == 0
 
 
-@pytest.mark.parametrize("chunk", [0, 2])  # 16- and 8-token chunks
-@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
-                                   (1, 16, 32), (1, 32, 64), (2, 17, 96), (1, 9, 32)])
-def test_bf16_ragged_fused2_kernel(bm, shape, chunk):
-    """The per-token fused kernel in phases (pre-pass of the chunk's per-token
-    work, then the scan): one, two and many chunks, ragged last chunks, a last
-    CTA whose 32 channels are partly past d_inner (and an odd channel count,
-    so a lane's partner channel can be past the end)."""
-    b, L, D = shape
-    inp, par = W.make_case(b, L, D, 16, "bf16", seed=600 + L + D)
-    ref = oracle.layer_fwd(inp, par)
-    flags = (2 << bm.BIMAMBA_FAMILY_SHIFT) | ALT | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
-    got32 = run_layer(bm, inp, par, torch.float32, flags)
-    assert U.normwise(got32, ref) <= U.GUARD
-    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
-    assert U.bf16_out_ok(got16, ref)
-    assert bm.bimamba_device_error() == 0
-
-
-@pytest.mark.parametrize("chunk", [0, 2])
-@pytest.mark.parametrize("L", [1, 7, 8, 9, 16, 17, 33, 100])
-def test_fused2_kernel_fp32(bm, L, chunk):
-    inp, par = W.make_case(2, L, 36, 16, "fp32", seed=700 + L)
-    ref = oracle.layer_fwd(inp, par)
-    got = run_layer(bm, inp, par, torch.float32, (2 << 18) | ALT | (chunk << 16))
-    assert U.normwise(got, ref) <= U.TOL_FP32, L
-
-
-@pytest.mark.parametrize("flag", ["fwd", "rev"])
-def test_fused2_kernel_single_direction(bm, flag):
-    inp, par = W.make_case(1, 200, 64, 16, "fp32", seed=17)
-    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
-    ref = oracle.layer_fwd(inp, par, flags=f)
-    fl = bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY
-    got = run_layer(bm, inp, par, torch.float32, (2 << 18) | ALT | fl)
-    assert U.normwise(got, ref) <= U.TOL_FP32
-
-
-@pytest.mark.parametrize("variant", [0, ALT])  # shuffles, shared-memory exchange
-@pytest.mark.parametrize("chunk", [2, 3])
-def test_split_kernel_variants(bm, chunk, variant):
-    for L, D in ((150, 40), (33, 8), (1, 16)):
-        inp, par = W.make_case(2, L, D, 16, "bf16", seed=18 + L)
-        ref = oracle.layer_fwd(inp, par)
-        got = run_layer(bm, inp, par, torch.float32, SPLIT | variant | (chunk << 16))
-        assert U.normwise(got, ref) <= U.GUARD, (L, D)
-
-
-PSCAN = (3 << 18) | 0x8000  # the chunked parallel scan (8 pieces of 8 steps per channel and chunk)
+PSCAN = 3 << 18  # the chunked parallel scan (8 pieces of 8 steps per channel and chunk)
 
 
 @pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
@@ -175,8 +127,8 @@ def test_ragged_pscan_kernel(bm, shape, dtype):
     ragged last chunks (where the reverse walk starts with identity steps),
     and channel counts that leave the last CTA's 8 channels partly empty."""
     b, L, D = shape
-    if dtype == "fp32" and D % 4:
-        pytest.skip("fp32 rows must be 16-byte units for the TMA path")
+    if D * (4 if dtype == "fp32" else 2) % 16:
+        pytest.skip("rows must be 16-byte units for the TMA-fed kernels")
     inp, par = W.make_case(b, L, D, 16, dtype, seed=900 + L + D)
     ref = oracle.layer_fwd(inp, par)
     got32 = run_layer(bm, inp, par, torch.float32, PSCAN)
@@ -201,69 +153,18 @@ def test_pscan_single_direction_and_general_A(bm, flag):
     assert U.normwise(got, ref) <= U.TOL_FP32
 
 
-SPLIT = 3 << 18  # the split-state kernel family (4 lanes x 4 states per channel)
-
-
-@pytest.mark.parametrize("chunk", [2, 3])  # 32 and 64 tokens
-@pytest.mark.parametrize("nwd", [1, 2])    # warps per direction per CTA
-@pytest.mark.parametrize("shape", [(1, 257, 72), (3, 100, 40), (2, 33, 8), (1, 95, 24), (2, 1, 16),
-                                   (1, 32, 32), (1, 64, 48), (1, 65, 8), (1, 200, 16)])
-def test_bf16_ragged_split_kernel(bm, shape, nwd, chunk):
-    """The split-state kernel: one, two and many chunks, a ragged last chunk
-    (both directions start their walk at a different end of it), and channel
-    counts that leave the last CTA's 8 or 16 channels partly empty."""
-    b, L, D = shape
-    inp, par = W.make_case(b, L, D, 16, "bf16", seed=400 + L + D)
-    ref = oracle.layer_fwd(inp, par)
-    flags = SPLIT | (nwd << 8) | (chunk << bm.BIMAMBA_CHUNK_SHIFT)
-    got32 = run_layer(bm, inp, par, torch.float32, flags)
-    assert U.normwise(got32, ref) <= U.GUARD
-    got16 = run_layer(bm, inp, par, torch.bfloat16, flags)
-    assert U.bf16_out_ok(got16, ref)
-    assert bm.bimamba_device_error() == 0
-
-
-@pytest.mark.parametrize("L", [1, 3, 31, 32, 33, 63, 64, 65, 127, 129])
-@pytest.mark.parametrize("flags", [SPLIT, SPLIT | (2 << 8) | (3 << 16)])
-def test_split_kernel_fp32(bm, L, flags):
-    inp, par = W.make_case(2, L, 20, 16, "fp32", seed=500 + L)
-    ref = oracle.layer_fwd(inp, par)
-    got = run_layer(bm, inp, par, torch.float32, flags)
-    assert U.normwise(got, ref) <= U.TOL_FP32, (L, hex(flags))
-
-
-@pytest.mark.parametrize("flag", ["fwd", "rev"])
-def test_split_kernel_single_direction(bm, flag):
-    inp, par = W.make_case(1, 300, 24, 16, "fp32", seed=13)
-    f = oracle.FWD_ONLY if flag == "fwd" else oracle.REV_ONLY
-    ref = oracle.layer_fwd(inp, par, flags=f)
-    fl = bm.BIMAMBA_FWD_ONLY if flag == "fwd" else bm.BIMAMBA_REV_ONLY
-    got = run_layer(bm, inp, par, torch.float32, SPLIT | fl)
-    assert U.normwise(got, ref) <= U.TOL_FP32
-
-
-def test_split_kernel_general_A_and_D(bm):
-    inp, par = W.make_case(1, 180, 32, 16, "fp32", seed=15)
-    g = torch.Generator().manual_seed(19)
-    par = dict(par)
-    par["A"] = -torch.exp(torch.rand(par["A"].shape, generator=g) * 5.0 - 3.0)
-    par["D"] = torch.rand(par["D"].shape, generator=g) * 2.0 - 1.0
-    ref = oracle.layer_fwd(inp, par)
-    got = run_layer(bm, inp, par, torch.float32, SPLIT | (2 << 8))
-    assert U.normwise(got, ref) <= U.TOL_FP32
-
-
-def test_split_kernel_rejects_staging(bm):
+def test_pscan_rejects_staging(bm):
     inp, par = W.make_case(1, 64, 16, 16, "bf16", seed=1, device="cuda")
     with pytest.raises(bm.BimambaError) as e:
-        bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, flags=SPLIT | bm.BIMAMBA_NO_TMA)
+        bm.bimamba_layer_fwd(inp["x"], inp["z"], inp["dt"], inp["B"], inp["C"], par, flags=PSCAN | bm.BIMAMBA_NO_TMA)
     assert e.value.status == bm.BIMAMBA_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("flags", [SPLIT | ALT, (8 << 8) | (1 << 18) | ALT, PSCAN])
+@pytest.mark.parametrize("flags", [(8 << 8) | (1 << 18) | WIDE, PSCAN])
 @pytest.mark.parametrize("L", [4096, 65536])
-def test_long_sequence_split_sampled(bm, L, flags):
-    """b=1, D=4096, bf16, seed 2: the split-state kernel at long L."""
+def test_long_sequence_other_kernels_sampled(bm, L, flags):
+    """b=1, D=4096, bf16, seed 2: the 4-warp chunked kernel and the parallel
+    scan at long L (the default kernel is checked by test_long_sequence_sampled)."""
     err, ok16 = _sampled_layer_check(bm, W.LONG_SEQ[L], 12, flags)
     assert err <= U.GUARD and ok16
 
@@ -344,7 +245,7 @@ def _sampled_layer_check(bm, w: W.Workload, nchan: int, flags=0):
     return U.normwise(g32, ref), U.bf16_out_ok(g16, ref)
 
 
-@pytest.mark.parametrize("flags", [0, 1 << 18, (2 << 18) | 0x2000, (2 << 18) | 0x2000 | (2 << 16)])
+@pytest.mark.parametrize("flags", [0, 1 << 18, (2 << 18) | (2 << 8) | (1 << 16)])
 def test_layer_1p3b_shape_sampled(bm, flags):
     """b=8, L=2048, D=4096, bf16, seed 1 -- the launch configuration the
     bench times (flags 0) and the chunked kernel; 48 channels of every batch

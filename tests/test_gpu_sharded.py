@@ -13,7 +13,7 @@ from tests import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
-FAMILIES = {"fused": 2 << 18, "chunked": 1 << 18, "split": 3 << 18}
+FAMILIES = {"fused": 2 << 18, "chunked": 1 << 18, "pscan": 3 << 18}
 
 
 @pytest.fixture(scope="module")

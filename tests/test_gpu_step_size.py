@@ -123,14 +123,10 @@ LAYER_KERNELS = {
     "fused_g2": 2 << 8 | 2 << 18,
     "fused_g1": 1 << 8 | 2 << 18,
     "fused_g2_peruse": 2 << 8 | 1 << 16 | 2 << 18,
-    "fused2_t16": 2 << 18 | 0x2000,
-    "fused2_t8": 2 << 18 | 0x2000 | 2 << 16,
     "chunked_g8": 8 << 8 | 1 << 18,
     "chunked_g4": 4 << 8 | 1 << 18,
     "staged": 4 << 8 | 0x4000,
-    "split_w1_t32": 3 << 18,
-    "split_w2_t64": 2 << 8 | 3 << 16 | 3 << 18,
-    "pscan": 3 << 18 | 0x8000,
+    "pscan": 3 << 18,
     "chunked_g8_4warp": 8 << 8 | 1 << 18 | 0x2000,
 }
 
