@@ -668,8 +668,7 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
         // CTA and B/C read straight from the tile (measured 6.79 against
         // 7.20 ms at batch 1, L 65536, d_inner 4096: 1024 CTAs spread over the
         // SMs evenly).  BIMAMBA_CHUNKED_WIDE keeps the 4-warp CTAs with B/C
-        // widened once per chunk.  The alternative-variant flag keeps the 4-warp CTAs with
-        // B/C widened once per chunk.
+        // widened once per chunk.
         if (gt == 8 && tt == 32 && !(flags & BIMAMBA_CHUNKED_WIDE)) {
             // the group loop fully unrolled: 6.24 against 6.77 ms at the same size
             if (with_carry) {

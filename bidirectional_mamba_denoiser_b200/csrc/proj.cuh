@@ -35,28 +35,44 @@ namespace bimamba {
 // One warp per token row, 8 rows per CTA of 256 threads: lane l holds the
 // 16-byte chunks l, l + 32, ... (CPL of them, d <= 256 CPL) in registers, so
 // the mean, the centred sum of squares and the output need one read of the
-// row and warp shuffles only.  d % 8 == 0; batch row = row / L.
+// row and warp shuffles only.  The chunks stay packed bf16 and are widened
+// at each of the three uses (exact), so that a thread needs 4 registers per
+// chunk rather than 8: up to d = 2048, 64 registers a thread and 32 rows
+// (warps) resident per SM keep twice as many rows' loads in flight.
+// d % 8 == 0; batch row = row / L.
+// Widening as opaque single instructions: the compiler would otherwise keep
+// the widened fp32 row from the first use to the last (the 8 registers a
+// chunk that packing saves).
+__device__ __forceinline__ float bf16_lo(uint32_t w) {
+    uint32_t o;
+    asm volatile("shl.b32 %0, %1, 16;" : "=r"(o) : "r"(w));
+    return __uint_as_float(o);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w) {
+    uint32_t o;
+    asm volatile("and.b32 %0, %1, 0xffff0000;" : "=r"(o) : "r"(w));
+    return __uint_as_float(o);
+}
+
 template <int CPL>
-__global__ void __launch_bounds__(256) adaln_kernel(const __nv_bfloat16* x, const float* gamma, const float* beta,
+__global__ void __launch_bounds__(256, CPL <= 8 ? 4 : 1) adaln_kernel(const __nv_bfloat16* x, const float* gamma, const float* beta,
                                                     __nv_bfloat16* out, int64_t rows, int64_t L, int d, float eps) {
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
     const __nv_bfloat16* xr = x + row * d;
-    float v[CPL][8];
-    float s = 0.f;
+    uint4 q[CPL];
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
         const int c = 8 * (lane + 32 * i);
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (c < d) q = *reinterpret_cast<const uint4*>(xr + c);
-        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+        q[i] = c < d ? *reinterpret_cast<const uint4*>(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float s = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
-            v[i][2 * u] = __uint_as_float(w4[u] << 16);
-            v[i][2 * u + 1] = __uint_as_float(w4[u] & 0xffff0000u);
-            s += v[i][2 * u] + v[i][2 * u + 1];
-        }
+    for (int i = 0; i < CPL; ++i) {
+        const uint32_t w4[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s += bf16_lo(w4[u]) + bf16_hi(w4[u]);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
@@ -65,8 +81,13 @@ __global__ void __launch_bounds__(256) adaln_kernel(const __nv_bfloat16* x, cons
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
         if (8 * (lane + 32 * i) < d) {
+            const uint32_t w4[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) q2 = fmaf(v[i][u] - mu, v[i][u] - mu, q2);
+            for (int u = 0; u < 4; ++u) {
+                const float e0 = bf16_lo(w4[u]) - mu, e1 = bf16_hi(w4[u]) - mu;
+                q2 = fmaf(e0, e0, q2);
+                q2 = fmaf(e1, e1, q2);
+            }
         }
     }
 #pragma unroll
@@ -83,15 +104,16 @@ __global__ void __launch_bounds__(256) adaln_kernel(const __nv_bfloat16* x, cons
         const float4 b0 = *reinterpret_cast<const float4*>(be + c), b1 = *reinterpret_cast<const float4*>(be + c + 4);
         const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
         const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        uint32_t w4[4];
+        const uint32_t w4[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+        uint32_t o4[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const float a0 = fmaf(gg[2 * u], (v[i][2 * u] - mu) * rstd, bb[2 * u]);
-            const float a1 = fmaf(gg[2 * u + 1], (v[i][2 * u + 1] - mu) * rstd, bb[2 * u + 1]);
+            const float a0 = fmaf(gg[2 * u], (bf16_lo(w4[u]) - mu) * rstd, bb[2 * u]);
+            const float a1 = fmaf(gg[2 * u + 1], (bf16_hi(w4[u]) - mu) * rstd, bb[2 * u + 1]);
             const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-            w4[u] = *reinterpret_cast<const uint32_t*>(&h);
+            o4[u] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        *reinterpret_cast<uint4*>(out + row * d + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        *reinterpret_cast<uint4*>(out + row * d + c) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
 }
 
