@@ -691,9 +691,9 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
         # dense equivalent that also multiplies the masked zeros) are reported
         # beside it.
         res["roofline"] = roofline_hbm(mamba2_bytes(w.batch, w.L, H, P, N), call_ms, w.name,
-                                       "m2_prep + m2_ssd_kernel (both directions)")
+                                       "m2_prep + m2_ssd dual-form kernel (both directions)")
         res["tensor_executed"] = roofline_tensor(mamba2_ssd_flops(w.batch, w.L, H, P, N), call_ms, w.name,
-                                                 "m2_ssd_kernel executed MMA")
+                                                 "m2_ssd dual-form kernel executed MMA")
         res["fp32_equivalent"] = roofline_fma(flops, call_ms, clocks, w.name, "recurrence-equivalent")
     else:
         res["roofline"] = roofline_fma(flops, call_ms, clocks, w.name, "m2_prep_kernel + 2 x m2_scan_kernel")

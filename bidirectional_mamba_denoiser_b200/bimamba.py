@@ -34,6 +34,7 @@ BIMAMBA_NO_TMA = 0x4000
 BIMAMBA_CHUNK_SHIFT = 16
 BIMAMBA_FAMILY_SHIFT = 18
 BIMAMBA_CHUNKED_WIDE = 0x2000
+BIMAMBA_M2_NO_CLUSTER = 0x8000
 BIMAMBA_TEST_STARVE = 0x100000
 
 D_STATE = 16

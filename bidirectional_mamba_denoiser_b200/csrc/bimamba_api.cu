@@ -922,13 +922,14 @@ namespace {
 size_t m2_round(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct M2Layout {
-    size_t v, dl, yf, yb, tiles, total;
+    size_t v, dl, yf, yb, tiles, sync, total;
 };
 
 // Workspace: conv features [2][batch][L][CH] fp32 (step-by-step path),
 // step sizes [2][batch][H][L], forward and reverse outputs [batch][L][H*P]
 // each, all fp32, then the fp16 C/B tiles of the tensor-core path
-// [2][batch][ceil(L/128)][2][128 x 128]; each part 256-byte aligned.
+// [2][batch][ceil(L/128)][2][128 x 128], then its ticket counter and one
+// flag per (batch row, head), int32; each part 256-byte aligned.
 M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
     const size_t CH = (size_t)H * P + 2 * (size_t)N;
     const size_t nc = (size_t)((L + bimamba::kSQ - 1) / bimamba::kSQ);
@@ -938,7 +939,8 @@ M2Layout m2_layout(int batch, int64_t L, int H, int P, int N) {
     l.yf = l.dl + m2_round(2 * (size_t)batch * (size_t)H * (size_t)L * 4);
     l.yb = l.yf + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
     l.tiles = l.yb + m2_round((size_t)batch * (size_t)L * (size_t)H * P * 4);
-    l.total = l.tiles + 2 * (size_t)batch * nc * 2 * (size_t)bimamba::kTileBytes;
+    l.sync = l.tiles + m2_round(2 * (size_t)batch * nc * 2 * (size_t)bimamba::kTileBytes);
+    l.total = l.sync + (1 + (size_t)batch * H) * 4;
     return l;
 }
 
@@ -950,19 +952,18 @@ bool m2_sizes_ok(int batch, int64_t L, int H) {
 
 // Chunked dual form on the tensor cores: the C/B chunk tiles, then the
 // directions' chunk scans, which compute the x features and step sizes
-// themselves -- both in one launch as clusters of two CTAs that meet halfway
-// when one direction's grid leaves SMs idle, else the forward then the
-// reverse (two or three launches; when L is not a whole number of chunks, the
+// themselves -- both in one launch, as clusters of two CTAs that meet halfway
+// when one direction's grid leaves SMs idle, else as ticket-ordered CTAs
+// (forwards first, each reverse after its forward; the ticket counter and
+// flags are cleared first).  When L is not a whole number of chunks, the
 // ragged chunk's tiles are cleared first so that its rows past the end read
-// zeros).
+// zeros.
 template <typename Tin, typename Tout>
-int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
+int launch_m2_ssd(const bimamba::M2Params& k, bool no_cluster, cudaStream_t st) {
     auto kc = &bimamba::m2_ssd_cluster_kernel<Tin, Tout>;
-    auto k0 = &bimamba::m2_ssd_kernel<0, Tin, Tout>;
-    auto k1 = &bimamba::m2_ssd_kernel<1, Tin, Tout>;
+    auto kt = &bimamba::m2_ssd_ticket_kernel<Tin, Tout>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kc), bimamba::kSsdSmem);
-    if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k0), bimamba::kSsdSmem);
-    if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(k1), bimamba::kSsdSmem);
+    if (!rc) rc = ensure_smem(reinterpret_cast<const void*>(kt), bimamba::kSsdSmem);
     if (rc) return rc;
     const int64_t nc = (k.L + bimamba::kSQ - 1) / bimamba::kSQ;
     if (k.L % bimamba::kSQ) {  // the ragged chunk: the forward's last, the reverse's first in step order
@@ -978,19 +979,19 @@ int launch_m2_ssd(const bimamba::M2Params& k, cudaStream_t st) {
     bimamba::m2_prep_kernel<Tin, true><<<g1, 128, 0, st>>>(k);
     if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
     // one direction's grid within one wave (2 CTAs per SM): both directions at once, as
-    // clusters that meet halfway; else the forward, then the reverse (measured faster
-    // there: 0.80 against 0.89 ms at batch 8, L 2048, 120 heads)
+    // clusters that meet halfway; else ticket-ordered CTAs (the clustered form measured
+    // 0.89 against 0.80 ms for a forward launch and then a reverse one at batch 8, L 2048,
+    // 120 heads)
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return BIMAMBA_ERR_CUDA;
-    if ((int64_t)k.H * k.batch <= 2LL * sms) {
+    if (!no_cluster && (int64_t)k.H * k.batch <= 2LL * sms) {
         kc<<<dim3((unsigned)(2 * k.H), (unsigned)k.batch), 128, bimamba::kSsdSmem, st>>>(k);
         return launch_status();
     }
-    const dim3 g2((unsigned)k.H, (unsigned)k.batch);
-    k0<<<g2, 128, bimamba::kSsdSmem, st>>>(k);
-    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    k1<<<g2, 128, bimamba::kSsdSmem, st>>>(k);
+    const int64_t n1 = (int64_t)k.H * k.batch;
+    if (cudaMemsetAsync(k.sync, 0, (size_t)(1 + n1) * sizeof(int), st) != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    kt<<<(unsigned)(2 * n1), 128, bimamba::kSsdSmem, st>>>(k);
     return launch_status();
 }
 
@@ -1152,7 +1153,7 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
                        unsigned flags, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     if (!in || !p || !out || !m2_sizes_ok(batch, L, nheads)) return BIMAMBA_ERR_INVALID_ARG;
     if (headdim != bimamba::kM2P || d_state != bimamba::kM2N) return BIMAMBA_ERR_UNSUPPORTED;
-    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_NO_TMA | BIMAMBA_TEST_STARVE))
+    if (flags & ~(BIMAMBA_FWD_ONLY | BIMAMBA_REV_ONLY | BIMAMBA_NO_TMA | BIMAMBA_TEST_STARVE | BIMAMBA_M2_NO_CLUSTER))
         return BIMAMBA_ERR_UNSUPPORTED;
     if ((flags & BIMAMBA_FWD_ONLY) && (flags & BIMAMBA_REV_ONLY)) return BIMAMBA_ERR_INVALID_ARG;
     if (!dtype_ok(in->dtype) || !dtype_ok(out_dtype)) return BIMAMBA_ERR_UNSUPPORTED;
@@ -1197,12 +1198,15 @@ int bimamba2_layer_fwd(const bimamba2_inputs_t* in, const bimamba2_params_t* p, 
     k.dir_scale[1] = (flags & BIMAMBA_FWD_ONLY) ? 0.f : 1.f;
     k.starve = (flags & BIMAMBA_TEST_STARVE) ? 1 : 0;
     k.wait_limit = k.starve ? kStarveWaitCycles : kWaitCycles;
+    k.meet_limit = k.starve ? kStarveWaitCycles : kWaitCycles;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = in->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
     if (in_bf && !(flags & BIMAMBA_NO_TMA)) {
         k.tiles = ws + lay.tiles;
-        if (out_bf) return launch_m2_ssd<bf16, bf16>(k, st);
-        return launch_m2_ssd<bf16, float>(k, st);
+        k.sync = reinterpret_cast<int*>(ws + lay.sync);
+        const bool no_cluster = (flags & BIMAMBA_M2_NO_CLUSTER) != 0;
+        if (out_bf) return launch_m2_ssd<bf16, bf16>(k, no_cluster, st);
+        return launch_m2_ssd<bf16, float>(k, no_cluster, st);
     }
     if (in_bf && out_bf) return launch_m2<bf16, bf16>(k, st);
     if (in_bf) return launch_m2<bf16, float>(k, st);

@@ -223,41 +223,42 @@ struct TmaWorker {
                 return group_transpose_reduce<G, Ge::CPW>(pp, j);
             else
                 return 0.f;
-        }
-        float pp[G];
+        } else {
+            float pp[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const int s = G * e + g;
-            const float2 q2 = ed2[s * Ge::CPW + c];
-            const float* row = bc + row_of(s) * 2 * kNState;
-            float acc = 0.f;
-            if constexpr (Ge::S == 1) {
-                const float ea = ex2_approx(q2.x * A2[0]);
-                h[0] = fmaf(ea, h[0], q2.y * row[bc_quad_index(j)]);
-                if constexpr (WITH_Y) acc = row[bc_quad_index(j) + 2] * h[0];
-            } else {
-                const float2 dd = make_float2(q2.x, q2.x);
-                const float2 du = make_float2(q2.y, q2.y);
-                float2 acc2 = make_float2(0.f, 0.f);
+            for (int g = 0; g < G; ++g) {
+                const int s = G * e + g;
+                const float2 q2 = ed2[s * Ge::CPW + c];
+                const float* row = bc + row_of(s) * 2 * kNState;
+                float acc = 0.f;
+                if constexpr (Ge::S == 1) {
+                    const float ea = ex2_approx(q2.x * A2[0]);
+                    h[0] = fmaf(ea, h[0], q2.y * row[bc_quad_index(j)]);
+                    if constexpr (WITH_Y) acc = row[bc_quad_index(j) + 2] * h[0];
+                } else {
+                    const float2 dd = make_float2(q2.x, q2.x);
+                    const float2 du = make_float2(q2.y, q2.y);
+                    float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int pq = 0; pq < Ge::S / 2; ++pq) {
-                    const float4 bcq = *reinterpret_cast<const float4*>(row + (j * Ge::S / 2 + pq) * 4);
-                    const float2 v = mul2(dd, make_float2(A2[2 * pq], A2[2 * pq + 1]));
-                    const float2 ea = make_float2(ex2_approx(v.x), ex2_approx(v.y));
-                    const float2 drive = mul2(du, make_float2(bcq.x, bcq.y));
-                    const float2 hh = fma2(ea, make_float2(h[2 * pq], h[2 * pq + 1]), drive);
-                    h[2 * pq] = hh.x;
-                    h[2 * pq + 1] = hh.y;
-                    if constexpr (WITH_Y) acc2 = fma2(make_float2(bcq.z, bcq.w), hh, acc2);
+                    for (int pq = 0; pq < Ge::S / 2; ++pq) {
+                        const float4 bcq = *reinterpret_cast<const float4*>(row + (j * Ge::S / 2 + pq) * 4);
+                        const float2 v = mul2(dd, make_float2(A2[2 * pq], A2[2 * pq + 1]));
+                        const float2 ea = make_float2(ex2_approx(v.x), ex2_approx(v.y));
+                        const float2 drive = mul2(du, make_float2(bcq.x, bcq.y));
+                        const float2 hh = fma2(ea, make_float2(h[2 * pq], h[2 * pq + 1]), drive);
+                        h[2 * pq] = hh.x;
+                        h[2 * pq + 1] = hh.y;
+                        if constexpr (WITH_Y) acc2 = fma2(make_float2(bcq.z, bcq.w), hh, acc2);
+                    }
+                    acc = acc2.x + acc2.y;
                 }
-                acc = acc2.x + acc2.y;
+                pp[g] = acc;
             }
-            pp[g] = acc;
+            if constexpr (WITH_Y)
+                return group_transpose_reduce<G, Ge::CPW>(pp, j);
+            else
+                return 0.f;
         }
-        if constexpr (WITH_Y)
-            return group_transpose_reduce<G, Ge::CPW>(pp, j);
-        else
-            return 0.f;
     }
 };
 

@@ -68,10 +68,15 @@ struct M2Params {
     int H, CH, batch;
     float dir_scale[2];    // 1, or 0 for a disabled direction (test flags)
     long long wait_limit;  // SM clocks a wait for a tile or a product may take (tensor-core path)
+    long long meet_limit;  // SM clocks a reverse CTA may wait for its forward (tensor-core path)
     int starve;            // test aid (tensor-core path): issue no tile copies, so every wait gives up
     // tensor-core path: the prep kernel writes only the fp16 C/B tiles
     // ([2][batch][ceil(L/128)][C | B] x 128 x 128, rows in step order)
     unsigned char* tiles;
+    // tensor-core path, directions as separate CTAs of one launch: [0] the
+    // next ticket, [1 + b H + h] set once the forward (head h, batch row b)
+    // has stored its y; zeroed before the launch
+    int* sync;
     // block-cached decoding (step-by-step scan): the forward direction's cached
     // state [batch][H][P][N] fp32 and conv tail [batch][3][CH] (xBC rows before
     // token 0, oldest first); nullptr = zero state / zero halo / no commit

@@ -45,7 +45,7 @@ namespace bimamba {
 
 constexpr int kSQ = kM2Chunk;               // steps per chunk (= MMA M)
 constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
-// shared memory of m2_ssd_kernel
+// shared memory of one dual-form CTA (either kernel)
 constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
               kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90728, kSsdX = 90752, kSsdE = 101232,
               kSsdCW = 101744, kSsdCB = 102256, kSsdSmem = 102384;
@@ -92,7 +92,7 @@ __device__ __forceinline__ void cluster_meet() {
 // it the forward stores y for every chunk (p.YF) and the reverse, launched
 // after it, gates every chunk with that y.
 template <int DIR, typename Tin, typename Tout, bool CL>
-__device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm, const int h) {
+__device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm, const int h, const int b) {
     constexpr int Q = kSQ, P = kM2P;
     static_assert(sizeof(Tin) == 2, "the dual form reads bf16 inputs");
     unsigned char* sC = sm + kSsdC;
@@ -110,7 +110,6 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
     float* sCB = reinterpret_cast<float*>(sm + kSsdCB);    // [32]: conv bias
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int b = blockIdx.y;
     const int64_t L = p.L;
     const int H = p.H, HP = H * P;
     const int nc = (int)((L + Q - 1) / Q);
@@ -472,17 +471,69 @@ template <typename Tin, typename Tout>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 2) m2_ssd_cluster_kernel(const M2Params p) {
     extern __shared__ __align__(128) unsigned char sm[];
     if (blockIdx.x & 1)
-        m2_ssd_dir<1, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1));
+        m2_ssd_dir<1, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1), (int)blockIdx.y);
     else
-        m2_ssd_dir<0, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1));
+        m2_ssd_dir<0, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1), (int)blockIdx.y);
 }
 
-// grid (H, batch), block 128, dynamic shared memory kSsdSmem: one direction;
-// the forward launch stores y_0, the reverse launch after it gates.
-template <int DIR, typename Tin, typename Tout>
-__global__ void __launch_bounds__(128, 2) m2_ssd_kernel(const M2Params p) {
+// Both directions as separate CTAs of one launch, for calls whose
+// per-direction grid fills the GPU: grid (2 H batch), block 128, dynamic
+// shared memory kSsdSmem.  Each CTA takes a ticket from p.sync[0] when it
+// starts; tickets [0, H batch) run the forward of (h, b) = (ticket mod H,
+// ticket / H) and store its y for every chunk, the rest the reverse of the
+// same pairs in the same order, which gates with that y.  A reverse CTA
+// waits for its forward's flag before its first chunk.  The forward CTA holds
+// a smaller ticket, so it has started by then and only waits on its own
+// copies and products: the wait always ends.  It is still bounded (p.meet_limit,
+// ~2 s; on timeout bit 1 of the device error word is set and the CTA carries
+// on).
+// Compared with a forward launch followed by a reverse launch, the reverse
+// CTAs fill the SMs the forward's last partial wave leaves idle.
+constexpr unsigned kErrPartnerTimeout = 2u;
+
+__device__ __forceinline__ void m2_flag_release(int* f) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(1) : "memory");
+}
+__device__ __forceinline__ int m2_flag_acquire(const int* f) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(128, 2) m2_ssd_ticket_kernel(const M2Params p) {
     extern __shared__ __align__(128) unsigned char sm[];
-    m2_ssd_dir<DIR, Tin, Tout, false>(p, sm, (int)blockIdx.x);
+    __shared__ int ticket;
+    if (threadIdx.x == 0) ticket = atomicAdd(p.sync, 1);
+    __syncthreads();
+    const int n1 = p.H * p.batch;
+    const int tk = ticket;
+    if (tk < n1) {
+        m2_ssd_dir<0, Tin, Tout, false>(p, sm, tk % p.H, tk / p.H);
+        // every thread's y stores are visible device-wide before the flag
+        __threadfence();
+        __syncthreads();
+        // (under the starving test aid the flag is never set, so that the
+        // reverse's bounded wait is exercised too)
+        if (threadIdx.x == 0 && !p.starve) m2_flag_release(p.sync + 1 + tk);
+    } else {
+        const int x = tk - n1;
+        if (threadIdx.x == 0) {
+            const int* f = p.sync + 1 + x;
+            if (!m2_flag_acquire(f)) {
+                const long long t0 = clock64();
+                while (!m2_flag_acquire(f)) {
+                    if (clock64() - t0 > p.meet_limit) {
+                        atomicOr(&g_device_error, kErrPartnerTimeout);
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+            }
+        }
+        __syncthreads();
+        m2_ssd_dir<1, Tin, Tout, false>(p, sm, x % p.H, x / p.H);
+    }
 }
 
 }  // namespace bimamba

@@ -92,6 +92,11 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * widened to fp32 once per chunk, instead of one warp per direction reading
  * B/C from the tile (tuning knob). */
 #define BIMAMBA_CHUNKED_WIDE 0x2000u
+/* bimamba2_layer_fwd, tensor-core path: run the two directions as separate
+ * ticket-ordered CTAs of one launch even when one direction's grid fits in
+ * one wave, where the clustered form is otherwise taken (test aid; the result
+ * does not depend on it beyond fp32 rounding order). */
+#define BIMAMBA_M2_NO_CLUSTER 0x8000u
 /* Test aid for the failure path: the TMA-fed kernels issue no tile loads,
  * so every wait for a tile gives up (after ~0.1 ms instead of ~2 s); the
  * kernel still finishes, its output is undefined, and bit 0 of
@@ -288,7 +293,8 @@ typedef struct {
 
 /* Bytes of device workspace bimamba2_layer_fwd needs (fp32 conv features of
  * both directions, step sizes, the forward and reverse outputs, the tensor
- * path's C/B tiles); 0 for invalid sizes. */
+ * path's C/B tiles, its ticket counter and per-(batch row, head) flags); 0
+ * for invalid sizes. */
 size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, int d_state);
 
 /* The full-sequence Mamba-2 mixer.  out: [batch][L][nheads*headdim] of
@@ -301,14 +307,20 @@ size_t bimamba2_workspace_bytes(int batch, int64_t L, int nheads, int headdim, i
  * from xbc and dt themselves: when batch * nheads <= 2 x the SM count both
  * run in one launch as the two CTAs of a thread-block cluster (each stores
  * its y over the first half of its walk and, after meeting at a cluster
- * barrier, combines and gates over the second half), else the forward and
- * then the reverse (which gates); plus a clearing of the ragged chunk's tiles
- * when L % 128 != 0.  fp32 inputs, or flags with
+ * barrier, combines and gates over the second half), else in one launch as
+ * separate CTAs ordered by tickets taken at their start (the forwards first,
+ * storing y; each reverse waits for its own forward's flag, then gates; the
+ * counter and flags are cleared by a memset before the launch); plus a
+ * clearing of the ragged chunk's tiles when L % 128 != 0.  A reverse CTA's
+ * wait is bounded (~2 s): on timeout bit 1 of bimamba_device_error() is set
+ * and the output is undefined.  fp32 inputs, or flags with
  * BIMAMBA_NO_TMA, run the step-by-step scan on the CUDA cores in fp32: three
- * launches.  Other flags: BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY (test aids);
+ * launches.  Other flags: BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY, BIMAMBA_M2_NO_CLUSTER (test aids);
  * BIMAMBA_TEST_STARVE (tensor-core path: no tile copies are issued, every
- * wait gives up after ~0.1 ms and sets bit 0 of bimamba_device_error(); the
- * output is undefined).  Nothing is launched when a check fails.  Returns
+ * wait gives up after ~0.1 ms and sets bit 0 of bimamba_device_error(); in
+ * the ticket-ordered form no forward sets its flag either, so every reverse
+ * CTA's wait gives up after ~0.1 ms and sets bit 1; the output is
+ * undefined).  Nothing is launched when a check fails.  Returns
  * BIMAMBA_OK or a negative status. */
 int bimamba2_layer_fwd(const bimamba2_inputs_t *in, const bimamba2_params_t *p,
                        void *out, bimamba_dtype_t out_dtype,
@@ -405,7 +417,8 @@ int bimamba_features(const bimamba_inputs_t *in, const bimamba_params_t *p, int 
 
 /* Read (and, if reset != 0, clear) the error word of the current device.
  * Kernels never wait without bound: a wait for a tile that gives up after
- * about two seconds sets bit 0 (a tile load that never arrived) and the kernel
+ * about two seconds sets bit 0 (a tile load that never arrived), a Mamba-2
+ * reverse CTA's wait for its forward that gives up sets bit 1, and the kernel
  * finishes with undefined output instead of hanging.  Synchronises the
  * device.  Returns the word, or BIMAMBA_ERR_CUDA if it cannot be read. */
 int bimamba_device_error(int reset);

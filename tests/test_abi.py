@@ -214,10 +214,13 @@ def _m2_call(inp=None, par=None, out=FAKE + 0x50000, out_dtype=bm.BIMAMBA_BF16, 
 
 def test_mamba2_workspace_bytes():
     # conv features 2*b*L*CH + step sizes 2*b*H*L + forward and reverse outputs 2*b*L*H*P,
-    # fp32, then fp16 C and B tiles of 128 x 128 per chunk of 128 steps and direction
+    # fp32, then fp16 C and B tiles of 128 x 128 per chunk of 128 steps and direction, then
+    # the ticket counter and one flag per (batch row, head), int32 (every part a multiple of
+    # 256 bytes at this size)
     b, L, H = 8, 2048, 120
     CH = H * 32 + 256
-    want = 2 * b * L * CH * 4 + 2 * b * H * L * 4 + 2 * b * L * H * 32 * 4 + 2 * b * (L // 128) * 2 * 128 * 128 * 2
+    want = (2 * b * L * CH * 4 + 2 * b * H * L * 4 + 2 * b * L * H * 32 * 4 + 2 * b * (L // 128) * 2 * 128 * 128 * 2
+            + (1 + b * H) * 4)
     assert bm.bimamba2_workspace_bytes(b, L, H) == want
     assert bm.bimamba2_workspace_bytes(0, 10, 4) == 0
     assert bm.bimamba2_workspace_bytes(1, 0, 4) == 0

@@ -56,35 +56,58 @@ def test_bf16_inputs(bm, path):
     assert U.bf16_out_ok(got16, want)
 
 
+# the two launch forms of the tensor path: clusters whose CTAs meet halfway
+# (chosen while batch * nheads <= 2 x the SM count), and ticket-ordered CTAs
+# (forwards first, each reverse after its forward; forced by the flag)
+FORMS = {"cluster": 0, "tickets": 0x8000}
+
+
 @pytest.mark.parametrize("shape", [(3, 300, 120), (1, 383, 300), (3, 129, 100)])
 def test_tensor_path_both_launch_forms(bm, shape):
-    """batch * nheads above 2 x the SM count runs the forward and reverse
-    launches one after the other, at or below it one clustered launch whose
-    CTAs meet halfway: both, with ragged L (the chunks of the two directions
-    aligned in token space), within the 2e-3 bound."""
+    """batch * nheads above 2 x the SM count (360, 300 and 300 (head, batch
+    row) pairs against 296) takes the ticket-ordered form without the flag;
+    here with ragged L (the chunks of the two directions aligned in token
+    space) and, in the 3-row cases, reverse CTAs of one batch row waiting on
+    forwards of another.  Each form once more below the threshold, forced."""
     b, L, H = shape
     inp, par = W.make_mamba2_case(b, L, H, P, N, "bf16", seed=66 + L)
     want = oracle.mamba2_layer_fwd(inp, par)
     got = run(bm, inp, par, torch.float32)
     assert bm.bimamba_device_error() == 0
     assert U.normwise(got, want) <= U.TOL_BF16
+    small, spar = W.make_mamba2_case(2, 300, 40, P, N, "bf16", seed=67)
+    swant = oracle.mamba2_layer_fwd(small, spar)
+    for flags in FORMS.values():
+        assert U.normwise(run(bm, small, spar, torch.float32, flags=flags), swant) <= U.TOL_BF16
 
 
+@pytest.mark.parametrize("form", sorted(FORMS))
 @pytest.mark.parametrize("L", [1, 2, 127, 128, 129, 256, 383])
-def test_tensor_path_ragged_lengths(bm, L):
-    """Chunks of 128 steps: lengths around the chunk edge, both directions."""
+def test_tensor_path_ragged_lengths(bm, L, form):
+    """Chunks of 128 steps: lengths around the chunk edge, both directions,
+    both launch forms."""
     inp, par = W.make_mamba2_case(2, L, 3, P, N, "bf16", seed=70 + L)
-    got = run(bm, inp, par, torch.float32)
+    got = run(bm, inp, par, torch.float32, flags=FORMS[form])
+    assert bm.bimamba_device_error() == 0
     assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
 
 
+@pytest.mark.parametrize("form", sorted(FORMS))
 @pytest.mark.parametrize("which", ["fwd", "rev"])
-def test_tensor_path_direction_flags(bm, which):
+def test_tensor_path_direction_flags(bm, which, form):
     inp, par = W.make_mamba2_case(1, 200, 2, P, N, "bf16", seed=71)
     f_or = oracle.FWD_ONLY if which == "fwd" else oracle.REV_ONLY
     f_bm = bm.BIMAMBA_FWD_ONLY if which == "fwd" else bm.BIMAMBA_REV_ONLY
-    got = run(bm, inp, par, torch.float32, flags=f_bm)
+    got = run(bm, inp, par, torch.float32, flags=f_bm | FORMS[form])
     assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par, flags=f_or)) <= U.TOL_BF16
+
+
+def test_tensor_path_tickets_bf16_output(bm):
+    """The ticket-ordered form with bf16 output: within one bf16 rounding + 2e-3."""
+    inp, par = W.make_mamba2_case(3, 260, 5, P, N, "bf16", seed=74)
+    want = oracle.mamba2_layer_fwd(inp, par)
+    got16 = run(bm, inp, par, torch.bfloat16, flags=FORMS["tickets"])
+    assert U.bf16_out_ok(got16, want)
 
 
 @pytest.mark.parametrize("dt_value", [4.0, -9.0])
@@ -95,15 +118,20 @@ def test_tensor_path_extreme_step_sizes(bm, dt_value):
     assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
 
 
-def test_tensor_path_starved_waits_give_up(bm):
+@pytest.mark.parametrize("form", sorted(FORMS))
+def test_tensor_path_starved_waits_give_up(bm, form):
     """With BIMAMBA_TEST_STARVE no tile copy is issued: every wait for a tile
-    gives up after ~0.1 ms, bit 0 of the device error word is set, the
-    kernel finishes, and the context still works afterwards."""
+    gives up after ~0.1 ms and bit 0 of the device error word is set; in the
+    ticket-ordered form no forward sets its flag either, so every reverse
+    CTA's wait for it gives up too and sets bit 1.  The kernel finishes, and
+    the context still works afterwards."""
     inp, par = W.make_mamba2_case(1, 130, 2, P, N, "bf16", seed=73)
     assert bm.bimamba_device_error(reset=True) >= 0
-    run(bm, inp, par, torch.float32, flags=bm.BIMAMBA_TEST_STARVE)
-    assert bm.bimamba_device_error(reset=True) & 1
-    got = run(bm, inp, par, torch.float32)
+    run(bm, inp, par, torch.float32, flags=bm.BIMAMBA_TEST_STARVE | FORMS[form])
+    word = bm.bimamba_device_error(reset=True)
+    assert word & 1
+    assert bool(word & 2) == (form == "tickets")
+    got = run(bm, inp, par, torch.float32, flags=FORMS[form])
     assert U.normwise(got, oracle.mamba2_layer_fwd(inp, par)) <= U.TOL_BF16
     assert bm.bimamba_device_error(reset=True) == 0
 
