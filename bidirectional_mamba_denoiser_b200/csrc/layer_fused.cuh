@@ -264,7 +264,7 @@ __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int G, typename Tin, typename Tout, int DIR, bool CARRY, bool F32BC>
+template <int G, typename Tin, typename Tout, int DIR, bool CARRY, bool F32BC, int UNR = 4>
 __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, const KParams& p, unsigned char* base,
                                                       int lane) {
     using Ge = FusedGeo<G, Tin, F32BC>;
@@ -351,7 +351,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         float* wsw = p.ws + chunk_row * D + wp.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wp.d;
         typename Wp::Elem nxt = wp.element(0, 0 >= s_lo && 0 < s_hi, xt, dtt);
-#pragma unroll 2
+#pragma unroll (UNR)
         for (int s = 0; s < T; ++s) {
             const bool valid = s >= s_lo && s < s_hi;
             const typename Wp::Elem cur = nxt;
@@ -392,7 +392,9 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     if (CARRY && p.delta_sum[DIR] && wp.dvalid) p.delta_sum[DIR][(int64_t)b * D + wp.d] = dsum;
 }
 
-template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false>
+// The token loop unrolled by 4 (measured 1.116 against 1.154 ms for 2, 1.25
+// for 8 and 1.41 for all 16 at batch 8, L 2048, d_inner 4096).
+template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false, int UNR = 4>
 __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constant__ FusedMaps maps, const KParams p) {
     using Ge = FusedGeo<G, Tin, F32BC>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
@@ -406,9 +408,9 @@ __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constan
     }
     __syncthreads();
     if (warp == 0)
-        fused_layer_direction<G, Tin, Tout, 0, CARRY, F32BC>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 0, CARRY, F32BC, UNR>(maps, p, base, lane);
     else
-        fused_layer_direction<G, Tin, Tout, 1, CARRY, F32BC>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 1, CARRY, F32BC, UNR>(maps, p, base, lane);
 }
 
 // Forward scan over P = p.L tokens from zero: final state and conv tail.
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(32, 16) fused_prefix_kernel(const __grid_const
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         wp.window(xt);
         auto nxt = wp.element(0, 0 < nvalid, xt, dtt);
-#pragma unroll 2
+#pragma unroll 4
         for (int s = 0; s < T; ++s) {
             const auto cur = nxt;
             if (s + 1 < T) nxt = wp.element(s + 1, s + 1 < nvalid, xt, dtt);
