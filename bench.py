@@ -430,8 +430,8 @@ def l_sweep(args, bm, rank, world, dev, stream, flags, lengths=(4096, 16384, 655
 def run_chunked(args, w, bm, rank, world, dev, stream):
     """long --segments k: the batch-1 layer scanned as k segments side by side
     (sharded.ChunkedLayer: a pass from zero, the carry composition, a second
-    pass), for comparison with the single-pass kernels.  The extended
-    segments are built before the timed region."""
+    pass), for comparison with the single-pass kernels.  The segment views
+    and their conv halos are set up before the timed region."""
     from bidirectional_mamba_denoiser_b200 import sharded as SH
     ops = SH.CudaOps(flags_of(args, bm))
     plans = []
@@ -817,7 +817,7 @@ def run_sharded(args, w, bm, rank, world, dev, stream):
     ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
     ms_max = max_over_ranks(ms, world)
     step_ms = ms / args.steps
-    elems = w.batch * (Ls + 2 * SH.HALO) * w.d_inner
+    elems = w.batch * Ls * w.d_inner
     res = {
         "value": whole_job_rate(w.batch * Ls * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps, "gpu_launches": 3 * args.steps, "scaling": "strong",
@@ -837,10 +837,11 @@ def run_sharded(args, w, bm, rank, world, dev, stream):
             edges = torch.stack([SH.halo_edges(one)] * R)
             mid = R // 2  # a middle segment: both halos and both carries are real
 
+            halo = SH.neighbour_halos(edges, mid)
+
             def share(i):
-                ext = SH.extend_segment(one, *SH.neighbour_halos(edges, mid))
-                SH.pass_from_zero(ext, p1, ops)
-                SH.pass_with_carries(ext, p1, h_all, ds_all, mid, ops)
+                SH.pass_from_zero(one, halo, p1, ops)
+                SH.pass_with_carries(one, halo, p1, h_all, ds_all, mid, ops)
 
             k = max(3, args.steps // 4)
             ms_r, _ = timed(share, k, 2, 1, dev, stream)

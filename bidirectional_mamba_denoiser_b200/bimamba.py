@@ -61,7 +61,8 @@ class FwdState(ctypes.Structure):
 
 
 class Carry(ctypes.Structure):
-    _fields_ = [("h_in", ctypes.c_void_p * 2), ("h_out", ctypes.c_void_p * 2), ("delta_sum", ctypes.c_void_p * 2)]
+    _fields_ = [("h_in", ctypes.c_void_p * 2), ("h_out", ctypes.c_void_p * 2), ("delta_sum", ctypes.c_void_p * 2),
+                ("conv_halo", ctypes.c_void_p * 2)]
 
 
 class Params2(ctypes.Structure):
@@ -245,11 +246,13 @@ def _dir_pair(t):
 
 
 def bimamba_layer_fwd_carry(x, z, dt, B, C, params: dict, h_in=None, h_out=None, delta_sum=None, out=None,
-                            out_dtype=None, flags: int = 0, workspace=None, stream=None):
+                            out_dtype=None, flags: int = 0, workspace=None, stream=None, conv_halo=None):
     """bimamba_layer_fwd with scan carries.  h_in, h_out: [2, b, D, 16] fp32
     (or (fwd, rev) pairs, entries may be None): the states entering / leaving
     each direction; delta_sum: [2, b, D] fp32, each direction's sum of step
-    sizes.  Returns out [b, L, D]."""
+    sizes; conv_halo: [2, b, 3, D] of x's dtype (or a (before, after) pair):
+    the x rows of the three tokens before token 0 and after token L-1 that the
+    convs read instead of zeros.  Returns out [b, L, D]."""
     b, L, D = x.shape
     N = (B[0] if isinstance(B, (tuple, list)) else B).shape[-1]
     if out is None:
@@ -263,6 +266,7 @@ def bimamba_layer_fwd_carry(x, z, dt, B, C, params: dict, h_in=None, h_out=None,
     car.h_in[0], car.h_in[1] = _dir_pair(h_in)
     car.h_out[0], car.h_out[1] = _dir_pair(h_out)
     car.delta_sum[0], car.delta_sum[1] = _dir_pair(delta_sum)
+    car.conv_halo[0], car.conv_halo[1] = _dir_pair(conv_halo)
     rc = lib.bimamba_layer_fwd_carry(ctypes.byref(inp), ctypes.byref(par), ctypes.byref(car), _ptr(out),
                                      _dtype_code(out.dtype), b, L, D, N, flags, _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))

@@ -616,12 +616,14 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     bool with_carry = false;
     if (carry) {
         for (int r = 0; r < 2; ++r) {
-            if (!aligned(carry->h_in[r], 4) || !aligned(carry->h_out[r], 4) || !aligned(carry->delta_sum[r], 4))
+            if (!aligned(carry->h_in[r], 4) || !aligned(carry->h_out[r], 4) || !aligned(carry->delta_sum[r], 4) ||
+                !aligned(carry->conv_halo[r], elem_size(in->dtype)))
                 return BIMAMBA_ERR_MISALIGNED;
             k.carry_in[r] = carry->h_in[r];
             k.carry_out[r] = carry->h_out[r];
             k.delta_sum[r] = carry->delta_sum[r];
-            with_carry = with_carry || carry->h_in[r] || carry->h_out[r] || carry->delta_sum[r];
+            k.conv_halo[r] = carry->conv_halo[r];
+            with_carry = with_carry || carry->h_in[r] || carry->h_out[r] || carry->delta_sum[r] || carry->conv_halo[r];
         }
     }
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);

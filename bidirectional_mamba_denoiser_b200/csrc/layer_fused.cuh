@@ -338,6 +338,10 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         const Tin* zt = reinterpret_cast<const Tin*>(sb + Ge::XB + Ge::DTB);
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
+        if (CARRY && i == 0 && p.conv_halo[DIR])  // forward: tile rows 0..2 = tokens -3..-1; reverse: rows of L..L+2
+            put_conv_halo(reinterpret_cast<Tin*>(wbase + st * Ge::STAGE), Ge::CW,
+                          DIR == 0 ? 0 : (int)(L - (int64_t)k * T), 0, ct0, Ge::CW,
+                          static_cast<const Tin*>(p.conv_halo[DIR]) + (int64_t)b * 3 * D, D, lane);
         if (gated) {
             cp_async_wait_all();
             __syncwarp();

@@ -198,6 +198,10 @@ __device__ __forceinline__ void pscan_direction(const LayerMaps& maps, const KPa
         const Tin* zt = reinterpret_cast<const Tin*>(sb + Ge::XB + Ge::DTB);
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
+        if (CARRY && i == 0 && p.conv_halo[DIR])  // forward: tile rows 0..2 = tokens -3..-1; reverse: rows of L..L+2
+            put_conv_halo(reinterpret_cast<Tin*>(dir_base + st * Ge::STAGE), Ge::XW,
+                          DIR == 0 ? 0 : (int)(L - (int64_t)k * T), ct0 % Ge::XW + wg * Ge::CPW, c0w, Ge::CPW,
+                          static_cast<const Tin*>(p.conv_halo[DIR]) + (int64_t)b * 3 * D, D, lane);
 
         // 1. B and C as fp32 pairs in step order (the previous chunk's are
         // no longer read: every warp of the direction is past its scan)

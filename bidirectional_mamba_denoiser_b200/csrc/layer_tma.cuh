@@ -359,6 +359,10 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         const Tin* zt = reinterpret_cast<const Tin*>(sb + Ge::XB + Ge::DTB);
         const Tin* Bt = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB);
         const Tin* Ct = reinterpret_cast<const Tin*>(sb + Ge::XB + 2 * Ge::DTB + Ge::BB);
+        if (CARRY && i == 0 && p.conv_halo[DIR])  // forward: tile rows 0..2 = tokens -3..-1; reverse: rows of L..L+2
+            put_conv_halo(reinterpret_cast<Tin*>(dir_base + st * Ge::STAGE), Ge::XW,
+                          DIR == 0 ? 0 : (int)(L - (int64_t)k * T), ct0 % Ge::XW + wg * Ge::CPW, c0w, Ge::CPW,
+                          static_cast<const Tin*>(p.conv_halo[DIR]) + (int64_t)b * 3 * D, D, lane);
         float* bc = bc32 + (i & 1) * (T * kNState * 2);
         if constexpr (!DIRECT) convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
         // every warp of the direction is past the previous chunk (and, unless

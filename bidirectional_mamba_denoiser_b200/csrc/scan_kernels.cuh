@@ -135,6 +135,9 @@ struct KParams {
     const float* carry_in[2];  // [batch][D][16]: state entering the direction's first step (else 0)
     float* carry_out[2];       // [batch][D][16]: state after the direction's last step
     float* delta_sum[2];       // [batch][D]: sum of the step sizes over the sequence
+    // [batch][3][D] of the input type, rows in token order: the x the conv reads
+    // outside [0, L) (forward: tokens -3..-1; reverse: tokens L..L+2), else zeros
+    const void* conv_halo[2];
     int64_t L;             // sequence (or block) length
     int64_t M;             // meeting point of the two directions (layer)
     int D;

@@ -67,6 +67,23 @@ __device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// A segment's conv halo written over the zeros that a TMA x tile holds
+// outside the sequence: rows r0 .. r0+2 of the tile (row stride xw
+// elements), columns col0 + [0, nch) = channels d0 + [0, nch), from halo_b
+// ([3][D], rows in token order).  One warp; the proxy fence orders these
+// generic-proxy writes before a later TMA refill of the same stage, and the
+// warp sync before the warp's own reads of the tile.
+template <typename T>
+__device__ __forceinline__ void put_conv_halo(T* tile, int xw, int r0, int col0, int d0, int nch, const T* halo_b,
+                                              int D, int lane) {
+    for (int e = lane; e < 3 * nch; e += 32) {
+        const int q = e / nch, c = e % nch;
+        if (d0 + c < D) tile[(r0 + q) * xw + col0 + c] = halo_b[(int64_t)q * D + d0 + c];
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+}
+
 // 3-D tiled TMA load into shared memory, completing on `bar` (transaction
 // bytes).  Coordinates are element indices, innermost first; a box that
 // reaches outside the tensor reads zeros there.

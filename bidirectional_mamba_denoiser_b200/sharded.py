@@ -11,18 +11,17 @@ aggregates ([2, b, D, 16] states and [2, b, D] step-size sums), and each
 composes the states entering its own segment and scans again from them.
 The causal and anti-causal convs also reach three tokens into the
 neighbouring segments, so the ranks first exchange their first and last
-three x rows (the halos).
+three x rows (the halos), which the layer kernels read in place of the zeros
+outside the segment: the segment itself is passed as it is.
 
 Per rank, in order (all arithmetic in the CUDA library):
-  1. ``halo_edges``: the segment's first and last 3 x rows; all-gathered.
-  2. ``extend_segment``: the segment with its halo tokens on both sides; the
-     halo tokens get dt = -inf, i.e. step size exactly 0, so they only feed
-     the conv and leave the state unchanged.
-  3. ``pass_from_zero``: ``bimamba_layer_fwd_carry`` from zero states, for
+  1. ``halo_edges``: the segment's first and last 3 x rows; all-gathered;
+     ``neighbour_halos`` picks the rows before and after this segment.
+  2. ``pass_from_zero``: ``bimamba_layer_fwd_carry`` from zero states, for
      h_out and delta_sum (its output is not used); all-gathered.
-  4. ``pass_with_carries``: ``bimamba_compose_carries`` for this segment's
-     entering states, then ``bimamba_layer_fwd_carry`` from them; the
-     segment's rows of that output are the result.
+  3. ``pass_with_carries``: ``bimamba_compose_carries`` for this segment's
+     entering states, then ``bimamba_layer_fwd_carry`` from them: the
+     segment's layer output.
 
 The collectives are three small all-gathers (the halo rows, the final
 states, the step-size sums: a few hundred KB in all), the exchange step of a
@@ -51,10 +50,10 @@ class CudaOps:
         self.bm = bm
         self.flags = flags
 
-    def layer_carry(self, ext: dict, params: dict, h_in=None, h_out=None, delta_sum=None, out=None):
-        return self.bm.bimamba_layer_fwd_carry(ext["x"], ext["z"], ext["dt"], ext["B"], ext["C"], params,
+    def layer_carry(self, seg: dict, params: dict, halo, h_in=None, h_out=None, delta_sum=None, out=None):
+        return self.bm.bimamba_layer_fwd_carry(seg["x"], seg["z"], seg["dt"], seg["B"], seg["C"], params,
                                               h_in=h_in, h_out=h_out, delta_sum=delta_sum, out=out,
-                                              flags=self.flags)
+                                              flags=self.flags, conv_halo=halo)
 
     def compose(self, h_all, ds_all, params: dict, seg: int):
         return self.bm.bimamba_compose_carries(h_all, ds_all, params, seg)
@@ -71,55 +70,33 @@ def halo_edges(seg: dict) -> torch.Tensor:
 def neighbour_halos(all_edges: torch.Tensor, rank: int):
     """From the gathered edges [R, 2, b, 3, D]: the x rows just before the
     segment (rank - 1's last three; zeros at the sequence start) and just
-    after it (rank + 1's first three; zeros at the end)."""
+    after it (rank + 1's first three; zeros at the end), as the conv halos
+    (before, after) of the segment's layer calls, [b, 3, D] each."""
     R = all_edges.shape[0]
     zeros = torch.zeros_like(all_edges[0, 0])
     left = all_edges[rank - 1, 1] if rank > 0 else zeros
     right = all_edges[rank + 1, 0] if rank < R - 1 else zeros
-    return left, right
+    return left.contiguous(), right.contiguous()
 
 
-def extend_segment(seg: dict, left: torch.Tensor, right: torch.Tensor) -> dict:
-    """The segment's inputs with HALO tokens on each side: x from the
-    neighbours, dt = -inf (step size 0: the state passes unchanged), z, B, C
-    zero.  x, z [b, Ls, D]; dt [2, b, Ls, D]; B, C [2, b, Ls, 16]."""
-    def pad(t, dim, value=0.0):
-        shape = list(t.shape)
-        shape[dim] = HALO
-        p = torch.full(shape, value, device=t.device, dtype=t.dtype)
-        return torch.cat([p, t, p], dim=dim).contiguous()
-    return {
-        "x": torch.cat([left.to(seg["x"].dtype), seg["x"], right.to(seg["x"].dtype)], dim=1).contiguous(),
-        "z": pad(seg["z"], 1),
-        "dt": pad(seg["dt"], 2, float("-inf")),
-        "B": pad(seg["B"], 2),
-        "C": pad(seg["C"], 2),
-    }
-
-
-def pass_from_zero(ext: dict, params: dict, ops) -> tuple[torch.Tensor, torch.Tensor]:
-    """The extended segment scanned from zero states: (h_out [2, b, D, 16],
+def pass_from_zero(seg: dict, halo, params: dict, ops) -> tuple[torch.Tensor, torch.Tensor]:
+    """The segment scanned from zero states: (h_out [2, b, D, 16],
     delta_sum [2, b, D]) of ops.state_dtype."""
-    b, _, D = ext["x"].shape
-    N = ext["B"].shape[-1]
-    dev = ext["x"].device
+    b, _, D = seg["x"].shape
+    N = seg["B"].shape[-1]
+    dev = seg["x"].device
     h_out = torch.empty(2, b, D, N, device=dev, dtype=ops.state_dtype)
     ds = torch.empty(2, b, D, device=dev, dtype=ops.state_dtype)
-    ops.layer_carry(ext, params, h_out=h_out, delta_sum=ds)
+    ops.layer_carry(seg, params, halo, h_out=h_out, delta_sum=ds)
     return h_out, ds
 
 
-def pass_with_carries(ext: dict, params: dict, h_all: torch.Tensor, ds_all: torch.Tensor, rank: int, ops,
+def pass_with_carries(seg: dict, halo, params: dict, h_all: torch.Tensor, ds_all: torch.Tensor, rank: int, ops,
                       out=None) -> torch.Tensor:
-    """The extended segment scanned from the states the other segments hand
-    it; returns the segment's own rows of the layer output."""
+    """The segment scanned from the states the other segments hand it: its
+    layer output [b, Ls, D] (written to out if given)."""
     h_in = ops.compose(h_all, ds_all, params, rank)
-    y = ops.layer_carry(ext, params, h_in=h_in)
-    seg = y[:, HALO:y.shape[1] - HALO]
-    if out is not None:
-        out.copy_(seg)
-        return out
-    return seg
+    return ops.layer_carry(seg, params, halo, h_in=h_in, out=out)
 
 
 def _all_gather(t: torch.Tensor, group=None) -> torch.Tensor:
@@ -136,10 +113,9 @@ def sharded_layer_fwd(seg: dict, params: dict, group=None, ops=None, out=None) -
     import torch.distributed as dist
     ops = ops or CudaOps()
     rank = dist.get_rank(group)
-    left, right = neighbour_halos(_all_gather(halo_edges(seg), group), rank)
-    ext = extend_segment(seg, left, right)
-    h_out, ds = pass_from_zero(ext, params, ops)
-    return pass_with_carries(ext, params, _all_gather(h_out, group), _all_gather(ds, group), rank, ops, out=out)
+    halo = neighbour_halos(_all_gather(halo_edges(seg), group), rank)
+    h_out, ds = pass_from_zero(seg, halo, params, ops)
+    return pass_with_carries(seg, halo, params, _all_gather(h_out, group), _all_gather(ds, group), rank, ops, out=out)
 
 
 def split_sequence(inputs: dict, lengths: Sequence[int]) -> list[dict]:
@@ -158,13 +134,14 @@ def emulate_sharded(inputs: dict, params: dict, lengths: Sequence[int], ops=None
     """The sharded computation for all segments in this process (stacking in
     place of the all-gathers); returns the full output [b, L, D]."""
     ops = ops or CudaOps()
-    segs = split_sequence(inputs, lengths)
+    segs = [{k: v.contiguous() for k, v in s.items()} for s in split_sequence(inputs, lengths)]
     all_edges = torch.stack([halo_edges(s) for s in segs])
-    exts = [extend_segment(s, *neighbour_halos(all_edges, r)) for r, s in enumerate(segs)]
-    aggs = [pass_from_zero(e, params, ops) for e in exts]
+    halos = [neighbour_halos(all_edges, r) for r in range(len(segs))]
+    aggs = [pass_from_zero(s, halos[r], params, ops) for r, s in enumerate(segs)]
     h_all = torch.stack([a[0] for a in aggs])
     ds_all = torch.stack([a[1] for a in aggs])
-    return torch.cat([pass_with_carries(e, params, h_all, ds_all, r, ops) for r, e in enumerate(exts)], dim=1)
+    return torch.cat([pass_with_carries(s, halos[r], params, h_all, ds_all, r, ops) for r, s in enumerate(segs)],
+                     dim=1)
 
 
 class ChunkedLayer:
@@ -172,14 +149,15 @@ class ChunkedLayer:
     segments that one GPU scans side by side, as the rows of a batch: the
     chunked form of the scan, with carries, inside one device.
 
-    ``__init__`` builds the extended segments once (each with its 3-token
-    halos, stacked into [nseg, Ls + 6, D] inputs); ``run`` is then the scan
-    itself: one layer pass from zero states for every segment's final states
-    and step-size sums, the composition of the carries entering each segment
-    (nseg small launches), and a second layer pass from them.  It exists to
-    measure this schedule against the single-pass kernels, which walk the
-    whole sequence in one chain per (channel, direction) and so need no
-    second pass."""
+    The segments are views of the inputs ([1, L, ...] read as [nseg, L/nseg,
+    ...]: no copy); ``__init__`` gathers each segment's conv halos (3 x rows
+    on each side) once.  ``run`` is then the scan itself: one layer pass from
+    zero states for every segment's final states and step-size sums, the
+    composition of the carries entering each segment (nseg small launches),
+    and a second layer pass from them, whose output rows are the layer's.  It
+    exists to measure this schedule against the single-pass kernels, which
+    walk the whole sequence in one chain per (channel, direction) and so need
+    no second pass."""
 
     def __init__(self, inputs: dict, params: dict, nseg: int, ops=None):
         x = inputs["x"]
@@ -191,32 +169,35 @@ class ChunkedLayer:
         self.ops = ops or CudaOps()
         self.params = params
         self.nseg, self.Ls = nseg, L // nseg
-        segs = split_sequence(inputs, [self.Ls] * nseg)
-        all_edges = torch.stack([halo_edges(s) for s in segs])
-        exts = [extend_segment(s, *neighbour_halos(all_edges, r)) for r, s in enumerate(segs)]
-        self.ext = {"x": torch.cat([e["x"] for e in exts], 0).contiguous(),
-                    "z": torch.cat([e["z"] for e in exts], 0).contiguous(),
-                    "dt": torch.cat([e["dt"] for e in exts], 1).contiguous(),
-                    "B": torch.cat([e["B"] for e in exts], 1).contiguous(),
-                    "C": torch.cat([e["C"] for e in exts], 1).contiguous()}
+        Ls = self.Ls
         D, N = x.shape[2], inputs["B"].shape[-1]
+        self.seg = {"x": x.contiguous().view(nseg, Ls, D), "z": inputs["z"].contiguous().view(nseg, Ls, D),
+                    "dt": inputs["dt"].contiguous().view(2, nseg, Ls, D),
+                    "B": inputs["B"].contiguous().view(2, nseg, Ls, N),
+                    "C": inputs["C"].contiguous().view(2, nseg, Ls, N)}
+        xs = self.seg["x"]
+        before = torch.zeros(nseg, HALO, D, device=x.device, dtype=x.dtype)
+        after = torch.zeros_like(before)
+        before[1:] = xs[:-1, Ls - HALO:]
+        after[:-1] = xs[1:, :HALO]
+        self.halo = (before, after)
         dev = x.device
         self.h_out = torch.empty(2, nseg, D, N, device=dev, dtype=self.ops.state_dtype)
         self.ds = torch.empty(2, nseg, D, device=dev, dtype=self.ops.state_dtype)
         self.h_all = torch.empty(nseg, 2, 1, D, N, device=dev, dtype=self.ops.state_dtype)
         self.ds_all = torch.empty(nseg, 2, 1, D, device=dev, dtype=self.ops.state_dtype)
         self.h_in = torch.empty(2, nseg, D, N, device=dev, dtype=self.ops.state_dtype)
-        self.y = torch.empty(nseg, self.Ls + 2 * HALO, D, device=dev, dtype=x.dtype)
+        self.y = torch.empty(nseg, Ls, D, device=dev, dtype=x.dtype)
 
     def run(self) -> torch.Tensor:
-        """[nseg, Ls + 6, D]: each segment's extended rows of the layer output."""
-        self.ops.layer_carry(self.ext, self.params, h_out=self.h_out, delta_sum=self.ds)
+        """[nseg, Ls, D]: each segment's rows of the layer output."""
+        self.ops.layer_carry(self.seg, self.params, self.halo, h_out=self.h_out, delta_sum=self.ds)
         self.h_all.copy_(self.h_out.permute(1, 0, 2, 3).unsqueeze(2))
         self.ds_all.copy_(self.ds.permute(1, 0, 2).unsqueeze(2))
         for s in range(self.nseg):
             self.h_in[:, s] = self.ops.compose(self.h_all, self.ds_all, self.params, s)[:, 0]
-        return self.ops.layer_carry(self.ext, self.params, h_in=self.h_in, out=self.y)
+        return self.ops.layer_carry(self.seg, self.params, self.halo, h_in=self.h_in, out=self.y)
 
     def output(self, y: torch.Tensor) -> torch.Tensor:
-        """The layer output [1, L, D] from run()'s result."""
-        return y[:, HALO:HALO + self.Ls].reshape(1, self.nseg * self.Ls, y.shape[-1])
+        """The layer output [1, L, D] from run()'s result (a view)."""
+        return y.view(1, self.nseg * self.Ls, y.shape[-1])

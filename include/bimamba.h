@@ -157,21 +157,25 @@ int bimamba_layer_fwd(const bimamba_inputs_t *in, const bimamba_params_t *p,
  *   h_out      [batch][d_inner][d_state]: the state after the direction's last
  *              step (forward: after token L-1; reverse: after token 0)
  *   delta_sum  [batch][d_inner]: sum over the L tokens of the direction's step
- *              size softplus(dt + dt_bias) */
+ *              size softplus(dt + dt_bias)
+ *   conv_halo  [batch][3][d_inner] of the input dtype, rows in token order,
+ *              aligned to its element: the x the direction's conv reads outside
+ *              [0, L) (forward: the three tokens before token 0; reverse: the
+ *              three after token L-1), instead of zeros */
 typedef struct {
     const float *h_in[2];
     float *h_out[2];
     float *delta_sum[2];
+    const void *conv_halo[2];
 } bimamba_carry_t;
 
 /* bimamba_layer_fwd with carries: the recurrences of §3.2 Eq. (4)-(5) start
  * from carry->h_in and report their final states and step-size sums.  With
  * these a sequence cut into segments (one per GPU) is scanned exactly: run
  * each segment from zero for h_out and delta_sum, compose the carries with
- * bimamba_compose_carries, run again from them.  The conv still reads zeros
- * outside [0, L): a segment's inputs are extended by the three neighbouring
- * tokens on each side with dt = -inf there (step size exactly 0, so those
- * tokens leave the state unchanged and only feed the conv).  h_in may alias
+ * bimamba_compose_carries, run again from them.  The conv reads the
+ * neighbouring segments' x rows from conv_halo (zeros where it is NULL), so
+ * a segment is passed as it is, with no copy.  h_in may alias
  * h_out only if both are the same direction's (each state word is read
  * before it is written, by the same thread).  Runs the TMA-fed kernel
  * families only: inputs that bimamba_layer_fwd would run on its fallback

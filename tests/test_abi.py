@@ -342,6 +342,10 @@ def test_layer_carry_rejects():
     assert _layer_carry(_carry(h_out=(FAKE + 0x40000, None)), flags=bm.BIMAMBA_NO_TMA) == bm.BIMAMBA_ERR_UNSUPPORTED
     for name in ("h_in", "h_out", "delta_sum"):
         assert _layer_carry(_carry(**{name: (None, FAKE + 0x40002)})) == bm.BIMAMBA_ERR_MISALIGNED
+    # conv halos: aligned to the input element (bf16 here); a halo alone runs with carries
+    assert _layer_carry(_carry(conv_halo=(FAKE + 0x40001, None))) == bm.BIMAMBA_ERR_MISALIGNED
+    assert _layer_carry(_carry(conv_halo=(None, FAKE + 0x40000)), flags=bm.BIMAMBA_NO_TMA) == \
+        bm.BIMAMBA_ERR_UNSUPPORTED
     assert _layer_carry(_carry(h_out=(FAKE + 0x40000, None)), batch=0) == bm.BIMAMBA_ERR_INVALID_ARG
 
 

@@ -1,8 +1,7 @@
 """Host logic of the sequence-sharded layer (bidirectional_mamba_denoiser_b200/
-sharded.py), on CPU: halo selection, segment extension, and the whole
-exchange (all-gathers over real gloo groups of 2 and 3 ranks) with a plain
-fp64 numpy stand-in for the CUDA compute steps, against the oracle's
-full-sequence layer."""
+sharded.py), on CPU: halo selection and the whole exchange (all-gathers over
+real gloo groups of 2 and 3 ranks) with a plain fp64 numpy stand-in for the
+CUDA compute steps, against the oracle's full-sequence layer."""
 import os
 import socket
 
@@ -20,18 +19,21 @@ from bidirectional_mamba_denoiser_b200 import workloads as W
 class NumpyOps:
     """The two compute steps in plain fp64 numpy: the layer with carries
     (the recurrences of §3.2 Eq. (4)-(6) started from h_in, reporting the
-    final states and the step-size sums) and the carry composition."""
+    final states and the step-size sums; the convs reading the halo rows
+    outside the segment) and the carry composition."""
 
     state_dtype = torch.float64
 
-    def layer_carry(self, ext, params, h_in=None, h_out=None, delta_sum=None, out=None):
-        x = ext["x"].double().numpy()
-        z = ext["z"].double().numpy()
-        dt, B, C = (ext[k].double().numpy() for k in ("dt", "B", "C"))
+    def layer_carry(self, seg, params, halo, h_in=None, h_out=None, delta_sum=None, out=None):
+        x = seg["x"].double().numpy()
+        z = seg["z"].double().numpy()
+        dt, B, C = (seg[k].double().numpy() for k in ("dt", "B", "C"))
         A, Dk, bias, w, cb = (params[k].double().numpy() for k in ("A", "D", "dt_bias", "conv_w", "conv_b"))
         b, L, D = x.shape
         N = B.shape[-1]
-        xp = np.concatenate([np.zeros((b, 3, D)), x, np.zeros((b, 3, D))], axis=1)
+        left, right = ((np.zeros((b, 3, D)), np.zeros((b, 3, D))) if halo is None
+                       else (halo[0].double().numpy(), halo[1].double().numpy()))
+        xp = np.concatenate([left, x, right], axis=1)
         y = np.zeros((2, b, L, D))
         for r in range(2):
             # forward: tap k on x[t-3+k]; reverse: tap k on x[t+3-k] (xp is x shifted by 3)
@@ -83,11 +85,7 @@ def test_neighbour_halos_and_extension():
     left0, _ = SH.neighbour_halos(edges, 0)
     _, right2 = SH.neighbour_halos(edges, 2)
     assert not left0.any() and not right2.any()
-    ext = SH.extend_segment(segs[1], left, right)
-    assert torch.equal(ext["x"], inp["x"][:, 3:18])
-    assert torch.isneginf(ext["dt"][:, :, :3]).all() and torch.isneginf(ext["dt"][:, :, -3:]).all()
-    assert torch.equal(ext["dt"][:, :, 3:-3], segs[1]["dt"])
-    assert not ext["B"][:, :, :3].any() and not ext["z"][:, -3:].any()
+    assert left.is_contiguous() and right.is_contiguous()
     with pytest.raises(ValueError):
         SH.halo_edges({"x": inp["x"][:, :2]})
 
@@ -100,15 +98,31 @@ def test_emulated_segments_match_the_full_layer(lengths):
     assert np.abs(got.numpy() - want).max() <= 1e-10 * np.abs(want).max()
 
 
+@pytest.mark.parametrize("nseg", [2, 5])
+def test_chunked_layer_views_and_halos(nseg):
+    """ChunkedLayer: one sequence read as nseg batch rows (views, no copy),
+    each row's conv halos the neighbouring rows' edge tokens (zeros at the
+    ends); two passes and the composition give the full-sequence layer."""
+    inp, par = _case(40, b=1)
+    plan = SH.ChunkedLayer(inp, par, nseg, ops=NumpyOps())
+    assert plan.seg["x"].data_ptr() == inp["x"].data_ptr()
+    before, after = plan.halo
+    Ls = 40 // nseg
+    assert not before[0].any() and not after[-1].any()
+    assert torch.equal(before[1], inp["x"][0, Ls - 3:Ls]) and torch.equal(after[0], inp["x"][0, Ls:Ls + 3])
+    got = plan.output(plan.run())
+    want = oracle.layer_fwd(inp, par)
+    assert np.abs(got.numpy() - want).max() <= 1e-10 * np.abs(want).max()
+
+
 def test_composed_carries_are_the_prefix_and_suffix_states():
     # the forward carry entering a segment is the state of the scan over everything before it
     inp, par = _case(30)
     lengths = [12, 18]
     segs = SH.split_sequence(inp, lengths)
     edges = torch.stack([SH.halo_edges(s) for s in segs])
-    exts = [SH.extend_segment(s, *SH.neighbour_halos(edges, r)) for r, s in enumerate(segs)]
     ops = NumpyOps()
-    aggs = [SH.pass_from_zero(e, par, ops) for e in exts]
+    aggs = [SH.pass_from_zero(s, SH.neighbour_halos(edges, r), par, ops) for r, s in enumerate(segs)]
     h_in = ops.compose(torch.stack([a[0] for a in aggs]), torch.stack([a[1] for a in aggs]), par, 1)
     head = {k: (v[:, :12] if k in ("x", "z") else v[:, :, :12]) for k, v in inp.items()}
     h_prefix, _ = oracle.prefix_state(head, par)
