@@ -435,11 +435,13 @@ int pick_family(int64_t lanes_total, unsigned flags) {
     return lanes_total >= 148LL * 8 * 32 ? 2 : 1;
 }
 
-// Group size of the fused kernel: 2 lanes x 8 states measured fastest at
-// batch 8, L 2048, d_inner 4096 (1.11 ms against 1.14 ms at 4 lanes).
+// Group size of the fused kernel: one lane per channel with all 16 states
+// measured fastest at batch 8, L 2048, d_inner 4096 with the token loop
+// unrolled by 4 (1.096 ms against 1.122 ms for 2 lanes x 8 states, 1.175 at
+// 4 and 1.276 at 8).
 int pick_group_fused(unsigned flags) {
     const unsigned f = (flags & BIMAMBA_LANES_MASK) >> BIMAMBA_LANES_SHIFT;
-    return f ? (int)f : 2;
+    return f ? (int)f : 1;
 }
 
 // Chunk length of the chunked kernel: forced by the flags, else 16 tokens
@@ -646,17 +648,18 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     const bool group_ok = forced == 0 || forced == 1 || forced == 2 || forced == 4 || forced == 8;
     if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
         tma_eligible(in, d_inner, true, true)) {
-        if (with_carry) {  // carries: the 2-lane groups (the group size changes only the speed)
-            if (in_bf && out_bf) return launch_fused_layer<2, bf16, bf16, true>(k, in, st);
-            if (in_bf) return launch_fused_layer<2, bf16, float, true>(k, in, st);
-            if (out_bf) return launch_fused_layer<2, float, bf16, true>(k, in, st);
-            return launch_fused_layer<2, float, float, true>(k, in, st);
+        if (with_carry) {  // carries: one lane per channel (the group size changes only the speed)
+            if (in_bf && out_bf) return launch_fused_layer<1, bf16, bf16, true>(k, in, st);
+            if (in_bf) return launch_fused_layer<1, bf16, float, true>(k, in, st);
+            if (out_bf) return launch_fused_layer<1, float, bf16, true>(k, in, st);
+            return launch_fused_layer<1, float, float, true>(k, in, st);
         }
         const int gf = pick_group_fused(flags);
         // B/C widened to fp32 once per chunk at 2 lanes per group (measured
         // 1.164 against 1.176 ms at batch 8, L 2048); the chunk field's 1
-        // selects the per-use widening
-        const bool f32bc = gf == 2 ? chunk_field != 1 : chunk_field == 2;
+        // selects the per-use widening there, its 2 the widening at 4 lanes.
+        // One lane per channel always widens them once per chunk.
+        const bool f32bc = (gf == 2 && chunk_field != 1) || (gf == 4 && chunk_field == 2);
         if (in_bf && out_bf) return fused_layer_by_group<bf16, bf16>(gf, f32bc, k, in, st);
         if (in_bf) return fused_layer_by_group<bf16, float>(gf, f32bc, k, in, st);
         if (out_bf) return fused_layer_by_group<float, bf16>(gf, f32bc, k, in, st);

@@ -80,9 +80,10 @@ typedef enum { BIMAMBA_F32 = 0, BIMAMBA_BF16 = 1 } bimamba_dtype_t;
  * size).  1: chunked -- G lanes share one channel's states, for few channels
  * (batch 1, long sequences).  2: per-token fused -- one lane per channel,
  * groups of G lanes share B/C across G channels, for many channels.  With
- * family 2 the lane field (bits 8..12) is the group size (1, 2, 4 or 8); at 2
- * lanes B/C are widened to fp32 once per chunk unless the chunk field is 1,
- * at 4 only if it is 2.  3: chunked parallel scan -- per 64-token chunk a
+ * family 2 the lane field (bits 8..12) is the group size (1, 2, 4 or 8; 0 =
+ * 1: a lane per channel with all 16 states and B/C widened to fp32 once per
+ * chunk); at 2 lanes B/C are widened once per chunk unless the chunk field
+ * is 1, at 4 only if it is 2.  3: chunked parallel scan -- per 64-token chunk a
  * channel's 8 lanes scan 8-step pieces and combine their carries with warp
  * shuffles (the lane and chunk fields are not read).  Tuning knobs: the
  * result does not depend on the family beyond fp32 rounding order. */
@@ -181,8 +182,9 @@ typedef struct {
  * families only: inputs that bimamba_layer_fwd would run on its fallback
  * kernels (pointers not 16-byte aligned, d_inner % 8 != 0, or flags with
  * BIMAMBA_NO_TMA or a fallback lane count) return BIMAMBA_ERR_UNSUPPORTED; with
- * carries the per-token family runs 2-lane groups and the chunked family its
- * automatic chunk length, whatever the lane-group and chunk flags ask.
+ * carries the per-token family runs one lane per channel and the chunked
+ * family its automatic chunk length, whatever the lane-group and chunk flags
+ * ask.
  * carry == NULL returns BIMAMBA_ERR_INVALID_ARG.  Other arguments, checks
  * and errors: as bimamba_layer_fwd.  One kernel launch. */
 int bimamba_layer_fwd_carry(const bimamba_inputs_t *in, const bimamba_params_t *p, const bimamba_carry_t *carry,
