@@ -660,8 +660,10 @@ def mamba2_oracle_rate(w: W.Workload, inputs, params, budget_s: float):
 
 
 def run_mamba2(args, w, bm, rank, world, dev, stream):
-    """mamba2 / mamba2_long: steps of bimamba2_layer_fwd (three launches each)."""
+    """mamba2 / mamba2_long: steps of bimamba2_layer_fwd (two launches each on
+    the tensor-core path, three on the CUDA-core one)."""
     H, P, N = w.extra["nheads"], w.extra["headdim"], w.d_state
+    flags = flags_of(args, bm)
     sets = [W.make_mamba2_case(w.batch, w.L, H, P, N, w.dtype, w.seed + 1000 * i + rank, device=dev)
             for i in range(2)]
     out = torch.empty(w.batch, w.L, H * P, device=dev, dtype=W.torch_dtype(w.dtype))
@@ -669,14 +671,15 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
 
     def step(i):
         inp, par = sets[i % 2]
-        bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out=out, workspace=ws, stream=stream)
+        bm.bimamba2_layer_fwd(inp["xbc"], inp["z"], inp["dt"], par, out=out, workspace=ws, stream=stream,
+                              flags=flags)
 
     ms, clocks = timed(step, args.steps, args.warmup, world, dev, stream)
     ms_max = max_over_ranks(ms, world)
     call_ms = ms / args.steps
     tokens = w.batch * w.L
     flops = 4.0 * P * N * H * 2 * tokens  # the recurrence: two FMAs per state per token and direction
-    tensor_path = w.dtype == "bf16"
+    tensor_path = w.dtype == "bf16" and not (flags & bm.BIMAMBA_NO_TMA)
     res = {
         "value": whole_job_rate(tokens * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
@@ -704,7 +707,7 @@ def run_mamba2(args, w, bm, rank, world, dev, stream):
         k2 = max(3, min(args.steps, 20))
 
         def call(d, o, st):
-            bm.bimamba2_layer_fwd(d["xbc"], d["z"], d["dt"], par, out=o, workspace=ws, stream=st)
+            bm.bimamba2_layer_fwd(d["xbc"], d["z"], d["dt"], par, out=o, workspace=ws, stream=st, flags=flags)
 
         ms2 = e2e_pipelined(call, host, out.shape, out.dtype, k2, world, dev, stream)
         res["e2e"] = {"value": round(whole_job_rate(tokens * k2, world, ms2 / 1e3), 4),
