@@ -396,8 +396,9 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     if (CARRY && p.delta_sum[DIR] && wp.dvalid) p.delta_sum[DIR][(int64_t)b * D + wp.d] = dsum;
 }
 
-// The token loop unrolled by 4 (measured 1.116 against 1.154 ms for 2, 1.25
-// for 8 and 1.41 for all 16 at batch 8, L 2048, d_inner 4096).
+// The token loop unrolled by 4 (with 2-lane groups: 1.116 against 1.154 ms
+// for 2, 1.25 for 8 and 1.41 for all 16 at batch 8, L 2048, d_inner 4096;
+// with one lane per channel 1.096 against 1.137 for 2 and 1.20 for 8).
 template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false, int UNR = 4>
 __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constant__ FusedMaps maps, const KParams p) {
     using Ge = FusedGeo<G, Tin, F32BC>;
