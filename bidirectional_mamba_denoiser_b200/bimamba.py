@@ -335,8 +335,8 @@ def bimamba_out_proj(y, w_out, out=None, stream=None):
 def bimamba_layer_fwd_noalloc(x, z, dt, B, C, params: dict, out=None, out_dtype=None, flags: int = 0,
                               stream=None):
     """bimamba_layer_fwd for callers that cannot allocate device memory: the
-    library's built-in 64 MiB scratch replaces the workspace (batch * L *
-    d_inner <= 16,777,216).  Calls that overlap on the GPU race on that
+    library's built-in 64 MiB scratch replaces the workspace (sizes whose
+    bimamba_workspace_bytes fits in it).  Calls that overlap on the GPU race on that
     scratch.  ``out`` is still the caller's; pass it in to allocate nothing
     here either."""
     b, L, D = x.shape

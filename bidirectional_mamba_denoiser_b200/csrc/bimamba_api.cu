@@ -235,6 +235,16 @@ bool tma_eligible(const bimamba_inputs_t* in, int d_inner, bool need_reverse, bo
 constexpr int kTWD = 4;  // warps per direction per CTA
 constexpr int kTNS = 2;  // pipeline stages
 
+// The layer's workspace: the directions' fp32 partial outputs [batch][L][D],
+// then (256-byte aligned) the fp32 B/C quads [2][batch][L][32] of the
+// chunked kernel at 8 lanes per channel.
+size_t layer_ws_bcq_offset(int batch, int64_t L, int d_inner) {
+    return ((size_t)batch * (size_t)L * (size_t)d_inner * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+size_t layer_ws_bcq_bytes(int batch, int64_t L) {
+    return 2 * (size_t)batch * (size_t)L * 2 * bimamba::kNState * sizeof(float);
+}
+
 template <int G, int T, typename Tin, int NWD = kTWD>
 bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int64_t L, int D, bool reverse,
                bool gated) {
@@ -262,13 +272,27 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
+// BCQ: B and C widened to fp32 quads in the workspace first (one small
+// launch), then read by TMA in the layout the states use, with no widening in
+// the scan loop.
 template <int G, int T, typename Tin, typename Tout, bool CARRY = false, int NWD = kTWD, bool DIRECT = false,
-          bool FULL_UNROLL = false>
+          bool FULL_UNROLL = false, bool BCQ = false>
 int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin, DIRECT>;
+    using Ge = bimamba::TmaGeo<G, T, NWD, kTNS, Tin, DIRECT, BCQ>;
     bimamba::LayerMaps maps;
     if (!fill_maps<G, T, Tin, NWD>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT, FULL_UNROLL>;
+    if constexpr (BCQ) {
+        const int64_t rows = 2 * (int64_t)k.batch * k.L;
+        const int64_t blocks = (rows + 255) / 256;
+        bimamba::widen_bc_kernel<Tin><<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(k);
+        if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+        const size_t per_dir = (size_t)k.batch * (size_t)k.L * 2 * bimamba::kNState;
+        for (int r = 0; r < 2; ++r)
+            if (!map3d(&maps.B[r], k.bcq + r * per_dir, false, 2 * bimamba::kNState, (uint64_t)k.L,
+                       (uint64_t)k.batch, 2 * bimamba::kNState, T))
+                return BIMAMBA_ERR_CUDA;
+    }
+    auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT, FULL_UNROLL, BCQ>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -525,7 +549,7 @@ void fill_inputs(KParams& k, const bimamba_inputs_t* in) {
 
 extern "C" {
 
-int bimamba_abi_version(void) { return 1; }
+int bimamba_abi_version(void) { return 2; }
 
 const char* bimamba_status_string(int status) {
     switch (status) {
@@ -576,7 +600,7 @@ int bimamba_features(const bimamba_inputs_t* in, const bimamba_params_t* p, int 
 size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags) {
     (void)flags;
     if (batch <= 0 || batch > kMaxBatch || L <= 0 || d_inner <= 0 || d_state != bimamba::kNState) return 0;
-    return (size_t)batch * (size_t)L * (size_t)d_inner * sizeof(float);
+    return layer_ws_bcq_offset(batch, L, d_inner) + layer_ws_bcq_bytes(batch, L);
 }
 
 }  // extern "C"
@@ -608,6 +632,7 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     fill_params(k, p);
     k.out = out;
     k.ws = static_cast<float*>(workspace);
+    k.bcq = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + layer_ws_bcq_offset(batch, L, d_inner));
     k.L = L;
     k.M = L / 2;
     k.D = d_inner;
@@ -671,22 +696,23 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
         // with carries the chunk length is the automatic one (the flag is not honoured)
         const int tt = with_carry ? pick_chunk_tma(0, gt) : pick_chunk_tma(flags, gt);
         // 8 lanes per channel with 32-token chunks: one warp per direction per
-        // CTA and B/C read straight from the tile (measured 6.79 against
-        // 7.20 ms at batch 1, L 65536, d_inner 4096: 1024 CTAs spread over the
-        // SMs evenly).  BIMAMBA_CHUNKED_WIDE keeps the 4-warp CTAs with B/C
-        // widened once per chunk.
+        // CTA (measured 6.79 against 7.20 ms for 4-warp CTAs at batch 1,
+        // L 65536, d_inner 4096: 1024 CTAs spread over the SMs evenly), the
+        // group loop fully unrolled (6.24 against 6.77 ms), and B/C widened
+        // to fp32 quads once per call in the workspace instead of by every
+        // lane at each use.  BIMAMBA_CHUNKED_WIDE keeps the 4-warp CTAs with
+        // B/C widened once per chunk in shared memory.
         if (gt == 8 && tt == 32 && !(flags & BIMAMBA_CHUNKED_WIDE)) {
-            // the group loop fully unrolled: 6.24 against 6.77 ms at the same size
             if (with_carry) {
-                if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, true, true>(k, in, st);
-                if (in_bf) return launch_layer_tma<8, 32, bf16, float, true, 1, true, true>(k, in, st);
-                if (out_bf) return launch_layer_tma<8, 32, float, bf16, true, 1, true, true>(k, in, st);
-                return launch_layer_tma<8, 32, float, float, true, 1, true, true>(k, in, st);
+                if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, true, 1, false, true, true>(k, in, st);
+                if (in_bf) return launch_layer_tma<8, 32, bf16, float, true, 1, false, true, true>(k, in, st);
+                if (out_bf) return launch_layer_tma<8, 32, float, bf16, true, 1, false, true, true>(k, in, st);
+                return launch_layer_tma<8, 32, float, float, true, 1, false, true, true>(k, in, st);
             }
-            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, true, true>(k, in, st);
-            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, true, true>(k, in, st);
-            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, true, true>(k, in, st);
-            return launch_layer_tma<8, 32, float, float, false, 1, true, true>(k, in, st);
+            if (in_bf && out_bf) return launch_layer_tma<8, 32, bf16, bf16, false, 1, false, true, true>(k, in, st);
+            if (in_bf) return launch_layer_tma<8, 32, bf16, float, false, 1, false, true, true>(k, in, st);
+            if (out_bf) return launch_layer_tma<8, 32, float, bf16, false, 1, false, true, true>(k, in, st);
+            return launch_layer_tma<8, 32, float, float, false, 1, false, true, true>(k, in, st);
         }
         if (with_carry) {
             if (in_bf && out_bf) return layer_tma_carry_by_lanes<bf16, bf16>(gt, k, in, st);

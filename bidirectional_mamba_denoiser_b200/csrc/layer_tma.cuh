@@ -43,15 +43,17 @@ struct LayerMaps {
     CUtensorMap x;      // [batch][L][D]      box {CW, T+3, 1}
     CUtensorMap z;      // [batch][L][D]      box {CW, T, 1}
     CUtensorMap dt[2];  // [batch][L][D]      box {CW, T, 1}
-    CUtensorMap B[2];   // [batch][L][16]     box {16, T, 1}
-    CUtensorMap C[2];   // [batch][L][16]     box {16, T, 1}
+    CUtensorMap B[2];   // [batch][L][16]     box {16, T, 1}; with BCQ: fp32 quads [batch][L][32], box {32, T, 1}
+    CUtensorMap C[2];   // [batch][L][16]     box {16, T, 1}; unused with BCQ
 };
 
 constexpr int align128(int v) { return (v + 127) & ~127; }
 
 // DIRECT: B and C are read straight from the TMA tiles, so the fp32 B/C
-// buffers are not allocated.
-template <int G, int T, int NWD, int NS, typename Tin, bool DIRECT = false>
+// buffers are not allocated.  BCQ: B and C arrive already widened to fp32
+// quads (widen_bc_kernel), one TMA tile per chunk in the layout of the fp32
+// B/C buffer, which the states read in place.
+template <int G, int T, int NWD, int NS, typename Tin, bool DIRECT = false, bool BCQ = false>
 struct TmaGeo {
     static_assert(G == 4 || G == 8 || G == 16, "lanes per channel");
     static_assert(T % G == 0 && T <= 253, "chunk");
@@ -66,20 +68,62 @@ struct TmaGeo {
     static constexpr int XB = align128((T + 3) * XW * ESZ);
     static constexpr int DTB = align128(T * XW * ESZ);
     static constexpr int BB = align128(T * kNState * ESZ);
-    static constexpr int STAGE = XB + 2 * DTB + 2 * BB;   // x, dt, z, B, C
     static constexpr int BC32 = T * kNState * 2 * 4;      // one fp32 B/C buffer
+    static constexpr int STAGE = XB + 2 * DTB + (BCQ ? align128(BC32) : 2 * BB);  // x, dt, z, B and C
     static constexpr int ED2 = T * CPW * 8;               // per warp: (delta, delta*u)
     static constexpr int EDU = T * CPW * 4;               // per warp: D*u
     static constexpr int OWS = T * CPW * 4;               // per warp: partner's y
     static constexpr int WARP_BYTES = ED2 + EDU + OWS;
-    static constexpr int DIR_BYTES = NS * STAGE + (DIRECT ? 0 : 2 * BC32);
+    static constexpr int DIR_BYTES = NS * STAGE + ((DIRECT || BCQ) ? 0 : 2 * BC32);
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
     static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;  // + alignment slack
-    static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * XW + T * XW + 2 * T * kNState) * ESZ);
+    static constexpr uint32_t TX_BASE =
+        (uint32_t)(((T + 3) * XW + T * XW) * ESZ + (BCQ ? BC32 : 2 * T * kNState * ESZ));
     static constexpr uint32_t TX_Z = (uint32_t)(T * XW * ESZ);
     static_assert((XW * ESZ) % 16 == 0 && XW % CW == 0, "TMA box rows must be whole 16-byte units");
+    static_assert(!(BCQ && DIRECT), "one source of B/C");
 };
+
+// B and C of both directions widened to fp32 once per call, for the chunked
+// kernel's BCQ form: bcq[r][b][t] = 8 quads (B_2q, B_2q+1, C_2q, C_2q+1), the
+// layout of its fp32 B/C buffer (bf16 widening is exact).  One thread per
+// (direction, batch row, token); grid-stride.
+template <typename Tin>
+__global__ void __launch_bounds__(256) widen_bc_kernel(const KParams p) {
+    const int64_t rows = (int64_t)p.batch * p.L;
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < 2 * rows; i += (int64_t)gridDim.x * 256) {
+        const int r = (int)(i / rows);
+        const int64_t bt = i - r * rows;
+        const Tin* Bp = static_cast<const Tin*>(p.B[r]) + bt * kNState;
+        const Tin* Cp = static_cast<const Tin*>(p.C[r]) + bt * kNState;
+        float bv[kNState], cv[kNState];
+        if constexpr (sizeof(Tin) == 2) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 wb = reinterpret_cast<const uint4*>(Bp)[h];
+                const uint4 wc = reinterpret_cast<const uint4*>(Cp)[h];
+                const uint32_t b4[4] = {wb.x, wb.y, wb.z, wb.w}, c4[4] = {wc.x, wc.y, wc.z, wc.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {  // the bf16 bits are the high half of the fp32
+                    bv[8 * h + 2 * u] = __uint_as_float(b4[u] << 16);
+                    bv[8 * h + 2 * u + 1] = __uint_as_float(b4[u] & 0xffff0000u);
+                    cv[8 * h + 2 * u] = __uint_as_float(c4[u] << 16);
+                    cv[8 * h + 2 * u + 1] = __uint_as_float(c4[u] & 0xffff0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int n = 0; n < kNState; ++n) {
+                bv[n] = ldf(Bp, n);
+                cv[n] = ldf(Cp, n);
+            }
+        }
+        float4* o = reinterpret_cast<float4*>(p.bcq + i * 2 * kNState);
+#pragma unroll
+        for (int q = 0; q < kNState / 2; ++q) o[q] = make_float4(bv[2 * q], bv[2 * q + 1], cv[2 * q], cv[2 * q + 1]);
+    }
+}
 
 // fp32 B/C layout per token: 8 quads (B_2p, B_2p+1, C_2p, C_2p+1), so that a
 // lane's state pairs and their B and C are register pairs.
@@ -262,10 +306,10 @@ struct TmaWorker {
     }
 };
 
-template <int G, int T, int NWD, int NS, typename Tin>
+template <int G, int T, int NWD, int NS, typename Tin, bool BCQ = false>
 __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char* dir_base, uint64_t* full, int r,
                                             int i, int k, bool gated, int ct0, int b, int starve) {
-    using Ge = TmaGeo<G, T, NWD, NS, Tin>;
+    using Ge = TmaGeo<G, T, NWD, NS, Tin, false, BCQ>;
     if (starve) return;
     const int st = i % NS;
     unsigned char* sb = dir_base + st * Ge::STAGE;
@@ -277,15 +321,15 @@ __device__ __forceinline__ void issue_chunk(const LayerMaps& maps, unsigned char
     tma_load_3d(sb + Ge::XB, &maps.dt[r], bar, x0, row0, b);
     if (gated) tma_load_3d(sb + Ge::XB + Ge::DTB, &maps.z, bar, x0, row0, b);
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB, &maps.B[r], bar, 0, row0, b);
-    tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
+    if constexpr (!BCQ) tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
 template <int G, int T, int NWD, int NS, typename Tin, typename Tout, int DIR, bool CARRY, bool DIRECT,
-          bool FULL_UNROLL = false>
+          bool FULL_UNROLL = false, bool BCQ = false>
 __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KParams& p, unsigned char* base,
                                                 int wg, int lane) {
-    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT>;
+    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT, BCQ>;
     using Wk = TmaWorker<G, T, NWD, NS, Tin, DIR>;
     unsigned char* dir_base = base + DIR * Ge::DIR_BYTES;
     float* bc32 = reinterpret_cast<float*>(dir_base + NS * Ge::STAGE);
@@ -317,7 +361,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     if (leader) {
         for (int i = 0; i < NS && i < nc; ++i) {
             const int k = DIR == 0 ? i : nc - 1 - i;
-            issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i, k, i >= meet, ct0, b, p.starve);
+            issue_chunk<G, T, NWD, NS, Tin, BCQ>(maps, dir_base, full, DIR, i, k, i >= meet, ct0, b, p.starve);
         }
     }
 
@@ -363,8 +407,9 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
             put_conv_halo(reinterpret_cast<Tin*>(dir_base + st * Ge::STAGE), Ge::XW,
                           DIR == 0 ? 0 : (int)(L - (int64_t)k * T), ct0 % Ge::XW + wg * Ge::CPW, c0w, Ge::CPW,
                           static_cast<const Tin*>(p.conv_halo[DIR]) + (int64_t)b * 3 * D, D, lane);
-        float* bc = bc32 + (i & 1) * (T * kNState * 2);
-        if constexpr (!DIRECT) convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
+        float* bc = BCQ ? reinterpret_cast<float*>(dir_base + st * Ge::STAGE + Ge::XB + 2 * Ge::DTB)
+                        : bc32 + (i & 1) * (T * kNState * 2);
+        if constexpr (!DIRECT && !BCQ) convert_bc<T, Tin>(Bt, Ct, bc, gtid, NWD * 32, true);
         // every warp of the direction is past the previous chunk (and, unless
         // DIRECT, the fp32 B/C rows of this one are written)
         if constexpr (NWD == 1)
@@ -373,8 +418,8 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
             named_bar_sync(1 + DIR, NWD * 32);
         if (leader && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
-            issue_chunk<G, T, NWD, NS, Tin>(maps, dir_base, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2,
-                                            i2 >= meet, ct0, b, p.starve);
+            issue_chunk<G, T, NWD, NS, Tin, BCQ>(maps, dir_base, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2,
+                                                 i2 >= meet, ct0, b, p.starve);
         }
 
         wk.template elements<CARRY>(xt, dtt, s_lo, s_hi, ed2, edu);
@@ -417,17 +462,19 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     }
 }
 
-// Resident CTAs per SM the register budget is sized for.
-template <int G, int T>
+// Resident CTAs per SM the register budget is sized for.  One warp per
+// direction: 7 two-warp CTAs, so that the 1024 CTAs of a 4096-channel batch
+// row (4 channels each) are resident at once on 148 SMs.
+template <int G, int T, int NWD>
 constexpr int layer_min_blocks() {
-    return (T <= 16 || G >= 16) ? 4 : 3;
+    return NWD == 1 ? 7 : (T <= 16 || G >= 16) ? 4 : 3;
 }
 
 template <int G, int T, int NWD, int NS, typename Tin, typename Tout, bool CARRY = false, bool DIRECT = false,
-          bool FULL_UNROLL = false>
-__global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
+          bool FULL_UNROLL = false, bool BCQ = false>
+__global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T, NWD>()))
     layer_tma_kernel(const __grid_constant__ LayerMaps maps, const KParams p) {
-    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT>;
+    using Ge = TmaGeo<G, T, NWD, NS, Tin, DIRECT, BCQ>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~static_cast<uintptr_t>(127));
@@ -439,9 +486,10 @@ __global__ void __launch_bounds__(2 * NWD * 32, (layer_min_blocks<G, T>()))
     }
     __syncthreads();
     if (warp < NWD)
-        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY, DIRECT, FULL_UNROLL>(maps, p, base, warp, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 0, CARRY, DIRECT, FULL_UNROLL, BCQ>(maps, p, base, warp, lane);
     else
-        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY, DIRECT, FULL_UNROLL>(maps, p, base, warp - NWD, lane);
+        layer_direction<G, T, NWD, NS, Tin, Tout, 1, CARRY, DIRECT, FULL_UNROLL, BCQ>(maps, p, base, warp - NWD,
+                                                                                     lane);
 }
 
 // ---------------------------------------------------------------- prefix

@@ -127,6 +127,7 @@ struct KParams {
     const float* conv_b;   // [2][D] or nullptr
     void* out;             // [batch][L][D]
     float* ws;             // [batch][L][D] fp32 (layer only)
+    float* bcq;            // [2][batch][L][8][4] fp32: B/C quads (chunked layer at 8 lanes)
     const float* h_in;     // [batch][D][16]   (block step)
     const void* tail_in;   // [batch][3][D]    (block step)
     float* h_out;          // [batch][D][16]   (prefix, block commit) or nullptr

@@ -134,7 +134,9 @@ typedef struct {
 
 /* Bytes of device workspace bimamba_layer_fwd needs: one fp32 per
  * (batch, token, channel) for the half-sequence partial outputs the two
- * directions hand each other.  Returns 0 for invalid sizes. */
+ * directions hand each other, rounded up to 256 bytes, plus 32 fp32 per
+ * (direction, batch, token) for B and C widened once per call (the chunked
+ * kernel at 8 lanes per channel).  Returns 0 for invalid sizes. */
 size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, unsigned flags);
 
 /* Full-sequence bidirectional layer (§3.2 Eq. (4)-(6)).
@@ -143,7 +145,8 @@ size_t bimamba_workspace_bytes(int batch, int64_t L, int d_inner, int d_state, u
  *   out         [batch][L][d_inner] of out_dtype
  *   workspace   >= bimamba_workspace_bytes(...) bytes of device memory, 16-byte
  *               aligned, contents ignored on entry and undefined on exit
- * One kernel launch. */
+ * One kernel launch (two for the chunked kernel at 8 lanes per channel: the
+ * B/C widening, then the layer). */
 int bimamba_layer_fwd(const bimamba_inputs_t *in, const bimamba_params_t *p,
                       void *out, bimamba_dtype_t out_dtype,
                       int batch, int64_t L, int d_inner, int d_state, unsigned flags,
@@ -214,9 +217,10 @@ int bimamba_compose_carries(const float *h_out_all, const float *delta_sum_all, 
  * bimamba_layer_fwd computes.
  *   Instead of a caller's workspace it uses a scratch array built into the
  * library: 64 MiB that every GPU loading the library holds until the process
- * exits.  It therefore accepts batch * L * d_inner <= 16,777,216 (the
- * workspace bimamba_workspace_bytes reports must fit in 64 MiB) and returns
- * BIMAMBA_ERR_WORKSPACE above that.  It allocates and frees nothing.
+ * exits.  It therefore accepts the sizes whose bimamba_workspace_bytes fits
+ * in 64 MiB (batch * L * (4 d_inner + 256) bytes, about batch * L * d_inner
+ * <= 16.5 M at d_inner 4096) and returns BIMAMBA_ERR_WORKSPACE above that.
+ * It allocates and frees nothing.
  *   The first call in a CUDA context looks up the scratch array's device
  * address (cudaGetSymbolAddress, with the device current) and caches it for
  * that context; a context created anew (after cudaDeviceReset, say) looks it

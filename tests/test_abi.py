@@ -40,15 +40,16 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert bm.lib.bimamba_abi_version() == 1
+    assert bm.lib.bimamba_abi_version() == 2
     for s in (0, -1, -2, -3, -4, -5):
         assert bm.status_string(s) and bm.status_string(s) != "unknown status"
     assert bm.status_string(-99) == "unknown status"
 
 
 def test_workspace_bytes():
-    assert bm.bimamba_workspace_bytes(8, 2048, 4096) == 8 * 2048 * 4096 * 4
-    assert bm.bimamba_workspace_bytes(1, 1, 1) == 4
+    # fp32 partial outputs [b][L][D] rounded up to 256 bytes, then fp32 B/C quads [2][b][L][32]
+    assert bm.bimamba_workspace_bytes(8, 2048, 4096) == 8 * 2048 * 4096 * 4 + 2 * 8 * 2048 * 32 * 4
+    assert bm.bimamba_workspace_bytes(1, 1, 1) == 256 + 2 * 32 * 4
     assert bm.bimamba_workspace_bytes(0, 10, 10) == 0
     assert bm.bimamba_workspace_bytes(1, 0, 10) == 0
     assert bm.bimamba_workspace_bytes(1, 10, 10, d_state=8) == 0
@@ -417,9 +418,10 @@ def test_header_serves_a_plain_c_program(tmp_path):
 #include <string.h>
 #include "bimamba.h"
 int main(void) {
-    if (bimamba_abi_version() != 1) return 1;
+    if (bimamba_abi_version() != 2) return 1;
     if (strlen(bimamba_status_string(BIMAMBA_ERR_INVALID_ARG)) == 0) return 2;
-    if (bimamba_workspace_bytes(8, 2048, 4096, 16, 0) != (size_t)8 * 2048 * 4096 * 4) return 3;
+    if (bimamba_workspace_bytes(8, 2048, 4096, 16, 0) != (size_t)8 * 2048 * 4096 * 4 + (size_t)2 * 8 * 2048 * 32 * 4)
+        return 3;
     if (bimamba2_workspace_bytes(0, 10, 4, 32, 128) != 0) return 4;
     /* a call with no inputs is rejected before anything is launched */
     if (bimamba_layer_fwd(NULL, NULL, NULL, BIMAMBA_BF16, 1, 16, 32, 16, 0, NULL, 0, NULL) !=

@@ -81,14 +81,14 @@ def test_noalloc_matches_layer_fwd_twice(bm, shape, out_dtype, flags):
 
 
 def _oversize_inputs():
-    L = 4096 + 8  # batch * L * d_inner = 16,809,984 > 16,777,216
+    L = 4096 + 8  # workspace 4104 * (4096 * 4 + 256) bytes > 64 MiB
     x = torch.empty(1, L, 4096, device="cuda", dtype=torch.bfloat16)
     bc = torch.empty(2, 1, L, 16, device="cuda", dtype=torch.bfloat16)
     return {"x": x, "z": x, "dt": torch.stack([x, x]), "B": bc, "C": bc}
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(bm):
-    """batch * L * d_inner above 16,777,216 does not fit the 64 MiB scratch:
+    """A workspace above 64 MiB does not fit the scratch:
     the call returns BIMAMBA_ERR_WORKSPACE and launches nothing."""
     inp = _oversize_inputs()
     _, par = W.make_case(1, 4, 4096, 16, "bf16", seed=1, device="cuda")
