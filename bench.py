@@ -383,6 +383,20 @@ def flags_of(args, bm):
             | (args.family << bm.BIMAMBA_FAMILY_SHIFT) | args.flags)
 
 
+def layer_launches(batch: int, d_inner: int, args, carry: bool = False) -> int:
+    """The library's kernel launches per layer call: two (B/C widening, then
+    the layer) for the chunked family at 8 lanes per channel with 32-token
+    chunks, one otherwise."""
+    fam = args.family or (2 if 2 * batch * d_inner >= SMS * 8 * 32 else 1)
+    if fam != 1 or (args.flags & 0x2000):  # BIMAMBA_CHUNKED_WIDE
+        return 1
+    lanes = args.lanes or (4 if 2 * batch * d_inner * 4 >= SMS * 1024 else 8)
+    chunk = 32 if lanes >= 8 else 16
+    if args.chunk and not carry:
+        chunk = 16 if args.chunk == 1 else 32
+    return 2 if (lanes == 8 and chunk == 32) else 1
+
+
 def kernel_name(w: W.Workload, args) -> str:
     if args.workload in ("block", "decode"):
         return "async_block_kernel"
@@ -452,7 +466,7 @@ def run_chunked(args, w, bm, rank, world, dev, stream):
     return {
         "value": whole_job_rate(w.batch * w.L * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
-        "gpu_launches": args.steps * (2 + args.segments + 2),
+        "gpu_launches": args.steps * (2 * layer_launches(args.segments, w.d_inner, args, carry=True) + args.segments),
         "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, "fused_layer_kernel x 2 passes"),
         "hbm": hbm_fraction(layer_bytes(w.batch, w.L, w.d_inner, w.d_state, 2), call_ms),
         "clocks": clocks,
@@ -492,7 +506,7 @@ def run_layer_like(args, w, bm, rank, world, dev, stream):
     res = {
         "value": whole_job_rate(w.batch * w.L * calls * args.steps, world, ms_max / 1e3),
         "ms_per_step": ms_max / args.steps,
-        "gpu_launches": args.steps * calls,
+        "gpu_launches": args.steps * calls * layer_launches(w.batch, w.d_inner, args),
         "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args)),
         "hbm": hbm_fraction(layer_bytes(w.batch, w.L, w.d_inner, w.d_state, 2), call_ms),
         "clocks": clocks,
@@ -824,7 +838,8 @@ def run_sharded(args, w, bm, rank, world, dev, stream):
     elems = w.batch * Ls * w.d_inner
     res = {
         "value": whole_job_rate(w.batch * Ls * args.steps, world, ms_max / 1e3),
-        "ms_per_step": ms_max / args.steps, "gpu_launches": 3 * args.steps, "scaling": "strong",
+        "ms_per_step": ms_max / args.steps, "scaling": "strong",
+        "gpu_launches": (2 * layer_launches(w.batch, w.d_inner, args, carry=True) + 1) * args.steps,
         "roofline": roofline(MUFU_PER_ELEM_LAYER * elems, step_ms / 2, clocks, w.name, kernel_name(w, args)),
         "clocks": clocks,
         "method": "two layer passes per segment (from zero for the aggregates, then from the composed carries)",
