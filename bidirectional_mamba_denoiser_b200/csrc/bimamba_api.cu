@@ -272,6 +272,22 @@ bool fill_maps(bimamba::LayerMaps& m, const bimamba_inputs_t* in, int batch, int
     return ok;
 }
 
+// Both directions' B and C widened to fp32 quads into k.bcq (one small
+// launch), and the two tensor maps over them (boxes of T tokens) in maps_b.
+template <typename Tin>
+int widen_bc(const KParams& k, int T, CUtensorMap* maps_b, cudaStream_t st) {
+    const int64_t rows = 2 * (int64_t)k.batch * k.L;
+    const int64_t blocks = (rows + 255) / 256;
+    bimamba::widen_bc_kernel<Tin><<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const size_t per_dir = (size_t)k.batch * (size_t)k.L * 2 * bimamba::kNState;
+    for (int r = 0; r < 2; ++r)
+        if (!map3d(&maps_b[r], k.bcq + r * per_dir, false, 2 * bimamba::kNState, (uint64_t)k.L, (uint64_t)k.batch,
+                   2 * bimamba::kNState, (uint32_t)T))
+            return BIMAMBA_ERR_CUDA;
+    return BIMAMBA_OK;
+}
+
 // BCQ: B and C widened to fp32 quads in the workspace first (one small
 // launch), then read by TMA in the layout the states use, with no widening in
 // the scan loop.
@@ -282,15 +298,8 @@ int launch_layer_tma(const KParams& k, const bimamba_inputs_t* in, cudaStream_t 
     bimamba::LayerMaps maps;
     if (!fill_maps<G, T, Tin, NWD>(maps, in, k.batch, k.L, k.D, true, true)) return BIMAMBA_ERR_CUDA;
     if constexpr (BCQ) {
-        const int64_t rows = 2 * (int64_t)k.batch * k.L;
-        const int64_t blocks = (rows + 255) / 256;
-        bimamba::widen_bc_kernel<Tin><<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(k);
-        if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
-        const size_t per_dir = (size_t)k.batch * (size_t)k.L * 2 * bimamba::kNState;
-        for (int r = 0; r < 2; ++r)
-            if (!map3d(&maps.B[r], k.bcq + r * per_dir, false, 2 * bimamba::kNState, (uint64_t)k.L,
-                       (uint64_t)k.batch, 2 * bimamba::kNState, T))
-                return BIMAMBA_ERR_CUDA;
+        int rc = widen_bc<Tin>(k, T, maps.B, st);
+        if (rc) return rc;
     }
     auto kern = &bimamba::layer_tma_kernel<G, T, NWD, kTNS, Tin, Tout, CARRY, DIRECT, FULL_UNROLL, BCQ>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
@@ -407,12 +416,18 @@ bool fill_fused_maps(bimamba::FusedMaps& m, const bimamba_inputs_t* in, int batc
     return ok;
 }
 
-template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false>
+// BCQ (one lane per channel): B and C widened to fp32 quads in the workspace
+// first, then read by TMA with no per-chunk widening.
+template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false, bool BCQ = false>
 int launch_fused_layer(const KParams& k, const bimamba_inputs_t* in, cudaStream_t st) {
-    using Ge = bimamba::FusedGeo<G, Tin, F32BC>;
+    using Ge = bimamba::FusedGeo<G, Tin, F32BC, BCQ>;
     bimamba::FusedMaps maps;
     if (!fill_fused_maps<G, Tin>(maps, in, k.batch, k.L, k.D, true)) return BIMAMBA_ERR_CUDA;
-    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout, CARRY, F32BC>;
+    if constexpr (BCQ) {
+        int rc = widen_bc<Tin>(k, (int)Ge::T, maps.B, st);
+        if (rc) return rc;
+    }
+    auto kern = &bimamba::fused_layer_kernel<G, Tin, Tout, CARRY, F32BC, 4, BCQ>;
     int rc = ensure_smem(reinterpret_cast<const void*>(kern), Ge::SMEM);
     if (rc) return rc;
     dim3 grid((unsigned)((k.D + Ge::CW - 1) / Ge::CW), (unsigned)k.batch);
@@ -430,7 +445,7 @@ int fused_layer_by_group(int g, bool f32bc, const KParams& k, const bimamba_inpu
         return BIMAMBA_ERR_UNSUPPORTED;
     }
     switch (g) {
-        case 1: return launch_fused_layer<1, Tin, Tout>(k, in, st);
+        case 1: return launch_fused_layer<1, Tin, Tout, false, false, true>(k, in, st);
         case 2: return launch_fused_layer<2, Tin, Tout>(k, in, st);
         case 4: return launch_fused_layer<4, Tin, Tout>(k, in, st);
         case 8: return launch_fused_layer<8, Tin, Tout>(k, in, st);
@@ -675,10 +690,10 @@ int layer_fwd_impl(const bimamba_inputs_t* in, const bimamba_params_t* p, const 
     if (!(flags & BIMAMBA_NO_TMA) && fam == 2 && group_ok &&
         tma_eligible(in, d_inner, true, true)) {
         if (with_carry) {  // carries: one lane per channel (the group size changes only the speed)
-            if (in_bf && out_bf) return launch_fused_layer<1, bf16, bf16, true>(k, in, st);
-            if (in_bf) return launch_fused_layer<1, bf16, float, true>(k, in, st);
-            if (out_bf) return launch_fused_layer<1, float, bf16, true>(k, in, st);
-            return launch_fused_layer<1, float, float, true>(k, in, st);
+            if (in_bf && out_bf) return launch_fused_layer<1, bf16, bf16, true, false, true>(k, in, st);
+            if (in_bf) return launch_fused_layer<1, bf16, float, true, false, true>(k, in, st);
+            if (out_bf) return launch_fused_layer<1, float, bf16, true, false, true>(k, in, st);
+            return launch_fused_layer<1, float, float, true, false, true>(k, in, st);
         }
         const int gf = pick_group_fused(flags);
         // B/C widened to fp32 once per chunk at 2 lanes per group (measured

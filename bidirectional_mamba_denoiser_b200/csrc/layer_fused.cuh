@@ -34,13 +34,15 @@ struct FusedMaps {
     CUtensorMap x;      // [batch][L][D]    box {32, T+3, 1}
     CUtensorMap z;      // [batch][L][D]    box {32, T, 1}
     CUtensorMap dt[2];  // [batch][L][D]    box {32, T, 1}
-    CUtensorMap B[2];   // [batch][L][16]   box {16, T, 1}
-    CUtensorMap C[2];   // [batch][L][16]   box {16, T, 1}
+    CUtensorMap B[2];   // [batch][L][16]   box {16, T, 1}; with BCQ: fp32 quads [batch][L][32], box {32, T, 1}
+    CUtensorMap C[2];   // [batch][L][16]   box {16, T, 1}; unused with BCQ
 };
 
 // F32BC: B and C are widened to fp32 once per chunk (into a per-warp buffer)
-// instead of at every use.
-template <int G, typename Tin, bool F32BC = false>
+// instead of at every use.  BCQ (one lane per channel): B and C arrive
+// already widened to fp32 quads (B_2q, B_2q+1, C_2q, C_2q+1) per token,
+// written once per call by widen_bc_kernel, and are read from the TMA tile.
+template <int G, typename Tin, bool F32BC = false, bool BCQ = false>
 struct FusedGeo {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "lanes per group");
     static constexpr int T = 16;                // tokens per chunk
@@ -51,18 +53,21 @@ struct FusedGeo {
     static constexpr int XB = (((T + 3) * CW * ESZ) + 127) & ~127;
     static constexpr int DTB = ((T * CW * ESZ) + 127) & ~127;
     static constexpr int BB = ((T * kNState * ESZ) + 127) & ~127;
-    static constexpr int STAGE = XB + 2 * DTB + 2 * BB;  // x, dt, z, B, C
+    static constexpr int BQB = ((T * 2 * kNState * 4) + 127) & ~127;  // the fp32 quads of a chunk
+    static constexpr int STAGE = XB + 2 * DTB + (BCQ ? BQB : 2 * BB);  // x, dt, z, B and C
     static constexpr int OWS = T * CW * 4;               // partner's y of a chunk
     // With G == 1 every lane needs all 16 B and C of a token, and with F32BC
     // they are wanted as fp32 anyway: they are converted once per chunk
     // (T x 32 floats) instead of per use.
-    static constexpr int BCF = (G == 1 || F32BC) ? T * 2 * kNState * 4 : 0;
+    static constexpr int BCF = (!BCQ && (G == 1 || F32BC)) ? T * 2 * kNState * 4 : 0;
     static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF;
     static constexpr int BAR_OFF = 2 * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
-    static constexpr uint32_t TX_BASE = (uint32_t)(((T + 3) * CW + T * CW + 2 * T * kNState) * ESZ);
+    static constexpr uint32_t TX_BASE =
+        (uint32_t)(((T + 3) * CW + T * CW) * ESZ + (BCQ ? T * 2 * kNState * 4 : 2 * T * kNState * ESZ));
     static constexpr uint32_t TX_Z = (uint32_t)(T * CW * ESZ);
     static_assert(T + 3 <= 256 && CW <= 256, "TMA box dimensions");
+    static_assert(!BCQ || G == 1, "fp32 quads: one lane per channel");
 };
 
 // S consecutive B (or C) values of a token row, as fp32.
@@ -95,9 +100,9 @@ __device__ __forceinline__ void load_row(const float* p, float (&v)[S]) {
     load_states<S>(p, v);
 }
 
-template <int G, typename Tin, typename Tout, int DIR, bool LAYER, bool F32BC = false>
+template <int G, typename Tin, typename Tout, int DIR, bool LAYER, bool F32BC = false, bool BCQ = false>
 struct FusedWarp {
-    using Ge = FusedGeo<G, Tin, F32BC>;
+    using Ge = FusedGeo<G, Tin, F32BC, BCQ>;
     static constexpr int T = Ge::T, NS = Ge::NS, S = Ge::S;
 
     // own channel (per-token work and output)
@@ -172,13 +177,22 @@ struct FusedWarp {
     // gathered from the group's lanes); returns sum_n C h of the own channel
     // (WITH_Y), before the D skip.
     // G == 1: the lane's own channel, all 16 states; B and C of the token
-    // come as fp32 from the per-chunk buffer bcf ([T][B 16 | C 16]).
+    // come as fp32 from the per-chunk buffer bcf ([T][B 16 | C 16]), or with
+    // BCQ from the chunk's tile of fp32 quads ([T][8][B B C C]).
     template <bool WITH_Y>
     __device__ __forceinline__ float scan1(int s, const Elem& e, const float* bcf) {
         const float* rowp = bcf + row_of(s) * 2 * kNState;
         float bv[kNState], cvv[kNState];
-        load_states<kNState>(rowp, bv);
-        if constexpr (WITH_Y) load_states<kNState>(rowp + kNState, cvv);
+        if constexpr (BCQ) {
+#pragma unroll
+            for (int q = 0; q < kNState / 2; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(rowp + 4 * q);
+                bv[2 * q] = v.x; bv[2 * q + 1] = v.y; cvv[2 * q] = v.z; cvv[2 * q + 1] = v.w;
+            }
+        } else {
+            load_states<kNState>(rowp, bv);
+            if constexpr (WITH_Y) load_states<kNState>(rowp + kNState, cvv);
+        }
         const float2 dd = make_float2(e.dl, e.dl);
         const float2 uu = make_float2(e.du, e.du);
         float2 acc2 = make_float2(0.f, 0.f);
@@ -246,10 +260,10 @@ __device__ __forceinline__ void fused_convert_bc(const Tin* Bt, const Tin* Ct, f
     for (int r = 0; r < T; ++r) bcf[r * 2 * kNState + lane] = ldf(src, r * kNState + n);
 }
 
-template <int G, typename Tin, bool F32BC = false>
+template <int G, typename Tin, bool F32BC = false, bool BCQ = false>
 __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char* wbase, uint64_t* full, int r,
                                             int i, int k, bool gated, int ct0, int b, int starve) {
-    using Ge = FusedGeo<G, Tin, F32BC>;
+    using Ge = FusedGeo<G, Tin, F32BC, BCQ>;
     if (starve) return;
     const int st = i % Ge::NS;
     unsigned char* sb = wbase + st * Ge::STAGE;
@@ -260,16 +274,16 @@ __device__ __forceinline__ void fused_issue(const FusedMaps& maps, unsigned char
     tma_load_3d(sb + Ge::XB, &maps.dt[r], bar, ct0, row0, b);
     if (gated) tma_load_3d(sb + Ge::XB + Ge::DTB, &maps.z, bar, ct0, row0, b);
     tma_load_3d(sb + Ge::XB + 2 * Ge::DTB, &maps.B[r], bar, 0, row0, b);
-    tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
+    if constexpr (!BCQ) tma_load_3d(sb + Ge::XB + 2 * Ge::DTB + Ge::BB, &maps.C[r], bar, 0, row0, b);
 }
 
 // CARRY: start from p.carry_in, report p.carry_out and p.delta_sum (each where non-null).
-template <int G, typename Tin, typename Tout, int DIR, bool CARRY, bool F32BC, int UNR = 4>
+template <int G, typename Tin, typename Tout, int DIR, bool CARRY, bool F32BC, int UNR = 4, bool BCQ = false>
 __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, const KParams& p, unsigned char* base,
                                                       int lane) {
-    using Ge = FusedGeo<G, Tin, F32BC>;
+    using Ge = FusedGeo<G, Tin, F32BC, BCQ>;
     constexpr int T = Ge::T, NS = Ge::NS, S = Ge::S;
-    using Wp = FusedWarp<G, Tin, Tout, DIR, true, F32BC>;
+    using Wp = FusedWarp<G, Tin, Tout, DIR, true, F32BC, BCQ>;
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
     float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS);
@@ -299,7 +313,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     float dsum = 0.f;  // step sizes of the own channel so far
     if (lane == 0)
         for (int i = 0; i < NS && i < nc; ++i)
-            fused_issue<G, Tin, F32BC>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b,
+            fused_issue<G, Tin, F32BC, BCQ>(maps, wbase, full, DIR, i, DIR == 0 ? i : nc - 1 - i, i >= meet, ct0, b,
                                        p.starve);
 
 #pragma unroll 1
@@ -313,7 +327,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         // the previous chunk's stage is free (this warp is past it): refill it
         if (lane == 0 && i >= 1 && i - 1 + NS < nc) {
             const int i2 = i - 1 + NS;
-            fused_issue<G, Tin, F32BC>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b,
+            fused_issue<G, Tin, F32BC, BCQ>(maps, wbase, full, DIR, i2, DIR == 0 ? i2 : nc - 1 - i2, i2 >= meet, ct0, b,
                                        p.starve);
         }
         const int nvalid = (int)((L - (int64_t)k * T < T) ? (L - (int64_t)k * T) : T);
@@ -346,7 +360,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             cp_async_wait_all();
             __syncwarp();
         }
-        if constexpr (G == 1 || F32BC) {
+        if constexpr (!BCQ && (G == 1 || F32BC)) {
             __syncwarp();
             fused_convert_bc<T, Tin>(Bt, Ct, bcf, lane, true);
             __syncwarp();
@@ -363,7 +377,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
             if (s + 1 < T) nxt = wp.element(s + 1, s + 1 >= s_lo && s + 1 < s_hi, xt, dtt);
             float yr;
             if constexpr (G == 1)
-                yr = wp.template scan1<true>(s, cur, bcf);
+                yr = wp.template scan1<true>(s, cur, BCQ ? reinterpret_cast<const float*>(Bt) : bcf);
             else
                 yr = wp.template scan<true>(s, cur, Bt, Ct, bcf);
             const float y = (yr + cur.Du) * scale;
@@ -399,9 +413,9 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
 // The token loop unrolled by 4 (with 2-lane groups: 1.116 against 1.154 ms
 // for 2, 1.25 for 8 and 1.41 for all 16 at batch 8, L 2048, d_inner 4096;
 // with one lane per channel 1.096 against 1.137 for 2 and 1.20 for 8).
-template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false, int UNR = 4>
+template <int G, typename Tin, typename Tout, bool CARRY = false, bool F32BC = false, int UNR = 4, bool BCQ = false>
 __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constant__ FusedMaps maps, const KParams p) {
-    using Ge = FusedGeo<G, Tin, F32BC>;
+    using Ge = FusedGeo<G, Tin, F32BC, BCQ>;
     extern __shared__ __align__(128) unsigned char smem_dyn[];
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 127) & ~static_cast<uintptr_t>(127));
@@ -413,9 +427,9 @@ __global__ void __launch_bounds__(64, 8) fused_layer_kernel(const __grid_constan
     }
     __syncthreads();
     if (warp == 0)
-        fused_layer_direction<G, Tin, Tout, 0, CARRY, F32BC, UNR>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 0, CARRY, F32BC, UNR, BCQ>(maps, p, base, lane);
     else
-        fused_layer_direction<G, Tin, Tout, 1, CARRY, F32BC, UNR>(maps, p, base, lane);
+        fused_layer_direction<G, Tin, Tout, 1, CARRY, F32BC, UNR, BCQ>(maps, p, base, lane);
 }
 
 // Forward scan over P = p.L tokens from zero: final state and conv tail.
