@@ -58,7 +58,7 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 # (a step reads the same bytes whatever the prefix length).
 NCU_TRAFFIC = {
 
-    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1308.5e6,
+    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): None,  # kernel changed since the last capture
     ("mamba2_1p3b_b8_L2048_H120x32_N128_bf16", "m2_prep + m2_ssd dual-form kernel (both directions)"): 1027.8e6,
     ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1448.1e6,
     ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1448.1e6,
@@ -385,9 +385,11 @@ def flags_of(args, bm):
 
 def layer_launches(batch: int, d_inner: int, args, carry: bool = False) -> int:
     """The library's kernel launches per layer call: two (B/C widening, then
-    the layer) for the chunked family at 8 lanes per channel with 32-token
-    chunks, one otherwise."""
+    the layer) for the per-token family at one lane per channel and for the
+    chunked family at 8 lanes per channel with 32-token chunks, one otherwise."""
     fam = args.family or (2 if 2 * batch * d_inner >= SMS * 8 * 32 else 1)
+    if fam == 2:
+        return 2 if (carry or args.lanes in (0, 1)) else 1
     if fam != 1 or (args.flags & 0x2000):  # BIMAMBA_CHUNKED_WIDE
         return 1
     lanes = args.lanes or (4 if 2 * batch * d_inner * 4 >= SMS * 1024 else 8)
