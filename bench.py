@@ -58,7 +58,7 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 # (a step reads the same bytes whatever the prefix length).
 NCU_TRAFFIC = {
 
-    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): None,  # kernel changed since the last capture
+    ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1311.6e6,
     ("mamba2_1p3b_b8_L2048_H120x32_N128_bf16", "m2_prep + m2_ssd dual-form kernel (both directions)"): 1027.8e6,
     ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1448.1e6,
     ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1448.1e6,
