@@ -1034,12 +1034,12 @@ int launch_m2_ssd(const bimamba::M2Params& k, bool no_cluster, cudaStream_t st) 
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return BIMAMBA_ERR_CUDA;
     if (!no_cluster && (int64_t)k.H * k.batch <= 2LL * sms) {
-        kc<<<dim3((unsigned)(2 * k.H), (unsigned)k.batch), 128, bimamba::kSsdSmem, st>>>(k);
+        kc<<<dim3((unsigned)(2 * k.H), (unsigned)k.batch), bimamba::kSsdThreads, bimamba::kSsdSmem, st>>>(k);
         return launch_status();
     }
     const int64_t n1 = (int64_t)k.H * k.batch;
     if (cudaMemsetAsync(k.sync, 0, (size_t)(1 + n1) * sizeof(int), st) != cudaSuccess) return BIMAMBA_ERR_CUDA;
-    kt<<<(unsigned)(2 * n1), 128, bimamba::kSsdSmem, st>>>(k);
+    kt<<<(unsigned)(2 * n1), bimamba::kSsdThreads, bimamba::kSsdSmem, st>>>(k);
     return launch_status();
 }
 

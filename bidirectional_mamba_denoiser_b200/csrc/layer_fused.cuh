@@ -55,12 +55,12 @@ struct FusedGeo {
     static constexpr int BB = ((T * kNState * ESZ) + 127) & ~127;
     static constexpr int BQB = ((T * 2 * kNState * 4) + 127) & ~127;  // the fp32 quads of a chunk
     static constexpr int STAGE = XB + 2 * DTB + (BCQ ? BQB : 2 * BB);  // x, dt, z, B and C
-    static constexpr int OWS = T * CW * 4;               // partner's y of a chunk
+    static constexpr int OWS = T * CW * 4;               // partner's y of a chunk (double-buffered)
     // With G == 1 every lane needs all 16 B and C of a token, and with F32BC
     // they are wanted as fp32 anyway: they are converted once per chunk
     // (T x 32 floats) instead of per use.
     static constexpr int BCF = (!BCQ && (G == 1 || F32BC)) ? T * 2 * kNState * 4 : 0;
-    static constexpr int WARP_BYTES = NS * STAGE + OWS + BCF;
+    static constexpr int WARP_BYTES = NS * STAGE + 2 * OWS + BCF;
     static constexpr int BAR_OFF = 2 * WARP_BYTES;
     static constexpr int SMEM = BAR_OFF + 2 * NS * 8 + 128;
     static constexpr uint32_t TX_BASE =
@@ -286,7 +286,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     using Wp = FusedWarp<G, Tin, Tout, DIR, true, F32BC, BCQ>;
     unsigned char* wbase = base + DIR * Ge::WARP_BYTES;
     float* ows = reinterpret_cast<float*>(wbase + NS * Ge::STAGE);
-    float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + Ge::OWS);
+    float* bcf = reinterpret_cast<float*>(wbase + NS * Ge::STAGE + 2 * Ge::OWS);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + Ge::BAR_OFF) + DIR * NS;
     const int b = blockIdx.y;
     const int ct0 = blockIdx.x * Ge::CW;
@@ -296,6 +296,20 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
     const int hF = nc / 2;
     const int meet = DIR == 0 ? hF : nc - hF;
     const float scale = p.dir_scale[DIR];
+    // cp.async of the partner's fp32 y of chunk ii (T rows x 32 channels,
+    // 16-byte pieces; D % 4 == 0 on this path) into buffer ii & 1
+    auto fetch_partner = [&](int ii) {
+        const int kk = DIR == 0 ? ii : nc - 1 - ii;
+        const int64_t row = (int64_t)b * L + (int64_t)kk * T;
+        float* dst = ows + (ii & 1) * (T * Ge::CW);
+        for (int e = lane; e < T * 8; e += 32) {
+            const int r = e >> 3, q = e & 7;
+            const bool ok = (int64_t)kk * T + r < L && ct0 + 4 * q < D;
+            const float* src = p.ws + (row + (ok ? r : 0)) * D + (ok ? ct0 + 4 * q : 0);
+            cp_async<16>(dst + r * Ge::CW + 4 * q, src, ok);
+        }
+        cp_async_commit();
+    };
 
     Wp wp;
     wp.setup(p, ct0, lane);
@@ -334,16 +348,11 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
         const int s_lo = DIR == 0 ? 0 : T - nvalid;
         const int s_hi = DIR == 0 ? nvalid : T;
         const int64_t chunk_row = (int64_t)b * L + (int64_t)k * T;
-        if (gated) {
-            // partner's y: T rows x 32 channels, 16-byte pieces (D % 4 == 0 here)
-            for (int e = lane; e < T * 8; e += 32) {
-                const int r = e >> 3, q = e & 7;
-                const bool ok = (int64_t)k * T + r < L && ct0 + 4 * q < D;
-                const float* src = p.ws + (chunk_row + (ok ? r : 0)) * D + (ok ? ct0 + 4 * q : 0);
-                cp_async<16>(ows + r * Ge::CW + 4 * q, src, ok);
-            }
-            cp_async_commit();
-        }
+        // The partner's y of the gated chunks, one chunk ahead (buffer i & 1):
+        // the copy of chunk i+1 runs under the scan of chunk i.  All of it was
+        // stored before the meeting barrier.
+        if (i == meet) fetch_partner(i);
+        if (gated && i + 1 < nc) fetch_partner(i + 1);
         const int st = i % NS;
         mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
         const unsigned char* sb = wbase + st * Ge::STAGE;
@@ -357,9 +366,13 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
                           DIR == 0 ? 0 : (int)(L - (int64_t)k * T), 0, ct0, Ge::CW,
                           static_cast<const Tin*>(p.conv_halo[DIR]) + (int64_t)b * 3 * D, D, lane);
         if (gated) {
-            cp_async_wait_all();
+            if (i + 1 < nc)
+                cp_async_wait_pending<1>();  // chunk i's copies; i+1's may still run
+            else
+                cp_async_wait_all();
             __syncwarp();
         }
+        const float* owc = ows + (i & 1) * (T * Ge::CW);
         if constexpr (!BCQ && (G == 1 || F32BC)) {
             __syncwarp();
             fused_convert_bc<T, Tin>(Bt, Ct, bcf, lane, true);
@@ -387,7 +400,7 @@ __device__ __forceinline__ void fused_layer_direction(const FusedMaps& maps, con
                     wsw[(int64_t)tr * D] = y;
                 } else {
                     const float zv = ldf(zt, tr * Ge::CW + lane);
-                    stf(outw, (int64_t)tr * D, (y + ows[tr * Ge::CW + lane]) * silu(zv));
+                    stf(outw, (int64_t)tr * D, (y + owc[tr * Ge::CW + lane]) * silu(zv));
                 }
             }
         }

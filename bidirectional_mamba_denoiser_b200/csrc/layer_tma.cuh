@@ -72,8 +72,8 @@ struct TmaGeo {
     static constexpr int STAGE = XB + 2 * DTB + (BCQ ? align128(BC32) : 2 * BB);  // x, dt, z, B and C
     static constexpr int ED2 = T * CPW * 8;               // per warp: (delta, delta*u)
     static constexpr int EDU = T * CPW * 4;               // per warp: D*u
-    static constexpr int OWS = T * CPW * 4;               // per warp: partner's y
-    static constexpr int WARP_BYTES = ED2 + EDU + OWS;
+    static constexpr int OWS = T * CPW * 4;               // per warp: partner's y of a chunk
+    static constexpr int WARP_BYTES = ED2 + EDU + 2 * OWS;  // partner's y double-buffered
     static constexpr int DIR_BYTES = NS * STAGE + ((DIRECT || BCQ) ? 0 : 2 * BC32);
     static constexpr int WARP_OFF = 2 * DIR_BYTES;
     static constexpr int BAR_OFF = WARP_OFF + 2 * NWD * WARP_BYTES;
@@ -349,6 +349,24 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
     const int gtid = wg * 32 + lane;
     const float scale = p.dir_scale[DIR];
     const int c0w = ct0 + wg * Ge::CPW;  // first channel of this warp
+    // cp.async of the partner's fp32 y of chunk ii into buffer ii & 1, in pieces
+    // of PC = min(4, CPW) channels.  D is a multiple of 4 on this path and c0w
+    // a multiple of PC, so a piece that starts inside a row ends inside it and
+    // is aligned to its size.
+    auto fetch_partner = [&](int ii) {
+        constexpr int PC = Ge::CPW < 4 ? Ge::CPW : 4;
+        constexpr int PIECES = Ge::CPW / PC;
+        const int kk = DIR == 0 ? ii : nc - 1 - ii;
+        const int64_t row = (int64_t)b * L + (int64_t)kk * T;
+        float* dst = ows + (ii & 1) * (T * Ge::CPW);
+        for (int e = lane; e < T * PIECES; e += 32) {
+            const int r = e / PIECES, q = e % PIECES;
+            const bool ok = (int64_t)kk * T + r < L && c0w + PC * q < D;
+            const float* src = p.ws + (row + (ok ? r : 0)) * D + (ok ? c0w + PC * q : 0);
+            cp_async<PC * 4>(dst + r * Ge::CPW + PC * q, src, ok);
+        }
+        cp_async_commit();
+    };
 
     Wk wk;
     wk.setup(p, ct0, wg, lane);
@@ -379,21 +397,11 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         const int s_hi = DIR == 0 ? nvalid : T;
         const int64_t chunk_row = (int64_t)b * L + (int64_t)k * T;  // global row of the chunk's token kT
 
-        // partner's y of this chunk -> shared memory (waited for before the scan),
-        // in pieces of PC = min(4, CPW) channels.  D is a multiple of 4 on this
-        // path and c0w a multiple of PC, so a piece that starts inside a row
-        // ends inside it and is aligned to its size.
-        if (gated) {
-            constexpr int PC = Ge::CPW < 4 ? Ge::CPW : 4;
-            constexpr int PIECES = Ge::CPW / PC;
-            for (int e = lane; e < T * PIECES; e += 32) {
-                const int r = e / PIECES, q = e % PIECES;
-                const bool ok = (int64_t)k * T + r < L && c0w + PC * q < D;
-                const float* src = p.ws + (chunk_row + (ok ? r : 0)) * D + (ok ? c0w + PC * q : 0);
-                cp_async<PC * 4>(ows + r * Ge::CPW + PC * q, src, ok);
-            }
-            cp_async_commit();
-        }
+        // The partner's y of the gated chunks -> shared memory, one chunk ahead
+        // (buffer i & 1), so that the copy of chunk i+1 runs under the scan of
+        // chunk i.  All of it was stored before the meeting barrier.
+        if (i == meet) fetch_partner(i);
+        if (gated && i + 1 < nc) fetch_partner(i + 1);
 
         const int st = i % NS;
         mbar_wait_bounded(full + st, (uint32_t)((i / NS) & 1), p.wait_limit);
@@ -423,8 +431,14 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
         }
 
         wk.template elements<CARRY>(xt, dtt, s_lo, s_hi, ed2, edu);
-        if (gated) cp_async_wait_all();
+        if (gated) {
+            if (i + 1 < nc)
+                cp_async_wait_pending<1>();  // chunk i's copies; i+1's may still run
+            else
+                cp_async_wait_all();
+        }
         __syncwarp();
+        const float* owc = ows + (i & 1) * (T * Ge::CPW);
 
         float* wsw = p.ws + chunk_row * D + wk.d;
         Tout* outw = static_cast<Tout*>(p.out) + chunk_row * D + wk.d;
@@ -439,7 +453,7 @@ __device__ __forceinline__ void layer_direction(const LayerMaps& maps, const KPa
                     wsw[(int64_t)tr * D] = y;
                 } else {
                     const float zv = ldf(zt, tr * Ge::XW + wk.tc);
-                    stf(outw, (int64_t)tr * D, (y + ows[tr * Ge::CPW + wk.c]) * silu(zv));
+                    stf(outw, (int64_t)tr * D, (y + owc[tr * Ge::CPW + wk.c]) * silu(zv));
                 }
             }
         }

@@ -15,15 +15,17 @@
 //   Y1  = M (delta x), M = G o e^{c_t - c_s} [s <= t]   (Q x P, K = Q)
 //                                                        -> TMEM cols [128, 160)
 //   y_t = Y1 + e^{c_t} Y2 + D x_t
-// One CTA = one (head, batch row) in one direction, 128 threads; thread t
-// owns step t of the chunk (TMEM lane t) for the per-step work and state
-// row n = t for the state epilogue.  The per-step work starts from the
-// inputs: the head's 32 xBC channels of step t arrive raw by cp.async into a
+// One CTA = one (head, batch row) in one direction, 256 threads: threads t
+// and t + 128 own step t of the chunk (TMEM lane t) for the per-step work and
+// state row n = t for the state epilogue, each for one half of the 32
+// channels (and of the M row's four 32-column blocks), so that an SM's two
+// CTAs give it 16 warps.  The per-step work starts from the inputs: the
+// head's 32 xBC channels of step t arrive raw by cp.async into a
 // shared-memory ring of 3 + 128 rows (the first three hold the last three
 // steps of the previous chunk, the conv's halo, in step order -- so that the
-// causal forward and the anti-causal reverse conv are the same code), thread
-// t computes the conv + SiLU of its step from rows t..t+3, and its step size
-// softplus(dt + bias) from dt.  The chunk's C and B arrive as fp16 tiles (in
+// causal forward and the anti-causal reverse conv are the same code), the
+// conv + SiLU of step t comes from rows t..t+3, and its step size
+// softplus(dt + bias) from dt (computed by both threads of the step).  The chunk's C and B arrive as fp16 tiles (in
 // the canonical K-major form, rows in step order so that the reverse
 // direction needs no other code; written by m2_prep_kernel<Tin, true>) by
 // bulk copies; the B tile of the next chunk is fetched as soon as the
@@ -51,6 +53,7 @@ constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 8
               kSsdCW = 101744, kSsdCB = 102256, kSsdSmem = 102384;
 constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
 constexpr int kSsdXStride = 40;  // bf16 per xBC row in shared memory (80 B: conflict-free 16-byte accesses)
+constexpr int kSsdThreads = 256;  // threads of a dual-form CTA: two per step of the chunk
 
 // 8 fp32 values -> 8 fp16 in one 16-byte store.
 __device__ __forceinline__ void st_half8(unsigned char* dst, const float* v) {
@@ -95,6 +98,7 @@ template <int DIR, typename Tin, typename Tout, bool CL>
 __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm, const int h, const int b) {
     constexpr int Q = kSQ, P = kM2P;
     static_assert(sizeof(Tin) == 2, "the dual form reads bf16 inputs");
+    static_assert(kSsdThreads == 2 * Q, "two threads per step");
     unsigned char* sC = sm + kSsdC;
     unsigned char* sB = sm + kSsdB;
     unsigned char* sDX = sm + kSsdDX;
@@ -109,7 +113,11 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
     float* sCW = reinterpret_cast<float*>(sm + kSsdCW);  // [4][32]: conv tap j of the head's channel p
     float* sCB = reinterpret_cast<float*>(sm + kSsdCB);    // [32]: conv bias
     int* bigspan = reinterpret_cast<int*>(sm + kSsdTot + 16);  // [4]: block j's decay span exceeds kSsdSpanMax
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int tid = threadIdx.x;
+    const int t = tid & (Q - 1);      // the step (TMEM lane, state row) this thread works on
+    const int hf = tid >> 7;          // which half of the step's 32 channels: 16 hf .. 16 hf + 15
+    const int warp = (tid >> 5) & 3;  // the step block, = the TMEM lane quarter this warp may access
+    const int lane = tid & 31;
     const int64_t L = p.L;
     const int H = p.H, HP = H * P;
     const int nc = (int)((L + Q - 1) / Q);
@@ -125,43 +133,44 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
     const float Dsk = p.Dskip[DIR * H + h];
     const float scale = p.dir_scale[DIR];
 
-    if (t == 0) {
+    if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc<256>(tmem_slot);
-    for (int e = t; e < 8192 / 16; e += 128) reinterpret_cast<uint4*>(sS)[e] = make_uint4(0u, 0u, 0u, 0u);
-    if (t < P) {
-        const int64_t ch = (int64_t)DIR * CH + (int64_t)h * P + t;
+    if (tid < 32) tmem_alloc<256>(tmem_slot);
+    for (int e = tid; e < 8192 / 16; e += kSsdThreads) reinterpret_cast<uint4*>(sS)[e] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < P) {
+        const int64_t ch = (int64_t)DIR * CH + (int64_t)h * P + tid;
         const float4 w = reinterpret_cast<const float4*>(p.conv_w)[ch];
-        sCW[t] = w.x;
-        sCW[32 + t] = w.y;
-        sCW[64 + t] = w.z;
-        sCW[96 + t] = w.w;
-        sCB[t] = p.conv_b ? p.conv_b[ch] : 0.f;
+        sCW[tid] = w.x;
+        sCW[32 + tid] = w.y;
+        sCW[64 + tid] = w.z;
+        sCW[96 + tid] = w.w;
+        sCB[tid] = p.conv_b ? p.conv_b[ch] : 0.f;
     }
-    if (t < 3 * 4)  // the first chunk's halo: zeros (before token 0 forward, past token L-1 in reverse)
-        reinterpret_cast<uint4*>(sX + (t >> 2) * kSsdXStride)[t & 3] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < 3 * 4)  // the first chunk's halo: zeros (before token 0 forward, past token L-1 in reverse)
+        reinterpret_cast<uint4*>(sX + (tid >> 2) * kSsdXStride)[tid & 3] = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const uint32_t ch16 = (uint32_t)(16 * hf);  // this thread's 16 columns of a 32-column block
     {
-        float zero[32];
+        float zero[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) zero[i] = 0.f;
-        tmem_st32(tmem + 192 + lb, zero);  // state row n = t starts at 0
+        for (int i = 0; i < 16; ++i) zero[i] = 0.f;
+        tmem_st16(tmem + 192 + ch16 + lb, zero);  // state row n = t starts at 0
     }
-    if (t == 0 && !p.starve) {
+    if (tid == 0 && !p.starve) {
         mbar_arrive_expect_tx(bars + 0, kTileBytes);
         bulk_g2s(sB, tileb + kTileBytes, kTileBytes, bars + 0);
         mbar_arrive_expect_tx(bars + 1, kTileBytes);
         bulk_g2s(sC, tileb, kTileBytes, bars + 1);
     }
-    // step t of chunk kk: the head's xBC row into row 3 + t of sX (zeros past either end) and
-    // dt into a register, used one chunk later
+    // step t of chunk kk: this half's 16 xBC channels of the head into row 3 + t of sX (zeros past
+    // either end) and dt into a register, used one chunk later
     float dt_next = 0.f;
     bool ok_next = false;
     auto fetch_step = [&](int kk) {
@@ -169,7 +178,10 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         const bool ok = tk >= 0 && tk < L;
         const Tin* src = Xr + (ok ? tk : 0) * CH;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cp_async<16>(sX + (3 + t) * kSsdXStride + 8 * i, src + 8 * i, ok);
+        for (int ii = 0; ii < 2; ++ii) {
+            const int i = 2 * hf + ii;
+            cp_async<16>(sX + (3 + t) * kSsdXStride + 8 * i, src + 8 * i, ok);
+        }
         cp_async_commit();
         dt_next = ok ? ldf(DTr, tk * H) : 0.f;
         ok_next = ok;
@@ -186,24 +198,21 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         const uint32_t ph = (uint32_t)(k & 1);
         const bool gated = CL ? k >= meetk : DIR == 1;
         if (CL && k == meetk) cluster_meet();
-        // ---- step t of chunk k: x and delta
-        float x[32];
-        // a gated chunk's partner y and z in the row-contiguous mapping of the output stores:
-        // row 32 warp + 4 i + lane / 8, channels 4 (lane % 8) .. + 3
-        float4 yfc[8];
-        uint2 zc[8];
-        uint32_t sraw[32];
-        tmem_ld32_async(tmem + 192 + lb, sraw);  // carried state row n = t; waited for after the scan
+        // ---- step t of chunk k: x (this half's 16 channels) and delta
+        float x[16];
+        uint32_t sraw[16];
+        tmem_ld16_async(tmem + 192 + ch16 + lb, sraw);  // carried state row n = t; waited for after the scan
         const float dtk = dt_next;
         const bool okk = ok_next;
         // the next chunk's tiles into L2 a chunk ahead of their copies into shared memory
-        if (t == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
+        if (tid == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
         cp_async_wait_all();
         __syncthreads();  // every xBC row of the chunk is in shared memory
         // conv + SiLU of step t: rows t..t+3 hold steps t-3..t, and tap j multiplies step t-3+j in
         // both directions (the reverse scan's steps run backwards in time)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // channels 8i .. 8i+7, in pairs
+        for (int ii = 0; ii < 2; ++ii) {  // channels 8i .. 8i+7, in pairs
+            const int i = 2 * hf + ii;
             float2 acc[4];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -226,29 +235,31 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                x[8 * i + 2 * u] = silu(acc[u].x);
-                x[8 * i + 2 * u + 1] = silu(acc[u].y);
+                x[8 * ii + 2 * u] = silu(acc[u].x);
+                x[8 * ii + 2 * u + 1] = silu(acc[u].y);
             }
         }
         const float dl = okk ? softplus(dtk + bias) : 0.f;
-        // ---- c_t: inclusive scan of delta A (log2 units) over the chunk
+        // ---- c_t: inclusive scan of delta A (log2 units) over the chunk (both halves alike)
         float a = dl * A2;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const float v = __shfl_up_sync(0xffffffffu, a, off);
             if (lane >= off) a += v;
         }
-        if (lane == 31) wtot[warp] = a;
+        if (lane == 31 && hf == 0) wtot[warp] = a;
         __syncthreads();
         if (t >= Q - 3) {  // the conv has read every row: the last three steps become the next halo
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int ii = 0; ii < 2; ++ii) {
+                const int i = 2 * hf + ii;
                 reinterpret_cast<uint4*>(sX + (t + 3 - Q) * kSsdXStride)[i] =
                     reinterpret_cast<const uint4*>(sX + (t + 3) * kSsdXStride)[i];
+            }
         }
         // ---- G = C B^T and Y2 = C S_^T need only the tiles and the state of the previous
         // chunk: they run on the tensor cores while the steps below are computed
-        if (t == 0) {
+        if (tid == 0) {
             mbar_wait_bounded(bars + 0, ph, p.wait_limit);
             mbar_wait_bounded(bars + 1, ph, p.wait_limit);
             tmem_fence_after_sync();
@@ -266,57 +277,45 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         for (int w = 0; w < warp; ++w) base += wtot[w];
         const float c = a + base;
         const float cend = wtot[0] + wtot[1] + wtot[2] + wtot[3];
-        c2s[t] = c;
         {
             // block j = warp: step s's factor 2^(c_{32j} - c_s) >= 1, usable while the span is small
             const float cref = __shfl_sync(0xffffffffu, c, 0);
-            sE[t] = ex2_approx(fminf(cref - c, kSsdSpanMax));
             const float span = cref - __shfl_sync(0xffffffffu, c, 31);
-            if (lane == 0) bigspan[warp] = span > kSsdSpanMax ? 1 : 0;
+            if (hf == 0) {
+                c2s[t] = c;
+                sE[t] = ex2_approx(fminf(cref - c, kSsdSpanMax));
+                if (lane == 0) bigspan[warp] = span > kSsdSpanMax ? 1 : 0;
+            }
         }
-        // ---- delta x and W rows of step t (MN-major [s][p])
+        // ---- delta x and W rows of step t (MN-major [s][p]), this half's channels
         {
             const float wdec = ex2_approx(cend - c);
-            float dx[32];
+            float dx[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) dx[i] = dl * x[i];
+            for (int i = 0; i < 16; ++i) dx[i] = dl * x[i];
 #pragma unroll
-            for (int pg = 0; pg < 4; ++pg) st_half8(sDX + f16_mnmajor(8 * pg, t, P), dx + 8 * pg);
+            for (int pg = 0; pg < 2; ++pg) st_half8(sDX + f16_mnmajor(16 * hf + 8 * pg, t, P), dx + 8 * pg);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) dx[i] *= wdec;
+            for (int i = 0; i < 16; ++i) dx[i] *= wdec;
 #pragma unroll
-            for (int pg = 0; pg < 4; ++pg) st_half8(sW + f16_mnmajor(8 * pg, t, P), dx + 8 * pg);
+            for (int pg = 0; pg < 2; ++pg) st_half8(sW + f16_mnmajor(16 * hf + 8 * pg, t, P), dx + 8 * pg);
         }
         if (k + 1 < nc) fetch_step(k + 1);  // the conv and the halo copy are done with this chunk's rows
-        // ---- carried state row n = t decays over the whole chunk
+        // ---- carried state row n = t (this half's columns) decays over the whole chunk
         {
             tmem_wait_ld(sraw);
-            float s[32];
+            float s[16];
             const float f = ex2_approx(cend);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(sraw[i]) * f;
-            tmem_st32(tmem + 192 + lb, s);
-        }
-        if (gated) {  // in flight while the products run
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 32 * warp + 4 * i + (lane >> 3);
-                const int64_t tk = DIR == 0 ? (int64_t)k * Q + r : (int64_t)(nc - k) * Q - 1 - r;
-                yfc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                zc[i] = make_uint2(0u, 0u);
-                if (tk >= 0 && tk < L) {
-                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
-                    yfc[i] = *reinterpret_cast<const float4*>(partner_y + o);
-                    zc[i] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
-                }
-            }
+            for (int i = 0; i < 16; ++i) s[i] = __uint_as_float(sraw[i]) * f;
+            tmem_st16(tmem + 192 + ch16 + lb, s);
         }
         fence_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
         tmem_fence_after_sync();
         // ---- S^T += B^T W (onto the decayed state)
-        if (t == 0) {
+        if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 umma_f16(tmem + 192, umma_desc(aB + ks * 4096, 2048, 128), umma_desc(aW + ks * 1024, 512, 128),
@@ -324,115 +323,131 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             umma_commit(bars + 4);
         }
         mbar_wait_bounded(bars + 2, ph, p.wait_limit);
+        tmem_fence_after_sync();
+        // ---- M row t (into C's buffer, K-major [t][s]): this half's column blocks jb = hf, hf + 2.
+        // Columns s >= 32 jb reach step t = 32 warp + lane only for jb <= warp;
+        // e^(c_t - c_s) = 2^(c_t - c_{32jb}) 2^(c_{32jb} - c_s) while block jb's span is small
+#pragma unroll 1
+        for (int jj = 0; jj < 2; ++jj) {
+            const int jb = hf + 2 * jj;
+            uint32_t gr[32];
+            if (jb <= warp) tmem_ld32_async(tmem + 32 * jb + lb, gr);
+            tmem_wait_ld(gr);
+            float m[32];
+            if (jb <= warp) {
+                const float cref = c2s[32 * jb];
+                if (!bigspan[jb]) {
+                    const float F = ex2_approx(c - cref);
+                    const float2 FF = make_float2(F, F);
+                    const float4* e4 = reinterpret_cast<const float4*>(sE + 32 * jb);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 ev = e4[i / 4];
+                        const float2 m01 = mul2(make_float2(__uint_as_float(gr[i]), __uint_as_float(gr[i + 1])),
+                                                mul2(FF, make_float2(ev.x, ev.y)));
+                        const float2 m23 = mul2(make_float2(__uint_as_float(gr[i + 2]), __uint_as_float(gr[i + 3])),
+                                                mul2(FF, make_float2(ev.z, ev.w)));
+                        m[i] = m01.x; m[i + 1] = m01.y; m[i + 2] = m23.x; m[i + 3] = m23.y;
+                    }
+                    if (jb == warp) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i > lane) m[i] = 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = 32 * jb + i;
+                        m[i] = s <= t ? __uint_as_float(gr[i]) * ex2_approx(c - c2s[s]) : 0.f;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) m[i] = 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) st_half8(sC + f16_kmajor(t, 32 * jb + 8 * q, Q), m + 8 * q);
+        }
+        // ---- the new state row n = t (this half's columns) as the fp16 operand of the next C S_^T
         mbar_wait_bounded(bars + 4, ph, p.wait_limit);
         tmem_fence_after_sync();
-        if (t == 0 && k + 1 < nc && !p.starve) {  // B's buffer is free: next chunk's B tile
+        if (tid == 0 && k + 1 < nc && !p.starve) {  // B's buffer is free: next chunk's B tile
             mbar_arrive_expect_tx(bars + 0, kTileBytes);
             bulk_g2s(sB, tileb + (int64_t)(k + 1) * 2 * kTileBytes + kTileBytes, kTileBytes, bars + 0);
         }
-        // ---- M row t (into C's buffer, K-major [t][s]) and the new state row n = t
-        // columns s >= 32j reach step t = 32 warp + lane only for j <= warp;
-        // e^(c_t - c_s) = 2^(c_t - c_{32j}) 2^(c_{32j} - c_s) while block j's span is small
         {
-            uint32_t sn[32];
-            tmem_ld32_async(tmem + 192 + lb, sn);
-#pragma unroll 1
-            for (int j = 0; j < 4; j += 2) {
-                uint32_t g0[32], g1[32];
-                if (j <= warp) tmem_ld32_async(tmem + 32 * j + lb, g0);
-                if (j + 1 <= warp) tmem_ld32_async(tmem + 32 * (j + 1) + lb, g1);
-                tmem_wait_ld(g0);
-                tmem_wait_ld(g1);
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int jb = j + jj;
-                    uint32_t (&gr)[32] = jj == 0 ? g0 : g1;
-                    float m[32];
-                    if (jb <= warp) {
-                        const float cref = c2s[32 * jb];
-                        if (!bigspan[jb]) {
-                            const float F = ex2_approx(c - cref);
-                            const float2 FF = make_float2(F, F);
-                            const float4* e4 = reinterpret_cast<const float4*>(sE + 32 * jb);
-#pragma unroll
-                            for (int i = 0; i < 32; i += 4) {
-                                const float4 ev = e4[i / 4];
-                                const float2 m01 = mul2(make_float2(__uint_as_float(gr[i]), __uint_as_float(gr[i + 1])),
-                                                        mul2(FF, make_float2(ev.x, ev.y)));
-                                const float2 m23 = mul2(make_float2(__uint_as_float(gr[i + 2]), __uint_as_float(gr[i + 3])),
-                                                        mul2(FF, make_float2(ev.z, ev.w)));
-                                m[i] = m01.x; m[i + 1] = m01.y; m[i + 2] = m23.x; m[i + 3] = m23.y;
-                            }
-                            if (jb == warp) {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    if (i > lane) m[i] = 0.f;
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const int s = 32 * jb + i;
-                                m[i] = s <= t ? __uint_as_float(gr[i]) * ex2_approx(c - c2s[s]) : 0.f;
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) m[i] = 0.f;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) st_half8(sC + f16_kmajor(t, 32 * jb + 8 * q, Q), m + 8 * q);
-                }
-            }
+            uint32_t sn[16];
+            tmem_ld16_async(tmem + 192 + ch16 + lb, sn);
             tmem_wait_ld(sn);
-            float sv[32];
+            float sv[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(sn[i]);
+            for (int i = 0; i < 16; ++i) sv[i] = __uint_as_float(sn[i]);
 #pragma unroll
-            for (int pg = 0; pg < 4; ++pg) st_half8(sS + f16_mnmajor(8 * pg, t, P), sv + 8 * pg);
+            for (int pg = 0; pg < 2; ++pg) st_half8(sS + f16_mnmajor(16 * hf + 8 * pg, t, P), sv + 8 * pg);
         }
         fence_async_smem();
         tmem_fence_before_sync();
         __syncthreads();
         tmem_fence_after_sync();
         // ---- Y1 = M (delta x)
-        if (t == 0) {
+        if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 umma_f16(tmem + 128, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aDX + ks * 1024, 512, 128), ID_Y,
                          ks > 0);
             umma_commit(bars + 3);
         }
+        // a gated chunk's partner y and z, in flight while Y1 runs, in the row-contiguous mapping
+        // of the output stores: row 32 warp + 4 i + lane / 8 (i = 4 hf .. 4 hf + 3), channels
+        // 4 (lane % 8) .. + 3
+        float4 yfc[4];
+        uint2 zc[4];
+        if (gated) {
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int r = 32 * warp + 4 * (4 * hf + ii) + (lane >> 3);
+                const int64_t tk = DIR == 0 ? (int64_t)k * Q + r : (int64_t)(nc - k) * Q - 1 - r;
+                yfc[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
+                zc[ii] = make_uint2(0u, 0u);
+                if (tk >= 0 && tk < L) {
+                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
+                    yfc[ii] = *reinterpret_cast<const float4*>(partner_y + o);
+                    zc[ii] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
+                }
+            }
+        }
         mbar_wait_bounded(bars + 3, ph, p.wait_limit);
         tmem_fence_after_sync();
-        if (t == 0 && k + 1 < nc && !p.starve) {  // C's buffer is free: next chunk's C tile
+        if (tid == 0 && k + 1 < nc && !p.starve) {  // C's buffer is free: next chunk's C tile
             mbar_arrive_expect_tx(bars + 1, kTileBytes);
             bulk_g2s(sC, tileb + (int64_t)(k + 1) * 2 * kTileBytes, kTileBytes, bars + 1);
         }
-        // ---- output of step t: the row goes through this warp's 32-row staging block (the
-        // delta x / W buffers, free once Y1 is done; 16-byte chunks XOR-swizzled by row) and is
-        // stored row-contiguously, four whole 128-byte rows per warp instruction
+        // ---- output of step t: the two halves of each row go through the row block's 32-row
+        // staging block (the delta x / W buffers, free once Y1 is done; 16-byte chunks
+        // XOR-swizzled by row) and are stored row-contiguously, four whole 128-byte rows per warp
+        // instruction
         {
-            uint32_t r1[32], r2[32];
-            tmem_ld32_async(tmem + 128 + lb, r1);
-            tmem_ld32_async(tmem + 160 + lb, r2);
+            uint32_t r1[16], r2[16];
+            tmem_ld16_async(tmem + 128 + ch16 + lb, r1);
+            tmem_ld16_async(tmem + 160 + ch16 + lb, r2);
             tmem_wait_ld(r1);
             tmem_wait_ld(r2);
             const float e = ex2_approx(c);
             float4* stg = reinterpret_cast<float4*>(sDX) + warp * 256;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 float4 v;
                 v.x = (__uint_as_float(r1[4 * q]) + e * __uint_as_float(r2[4 * q]) + Dsk * x[4 * q]) * scale;
                 v.y = (__uint_as_float(r1[4 * q + 1]) + e * __uint_as_float(r2[4 * q + 1]) + Dsk * x[4 * q + 1]) * scale;
                 v.z = (__uint_as_float(r1[4 * q + 2]) + e * __uint_as_float(r2[4 * q + 2]) + Dsk * x[4 * q + 2]) * scale;
                 v.w = (__uint_as_float(r1[4 * q + 3]) + e * __uint_as_float(r2[4 * q + 3]) + Dsk * x[4 * q + 3]) * scale;
-                stg[lane * 8 + (q ^ (lane & 7))] = v;
+                stg[lane * 8 + ((4 * hf + q) ^ (lane & 7))] = v;
             }
-            __syncwarp();
+            named_bar_sync(1 + warp, 64);  // the row block's two warps (warp, warp + 4) wrote its staging block
             const int cq = lane & 7;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 4 * i + (lane >> 3);
+            for (int ii = 0; ii < 4; ++ii) {
+                const int r = 4 * (4 * hf + ii) + (lane >> 3);
                 const float4 v = stg[r * 8 + (cq ^ (r & 7))];
                 const int step = 32 * warp + r;
                 const int64_t tk = DIR == 0 ? (int64_t)k * Q + step : (int64_t)(nc - k) * Q - 1 - step;
@@ -442,13 +457,13 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
                         *reinterpret_cast<float4*>(own_y + o) = v;
                     } else {
                         // bf16 -> fp32 is exact: the bf16 bits are the high half
-                        const float z0 = __uint_as_float(zc[i].x << 16), z1 = __uint_as_float(zc[i].x & 0xffff0000u);
-                        const float z2 = __uint_as_float(zc[i].y << 16), z3 = __uint_as_float(zc[i].y & 0xffff0000u);
+                        const float z0 = __uint_as_float(zc[ii].x << 16), z1 = __uint_as_float(zc[ii].x & 0xffff0000u);
+                        const float z2 = __uint_as_float(zc[ii].y << 16), z3 = __uint_as_float(zc[ii].y & 0xffff0000u);
                         float ov[4];
-                        ov[0] = (yfc[i].x + v.x) * silu(z0);
-                        ov[1] = (yfc[i].y + v.y) * silu(z1);
-                        ov[2] = (yfc[i].z + v.z) * silu(z2);
-                        ov[3] = (yfc[i].w + v.w) * silu(z3);
+                        ov[0] = (yfc[ii].x + v.x) * silu(z0);
+                        ov[1] = (yfc[ii].y + v.y) * silu(z1);
+                        ov[2] = (yfc[ii].z + v.z) * silu(z2);
+                        ov[3] = (yfc[ii].w + v.w) * silu(z3);
                         store4(static_cast<Tout*>(p.out) + o, ov);
                     }
                 }
@@ -461,14 +476,14 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
     if (CL && meetk >= nc) cluster_meet();  // a one-chunk sequence: the reverse CTA meets after its chunk
     tmem_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc<256>(tmem);
+    if (tid < 32) tmem_dealloc<256>(tmem);
 }
 
 // grid (2 H, batch) in clusters of 2: CTA 2h runs head h forward, CTA 2h+1 in
 // reverse; block 128, dynamic shared memory kSsdSmem.  For calls whose
 // per-direction grid leaves SMs idle: both directions run at once.
 template <typename Tin, typename Tout>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 2) m2_ssd_cluster_kernel(const M2Params p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSsdThreads, 2) m2_ssd_cluster_kernel(const M2Params p) {
     extern __shared__ __align__(128) unsigned char sm[];
     if (blockIdx.x & 1)
         m2_ssd_dir<1, Tin, Tout, true>(p, sm, (int)(blockIdx.x >> 1), (int)blockIdx.y);
@@ -501,7 +516,7 @@ __device__ __forceinline__ int m2_flag_acquire(const int* f) {
 }
 
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(128, 2) m2_ssd_ticket_kernel(const M2Params p) {
+__global__ void __launch_bounds__(kSsdThreads, 2) m2_ssd_ticket_kernel(const M2Params p) {
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int ticket;
     if (threadIdx.x == 0) ticket = atomicAdd(p.sync, 1);
