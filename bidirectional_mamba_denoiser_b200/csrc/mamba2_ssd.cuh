@@ -192,6 +192,9 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
     constexpr uint32_t ID_G = umma_idesc_f16(128, 128, false, false);
     constexpr uint32_t ID_Y = umma_idesc_f16(128, 32, false, true);
     constexpr uint32_t ID_S = umma_idesc_f16(128, 32, true, true);
+    // The operands' descriptors at K step 0 (C and M K-major; B K-major for G and MN-major for
+    // the state update; the state, delta x and W MN-major), formed where the MMAs are issued:
+    // each chain of eight MMAs advances them.
 
 #pragma unroll 1
     for (int k = 0; k < nc; ++k) {
@@ -263,14 +266,9 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             mbar_wait_bounded(bars + 0, ph, p.wait_limit);
             mbar_wait_bounded(bars + 1, ph, p.wait_limit);
             tmem_fence_after_sync();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 0, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aB + ks * 256, 128, 2048), ID_G,
-                         ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 160, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aS + ks * 1024, 512, 128), ID_Y,
-                         ks > 0);
+            umma_f16_k8<256 / 16, 256 / 16>(tmem + 0, umma_desc(aC, 128, 2048), umma_desc(aB, 128, 2048), ID_G, false);
+            umma_f16_k8<256 / 16, 1024 / 16>(tmem + 160, umma_desc(aC, 128, 2048), umma_desc(aS, 512, 128), ID_Y,
+                                             false);
             umma_commit(bars + 2);
         }
         float base = 0.f;
@@ -316,10 +314,8 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         tmem_fence_after_sync();
         // ---- S^T += B^T W (onto the decayed state)
         if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 192, umma_desc(aB + ks * 4096, 2048, 128), umma_desc(aW + ks * 1024, 512, 128),
-                         ID_S, true);
+            umma_f16_k8<4096 / 16, 1024 / 16>(tmem + 192, umma_desc(aB, 2048, 128), umma_desc(aW, 512, 128), ID_S,
+                                              true);
             umma_commit(bars + 4);
         }
         mbar_wait_bounded(bars + 2, ph, p.wait_limit);
@@ -391,10 +387,8 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         tmem_fence_after_sync();
         // ---- Y1 = M (delta x)
         if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma_f16(tmem + 128, umma_desc(aC + ks * 256, 128, 2048), umma_desc(aDX + ks * 1024, 512, 128), ID_Y,
-                         ks > 0);
+            umma_f16_k8<256 / 16, 1024 / 16>(tmem + 128, umma_desc(aC, 128, 2048), umma_desc(aDX, 512, 128), ID_Y,
+                                             false);
             umma_commit(bars + 3);
         }
         // a gated chunk's partner y and z, in flight while Y1 runs, in the row-contiguous mapping

@@ -72,6 +72,37 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t 
         "l"(da), "l"(db), "r"(idesc), "r"(accumulate ? 1u : 0u));
 }
 
+// Eight MMAs accumulating along K in one asm block: operand descriptors da,
+// db for the first K step, advanced by the immediates A_STEP and B_STEP
+// (descriptor units: 16 bytes of start address) per step; the first MMA
+// accumulates onto D only if `accumulate`.  Each MMA then costs one
+// instruction plus two 64-bit adds in the issuing thread, which matters when
+// that thread shares its SM's schedulers with many busy warps.
+template <int A_STEP, int B_STEP>
+__device__ __forceinline__ void umma_f16_k8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+        "add.s64 a, a, %6;\n\tadd.s64 b, b, %7;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(1u), "n"(A_STEP), "n"(B_STEP));
+}
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
