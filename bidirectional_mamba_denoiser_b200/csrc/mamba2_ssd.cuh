@@ -299,6 +299,25 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             for (int pg = 0; pg < 2; ++pg) st_half8(sW + f16_mnmajor(16 * hf + 8 * pg, t, P), dx + 8 * pg);
         }
         if (k + 1 < nc) fetch_step(k + 1);  // the conv and the halo copy are done with this chunk's rows
+        // a gated chunk's partner y and z, in flight while the products run, in the row-contiguous mapping
+        // of the output stores: row 32 warp + 4 i + lane / 8 (i = 4 hf .. 4 hf + 3), channels
+        // 4 (lane % 8) .. + 3
+        float4 yfc[4];
+        uint2 zc[4];
+        if (gated) {
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int r = 32 * warp + 4 * (4 * hf + ii) + (lane >> 3);
+                const int64_t tk = DIR == 0 ? (int64_t)k * Q + r : (int64_t)(nc - k) * Q - 1 - r;
+                yfc[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
+                zc[ii] = make_uint2(0u, 0u);
+                if (tk >= 0 && tk < L) {
+                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
+                    yfc[ii] = *reinterpret_cast<const float4*>(partner_y + o);
+                    zc[ii] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
+                }
+            }
+        }
         // ---- carried state row n = t (this half's columns) decays over the whole chunk
         {
             tmem_wait_ld(sraw);
@@ -390,25 +409,6 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             umma_f16_k8<256 / 16, 1024 / 16>(tmem + 128, umma_desc(aC, 128, 2048), umma_desc(aDX, 512, 128), ID_Y,
                                              false);
             umma_commit(bars + 3);
-        }
-        // a gated chunk's partner y and z, in flight while Y1 runs, in the row-contiguous mapping
-        // of the output stores: row 32 warp + 4 i + lane / 8 (i = 4 hf .. 4 hf + 3), channels
-        // 4 (lane % 8) .. + 3
-        float4 yfc[4];
-        uint2 zc[4];
-        if (gated) {
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int r = 32 * warp + 4 * (4 * hf + ii) + (lane >> 3);
-                const int64_t tk = DIR == 0 ? (int64_t)k * Q + r : (int64_t)(nc - k) * Q - 1 - r;
-                yfc[ii] = make_float4(0.f, 0.f, 0.f, 0.f);
-                zc[ii] = make_uint2(0u, 0u);
-                if (tk >= 0 && tk < L) {
-                    const int64_t o = ((int64_t)b * L + tk) * HP + (int64_t)h * P + 4 * (lane & 7);
-                    yfc[ii] = *reinterpret_cast<const float4*>(partner_y + o);
-                    zc[ii] = *reinterpret_cast<const uint2*>(static_cast<const Tin*>(p.z) + o);
-                }
-            }
         }
         mbar_wait_bounded(bars + 3, ph, p.wait_limit);
         tmem_fence_after_sync();
