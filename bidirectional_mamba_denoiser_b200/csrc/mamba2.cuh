@@ -126,10 +126,14 @@ constexpr int kM2Chunk = 128;  // steps per chunk of the tensor-core path
 // every channel to V (fp32) and the step sizes to DL.  TILES = true
 // (tensor-core path, whose scan kernel computes the x channels and step
 // sizes itself): grid (ceil(L / 32), 1, 2 * batch), block 128 = 4 token
-// groups x the 32 threads of the B and C channels, written as fp16 rows of
-// the chunk tiles at the token's step (forward: token t is step t; reverse:
-// step nc*128-1-t, the chunks of both directions covering the same tokens),
-// in the canonical K-major layout.
+// groups x the 32 threads of the B and C channels, written in fp16 into the
+// chunk tiles at the token's step (forward: token t is step t; reverse: step
+// nc*128-1-t, the chunks of both directions covering the same tokens).  C is
+// K-major [step][n] (a 16-byte row of 8 channels per token); B is MN-major
+// with the 8-n groups adjacent (f16_mn_kfast(step, n): a 16-byte run of 8
+// steps per channel, stored once per 8-token group), the layout in which the
+// scan kernel appends the state's fp16 copy to make one operand of G and
+// C S^T.
 template <typename Tin, bool TILES>
 __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     constexpr int TT = kM2PrepT;
@@ -166,6 +170,15 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
             else
                 xw[k].zero();
         }
+        // TILES, B channels: the group's 8 steps of each of the thread's 8 channels, as fp16
+        // pairs (a token's step within the group is k forward, 7 - k in reverse)
+        uint32_t hb[8][4];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) hb[q][u] = 0u;
+        const int HPc = H * kM2P;
+        const bool isB = TILES && c0 < HPc + kM2N;
 #pragma unroll
         for (int k = 0; k < TT; ++k) {
             const int64_t t = t0 + k;
@@ -184,21 +197,41 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
                 float4* dst = reinterpret_cast<float4*>(V + t * CH);
                 dst[0] = make_float4(v[0], v[1], v[2], v[3]);
                 dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else if (isB) {
+                // fp16 bits of v[q] into half (step within the group) of hb[q]
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t hv = (uint32_t)__half_as_ushort(__float2half_rn(v[q]));
+                    if (r == 0) {
+                        hb[q][k >> 1] |= (k & 1) ? hv << 16 : hv;
+                    } else {
+                        hb[q][(TT - 1 - k) >> 1] |= ((TT - 1 - k) & 1) ? hv << 16 : hv;
+                    }
+                }
             } else {
                 const __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
                 const __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
                 const uint4 q = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
                                            *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
-                const int HP = H * kM2P;
-                const bool isB = c0 < HP + kM2N;
-                const int n0 = c0 - HP - (isB ? 0 : kM2N);
+                const int n0 = c0 - HPc - kM2N;
                 const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
                 const int64_t step = r == 0 ? t : nc * kM2Chunk - 1 - t;  // chunks aligned in token space
                 unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + step / kM2Chunk) *
                                                  (2 * kM2Chunk * kM2N * 2);
-                *reinterpret_cast<uint4*>(T + (isB ? kM2Chunk * kM2N * 2 : 0) +
-                                          f16_kmajor((int)(step % kM2Chunk), n0, kM2N)) = q;
+                *reinterpret_cast<uint4*>(T + f16_kmajor((int)(step % kM2Chunk), n0, kM2N)) = q;
             }
+        }
+        if (isB && t0 < L) {  // the group's 8 steps of each channel: one 16-byte run per channel
+            static_assert(TT == 8, "one 8-step group per thread");
+            const int n0 = c0 - HPc;
+            const int64_t nc = (L + kM2Chunk - 1) / kM2Chunk;
+            const int64_t s0 = r == 0 ? t0 : nc * kM2Chunk - TT - t0;  // the group's first step
+            unsigned char* T = p.tiles + (((int64_t)r * p.batch + b) * nc + s0 / kM2Chunk) * (2 * kM2Chunk * kM2N * 2) +
+                               kM2Chunk * kM2N * 2;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4*>(T + f16_mn_kfast((int)(s0 % kM2Chunk), n0 + q, kM2N)) =
+                    make_uint4(hb[q][0], hb[q][1], hb[q][2], hb[q][3]);
         }
     }
     if (!TILES && blockIdx.y == 0) {

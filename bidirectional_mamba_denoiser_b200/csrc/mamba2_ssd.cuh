@@ -9,11 +9,12 @@
 // (the same recurrence as the step-by-step scan, summed in closed form; the
 // state-space-dual view of Mamba-2 the pages cite).  Four matrix products:
 //   G   = C B^T                     (Q x Q, K = N)      -> TMEM cols [0, 128)
-//   Y2  = C S_^T                    (Q x P, K = N)      -> TMEM cols [160, 192)
+//   Y2  = C S_^T                    (Q x P, K = N)      -> TMEM cols [128, 160)
+//         (one product: C times the B tile with the state's fp16 copy appended)
 //   S^T = e^{c_end} S_^T + B^T W    (N x P, K = Q), W_s = e^{c_end - c_s} delta_s x_s
 //                                                        -> TMEM cols [192, 224)
 //   Y1  = M (delta x), M = G o e^{c_t - c_s} [s <= t]   (Q x P, K = Q)
-//                                                        -> TMEM cols [128, 160)
+//                                                        -> TMEM cols [160, 192)
 //   y_t = Y1 + e^{c_t} Y2 + D x_t
 // One CTA = one (head, batch row) in one direction, 256 threads: threads t
 // and t + 128 own step t of the chunk (TMEM lane t) for the per-step work and
@@ -25,10 +26,13 @@
 // steps of the previous chunk, the conv's halo, in step order -- so that the
 // causal forward and the anti-causal reverse conv are the same code), the
 // conv + SiLU of step t comes from rows t..t+3, and its step size
-// softplus(dt + bias) from dt (computed by both threads of the step).  The chunk's C and B arrive as fp16 tiles (in
-// the canonical K-major form, rows in step order so that the reverse
-// direction needs no other code; written by m2_prep_kernel<Tin, true>) by
-// bulk copies; the B tile of the next chunk is fetched as soon as the
+// softplus(dt + bias) from dt (computed by both threads of the step).  The
+// chunk's C and B arrive as fp16 tiles by bulk copies (written by
+// m2_prep_kernel<Tin, true>, in step order so that the reverse direction needs
+// no other code): C K-major [step][n]; B MN-major with its 8-n groups
+// adjacent, followed in shared memory by the carried state's fp16 copy in the
+// same layout, so that G and C S_^T are one product of N = 160.  The B tile
+// of the next chunk is fetched as soon as the
 // products that read B are done, the C tile once M (which reuses C's
 // buffer) has been consumed, and the next chunk's xBC rows and step sizes
 // once this chunk's conv has read them.  Every mbarrier wait is bounded.
@@ -48,7 +52,7 @@ namespace bimamba {
 constexpr int kSQ = kM2Chunk;               // steps per chunk (= MMA M)
 constexpr int kTileBytes = kSQ * kM2N * 2;  // one fp16 C or B tile
 // shared memory of one dual-form CTA (either kernel)
-constexpr int kSsdC = 0, kSsdB = 32768, kSsdDX = 65536, kSsdW = 73728, kSsdS = 81920, kSsdC2 = 90112,
+constexpr int kSsdC = 0, kSsdB = 32768, kSsdS = 65536, kSsdDX = 73728, kSsdW = 81920, kSsdC2 = 90112,
               kSsdTot = 90624, kSsdBar = 90688, kSsdTmem = 90728, kSsdX = 90752, kSsdE = 101232,
               kSsdCW = 101744, kSsdCB = 102256, kSsdSmem = 102384;
 constexpr float kSsdSpanMax = 100.f;  // largest log2 decay span of a 32-step block taken in factored form
@@ -187,11 +191,13 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         ok_next = ok;
     };
     fetch_step(0);
-    const uint32_t aC = smem_addr(sC), aB = smem_addr(sB), aDX = smem_addr(sDX), aW = smem_addr(sW),
-                   aS = smem_addr(sS);
-    constexpr uint32_t ID_G = umma_idesc_f16(128, 128, false, false);
+    const uint32_t aC = smem_addr(sC), aB = smem_addr(sB), aDX = smem_addr(sDX), aW = smem_addr(sW);
+    // [G | Y2] = C [B ; S_]^T: the B tile and the state's fp16 copy right after it form one
+    // MN-major operand of 160 rows (f16_mn_kfast layout, 8-MN groups 2048 bytes apart)
+    constexpr uint32_t ID_GY = umma_idesc_f16(128, 160, false, true);
     constexpr uint32_t ID_Y = umma_idesc_f16(128, 32, false, true);
-    constexpr uint32_t ID_S = umma_idesc_f16(128, 32, true, true);
+    // S^T += B^T W: the same B tile read K-major (rows = states n, K = steps s)
+    constexpr uint32_t ID_S = umma_idesc_f16(128, 32, false, true);
     // The operands' descriptors at K step 0 (C and M K-major; B K-major for G and MN-major for
     // the state update; the state, delta x and W MN-major), formed where the MMAs are issued:
     // each chain of eight MMAs advances them.
@@ -266,9 +272,8 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             mbar_wait_bounded(bars + 0, ph, p.wait_limit);
             mbar_wait_bounded(bars + 1, ph, p.wait_limit);
             tmem_fence_after_sync();
-            umma_f16_k8<256 / 16, 256 / 16>(tmem + 0, umma_desc(aC, 128, 2048), umma_desc(aB, 128, 2048), ID_G, false);
-            umma_f16_k8<256 / 16, 1024 / 16>(tmem + 160, umma_desc(aC, 128, 2048), umma_desc(aS, 512, 128), ID_Y,
-                                             false);
+            umma_f16_k8<256 / 16, 256 / 16>(tmem + 0, umma_desc(aC, 128, 2048), umma_desc(aB, 128, 2048), ID_GY,
+                                            false);
             umma_commit(bars + 2);
         }
         float base = 0.f;
@@ -398,7 +403,7 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
 #pragma unroll
             for (int i = 0; i < 16; ++i) sv[i] = __uint_as_float(sn[i]);
 #pragma unroll
-            for (int pg = 0; pg < 2; ++pg) st_half8(sS + f16_mnmajor(16 * hf + 8 * pg, t, P), sv + 8 * pg);
+            for (int pg = 0; pg < 2; ++pg) st_half8(sS + f16_mn_kfast(16 * hf + 8 * pg, t, kM2N), sv + 8 * pg);
         }
         fence_async_smem();
         tmem_fence_before_sync();
@@ -406,7 +411,7 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         tmem_fence_after_sync();
         // ---- Y1 = M (delta x)
         if (tid == 0) {
-            umma_f16_k8<256 / 16, 1024 / 16>(tmem + 128, umma_desc(aC, 128, 2048), umma_desc(aDX, 512, 128), ID_Y,
+            umma_f16_k8<256 / 16, 1024 / 16>(tmem + 160, umma_desc(aC, 128, 2048), umma_desc(aDX, 512, 128), ID_Y,
                                              false);
             umma_commit(bars + 3);
         }
@@ -422,8 +427,8 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         // instruction
         {
             uint32_t r1[16], r2[16];
-            tmem_ld16_async(tmem + 128 + ch16 + lb, r1);
-            tmem_ld16_async(tmem + 160 + ch16 + lb, r2);
+            tmem_ld16_async(tmem + 160 + ch16 + lb, r1);
+            tmem_ld16_async(tmem + 128 + ch16 + lb, r2);
             tmem_wait_ld(r1);
             tmem_wait_ld(r2);
             const float e = ex2_approx(c);

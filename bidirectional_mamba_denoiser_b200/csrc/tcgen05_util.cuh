@@ -26,6 +26,17 @@ __host__ __device__ constexpr int f16_mnmajor(int m, int k, int MN) {
     return ((k >> 3) * (MN >> 3) + (m >> 3)) * 128 + (k & 7) * 16 + (m & 7) * 2;
 }
 
+// Byte offset of fp16 element (m, k) of an MN-major operand whose core
+// matrices (8 k-rows x 16 bytes along MN) run along K first: 8-k groups 128
+// bytes apart (LBO 128), 8-MN groups Kd / 8 core matrices apart (SBO Kd * 16).
+// Several such operands with the same Kd placed one after the other form one
+// operand with their MN extents added.  The same bytes read as a K-major
+// operand with the roles of the two indices exchanged (rows = k, K = m) have
+// LBO Kd * 16 and SBO 128.
+__host__ __device__ constexpr int f16_mn_kfast(int m, int k, int Kd) {
+    return ((m >> 3) * (Kd >> 3) + (k >> 3)) * 128 + (k & 7) * 16 + (m & 7) * 2;
+}
+
 // Shared-memory matrix descriptor: start address, leading and stride byte
 // offsets (16-byte units), version 1, no swizzle.
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
