@@ -59,7 +59,7 @@ MUFU_PER_ELEM_FWD = 20        # one direction: 16 state exps + SiLU 2 + softplus
 NCU_TRAFFIC = {
 
     ("layer_1p3b_b8_L2048_D4096_bf16", "fused_layer_kernel"): 1307.9e6,
-    ("mamba2_1p3b_b8_L2048_H120x32_N128_bf16", "m2_prep + m2_ssd dual-form kernel (both directions)"): 1026.6e6,
+    ("mamba2_1p3b_b8_L2048_H120x32_N128_bf16", "m2_prep + m2_ssd dual-form kernel (both directions)"): 1026.2e6,
     ("long_b1_L16384_D4096_bf16", "layer_tma_kernel"): 1457.4e6,
     ("long_b1_L65536_D4096_bf16", "layer_tma_kernel"): 4 * 1457.4e6,
     ("block_cached_b16_P65536_G32_D4096_bf16", "async_block_kernel"): 22.2e6,
