@@ -142,6 +142,10 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
     const int c0 = TILES ? H * kM2P + (int)(threadIdx.x & 31) * 8 : (blockIdx.y * 128 + threadIdx.x) * 8;
     const int64_t t0 = TILES ? ((int64_t)blockIdx.x * 4 + (threadIdx.x >> 5)) * TT : (int64_t)blockIdx.x * TT;
     const int r = blockIdx.z / p.batch, b = blockIdx.z % p.batch;
+    // per thread 8 rows of 16 bytes, rows of neighbouring threads 144 bytes apart (2-way bank
+    // conflicts at most for the 16 B-channel threads of a warp)
+    constexpr int kBStageStride = 144;
+    __shared__ __align__(16) unsigned char bstage[TILES ? 128 * kBStageStride : 16];
     if (c0 < CH) {
         const Tin* X = static_cast<const Tin*>(p.xbc[r]) + (int64_t)b * L * CH + c0;
         float w[8][4], cb[8];
@@ -170,15 +174,16 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
             else
                 xw[k].zero();
         }
-        // TILES, B channels: the group's 8 steps of each of the thread's 8 channels, as fp16
-        // pairs (a token's step within the group is k forward, 7 - k in reverse)
-        uint32_t hb[8][4];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) hb[q][u] = 0u;
+        // TILES, B channels: the group's 8 steps of each of the thread's 8 channels gather in
+        // fp16 in the thread's own shared-memory rows (one 16-byte row per channel; a token's step
+        // within the group is k forward, 7 - k in reverse; steps past the end stay zero)
         const int HPc = H * kM2P;
         const bool isB = TILES && c0 < HPc + kM2N;
+        unsigned char* brow = bstage + threadIdx.x * kBStageStride;
+        if (isB) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(brow + 16 * q)[0] = make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
         for (int k = 0; k < TT; ++k) {
             const int64_t t = t0 + k;
@@ -198,16 +203,9 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
                 dst[0] = make_float4(v[0], v[1], v[2], v[3]);
                 dst[1] = make_float4(v[4], v[5], v[6], v[7]);
             } else if (isB) {
-                // fp16 bits of v[q] into half (step within the group) of hb[q]
+                const int sl = r == 0 ? k : TT - 1 - k;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t hv = (uint32_t)__half_as_ushort(__float2half_rn(v[q]));
-                    if (r == 0) {
-                        hb[q][k >> 1] |= (k & 1) ? hv << 16 : hv;
-                    } else {
-                        hb[q][(TT - 1 - k) >> 1] |= ((TT - 1 - k) & 1) ? hv << 16 : hv;
-                    }
-                }
+                for (int q = 0; q < 8; ++q) reinterpret_cast<__half*>(brow + 16 * q)[sl] = __float2half_rn(v[q]);
             } else {
                 const __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
                 const __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
@@ -231,7 +229,7 @@ __global__ void __launch_bounds__(128) m2_prep_kernel(const M2Params p) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 *reinterpret_cast<uint4*>(T + f16_mn_kfast((int)(s0 % kM2Chunk), n0 + q, kM2N)) =
-                    make_uint4(hb[q][0], hb[q][1], hb[q][2], hb[q][3]);
+                    reinterpret_cast<const uint4*>(brow + 16 * q)[0];
         }
     }
     if (!TILES && blockIdx.y == 0) {
