@@ -216,7 +216,11 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         // the next chunk's tiles into L2 a chunk ahead of their copies into shared memory
         if (tid == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
         cp_async_wait_all();
-        __syncthreads();  // every xBC row of the chunk is in shared memory
+        // every xBC row of the chunk is in shared memory, and the previous chunk's epilogue is
+        // done with the staging block and with its TMEM reads
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
         // conv + SiLU of step t: rows t..t+3 hold steps t-3..t, and tap j multiplies step t-3+j in
         // both directions (the reverse scan's steps run backwards in time)
 #pragma unroll
@@ -468,9 +472,6 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
                 }
             }
         }
-        tmem_fence_before_sync();
-        __syncthreads();
-        tmem_fence_after_sync();
     }
     if (CL && meetk >= nc) cluster_meet();  // a one-chunk sequence: the reverse CTA meets after its chunk
     tmem_fence_before_sync();
