@@ -18,6 +18,7 @@
 #include "layer_tma.cuh"
 #include "mamba2.cuh"
 #include "mamba2_ssd.cuh"
+#include "mamba2_block.cuh"
 #include "proj.cuh"
 #include "scan_kernels.cuh"
 
@@ -1057,6 +1058,31 @@ int launch_m2(const bimamba::M2Params& k, cudaStream_t st) {
     return launch_status();
 }
 
+// The block step with bf16 inputs, a block of at most 32 steps and a multiple of
+// 4 heads: the features and step sizes as for the step-by-step scan, then the
+// block's closed form on the tensor cores (m2_block_mma_kernel), then the
+// combination and gate.
+template <typename Tout>
+int launch_m2_block_mma(const bimamba::M2Params& k, cudaStream_t st) {
+    const dim3 g1((unsigned)((k.L + bimamba::kM2PrepT - 1) / bimamba::kM2PrepT), (unsigned)((k.CH + 1023) / 1024),
+                  (unsigned)(2 * k.batch));
+    bimamba::m2_prep_kernel<bf16, false><<<g1, 128, 0, st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    bimamba::m2_block_gram_kernel<<<dim3((unsigned)k.batch, 2, bimamba::kM2BlkT / bimamba::kM2GramRows), 128, 0,
+                                    st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const int smem = k.S_out ? bimamba::kBlkSmemCommit : bimamba::kBlkSmemStep;
+    int rc = ensure_smem(reinterpret_cast<const void*>(&bimamba::m2_block_mma_kernel), bimamba::kBlkSmemCommit);
+    if (rc) return rc;
+    bimamba::m2_block_mma_kernel<<<dim3((unsigned)(k.H / bimamba::kM2BlkHeads), (unsigned)k.batch, 2), 128, smem,
+                                   st>>>(k);
+    if (cudaGetLastError() != cudaSuccess) return BIMAMBA_ERR_CUDA;
+    const int64_t n4 = (int64_t)k.batch * k.L * k.H * bimamba::kM2P / 4;
+    const int64_t blocks = (n4 + 255) / 256;
+    bimamba::m2_combine_kernel<bf16, Tout><<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, st>>>(k);
+    return launch_status();
+}
+
 // Shared checks of the Mamba-2 entry points: parameters and the 16-byte
 // alignment the kernels' vector accesses need.
 int m2_check_params(const bimamba2_params_t* p) {
@@ -1166,6 +1192,7 @@ int bimamba2_block_step(const bimamba2_fwd_state_t* prefix_state, const bimamba2
     k.DL = reinterpret_cast<float*>(ws + lay.dl);
     k.YF = reinterpret_cast<float*>(ws + lay.yf);
     k.YB = reinterpret_cast<float*>(ws + lay.yb);
+    k.tiles = ws + lay.tiles;  // the tensor-core block step's G [2][batch][32][32] fp32
     k.L = block_len;
     k.H = nheads;
     k.CH = nheads * headdim + 2 * d_state;
@@ -1176,9 +1203,14 @@ int bimamba2_block_step(const bimamba2_fwd_state_t* prefix_state, const bimamba2
     k.tail_in = prefix_state->conv_xbc;
     k.S_out = new_state ? new_state->S : nullptr;
     k.tail_out = new_state ? new_state->conv_xbc : nullptr;
+    k.wait_limit = kWaitCycles;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     const bool in_bf = block->dtype == BIMAMBA_BF16, out_bf = out_dtype == BIMAMBA_BF16;
-    if (in_bf && out_bf) rc = launch_m2<bf16, bf16>(k, st);
+    // bf16 inputs (tolerance 2e-3, fp16 operands suffice), a block of at most 32 steps and a
+    // multiple of 4 heads: the tensor-core closed form; otherwise the step-by-step scan
+    const bool mma = in_bf && block_len <= bimamba::kM2BlkT && nheads % bimamba::kM2BlkHeads == 0;
+    if (mma) rc = out_bf ? launch_m2_block_mma<bf16>(k, st) : launch_m2_block_mma<float>(k, st);
+    else if (in_bf && out_bf) rc = launch_m2<bf16, bf16>(k, st);
     else if (in_bf) rc = launch_m2<bf16, float>(k, st);
     else if (out_bf) rc = launch_m2<float, bf16>(k, st);
     else rc = launch_m2<float, float>(k, st);

@@ -276,3 +276,69 @@ def test_block_step_without_commit_leaves_state(bm):
     bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(S, S0) and torch.equal(tail, t0)
+
+
+# bf16 inputs, a block of at most 32 steps and a multiple of 4 heads: the block
+# step's closed form on the tensor cores (fp16 operands, fp32 state), within the
+# dual form's 2e-3 bound.
+@pytest.mark.parametrize("G,H", [(32, 4), (31, 8), (17, 4), (1, 4)])
+def test_block_chain_tensor_path(bm, G, H):
+    """Prefix of 100 tokens, then two committed blocks of G; expected values
+    from the layer oracle by the definition of the block step (forward: the
+    full-sequence forward restricted to the block; reverse: the layer on the
+    block alone).  The second block checks the first commit's state; the
+    tail is compared bit for bit."""
+    b, Pn = 2, 100
+    inp, par = W.make_mamba2_case(b, Pn + 2 * G, H, P, N, "bf16", seed=90 + G)
+    d, p = U.to_device(inp), U.to_device(par)
+    pre = _tok(d, 0, Pn)
+    S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
+    for k in range(2):
+        lo, hi = Pn + k * G, Pn + (k + 1) * G
+        blk = _tok(d, lo, hi)
+        out = bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=torch.float32,
+                                     new_state=(S, tail))
+        torch.cuda.synchronize()
+        assert bm.bimamba_device_error() == 0
+        _, yf, _ = oracle.mamba2_layer_fwd(_tok(inp, 0, hi), par, return_dirs=True)
+        bi = _tok(inp, lo, hi)
+        _, _, yr = oracle.mamba2_layer_fwd(bi, par, return_dirs=True)
+        z = bi["z"].double().numpy()
+        want = (yf[:, lo:hi] + yr) * (z / (1.0 + np.exp(-z)))
+        assert U.normwise(U.to_cpu64(out), want) <= U.TOL_BF16, k
+        want_tail = inp["xbc"][0, :, hi - 3:hi].double().numpy()
+        assert np.array_equal(U.to_cpu64(tail), want_tail), k
+
+
+@pytest.mark.parametrize("which", ["fwd", "rev", "bf16_out"])
+def test_block_step_tensor_path_flags_and_output(bm, which):
+    """One block of 32 after a 64-token prefix, without commit: a single
+    direction by flag, or bf16 output (within one bf16 rounding + 2e-3); the
+    cached state is left unchanged."""
+    b, H, Pn, G = 2, 4, 64, 32
+    inp, par = W.make_mamba2_case(b, Pn + G, H, P, N, "bf16", seed=97)
+    d, p = U.to_device(inp), U.to_device(par)
+    pre = _tok(d, 0, Pn)
+    S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
+    S0, t0 = S.clone(), tail.clone()
+    blk = _tok(d, Pn, Pn + G)
+    flags = {"fwd": bm.BIMAMBA_FWD_ONLY, "rev": bm.BIMAMBA_REV_ONLY, "bf16_out": 0}[which]
+    out_dtype = torch.bfloat16 if which == "bf16_out" else torch.float32
+    out = bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=out_dtype, flags=flags)
+    torch.cuda.synchronize()
+    assert bm.bimamba_device_error() == 0
+    _, yf, _ = oracle.mamba2_layer_fwd(_tok(inp, 0, Pn + G), par, return_dirs=True)
+    bi = _tok(inp, Pn, Pn + G)
+    _, _, yr = oracle.mamba2_layer_fwd(bi, par, return_dirs=True)
+    yf, yr = yf[:, Pn:], yr
+    if which == "fwd":
+        yr = np.zeros_like(yr)
+    elif which == "rev":
+        yf = np.zeros_like(yf)
+    z = bi["z"].double().numpy()
+    want = (yf + yr) * (z / (1.0 + np.exp(-z)))
+    if which == "bf16_out":
+        assert U.bf16_out_ok(U.to_cpu64(out), want)
+    else:
+        assert U.normwise(U.to_cpu64(out), want) <= U.TOL_BF16
+    assert torch.equal(S, S0) and torch.equal(tail, t0)
