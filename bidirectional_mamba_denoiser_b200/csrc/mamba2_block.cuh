@@ -61,14 +61,27 @@ __global__ void __launch_bounds__(128) m2_block_gram_kernel(const M2Params p) {
     auto row_of = [&](int t) -> const float* {
         return Vb + (DIR == 0 ? (int64_t)t : L - 1 - t) * CH + HP;
     };
-    for (int e = tid; e < T * N; e += 128) {
-        const int t = e / N, n = e % N;
-        sBr[t * RS + n] = t < L ? row_of(t)[n] : 0.f;
+    // 16-byte loads, all of a thread's issued together
+    float4 bq[T * N / 4 / 128];
+#pragma unroll
+    for (int j = 0; j < T * N / 4 / 128; ++j) {
+        const int e = tid + 128 * j, t = e / (N / 4), q = e % (N / 4);
+        bq[j] = t < L ? reinterpret_cast<const float4*>(row_of(t))[q] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int e = tid; e < R * N; e += 128) {
-        const int t = e / N, n = e % N;
-        sCr[t * RS + n] = t0 + t < L ? row_of(t0 + t)[N + n] : 0.f;
+    const int ec = tid, tc = ec / (N / 4), qc = ec % (N / 4);  // R * N / 4 == 128: one C load each
+    const float4 cq = t0 + tc < L ? reinterpret_cast<const float4*>(row_of(t0 + tc) + N)[qc]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < T * N / 4 / 128; ++j) {
+        const int e = tid + 128 * j, t = e / (N / 4), q = e % (N / 4);
+        float* d = sBr + t * RS + 4 * q;
+        d[0] = bq[j].x; d[1] = bq[j].y; d[2] = bq[j].z; d[3] = bq[j].w;
     }
+    {
+        float* d = sCr + tc * RS + 4 * qc;
+        d[0] = cq.x; d[1] = cq.y; d[2] = cq.z; d[3] = cq.w;
+    }
+    static_assert(R * N / 4 == 128, "one 16-byte C load per thread");
     __syncthreads();
     const int tl = tid >> 5, s = tid & 31;
     float g = 0.f;
