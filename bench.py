@@ -799,9 +799,15 @@ def run_decode(args, w, bm, rank, world, dev, stream):
         roof = roofline(MUFU_PER_ELEM_LAYER * elems, call_ms, clocks, w.name, kernel_name(w, args))
         hbm = hbm_fraction(block_bytes(w), call_ms)
     else:
-        # conv features, forward and reverse scans per call; a commit adds the conv tail
-        launches = reps * (3 * K * layers + layers)
+        # bf16 blocks of at most 32 steps over a multiple of 4 heads: conv features, the block's
+        # Gram matrix, its closed form on the tensor cores and the combination; else the conv
+        # features, both directions' step-by-step scans and the combination.  A commit adds the
+        # conv tail.
+        tensor = w.dtype == "bf16" and G <= 32 and H % 4 == 0
+        launches = reps * ((4 if tensor else 3) * K * layers + layers)
         roof = roofline_fma(4.0 * Pd * w.d_state * H * 2 * w.batch * G, call_ms, clocks, w.name,
+                            "m2_prep + m2_block_gram + m2_block_mma + m2_combine (block step; the "
+                            "recurrence's FP32-equivalent work)" if tensor else
                             "m2_prep + 2 x m2_scan_kernel (block step)")
         state = w.batch * H * Pd * w.d_state * 4 + w.batch * 3 * (w.d_inner + 2 * w.d_state) * 2
         hbm = hbm_fraction(mamba2_bytes(w.batch, G, H, Pd, w.d_state) + state + state // K, call_ms)

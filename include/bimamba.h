@@ -365,7 +365,10 @@ int bimamba2_prefix_state(const bimamba2_inputs_t *prefix, const bimamba2_params
  * new_state is not NULL the forward state and conv tail after the block are
  * written there (commit); new_state may be prefix_state itself.  workspace:
  * at least bimamba2_workspace_bytes(batch, block_len, ...) bytes.  Flags:
- * BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY or 0.  Step-by-step scan on the CUDA
+ * BIMAMBA_FWD_ONLY, BIMAMBA_REV_ONLY or 0.  bf16 inputs with block_len <= 32
+ * and nheads % 4 == 0: the block's closed form, C S^T and the state update on
+ * the tensor cores with fp16 operands (within the 2e-3 bound for bf16 I/O);
+ * 4 launches, 5 with a commit.  Otherwise the step-by-step scan on the CUDA
  * cores in fp32; 3 launches, 4 with a commit. */
 int bimamba2_block_step(const bimamba2_fwd_state_t *prefix_state, const bimamba2_inputs_t *block,
                         int64_t block_len, const bimamba2_params_t *p,
