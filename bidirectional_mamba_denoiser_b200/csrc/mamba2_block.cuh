@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(128) m2_block_gram_kernel(const M2Params p) {
 // m2_scan_kernel, and, forward with p.S_out, the state after the block.  Which
 // products run depends on the CTA: the reverse starts from zero (no C S_^T)
 // and keeps no state, and the forward updates the state only on a commit.
-__global__ void __launch_bounds__(128, 3) m2_block_mma_kernel(const M2Params p) {
+__global__ void __launch_bounds__(128, 4) m2_block_mma_kernel(const M2Params p) {
     constexpr int T = kM2BlkT, P = kM2P, N = kM2N;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
@@ -185,14 +185,17 @@ __global__ void __launch_bounds__(128, 3) m2_block_mma_kernel(const M2Params p) 
     // the fp16 operand of C S_^T
     if (with_state && !commit) {
         const float4* srow = reinterpret_cast<const float4*>(p.S_in + (((int64_t)b * H + h) * P + lane) * N);
-        float4 v4[N / 4];
 #pragma unroll
-        for (int i = 0; i < N / 4; ++i) v4[i] = srow[i];
+        for (int hh = 0; hh < 2; ++hh) {  // two halves of 64 states, each half's loads issued together
+            float4 v4[N / 8];
 #pragma unroll
-        for (int g = 0; g < N / 8; ++g) {
-            const float v[8] = {v4[2 * g].x, v4[2 * g].y, v4[2 * g].z, v4[2 * g].w,
-                                v4[2 * g + 1].x, v4[2 * g + 1].y, v4[2 * g + 1].z, v4[2 * g + 1].w};
-            st_half8(sS16 + f16_kmajor(tid, 8 * g, N), v);
+            for (int i = 0; i < N / 8; ++i) v4[i] = srow[hh * (N / 8) + i];
+#pragma unroll
+            for (int g = 0; g < N / 16; ++g) {
+                const float v[8] = {v4[2 * g].x, v4[2 * g].y, v4[2 * g].z, v4[2 * g].w,
+                                    v4[2 * g + 1].x, v4[2 * g + 1].y, v4[2 * g + 1].z, v4[2 * g + 1].w};
+                st_half8(sS16 + f16_kmajor(tid, hh * (N / 2) + 8 * g, N), v);
+            }
         }
     }
     // ---- x of this thread's channel (h, p = lane) at every step
