@@ -1145,8 +1145,23 @@ int bimamba2_prefix_state(const bimamba2_inputs_t* prefix, const bimamba2_params
     const dim3 g2((unsigned)nheads, (unsigned)batch);
     const dim3 g3((unsigned)((k.CH + 127) / 128), (unsigned)batch);
     if (prefix->dtype == BIMAMBA_BF16) {
-        bimamba::m2_prep_kernel<bf16, false><<<g1, 128, 0, st>>>(k);
-        bimamba::m2_scan_kernel<false, bf16><<<g2, 32, 0, st>>>(k);
+        // bf16 inputs (the 2e-3 bound): the chunked dual form's state updates on the tensor cores,
+        // from the B tiles of direction 0
+        k.tiles = ws + lay.tiles;
+        k.wait_limit = kWaitCycles;
+        const int64_t nc = (P + bimamba::kSQ - 1) / bimamba::kSQ;
+        if (P % bimamba::kSQ) {  // the last chunk's rows past the end read zeros
+            const size_t pair = 2 * (size_t)bimamba::kTileBytes;
+            if (cudaMemset2DAsync(k.tiles + (nc - 1) * pair, (size_t)nc * pair, 0, pair, (size_t)batch, st) !=
+                cudaSuccess)
+                return BIMAMBA_ERR_CUDA;
+        }
+        const int64_t tok_per_cta = 4 * bimamba::kM2PrepT;
+        const dim3 gt((unsigned)((P + tok_per_cta - 1) / tok_per_cta), 1u, (unsigned)batch);  // direction 0 only
+        bimamba::m2_prep_kernel<bf16, true><<<gt, 128, 0, st>>>(k);
+        rc = ensure_smem(reinterpret_cast<const void*>(&bimamba::m2_ssd_prefix_kernel), bimamba::kSsdSmem);
+        if (rc) return rc;
+        bimamba::m2_ssd_prefix_kernel<<<g2, bimamba::kSsdThreads, bimamba::kSsdSmem, st>>>(k);
         bimamba::m2_tail_kernel<bf16><<<g3, 128, 0, st>>>(k);
     } else {
         bimamba::m2_prep_kernel<float, false><<<g1, 128, 0, st>>>(k);

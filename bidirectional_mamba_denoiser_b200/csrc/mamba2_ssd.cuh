@@ -97,8 +97,10 @@ __device__ __forceinline__ void cluster_meet() {
 
 // CL: the two directions run as a cluster and meet halfway (above).  Without
 // it the forward stores y for every chunk (p.YF) and the reverse, launched
-// after it, gates every chunk with that y.
-template <int DIR, typename Tin, typename Tout, bool CL>
+// after it, gates every chunk with that y.  PREFIX (forward, no cluster): the
+// prefix state of block-cached decoding -- only the state update runs (no G,
+// C S_^T, M or output), from zero, and the final state goes to p.S_out.
+template <int DIR, typename Tin, typename Tout, bool CL, bool PREFIX = false>
 __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm, const int h, const int b) {
     constexpr int Q = kSQ, P = kM2P;
     static_assert(sizeof(Tin) == 2, "the dual form reads bf16 inputs");
@@ -167,11 +169,14 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         for (int i = 0; i < 16; ++i) zero[i] = 0.f;
         tmem_st16(tmem + 192 + ch16 + lb, zero);  // state row n = t starts at 0
     }
+    static_assert(!PREFIX || (DIR == 0 && !CL), "the prefix state is the forward's");
     if (tid == 0 && !p.starve) {
         mbar_arrive_expect_tx(bars + 0, kTileBytes);
         bulk_g2s(sB, tileb + kTileBytes, kTileBytes, bars + 0);
-        mbar_arrive_expect_tx(bars + 1, kTileBytes);
-        bulk_g2s(sC, tileb, kTileBytes, bars + 1);
+        if constexpr (!PREFIX) {
+            mbar_arrive_expect_tx(bars + 1, kTileBytes);
+            bulk_g2s(sC, tileb, kTileBytes, bars + 1);
+        }
     }
     // step t of chunk kk: this half's 16 xBC channels of the head into row 3 + t of sX (zeros past
     // either end) and dt into a register, used one chunk later
@@ -214,7 +219,12 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         const float dtk = dt_next;
         const bool okk = ok_next;
         // the next chunk's tiles into L2 a chunk ahead of their copies into shared memory
-        if (tid == 0 && k + 1 < nc && !p.starve) prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
+        if (tid == 0 && k + 1 < nc && !p.starve) {
+            if constexpr (PREFIX)
+                prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes + kTileBytes, kTileBytes);
+            else
+                prefetch_l2(tileb + (int64_t)(k + 1) * 2 * kTileBytes, 2 * kTileBytes);
+        }
         cp_async_wait_all();
         // every xBC row of the chunk is in shared memory, and the previous chunk's epilogue is
         // done with the staging block and with its TMEM reads
@@ -272,7 +282,7 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         }
         // ---- G = C B^T and Y2 = C S_^T need only the tiles and the state of the previous
         // chunk: they run on the tensor cores while the steps below are computed
-        if (tid == 0) {
+        if (!PREFIX && tid == 0) {
             mbar_wait_bounded(bars + 0, ph, p.wait_limit);
             mbar_wait_bounded(bars + 1, ph, p.wait_limit);
             tmem_fence_after_sync();
@@ -288,7 +298,7 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             // block j = warp: step s's factor 2^(c_{32j} - c_s) >= 1, usable while the span is small
             const float cref = __shfl_sync(0xffffffffu, c, 0);
             const float span = cref - __shfl_sync(0xffffffffu, c, 31);
-            if (hf == 0) {
+            if (!PREFIX && hf == 0) {
                 c2s[t] = c;
                 sE[t] = ex2_approx(fminf(cref - c, kSsdSpanMax));
                 if (lane == 0) bigspan[warp] = span > kSsdSpanMax ? 1 : 0;
@@ -300,8 +310,10 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
             float dx[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) dx[i] = dl * x[i];
+            if constexpr (!PREFIX) {
 #pragma unroll
-            for (int pg = 0; pg < 2; ++pg) st_half8(sDX + f16_mnmajor(16 * hf + 8 * pg, t, P), dx + 8 * pg);
+                for (int pg = 0; pg < 2; ++pg) st_half8(sDX + f16_mnmajor(16 * hf + 8 * pg, t, P), dx + 8 * pg);
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) dx[i] *= wdec;
 #pragma unroll
@@ -342,9 +354,22 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         tmem_fence_after_sync();
         // ---- S^T += B^T W (onto the decayed state)
         if (tid == 0) {
+            if constexpr (PREFIX) {
+                mbar_wait_bounded(bars + 0, ph, p.wait_limit);
+                tmem_fence_after_sync();
+            }
             umma_f16_k8<4096 / 16, 1024 / 16>(tmem + 192, umma_desc(aB, 2048, 128), umma_desc(aW, 512, 128), ID_S,
                                               true);
             umma_commit(bars + 4);
+        }
+        if constexpr (PREFIX) {  // the state is all a prefix needs
+            mbar_wait_bounded(bars + 4, ph, p.wait_limit);
+            tmem_fence_after_sync();
+            if (tid == 0 && k + 1 < nc && !p.starve) {  // B's buffer is free: next chunk's B tile
+                mbar_arrive_expect_tx(bars + 0, kTileBytes);
+                bulk_g2s(sB, tileb + (int64_t)(k + 1) * 2 * kTileBytes + kTileBytes, kTileBytes, bars + 0);
+            }
+            continue;
         }
         mbar_wait_bounded(bars + 2, ph, p.wait_limit);
         tmem_fence_after_sync();
@@ -474,9 +499,25 @@ __device__ __forceinline__ void m2_ssd_dir(const M2Params& p, unsigned char* sm,
         }
     }
     if (CL && meetk >= nc) cluster_meet();  // a one-chunk sequence: the reverse CTA meets after its chunk
+    if constexpr (PREFIX) {  // the final state: row n = t, this half's channels p
+        uint32_t sn[16];
+        tmem_ld16_async(tmem + 192 + ch16 + lb, sn);
+        tmem_wait_ld(sn);
+        float* so = p.S_out + ((int64_t)b * H + h) * P * kM2N + t;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) so[(int64_t)(16 * hf + i) * kM2N] = __uint_as_float(sn[i]);
+    }
     tmem_fence_before_sync();
     __syncthreads();
     if (tid < 32) tmem_dealloc<256>(tmem);
+}
+
+// The forward prefix state of block-cached decoding on the tensor cores
+// (bf16 inputs): grid (H, batch), block kSsdThreads, dynamic shared memory
+// kSsdSmem; the B tiles from m2_prep_kernel<bf16, true>.
+__global__ void __launch_bounds__(kSsdThreads, 2) m2_ssd_prefix_kernel(const M2Params p) {
+    extern __shared__ __align__(128) unsigned char sm[];
+    m2_ssd_dir<0, __nv_bfloat16, float, false, true>(p, sm, (int)blockIdx.x, (int)blockIdx.y);
 }
 
 // grid (2 H, batch) in clusters of 2: CTA 2h runs head h forward, CTA 2h+1 in

@@ -249,7 +249,9 @@ def test_block_chain_from_prefix_state(bm, dtype):
     d, p = U.to_device(inp), U.to_device(par)
     pre = _tok(d, 0, Pn)
     S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
-    tol = U.TOL_FP32 if dtype == "fp32" else U.GUARD
+    # bf16 inputs: the prefix state comes from the dual form's state updates on the tensor cores
+    # (fp16 operands), held to the 2e-3 bound of bf16 I/O; the blocks (G 37) run the fp32 scan
+    tol = U.TOL_FP32 if dtype == "fp32" else U.TOL_BF16
     for k in range(2):
         lo, hi = Pn + k * G, Pn + (k + 1) * G
         blk = _tok(d, lo, hi)
