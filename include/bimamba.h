@@ -349,9 +349,12 @@ typedef struct {
 /* Forward scan of the Mamba-2 mixer over a prefix of P tokens from a zero
  * state: writes state_out->S and state_out->conv_xbc.  Reads prefix->xbc[0]
  * and prefix->dt[0] (the rest may be NULL).  workspace: at least
- * bimamba2_workspace_bytes(batch, P, ...) bytes, 256-byte aligned.  Three
- * launches (conv features, forward scan with the final state, conv tail);
- * step-by-step scan on the CUDA cores in fp32. */
+ * bimamba2_workspace_bytes(batch, P, ...) bytes, 256-byte aligned.  bf16
+ * inputs: the chunked dual form's state updates on the tensor cores (fp16
+ * operands, fp32 state; within the 2e-3 bound of bf16 I/O): the C/B tiles,
+ * the state pass, the conv tail (3 launches and a memset when P % 128 != 0).
+ * fp32 inputs: conv features, the step-by-step forward scan on the CUDA cores
+ * in fp32, the conv tail (3 launches). */
 int bimamba2_prefix_state(const bimamba2_inputs_t *prefix, const bimamba2_params_t *p,
                           int batch, int64_t P, int nheads, int headdim, int d_state,
                           bimamba2_fwd_state_t *state_out, void *workspace, size_t workspace_bytes,
