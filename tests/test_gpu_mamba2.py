@@ -344,3 +344,28 @@ def test_block_step_tensor_path_flags_and_output(bm, which):
     else:
         assert U.normwise(U.to_cpu64(out), want) <= U.TOL_BF16
     assert torch.equal(S, S0) and torch.equal(tail, t0)
+
+
+@pytest.mark.parametrize("Pn", [128, 300, 1])
+def test_prefix_state_tensor_path_lengths(bm, Pn):
+    """bf16 prefixes of one whole chunk, several chunks with a ragged last one,
+    and a single token (the prefix state's state updates on the tensor cores),
+    each followed by one committed block of 32: the block's output against the
+    layer oracle by the block step's definition, and the tail bit for bit."""
+    b, H, G = 2, 4, 32
+    inp, par = W.make_mamba2_case(b, Pn + G, H, P, N, "bf16", seed=110 + Pn)
+    d, p = U.to_device(inp), U.to_device(par)
+    pre = _tok(d, 0, Pn)
+    S, tail = bm.bimamba2_prefix_state(pre["xbc"], pre["dt"], p)
+    blk = _tok(d, Pn, Pn + G)
+    out = bm.bimamba2_block_step((S, tail), blk["xbc"], blk["z"], blk["dt"], p, out_dtype=torch.float32,
+                                 new_state=(S, tail))
+    torch.cuda.synchronize()
+    assert bm.bimamba_device_error() == 0
+    _, yf, _ = oracle.mamba2_layer_fwd(_tok(inp, 0, Pn + G), par, return_dirs=True)
+    bi = _tok(inp, Pn, Pn + G)
+    _, _, yr = oracle.mamba2_layer_fwd(bi, par, return_dirs=True)
+    z = bi["z"].double().numpy()
+    want = (yf[:, Pn:] + yr) * (z / (1.0 + np.exp(-z)))
+    assert U.normwise(U.to_cpu64(out), want) <= U.TOL_BF16
+    assert np.array_equal(U.to_cpu64(tail), inp["xbc"][0, :, Pn + G - 3:Pn + G].double().numpy())
